@@ -1,0 +1,52 @@
+"""Seeded synthetic inputs shared by the CUDA path's tests, the bench and the oracle checks.
+
+This module holds no attention arithmetic: it only draws i.i.d. N(0, 1) values
+with torch's CPU generator and rounds them to bf16, the activations' dtype.
+Seeds 0, 1, 2, 3 draw q, k, v and dO respectively (an offset shifts all four).
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import torch
+
+
+@dataclass(frozen=True)
+class Shape:
+    """One attention problem: batch B, query heads H, kv heads Hkv, head dim D,
+    sequence length N, group size G (G == N means dense causal)."""
+    name: str
+    B: int
+    H: int
+    Hkv: int
+    D: int
+    N: int
+    G: int
+
+    def dense(self) -> "Shape":
+        return Shape(self.name + "-dense", self.B, self.H, self.Hkv, self.D, self.N, self.N)
+
+
+# The five workload shapes: group size a quarter of the sequence, half the
+# (query) heads shifted by half a group.
+TINY = Shape("tiny", 1, 4, 4, 64, 1024, 256)
+LLAMA2_7B_8K = Shape("llama2-7b-n8192", 1, 32, 32, 128, 8192, 2048)
+QWEN3_8B_16K = Shape("qwen3-8b-gqa-n16384", 1, 32, 8, 128, 16384, 4096)
+LLAMA2_70B_32K = Shape("llama2-70b-gqa-n32768", 1, 64, 8, 128, 32768, 8192)
+LLAMA2_7B_100K = Shape("llama2-7b-n102400", 1, 32, 32, 128, 102400, 25600)
+WORKLOADS = [TINY, LLAMA2_7B_8K, QWEN3_8B_16K, LLAMA2_70B_32K, LLAMA2_7B_100K]
+
+
+def randn_bf16(shape, seed: int) -> torch.Tensor:
+    """fp32 N(0,1) from a seeded CPU generator, rounded to bf16 (RNE)."""
+    g = torch.Generator().manual_seed(seed)
+    return torch.randn(*shape, generator=g, dtype=torch.float32).to(torch.bfloat16)
+
+
+def make_inputs(s: Shape, seed_offset: int = 0):
+    """(q, k, v, dO) as CPU bf16 tensors: q, dO [B,N,H,D]; k, v [B,N,Hkv,D]."""
+    q = randn_bf16((s.B, s.N, s.H, s.D), 0 + seed_offset)
+    k = randn_bf16((s.B, s.N, s.Hkv, s.D), 1 + seed_offset)
+    v = randn_bf16((s.B, s.N, s.Hkv, s.D), 2 + seed_offset)
+    do = randn_bf16((s.B, s.N, s.H, s.D), 3 + seed_offset)
+    return q, k, v, do
