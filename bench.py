@@ -1,0 +1,402 @@
+#!/usr/bin/env python
+"""Benchmark of S2-Attn forward + backward on B200 GPUs (one process per GPU).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pass of the whole hot path over one batch: s2attn_forward (one
+kernel) then s2attn_backward (preprocess, dK/dV, dQ kernels), through the C ABI.
+The headline is effective fwd+bwd TFLOP/s, FLOPs counted as
+4*B*H*N*G*D/2 forward and 2.5x that backward.  Rank 0 prints one JSON line.
+
+Under torchrun (N > 1) every rank runs the same workload on its own batch
+(weak scaling, no collective on the data path); the time is the max over ranks.
+
+--impl reference times the fp64 CPU oracle (the only reference there is) on a
+bounded sample of the same workload, on this machine's host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from sparse_attention_attn_b200 import inputs as I  # noqa: E402
+
+METRIC = "S2-Attn fwd+bwd TFLOP/s & tokens/s on 1 B200; % of BF16 tensor peak"
+KERNEL_NAMES = {0: "s2_fwd_kernel", 1: "s2_bwd_pre_kernel", 2: "s2_bwd_dkdv_kernel", 3: "s2_bwd_dq_kernel"}
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def effective_flops(s: I.Shape):
+    fwd = 4.0 * s.B * s.H * s.N * s.G * s.D * 0.5
+    return fwd, 2.5 * fwd
+
+
+def kernel_algorithmic(s: I.Shape):
+    """Per-launch algorithmic work of each kernel.  The UMMA kernels are
+    credited the GEMMs they must issue on the causal half of every group
+    (2*B*H*N*G*D/2 FLOPs per GEMM): forward 2 (S, O), dK/dV 4 (S, dP, dV, dK),
+    dQ 3 (S, dP, dQ).  The preprocess moves bytes: O and dO read, Delta and
+    lse*log2(e) written, lse read."""
+    gemm = 2.0 * s.B * s.H * s.N * s.G * s.D * 0.5
+    rows = s.B * s.H * s.N
+    return {0: ("tensor", 2 * gemm), 2: ("tensor", 4 * gemm), 3: ("tensor", 3 * gemm),
+            1: ("hbm", 2.0 * rows * s.D * 2 + rows * 4 * 3)}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            return json.load(fh), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling during the timed region."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        self.gpu = gpu_index
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as fh:
+            for line in fh:
+                f = [x.strip() for x in line.split(",")]
+                if len(f) < 9:
+                    continue
+                try:
+                    sm.append(float(f[1]))
+                    mx = float(f[2])
+                except ValueError:
+                    continue
+                for name, val in zip(names, f[5:9]):
+                    if val.lower().startswith("active"):
+                        reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def oracle_sample(shape: I.Shape, budget_s: float, seed_offset: int = 0):
+    """Time the fp64 oracle on whole (b, h, group) units of the workload until
+    `budget_s` seconds have passed (at least one unit).  Returns
+    (seconds, units, effective flops done, threads)."""
+    import oracle.s2_ref as ref
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = os.cpu_count()
+    g = torch.Generator().manual_seed(1234 + seed_offset)
+    # one unit's inputs: the group's rows of one head (same distribution as the workload)
+    fwd_unit = 4.0 * shape.G * shape.G * shape.D * 0.5
+    t0 = time.perf_counter()
+    units = 0
+    while True:
+        qg, kg, vg, dog = (torch.randn(shape.G, shape.D, generator=g).to(torch.bfloat16).double().numpy()
+                           for _ in range(4))
+        scale = 1.0 / np.sqrt(shape.D)
+        ref.group_causal_attention(qg, kg, vg, scale)
+        ref.group_causal_attention_grad(qg, kg, vg, dog, scale)
+        units += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    return el, units, units * fwd_unit * 3.5, threads
+
+
+def run_reference(args, shape, world, rank):
+    if rank != 0:
+        return
+    fwd, bwd = effective_flops(shape)
+    for _ in range(args.warmup):
+        oracle_sample(shape, 0.0)
+    total_s, total_units, total_flops, threads = 0.0, 0, 0.0, 1
+    for _ in range(args.steps):
+        el, u, fl, threads = oracle_sample(shape, args.ref_step_seconds)
+        total_s += el
+        total_units += u
+        total_flops += fl
+    tflops = total_flops / total_s / 1e12
+    tokens_per_s = total_units * shape.G / total_s
+    ms_per_step = 1e3 * (fwd + bwd) / (tflops * 1e12)  # time the oracle would take for one full step
+    line = {
+        "impl": "reference", "metric": METRIC, "value": tflops, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "tokens_per_s": tokens_per_s,
+        "config": {"workload": shape.name, "B": shape.B, "H": shape.H, "Hkv": shape.Hkv, "D": shape.D,
+                   "N": shape.N, "G": shape.G},
+        "cpu_baseline": {"value": tflops, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{total_units} whole (head, group) units of G={shape.G} rows, "
+                                   f"fwd+bwd, over {args.steps} steps"},
+        "e2e": {"value": tflops, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, shape, world, rank, local):
+    import sparse_attention_attn_b200 as s2
+    from sparse_attention_attn_b200 import _lib
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    q, k, v, do = I.make_inputs(shape, seed_offset=10 * rank)
+    qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
+    o = torch.empty_like(qd)
+    lse = torch.empty((shape.B, shape.H, shape.N), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
+    ws = torch.empty(s2.bwd_workspace_bytes(shape.B, shape.H, shape.Hkv, shape.N, shape.D, shape.G),
+                     dtype=torch.uint8, device=dev)
+    launches = [0]
+
+    def step():
+        s2.s2attn_forward(qd, kd, vd, shape.G, out=o, lse=lse)
+        launches[0] += _lib.s2attn_last_launch_count()
+        s2.s2attn_backward(qd, kd, vd, o, lse, dod, shape.G, dq=dq, dk=dk, dv=dv, workspace=ws)
+        launches[0] += _lib.s2attn_last_launch_count()
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    if s2.device_status() != 0 or s2.device_status(ws) != 0:
+        raise RuntimeError("device status reports a timeout during warm-up")
+
+    # ---- device-timed region (inputs resident in HBM) ----
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    cap = 4 * args.steps + 8
+    assert _lib.s2attn_profile_start(cap) == 0
+    launches[0] = 0
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms_total = e0.elapsed_time(e1)
+    ms_arr = (ctypes.c_float * cap)()
+    id_arr = (ctypes.c_int * cap)()
+    n_rec = _lib.s2attn_profile_stop(ctypes.addressof(ms_arr), ctypes.addressof(id_arr), cap)
+    clk = clocks.stop()
+    gpu_launches = launches[0]
+    per_kernel = {}
+    for i in range(max(n_rec, 0)):
+        per_kernel.setdefault(id_arr[i], []).append(ms_arr[i])
+    ms_step = max_over_ranks(ms_total / args.steps, world, dev)
+    if s2.device_status() != 0 or s2.device_status(ws) != 0:
+        raise RuntimeError("device status reports a timeout in the timed region")
+
+    # ---- end-to-end through the public API with pinned host buffers ----
+    hq, hk, hv, hdo = (t.pin_memory() for t in (q, k, v, do))
+    hdq, hdk, hdv = (torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (dq, dk, dv))
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo))
+    d2h = sum(t.numel() * t.element_size() for t in (hdq, hdk, hdv))
+
+    def e2e_step():
+        qd.copy_(hq, non_blocking=True)
+        kd.copy_(hk, non_blocking=True)
+        vd.copy_(hv, non_blocking=True)
+        dod.copy_(hdo, non_blocking=True)
+        step()
+        hdq.copy_(dq, non_blocking=True)
+        hdk.copy_(dk, non_blocking=True)
+        hdv.copy_(dv, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 20))
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    f1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms_e2e = max_over_ranks(f0.elapsed_time(f1) / e2e_steps, world, dev)
+
+    # ---- report ----
+    fwd, bwd = effective_flops(shape)
+    total_flops = (fwd + bwd) * world
+    tflops = total_flops / (ms_step * 1e-3) / 1e12
+    tokens = shape.B * shape.N * world / (ms_step * 1e-3)
+    peaks, peak_src = load_peaks()
+    alg = kernel_algorithmic(shape)
+    kern = {}
+    for kid, times in per_kernel.items():
+        avg = sum(times) / len(times)
+        bound, work = alg[kid]
+        if bound == "tensor":
+            ach = work / (avg * 1e-3) / 1e12
+            kern[KERNEL_NAMES[kid]] = {"avg_ms": avg, "launches": len(times), "achieved": ach,
+                                       "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"]}
+        else:
+            ach = work / (avg * 1e-3) / 1e9
+            kern[KERNEL_NAMES[kid]] = {"avg_ms": avg, "launches": len(times), "achieved": ach,
+                                       "unit": "GB/s", "frac": ach / peaks["hbm_gbs"]}
+    dom_id = max(per_kernel, key=lambda kid: sum(per_kernel[kid])) if per_kernel else 2
+    dom = kern.get(KERNEL_NAMES[dom_id], {})
+    bound = alg[dom_id][0]
+    roofline = {
+        "kernel": KERNEL_NAMES[dom_id], "bound": bound, "achieved": dom.get("achieved"),
+        "peak": peaks["bf16_tflops"] if bound == "tensor" else peaks["hbm_gbs"],
+        "unit": "TFLOP/s" if bound == "tensor" else "GB/s", "frac": dom.get("frac"),
+        "traffic": None, "peak_source": f"{peak_src} ({'bf16_tflops burst' if bound == 'tensor' else 'hbm_gbs'})",
+        "share": (sum(per_kernel[dom_id]) / sum(sum(v) for v in per_kernel.values())) if per_kernel else None,
+    }
+    line = {
+        "metric": METRIC, "value": tflops, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "tokens_per_s": tokens,
+        "frac_of_bf16_peak": tflops / (peaks["bf16_tflops"] * world),
+        "config": {"workload": shape.name, "B": shape.B, "H": shape.H, "Hkv": shape.Hkv, "D": shape.D,
+                   "N": shape.N, "G": shape.G, "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "l2": "inputs larger than L2 (q,k,v,dO,o = %d MiB), no flush" %
+                         ((4 * qd.numel() + 2 * kd.numel()) * 2 >> 20)},
+        "e2e": {"value": total_flops / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
+        "gpu_launches": gpu_launches,
+        "roofline": roofline,
+        "kernels": kern,
+        "clocks": clk,
+    }
+    if args.dense_ratio and rank == 0:
+        line["dense_comparison"] = dense_ratio(shape, dev, args)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        el, units, fl, threads = oracle_sample(shape, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": fl / el / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                                "sample": f"{units} whole (head, group) units of G={shape.G} rows, fwd+bwd, "
+                                          f"{el:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def dense_ratio(shape: I.Shape, dev, args):
+    """Same inputs through the same kernels with G = N (dense causal): time ratio."""
+    import sparse_attention_attn_b200 as s2
+    dense = shape.dense()
+    q, k, v, do = (t.to(dev) for t in I.make_inputs(dense))
+    ws = torch.empty(s2.bwd_workspace_bytes(dense.B, dense.H, dense.Hkv, dense.N, dense.D, dense.G),
+                     dtype=torch.uint8, device=dev)
+
+    def timed(G, steps):
+        for _ in range(3):
+            o, lse = s2.s2attn_forward(q, k, v, G)
+            s2.s2attn_backward(q, k, v, o, lse, do, G, workspace=ws)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(steps):
+            o, lse = s2.s2attn_forward(q, k, v, G)
+            s2.s2attn_backward(q, k, v, o, lse, do, G, workspace=ws)
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / steps
+
+    n = max(5, min(args.steps, 20))
+    t_s2 = timed(shape.G, n)
+    t_dense = timed(shape.N, n)
+    return {"s2_ms": t_s2, "dense_ms": t_dense, "speedup": t_dense / t_s2}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=I.LLAMA2_7B_8K.name,
+                    choices=[s.name for s in I.WORKLOADS])
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--ref-step-seconds", type=float, default=5.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--dense-ratio", action="store_true", help="also time G=N on the same inputs")
+    args = ap.parse_args()
+    shape = {s.name: s for s in I.WORKLOADS}[args.workload]
+    world, rank, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            run_reference(args, shape, world, rank)
+        else:
+            run_ours(args, shape, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -57,6 +57,8 @@ __all__ = [
     "s2_attention_bwd",
     "s2_attention_fwd_maskform",
     "s2_unit",
+    "group_suffix_attention",
+    "s2_unit_suffix",
     "s2_effective_flops",
 ]
 
@@ -275,6 +277,58 @@ def s2_unit(q, k, v, do, G: int, b: int, h: int, g: int,
         dqg, dkg, dvg, delta = group_causal_attention_grad(qg, kg, vg, dog, scale)
         out.update(dq=dqg, dk_part=dkg, dv_part=dvg, delta=delta)
     return out
+
+
+def group_suffix_attention(qg, kg, vg, dog, i0: int, scale: float):
+    """Causal attention of one group restricted to its last rows [i0, n).
+
+    Query rows i >= i0 see keys [0, i], so their o, lse and dq are exactly
+    those of the whole group; and key rows j >= i0 are seen only by query rows
+    i >= j >= i0, so dk and dv of rows [i0, n) are exact as well.  Same
+    definitions as group_causal_attention(_grad), evaluated on the
+    (n - i0) x n block of scores only.  Returns (o, lse, dq, dk, dv, delta)
+    for rows [i0, n).
+    """
+    n = qg.shape[0]
+    qs, dos = qg[i0:], dog[i0:]
+    s = scale * (qs @ kg.T)
+    vis = np.arange(n)[None, :] <= np.arange(i0, n)[:, None]
+    s = np.where(vis, s, -np.inf)
+    m = s.max(axis=1, keepdims=True)
+    e = np.exp(s - m)
+    l = e.sum(axis=1, keepdims=True)
+    p = e / l
+    o = p @ vg
+    lse = (m + np.log(l))[:, 0]
+    dp = dos @ vg.T
+    delta = np.sum(dos * o, axis=1)
+    ds = p * (dp - delta[:, None])
+    dq = scale * (ds @ kg)
+    dk = scale * (ds.T @ qs)
+    dv = p.T @ dos
+    return o, lse, dq, dk[i0:], dv[i0:], delta
+
+
+def s2_unit_suffix(q, k, v, do, G: int, b: int, h: int, g: int, m: int,
+                   scale: float | None = None):
+    """Oracle for the last m rolled rows of unit (b, h, g), at original positions.
+
+    Returns a dict like s2_unit: rows, o, lse, dq, delta, and this head's
+    contribution dk_part / dv_part to its kv-head at those rows.
+    """
+    B, N, H, D = q.shape
+    Hkv = k.shape[2]
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    s = shift_of_head(h, H, N, G)
+    kh = kv_head_of(h, H, Hkv)
+    rows_all = (np.arange(g * G, (g + 1) * G) + s) % N
+    qg = np.asarray(q[b, rows_all, h], dtype=np.float64)
+    kg = np.asarray(k[b, rows_all, kh], dtype=np.float64)
+    vg = np.asarray(v[b, rows_all, kh], dtype=np.float64)
+    dog = np.asarray(do[b, rows_all, h], dtype=np.float64)
+    o, lse, dq, dk, dv, delta = group_suffix_attention(qg, kg, vg, dog, G - m, scale)
+    return {"rows": rows_all[G - m:], "o": o, "lse": lse, "dq": dq, "dk_part": dk,
+            "dv_part": dv, "delta": delta, "kv_head": kh, "shift": s}
 
 
 def s2_effective_flops(B: int, H: int, N: int, G: int, D: int):

@@ -1,0 +1,106 @@
+"""ctypes binding of libs2attn.so: the C ABI of include/s2attn.h, same names.
+
+Argument marshalling only.  Every step of the attention runs in the library's
+CUDA kernels; there is no Python or CPU fallback: if the library is missing or
+the device is not a B200, calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libs2attn.so")
+
+S2ATTN_OK = 0
+S2ATTN_ERR_INVALID_ARG = 1
+S2ATTN_ERR_UNSUPPORTED = 2
+S2ATTN_ERR_MISALIGNED = 3
+S2ATTN_ERR_CUDA = 4
+S2ATTN_ERR_DEVICE_TIMEOUT = 5
+S2ATTN_ERR_WORKSPACE = 6
+
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+
+# name -> (restype, argtypes); mirrors include/s2attn.h
+SIGNATURES = {
+    "s2attn_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]),
+    "s2attn_bwd_workspace_bytes": (ctypes.c_size_t, [_i, _i, _i, _i, _i, _i]),
+    "s2attn_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
+                        _vp, ctypes.c_size_t, _vp]),
+    "s2attn_device_status": (_i, [_vp, _vp]),
+    "s2attn_status_string": (ctypes.c_char_p, [_i]),
+    "s2attn_selftest_wait_timeout": (_i, [_vp, ctypes.c_uint64, _vp]),
+    "s2attn_last_launch_count": (_i, []),
+    "s2attn_profile_start": (_i, [_i]),
+    "s2attn_profile_stop": (_i, [_vp, _vp, _i]),
+}
+
+_lib = None
+
+
+class S2AttnError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {status_string(status)} ({status})")
+
+
+def load() -> ctypes.CDLL:
+    """Load libs2attn.so (built in-tree).  Raises if it is missing."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing; build it with `python -m sparse_attention_attn_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return load().s2attn_status_string(int(status)).decode()
+
+
+def _check(fn: str, status: int) -> None:
+    if status != S2ATTN_OK:
+        raise S2AttnError(fn, status)
+
+
+def s2attn_fwd(q, k, v, o, lse, B, H, Hkv, N, D, G, stream) -> int:
+    """Raw C call with integer device pointers; returns the status code."""
+    return load().s2attn_fwd(q, k, v, o, lse, B, H, Hkv, N, D, G, stream)
+
+
+def s2attn_bwd_workspace_bytes(B, H, Hkv, N, D, G) -> int:
+    return load().s2attn_bwd_workspace_bytes(B, H, Hkv, N, D, G)
+
+
+def s2attn_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, Hkv, N, D, G, workspace, workspace_bytes,
+               stream) -> int:
+    return load().s2attn_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, Hkv, N, D, G, workspace,
+                             workspace_bytes, stream)
+
+
+def s2attn_device_status(workspace, stream) -> int:
+    return load().s2attn_device_status(workspace, stream)
+
+
+def s2attn_selftest_wait_timeout(status_out, limit_ns, stream) -> int:
+    return load().s2attn_selftest_wait_timeout(status_out, limit_ns, stream)
+
+
+def s2attn_last_launch_count() -> int:
+    return load().s2attn_last_launch_count()
+
+
+def s2attn_profile_start(max_launches) -> int:
+    return load().s2attn_profile_start(max_launches)
+
+
+def s2attn_profile_stop(ms, kernel_ids, capacity) -> int:
+    return load().s2attn_profile_stop(ms, kernel_ids, capacity)

@@ -1,0 +1,585 @@
+// S2-Attn backward for sm_100a.
+//
+// Analytic gradient of softmax attention inside each rolled group, with P
+// recomputed from the saved log-sum-exp (LongQLoRA community post, section 03,
+// Shift Short Attention, used in training; the gradient formulas are those of
+// plain softmax attention):
+//   dP = dO V^T,  Delta_i = sum_d dO_id O_id,  dS = P * (dP - Delta),
+//   dQ = scale dS K,  dK = scale dS^T Q,  dV = P^T dO.
+//
+// Three kernels run in order on one stream:
+//   s2_bwd_pre_kernel   Delta and lse*log2(e) per query row (HBM-bound).
+//   s2_bwd_dkdv_kernel  one CTA per 128-row kv tile of a kv-head; loops over the
+//                       kv-head's query heads and the query tiles from the
+//                       diagonal to the end of the group.  S^T = K Q^T and
+//                       dP^T = V dO^T land in TMEM, P^T and dS^T (bf16) are
+//                       written back over them and feed dV += P^T dO and
+//                       dK += dS^T Q straight from TMEM; dK/dV accumulate in
+//                       TMEM for the whole loop (no atomics).
+//   s2_bwd_dq_kernel    one CTA per 128-row query tile; loops over the kv tiles
+//                       from the group start to the diagonal: S, dP in TMEM,
+//                       dS over dP, dQ += dS K in TMEM.
+//
+// Warp roles of the two UMMA kernels (320 threads): warp 0 TMA producer,
+// warp 1 TMEM owner + UMMA issuer, warps 2..9 elementwise (thread = one TMEM
+// lane = one tile row; warps 2..5 take columns [0,64), warps 6..9 [64,128)).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "s2_common.cuh"
+#include "s2_ptx.cuh"
+
+namespace s2 {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+__device__ __forceinline__ uint4 ldg_stream(const uint4* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ float dot_bf16x2(uint32_t a, uint32_t b) {
+  const float2 fa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&a));
+  const float2 fb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&b));
+  return fmaf(fa.x, fb.x, fa.y * fb.y);
+}
+
+// ------------------------------------------------------------------ preprocess
+
+template <int D>
+__global__ void __launch_bounds__(256) s2_bwd_pre_kernel(const BwdPreArgs a) {
+  constexpr int LPR = D / 8;     // lanes per row: one 16-byte chunk each
+  constexpr int RPW = 32 / LPR;  // rows per warp per step
+  const Dims& d = a.d;
+  const long long rows = static_cast<long long>(d.B) * d.N * d.H;
+  const int lane = threadIdx.x & 31;
+  const long long warp_id = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const long long n_warps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+  const int sub = lane / LPR, part = lane % LPR;
+  const uint4* o = static_cast<const uint4*>(a.o);
+  const uint4* g = static_cast<const uint4*>(a.dO);
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    a.status[0] = 0u;
+    a.status[1] = 0u;
+  }
+  for (long long base = warp_id * RPW; base < rows; base += n_warps * RPW) {
+    const long long row = base + sub;  // (b * N + t) * H + h
+    float acc = 0.f;
+    if (row < rows) {
+      const uint4 ov = ldg_stream(o + row * (D / 8) + part);
+      const uint4 gv = ldg_stream(g + row * (D / 8) + part);
+      acc = dot_bf16x2(ov.x, gv.x) + dot_bf16x2(ov.y, gv.y) + dot_bf16x2(ov.z, gv.z) +
+            dot_bf16x2(ov.w, gv.w);
+    }
+#pragma unroll
+    for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (row < rows && part == 0) {
+      const int h = static_cast<int>(row % d.H);
+      const long long bt = row / d.H;
+      const int t = static_cast<int>(bt % d.N);
+      const int b = static_cast<int>(bt / d.N);
+      const size_t idx = (static_cast<size_t>(b) * d.H + h) * d.N + t;
+      a.delta[idx] = acc;
+      a.lse2[idx] = a.lse[idx] * kLog2e;
+    }
+  }
+}
+
+// ------------------------------------------------------------------ dK / dV
+
+template <int D>
+struct DkvCfg {
+  static constexpr int STAGES = 2;
+  static constexpr int ATOM_BYTES = kTile * 128;
+  static constexpr int TILE_BYTES = kTile * D * 2;
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = TILE_BYTES;
+  static constexpr int OFF_Q = 2 * TILE_BYTES;
+  static constexpr int OFF_DO = OFF_Q + STAGES * TILE_BYTES;
+  static constexpr int OFF_ROW = OFF_DO + STAGES * TILE_BYTES;  // per stage: lse2[128], delta[128]
+  static constexpr int SMEM_BYTES = OFF_ROW + STAGES * 1024 + 1024;
+  static constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DV = 256, TM_DK = 256 + D;
+  static constexpr int THREADS = 320;
+};
+
+// A-operand column of k-step kk when a 128-wide bf16 operand was written by
+// two warp halves into columns [0,32) and [64,96) of a 128-column region.
+__device__ __forceinline__ uint32_t split_acol(int kk) { return kk * 8 + (kk >= 4 ? 32 : 0); }
+
+template <int D>
+__global__ void __launch_bounds__(320, 1)
+    s2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmG,
+                       const BwdArgs a) {
+  using C = DkvCfg<D>;
+  constexpr int ST = C::STAGES;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  __shared__ __align__(8) uint64_t bar_kv, bar_full[ST], bar_empty[ST], bar_sdp, bar_pds, bar_done,
+      bar_drain;
+  __shared__ uint32_t tmem_slot;
+  __shared__ uint32_t abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const Dims& d = a.d;
+  const TileWork w = decode_kv_tile(d, blockIdx.x);
+  const int sh = shift_of_head(d, w.h);
+  const int tk0 = original_row(d, w.g * d.G + w.tile * kTile, sh);
+  const int nq = d.tiles - w.tile;
+  const int iters = d.rep * nq;
+  WaitCtx wc{&abort_flag, a.status, a.wait_limit_ns};
+
+  const uint32_t s0 = smem_u32(smem);
+  const uint32_t sK = s0 + C::OFF_K, sV = s0 + C::OFF_V;
+  auto sQ = [&](int s) { return s0 + C::OFF_Q + s * C::TILE_BYTES; };
+  auto sG = [&](int s) { return s0 + C::OFF_DO + s * C::TILE_BYTES; };
+  auto sRow = [&](int s) { return s0 + C::OFF_ROW + s * 1024; };
+
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(smem_u32(&bar_kv), 1);
+    for (int s = 0; s < ST; ++s) {
+      mbar_init(smem_u32(&bar_full[s]), 1);
+      mbar_init(smem_u32(&bar_empty[s]), 1);
+    }
+    mbar_init(smem_u32(&bar_sdp), 1);
+    mbar_init(smem_u32(&bar_pds), 256);
+    mbar_init(smem_u32(&bar_done), 1);
+    mbar_init(smem_u32(&bar_drain), 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      tma_prefetch_desc(&tmG);
+      mbar_arrive_expect_tx(smem_u32(&bar_kv), 2 * C::TILE_BYTES);
+      for (int c = 0; c < D / 64; ++c) {
+        tma_load_4d(sK + c * C::ATOM_BYTES, &tmK, smem_u32(&bar_kv), c * 64, w.kvh, tk0, w.b);
+        tma_load_4d(sV + c * C::ATOM_BYTES, &tmV, smem_u32(&bar_kv), c * 64, w.kvh, tk0, w.b);
+      }
+      int issued = 0;
+      for (int it = 0; it < iters; ++it) {
+        const int s = it % ST, n = it / ST;
+        if (n > 0 && !mbar_wait(smem_u32(&bar_empty[s]), (n - 1) & 1, wc, 110)) break;
+        const int h = w.kvh * d.rep + it / nq;
+        const int i = w.tile + it % nq;
+        const int tq0 = original_row(d, w.g * d.G + i * kTile, sh);
+        const uint32_t bar = smem_u32(&bar_full[s]);
+        mbar_arrive_expect_tx(bar, 2 * C::TILE_BYTES + 1024);
+        for (int c = 0; c < D / 64; ++c) {
+          tma_load_4d(sQ(s) + c * C::ATOM_BYTES, &tmQ, bar, c * 64, h, tq0, w.b);
+          tma_load_4d(sG(s) + c * C::ATOM_BYTES, &tmG, bar, c * 64, h, tq0, w.b);
+        }
+        const size_t ro = (static_cast<size_t>(w.b) * d.H + h) * d.N + tq0;
+        bulk_load(sRow(s), a.lse2 + ro, 512, bar);
+        bulk_load(sRow(s) + 512, a.delta + ro, 512, bar);
+        ++issued;
+      }
+      if (*wc.abort) {
+        drain_wait(smem_u32(&bar_kv), 0);
+        for (int s = 0; s < ST && s < issued; ++s) drain_wait(smem_u32(&bar_full[s]), ((issued - 1 - s) / ST) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idS = make_idesc_bf16(128, 128, 0, 0);  // S^T = K Q^T, dP^T = V dO^T
+      const uint32_t idG = make_idesc_bf16(128, D, 0, 1);    // dV += P^T dO, dK += dS^T Q
+      bool ok = mbar_wait(smem_u32(&bar_kv), 0, wc, 120);
+      for (int it = 0; ok && it < iters; ++it) {
+        const int s = it % ST;
+        if (!mbar_wait(smem_u32(&bar_full[s]), (it / ST) & 1, wc, 121)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::ATOM_BYTES + (kk & 3) * 32;
+          umma_ss(tmem + C::TM_S, make_sdesc_sw128(sK + off, 16, 1024),
+                  make_sdesc_sw128(sQ(s) + off, 16, 1024), idS, kk > 0);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::ATOM_BYTES + (kk & 3) * 32;
+          umma_ss(tmem + C::TM_DP, make_sdesc_sw128(sV + off, 16, 1024),
+                  make_sdesc_sw128(sG(s) + off, 16, 1024), idS, kk > 0);
+        }
+        umma_commit(smem_u32(&bar_sdp));
+        if (!mbar_wait(smem_u32(&bar_pds), it & 1, wc, 122)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_ts(tmem + C::TM_DV, tmem + C::TM_S + split_acol(kk),
+                  make_sdesc_sw128(sG(s) + kk * 2048, C::ATOM_BYTES, 1024), idG, (it > 0 || kk > 0));
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_ts(tmem + C::TM_DK, tmem + C::TM_DP + split_acol(kk),
+                  make_sdesc_sw128(sQ(s) + kk * 2048, C::ATOM_BYTES, 1024), idG, (it > 0 || kk > 0));
+        umma_commit(smem_u32(&bar_empty[s]));
+      }
+      umma_commit(smem_u32(&bar_done));
+      umma_commit(smem_u32(&bar_drain));
+      drain_wait(smem_u32(&bar_drain), 0);
+    }
+  } else {
+    const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const int row = quarter * 32 + lane;  // kv row inside the tile
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const float sl2 = a.scale_log2;
+    bool ok = true;
+    for (int it = 0; it < iters; ++it) {
+      const int s = it % ST;
+      const int i = w.tile + it % nq;
+      if (lane == 0)
+        ok = mbar_wait(smem_u32(&bar_full[s]), (it / ST) & 1, wc, 130) &&
+             mbar_wait(smem_u32(&bar_sdp), it & 1, wc, 131);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      tc_fence_after();
+      const float* lrow = reinterpret_cast<const float*>(smem + C::OFF_ROW + s * 1024) + half * 64;
+      const float* drow = lrow + 128;
+      uint32_t sr[2][32];
+      tmem_ld32(tmem + lane_off + C::TM_S + half * 64, sr[0]);
+      tmem_ld32(tmem + lane_off + C::TM_S + half * 64 + 32, sr[1]);
+      tmem_wait_ld();
+      const bool diag = (i == w.tile);
+      float p[64];
+      uint32_t pk[32];
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        float v = ex2_approx(fmaf(__uint_as_float(sr[c >> 5][c & 31]), sl2, -lrow[c]));
+        if (diag && half * 64 + c < row) v = 0.f;  // query before key in rolled order
+        p[c] = v;
+      }
+#pragma unroll
+      for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(p[2 * c], p[2 * c + 1]);
+      tmem_st32(tmem + lane_off + C::TM_S + half * 64, pk);
+      uint32_t dr[2][32];
+      tmem_ld32(tmem + lane_off + C::TM_DP + half * 64, dr[0]);
+      tmem_ld32(tmem + lane_off + C::TM_DP + half * 64 + 32, dr[1]);
+      tmem_wait_ld();
+      uint32_t dk[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        const float a0 = p[2 * c] * (__uint_as_float(dr[(2 * c) >> 5][(2 * c) & 31]) - drow[2 * c]);
+        const float a1 =
+            p[2 * c + 1] * (__uint_as_float(dr[(2 * c + 1) >> 5][(2 * c + 1) & 31]) - drow[2 * c + 1]);
+        dk[c] = pack_bf16x2(a0, a1);
+      }
+      tmem_st32(tmem + lane_off + C::TM_DP + half * 64, dk);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(smem_u32(&bar_pds));
+    }
+    if (ok) {
+      if (lane == 0) ok = mbar_wait(smem_u32(&bar_done), 0, wc, 132);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+    }
+    if (ok) {
+      tc_fence_after();
+      const size_t grow = (static_cast<size_t>(w.b) * d.N + tk0 + row) * d.Hkv + w.kvh;
+      __nv_bfloat16* dvrow = static_cast<__nv_bfloat16*>(a.dv) + grow * D + half * (D / 2);
+      __nv_bfloat16* dkrow = static_cast<__nv_bfloat16*>(a.dk) + grow * D + half * (D / 2);
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tmem + lane_off + C::TM_DV + half * (D / 2) + c * 32, r);
+        tmem_wait_ld();
+        uint4* dst = reinterpret_cast<uint4*>(dvrow + c * 32);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          dst[q] = make_uint4(pack_bf16x2(__uint_as_float(r[8 * q]), __uint_as_float(r[8 * q + 1])),
+                              pack_bf16x2(__uint_as_float(r[8 * q + 2]), __uint_as_float(r[8 * q + 3])),
+                              pack_bf16x2(__uint_as_float(r[8 * q + 4]), __uint_as_float(r[8 * q + 5])),
+                              pack_bf16x2(__uint_as_float(r[8 * q + 6]), __uint_as_float(r[8 * q + 7])));
+        tmem_ld32(tmem + lane_off + C::TM_DK + half * (D / 2) + c * 32, r);
+        tmem_wait_ld();
+        const float sc = a.scale;
+        dst = reinterpret_cast<uint4*>(dkrow + c * 32);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          dst[q] = make_uint4(
+              pack_bf16x2(__uint_as_float(r[8 * q]) * sc, __uint_as_float(r[8 * q + 1]) * sc),
+              pack_bf16x2(__uint_as_float(r[8 * q + 2]) * sc, __uint_as_float(r[8 * q + 3]) * sc),
+              pack_bf16x2(__uint_as_float(r[8 * q + 4]) * sc, __uint_as_float(r[8 * q + 5]) * sc),
+              pack_bf16x2(__uint_as_float(r[8 * q + 6]) * sc, __uint_as_float(r[8 * q + 7]) * sc));
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------ dQ
+
+template <int D>
+struct DqCfg {
+  static constexpr int STAGES = 2;
+  static constexpr int ATOM_BYTES = kTile * 128;
+  static constexpr int TILE_BYTES = kTile * D * 2;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_DO = TILE_BYTES;
+  static constexpr int OFF_K = 2 * TILE_BYTES;
+  static constexpr int OFF_V = OFF_K + STAGES * TILE_BYTES;
+  static constexpr int SMEM_BYTES = OFF_V + STAGES * TILE_BYTES + 1024;
+  static constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DQ = 256;
+  static constexpr int THREADS = 320;
+};
+
+template <int D>
+__global__ void __launch_bounds__(320, 1)
+    s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmG,
+                     const BwdArgs a) {
+  using C = DqCfg<D>;
+  constexpr int ST = C::STAGES;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  __shared__ __align__(8) uint64_t bar_q, bar_k[ST], bar_v[ST], bar_empty[ST], bar_sdp, bar_ds,
+      bar_done, bar_drain;
+  __shared__ uint32_t tmem_slot;
+  __shared__ uint32_t abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const Dims& d = a.d;
+  const TileWork w = decode_q_tile(d, blockIdx.x);
+  const int sh = shift_of_head(d, w.h);
+  const int tq0 = original_row(d, w.g * d.G + w.tile * kTile, sh);
+  const int nkv = w.tile + 1;
+  WaitCtx wc{&abort_flag, a.status, a.wait_limit_ns};
+
+  const uint32_t s0 = smem_u32(smem);
+  const uint32_t sQ = s0 + C::OFF_Q, sG = s0 + C::OFF_DO;
+  auto sK = [&](int s) { return s0 + C::OFF_K + s * C::TILE_BYTES; };
+  auto sV = [&](int s) { return s0 + C::OFF_V + s * C::TILE_BYTES; };
+
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(smem_u32(&bar_q), 1);
+    for (int s = 0; s < ST; ++s) {
+      mbar_init(smem_u32(&bar_k[s]), 1);
+      mbar_init(smem_u32(&bar_v[s]), 1);
+      mbar_init(smem_u32(&bar_empty[s]), 1);
+    }
+    mbar_init(smem_u32(&bar_sdp), 1);
+    mbar_init(smem_u32(&bar_ds), 256);
+    mbar_init(smem_u32(&bar_done), 1);
+    mbar_init(smem_u32(&bar_drain), 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      tma_prefetch_desc(&tmG);
+      mbar_arrive_expect_tx(smem_u32(&bar_q), 2 * C::TILE_BYTES);
+      for (int c = 0; c < D / 64; ++c) {
+        tma_load_4d(sQ + c * C::ATOM_BYTES, &tmQ, smem_u32(&bar_q), c * 64, w.h, tq0, w.b);
+        tma_load_4d(sG + c * C::ATOM_BYTES, &tmG, smem_u32(&bar_q), c * 64, w.h, tq0, w.b);
+      }
+      int issued = 0;
+      for (int j = 0; j < nkv; ++j) {
+        const int s = j % ST, n = j / ST;
+        if (n > 0 && !mbar_wait(smem_u32(&bar_empty[s]), (n - 1) & 1, wc, 210)) break;
+        const int tk0 = original_row(d, w.g * d.G + j * kTile, sh);
+        mbar_arrive_expect_tx(smem_u32(&bar_k[s]), C::TILE_BYTES);
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_4d(sK(s) + c * C::ATOM_BYTES, &tmK, smem_u32(&bar_k[s]), c * 64, w.kvh, tk0, w.b);
+        mbar_arrive_expect_tx(smem_u32(&bar_v[s]), C::TILE_BYTES);
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_4d(sV(s) + c * C::ATOM_BYTES, &tmV, smem_u32(&bar_v[s]), c * 64, w.kvh, tk0, w.b);
+        ++issued;
+      }
+      if (*wc.abort) {
+        drain_wait(smem_u32(&bar_q), 0);
+        for (int s = 0; s < ST && s < issued; ++s) {
+          const int last = (issued - 1 - s) / ST;
+          drain_wait(smem_u32(&bar_k[s]), last & 1);
+          drain_wait(smem_u32(&bar_v[s]), last & 1);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idS = make_idesc_bf16(128, 128, 0, 0);  // S = Q K^T, dP = dO V^T
+      const uint32_t idQ = make_idesc_bf16(128, D, 0, 1);    // dQ += dS K (K MN-major)
+      bool ok = mbar_wait(smem_u32(&bar_q), 0, wc, 220);
+      for (int j = 0; ok && j < nkv; ++j) {
+        const int s = j % ST;
+        if (!mbar_wait(smem_u32(&bar_k[s]), (j / ST) & 1, wc, 221)) break;
+        if (!mbar_wait(smem_u32(&bar_v[s]), (j / ST) & 1, wc, 222)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::ATOM_BYTES + (kk & 3) * 32;
+          umma_ss(tmem + C::TM_S, make_sdesc_sw128(sQ + off, 16, 1024),
+                  make_sdesc_sw128(sK(s) + off, 16, 1024), idS, kk > 0);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::ATOM_BYTES + (kk & 3) * 32;
+          umma_ss(tmem + C::TM_DP, make_sdesc_sw128(sG + off, 16, 1024),
+                  make_sdesc_sw128(sV(s) + off, 16, 1024), idS, kk > 0);
+        }
+        umma_commit(smem_u32(&bar_sdp));
+        if (!mbar_wait(smem_u32(&bar_ds), j & 1, wc, 223)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_ts(tmem + C::TM_DQ, tmem + C::TM_DP + split_acol(kk),
+                  make_sdesc_sw128(sK(s) + kk * 2048, C::ATOM_BYTES, 1024), idQ, (j > 0 || kk > 0));
+        umma_commit(smem_u32(&bar_empty[s]));
+      }
+      umma_commit(smem_u32(&bar_done));
+      umma_commit(smem_u32(&bar_drain));
+      drain_wait(smem_u32(&bar_drain), 0);
+    }
+  } else {
+    const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const int row = quarter * 32 + lane;  // query row inside the tile
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const float sl2 = a.scale_log2;
+    const int t = tq0 + row;
+    const size_t ridx = (static_cast<size_t>(w.b) * d.H + w.h) * d.N + t;
+    const float lse2 = a.lse2[ridx];
+    const float delta = a.delta[ridx];
+    bool ok = true;
+    for (int j = 0; j < nkv; ++j) {
+      if (lane == 0) ok = mbar_wait(smem_u32(&bar_sdp), j & 1, wc, 230);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sr[2][32], dr[2][32];
+      tmem_ld32(tmem + lane_off + C::TM_S + half * 64, sr[0]);
+      tmem_ld32(tmem + lane_off + C::TM_S + half * 64 + 32, sr[1]);
+      tmem_ld32(tmem + lane_off + C::TM_DP + half * 64, dr[0]);
+      tmem_ld32(tmem + lane_off + C::TM_DP + half * 64 + 32, dr[1]);
+      tmem_wait_ld();
+      const bool diag = (j == nkv - 1);
+      uint32_t pk[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        float v0 = ex2_approx(fmaf(__uint_as_float(sr[(2 * c) >> 5][(2 * c) & 31]), sl2, -lse2));
+        float v1 = ex2_approx(fmaf(__uint_as_float(sr[(2 * c + 1) >> 5][(2 * c + 1) & 31]), sl2, -lse2));
+        if (diag && half * 64 + 2 * c > row) v0 = 0.f;  // key after query in rolled order
+        if (diag && half * 64 + 2 * c + 1 > row) v1 = 0.f;
+        v0 *= __uint_as_float(dr[(2 * c) >> 5][(2 * c) & 31]) - delta;
+        v1 *= __uint_as_float(dr[(2 * c + 1) >> 5][(2 * c + 1) & 31]) - delta;
+        pk[c] = pack_bf16x2(v0, v1);
+      }
+      tmem_st32(tmem + lane_off + C::TM_DP + half * 64, pk);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(smem_u32(&bar_ds));
+    }
+    if (ok) {
+      if (lane == 0) ok = mbar_wait(smem_u32(&bar_done), 0, wc, 232);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+    }
+    if (ok) {
+      tc_fence_after();
+      __nv_bfloat16* dqrow = static_cast<__nv_bfloat16*>(a.dq) +
+                             ((static_cast<size_t>(w.b) * d.N + t) * d.H + w.h) * D + half * (D / 2);
+      const float sc = a.scale;
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tmem + lane_off + C::TM_DQ + half * (D / 2) + c * 32, r);
+        tmem_wait_ld();
+        uint4* dst = reinterpret_cast<uint4*>(dqrow + c * 32);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          dst[q] = make_uint4(
+              pack_bf16x2(__uint_as_float(r[8 * q]) * sc, __uint_as_float(r[8 * q + 1]) * sc),
+              pack_bf16x2(__uint_as_float(r[8 * q + 2]) * sc, __uint_as_float(r[8 * q + 3]) * sc),
+              pack_bf16x2(__uint_as_float(r[8 * q + 4]) * sc, __uint_as_float(r[8 * q + 5]) * sc),
+              pack_bf16x2(__uint_as_float(r[8 * q + 6]) * sc, __uint_as_float(r[8 * q + 7]) * sc));
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------ launchers
+
+static bool set_smem_attr(const void* fn, int bytes) {
+  return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
+}
+
+template <int D>
+cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const CUtensorMap& tg, const BwdPreArgs& pre, const BwdArgs& a, int num_sms,
+                       cudaStream_t stream, int* launches) {
+  using K3 = DkvCfg<D>;
+  using K4 = DqCfg<D>;
+  if (!set_smem_attr(reinterpret_cast<const void*>(s2_bwd_dkdv_kernel<D>), K3::SMEM_BYTES) ||
+      !set_smem_attr(reinterpret_cast<const void*>(s2_bwd_dq_kernel<D>), K4::SMEM_BYTES))
+    return cudaErrorInvalidValue;
+  const long long rows = static_cast<long long>(a.d.B) * a.d.N * a.d.H;
+  const long long want = (rows * (D / 8) + 255) / 256;
+  const int pre_grid = static_cast<int>(want < 16LL * num_sms ? want : 16LL * num_sms);
+  prof_before(stream, kKernelBwdPre);
+  s2_bwd_pre_kernel<D><<<pre_grid, 256, 0, stream>>>(pre);
+  cudaError_t e = cudaGetLastError();
+  prof_after(stream);
+  if (e != cudaSuccess) return e;
+  const int grid_kv = a.d.B * a.d.Hkv * a.d.n_groups * a.d.tiles;
+  prof_before(stream, kKernelBwdDkDv);
+  s2_bwd_dkdv_kernel<D><<<grid_kv, K3::THREADS, K3::SMEM_BYTES, stream>>>(tq, tk, tv, tg, a);
+  e = cudaGetLastError();
+  prof_after(stream);
+  if (e != cudaSuccess) return e;
+  const int grid_q = a.d.B * a.d.H * a.d.n_groups * a.d.tiles;
+  prof_before(stream, kKernelBwdDq);
+  s2_bwd_dq_kernel<D><<<grid_q, K4::THREADS, K4::SMEM_BYTES, stream>>>(tq, tk, tv, tg, a);
+  e = cudaGetLastError();
+  prof_after(stream);
+  if (launches) *launches = 3;
+  return e;
+}
+
+template cudaError_t launch_bwd<64>(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
+                                    const CUtensorMap&, const BwdPreArgs&, const BwdArgs&, int,
+                                    cudaStream_t, int*);
+template cudaError_t launch_bwd<128>(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
+                                     const CUtensorMap&, const BwdPreArgs&, const BwdArgs&, int,
+                                     cudaStream_t, int*);
+
+}  // namespace s2

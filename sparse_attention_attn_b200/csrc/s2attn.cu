@@ -1,0 +1,365 @@
+// Host side of the C ABI declared in include/s2attn.h: argument validation,
+// TMA tensor-map encoding, kernel launches and status reporting.
+//
+// Nothing here allocates device memory: every buffer belongs to the caller.
+// The only library-owned device state is the forward's status block, a
+// file-scope __device__ array.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstdlib>
+#include <mutex>
+#include <vector>
+
+#include "s2_common.cuh"
+#include "s2_ptx.cuh"
+#include "s2attn.h"
+
+namespace s2 {
+template <int D>
+cudaError_t launch_fwd(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const FwdArgs&,
+                       cudaStream_t);
+template <int D>
+cudaError_t launch_bwd(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
+                       const BwdPreArgs&, const BwdArgs&, int, cudaStream_t, int*);
+}  // namespace s2
+
+namespace {
+
+using namespace s2;
+
+__device__ uint32_t g_fwd_status[4];  // [0] error code, [1] where
+
+thread_local int g_last_launches = 0;
+
+constexpr size_t kStatusBytes = 256;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// Per-device facts cached on first use: is it sm_100, how many SMs.
+struct DeviceInfo {
+  bool ok = false;
+  int sms = 0;
+};
+
+bool device_info(DeviceInfo* out) {
+  static std::mutex mu;
+  static DeviceInfo cache[64];
+  static bool known[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!known[dev]) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return false;
+    cache[dev].ok = (major == 10 && minor == 0);
+    cache[dev].sms = sms;
+    known[dev] = true;
+  }
+  *out = cache[dev];
+  return true;
+}
+
+unsigned long long wait_limit_ns() {
+  static unsigned long long v = [] {
+    const char* e = std::getenv("S2ATTN_WAIT_LIMIT_MS");
+    long long ms = e ? std::atoll(e) : 2000;
+    if (ms <= 0) ms = 2000;
+    return static_cast<unsigned long long>(ms) * 1000000ull;
+  }();
+  return v;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Shape rules shared by forward and backward.  Pure host logic: no CUDA call.
+int validate_shape(int B, int H, int Hkv, int N, int D, int G) {
+  if (B <= 0 || H <= 0 || Hkv <= 0 || N <= 0 || D <= 0 || G <= 0) return S2ATTN_ERR_INVALID_ARG;
+  if (H % Hkv != 0 || G > N || N % G != 0) return S2ATTN_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return S2ATTN_ERR_UNSUPPORTED;
+  if (N % kTile != 0 || G % kTile != 0) return S2ATTN_ERR_UNSUPPORTED;
+  if (G < N) {
+    if (G % (2 * kTile) != 0) return S2ATTN_ERR_UNSUPPORTED;
+    if ((H / 2) % (H / Hkv) != 0) return S2ATTN_ERR_UNSUPPORTED;
+  }
+  // grid sizes and element offsets stay well inside 32/64-bit ranges
+  const long long q_tiles = static_cast<long long>(B) * H * (N / kTile);
+  if (q_tiles > (1LL << 30)) return S2ATTN_ERR_UNSUPPORTED;
+  if (static_cast<long long>(N) * H * D >= (1LL << 40)) return S2ATTN_ERR_UNSUPPORTED;
+  return S2ATTN_OK;
+}
+
+Dims make_dims(int B, int H, int Hkv, int N, int D, int G) {
+  Dims d;
+  d.B = B;
+  d.H = H;
+  d.Hkv = Hkv;
+  d.N = N;
+  d.D = D;
+  d.G = G;
+  d.rep = H / Hkv;
+  d.n_groups = N / G;
+  d.tiles = G / kTile;
+  return d;
+}
+
+// 4-D view {D, heads, N, B} of a bf16 [B, N, heads, D] tensor; box = one
+// 128-row x 64-column slab, 128-byte swizzle (the UMMA operand layout).
+bool make_map(CUtensorMap* m, const void* base, int B, int N, int heads, int D) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(heads),
+                        static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(B)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(heads) * D * 2,
+                           static_cast<cuuint64_t>(N) * heads * D * 2};
+  cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(kTile), 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+size_t rowstat_bytes(int B, int H, int N) {
+  return round_up(static_cast<size_t>(B) * H * N * sizeof(float), 256);
+}
+
+__global__ void s2_selftest_wait_kernel(uint32_t* status, unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ uint32_t abort_flag;
+  if (threadIdx.x == 0) {
+    status[0] = 0;
+    status[1] = 0;
+    abort_flag = 0;
+    mbar_init(smem_u32(&bar), 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    WaitCtx wc{&abort_flag, status, limit_ns};
+    mbar_wait(smem_u32(&bar), 0, wc, 999);  // nothing ever arrives: runs out, records, returns
+  }
+}
+
+// Per-host-thread launch timing.  Events are created once by
+// s2attn_profile_start and reused; no device memory is involved.
+struct ProfRecord {
+  cudaEvent_t start, stop;
+  int kernel;
+};
+struct ProfState {
+  bool on = false;
+  std::vector<ProfRecord> recs;
+  size_t used = 0;
+};
+thread_local ProfState g_prof;
+
+}  // namespace
+
+namespace s2 {
+void prof_before(cudaStream_t stream, int kernel_id) {
+  if (!g_prof.on || g_prof.used >= g_prof.recs.size()) return;
+  ProfRecord& r = g_prof.recs[g_prof.used];
+  r.kernel = kernel_id;
+  cudaEventRecord(r.start, stream);
+}
+void prof_after(cudaStream_t stream) {
+  if (!g_prof.on || g_prof.used >= g_prof.recs.size()) return;
+  cudaEventRecord(g_prof.recs[g_prof.used].stop, stream);
+  ++g_prof.used;
+}
+}  // namespace s2
+
+extern "C" {
+
+int s2attn_profile_start(int max_launches) {
+  if (max_launches <= 0 || max_launches > (1 << 20)) return S2ATTN_ERR_INVALID_ARG;
+  for (ProfRecord& r : g_prof.recs) {
+    cudaEventDestroy(r.start);
+    cudaEventDestroy(r.stop);
+  }
+  g_prof.recs.clear();
+  g_prof.used = 0;
+  g_prof.on = false;
+  for (int i = 0; i < max_launches; ++i) {
+    ProfRecord r{nullptr, nullptr, -1};
+    if (cudaEventCreate(&r.start) != cudaSuccess || cudaEventCreate(&r.stop) != cudaSuccess)
+      return S2ATTN_ERR_CUDA;
+    g_prof.recs.push_back(r);
+  }
+  g_prof.on = true;
+  return S2ATTN_OK;
+}
+
+int s2attn_profile_stop(float* ms, int* kernel_ids, int capacity) {
+  if (!g_prof.on) return 0;
+  g_prof.on = false;
+  const int n = static_cast<int>(g_prof.used);
+  int out = 0;
+  for (int i = 0; i < n && out < capacity; ++i) {
+    float t = 0.f;
+    if (cudaEventSynchronize(g_prof.recs[i].stop) != cudaSuccess ||
+        cudaEventElapsedTime(&t, g_prof.recs[i].start, g_prof.recs[i].stop) != cudaSuccess)
+      return -S2ATTN_ERR_CUDA;
+    if (ms) ms[out] = t;
+    if (kernel_ids) kernel_ids[out] = g_prof.recs[i].kernel;
+    ++out;
+  }
+  g_prof.used = 0;
+  return out;
+}
+
+
+const char* s2attn_status_string(int status) {
+  switch (status) {
+    case S2ATTN_OK: return "S2ATTN_OK";
+    case S2ATTN_ERR_INVALID_ARG: return "S2ATTN_ERR_INVALID_ARG";
+    case S2ATTN_ERR_UNSUPPORTED: return "S2ATTN_ERR_UNSUPPORTED";
+    case S2ATTN_ERR_MISALIGNED: return "S2ATTN_ERR_MISALIGNED";
+    case S2ATTN_ERR_CUDA: return "S2ATTN_ERR_CUDA";
+    case S2ATTN_ERR_DEVICE_TIMEOUT: return "S2ATTN_ERR_DEVICE_TIMEOUT";
+    case S2ATTN_ERR_WORKSPACE: return "S2ATTN_ERR_WORKSPACE";
+    default: return "S2ATTN_UNKNOWN_STATUS";
+  }
+}
+
+int s2attn_last_launch_count(void) { return g_last_launches; }
+
+size_t s2attn_bwd_workspace_bytes(int B, int H, int Hkv, int N, int D, int G) {
+  if (validate_shape(B, H, Hkv, N, D, G) != S2ATTN_OK) return 0;
+  return kStatusBytes + 2 * rowstat_bytes(B, H, N);
+}
+
+int s2attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+               int Hkv, int N, int D, int G, s2attn_stream_t stream) {
+  g_last_launches = 0;
+  if (!q || !k || !v || !o || !lse) return S2ATTN_ERR_INVALID_ARG;
+  int st = validate_shape(B, H, Hkv, N, D, G);
+  if (st != S2ATTN_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return S2ATTN_ERR_MISALIGNED;
+  DeviceInfo info;
+  if (!device_info(&info)) return S2ATTN_ERR_CUDA;
+  if (!info.ok) return S2ATTN_ERR_UNSUPPORTED;
+  CUtensorMap tq, tk, tv;
+  if (!make_map(&tq, q, B, N, H, D) || !make_map(&tk, k, B, N, Hkv, D) ||
+      !make_map(&tv, v, B, N, Hkv, D))
+    return S2ATTN_ERR_CUDA;
+  FwdArgs a;
+  a.d = make_dims(B, H, Hkv, N, D, G);
+  a.scale_log2 = static_cast<float>(1.4426950408889634 / __builtin_sqrt(static_cast<double>(D)));
+  a.o = o;
+  a.lse = lse;
+  void* status = nullptr;
+  if (cudaGetSymbolAddress(&status, g_fwd_status) != cudaSuccess) return S2ATTN_ERR_CUDA;
+  a.status = static_cast<uint32_t*>(status);
+  a.wait_limit_ns = wait_limit_ns();
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = (D == 64) ? launch_fwd<64>(tq, tk, tv, a, s) : launch_fwd<128>(tq, tk, tv, a, s);
+  if (e != cudaSuccess) return S2ATTN_ERR_CUDA;
+  g_last_launches = 1;
+  return S2ATTN_OK;
+}
+
+int s2attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+               const void* dO, void* dq, void* dk, void* dv, int B, int H, int Hkv, int N, int D,
+               int G, void* workspace, size_t workspace_bytes, s2attn_stream_t stream) {
+  g_last_launches = 0;
+  if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return S2ATTN_ERR_INVALID_ARG;
+  int st = validate_shape(B, H, Hkv, N, D, G);
+  if (st != S2ATTN_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+      !aligned16(dO) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return S2ATTN_ERR_MISALIGNED;
+  const size_t need = s2attn_bwd_workspace_bytes(B, H, Hkv, N, D, G);
+  if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return S2ATTN_ERR_WORKSPACE;
+  DeviceInfo info;
+  if (!device_info(&info)) return S2ATTN_ERR_CUDA;
+  if (!info.ok) return S2ATTN_ERR_UNSUPPORTED;
+  CUtensorMap tq, tk, tv, tg;
+  if (!make_map(&tq, q, B, N, H, D) || !make_map(&tk, k, B, N, Hkv, D) ||
+      !make_map(&tv, v, B, N, Hkv, D) || !make_map(&tg, dO, B, N, H, D))
+    return S2ATTN_ERR_CUDA;
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws);
+  float* delta = reinterpret_cast<float*>(ws + kStatusBytes);
+  float* lse2 = reinterpret_cast<float*>(ws + kStatusBytes + rowstat_bytes(B, H, N));
+  const Dims d = make_dims(B, H, Hkv, N, D, G);
+  BwdPreArgs pre;
+  pre.d = d;
+  pre.o = o;
+  pre.dO = dO;
+  pre.lse = lse;
+  pre.delta = delta;
+  pre.lse2 = lse2;
+  pre.status = status;
+  BwdArgs a;
+  a.d = d;
+  a.scale = static_cast<float>(1.0 / __builtin_sqrt(static_cast<double>(D)));
+  a.scale_log2 = static_cast<float>(1.4426950408889634 / __builtin_sqrt(static_cast<double>(D)));
+  a.delta = delta;
+  a.lse2 = lse2;
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  a.status = status;
+  a.wait_limit_ns = wait_limit_ns();
+  int launches = 0;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = (D == 64) ? launch_bwd<64>(tq, tk, tv, tg, pre, a, info.sms, s, &launches)
+                            : launch_bwd<128>(tq, tk, tv, tg, pre, a, info.sms, s, &launches);
+  g_last_launches = launches;
+  return e == cudaSuccess ? S2ATTN_OK : S2ATTN_ERR_CUDA;
+}
+
+int s2attn_device_status(void* workspace, s2attn_stream_t stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return S2ATTN_ERR_CUDA;
+  uint32_t words[2] = {0, 0};
+  const uint32_t zero[2] = {0, 0};
+  if (workspace) {
+    if (cudaMemcpy(words, workspace, sizeof(words), cudaMemcpyDeviceToHost) != cudaSuccess ||
+        cudaMemcpy(workspace, zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+      return S2ATTN_ERR_CUDA;
+  } else {
+    if (cudaMemcpyFromSymbol(words, g_fwd_status, sizeof(words)) != cudaSuccess ||
+        cudaMemcpyToSymbol(g_fwd_status, zero, sizeof(zero)) != cudaSuccess)
+      return S2ATTN_ERR_CUDA;
+  }
+  return words[0] == 0 ? S2ATTN_OK : static_cast<int>(words[0]);
+}
+
+int s2attn_selftest_wait_timeout(uint32_t* status_out, uint64_t limit_ns, s2attn_stream_t stream) {
+  if (!status_out || limit_ns == 0 || limit_ns > 10000000000ull) return S2ATTN_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(status_out) & 7u) != 0) return S2ATTN_ERR_MISALIGNED;
+  DeviceInfo info;
+  if (!device_info(&info)) return S2ATTN_ERR_CUDA;
+  if (!info.ok) return S2ATTN_ERR_UNSUPPORTED;
+  s2_selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(status_out, limit_ns);
+  return cudaGetLastError() == cudaSuccess ? S2ATTN_OK : S2ATTN_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,140 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+* a sweep of small shapes, whole tensors compared element by element;
+* the five workload shapes and the dense (G = N) runs at full size, in the
+  launch configuration the benchmark times, compared on sampled units: the last
+  rows of a rolled group (the rows with the most keys; for shifted heads the
+  wrap-around group), where the oracle's o, lse, dq and dk/dv are exact.
+
+Tolerances: O max-abs 1e-2 and relative Frobenius 5e-3; dQ, dK, dV relative
+Frobenius 1e-2 (bf16 inputs and outputs, fp32 accumulation).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle.s2_ref as ref
+from sparse_attention_attn_b200 import inputs as I
+from tests.parity_util import check_grad, check_o, max_abs, to64
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(shape: I.Shape, seed_offset=0):
+    import sparse_attention_attn_b200 as s2
+    q, k, v, do = I.make_inputs(shape, seed_offset)
+    dev = torch.device("cuda:0")
+    qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
+    o, lse = s2.s2attn_forward(qd, kd, vd, shape.G)
+    dq, dk, dv = s2.s2attn_backward(qd, kd, vd, o, lse, dod, shape.G)
+    assert s2.device_status() == 0
+    torch.cuda.synchronize()
+    return (q, k, v, do), (o, lse, dq, dk, dv)
+
+
+SMALL = [
+    # (B, N, H, Hkv, D, G)
+    (1, 1024, 4, 4, 64, 256),     # the tiny workload shape
+    (1, 128, 1, 1, 64, 128),      # one tile, dense
+    (2, 512, 4, 2, 128, 256),     # GQA, shifted, two batches
+    (1, 1024, 4, 1, 128, 1024),   # dense, one kv-head
+    (1, 768, 6, 2, 64, 256),      # three query heads per kv-head, shifted
+    (1, 512, 2, 2, 128, 512),     # dense, 4 tiles
+    (1, 1024, 8, 4, 128, 512),    # shifted GQA, D=128
+    (1, 512, 1, 1, 64, 256),      # H=1: every head shifted
+    (1, 2048, 2, 2, 128, 2048),   # dense causal, 16 tiles
+    (2, 1536, 4, 4, 64, 768),     # G/2 = 384: three-tile shift
+]
+
+
+@pytest.mark.parametrize("B,N,H,Hkv,D,G", SMALL)
+def test_small_whole_tensor(B, N, H, Hkv, D, G):
+    shape = I.Shape("small", B, H, Hkv, D, N, G)
+    (q, k, v, do), (o, lse, dq, dk, dv) = _run(shape, seed_offset=7)
+    q64, k64, v64, do64 = (to64(t) for t in (q, k, v, do))
+    o_ref, lse_ref = ref.s2_attention_fwd(q64, k64, v64, G)
+    dq_ref, dk_ref, dv_ref, _ = ref.s2_attention_bwd(q64, k64, v64, do64, G)
+    check_o(to64(o), o_ref)
+    assert max_abs(to64(lse), lse_ref) < 1e-3
+    check_grad("dQ", to64(dq), dq_ref)
+    check_grad("dK", to64(dk), dk_ref)
+    check_grad("dV", to64(dv), dv_ref)
+
+
+def _units(shape: I.Shape):
+    """Sampled (b, h, g) units: an unshifted head's first group, the last head's
+    last group (the wrap-around group when shifted), and a middle one."""
+    ng = shape.N // shape.G
+    units = [(0, 0, 0), (shape.B - 1, shape.H - 1, ng - 1)]
+    if shape.H > 2:
+        units.append((0, shape.H // 2, ng // 2))
+    return units
+
+
+def _check_full_size(shape: I.Shape, m: int):
+    (q, k, v, do), (o, lse, dq, dk, dv) = _run(shape)
+    o, lse, dq, dk, dv = (t.cpu() for t in (o, lse, dq, dk, dv))
+    rep = shape.H // shape.Hkv
+    msgs = []
+    for b, h, g in _units(shape):
+        u = ref.s2_unit_suffix(q, k, v, do, shape.G, b, h, g, m)
+        rows = u["rows"]
+        msgs.append(check_o(to64(o[b, rows, h]), u["o"], f"[b{b} h{h} g{g}]"))
+        assert max_abs(to64(lse[b, h, rows]), u["lse"]) < 1e-3
+        msgs.append(check_grad("dQ", to64(dq[b, rows, h]), u["dq"], f"[b{b} h{h} g{g}]"))
+        kh = u["kv_head"]
+        dk_ref = np.zeros_like(u["dk_part"])
+        dv_ref = np.zeros_like(u["dv_part"])
+        for h2 in range(kh * rep, (kh + 1) * rep):
+            u2 = u if h2 == h else ref.s2_unit_suffix(q, k, v, do, shape.G, b, h2, g, m)
+            assert np.array_equal(u2["rows"], rows)
+            dk_ref += u2["dk_part"]
+            dv_ref += u2["dv_part"]
+        msgs.append(check_grad("dK", to64(dk[b, rows, kh]), dk_ref, f"[b{b} kvh{kh} g{g}]"))
+        msgs.append(check_grad("dV", to64(dv[b, rows, kh]), dv_ref, f"[b{b} kvh{kh} g{g}]"))
+    print("\n".join(msgs))
+
+
+@pytest.mark.parametrize("shape", I.WORKLOADS[:4], ids=lambda s: s.name)
+def test_workload_sampled(shape):
+    _check_full_size(shape, m=min(shape.G, 2048))
+
+
+@pytest.mark.slow
+def test_workload_100k_sampled():
+    _check_full_size(I.LLAMA2_7B_100K, m=1024)
+
+
+@pytest.mark.parametrize("shape", [I.LLAMA2_7B_8K.dense()], ids=lambda s: s.name)
+def test_dense_sampled(shape):
+    _check_full_size(shape, m=1024)
+
+
+@pytest.mark.slow
+def test_dense_100k_sampled():
+    _check_full_size(I.LLAMA2_7B_100K.dense(), m=512)
+
+
+def test_launch_counts():
+    from sparse_attention_attn_b200 import _lib
+    import sparse_attention_attn_b200 as s2
+    shape = I.Shape("lc", 1, 2, 2, 64, 256, 128)
+    q, k, v, do = (t.cuda() for t in I.make_inputs(shape))
+    o, lse = s2.s2attn_forward(q, k, v, shape.G)
+    assert _lib.s2attn_last_launch_count() == 1
+    s2.s2attn_backward(q, k, v, o, lse, do, shape.G)
+    assert _lib.s2attn_last_launch_count() == 3
+
+
+def test_bounded_wait_times_out_cleanly():
+    """A wait on an mbarrier nothing arrives at gives up after its limit and
+    reports S2ATTN_ERR_DEVICE_TIMEOUT; the context stays usable."""
+    from sparse_attention_attn_b200 import _lib
+    st = torch.zeros(2, dtype=torch.int32, device="cuda")
+    rc = _lib.s2attn_selftest_wait_timeout(st.data_ptr(), 20_000_000, torch.cuda.current_stream().cuda_stream)
+    assert rc == 0
+    torch.cuda.synchronize()
+    assert int(st[0]) == _lib.S2ATTN_ERR_DEVICE_TIMEOUT and int(st[1]) == 999
+    # the context still works afterwards
+    x = torch.ones(1024, device="cuda")
+    assert float(x.sum()) == 1024.0

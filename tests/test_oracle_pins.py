@@ -236,6 +236,18 @@ def test_unit_matches_full():
     np.testing.assert_allclose(u["dv_part"] + u2["dv_part"], dv[1, u["rows"], 1], atol=1e-13, rtol=0)
 
 
+def test_suffix_matches_full_unit():
+    """The suffix oracle (used to sample long groups) equals the whole-group oracle on its rows."""
+    B, N, G, H, Hkv, D = 1, 64, 32, 4, 2, 6
+    q, k, v, do = _qkvdo(B, N, H, Hkv, D, seed=12)
+    for h, g in ((0, 1), (3, 1), (2, 0)):
+        full = ref.s2_unit(q, k, v, do, G, b=0, h=h, g=g)
+        suf = ref.s2_unit_suffix(q, k, v, do, G, b=0, h=h, g=g, m=12)
+        np.testing.assert_array_equal(suf["rows"], full["rows"][-12:])
+        for key in ("o", "lse", "dq", "dk_part", "dv_part", "delta"):
+            np.testing.assert_allclose(suf[key], full[key][-12:], rtol=0, atol=1e-12, err_msg=key)
+
+
 def test_rejects_mixed_shift_kv_head():
     q, k, v, _ = _qkvdo(1, 16, 4, 1, 4)
     with pytest.raises(ValueError):
