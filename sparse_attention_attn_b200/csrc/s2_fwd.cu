@@ -214,9 +214,8 @@ __global__ void __launch_bounds__(192, 1)
         const float p0 = ex2_approx(fmaf(__uint_as_float(sr[(2 * c) >> 5][(2 * c) & 31]), sl2, -m_run));
         const float p1 =
             ex2_approx(fmaf(__uint_as_float(sr[(2 * c + 1) >> 5][(2 * c + 1) & 31]), sl2, -m_run));
-        const uint32_t u = pack_bf16x2(p0, p1);
-        pk[c >> 5][c & 31] = u;
-        rs += __uint_as_float(u << 16) + __uint_as_float(u & 0xffff0000u);
+        pk[c >> 5][c & 31] = pack_bf16x2(p0, p1);
+        rs += p0 + p1;
       }
       l_run = l_run * alpha + rs;
       tmem_st32(tS, pk[0]);
