@@ -138,6 +138,33 @@ S2ATTN_API int s2attn_last_launch_count(void);
 S2ATTN_API int s2attn_profile_start(int max_launches);
 S2ATTN_API int s2attn_profile_stop(float* ms, int* kernel_ids, int capacity);
 
+/*
+ * Backward for callers that cannot allocate device memory (no counterpart in
+ * the papers: this is a deployment variant of s2attn_bwd).  Some callers have
+ * no way to get a workspace: they run under another runtime's memory budget
+ * without an allocator handle, inside plugin hosts that forbid cudaMalloc, or
+ * must not allocate between set-up and graph capture.  This call computes
+ * exactly what s2attn_bwd computes, with the same arguments minus the
+ * workspace, and allocates nothing: its scratch (s2attn_bwd_workspace_bytes of
+ * it) is a fixed 32 MiB device array inside the library, which every GPU that
+ * loads the library holds until the process exits.  That limits it to
+ * B * H * N <= 4194272 query rows (all five workload shapes fit); larger
+ * shapes return S2ATTN_ERR_WORKSPACE without launching anything.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current) and caches it; make that first call before any
+ *     stream capture.
+ *   - All calls share the array and it keeps the last call's contents; each
+ *     call rewrites what it reads.  Calls that overlap on the GPU (e.g. on two
+ *     streams) race on it and must be serialised by the caller.
+ *   - A bounded-wait timeout is recorded in the array's status block, which is
+ *     not readable through s2attn_device_status; use s2attn_bwd when the
+ *     device status is needed.
+ */
+S2ATTN_API int s2attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                                  const float* lse, const void* dO, void* dq, void* dk, void* dv,
+                                  int B, int H, int Hkv, int N, int D, int G,
+                                  s2attn_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

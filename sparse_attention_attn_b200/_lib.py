@@ -35,6 +35,8 @@ SIGNATURES = {
     "s2attn_last_launch_count": (_i, []),
     "s2attn_profile_start": (_i, [_i]),
     "s2attn_profile_stop": (_i, [_vp, _vp, _i]),
+    "s2attn_bwd_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
+                                _vp]),
 }
 
 _lib = None
@@ -104,3 +106,8 @@ def s2attn_profile_start(max_launches) -> int:
 
 def s2attn_profile_stop(ms, kernel_ids, capacity) -> int:
     return load().s2attn_profile_stop(ms, kernel_ids, capacity)
+
+
+def s2attn_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, B, H, Hkv, N, D, G, stream) -> int:
+    """Backward with the library's built-in scratch, for callers that cannot allocate."""
+    return load().s2attn_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, B, H, Hkv, N, D, G, stream)

@@ -363,3 +363,57 @@ int s2attn_selftest_wait_timeout(uint32_t* status_out, uint64_t limit_ns, s2attn
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Backward for callers that cannot allocate device memory.
+//
+// Some callers have no way to obtain device memory for a workspace: code that
+// runs under another runtime's memory budget with no allocator handle, plugin
+// hosts that forbid cudaMalloc, or programs that must not allocate between
+// set-up and capture.  For them the backward's scratch (status block, Delta and
+// lse*log2(e), s2attn_bwd_workspace_bytes of it) lives in this fixed array.
+// Every GPU that loads the library reserves it when the module is loaded and
+// keeps it until the process exits.  All calls share it and it keeps the last
+// call's contents; the backward's first kernel rewrites everything the later
+// kernels read (and clears the status words), so nothing needs clearing here.
+// Calls that overlap on the GPU (different streams, or devices sharing a
+// context) race on the array.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB
+static __device__ __align__(256) unsigned char g_bwd_scratch[kNoAllocScratchBytes];
+
+// Device address of g_bwd_scratch on the current device.  In host code the
+// array's name is only a host-side stand-in, so the address is looked up once
+// per device, with that device current, and cached.
+bool noalloc_scratch(void** out) {
+  static std::mutex mu;
+  static void* ptrs[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  std::lock_guard<std::mutex> lk(mu);
+  if (ptrs[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_bwd_scratch) != cudaSuccess || p == nullptr) return false;
+    ptrs[dev] = p;
+  }
+  *out = ptrs[dev];
+  return true;
+}
+
+}  // namespace
+
+extern "C" int s2attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                                  const float* lse, const void* dO, void* dq, void* dk, void* dv,
+                                  int B, int H, int Hkv, int N, int D, int G,
+                                  s2attn_stream_t stream) {
+  g_last_launches = 0;
+  const size_t need = s2attn_bwd_workspace_bytes(B, H, Hkv, N, D, G);
+  if (need > kNoAllocScratchBytes) return S2ATTN_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  // need == 0 means the shape is invalid: s2attn_bwd reports which error
+  if (need != 0 && !noalloc_scratch(&scratch)) return S2ATTN_ERR_CUDA;
+  return s2attn_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, Hkv, N, D, G, scratch,
+                    kNoAllocScratchBytes, stream);
+}
