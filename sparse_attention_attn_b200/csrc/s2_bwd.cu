@@ -89,26 +89,49 @@ __global__ void __launch_bounds__(256) s2_bwd_pre_kernel(const BwdPreArgs a) {
   }
 }
 
+// 32 fp32 values (bit patterns) times `scale` -> 32 bf16 at dst (64 bytes, 16-byte aligned).
+__device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const uint32_t (&r)[32], float scale) {
+  uint4* out = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    out[q] = make_uint4(pack_bf16x2(__uint_as_float(r[8 * q]) * scale, __uint_as_float(r[8 * q + 1]) * scale),
+                        pack_bf16x2(__uint_as_float(r[8 * q + 2]) * scale, __uint_as_float(r[8 * q + 3]) * scale),
+                        pack_bf16x2(__uint_as_float(r[8 * q + 4]) * scale, __uint_as_float(r[8 * q + 5]) * scale),
+                        pack_bf16x2(__uint_as_float(r[8 * q + 6]) * scale, __uint_as_float(r[8 * q + 7]) * scale));
+}
+
+
 // ------------------------------------------------------------------ dK / dV
+//
+// One CTA per 128-row kv tile; the query side streams in 64-row sub-tiles.
+// S^T and dP^T (128 kv rows x 64 query columns each) are double-buffered in
+// TMEM, so the UMMAs of sub-tile it+1 run while warps 2..9 turn sub-tile it
+// into P^T and dS^T.  TMEM: S^T [0,128) (two 64-column buffers), dP^T
+// [128,256), dV [256, 256+D), dK [256+D, 256+2D).
+
+constexpr int kSub = 64;  // rows of a streamed sub-tile
+
+// A-operand column of k-step kk (16 rows of K) when a 64-wide bf16 operand was
+// written by two warp halves at packed columns [0,16) and [32,48) of its
+// 64-column TMEM buffer (each half stays inside the fp32 columns it read).
+__device__ __forceinline__ uint32_t split_acol64(int kk) { return kk * 8 + (kk >= 2 ? 16 : 0); }
 
 template <int D>
 struct DkvCfg {
-  static constexpr int STAGES = 2;
-  static constexpr int ATOM_BYTES = kTile * 128;
-  static constexpr int TILE_BYTES = kTile * D * 2;
+  static constexpr int STAGES = 3;
+  static constexpr int KV_ATOM = kTile * 128;  // one 64-column slab of a 128-row tile
+  static constexpr int Q_ATOM = kSub * 128;    // one 64-column slab of a 64-row tile
+  static constexpr int KV_BYTES = kTile * D * 2;
+  static constexpr int Q_BYTES = kSub * D * 2;
   static constexpr int OFF_K = 0;
-  static constexpr int OFF_V = TILE_BYTES;
-  static constexpr int OFF_Q = 2 * TILE_BYTES;
-  static constexpr int OFF_DO = OFF_Q + STAGES * TILE_BYTES;
-  static constexpr int OFF_ROW = OFF_DO + STAGES * TILE_BYTES;  // per stage: lse2[128], delta[128]
-  static constexpr int SMEM_BYTES = OFF_ROW + STAGES * 1024 + 1024;
+  static constexpr int OFF_V = KV_BYTES;
+  static constexpr int OFF_Q = 2 * KV_BYTES;
+  static constexpr int OFF_DO = OFF_Q + STAGES * Q_BYTES;
+  static constexpr int OFF_ROW = OFF_DO + STAGES * Q_BYTES;  // per stage: lse2[64], delta[64]
+  static constexpr int SMEM_BYTES = OFF_ROW + STAGES * 512 + 1024;
   static constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DV = 256, TM_DK = 256 + D;
   static constexpr int THREADS = 320;
 };
-
-// A-operand column of k-step kk when a 128-wide bf16 operand was written by
-// two warp halves into columns [0,32) and [64,96) of a 128-column region.
-__device__ __forceinline__ uint32_t split_acol(int kk) { return kk * 8 + (kk >= 4 ? 32 : 0); }
 
 template <int D>
 __global__ void __launch_bounds__(320, 1)
@@ -120,8 +143,8 @@ __global__ void __launch_bounds__(320, 1)
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  __shared__ __align__(8) uint64_t bar_kv, bar_full[ST], bar_empty[ST], bar_sdp, bar_pds, bar_done,
-      bar_drain;
+  __shared__ __align__(8) uint64_t bar_kv, bar_full[ST], bar_empty[ST], bar_sdp[2], bar_pds[2],
+      bar_done, bar_drain;
   __shared__ uint32_t tmem_slot;
   __shared__ uint32_t abort_flag;
 
@@ -130,15 +153,15 @@ __global__ void __launch_bounds__(320, 1)
   const TileWork w = decode_kv_tile(d, blockIdx.x);
   const int sh = shift_of_head(d, w.h);
   const int tk0 = original_row(d, w.g * d.G + w.tile * kTile, sh);
-  const int nq = d.tiles - w.tile;
+  const int nq = 2 * (d.tiles - w.tile);  // 64-row query sub-tiles from the diagonal to the group end
   const int iters = d.rep * nq;
   WaitCtx wc{&abort_flag, a.status, a.wait_limit_ns};
 
   const uint32_t s0 = smem_u32(smem);
   const uint32_t sK = s0 + C::OFF_K, sV = s0 + C::OFF_V;
-  auto sQ = [&](int s) { return s0 + C::OFF_Q + s * C::TILE_BYTES; };
-  auto sG = [&](int s) { return s0 + C::OFF_DO + s * C::TILE_BYTES; };
-  auto sRow = [&](int s) { return s0 + C::OFF_ROW + s * 1024; };
+  auto sQ = [&](int s) { return s0 + C::OFF_Q + s * C::Q_BYTES; };
+  auto sG = [&](int s) { return s0 + C::OFF_DO + s * C::Q_BYTES; };
+  auto sRow = [&](int s) { return s0 + C::OFF_ROW + s * 512; };
 
   if (threadIdx.x == 0) {
     abort_flag = 0;
@@ -147,8 +170,10 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(smem_u32(&bar_full[s]), 1);
       mbar_init(smem_u32(&bar_empty[s]), 1);
     }
-    mbar_init(smem_u32(&bar_sdp), 1);
-    mbar_init(smem_u32(&bar_pds), 256);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&bar_sdp[i]), 1);
+      mbar_init(smem_u32(&bar_pds[i]), 256);
+    }
     mbar_init(smem_u32(&bar_done), 1);
     mbar_init(smem_u32(&bar_drain), 1);
     fence_barrier_init();
@@ -163,71 +188,89 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t tmem = tmem_slot;
 
   if (warp == 0) {
+    // ------------------------------------------------------------ producer
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
       tma_prefetch_desc(&tmG);
-      mbar_arrive_expect_tx(smem_u32(&bar_kv), 2 * C::TILE_BYTES);
+      mbar_arrive_expect_tx(smem_u32(&bar_kv), 2 * C::KV_BYTES);
       for (int c = 0; c < D / 64; ++c) {
-        tma_load_4d(sK + c * C::ATOM_BYTES, &tmK, smem_u32(&bar_kv), c * 64, w.kvh, tk0, w.b);
-        tma_load_4d(sV + c * C::ATOM_BYTES, &tmV, smem_u32(&bar_kv), c * 64, w.kvh, tk0, w.b);
+        tma_load_4d(sK + c * C::KV_ATOM, &tmK, smem_u32(&bar_kv), c * 64, w.kvh, tk0, w.b);
+        tma_load_4d(sV + c * C::KV_ATOM, &tmV, smem_u32(&bar_kv), c * 64, w.kvh, tk0, w.b);
       }
       int issued = 0;
       for (int it = 0; it < iters; ++it) {
         const int s = it % ST, n = it / ST;
         if (n > 0 && !mbar_wait(smem_u32(&bar_empty[s]), (n - 1) & 1, wc, 110)) break;
         const int h = w.kvh * d.rep + it / nq;
-        const int i = w.tile + it % nq;
-        const int tq0 = original_row(d, w.g * d.G + i * kTile, sh);
+        const int i64 = 2 * w.tile + it % nq;
+        const int tq0 = original_row(d, w.g * d.G + i64 * kSub, sh);
         const uint32_t bar = smem_u32(&bar_full[s]);
-        mbar_arrive_expect_tx(bar, 2 * C::TILE_BYTES + 1024);
+        mbar_arrive_expect_tx(bar, 2 * C::Q_BYTES + 512);
         for (int c = 0; c < D / 64; ++c) {
-          tma_load_4d(sQ(s) + c * C::ATOM_BYTES, &tmQ, bar, c * 64, h, tq0, w.b);
-          tma_load_4d(sG(s) + c * C::ATOM_BYTES, &tmG, bar, c * 64, h, tq0, w.b);
+          tma_load_4d(sQ(s) + c * C::Q_ATOM, &tmQ, bar, c * 64, h, tq0, w.b);
+          tma_load_4d(sG(s) + c * C::Q_ATOM, &tmG, bar, c * 64, h, tq0, w.b);
         }
         const size_t ro = (static_cast<size_t>(w.b) * d.H + h) * d.N + tq0;
-        bulk_load(sRow(s), a.lse2 + ro, 512, bar);
-        bulk_load(sRow(s) + 512, a.delta + ro, 512, bar);
+        bulk_load(sRow(s), a.lse2 + ro, 256, bar);
+        bulk_load(sRow(s) + 256, a.delta + ro, 256, bar);
         ++issued;
       }
       if (*wc.abort) {
         drain_wait(smem_u32(&bar_kv), 0);
-        for (int s = 0; s < ST && s < issued; ++s) drain_wait(smem_u32(&bar_full[s]), ((issued - 1 - s) / ST) & 1);
+        for (int s = 0; s < ST && s < issued; ++s)
+          drain_wait(smem_u32(&bar_full[s]), ((issued - 1 - s) / ST) & 1);
       }
     }
   } else if (warp == 1) {
+    // ------------------------------------------------------------ UMMA issuer
     if (lane == 0) {
-      const uint32_t idS = make_idesc_bf16(128, 128, 0, 0);  // S^T = K Q^T, dP^T = V dO^T
-      const uint32_t idG = make_idesc_bf16(128, D, 0, 1);    // dV += P^T dO, dK += dS^T Q
-      bool ok = mbar_wait(smem_u32(&bar_kv), 0, wc, 120);
+      const uint32_t idS = make_idesc_bf16(128, kSub, 0, 0);  // S^T = K Q^T, dP^T = V dO^T
+      const uint32_t idG = make_idesc_bf16(128, D, 0, 1);     // dV += P^T dO, dK += dS^T Q
+      auto issue_sdp = [&](int it, int s) {
+        const uint32_t bo = (it & 1) * kSub;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t ko = (kk >> 2) * C::KV_ATOM + (kk & 3) * 32;
+          const uint32_t qo = (kk >> 2) * C::Q_ATOM + (kk & 3) * 32;
+          umma_ss(tmem + C::TM_S + bo, make_sdesc_sw128(sK + ko, 16, 1024),
+                  make_sdesc_sw128(sQ(s) + qo, 16, 1024), idS, kk > 0);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t ko = (kk >> 2) * C::KV_ATOM + (kk & 3) * 32;
+          const uint32_t qo = (kk >> 2) * C::Q_ATOM + (kk & 3) * 32;
+          umma_ss(tmem + C::TM_DP + bo, make_sdesc_sw128(sV + ko, 16, 1024),
+                  make_sdesc_sw128(sG(s) + qo, 16, 1024), idS, kk > 0);
+        }
+        umma_commit(smem_u32(&bar_sdp[it & 1]));
+      };
+      bool ok = mbar_wait(smem_u32(&bar_kv), 0, wc, 120) &&
+                (iters == 0 || mbar_wait(smem_u32(&bar_full[0]), 0, wc, 121));
+      if (ok && iters > 0) {
+        tc_fence_after();
+        issue_sdp(0, 0);
+      }
       for (int it = 0; ok && it < iters; ++it) {
         const int s = it % ST;
-        if (!mbar_wait(smem_u32(&bar_full[s]), (it / ST) & 1, wc, 121)) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::ATOM_BYTES + (kk & 3) * 32;
-          umma_ss(tmem + C::TM_S, make_sdesc_sw128(sK + off, 16, 1024),
-                  make_sdesc_sw128(sQ(s) + off, 16, 1024), idS, kk > 0);
+        if (it + 1 < iters) {
+          const int s1 = (it + 1) % ST;
+          if (!mbar_wait(smem_u32(&bar_full[s1]), ((it + 1) / ST) & 1, wc, 122)) break;
+          tc_fence_after();
+          issue_sdp(it + 1, s1);  // its TMEM buffer's last readers were issued before: in order
         }
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::ATOM_BYTES + (kk & 3) * 32;
-          umma_ss(tmem + C::TM_DP, make_sdesc_sw128(sV + off, 16, 1024),
-                  make_sdesc_sw128(sG(s) + off, 16, 1024), idS, kk > 0);
-        }
-        umma_commit(smem_u32(&bar_sdp));
-        if (!mbar_wait(smem_u32(&bar_pds), it & 1, wc, 122)) break;
+        if (!mbar_wait(smem_u32(&bar_pds[it & 1]), (it >> 1) & 1, wc, 123)) break;
         tc_fence_after();
+        const uint32_t bo = (it & 1) * kSub;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          umma_ts(tmem + C::TM_DV, tmem + C::TM_S + split_acol(kk),
-                  make_sdesc_sw128(sG(s) + kk * 2048, C::ATOM_BYTES, 1024), idG, (it > 0 || kk > 0));
+        for (int kk = 0; kk < kSub / 16; ++kk)
+          umma_ts(tmem + C::TM_DV, tmem + C::TM_S + bo + split_acol64(kk),
+                  make_sdesc_sw128(sG(s) + kk * 2048, C::Q_ATOM, 1024), idG, (it > 0 || kk > 0));
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          umma_ts(tmem + C::TM_DK, tmem + C::TM_DP + split_acol(kk),
-                  make_sdesc_sw128(sQ(s) + kk * 2048, C::ATOM_BYTES, 1024), idG, (it > 0 || kk > 0));
+        for (int kk = 0; kk < kSub / 16; ++kk)
+          umma_ts(tmem + C::TM_DK, tmem + C::TM_DP + bo + split_acol64(kk),
+                  make_sdesc_sw128(sQ(s) + kk * 2048, C::Q_ATOM, 1024), idG, (it > 0 || kk > 0));
         umma_commit(smem_u32(&bar_empty[s]));
       }
       umma_commit(smem_u32(&bar_done));
@@ -235,6 +278,7 @@ __global__ void __launch_bounds__(320, 1)
       drain_wait(smem_u32(&bar_drain), 0);
     }
   } else {
+    // ------------------------------------------------------------ P^T, dS^T
     const int quarter = warp & 3;
     const int half = (warp - 2) >> 2;
     const int row = quarter * 32 + lane;  // kv row inside the tile
@@ -243,48 +287,52 @@ __global__ void __launch_bounds__(320, 1)
     bool ok = true;
     for (int it = 0; it < iters; ++it) {
       const int s = it % ST;
-      const int i = w.tile + it % nq;
+      const int qoff = (it % nq) * kSub;  // query sub-tile start minus kv tile start (rolled)
+      const uint32_t bo = (it & 1) * kSub + half * 32;
       if (lane == 0)
         ok = mbar_wait(smem_u32(&bar_full[s]), (it / ST) & 1, wc, 130) &&
-             mbar_wait(smem_u32(&bar_sdp), it & 1, wc, 131);
+             mbar_wait(smem_u32(&bar_sdp[it & 1]), (it >> 1) & 1, wc, 131);
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       tc_fence_after();
-      const float* lrow = reinterpret_cast<const float*>(smem + C::OFF_ROW + s * 1024) + half * 64;
-      const float* drow = lrow + 128;
-      uint32_t sr[2][32];
-      tmem_ld32(tmem + lane_off + C::TM_S + half * 64, sr[0]);
-      tmem_ld32(tmem + lane_off + C::TM_S + half * 64 + 32, sr[1]);
+      const float4* l4 = reinterpret_cast<const float4*>(smem + C::OFF_ROW + s * 512) + half * 8;
+      const float4* d4 = l4 + 16;
+      uint32_t sr[32], dr[32];
+      tmem_ld32(tmem + lane_off + C::TM_S + bo, sr);
+      tmem_ld32(tmem + lane_off + C::TM_DP + bo, dr);
       tmem_wait_ld();
-      const bool diag = (i == w.tile);
-      float p[64];
-      uint32_t pk[32];
+      float p[32];
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        float v = ex2_approx(fmaf(__uint_as_float(sr[c >> 5][c & 31]), sl2, -lrow[c]));
-        if (diag && half * 64 + c < row) v = 0.f;  // query before key in rolled order
-        p[c] = v;
+      for (int c4 = 0; c4 < 8; ++c4) {
+        const float4 l = l4[c4];
+        p[4 * c4 + 0] = ex2_approx(fmaf(__uint_as_float(sr[4 * c4 + 0]), sl2, -l.x));
+        p[4 * c4 + 1] = ex2_approx(fmaf(__uint_as_float(sr[4 * c4 + 1]), sl2, -l.y));
+        p[4 * c4 + 2] = ex2_approx(fmaf(__uint_as_float(sr[4 * c4 + 2]), sl2, -l.z));
+        p[4 * c4 + 3] = ex2_approx(fmaf(__uint_as_float(sr[4 * c4 + 3]), sl2, -l.w));
       }
+      if (qoff < kTile) {  // sub-tile overlaps the diagonal: query before key is masked
 #pragma unroll
-      for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(p[2 * c], p[2 * c + 1]);
-      tmem_st32(tmem + lane_off + C::TM_S + half * 64, pk);
-      uint32_t dr[2][32];
-      tmem_ld32(tmem + lane_off + C::TM_DP + half * 64, dr[0]);
-      tmem_ld32(tmem + lane_off + C::TM_DP + half * 64 + 32, dr[1]);
-      tmem_wait_ld();
-      uint32_t dk[32];
-#pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const float a0 = p[2 * c] * (__uint_as_float(dr[(2 * c) >> 5][(2 * c) & 31]) - drow[2 * c]);
-        const float a1 =
-            p[2 * c + 1] * (__uint_as_float(dr[(2 * c + 1) >> 5][(2 * c + 1) & 31]) - drow[2 * c + 1]);
-        dk[c] = pack_bf16x2(a0, a1);
+        for (int c = 0; c < 32; ++c)
+          if (qoff + half * 32 + c < row) p[c] = 0.f;
       }
-      tmem_st32(tmem + lane_off + C::TM_DP + half * 64, dk);
+      uint32_t pk[16], dk[16];
+#pragma unroll
+      for (int c = 0; c < 16; ++c) pk[c] = pack_bf16x2(p[2 * c], p[2 * c + 1]);
+      tmem_st16(tmem + lane_off + C::TM_S + bo, pk);
+#pragma unroll
+      for (int c4 = 0; c4 < 8; ++c4) {
+        const float4 dl = d4[c4];
+        dk[2 * c4] = pack_bf16x2(p[4 * c4] * (__uint_as_float(dr[4 * c4]) - dl.x),
+                                 p[4 * c4 + 1] * (__uint_as_float(dr[4 * c4 + 1]) - dl.y));
+        dk[2 * c4 + 1] = pack_bf16x2(p[4 * c4 + 2] * (__uint_as_float(dr[4 * c4 + 2]) - dl.z),
+                                     p[4 * c4 + 3] * (__uint_as_float(dr[4 * c4 + 3]) - dl.w));
+      }
+      tmem_st16(tmem + lane_off + C::TM_DP + bo, dk);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(smem_u32(&bar_pds));
+      mbar_arrive(smem_u32(&bar_pds[it & 1]));
     }
+    // ------------------------------------------------------------ epilogue
     if (ok) {
       if (lane == 0) ok = mbar_wait(smem_u32(&bar_done), 0, wc, 132);
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -294,29 +342,16 @@ __global__ void __launch_bounds__(320, 1)
       const size_t grow = (static_cast<size_t>(w.b) * d.N + tk0 + row) * d.Hkv + w.kvh;
       __nv_bfloat16* dvrow = static_cast<__nv_bfloat16*>(a.dv) + grow * D + half * (D / 2);
       __nv_bfloat16* dkrow = static_cast<__nv_bfloat16*>(a.dk) + grow * D + half * (D / 2);
+      const float sc = a.scale;
 #pragma unroll
       for (int c = 0; c < D / 64; ++c) {
         uint32_t r[32];
         tmem_ld32(tmem + lane_off + C::TM_DV + half * (D / 2) + c * 32, r);
         tmem_wait_ld();
-        uint4* dst = reinterpret_cast<uint4*>(dvrow + c * 32);
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-          dst[q] = make_uint4(pack_bf16x2(__uint_as_float(r[8 * q]), __uint_as_float(r[8 * q + 1])),
-                              pack_bf16x2(__uint_as_float(r[8 * q + 2]), __uint_as_float(r[8 * q + 3])),
-                              pack_bf16x2(__uint_as_float(r[8 * q + 4]), __uint_as_float(r[8 * q + 5])),
-                              pack_bf16x2(__uint_as_float(r[8 * q + 6]), __uint_as_float(r[8 * q + 7])));
+        store_row32(dvrow + c * 32, r, 1.f);
         tmem_ld32(tmem + lane_off + C::TM_DK + half * (D / 2) + c * 32, r);
         tmem_wait_ld();
-        const float sc = a.scale;
-        dst = reinterpret_cast<uint4*>(dkrow + c * 32);
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-          dst[q] = make_uint4(
-              pack_bf16x2(__uint_as_float(r[8 * q]) * sc, __uint_as_float(r[8 * q + 1]) * sc),
-              pack_bf16x2(__uint_as_float(r[8 * q + 2]) * sc, __uint_as_float(r[8 * q + 3]) * sc),
-              pack_bf16x2(__uint_as_float(r[8 * q + 4]) * sc, __uint_as_float(r[8 * q + 5]) * sc),
-              pack_bf16x2(__uint_as_float(r[8 * q + 6]) * sc, __uint_as_float(r[8 * q + 7]) * sc));
+        store_row32(dkrow + c * 32, r, sc);
       }
     }
   }
@@ -330,17 +365,24 @@ __global__ void __launch_bounds__(320, 1)
 }
 
 // ------------------------------------------------------------------ dQ
+//
+// One CTA per 128-row query tile; keys/values stream in 64-row sub-tiles from
+// the group start to the diagonal.  S and dP (128 x 64) are double-buffered in
+// TMEM so the UMMAs of sub-tile j+1 overlap the dS work on sub-tile j.
+// TMEM: S [0,128) (two buffers), dP [128,256), dQ [256, 256+D).
 
 template <int D>
 struct DqCfg {
-  static constexpr int STAGES = 2;
-  static constexpr int ATOM_BYTES = kTile * 128;
-  static constexpr int TILE_BYTES = kTile * D * 2;
+  static constexpr int STAGES = 4;
+  static constexpr int Q_ATOM = kTile * 128;
+  static constexpr int KV_ATOM = kSub * 128;
+  static constexpr int Q_BYTES = kTile * D * 2;
+  static constexpr int KV_BYTES = kSub * D * 2;
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_DO = TILE_BYTES;
-  static constexpr int OFF_K = 2 * TILE_BYTES;
-  static constexpr int OFF_V = OFF_K + STAGES * TILE_BYTES;
-  static constexpr int SMEM_BYTES = OFF_V + STAGES * TILE_BYTES + 1024;
+  static constexpr int OFF_DO = Q_BYTES;
+  static constexpr int OFF_K = 2 * Q_BYTES;
+  static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
+  static constexpr int SMEM_BYTES = OFF_V + STAGES * KV_BYTES + 1024;
   static constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DQ = 256;
   static constexpr int THREADS = 320;
 };
@@ -355,8 +397,8 @@ __global__ void __launch_bounds__(320, 1)
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  __shared__ __align__(8) uint64_t bar_q, bar_k[ST], bar_v[ST], bar_empty[ST], bar_sdp, bar_ds,
-      bar_done, bar_drain;
+  __shared__ __align__(8) uint64_t bar_q, bar_kv[ST], bar_empty[ST], bar_sdp[2], bar_ds[2], bar_done,
+      bar_drain;
   __shared__ uint32_t tmem_slot;
   __shared__ uint32_t abort_flag;
 
@@ -365,24 +407,25 @@ __global__ void __launch_bounds__(320, 1)
   const TileWork w = decode_q_tile(d, blockIdx.x);
   const int sh = shift_of_head(d, w.h);
   const int tq0 = original_row(d, w.g * d.G + w.tile * kTile, sh);
-  const int nkv = w.tile + 1;
+  const int nkv = 2 * (w.tile + 1);  // 64-row kv sub-tiles from the group start to the diagonal
   WaitCtx wc{&abort_flag, a.status, a.wait_limit_ns};
 
   const uint32_t s0 = smem_u32(smem);
   const uint32_t sQ = s0 + C::OFF_Q, sG = s0 + C::OFF_DO;
-  auto sK = [&](int s) { return s0 + C::OFF_K + s * C::TILE_BYTES; };
-  auto sV = [&](int s) { return s0 + C::OFF_V + s * C::TILE_BYTES; };
+  auto sK = [&](int s) { return s0 + C::OFF_K + s * C::KV_BYTES; };
+  auto sV = [&](int s) { return s0 + C::OFF_V + s * C::KV_BYTES; };
 
   if (threadIdx.x == 0) {
     abort_flag = 0;
     mbar_init(smem_u32(&bar_q), 1);
     for (int s = 0; s < ST; ++s) {
-      mbar_init(smem_u32(&bar_k[s]), 1);
-      mbar_init(smem_u32(&bar_v[s]), 1);
+      mbar_init(smem_u32(&bar_kv[s]), 1);
       mbar_init(smem_u32(&bar_empty[s]), 1);
     }
-    mbar_init(smem_u32(&bar_sdp), 1);
-    mbar_init(smem_u32(&bar_ds), 256);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&bar_sdp[i]), 1);
+      mbar_init(smem_u32(&bar_ds[i]), 256);
+    }
     mbar_init(smem_u32(&bar_done), 1);
     mbar_init(smem_u32(&bar_drain), 1);
     fence_barrier_init();
@@ -402,62 +445,72 @@ __global__ void __launch_bounds__(320, 1)
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
       tma_prefetch_desc(&tmG);
-      mbar_arrive_expect_tx(smem_u32(&bar_q), 2 * C::TILE_BYTES);
+      mbar_arrive_expect_tx(smem_u32(&bar_q), 2 * C::Q_BYTES);
       for (int c = 0; c < D / 64; ++c) {
-        tma_load_4d(sQ + c * C::ATOM_BYTES, &tmQ, smem_u32(&bar_q), c * 64, w.h, tq0, w.b);
-        tma_load_4d(sG + c * C::ATOM_BYTES, &tmG, smem_u32(&bar_q), c * 64, w.h, tq0, w.b);
+        tma_load_4d(sQ + c * C::Q_ATOM, &tmQ, smem_u32(&bar_q), c * 64, w.h, tq0, w.b);
+        tma_load_4d(sG + c * C::Q_ATOM, &tmG, smem_u32(&bar_q), c * 64, w.h, tq0, w.b);
       }
       int issued = 0;
       for (int j = 0; j < nkv; ++j) {
         const int s = j % ST, n = j / ST;
         if (n > 0 && !mbar_wait(smem_u32(&bar_empty[s]), (n - 1) & 1, wc, 210)) break;
-        const int tk0 = original_row(d, w.g * d.G + j * kTile, sh);
-        mbar_arrive_expect_tx(smem_u32(&bar_k[s]), C::TILE_BYTES);
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_4d(sK(s) + c * C::ATOM_BYTES, &tmK, smem_u32(&bar_k[s]), c * 64, w.kvh, tk0, w.b);
-        mbar_arrive_expect_tx(smem_u32(&bar_v[s]), C::TILE_BYTES);
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_4d(sV(s) + c * C::ATOM_BYTES, &tmV, smem_u32(&bar_v[s]), c * 64, w.kvh, tk0, w.b);
+        const int tk0 = original_row(d, w.g * d.G + j * kSub, sh);
+        const uint32_t bar = smem_u32(&bar_kv[s]);
+        mbar_arrive_expect_tx(bar, 2 * C::KV_BYTES);
+        for (int c = 0; c < D / 64; ++c) {
+          tma_load_4d(sK(s) + c * C::KV_ATOM, &tmK, bar, c * 64, w.kvh, tk0, w.b);
+          tma_load_4d(sV(s) + c * C::KV_ATOM, &tmV, bar, c * 64, w.kvh, tk0, w.b);
+        }
         ++issued;
       }
       if (*wc.abort) {
         drain_wait(smem_u32(&bar_q), 0);
-        for (int s = 0; s < ST && s < issued; ++s) {
-          const int last = (issued - 1 - s) / ST;
-          drain_wait(smem_u32(&bar_k[s]), last & 1);
-          drain_wait(smem_u32(&bar_v[s]), last & 1);
-        }
+        for (int s = 0; s < ST && s < issued; ++s)
+          drain_wait(smem_u32(&bar_kv[s]), ((issued - 1 - s) / ST) & 1);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t idS = make_idesc_bf16(128, 128, 0, 0);  // S = Q K^T, dP = dO V^T
-      const uint32_t idQ = make_idesc_bf16(128, D, 0, 1);    // dQ += dS K (K MN-major)
-      bool ok = mbar_wait(smem_u32(&bar_q), 0, wc, 220);
+      const uint32_t idS = make_idesc_bf16(128, kSub, 0, 0);  // S = Q K^T, dP = dO V^T
+      const uint32_t idQ = make_idesc_bf16(128, D, 0, 1);     // dQ += dS K (K MN-major)
+      auto issue_sdp = [&](int j, int s) {
+        const uint32_t bo = (j & 1) * kSub;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t qo = (kk >> 2) * C::Q_ATOM + (kk & 3) * 32;
+          const uint32_t ko = (kk >> 2) * C::KV_ATOM + (kk & 3) * 32;
+          umma_ss(tmem + C::TM_S + bo, make_sdesc_sw128(sQ + qo, 16, 1024),
+                  make_sdesc_sw128(sK(s) + ko, 16, 1024), idS, kk > 0);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t qo = (kk >> 2) * C::Q_ATOM + (kk & 3) * 32;
+          const uint32_t ko = (kk >> 2) * C::KV_ATOM + (kk & 3) * 32;
+          umma_ss(tmem + C::TM_DP + bo, make_sdesc_sw128(sG + qo, 16, 1024),
+                  make_sdesc_sw128(sV(s) + ko, 16, 1024), idS, kk > 0);
+        }
+        umma_commit(smem_u32(&bar_sdp[j & 1]));
+      };
+      bool ok = mbar_wait(smem_u32(&bar_q), 0, wc, 220) && mbar_wait(smem_u32(&bar_kv[0]), 0, wc, 221);
+      if (ok) {
+        tc_fence_after();
+        issue_sdp(0, 0);
+      }
       for (int j = 0; ok && j < nkv; ++j) {
         const int s = j % ST;
-        if (!mbar_wait(smem_u32(&bar_k[s]), (j / ST) & 1, wc, 221)) break;
-        if (!mbar_wait(smem_u32(&bar_v[s]), (j / ST) & 1, wc, 222)) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::ATOM_BYTES + (kk & 3) * 32;
-          umma_ss(tmem + C::TM_S, make_sdesc_sw128(sQ + off, 16, 1024),
-                  make_sdesc_sw128(sK(s) + off, 16, 1024), idS, kk > 0);
+        if (j + 1 < nkv) {
+          const int s1 = (j + 1) % ST;
+          if (!mbar_wait(smem_u32(&bar_kv[s1]), ((j + 1) / ST) & 1, wc, 222)) break;
+          tc_fence_after();
+          issue_sdp(j + 1, s1);
         }
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::ATOM_BYTES + (kk & 3) * 32;
-          umma_ss(tmem + C::TM_DP, make_sdesc_sw128(sG + off, 16, 1024),
-                  make_sdesc_sw128(sV(s) + off, 16, 1024), idS, kk > 0);
-        }
-        umma_commit(smem_u32(&bar_sdp));
-        if (!mbar_wait(smem_u32(&bar_ds), j & 1, wc, 223)) break;
+        if (!mbar_wait(smem_u32(&bar_ds[j & 1]), (j >> 1) & 1, wc, 223)) break;
         tc_fence_after();
+        const uint32_t bo = (j & 1) * kSub;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          umma_ts(tmem + C::TM_DQ, tmem + C::TM_DP + split_acol(kk),
-                  make_sdesc_sw128(sK(s) + kk * 2048, C::ATOM_BYTES, 1024), idQ, (j > 0 || kk > 0));
+        for (int kk = 0; kk < kSub / 16; ++kk)
+          umma_ts(tmem + C::TM_DQ, tmem + C::TM_DP + bo + split_acol64(kk),
+                  make_sdesc_sw128(sK(s) + kk * 2048, C::KV_ATOM, 1024), idQ, (j > 0 || kk > 0));
         umma_commit(smem_u32(&bar_empty[s]));
       }
       umma_commit(smem_u32(&bar_done));
@@ -476,32 +529,33 @@ __global__ void __launch_bounds__(320, 1)
     const float delta = a.delta[ridx];
     bool ok = true;
     for (int j = 0; j < nkv; ++j) {
-      if (lane == 0) ok = mbar_wait(smem_u32(&bar_sdp), j & 1, wc, 230);
+      const uint32_t bo = (j & 1) * kSub + half * 32;
+      const int koff = j * kSub - w.tile * kTile;  // kv sub-tile start minus query tile start
+      if (lane == 0) ok = mbar_wait(smem_u32(&bar_sdp[j & 1]), (j >> 1) & 1, wc, 230);
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       tc_fence_after();
-      uint32_t sr[2][32], dr[2][32];
-      tmem_ld32(tmem + lane_off + C::TM_S + half * 64, sr[0]);
-      tmem_ld32(tmem + lane_off + C::TM_S + half * 64 + 32, sr[1]);
-      tmem_ld32(tmem + lane_off + C::TM_DP + half * 64, dr[0]);
-      tmem_ld32(tmem + lane_off + C::TM_DP + half * 64 + 32, dr[1]);
+      uint32_t sr[32], dr[32];
+      tmem_ld32(tmem + lane_off + C::TM_S + bo, sr);
+      tmem_ld32(tmem + lane_off + C::TM_DP + bo, dr);
       tmem_wait_ld();
-      const bool diag = (j == nkv - 1);
-      uint32_t pk[32];
+      float p[32];
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        float v0 = ex2_approx(fmaf(__uint_as_float(sr[(2 * c) >> 5][(2 * c) & 31]), sl2, -lse2));
-        float v1 = ex2_approx(fmaf(__uint_as_float(sr[(2 * c + 1) >> 5][(2 * c + 1) & 31]), sl2, -lse2));
-        if (diag && half * 64 + 2 * c > row) v0 = 0.f;  // key after query in rolled order
-        if (diag && half * 64 + 2 * c + 1 > row) v1 = 0.f;
-        v0 *= __uint_as_float(dr[(2 * c) >> 5][(2 * c) & 31]) - delta;
-        v1 *= __uint_as_float(dr[(2 * c + 1) >> 5][(2 * c + 1) & 31]) - delta;
-        pk[c] = pack_bf16x2(v0, v1);
+      for (int c = 0; c < 32; ++c) p[c] = ex2_approx(fmaf(__uint_as_float(sr[c]), sl2, -lse2));
+      if (koff >= 0) {  // sub-tile overlaps the diagonal: key after query is masked
+#pragma unroll
+        for (int c = 0; c < 32; ++c)
+          if (koff + half * 32 + c > row) p[c] = 0.f;
       }
-      tmem_st32(tmem + lane_off + C::TM_DP + half * 64, pk);
+      uint32_t pk[16];
+#pragma unroll
+      for (int c = 0; c < 16; ++c)
+        pk[c] = pack_bf16x2(p[2 * c] * (__uint_as_float(dr[2 * c]) - delta),
+                            p[2 * c + 1] * (__uint_as_float(dr[2 * c + 1]) - delta));
+      tmem_st16(tmem + lane_off + C::TM_DP + bo, pk);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(smem_u32(&bar_ds));
+      mbar_arrive(smem_u32(&bar_ds[j & 1]));
     }
     if (ok) {
       if (lane == 0) ok = mbar_wait(smem_u32(&bar_done), 0, wc, 232);
@@ -511,20 +565,12 @@ __global__ void __launch_bounds__(320, 1)
       tc_fence_after();
       __nv_bfloat16* dqrow = static_cast<__nv_bfloat16*>(a.dq) +
                              ((static_cast<size_t>(w.b) * d.N + t) * d.H + w.h) * D + half * (D / 2);
-      const float sc = a.scale;
 #pragma unroll
       for (int c = 0; c < D / 64; ++c) {
         uint32_t r[32];
         tmem_ld32(tmem + lane_off + C::TM_DQ + half * (D / 2) + c * 32, r);
         tmem_wait_ld();
-        uint4* dst = reinterpret_cast<uint4*>(dqrow + c * 32);
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-          dst[q] = make_uint4(
-              pack_bf16x2(__uint_as_float(r[8 * q]) * sc, __uint_as_float(r[8 * q + 1]) * sc),
-              pack_bf16x2(__uint_as_float(r[8 * q + 2]) * sc, __uint_as_float(r[8 * q + 3]) * sc),
-              pack_bf16x2(__uint_as_float(r[8 * q + 4]) * sc, __uint_as_float(r[8 * q + 5]) * sc),
-              pack_bf16x2(__uint_as_float(r[8 * q + 6]) * sc, __uint_as_float(r[8 * q + 7]) * sc));
+        store_row32(dqrow + c * 32, r, a.scale);
       }
     }
   }
@@ -543,9 +589,10 @@ static bool set_smem_attr(const void* fn, int bytes) {
   return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
 }
 
+// Tensor maps: `*128` have 128-row boxes, `*64` 64-row boxes.  dK/dV streams
+// 64-row query sub-tiles against 128-row kv tiles; dQ the other way round.
 template <int D>
-cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const CUtensorMap& tg, const BwdPreArgs& pre, const BwdArgs& a, int num_sms,
+cudaError_t launch_bwd(const BwdMaps& m, const BwdPreArgs& pre, const BwdArgs& a, int num_sms,
                        cudaStream_t stream, int* launches) {
   using K3 = DkvCfg<D>;
   using K4 = DqCfg<D>;
@@ -562,24 +609,20 @@ cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
   if (e != cudaSuccess) return e;
   const int grid_kv = a.d.B * a.d.Hkv * a.d.n_groups * a.d.tiles;
   prof_before(stream, kKernelBwdDkDv);
-  s2_bwd_dkdv_kernel<D><<<grid_kv, K3::THREADS, K3::SMEM_BYTES, stream>>>(tq, tk, tv, tg, a);
+  s2_bwd_dkdv_kernel<D><<<grid_kv, K3::THREADS, K3::SMEM_BYTES, stream>>>(m.q64, m.k128, m.v128, m.g64, a);
   e = cudaGetLastError();
   prof_after(stream);
   if (e != cudaSuccess) return e;
   const int grid_q = a.d.B * a.d.H * a.d.n_groups * a.d.tiles;
   prof_before(stream, kKernelBwdDq);
-  s2_bwd_dq_kernel<D><<<grid_q, K4::THREADS, K4::SMEM_BYTES, stream>>>(tq, tk, tv, tg, a);
+  s2_bwd_dq_kernel<D><<<grid_q, K4::THREADS, K4::SMEM_BYTES, stream>>>(m.q128, m.k64, m.v64, m.g128, a);
   e = cudaGetLastError();
   prof_after(stream);
   if (launches) *launches = 3;
   return e;
 }
 
-template cudaError_t launch_bwd<64>(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
-                                    const CUtensorMap&, const BwdPreArgs&, const BwdArgs&, int,
-                                    cudaStream_t, int*);
-template cudaError_t launch_bwd<128>(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
-                                     const CUtensorMap&, const BwdPreArgs&, const BwdArgs&, int,
-                                     cudaStream_t, int*);
+template cudaError_t launch_bwd<64>(const BwdMaps&, const BwdPreArgs&, const BwdArgs&, int, cudaStream_t, int*);
+template cudaError_t launch_bwd<128>(const BwdMaps&, const BwdPreArgs&, const BwdArgs&, int, cudaStream_t, int*);
 
 }  // namespace s2

@@ -12,6 +12,7 @@
 #pragma once
 
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 namespace s2 {
@@ -101,6 +102,12 @@ struct BwdArgs {
   void* dv;                // bf16 [B, N, Hkv, D]
   uint32_t* status;
   unsigned long long wait_limit_ns;
+};
+
+// TMA descriptors of the backward: 128-row and 64-row boxes of each operand.
+struct BwdMaps {
+  CUtensorMap q128, k128, v128, g128;
+  CUtensorMap q64, k64, v64, g64;
 };
 
 // Optional per-kernel timing (s2attn_profile_start / _stop): the launchers

@@ -7,13 +7,15 @@
 // community post, section 03: attention only inside each group; section 04:
 // causal next-token objective).
 //
-// Warp roles (192 threads):
+// Warp roles (320 threads):
 //   warp 0      TMA producer: Q once, then K_j / V_j into a STAGES-deep ring.
 //   warp 1      TMEM owner and UMMA issuer: S_j = Q K_j^T (double-buffered in
 //               TMEM), O += P_j V_j with P_j read from TMEM.
-//   warps 2..5  softmax: thread = query row; S row from TMEM, running max and
-//               sum, P (bf16) written back over S, O rescaled in TMEM only
-//               when the running max grows by more than 2^8, epilogue.
+//   warps 2..9  softmax: two threads per query row (warps 2..5 the first 64
+//               key columns of a tile, warps 6..9 the last 64); S from TMEM,
+//               running max and sum, P (bf16) written back over S, O rescaled
+//               in TMEM only when the running max grows by more than 2^8,
+//               epilogue.
 //
 // TMEM (512 columns): S buffers at [0,128) and [128,256) (P over their first
 // 64 columns), O at [256, 256 + D).
@@ -29,28 +31,31 @@ namespace s2 {
 template <int D>
 struct FwdCfg {
   static constexpr int BM = kTile, BN = kTile;
-  static constexpr int STAGES = (D == 64) ? 4 : 3;
+  // K and V tiles share one ring of slots, filled in the order K0 V0 K1 V1 ...;
+  // a K slot is released as soon as its S UMMA completes.
+  static constexpr int SLOTS = (D == 64) ? 8 : 5;
   static constexpr int ATOM_BYTES = kTile * 128;  // one 64-column slab of a 128-row tile
   static constexpr int Q_BYTES = BM * D * 2;
   static constexpr int KV_BYTES = BN * D * 2;
-  static constexpr int OFF_K = Q_BYTES;
-  static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
-  static constexpr int SMEM_BYTES = OFF_V + STAGES * KV_BYTES + 1024;  // + alignment slack
+  static constexpr int OFF_KV = Q_BYTES;
+  static constexpr int SMEM_BYTES = OFF_KV + SLOTS * KV_BYTES + 1024;  // + alignment slack
   static constexpr uint32_t TM_O = 256;
-  static constexpr int THREADS = 192;
+  static constexpr int THREADS = 320;
 };
 
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     s2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdArgs a) {
   using C = FwdCfg<D>;
-  constexpr int ST = C::STAGES;
+  constexpr int NS = C::SLOTS;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  __shared__ __align__(8) uint64_t bar_q, bar_k[ST], bar_v[ST], bar_empty[ST], bar_s[2], bar_p[2],
-      bar_o, bar_drain;
+  __shared__ __align__(8) uint64_t bar_q, bar_full[NS], bar_empty[NS], bar_s[2], bar_p[2], bar_x[2],
+      bar_l, bar_o, bar_drain;
+  __shared__ float red_max[2][2][kTile];  // [tile parity][half][row] partial row maxima
+  __shared__ float red_sum[2][kTile];     // [half][row] partial row sums
   __shared__ uint32_t tmem_slot;
   __shared__ uint32_t abort_flag;
 
@@ -64,21 +69,21 @@ __global__ void __launch_bounds__(192, 1)
   WaitCtx wc{&abort_flag, a.status, a.wait_limit_ns};
 
   const uint32_t sQ = smem_u32(smem);
-  auto sK = [&](int s) { return sQ + C::OFF_K + s * C::KV_BYTES; };
-  auto sV = [&](int s) { return sQ + C::OFF_V + s * C::KV_BYTES; };
+  auto slot_addr = [&](int s) { return sQ + C::OFF_KV + s * C::KV_BYTES; };
 
   if (threadIdx.x == 0) {
     abort_flag = 0;
     mbar_init(smem_u32(&bar_q), 1);
-    for (int s = 0; s < ST; ++s) {
-      mbar_init(smem_u32(&bar_k[s]), 1);
-      mbar_init(smem_u32(&bar_v[s]), 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(smem_u32(&bar_full[s]), 1);
       mbar_init(smem_u32(&bar_empty[s]), 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&bar_s[i]), 1);
-      mbar_init(smem_u32(&bar_p[i]), 128);
+      mbar_init(smem_u32(&bar_p[i]), 8);  // one elected arrival per softmax warp
+      mbar_init(smem_u32(&bar_x[i]), 8);
     }
+    mbar_init(smem_u32(&bar_l), 8);
     mbar_init(smem_u32(&bar_o), 1);
     mbar_init(smem_u32(&bar_drain), 1);
     fence_barrier_init();
@@ -102,29 +107,23 @@ __global__ void __launch_bounds__(192, 1)
       for (int c = 0; c < D / 64; ++c)
         tma_load_4d(sQ + c * C::ATOM_BYTES, &tmQ, smem_u32(&bar_q), c * 64, w.h, tq0, w.b);
       int issued = 0;
-      for (int j = 0; j < nkv; ++j) {
-        const int s = j % ST, n = j / ST;
+      for (int L = 0; L < 2 * nkv; ++L) {  // load L: K_{L/2} (even) or V_{L/2} (odd)
+        const int s = L % NS, n = L / NS;
         if (n > 0 && !mbar_wait(smem_u32(&bar_empty[s]), (n - 1) & 1, wc, 10)) break;
-        const int tk0 = original_row(d, w.g * d.G + j * kTile, sh);
-        mbar_arrive_expect_tx(smem_u32(&bar_k[s]), C::KV_BYTES);
+        const int tk0 = original_row(d, w.g * d.G + (L >> 1) * kTile, sh);
+        const CUtensorMap* map = (L & 1) ? &tmV : &tmK;
+        mbar_arrive_expect_tx(smem_u32(&bar_full[s]), C::KV_BYTES);
         for (int c = 0; c < D / 64; ++c)
-          tma_load_4d(sK(s) + c * C::ATOM_BYTES, &tmK, smem_u32(&bar_k[s]), c * 64, w.kvh, tk0,
-                      w.b);
-        mbar_arrive_expect_tx(smem_u32(&bar_v[s]), C::KV_BYTES);
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_4d(sV(s) + c * C::ATOM_BYTES, &tmV, smem_u32(&bar_v[s]), c * 64, w.kvh, tk0,
-                      w.b);
+          tma_load_4d(slot_addr(s) + c * C::ATOM_BYTES, map, smem_u32(&bar_full[s]), c * 64, w.kvh,
+                      tk0, w.b);
         ++issued;
       }
       if (*wc.abort) {
         // never leave copies in flight into shared memory: wait (bounded) for
-        // the last fill of every stage and for Q
+        // the last fill of every slot and for Q
         drain_wait(smem_u32(&bar_q), 0);
-        for (int s = 0; s < ST && s < issued; ++s) {
-          const int last = (issued - 1 - s) / ST;
-          drain_wait(smem_u32(&bar_k[s]), last & 1);
-          drain_wait(smem_u32(&bar_v[s]), last & 1);
-        }
+        for (int s = 0; s < NS && s < issued; ++s)
+          drain_wait(smem_u32(&bar_full[s]), ((issued - 1 - s) / NS) & 1);
       }
     }
   } else if (warp == 1) {
@@ -132,37 +131,35 @@ __global__ void __launch_bounds__(192, 1)
     if (lane == 0) {
       const uint32_t idS = make_idesc_bf16(128, C::BN, 0, 0);  // Q K-major, K K-major
       const uint32_t idO = make_idesc_bf16(128, D, 0, 1);      // P from TMEM, V MN-major
-      auto issue_qk = [&](uint32_t tS, uint32_t k_base) {
+      // S_j = Q K_j^T into S buffer j&1; releases K_j's slot when done
+      auto issue_qk = [&](int j) -> bool {
+        const int L = 2 * j, s = L % NS;
+        if (!mbar_wait(smem_u32(&bar_full[s]), (L / NS) & 1, wc, 22)) return false;
+        tc_fence_after();
+        const uint32_t k_base = slot_addr(s);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::ATOM_BYTES + (kk & 3) * 32;
-          umma_ss(tS, make_sdesc_sw128(sQ + off, 16, 1024), make_sdesc_sw128(k_base + off, 16, 1024),
-                  idS, kk > 0);
+          umma_ss(tmem + (j & 1) * 128, make_sdesc_sw128(sQ + off, 16, 1024),
+                  make_sdesc_sw128(k_base + off, 16, 1024), idS, kk > 0);
         }
+        umma_commit(smem_u32(&bar_s[j & 1]));
+        umma_commit(smem_u32(&bar_empty[s]));
+        return true;
       };
-      bool ok = mbar_wait(smem_u32(&bar_q), 0, wc, 20) && mbar_wait(smem_u32(&bar_k[0]), 0, wc, 21);
-      if (ok) {
-        tc_fence_after();
-        issue_qk(tmem, sK(0));
-        umma_commit(smem_u32(&bar_s[0]));
-      }
+      bool ok = mbar_wait(smem_u32(&bar_q), 0, wc, 20) && issue_qk(0);
       for (int j = 0; ok && j < nkv; ++j) {
-        const int s = j % ST;
-        if (j + 1 < nkv) {
-          const int s1 = (j + 1) % ST;
-          if (!mbar_wait(smem_u32(&bar_k[s1]), ((j + 1) / ST) & 1, wc, 22)) break;
-          tc_fence_after();
-          issue_qk(tmem + ((j + 1) & 1) * 128, sK(s1));
-          umma_commit(smem_u32(&bar_s[(j + 1) & 1]));
-        }
+        if (j + 1 < nkv && !issue_qk(j + 1)) break;
+        const int L = 2 * j + 1, s = L % NS;
         if (!mbar_wait(smem_u32(&bar_p[j & 1]), (j >> 1) & 1, wc, 23)) break;
-        if (!mbar_wait(smem_u32(&bar_v[s]), (j / ST) & 1, wc, 24)) break;
+        if (!mbar_wait(smem_u32(&bar_full[s]), (L / NS) & 1, wc, 24)) break;
         tc_fence_after();
         const uint32_t tP = tmem + (j & 1) * 128;
+        const uint32_t v_base = slot_addr(s);
 #pragma unroll
         for (int kk = 0; kk < C::BN / 16; ++kk)
-          umma_ts(tmem + C::TM_O, tP + kk * 8,
-                  make_sdesc_sw128(sV(s) + kk * 2048, C::ATOM_BYTES, 1024), idO, (j > 0 || kk > 0));
+          umma_ts(tmem + C::TM_O, tP + kk * 8, make_sdesc_sw128(v_base + kk * 2048, C::ATOM_BYTES, 1024),
+                  idO, (j > 0 || kk > 0));
         umma_commit(smem_u32(&bar_o));
         umma_commit(smem_u32(&bar_empty[s]));
       }
@@ -172,7 +169,12 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax
+    // Two warpgroups share every query row: warps 2..5 take key columns
+    // [0,64) of each tile, warps 6..9 columns [64,128).  The two halves of a
+    // row exchange their partial maxima through shared memory each tile (and
+    // their partial sums once at the end); both then take identical decisions.
     const int quarter = warp & 3;  // TMEM lanes this warp may access
+    const int half = (warp - 2) >> 2;
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const float sl2 = a.scale_log2;
@@ -184,42 +186,52 @@ __global__ void __launch_bounds__(192, 1)
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       tc_fence_after();
-      uint32_t sr[4][32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr[c]);
+      uint32_t sr[2][32];
+      tmem_ld32(tS + half * 64, sr[0]);
+      tmem_ld32(tS + half * 64 + 32, sr[1]);
       tmem_wait_ld();
-      const bool diag = (j == nkv - 1);
-      float mx = neg_inf();
+      if (j == nkv - 1) {  // diagonal tile: keys after the query are masked
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        float v = __uint_as_float(sr[c >> 5][c & 31]);
-        if (diag && c > row) v = neg_inf();
-        sr[c >> 5][c & 31] = __float_as_uint(v);
-        mx = fmaxf(mx, v);
+        for (int c = 0; c < 64; ++c)
+          if (half * 64 + c > row) sr[c >> 5][c & 31] = __float_as_uint(neg_inf());
       }
-      mx *= sl2;
+      float m4[4] = {neg_inf(), neg_inf(), neg_inf(), neg_inf()};
+#pragma unroll
+      for (int c = 0; c < 64; ++c) m4[c & 3] = fmaxf(m4[c & 3], __uint_as_float(sr[c >> 5][c & 31]));
+      const float mh = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+      // exchange partial maxima with the other half of the row (double-buffered slot)
+      red_max[j & 1][half][row] = mh;
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(smem_u32(&bar_x[j & 1]));
+        ok = mbar_wait(smem_u32(&bar_x[j & 1]), (j >> 1) & 1, wc, 33);
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      const float mx = fmaxf(mh, red_max[j & 1][half ^ 1][row]) * sl2;
       float alpha = 1.f;
       bool resc = false;
       if (j == 0) {
         m_run = mx;
-      } else if (mx > m_run + 8.f) {
+      } else if (mx > m_run + 8.f) {  // rescale only when the max grows by more than 2^8
         alpha = ex2_approx(m_run - mx);
         m_run = mx;
         resc = true;
       }
-      uint32_t pk[2][32];
-      float rs = 0.f;
+      uint32_t pk[32];
+      float r4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
+      for (int c = 0; c < 32; ++c) {
         const float p0 = ex2_approx(fmaf(__uint_as_float(sr[(2 * c) >> 5][(2 * c) & 31]), sl2, -m_run));
         const float p1 =
             ex2_approx(fmaf(__uint_as_float(sr[(2 * c + 1) >> 5][(2 * c + 1) & 31]), sl2, -m_run));
-        pk[c >> 5][c & 31] = pack_bf16x2(p0, p1);
-        rs += p0 + p1;
+        pk[c] = pack_bf16x2(p0, p1);
+        r4[c & 3] += p0 + p1;
       }
-      l_run = l_run * alpha + rs;
-      tmem_st32(tS, pk[0]);
-      tmem_st32(tS + 32, pk[1]);
+      l_run = l_run * alpha + ((r4[0] + r4[1]) + (r4[2] + r4[3]));
+      // P (bf16) over the first 64 columns of this S buffer; both halves read
+      // their S columns before the exchange above, so no write races a read
+      tmem_st32(tS + half * 32, pk);
       if (__any_sync(0xffffffffu, resc)) {
         // O holds P_{j-1} V_{j-1} only once that UMMA has completed
         if (lane == 0) ok = mbar_wait(smem_u32(&bar_o), (j - 1) & 1, wc, 31);
@@ -227,34 +239,42 @@ __global__ void __launch_bounds__(192, 1)
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < D / 64; ++c) {
           uint32_t o[32];
-          tmem_ld32(tmem + lane_off + C::TM_O + c * 32, o);
+          const uint32_t to = tmem + lane_off + C::TM_O + half * (D / 2) + c * 32;
+          tmem_ld32(to, o);
           tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(tmem + lane_off + C::TM_O + c * 32, o);
+          tmem_st32(to, o);
         }
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(smem_u32(&bar_p[j & 1]));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bar_p[j & 1]));
     }
     // ------------------------------------------------------------ epilogue
     if (ok) {
-      if (lane == 0) ok = mbar_wait(smem_u32(&bar_o), (nkv - 1) & 1, wc, 32);
+      red_sum[half][row] = l_run;
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(smem_u32(&bar_l));
+        ok = mbar_wait(smem_u32(&bar_l), 0, wc, 34) && mbar_wait(smem_u32(&bar_o), (nkv - 1) & 1, wc, 32);
+      }
       ok = __shfl_sync(0xffffffffu, ok, 0);
     }
     if (ok) {
       tc_fence_after();
-      const float inv_l = 1.f / l_run;
+      const float l_tot = l_run + red_sum[half ^ 1][row];
+      const float inv_l = 1.f / l_tot;
       const int t = tq0 + row;
-      __nv_bfloat16* orow =
-          static_cast<__nv_bfloat16*>(a.o) + ((static_cast<size_t>(w.b) * d.N + t) * d.H + w.h) * D;
+      __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.o) +
+                            ((static_cast<size_t>(w.b) * d.N + t) * d.H + w.h) * D + half * (D / 2);
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < D / 64; ++c) {
         uint32_t o[32];
-        tmem_ld32(tmem + lane_off + C::TM_O + c * 32, o);
+        tmem_ld32(tmem + lane_off + C::TM_O + half * (D / 2) + c * 32, o);
         tmem_wait_ld();
         uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll
@@ -267,8 +287,9 @@ __global__ void __launch_bounds__(192, 1)
           dst[q] = v;
         }
       }
-      a.lse[(static_cast<size_t>(w.b) * d.H + w.h) * d.N + t] =
-          (m_run + __log2f(l_run)) * 0.69314718055994530942f;
+      if (half == 0)
+        a.lse[(static_cast<size_t>(w.b) * d.H + w.h) * d.N + t] =
+            (m_run + __log2f(l_tot)) * 0.69314718055994530942f;
     }
   }
 

@@ -21,8 +21,7 @@ template <int D>
 cudaError_t launch_fwd(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const FwdArgs&,
                        cudaStream_t);
 template <int D>
-cudaError_t launch_bwd(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
-                       const BwdPreArgs&, const BwdArgs&, int, cudaStream_t, int*);
+cudaError_t launch_bwd(const BwdMaps&, const BwdPreArgs&, const BwdArgs&, int, cudaStream_t, int*);
 }  // namespace s2
 
 namespace {
@@ -125,15 +124,15 @@ Dims make_dims(int B, int H, int Hkv, int N, int D, int G) {
 }
 
 // 4-D view {D, heads, N, B} of a bf16 [B, N, heads, D] tensor; box = one
-// 128-row x 64-column slab, 128-byte swizzle (the UMMA operand layout).
-bool make_map(CUtensorMap* m, const void* base, int B, int N, int heads, int D) {
+// box_rows x 64-column slab, 128-byte swizzle (the UMMA operand layout).
+bool make_map(CUtensorMap* m, const void* base, int B, int N, int heads, int D, int box_rows = kTile) {
   EncodeTiledFn enc = get_encode();
   if (!enc) return false;
   cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(heads),
                         static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(B)};
   cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(heads) * D * 2,
                            static_cast<cuuint64_t>(N) * heads * D * 2};
-  cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(kTile), 1};
+  cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(box_rows), 1};
   cuuint32_t es[4] = {1, 1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -299,9 +298,11 @@ int s2attn_bwd(const void* q, const void* k, const void* v, const void* o, const
   DeviceInfo info;
   if (!device_info(&info)) return S2ATTN_ERR_CUDA;
   if (!info.ok) return S2ATTN_ERR_UNSUPPORTED;
-  CUtensorMap tq, tk, tv, tg;
-  if (!make_map(&tq, q, B, N, H, D) || !make_map(&tk, k, B, N, Hkv, D) ||
-      !make_map(&tv, v, B, N, Hkv, D) || !make_map(&tg, dO, B, N, H, D))
+  BwdMaps maps;
+  if (!make_map(&maps.q128, q, B, N, H, D) || !make_map(&maps.k128, k, B, N, Hkv, D) ||
+      !make_map(&maps.v128, v, B, N, Hkv, D) || !make_map(&maps.g128, dO, B, N, H, D) ||
+      !make_map(&maps.q64, q, B, N, H, D, 64) || !make_map(&maps.k64, k, B, N, Hkv, D, 64) ||
+      !make_map(&maps.v64, v, B, N, Hkv, D, 64) || !make_map(&maps.g64, dO, B, N, H, D, 64))
     return S2ATTN_ERR_CUDA;
   unsigned char* ws = static_cast<unsigned char*>(workspace);
   uint32_t* status = reinterpret_cast<uint32_t*>(ws);
@@ -329,8 +330,8 @@ int s2attn_bwd(const void* q, const void* k, const void* v, const void* o, const
   a.wait_limit_ns = wait_limit_ns();
   int launches = 0;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = (D == 64) ? launch_bwd<64>(tq, tk, tv, tg, pre, a, info.sms, s, &launches)
-                            : launch_bwd<128>(tq, tk, tv, tg, pre, a, info.sms, s, &launches);
+  cudaError_t e = (D == 64) ? launch_bwd<64>(maps, pre, a, info.sms, s, &launches)
+                            : launch_bwd<128>(maps, pre, a, info.sms, s, &launches);
   g_last_launches = launches;
   return e == cudaSuccess ? S2ATTN_OK : S2ATTN_ERR_CUDA;
 }
