@@ -189,7 +189,8 @@ __global__ void __launch_bounds__(320, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
+    // (whole warp converged; one elected lane issues the copies)
+    if (elect_one()) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
@@ -199,14 +200,17 @@ __global__ void __launch_bounds__(320, 1)
         tma_load_4d(sK + c * C::KV_ATOM, &tmK, smem_u32(&bar_kv), c * 64, w.kvh, tk0, w.b);
         tma_load_4d(sV + c * C::KV_ATOM, &tmV, smem_u32(&bar_kv), c * 64, w.kvh, tk0, w.b);
       }
-      int issued = 0;
-      for (int it = 0; it < iters; ++it) {
-        const int s = it % ST, n = it / ST;
-        if (n > 0 && !mbar_wait(smem_u32(&bar_empty[s]), (n - 1) & 1, wc, 110)) break;
-        const int h = w.kvh * d.rep + it / nq;
-        const int i64 = 2 * w.tile + it % nq;
-        const int tq0 = original_row(d, w.g * d.G + i64 * kSub, sh);
-        const uint32_t bar = smem_u32(&bar_full[s]);
+    }
+    __syncwarp();
+    int issued = 0;
+    for (int it = 0; it < iters; ++it) {
+      const int s = it % ST, n = it / ST;
+      if (n > 0 && !warp_wait(smem_u32(&bar_empty[s]), (n - 1) & 1, wc, 110)) break;
+      const int h = w.kvh * d.rep + it / nq;
+      const int i64 = 2 * w.tile + it % nq;
+      const int tq0 = original_row(d, w.g * d.G + i64 * kSub, sh);
+      const uint32_t bar = smem_u32(&bar_full[s]);
+      if (elect_one()) {
         mbar_arrive_expect_tx(bar, 2 * C::Q_BYTES + 512);
         for (int c = 0; c < D / 64; ++c) {
           tma_load_4d(sQ(s) + c * C::Q_ATOM, &tmQ, bar, c * 64, h, tq0, w.b);
@@ -215,68 +219,82 @@ __global__ void __launch_bounds__(320, 1)
         const size_t ro = (static_cast<size_t>(w.b) * d.H + h) * d.N + tq0;
         bulk_load(sRow(s), a.lse2 + ro, 256, bar);
         bulk_load(sRow(s) + 256, a.delta + ro, 256, bar);
-        ++issued;
       }
-      if (*wc.abort) {
-        drain_wait(smem_u32(&bar_kv), 0);
-        for (int s = 0; s < ST && s < issued; ++s)
-          drain_wait(smem_u32(&bar_full[s]), ((issued - 1 - s) / ST) & 1);
-      }
+      __syncwarp();
+      ++issued;
+    }
+    if (*wc.abort && lane == 0) {
+      drain_wait(smem_u32(&bar_kv), 0);
+      for (int s = 0; s < ST && s < issued; ++s)
+        drain_wait(smem_u32(&bar_full[s]), ((issued - 1 - s) / ST) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ UMMA issuer
-    if (lane == 0) {
-      const uint32_t idS = make_idesc_bf16(128, kSub, 0, 0);  // S^T = K Q^T, dP^T = V dO^T
-      const uint32_t idG = make_idesc_bf16(128, D, 0, 1);     // dV += P^T dO, dK += dS^T Q
-      auto issue_sdp = [&](int it, int s) {
-        const uint32_t bo = (it & 1) * kSub;
+    // (whole warp converged; one elected lane issues each batch)
+    const uint32_t idS = make_idesc_bf16(128, kSub, 0, 0);  // S^T = K Q^T, dP^T = V dO^T
+    const uint32_t idG = make_idesc_bf16(128, D, 0, 1);     // dV += P^T dO, dK += dS^T Q
+    const uint64_t dK0 = make_sdesc_sw128(sK, 16, 1024);           // K-major (A)
+    const uint64_t dV0 = make_sdesc_sw128(sV, 16, 1024);
+    const uint64_t dQk = make_sdesc_sw128(sQ(0), 16, 1024);        // K-major (B of S^T)
+    const uint64_t dGk = make_sdesc_sw128(sG(0), 16, 1024);
+    const uint64_t dQm = make_sdesc_sw128(sQ(0), C::Q_ATOM, 1024);  // MN-major (B of dK)
+    const uint64_t dGm = make_sdesc_sw128(sG(0), C::Q_ATOM, 1024);  // MN-major (B of dV)
+    auto issue_sdp = [&](int it, int s) {
+      const uint32_t bo = (it & 1) * kSub;
+      const uint64_t dq = sdesc_advance(dQk, s * C::Q_BYTES), dg = sdesc_advance(dGk, s * C::Q_BYTES);
+      if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ko = (kk >> 2) * C::KV_ATOM + (kk & 3) * 32;
           const uint32_t qo = (kk >> 2) * C::Q_ATOM + (kk & 3) * 32;
-          umma_ss(tmem + C::TM_S + bo, make_sdesc_sw128(sK + ko, 16, 1024),
-                  make_sdesc_sw128(sQ(s) + qo, 16, 1024), idS, kk > 0);
+          umma_ss(tmem + C::TM_S + bo, sdesc_advance(dK0, ko), sdesc_advance(dq, qo), idS, kk > 0);
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ko = (kk >> 2) * C::KV_ATOM + (kk & 3) * 32;
           const uint32_t qo = (kk >> 2) * C::Q_ATOM + (kk & 3) * 32;
-          umma_ss(tmem + C::TM_DP + bo, make_sdesc_sw128(sV + ko, 16, 1024),
-                  make_sdesc_sw128(sG(s) + qo, 16, 1024), idS, kk > 0);
+          umma_ss(tmem + C::TM_DP + bo, sdesc_advance(dV0, ko), sdesc_advance(dg, qo), idS, kk > 0);
         }
         umma_commit(smem_u32(&bar_sdp[it & 1]));
-      };
-      bool ok = mbar_wait(smem_u32(&bar_kv), 0, wc, 120) &&
-                (iters == 0 || mbar_wait(smem_u32(&bar_full[0]), 0, wc, 121));
-      if (ok && iters > 0) {
-        tc_fence_after();
-        issue_sdp(0, 0);
       }
-      for (int it = 0; ok && it < iters; ++it) {
-        const int s = it % ST;
-        if (it + 1 < iters) {
-          const int s1 = (it + 1) % ST;
-          if (!mbar_wait(smem_u32(&bar_full[s1]), ((it + 1) / ST) & 1, wc, 122)) break;
-          tc_fence_after();
-          issue_sdp(it + 1, s1);  // its TMEM buffer's last readers were issued before: in order
-        }
-        if (!mbar_wait(smem_u32(&bar_pds[it & 1]), (it >> 1) & 1, wc, 123)) break;
+      __syncwarp();
+    };
+    bool ok = warp_wait(smem_u32(&bar_kv), 0, wc, 120) && warp_wait(smem_u32(&bar_full[0]), 0, wc, 121);
+    if (ok) {
+      tc_fence_after();
+      issue_sdp(0, 0);
+    }
+    for (int it = 0; ok && it < iters; ++it) {
+      const int s = it % ST;
+      if (it + 1 < iters) {
+        const int s1 = (it + 1) % ST;
+        if (!warp_wait(smem_u32(&bar_full[s1]), ((it + 1) / ST) & 1, wc, 122)) break;
         tc_fence_after();
-        const uint32_t bo = (it & 1) * kSub;
+        issue_sdp(it + 1, s1);  // its TMEM buffer's last readers were issued before: in order
+      }
+      if (!warp_wait(smem_u32(&bar_pds[it & 1]), (it >> 1) & 1, wc, 123)) break;
+      tc_fence_after();
+      const uint32_t bo = (it & 1) * kSub;
+      const uint64_t dg = sdesc_advance(dGm, s * C::Q_BYTES), dq = sdesc_advance(dQm, s * C::Q_BYTES);
+      if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < kSub / 16; ++kk)
-          umma_ts(tmem + C::TM_DV, tmem + C::TM_S + bo + split_acol64(kk),
-                  make_sdesc_sw128(sG(s) + kk * 2048, C::Q_ATOM, 1024), idG, (it > 0 || kk > 0));
+          umma_ts(tmem + C::TM_DV, tmem + C::TM_S + bo + split_acol64(kk), sdesc_advance(dg, kk * 2048),
+                  idG, (it > 0 || kk > 0));
 #pragma unroll
         for (int kk = 0; kk < kSub / 16; ++kk)
-          umma_ts(tmem + C::TM_DK, tmem + C::TM_DP + bo + split_acol64(kk),
-                  make_sdesc_sw128(sQ(s) + kk * 2048, C::Q_ATOM, 1024), idG, (it > 0 || kk > 0));
+          umma_ts(tmem + C::TM_DK, tmem + C::TM_DP + bo + split_acol64(kk), sdesc_advance(dq, kk * 2048),
+                  idG, (it > 0 || kk > 0));
         umma_commit(smem_u32(&bar_empty[s]));
       }
+      __syncwarp();
+    }
+    if (elect_one()) {
       umma_commit(smem_u32(&bar_done));
       umma_commit(smem_u32(&bar_drain));
       drain_wait(smem_u32(&bar_drain), 0);
     }
+    __syncwarp();
   } else {
     // ------------------------------------------------------------ P^T, dS^T
     const int quarter = warp & 3;
@@ -440,7 +458,8 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t tmem = tmem_slot;
 
   if (warp == 0) {
-    if (lane == 0) {
+    // (whole warp converged; one elected lane issues the copies)
+    if (elect_one()) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
@@ -450,73 +469,90 @@ __global__ void __launch_bounds__(320, 1)
         tma_load_4d(sQ + c * C::Q_ATOM, &tmQ, smem_u32(&bar_q), c * 64, w.h, tq0, w.b);
         tma_load_4d(sG + c * C::Q_ATOM, &tmG, smem_u32(&bar_q), c * 64, w.h, tq0, w.b);
       }
-      int issued = 0;
-      for (int j = 0; j < nkv; ++j) {
-        const int s = j % ST, n = j / ST;
-        if (n > 0 && !mbar_wait(smem_u32(&bar_empty[s]), (n - 1) & 1, wc, 210)) break;
-        const int tk0 = original_row(d, w.g * d.G + j * kSub, sh);
-        const uint32_t bar = smem_u32(&bar_kv[s]);
+    }
+    __syncwarp();
+    int issued = 0;
+    for (int j = 0; j < nkv; ++j) {
+      const int s = j % ST, n = j / ST;
+      if (n > 0 && !warp_wait(smem_u32(&bar_empty[s]), (n - 1) & 1, wc, 210)) break;
+      const int tk0 = original_row(d, w.g * d.G + j * kSub, sh);
+      const uint32_t bar = smem_u32(&bar_kv[s]);
+      if (elect_one()) {
         mbar_arrive_expect_tx(bar, 2 * C::KV_BYTES);
         for (int c = 0; c < D / 64; ++c) {
           tma_load_4d(sK(s) + c * C::KV_ATOM, &tmK, bar, c * 64, w.kvh, tk0, w.b);
           tma_load_4d(sV(s) + c * C::KV_ATOM, &tmV, bar, c * 64, w.kvh, tk0, w.b);
         }
-        ++issued;
       }
-      if (*wc.abort) {
-        drain_wait(smem_u32(&bar_q), 0);
-        for (int s = 0; s < ST && s < issued; ++s)
-          drain_wait(smem_u32(&bar_kv[s]), ((issued - 1 - s) / ST) & 1);
-      }
+      __syncwarp();
+      ++issued;
+    }
+    if (*wc.abort && lane == 0) {
+      drain_wait(smem_u32(&bar_q), 0);
+      for (int s = 0; s < ST && s < issued; ++s)
+        drain_wait(smem_u32(&bar_kv[s]), ((issued - 1 - s) / ST) & 1);
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      const uint32_t idS = make_idesc_bf16(128, kSub, 0, 0);  // S = Q K^T, dP = dO V^T
-      const uint32_t idQ = make_idesc_bf16(128, D, 0, 1);     // dQ += dS K (K MN-major)
-      auto issue_sdp = [&](int j, int s) {
-        const uint32_t bo = (j & 1) * kSub;
+    // (whole warp converged; one elected lane issues each batch)
+    const uint32_t idS = make_idesc_bf16(128, kSub, 0, 0);  // S = Q K^T, dP = dO V^T
+    const uint32_t idQ = make_idesc_bf16(128, D, 0, 1);     // dQ += dS K (K MN-major)
+    const uint64_t dQ0 = make_sdesc_sw128(sQ, 16, 1024);               // K-major (A)
+    const uint64_t dG0 = make_sdesc_sw128(sG, 16, 1024);
+    const uint64_t dKk = make_sdesc_sw128(sK(0), 16, 1024);            // K-major (B of S)
+    const uint64_t dVk = make_sdesc_sw128(sV(0), 16, 1024);
+    const uint64_t dKm = make_sdesc_sw128(sK(0), C::KV_ATOM, 1024);    // MN-major (B of dQ)
+    auto issue_sdp = [&](int j, int s) {
+      const uint32_t bo = (j & 1) * kSub;
+      const uint64_t dk = sdesc_advance(dKk, s * C::KV_BYTES), dv = sdesc_advance(dVk, s * C::KV_BYTES);
+      if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t qo = (kk >> 2) * C::Q_ATOM + (kk & 3) * 32;
           const uint32_t ko = (kk >> 2) * C::KV_ATOM + (kk & 3) * 32;
-          umma_ss(tmem + C::TM_S + bo, make_sdesc_sw128(sQ + qo, 16, 1024),
-                  make_sdesc_sw128(sK(s) + ko, 16, 1024), idS, kk > 0);
+          umma_ss(tmem + C::TM_S + bo, sdesc_advance(dQ0, qo), sdesc_advance(dk, ko), idS, kk > 0);
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t qo = (kk >> 2) * C::Q_ATOM + (kk & 3) * 32;
           const uint32_t ko = (kk >> 2) * C::KV_ATOM + (kk & 3) * 32;
-          umma_ss(tmem + C::TM_DP + bo, make_sdesc_sw128(sG + qo, 16, 1024),
-                  make_sdesc_sw128(sV(s) + ko, 16, 1024), idS, kk > 0);
+          umma_ss(tmem + C::TM_DP + bo, sdesc_advance(dG0, qo), sdesc_advance(dv, ko), idS, kk > 0);
         }
         umma_commit(smem_u32(&bar_sdp[j & 1]));
-      };
-      bool ok = mbar_wait(smem_u32(&bar_q), 0, wc, 220) && mbar_wait(smem_u32(&bar_kv[0]), 0, wc, 221);
-      if (ok) {
-        tc_fence_after();
-        issue_sdp(0, 0);
       }
-      for (int j = 0; ok && j < nkv; ++j) {
-        const int s = j % ST;
-        if (j + 1 < nkv) {
-          const int s1 = (j + 1) % ST;
-          if (!mbar_wait(smem_u32(&bar_kv[s1]), ((j + 1) / ST) & 1, wc, 222)) break;
-          tc_fence_after();
-          issue_sdp(j + 1, s1);
-        }
-        if (!mbar_wait(smem_u32(&bar_ds[j & 1]), (j >> 1) & 1, wc, 223)) break;
+      __syncwarp();
+    };
+    bool ok = warp_wait(smem_u32(&bar_q), 0, wc, 220) && warp_wait(smem_u32(&bar_kv[0]), 0, wc, 221);
+    if (ok) {
+      tc_fence_after();
+      issue_sdp(0, 0);
+    }
+    for (int j = 0; ok && j < nkv; ++j) {
+      const int s = j % ST;
+      if (j + 1 < nkv) {
+        const int s1 = (j + 1) % ST;
+        if (!warp_wait(smem_u32(&bar_kv[s1]), ((j + 1) / ST) & 1, wc, 222)) break;
         tc_fence_after();
-        const uint32_t bo = (j & 1) * kSub;
+        issue_sdp(j + 1, s1);
+      }
+      if (!warp_wait(smem_u32(&bar_ds[j & 1]), (j >> 1) & 1, wc, 223)) break;
+      tc_fence_after();
+      const uint32_t bo = (j & 1) * kSub;
+      const uint64_t dk = sdesc_advance(dKm, s * C::KV_BYTES);
+      if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < kSub / 16; ++kk)
-          umma_ts(tmem + C::TM_DQ, tmem + C::TM_DP + bo + split_acol64(kk),
-                  make_sdesc_sw128(sK(s) + kk * 2048, C::KV_ATOM, 1024), idQ, (j > 0 || kk > 0));
+          umma_ts(tmem + C::TM_DQ, tmem + C::TM_DP + bo + split_acol64(kk), sdesc_advance(dk, kk * 2048),
+                  idQ, (j > 0 || kk > 0));
         umma_commit(smem_u32(&bar_empty[s]));
       }
+      __syncwarp();
+    }
+    if (elect_one()) {
       umma_commit(smem_u32(&bar_done));
       umma_commit(smem_u32(&bar_drain));
       drain_wait(smem_u32(&bar_drain), 0);
     }
+    __syncwarp();
   } else {
     const int quarter = warp & 3;
     const int half = (warp - 2) >> 2;

@@ -99,74 +99,90 @@ __global__ void __launch_bounds__(320, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
+    // (whole warp converged; one elected lane issues the copies)
+    if (elect_one()) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
       mbar_arrive_expect_tx(smem_u32(&bar_q), C::Q_BYTES);
       for (int c = 0; c < D / 64; ++c)
         tma_load_4d(sQ + c * C::ATOM_BYTES, &tmQ, smem_u32(&bar_q), c * 64, w.h, tq0, w.b);
-      int issued = 0;
-      for (int L = 0; L < 2 * nkv; ++L) {  // load L: K_{L/2} (even) or V_{L/2} (odd)
-        const int s = L % NS, n = L / NS;
-        if (n > 0 && !mbar_wait(smem_u32(&bar_empty[s]), (n - 1) & 1, wc, 10)) break;
-        const int tk0 = original_row(d, w.g * d.G + (L >> 1) * kTile, sh);
-        const CUtensorMap* map = (L & 1) ? &tmV : &tmK;
+    }
+    __syncwarp();
+    int issued = 0;
+    for (int L = 0; L < 2 * nkv; ++L) {  // load L: K_{L/2} (even) or V_{L/2} (odd)
+      const int s = L % NS, n = L / NS;
+      if (n > 0 && !warp_wait(smem_u32(&bar_empty[s]), (n - 1) & 1, wc, 10)) break;
+      const int tk0 = original_row(d, w.g * d.G + (L >> 1) * kTile, sh);
+      const CUtensorMap* map = (L & 1) ? &tmV : &tmK;
+      if (elect_one()) {
         mbar_arrive_expect_tx(smem_u32(&bar_full[s]), C::KV_BYTES);
         for (int c = 0; c < D / 64; ++c)
           tma_load_4d(slot_addr(s) + c * C::ATOM_BYTES, map, smem_u32(&bar_full[s]), c * 64, w.kvh,
                       tk0, w.b);
-        ++issued;
       }
-      if (*wc.abort) {
-        // never leave copies in flight into shared memory: wait (bounded) for
-        // the last fill of every slot and for Q
-        drain_wait(smem_u32(&bar_q), 0);
-        for (int s = 0; s < NS && s < issued; ++s)
-          drain_wait(smem_u32(&bar_full[s]), ((issued - 1 - s) / NS) & 1);
-      }
+      __syncwarp();
+      ++issued;
+    }
+    if (*wc.abort && lane == 0) {
+      // never leave copies in flight into shared memory: wait (bounded) for
+      // the last fill of every slot and for Q
+      drain_wait(smem_u32(&bar_q), 0);
+      for (int s = 0; s < NS && s < issued; ++s)
+        drain_wait(smem_u32(&bar_full[s]), ((issued - 1 - s) / NS) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ UMMA issuer
-    if (lane == 0) {
-      const uint32_t idS = make_idesc_bf16(128, C::BN, 0, 0);  // Q K-major, K K-major
-      const uint32_t idO = make_idesc_bf16(128, D, 0, 1);      // P from TMEM, V MN-major
-      // S_j = Q K_j^T into S buffer j&1; releases K_j's slot when done
-      auto issue_qk = [&](int j) -> bool {
-        const int L = 2 * j, s = L % NS;
-        if (!mbar_wait(smem_u32(&bar_full[s]), (L / NS) & 1, wc, 22)) return false;
-        tc_fence_after();
-        const uint32_t k_base = slot_addr(s);
+    // (whole warp converged; one elected lane issues each batch)
+    const uint32_t idS = make_idesc_bf16(128, C::BN, 0, 0);  // Q K-major, K K-major
+    const uint32_t idO = make_idesc_bf16(128, D, 0, 1);      // P from TMEM, V MN-major
+    // operand descriptors: built once, then advanced by constants
+    const uint64_t dQ0 = make_sdesc_sw128(sQ, 16, 1024);                      // K-major
+    const uint64_t dK0 = make_sdesc_sw128(slot_addr(0), 16, 1024);            // K-major
+    const uint64_t dV0 = make_sdesc_sw128(slot_addr(0), C::ATOM_BYTES, 1024);  // MN-major
+    // S_j = Q K_j^T into S buffer j&1; releases K_j's slot when done
+    auto issue_qk = [&](int j) -> bool {
+      const int L = 2 * j, s = L % NS;
+      if (!warp_wait(smem_u32(&bar_full[s]), (L / NS) & 1, wc, 22)) return false;
+      tc_fence_after();
+      const uint64_t dk = sdesc_advance(dK0, s * C::KV_BYTES);
+      const uint32_t tS = tmem + (j & 1) * 128;
+      if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::ATOM_BYTES + (kk & 3) * 32;
-          umma_ss(tmem + (j & 1) * 128, make_sdesc_sw128(sQ + off, 16, 1024),
-                  make_sdesc_sw128(k_base + off, 16, 1024), idS, kk > 0);
+          umma_ss(tS, sdesc_advance(dQ0, off), sdesc_advance(dk, off), idS, kk > 0);
         }
         umma_commit(smem_u32(&bar_s[j & 1]));
         umma_commit(smem_u32(&bar_empty[s]));
-        return true;
-      };
-      bool ok = mbar_wait(smem_u32(&bar_q), 0, wc, 20) && issue_qk(0);
-      for (int j = 0; ok && j < nkv; ++j) {
-        if (j + 1 < nkv && !issue_qk(j + 1)) break;
-        const int L = 2 * j + 1, s = L % NS;
-        if (!mbar_wait(smem_u32(&bar_p[j & 1]), (j >> 1) & 1, wc, 23)) break;
-        if (!mbar_wait(smem_u32(&bar_full[s]), (L / NS) & 1, wc, 24)) break;
-        tc_fence_after();
-        const uint32_t tP = tmem + (j & 1) * 128;
-        const uint32_t v_base = slot_addr(s);
+      }
+      __syncwarp();
+      return true;
+    };
+    bool ok = warp_wait(smem_u32(&bar_q), 0, wc, 20) && issue_qk(0);
+    for (int j = 0; ok && j < nkv; ++j) {
+      if (j + 1 < nkv && !issue_qk(j + 1)) break;
+      const int L = 2 * j + 1, s = L % NS;
+      if (!warp_wait(smem_u32(&bar_p[j & 1]), (j >> 1) & 1, wc, 23)) break;
+      if (!warp_wait(smem_u32(&bar_full[s]), (L / NS) & 1, wc, 24)) break;
+      tc_fence_after();
+      const uint32_t tP = tmem + (j & 1) * 128;
+      const uint64_t dv = sdesc_advance(dV0, s * C::KV_BYTES);
+      if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < C::BN / 16; ++kk)
-          umma_ts(tmem + C::TM_O, tP + kk * 8, make_sdesc_sw128(v_base + kk * 2048, C::ATOM_BYTES, 1024),
-                  idO, (j > 0 || kk > 0));
+          umma_ts(tmem + C::TM_O, tP + kk * 8, sdesc_advance(dv, kk * 2048), idO, (j > 0 || kk > 0));
         umma_commit(smem_u32(&bar_o));
         umma_commit(smem_u32(&bar_empty[s]));
       }
-      // every issued UMMA completes before TMEM is released
+      __syncwarp();
+    }
+    // every issued UMMA completes before TMEM is released
+    if (elect_one()) {
       umma_commit(smem_u32(&bar_drain));
       drain_wait(smem_u32(&bar_drain), 0);
     }
+    __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax
     // Two warpgroups share every query row: warps 2..5 take key columns
