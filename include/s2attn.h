@@ -82,8 +82,9 @@ S2ATTN_API int s2attn_fwd(const void* q, const void* k, const void* v, void* o, 
                int B, int H, int Hkv, int N, int D, int G, s2attn_stream_t stream);
 
 /*
- * Bytes of device workspace s2attn_bwd needs: Delta (fp32 [B, H, N],
- * Delta_t = sum_d dO_td * O_td) plus a 256-byte device status block.
+ * Bytes of device workspace s2attn_bwd needs: a 256-byte device status block,
+ * then two fp32 [B, H, N] arrays written by the backward's first kernel:
+ * -Delta (Delta_t = sum_d dO_td * O_td) and -lse_t * log2(e).
  */
 S2ATTN_API size_t s2attn_bwd_workspace_bytes(int B, int H, int Hkv, int N, int D, int G);
 
@@ -120,6 +121,14 @@ S2ATTN_API const char* s2attn_status_string(int status);
  * to the device word *status_out.  No fault, trap or endless spin is involved.
  */
 S2ATTN_API int s2attn_selftest_wait_timeout(uint32_t* status_out, uint64_t limit_ns, s2attn_stream_t stream);
+
+/*
+ * Test hook for the forward kernel's FMA-pipe exponential: writes
+ * y_poly[i] = the kernel's 2^x (Cody-Waite split plus a minimax cubic) and
+ * y_ref[i] = CUDA's exp2f(x[i]) for n device floats.  Asynchronous on stream.
+ */
+S2ATTN_API int s2attn_selftest_exp2(const float* x, float* y_poly, float* y_ref, int n,
+                                    s2attn_stream_t stream);
 
 /* Number of kernel launches the last s2attn_fwd / s2attn_bwd call made on this host thread. */
 S2ATTN_API int s2attn_last_launch_count(void);

@@ -8,7 +8,8 @@
 //   dQ = scale dS K,  dK = scale dS^T Q,  dV = P^T dO.
 //
 // Three kernels run in order on one stream:
-//   s2_bwd_pre_kernel   Delta and lse*log2(e) per query row (HBM-bound).
+//   s2_bwd_pre_kernel   -Delta and -lse*log2(e) per query row (HBM-bound); stored
+//                       negated so each score needs one fused multiply-add.
 //   s2_bwd_dkdv_kernel  one CTA per 128-row kv tile of a kv-head; loops over the
 //                       kv-head's query heads and the query tiles from the
 //                       diagonal to the end of the group.  S^T = K Q^T and
@@ -83,8 +84,8 @@ __global__ void __launch_bounds__(256) s2_bwd_pre_kernel(const BwdPreArgs a) {
       const int t = static_cast<int>(bt % d.N);
       const int b = static_cast<int>(bt / d.N);
       const size_t idx = (static_cast<size_t>(b) * d.H + h) * d.N + t;
-      a.delta[idx] = acc;
-      a.lse2[idx] = a.lse[idx] * kLog2e;
+      a.ndelta[idx] = -acc;
+      a.nlse2[idx] = -a.lse[idx] * kLog2e;
     }
   }
 }
@@ -127,7 +128,7 @@ struct DkvCfg {
   static constexpr int OFF_V = KV_BYTES;
   static constexpr int OFF_Q = 2 * KV_BYTES;
   static constexpr int OFF_DO = OFF_Q + STAGES * Q_BYTES;
-  static constexpr int OFF_ROW = OFF_DO + STAGES * Q_BYTES;  // per stage: lse2[64], delta[64]
+  static constexpr int OFF_ROW = OFF_DO + STAGES * Q_BYTES;  // per stage: -lse2[64], -delta[64]
   static constexpr int SMEM_BYTES = OFF_ROW + STAGES * 512 + 1024;
   static constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DV = 256, TM_DK = 256 + D;
   static constexpr int THREADS = 320;
@@ -217,8 +218,8 @@ __global__ void __launch_bounds__(320, 1)
           tma_load_4d(sG(s) + c * C::Q_ATOM, &tmG, bar, c * 64, h, tq0, w.b);
         }
         const size_t ro = (static_cast<size_t>(w.b) * d.H + h) * d.N + tq0;
-        bulk_load(sRow(s), a.lse2 + ro, 256, bar);
-        bulk_load(sRow(s) + 256, a.delta + ro, 256, bar);
+        bulk_load(sRow(s), a.nlse2 + ro, 256, bar);
+        bulk_load(sRow(s) + 256, a.ndelta + ro, 256, bar);
       }
       __syncwarp();
       ++issued;
@@ -319,14 +320,19 @@ __global__ void __launch_bounds__(320, 1)
       tmem_ld32(tmem + lane_off + C::TM_S + bo, sr);
       tmem_ld32(tmem + lane_off + C::TM_DP + bo, dr);
       tmem_wait_ld();
+      const uint64_t sl2x2 = f2_pack(sl2, sl2);
       float p[32];
 #pragma unroll
-      for (int c4 = 0; c4 < 8; ++c4) {
+      for (int c4 = 0; c4 < 8; ++c4) {  // P^T = 2^(S^T * scale * log2 e - lse * log2 e)
         const float4 l = l4[c4];
-        p[4 * c4 + 0] = ex2_approx(fmaf(__uint_as_float(sr[4 * c4 + 0]), sl2, -l.x));
-        p[4 * c4 + 1] = ex2_approx(fmaf(__uint_as_float(sr[4 * c4 + 1]), sl2, -l.y));
-        p[4 * c4 + 2] = ex2_approx(fmaf(__uint_as_float(sr[4 * c4 + 2]), sl2, -l.z));
-        p[4 * c4 + 3] = ex2_approx(fmaf(__uint_as_float(sr[4 * c4 + 3]), sl2, -l.w));
+        const uint64_t x01 = f2_fma(f2_pack(__uint_as_float(sr[4 * c4]), __uint_as_float(sr[4 * c4 + 1])),
+                                    sl2x2, f2_pack(l.x, l.y));
+        const uint64_t x23 = f2_fma(f2_pack(__uint_as_float(sr[4 * c4 + 2]), __uint_as_float(sr[4 * c4 + 3])),
+                                    sl2x2, f2_pack(l.z, l.w));
+        p[4 * c4 + 0] = ex2_approx(f2_lo(x01));
+        p[4 * c4 + 1] = ex2_approx(f2_hi(x01));
+        p[4 * c4 + 2] = ex2_approx(f2_lo(x23));
+        p[4 * c4 + 3] = ex2_approx(f2_hi(x23));
       }
       if (qoff < kTile) {  // sub-tile overlaps the diagonal: query before key is masked
 #pragma unroll
@@ -338,12 +344,14 @@ __global__ void __launch_bounds__(320, 1)
       for (int c = 0; c < 16; ++c) pk[c] = pack_bf16x2(p[2 * c], p[2 * c + 1]);
       tmem_st16(tmem + lane_off + C::TM_S + bo, pk);
 #pragma unroll
-      for (int c4 = 0; c4 < 8; ++c4) {
+      for (int c4 = 0; c4 < 8; ++c4) {  // dS^T = P^T * (dP^T - Delta)
         const float4 dl = d4[c4];
-        dk[2 * c4] = pack_bf16x2(p[4 * c4] * (__uint_as_float(dr[4 * c4]) - dl.x),
-                                 p[4 * c4 + 1] * (__uint_as_float(dr[4 * c4 + 1]) - dl.y));
-        dk[2 * c4 + 1] = pack_bf16x2(p[4 * c4 + 2] * (__uint_as_float(dr[4 * c4 + 2]) - dl.z),
-                                     p[4 * c4 + 3] * (__uint_as_float(dr[4 * c4 + 3]) - dl.w));
+        const uint64_t d01 = f2_add(f2_pack(__uint_as_float(dr[4 * c4]), __uint_as_float(dr[4 * c4 + 1])),
+                                    f2_pack(dl.x, dl.y));
+        const uint64_t d23 = f2_add(f2_pack(__uint_as_float(dr[4 * c4 + 2]), __uint_as_float(dr[4 * c4 + 3])),
+                                    f2_pack(dl.z, dl.w));
+        dk[2 * c4] = f2_to_bf16x2(f2_mul(f2_pack(p[4 * c4], p[4 * c4 + 1]), d01));
+        dk[2 * c4 + 1] = f2_to_bf16x2(f2_mul(f2_pack(p[4 * c4 + 2], p[4 * c4 + 3]), d23));
       }
       tmem_st16(tmem + lane_off + C::TM_DP + bo, dk);
       tmem_wait_st();
@@ -561,8 +569,9 @@ __global__ void __launch_bounds__(320, 1)
     const float sl2 = a.scale_log2;
     const int t = tq0 + row;
     const size_t ridx = (static_cast<size_t>(w.b) * d.H + w.h) * d.N + t;
-    const float lse2 = a.lse2[ridx];
-    const float delta = a.delta[ridx];
+    const uint64_t nl2 = f2_pack(a.nlse2[ridx], a.nlse2[ridx]);    // -lse * log2 e
+    const uint64_t nd2 = f2_pack(a.ndelta[ridx], a.ndelta[ridx]);  // -Delta
+    const uint64_t sl2x2 = f2_pack(sl2, sl2);
     bool ok = true;
     for (int j = 0; j < nkv; ++j) {
       const uint32_t bo = (j & 1) * kSub + half * 32;
@@ -577,7 +586,11 @@ __global__ void __launch_bounds__(320, 1)
       tmem_wait_ld();
       float p[32];
 #pragma unroll
-      for (int c = 0; c < 32; ++c) p[c] = ex2_approx(fmaf(__uint_as_float(sr[c]), sl2, -lse2));
+      for (int c = 0; c < 16; ++c) {  // P = 2^(S * scale * log2 e - lse * log2 e)
+        const uint64_t x = f2_fma(f2_pack(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])), sl2x2, nl2);
+        p[2 * c] = ex2_approx(f2_lo(x));
+        p[2 * c + 1] = ex2_approx(f2_hi(x));
+      }
       if (koff >= 0) {  // sub-tile overlaps the diagonal: key after query is masked
 #pragma unroll
         for (int c = 0; c < 32; ++c)
@@ -585,9 +598,9 @@ __global__ void __launch_bounds__(320, 1)
       }
       uint32_t pk[16];
 #pragma unroll
-      for (int c = 0; c < 16; ++c)
-        pk[c] = pack_bf16x2(p[2 * c] * (__uint_as_float(dr[2 * c]) - delta),
-                            p[2 * c + 1] * (__uint_as_float(dr[2 * c + 1]) - delta));
+      for (int c = 0; c < 16; ++c)  // dS = P * (dP - Delta)
+        pk[c] = f2_to_bf16x2(f2_mul(f2_pack(p[2 * c], p[2 * c + 1]),
+                                    f2_add(f2_pack(__uint_as_float(dr[2 * c]), __uint_as_float(dr[2 * c + 1])), nd2)));
       tmem_st16(tmem + lane_off + C::TM_DP + bo, pk);
       tmem_wait_st();
       tc_fence_before();

@@ -86,8 +86,8 @@ struct BwdPreArgs {
   const void* o;           // bf16 [B, N, H, D]
   const void* dO;          // bf16 [B, N, H, D]
   const float* lse;        // fp32 [B, H, N]
-  float* delta;            // fp32 [B, H, N]: sum_d dO * O
-  float* lse2;             // fp32 [B, H, N]: lse * log2(e)
+  float* ndelta;           // fp32 [B, H, N]: -Delta = -sum_d dO * O
+  float* nlse2;            // fp32 [B, H, N]: -lse * log2(e)
   uint32_t* status;        // device status words, cleared here (first kernel of the call)
 };
 
@@ -95,8 +95,8 @@ struct BwdArgs {
   Dims d;
   float scale;             // 1/sqrt(D)
   float scale_log2;        // scale * log2(e)
-  const float* delta;      // fp32 [B, H, N]
-  const float* lse2;       // fp32 [B, H, N]
+  const float* ndelta;     // fp32 [B, H, N]: -Delta
+  const float* nlse2;      // fp32 [B, H, N]: -lse * log2(e)
   void* dq;                // bf16 [B, N, H, D]
   void* dk;                // bf16 [B, N, Hkv, D]
   void* dv;                // bf16 [B, N, Hkv, D]

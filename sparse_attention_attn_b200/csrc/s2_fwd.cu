@@ -43,6 +43,63 @@ struct FwdCfg {
   static constexpr int THREADS = 320;
 };
 
+// Cubic for 2^f on [-1/2, 1/2], minimax in relative error (derived by
+// derive_exp2_poly.py in this directory; max relative error 7.5e-5 in float32).
+constexpr float kExp2C0 = 9.999280572e-01f;
+constexpr float kExp2C1 = 6.932609677e-01f;
+constexpr float kExp2C2 = 2.426111251e-01f;
+constexpr float kExp2C3 = 5.517166853e-02f;
+
+// 2^x on the FMA pipe (Cody-Waite split x = n + f, n = round(x), f in
+// [-1/2, 1/2]; 2^n added to the exponent field).  x is clamped below at -126
+// so the result stays a (tiny) non-negative float; inputs here are <= 8.
+__device__ __forceinline__ float exp2_fma(float x) {
+  x = fmaxf(x, -126.f);
+  const float t = x + 12582912.f;  // 1.5 * 2^23: round(x) lands in the low mantissa bits
+  const float f = x - (t - 12582912.f);
+  const float p = fmaf(fmaf(fmaf(kExp2C3, f, kExp2C2), f, kExp2C1), f, kExp2C0);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// The same on a packed pair, with f32x2 arithmetic.
+__device__ __forceinline__ uint64_t exp2_fma2(uint64_t x) {
+  const uint64_t xc = f2_pack(fmaxf(f2_lo(x), -126.f), fmaxf(f2_hi(x), -126.f));
+  const uint64_t t = f2_add(xc, f2_pack(12582912.f, 12582912.f));
+  const uint64_t f = f2_add(xc, f2_add(t, f2_pack(-12582912.f, -12582912.f)) ^ 0x8000000080000000ull);
+  uint64_t p = f2_fma(f2_pack(kExp2C3, kExp2C3), f, f2_pack(kExp2C2, kExp2C2));
+  p = f2_fma(p, f, f2_pack(kExp2C1, kExp2C1));
+  p = f2_fma(p, f, f2_pack(kExp2C0, kExp2C0));
+  const uint32_t lo = __float_as_uint(f2_lo(p)) + (static_cast<uint32_t>(t) << 23);
+  const uint32_t hi = __float_as_uint(f2_hi(p)) + (static_cast<uint32_t>(t >> 32) << 23);
+  return (static_cast<uint64_t>(hi) << 32) | lo;
+}
+
+// P for 64 scores of one query row: p = 2^(s * sl2 - m), packed to bf16
+// pairs in pk; returns the fp32 sum.  Arguments and sums use packed f32x2
+// arithmetic; one pair in four takes its exponentials on the FMA pipe
+// (exp2_fma2), the rest on the MUFU (ex2.approx), which balances the pipes.
+__device__ __forceinline__ float softmax_row64(const uint32_t (&sr)[2][32], float sl2, float m,
+                                               uint32_t (&pk)[32]) {
+  const uint64_t sc2 = f2_pack(sl2, sl2), nm2 = f2_pack(-m, -m);
+  uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+  for (int c = 0; c < 32; ++c) {
+    const uint64_t x = f2_fma(f2_pack(__uint_as_float(sr[(2 * c) >> 5][(2 * c) & 31]),
+                                      __uint_as_float(sr[(2 * c + 1) >> 5][(2 * c + 1) & 31])),
+                              sc2, nm2);
+    uint64_t p;
+    if ((c & 3) == 0) {
+      p = exp2_fma2(x);
+    } else {
+      p = f2_pack(ex2_approx(f2_lo(x)), ex2_approx(f2_hi(x)));
+    }
+    pk[c] = f2_to_bf16x2(p);
+    acc[c & 3] = f2_add(acc[c & 3], p);
+  }
+  const uint64_t s = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
+  return f2_lo(s) + f2_hi(s);
+}
+
 template <int D>
 __global__ void __launch_bounds__(320, 1)
     s2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -215,36 +272,37 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
       for (int c = 0; c < 64; ++c) m4[c & 3] = fmaxf(m4[c & 3], __uint_as_float(sr[c >> 5][c & 31]));
       const float mh = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-      // exchange partial maxima with the other half of the row (double-buffered slot)
+      // exchange partial maxima with the other half of the row (double-buffered
+      // slot).  From the second tile on the exchange completes in the
+      // background: P is computed against the running max first and redone
+      // only if the row max grew by more than 2^8 (rare after the first tiles).
       red_max[j & 1][half][row] = mh;
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(smem_u32(&bar_x[j & 1]));
-        ok = mbar_wait(smem_u32(&bar_x[j & 1]), (j >> 1) & 1, wc, 33);
-      }
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) break;
-      const float mx = fmaxf(mh, red_max[j & 1][half ^ 1][row]) * sl2;
-      float alpha = 1.f;
-      bool resc = false;
+      if (lane == 0) mbar_arrive(smem_u32(&bar_x[j & 1]));
+      auto exchange = [&]() -> bool {
+        bool ok2 = true;
+        if (lane == 0) ok2 = mbar_wait(smem_u32(&bar_x[j & 1]), (j >> 1) & 1, wc, 33);
+        return __shfl_sync(0xffffffffu, ok2, 0);
+      };
       if (j == 0) {
-        m_run = mx;
-      } else if (mx > m_run + 8.f) {  // rescale only when the max grows by more than 2^8
-        alpha = ex2_approx(m_run - mx);
-        m_run = mx;
-        resc = true;
+        if (!exchange()) { ok = false; break; }
+        m_run = fmaxf(mh, red_max[0][half ^ 1][row]) * sl2;
       }
       uint32_t pk[32];
-      float r4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const float p0 = ex2_approx(fmaf(__uint_as_float(sr[(2 * c) >> 5][(2 * c) & 31]), sl2, -m_run));
-        const float p1 =
-            ex2_approx(fmaf(__uint_as_float(sr[(2 * c + 1) >> 5][(2 * c + 1) & 31]), sl2, -m_run));
-        pk[c] = pack_bf16x2(p0, p1);
-        r4[c & 3] += p0 + p1;
+      float rs = softmax_row64(sr, sl2, m_run, pk);
+      float alpha = 1.f;
+      bool resc = false;
+      if (j > 0) {
+        if (!exchange()) { ok = false; break; }
+        const float mx = fmaxf(mh, red_max[j & 1][half ^ 1][row]) * sl2;
+        if (mx > m_run + 8.f) {
+          alpha = ex2_approx(m_run - mx);
+          m_run = mx;
+          resc = true;
+          rs = softmax_row64(sr, sl2, m_run, pk);
+        }
       }
-      l_run = l_run * alpha + ((r4[0] + r4[1]) + (r4[2] + r4[3]));
+      l_run = l_run * alpha + rs;
       // P (bf16) over the first 64 columns of this S buffer; both halves read
       // their S columns before the exchange above, so no write races a read
       tmem_st32(tS + half * 32, pk);
@@ -330,6 +388,28 @@ cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
   cudaError_t e = cudaGetLastError();
   prof_after(stream);
   return e;
+}
+
+// Test hook: the FMA-pipe exp2 next to CUDA's exp2f on the same inputs.
+// (pairs go through the packed form the softmax uses; an odd last element
+// through the scalar form)
+__global__ void s2_exp2_selftest_kernel(const float* x, float* y_poly, float* y_ref, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i + 1 < n) {
+    const uint64_t p = exp2_fma2(f2_pack(x[i], x[i + 1]));
+    y_poly[i] = f2_lo(p);
+    y_poly[i + 1] = f2_hi(p);
+    y_ref[i] = exp2f(x[i]);
+    y_ref[i + 1] = exp2f(x[i + 1]);
+  } else if (i < n) {
+    y_poly[i] = exp2_fma(x[i]);
+    y_ref[i] = exp2f(x[i]);
+  }
+}
+
+cudaError_t launch_exp2_selftest(const float* x, float* y_poly, float* y_ref, int n, cudaStream_t stream) {
+  s2_exp2_selftest_kernel<<<((n + 1) / 2 + 255) / 256, 256, 0, stream>>>(x, y_poly, y_ref, n);
+  return cudaGetLastError();
 }
 
 template cudaError_t launch_fwd<64>(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,

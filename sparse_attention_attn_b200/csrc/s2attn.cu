@@ -22,6 +22,7 @@ cudaError_t launch_fwd(const CUtensorMap&, const CUtensorMap&, const CUtensorMap
                        cudaStream_t);
 template <int D>
 cudaError_t launch_bwd(const BwdMaps&, const BwdPreArgs&, const BwdArgs&, int, cudaStream_t, int*);
+cudaError_t launch_exp2_selftest(const float* x, float* y_poly, float* y_ref, int n, cudaStream_t stream);
 }  // namespace s2
 
 namespace {
@@ -306,23 +307,23 @@ int s2attn_bwd(const void* q, const void* k, const void* v, const void* o, const
     return S2ATTN_ERR_CUDA;
   unsigned char* ws = static_cast<unsigned char*>(workspace);
   uint32_t* status = reinterpret_cast<uint32_t*>(ws);
-  float* delta = reinterpret_cast<float*>(ws + kStatusBytes);
-  float* lse2 = reinterpret_cast<float*>(ws + kStatusBytes + rowstat_bytes(B, H, N));
+  float* ndelta = reinterpret_cast<float*>(ws + kStatusBytes);
+  float* nlse2 = reinterpret_cast<float*>(ws + kStatusBytes + rowstat_bytes(B, H, N));
   const Dims d = make_dims(B, H, Hkv, N, D, G);
   BwdPreArgs pre;
   pre.d = d;
   pre.o = o;
   pre.dO = dO;
   pre.lse = lse;
-  pre.delta = delta;
-  pre.lse2 = lse2;
+  pre.ndelta = ndelta;
+  pre.nlse2 = nlse2;
   pre.status = status;
   BwdArgs a;
   a.d = d;
   a.scale = static_cast<float>(1.0 / __builtin_sqrt(static_cast<double>(D)));
   a.scale_log2 = static_cast<float>(1.4426950408889634 / __builtin_sqrt(static_cast<double>(D)));
-  a.delta = delta;
-  a.lse2 = lse2;
+  a.ndelta = ndelta;
+  a.nlse2 = nlse2;
   a.dq = dq;
   a.dk = dk;
   a.dv = dv;
@@ -351,6 +352,16 @@ int s2attn_device_status(void* workspace, s2attn_stream_t stream) {
       return S2ATTN_ERR_CUDA;
   }
   return words[0] == 0 ? S2ATTN_OK : static_cast<int>(words[0]);
+}
+
+int s2attn_selftest_exp2(const float* x, float* y_poly, float* y_ref, int n, s2attn_stream_t stream) {
+  if (!x || !y_poly || !y_ref || n <= 0) return S2ATTN_ERR_INVALID_ARG;
+  DeviceInfo info;
+  if (!device_info(&info)) return S2ATTN_ERR_CUDA;
+  if (!info.ok) return S2ATTN_ERR_UNSUPPORTED;
+  return launch_exp2_selftest(x, y_poly, y_ref, n, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? S2ATTN_OK
+             : S2ATTN_ERR_CUDA;
 }
 
 int s2attn_selftest_wait_timeout(uint32_t* status_out, uint64_t limit_ns, s2attn_stream_t stream) {

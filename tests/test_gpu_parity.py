@@ -140,3 +140,23 @@ def test_bounded_wait_times_out_cleanly():
     # the context still works afterwards
     x = torch.ones(1024, device="cuda")
     assert float(x.sum()) == 1024.0
+
+
+def test_exp2_fma_against_cuda_exp2f():
+    """The forward's FMA-pipe 2^x stays within its derived relative error bound
+    (7.5e-5 plus float32 rounding) of CUDA's exp2f over the range softmax uses."""
+    from sparse_attention_attn_b200 import _lib
+    x = torch.cat([torch.linspace(-125.0, 8.0, 1_000_001), torch.linspace(-1.0, 1.0, 100_001)]).cuda()
+    yp, yr = torch.empty_like(x), torch.empty_like(x)
+    assert _lib.s2attn_selftest_exp2(x.data_ptr(), yp.data_ptr(), yr.data_ptr(), x.numel(),
+                                     torch.cuda.current_stream().cuda_stream) == 0
+    torch.cuda.synchronize()
+    rel = ((yp.double() - yr.double()).abs() / yr.double()).max().item()
+    assert rel < 8e-5, rel
+    # far below the clamp the result is a tiny non-negative number, never garbage
+    x2 = torch.tensor([-1e4, -300.0, -127.0, -126.0, float("-inf")], device="cuda")
+    yp2, yr2 = torch.empty_like(x2), torch.empty_like(x2)
+    _lib.s2attn_selftest_exp2(x2.data_ptr(), yp2.data_ptr(), yr2.data_ptr(), x2.numel(),
+                              torch.cuda.current_stream().cuda_stream)
+    torch.cuda.synchronize()
+    assert bool((yp2 >= 0).all()) and float(yp2.max()) < 1e-37
