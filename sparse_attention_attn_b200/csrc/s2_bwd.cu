@@ -10,16 +10,16 @@
 // Three kernels run in order on one stream:
 //   s2_bwd_pre_kernel   -Delta and -lse*log2(e) per query row (HBM-bound); stored
 //                       negated so each score needs one fused multiply-add.
-//   s2_bwd_dkdv_kernel  one CTA per 128-row kv tile of a kv-head; loops over the
-//                       kv-head's query heads and the query tiles from the
-//                       diagonal to the end of the group.  S^T = K Q^T and
+//   s2_bwd_dkdv_kernel  persistent; per 128-row kv tile of a kv-head it loops over
+//                       the kv-head's query heads and the query sub-tiles from
+//                       the diagonal to the end of the group.  S^T = K Q^T and
 //                       dP^T = V dO^T land in TMEM, P^T and dS^T (bf16) are
 //                       written back over them and feed dV += P^T dO and
 //                       dK += dS^T Q straight from TMEM; dK/dV accumulate in
 //                       TMEM for the whole loop (no atomics).
-//   s2_bwd_dq_kernel    one CTA per 128-row query tile; loops over the kv tiles
-//                       from the group start to the diagonal: S, dP in TMEM,
-//                       dS over dP, dQ += dS K in TMEM.
+//   s2_bwd_dq_kernel    persistent; per 128-row query tile it loops over the kv
+//                       sub-tiles from the group start to the diagonal: S, dP
+//                       in TMEM, dS over dP, dQ += dS K in TMEM.
 //
 // Warp roles of the two UMMA kernels (320 threads): warp 0 TMA producer,
 // warp 1 TMEM owner + UMMA issuer, warps 2..9 elementwise (thread = one TMEM
@@ -104,11 +104,16 @@ __device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const uint32_t (
 
 // ------------------------------------------------------------------ dK / dV
 //
-// One CTA per 128-row kv tile; the query side streams in 64-row sub-tiles.
+// Persistent: one CTA per SM walks its share of 128-row kv tiles (work items,
+// see PairSched).  The query side of each item streams in 64-row sub-tiles.
 // S^T and dP^T (128 kv rows x 64 query columns each) are double-buffered in
-// TMEM, so the UMMAs of sub-tile it+1 run while warps 2..9 turn sub-tile it
-// into P^T and dS^T.  TMEM: S^T [0,128) (two 64-column buffers), dP^T
-// [128,256), dV [256, 256+D), dK [256+D, 256+2D).
+// TMEM, so the UMMAs of sub-tile g+1 run while warps 2..9 turn sub-tile g into
+// P^T and dS^T; the buffers, the Q/dO stages and their barriers run on one
+// sub-tile counter across items.  K/V tiles are double-buffered across items,
+// so the next item's K/V load overlaps the current item.  TMEM: S^T [0,128)
+// (two 64-column buffers), dP^T [128,256), dV [256, 256+D), dK [256+D, 256+2D);
+// dV/dK are read out by the epilogue of an item before the next item's first
+// gradient UMMA overwrites them (acc_full / acc_free handshake).
 
 constexpr int kSub = 64;  // rows of a streamed sub-tile
 
@@ -124,14 +129,36 @@ struct DkvCfg {
   static constexpr int Q_ATOM = kSub * 128;    // one 64-column slab of a 64-row tile
   static constexpr int KV_BYTES = kTile * D * 2;
   static constexpr int Q_BYTES = kSub * D * 2;
-  static constexpr int OFF_K = 0;
-  static constexpr int OFF_V = KV_BYTES;
-  static constexpr int OFF_Q = 2 * KV_BYTES;
+  static constexpr int OFF_KV = 0;  // [2 buffers][K, V]
+  static constexpr int OFF_Q = 4 * KV_BYTES;
   static constexpr int OFF_DO = OFF_Q + STAGES * Q_BYTES;
   static constexpr int OFF_ROW = OFF_DO + STAGES * Q_BYTES;  // per stage: -lse2[64], -delta[64]
   static constexpr int SMEM_BYTES = OFF_ROW + STAGES * 512 + 1024;
   static constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DV = 256, TM_DK = 256 + D;
   static constexpr int THREADS = 320;
+};
+
+// Sub-tile cursor of the dK/dV kernel: item (kv tile) plus sub-tile index.
+struct DkvCursor {
+  ItemCursor ic;
+  TileWork w;
+  int it, iters, nq;
+  __device__ __forceinline__ void load(const Dims& d, const PairSched& ps) {
+    if (!ic.valid) return;
+    w = kv_item(d, ic.unit, ic.tile);
+    nq = 2 * (d.tiles - w.tile);  // 64-row query sub-tiles from the diagonal to the group end
+    iters = d.rep * nq;
+    it = 0;
+  }
+  __device__ __forceinline__ void first(const Dims& d, const PairSched& ps) {
+    ic.first(ps);
+    load(d, ps);
+  }
+  __device__ __forceinline__ void next(const Dims& d, const PairSched& ps) {
+    if (++it < iters) return;
+    ic.next(ps);
+    load(d, ps);
+  }
 };
 
 template <int D>
@@ -144,38 +171,37 @@ __global__ void __launch_bounds__(320, 1)
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  __shared__ __align__(8) uint64_t bar_kv, bar_full[ST], bar_empty[ST], bar_sdp[2], bar_pds[2],
-      bar_done, bar_drain;
+  __shared__ __align__(8) uint64_t bar_kv[2], bar_kv_empty[2], bar_full[ST], bar_empty[ST], bar_sdp[2],
+      bar_pds[2], bar_acc_full, bar_acc_free, bar_drain;
   __shared__ uint32_t tmem_slot;
   __shared__ uint32_t abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const Dims& d = a.d;
-  const TileWork w = decode_kv_tile(d, blockIdx.x);
-  const int sh = shift_of_head(d, w.h);
-  const int tk0 = original_row(d, w.g * d.G + w.tile * kTile, sh);
-  const int nq = 2 * (d.tiles - w.tile);  // 64-row query sub-tiles from the diagonal to the group end
-  const int iters = d.rep * nq;
+  const PairSched& ps = a.kv_sched;
   WaitCtx wc{&abort_flag, a.status, a.wait_limit_ns};
 
   const uint32_t s0 = smem_u32(smem);
-  const uint32_t sK = s0 + C::OFF_K, sV = s0 + C::OFF_V;
+  auto sK = [&](int kb) { return s0 + C::OFF_KV + kb * 2 * C::KV_BYTES; };
+  auto sV = [&](int kb) { return s0 + C::OFF_KV + kb * 2 * C::KV_BYTES + C::KV_BYTES; };
   auto sQ = [&](int s) { return s0 + C::OFF_Q + s * C::Q_BYTES; };
   auto sG = [&](int s) { return s0 + C::OFF_DO + s * C::Q_BYTES; };
   auto sRow = [&](int s) { return s0 + C::OFF_ROW + s * 512; };
 
   if (threadIdx.x == 0) {
     abort_flag = 0;
-    mbar_init(smem_u32(&bar_kv), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&bar_kv[i]), 1);
+      mbar_init(smem_u32(&bar_kv_empty[i]), 1);
+      mbar_init(smem_u32(&bar_sdp[i]), 1);
+      mbar_init(smem_u32(&bar_pds[i]), 8);  // one elected arrival per elementwise warp
+    }
     for (int s = 0; s < ST; ++s) {
       mbar_init(smem_u32(&bar_full[s]), 1);
       mbar_init(smem_u32(&bar_empty[s]), 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(smem_u32(&bar_sdp[i]), 1);
-      mbar_init(smem_u32(&bar_pds[i]), 256);
-    }
-    mbar_init(smem_u32(&bar_done), 1);
+    mbar_init(smem_u32(&bar_acc_full), 1);
+    mbar_init(smem_u32(&bar_acc_free), 8);
     mbar_init(smem_u32(&bar_drain), 1);
     fence_barrier_init();
   }
@@ -196,121 +222,164 @@ __global__ void __launch_bounds__(320, 1)
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
       tma_prefetch_desc(&tmG);
-      mbar_arrive_expect_tx(smem_u32(&bar_kv), 2 * C::KV_BYTES);
-      for (int c = 0; c < D / 64; ++c) {
-        tma_load_4d(sK + c * C::KV_ATOM, &tmK, smem_u32(&bar_kv), c * 64, w.kvh, tk0, w.b);
-        tma_load_4d(sV + c * C::KV_ATOM, &tmV, smem_u32(&bar_kv), c * 64, w.kvh, tk0, w.b);
-      }
     }
     __syncwarp();
-    int issued = 0;
-    for (int it = 0; it < iters; ++it) {
-      const int s = it % ST, n = it / ST;
-      if (n > 0 && !warp_wait(smem_u32(&bar_empty[s]), (n - 1) & 1, wc, 110)) break;
-      const int h = w.kvh * d.rep + it / nq;
-      const int i64 = 2 * w.tile + it % nq;
-      const int tq0 = original_row(d, w.g * d.G + i64 * kSub, sh);
-      const uint32_t bar = smem_u32(&bar_full[s]);
+    int gi = 0, kv_issued = 0;
+    bool ok = true;
+    ItemCursor ic;
+    for (ic.first(ps); ok && ic.valid; ic.next(ps)) {
+      const TileWork w = kv_item(d, ic.unit, ic.tile);
+      const int sh = shift_of_head(d, w.h);
+      const int kb = ic.n & 1;
+      if (ic.n >= 2 && !warp_wait(smem_u32(&bar_kv_empty[kb]), ((ic.n >> 1) - 1) & 1, wc, 109)) break;
+      const int tk0 = original_row(d, w.g * d.G + w.tile * kTile, sh);
       if (elect_one()) {
-        mbar_arrive_expect_tx(bar, 2 * C::Q_BYTES + 512);
+        mbar_arrive_expect_tx(smem_u32(&bar_kv[kb]), 2 * C::KV_BYTES);
         for (int c = 0; c < D / 64; ++c) {
-          tma_load_4d(sQ(s) + c * C::Q_ATOM, &tmQ, bar, c * 64, h, tq0, w.b);
-          tma_load_4d(sG(s) + c * C::Q_ATOM, &tmG, bar, c * 64, h, tq0, w.b);
+          tma_load_4d(sK(kb) + c * C::KV_ATOM, &tmK, smem_u32(&bar_kv[kb]), c * 64, w.kvh, tk0, w.b);
+          tma_load_4d(sV(kb) + c * C::KV_ATOM, &tmV, smem_u32(&bar_kv[kb]), c * 64, w.kvh, tk0, w.b);
         }
-        const size_t ro = (static_cast<size_t>(w.b) * d.H + h) * d.N + tq0;
-        bulk_load(sRow(s), a.nlse2 + ro, 256, bar);
-        bulk_load(sRow(s) + 256, a.ndelta + ro, 256, bar);
       }
       __syncwarp();
-      ++issued;
+      ++kv_issued;
+      const int nq = 2 * (d.tiles - w.tile);
+      const int iters = d.rep * nq;
+      for (int it = 0; it < iters; ++it, ++gi) {
+        const int s = gi % ST, f = gi / ST;
+        if (f > 0 && !warp_wait(smem_u32(&bar_empty[s]), (f - 1) & 1, wc, 110)) {
+          ok = false;
+          break;
+        }
+        const int h = w.kvh * d.rep + it / nq;
+        const int i64 = 2 * w.tile + it % nq;
+        const int tq0 = original_row(d, w.g * d.G + i64 * kSub, sh);
+        const uint32_t bar = smem_u32(&bar_full[s]);
+        if (elect_one()) {
+          mbar_arrive_expect_tx(bar, 2 * C::Q_BYTES + 512);
+          for (int c = 0; c < D / 64; ++c) {
+            tma_load_4d(sQ(s) + c * C::Q_ATOM, &tmQ, bar, c * 64, h, tq0, w.b);
+            tma_load_4d(sG(s) + c * C::Q_ATOM, &tmG, bar, c * 64, h, tq0, w.b);
+          }
+          const size_t ro = (static_cast<size_t>(w.b) * d.H + h) * d.N + tq0;
+          bulk_load(sRow(s), a.nlse2 + ro, 256, bar);
+          bulk_load(sRow(s) + 256, a.ndelta + ro, 256, bar);
+        }
+        __syncwarp();
+      }
     }
     if (*wc.abort && lane == 0) {
-      drain_wait(smem_u32(&bar_kv), 0);
-      for (int s = 0; s < ST && s < issued; ++s)
-        drain_wait(smem_u32(&bar_full[s]), ((issued - 1 - s) / ST) & 1);
+      // never leave copies in flight into shared memory: wait (bounded) for
+      // the last fill of every stage and K/V buffer
+      for (int kb = 0; kb < 2 && kb < kv_issued; ++kb)
+        drain_wait(smem_u32(&bar_kv[kb]), ((kv_issued - 1 - kb) >> 1) & 1);
+      for (int s = 0; s < ST && s < gi; ++s) drain_wait(smem_u32(&bar_full[s]), ((gi - 1 - s) / ST) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ UMMA issuer
     // (whole warp converged; one elected lane issues each batch)
     const uint32_t idS = make_idesc_bf16(128, kSub, 0, 0);  // S^T = K Q^T, dP^T = V dO^T
     const uint32_t idG = make_idesc_bf16(128, D, 0, 1);     // dV += P^T dO, dK += dS^T Q
-    const uint64_t dK0 = make_sdesc_sw128(sK, 16, 1024);           // K-major (A)
-    const uint64_t dV0 = make_sdesc_sw128(sV, 16, 1024);
-    const uint64_t dQk = make_sdesc_sw128(sQ(0), 16, 1024);        // K-major (B of S^T)
+    const uint64_t dK0 = make_sdesc_sw128(sK(0), 16, 1024);         // K-major (A)
+    const uint64_t dV0 = make_sdesc_sw128(sV(0), 16, 1024);
+    const uint64_t dQk = make_sdesc_sw128(sQ(0), 16, 1024);         // K-major (B of S^T)
     const uint64_t dGk = make_sdesc_sw128(sG(0), 16, 1024);
     const uint64_t dQm = make_sdesc_sw128(sQ(0), C::Q_ATOM, 1024);  // MN-major (B of dK)
     const uint64_t dGm = make_sdesc_sw128(sG(0), C::Q_ATOM, 1024);  // MN-major (B of dV)
-    auto issue_sdp = [&](int it, int s) {
-      const uint32_t bo = (it & 1) * kSub;
+    // S^T and dP^T of global sub-tile g (stage g % ST, K/V buffer kb)
+    auto issue_sdp = [&](int g, int kb) {
+      const int s = g % ST;
+      const uint32_t bo = (g & 1) * kSub;
+      const uint64_t dk = sdesc_advance(dK0, kb * 2 * C::KV_BYTES), dv = sdesc_advance(dV0, kb * 2 * C::KV_BYTES);
       const uint64_t dq = sdesc_advance(dQk, s * C::Q_BYTES), dg = sdesc_advance(dGk, s * C::Q_BYTES);
       if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ko = (kk >> 2) * C::KV_ATOM + (kk & 3) * 32;
           const uint32_t qo = (kk >> 2) * C::Q_ATOM + (kk & 3) * 32;
-          umma_ss(tmem + C::TM_S + bo, sdesc_advance(dK0, ko), sdesc_advance(dq, qo), idS, kk > 0);
+          umma_ss(tmem + C::TM_S + bo, sdesc_advance(dk, ko), sdesc_advance(dq, qo), idS, kk > 0);
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ko = (kk >> 2) * C::KV_ATOM + (kk & 3) * 32;
           const uint32_t qo = (kk >> 2) * C::Q_ATOM + (kk & 3) * 32;
-          umma_ss(tmem + C::TM_DP + bo, sdesc_advance(dV0, ko), sdesc_advance(dg, qo), idS, kk > 0);
+          umma_ss(tmem + C::TM_DP + bo, sdesc_advance(dv, ko), sdesc_advance(dg, qo), idS, kk > 0);
         }
-        umma_commit(smem_u32(&bar_sdp[it & 1]));
+        umma_commit(smem_u32(&bar_sdp[g & 1]));
       }
       __syncwarp();
     };
-    bool ok = warp_wait(smem_u32(&bar_kv), 0, wc, 120) && warp_wait(smem_u32(&bar_full[0]), 0, wc, 121);
-    if (ok) {
+    // make sub-tile g (cursor c) ready: its item's K/V and its Q/dO stage
+    auto wait_inputs = [&](const DkvCursor& c, int g) -> bool {
+      if (c.it == 0 && !warp_wait(smem_u32(&bar_kv[c.ic.n & 1]), (c.ic.n >> 1) & 1, wc, 120)) return false;
+      if (!warp_wait(smem_u32(&bar_full[g % ST]), (g / ST) & 1, wc, 121)) return false;
       tc_fence_after();
-      issue_sdp(0, 0);
+      return true;
+    };
+    DkvCursor cur, nxt;
+    cur.first(d, ps);
+    nxt = cur;
+    nxt.next(d, ps);
+    bool ok = true;
+    if (cur.ic.valid) {
+      ok = wait_inputs(cur, 0);
+      if (ok) issue_sdp(0, cur.ic.n & 1);
     }
-    for (int it = 0; ok && it < iters; ++it) {
-      const int s = it % ST;
-      if (it + 1 < iters) {
-        const int s1 = (it + 1) % ST;
-        if (!warp_wait(smem_u32(&bar_full[s1]), ((it + 1) / ST) & 1, wc, 122)) break;
-        tc_fence_after();
-        issue_sdp(it + 1, s1);  // its TMEM buffer's last readers were issued before: in order
+    for (int g = 0; ok && cur.ic.valid; ++g) {
+      if (nxt.ic.valid) {  // S^T/dP^T of the next sub-tile (possibly the next item's first)
+        if (!wait_inputs(nxt, g + 1)) break;
+        issue_sdp(g + 1, nxt.ic.n & 1);  // its TMEM buffer's last readers were issued before: in order
       }
-      if (!warp_wait(smem_u32(&bar_pds[it & 1]), (it >> 1) & 1, wc, 123)) break;
+      if (!warp_wait(smem_u32(&bar_pds[g & 1]), (g >> 1) & 1, wc, 123)) break;
+      if (cur.it == 0 && cur.ic.n > 0 &&
+          !warp_wait(smem_u32(&bar_acc_free), (cur.ic.n - 1) & 1, wc, 124))
+        break;
       tc_fence_after();
-      const uint32_t bo = (it & 1) * kSub;
+      const int s = g % ST;
+      const uint32_t bo = (g & 1) * kSub;
       const uint64_t dg = sdesc_advance(dGm, s * C::Q_BYTES), dq = sdesc_advance(dQm, s * C::Q_BYTES);
+      const bool last = (cur.it == cur.iters - 1);
       if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < kSub / 16; ++kk)
           umma_ts(tmem + C::TM_DV, tmem + C::TM_S + bo + split_acol64(kk), sdesc_advance(dg, kk * 2048),
-                  idG, (it > 0 || kk > 0));
+                  idG, (cur.it > 0 || kk > 0));
 #pragma unroll
         for (int kk = 0; kk < kSub / 16; ++kk)
           umma_ts(tmem + C::TM_DK, tmem + C::TM_DP + bo + split_acol64(kk), sdesc_advance(dq, kk * 2048),
-                  idG, (it > 0 || kk > 0));
+                  idG, (cur.it > 0 || kk > 0));
         umma_commit(smem_u32(&bar_empty[s]));
+        if (last) {
+          umma_commit(smem_u32(&bar_acc_full));
+          umma_commit(smem_u32(&bar_kv_empty[cur.ic.n & 1]));
+        }
       }
       __syncwarp();
+      cur = nxt;
+      nxt.next(d, ps);
     }
     if (elect_one()) {
-      umma_commit(smem_u32(&bar_done));
       umma_commit(smem_u32(&bar_drain));
       drain_wait(smem_u32(&bar_drain), 0);
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ P^T, dS^T
+    // ------------------------------------------------------------ P^T, dS^T, epilogue
     const int quarter = warp & 3;
     const int half = (warp - 2) >> 2;
     const int row = quarter * 32 + lane;  // kv row inside the tile
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const float sl2 = a.scale_log2;
+    const uint64_t sl2x2 = f2_pack(sl2, sl2);
     bool ok = true;
-    for (int it = 0; it < iters; ++it) {
-      const int s = it % ST;
-      const int qoff = (it % nq) * kSub;  // query sub-tile start minus kv tile start (rolled)
-      const uint32_t bo = (it & 1) * kSub + half * 32;
+    DkvCursor cur;
+    cur.first(d, ps);
+    for (int g = 0; cur.ic.valid; ++g) {
+      const int s = g % ST;
+      const int qoff = (cur.it % cur.nq) * kSub;  // query sub-tile start minus kv tile start (rolled)
+      const uint32_t bo = (g & 1) * kSub + half * 32;
       if (lane == 0)
-        ok = mbar_wait(smem_u32(&bar_full[s]), (it / ST) & 1, wc, 130) &&
-             mbar_wait(smem_u32(&bar_sdp[it & 1]), (it >> 1) & 1, wc, 131);
+        ok = mbar_wait(smem_u32(&bar_full[s]), (g / ST) & 1, wc, 130) &&
+             mbar_wait(smem_u32(&bar_sdp[g & 1]), (g >> 1) & 1, wc, 131);
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       tc_fence_after();
@@ -320,7 +389,6 @@ __global__ void __launch_bounds__(320, 1)
       tmem_ld32(tmem + lane_off + C::TM_S + bo, sr);
       tmem_ld32(tmem + lane_off + C::TM_DP + bo, dr);
       tmem_wait_ld();
-      const uint64_t sl2x2 = f2_pack(sl2, sl2);
       float p[32];
 #pragma unroll
       for (int c4 = 0; c4 < 8; ++c4) {  // P^T = 2^(S^T * scale * log2 e - lse * log2 e)
@@ -356,29 +424,33 @@ __global__ void __launch_bounds__(320, 1)
       tmem_st16(tmem + lane_off + C::TM_DP + bo, dk);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(smem_u32(&bar_pds[it & 1]));
-    }
-    // ------------------------------------------------------------ epilogue
-    if (ok) {
-      if (lane == 0) ok = mbar_wait(smem_u32(&bar_done), 0, wc, 132);
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-    }
-    if (ok) {
-      tc_fence_after();
-      const size_t grow = (static_cast<size_t>(w.b) * d.N + tk0 + row) * d.Hkv + w.kvh;
-      __nv_bfloat16* dvrow = static_cast<__nv_bfloat16*>(a.dv) + grow * D + half * (D / 2);
-      __nv_bfloat16* dkrow = static_cast<__nv_bfloat16*>(a.dk) + grow * D + half * (D / 2);
-      const float sc = a.scale;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bar_pds[g & 1]));
+      if (cur.it == cur.iters - 1) {
+        // ---------------------------------------------------- epilogue of this item
+        if (lane == 0) ok = mbar_wait(smem_u32(&bar_acc_full), cur.ic.n & 1, wc, 132);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        tc_fence_after();
+        const TileWork& w = cur.w;
+        const int tk0 = original_row(d, w.g * d.G + w.tile * kTile, shift_of_head(d, w.h));
+        const size_t grow = (static_cast<size_t>(w.b) * d.N + tk0 + row) * d.Hkv + w.kvh;
+        __nv_bfloat16* dvrow = static_cast<__nv_bfloat16*>(a.dv) + grow * D + half * (D / 2);
+        __nv_bfloat16* dkrow = static_cast<__nv_bfloat16*>(a.dk) + grow * D + half * (D / 2);
 #pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tmem + lane_off + C::TM_DV + half * (D / 2) + c * 32, r);
-        tmem_wait_ld();
-        store_row32(dvrow + c * 32, r, 1.f);
-        tmem_ld32(tmem + lane_off + C::TM_DK + half * (D / 2) + c * 32, r);
-        tmem_wait_ld();
-        store_row32(dkrow + c * 32, r, sc);
+        for (int c = 0; c < D / 64; ++c) {
+          uint32_t r[32], r2[32];
+          tmem_ld32(tmem + lane_off + C::TM_DV + half * (D / 2) + c * 32, r);
+          tmem_ld32(tmem + lane_off + C::TM_DK + half * (D / 2) + c * 32, r2);
+          tmem_wait_ld();
+          store_row32(dvrow + c * 32, r, 1.f);
+          store_row32(dkrow + c * 32, r2, a.scale);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bar_acc_free));
       }
+      cur.next(d, ps);
     }
   }
 
@@ -392,25 +464,47 @@ __global__ void __launch_bounds__(320, 1)
 
 // ------------------------------------------------------------------ dQ
 //
-// One CTA per 128-row query tile; keys/values stream in 64-row sub-tiles from
-// the group start to the diagonal.  S and dP (128 x 64) are double-buffered in
-// TMEM so the UMMAs of sub-tile j+1 overlap the dS work on sub-tile j.
-// TMEM: S [0,128) (two buffers), dP [128,256), dQ [256, 256+D).
+// Persistent: one CTA per SM walks its share of 128-row query tiles.  Keys and
+// values of each item stream in 64-row sub-tiles from the group start to the
+// diagonal.  S and dP (128 x 64) are double-buffered in TMEM so the UMMAs of
+// sub-tile g+1 overlap the dS work on sub-tile g; Q/dO are double-buffered
+// across items.  TMEM: S [0,128) (two buffers), dP [128,256), dQ [256, 256+D);
+// dQ is read out by the item's epilogue before the next item overwrites it.
 
 template <int D>
 struct DqCfg {
-  static constexpr int STAGES = 4;
+  static constexpr int STAGES = 3;
   static constexpr int Q_ATOM = kTile * 128;
   static constexpr int KV_ATOM = kSub * 128;
   static constexpr int Q_BYTES = kTile * D * 2;
   static constexpr int KV_BYTES = kSub * D * 2;
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_DO = Q_BYTES;
-  static constexpr int OFF_K = 2 * Q_BYTES;
+  static constexpr int OFF_Q = 0;  // [2 buffers][Q, dO]
+  static constexpr int OFF_K = 4 * Q_BYTES;
   static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
   static constexpr int SMEM_BYTES = OFF_V + STAGES * KV_BYTES + 1024;
   static constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DQ = 256;
   static constexpr int THREADS = 320;
+};
+
+struct DqCursor {
+  ItemCursor ic;
+  TileWork w;
+  int it, iters;
+  __device__ __forceinline__ void load(const Dims& d) {
+    if (!ic.valid) return;
+    w = q_item(d, ic.unit, ic.tile);
+    iters = 2 * (w.tile + 1);  // 64-row kv sub-tiles from the group start to the diagonal
+    it = 0;
+  }
+  __device__ __forceinline__ void first(const Dims& d, const PairSched& ps) {
+    ic.first(ps);
+    load(d);
+  }
+  __device__ __forceinline__ void next(const Dims& d, const PairSched& ps) {
+    if (++it < iters) return;
+    ic.next(ps);
+    load(d);
+  }
 };
 
 template <int D>
@@ -423,36 +517,36 @@ __global__ void __launch_bounds__(320, 1)
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  __shared__ __align__(8) uint64_t bar_q, bar_kv[ST], bar_empty[ST], bar_sdp[2], bar_ds[2], bar_done,
-      bar_drain;
+  __shared__ __align__(8) uint64_t bar_q[2], bar_q_empty[2], bar_kv[ST], bar_empty[ST], bar_sdp[2],
+      bar_ds[2], bar_acc_full, bar_acc_free, bar_drain;
   __shared__ uint32_t tmem_slot;
   __shared__ uint32_t abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const Dims& d = a.d;
-  const TileWork w = decode_q_tile(d, blockIdx.x);
-  const int sh = shift_of_head(d, w.h);
-  const int tq0 = original_row(d, w.g * d.G + w.tile * kTile, sh);
-  const int nkv = 2 * (w.tile + 1);  // 64-row kv sub-tiles from the group start to the diagonal
+  const PairSched& ps = a.q_sched;
   WaitCtx wc{&abort_flag, a.status, a.wait_limit_ns};
 
   const uint32_t s0 = smem_u32(smem);
-  const uint32_t sQ = s0 + C::OFF_Q, sG = s0 + C::OFF_DO;
+  auto sQ = [&](int qb) { return s0 + C::OFF_Q + qb * 2 * C::Q_BYTES; };
+  auto sG = [&](int qb) { return s0 + C::OFF_Q + qb * 2 * C::Q_BYTES + C::Q_BYTES; };
   auto sK = [&](int s) { return s0 + C::OFF_K + s * C::KV_BYTES; };
   auto sV = [&](int s) { return s0 + C::OFF_V + s * C::KV_BYTES; };
 
   if (threadIdx.x == 0) {
     abort_flag = 0;
-    mbar_init(smem_u32(&bar_q), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&bar_q[i]), 1);
+      mbar_init(smem_u32(&bar_q_empty[i]), 1);
+      mbar_init(smem_u32(&bar_sdp[i]), 1);
+      mbar_init(smem_u32(&bar_ds[i]), 8);  // one elected arrival per elementwise warp
+    }
     for (int s = 0; s < ST; ++s) {
       mbar_init(smem_u32(&bar_kv[s]), 1);
       mbar_init(smem_u32(&bar_empty[s]), 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(smem_u32(&bar_sdp[i]), 1);
-      mbar_init(smem_u32(&bar_ds[i]), 256);
-    }
-    mbar_init(smem_u32(&bar_done), 1);
+    mbar_init(smem_u32(&bar_acc_full), 1);
+    mbar_init(smem_u32(&bar_acc_free), 8);
     mbar_init(smem_u32(&bar_drain), 1);
     fence_barrier_init();
   }
@@ -466,117 +560,158 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t tmem = tmem_slot;
 
   if (warp == 0) {
-    // (whole warp converged; one elected lane issues the copies)
+    // ------------------------------------------------------------ producer
     if (elect_one()) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
       tma_prefetch_desc(&tmG);
-      mbar_arrive_expect_tx(smem_u32(&bar_q), 2 * C::Q_BYTES);
-      for (int c = 0; c < D / 64; ++c) {
-        tma_load_4d(sQ + c * C::Q_ATOM, &tmQ, smem_u32(&bar_q), c * 64, w.h, tq0, w.b);
-        tma_load_4d(sG + c * C::Q_ATOM, &tmG, smem_u32(&bar_q), c * 64, w.h, tq0, w.b);
-      }
     }
     __syncwarp();
-    int issued = 0;
-    for (int j = 0; j < nkv; ++j) {
-      const int s = j % ST, n = j / ST;
-      if (n > 0 && !warp_wait(smem_u32(&bar_empty[s]), (n - 1) & 1, wc, 210)) break;
-      const int tk0 = original_row(d, w.g * d.G + j * kSub, sh);
-      const uint32_t bar = smem_u32(&bar_kv[s]);
+    int gi = 0, q_issued = 0;
+    bool ok = true;
+    ItemCursor ic;
+    for (ic.first(ps); ok && ic.valid; ic.next(ps)) {
+      const TileWork w = q_item(d, ic.unit, ic.tile);
+      const int sh = shift_of_head(d, w.h);
+      const int qb = ic.n & 1;
+      if (ic.n >= 2 && !warp_wait(smem_u32(&bar_q_empty[qb]), ((ic.n >> 1) - 1) & 1, wc, 209)) break;
+      const int tq0 = original_row(d, w.g * d.G + w.tile * kTile, sh);
       if (elect_one()) {
-        mbar_arrive_expect_tx(bar, 2 * C::KV_BYTES);
+        mbar_arrive_expect_tx(smem_u32(&bar_q[qb]), 2 * C::Q_BYTES);
         for (int c = 0; c < D / 64; ++c) {
-          tma_load_4d(sK(s) + c * C::KV_ATOM, &tmK, bar, c * 64, w.kvh, tk0, w.b);
-          tma_load_4d(sV(s) + c * C::KV_ATOM, &tmV, bar, c * 64, w.kvh, tk0, w.b);
+          tma_load_4d(sQ(qb) + c * C::Q_ATOM, &tmQ, smem_u32(&bar_q[qb]), c * 64, w.h, tq0, w.b);
+          tma_load_4d(sG(qb) + c * C::Q_ATOM, &tmG, smem_u32(&bar_q[qb]), c * 64, w.h, tq0, w.b);
         }
       }
       __syncwarp();
-      ++issued;
+      ++q_issued;
+      const int iters = 2 * (w.tile + 1);
+      for (int j = 0; j < iters; ++j, ++gi) {
+        const int s = gi % ST, f = gi / ST;
+        if (f > 0 && !warp_wait(smem_u32(&bar_empty[s]), (f - 1) & 1, wc, 210)) {
+          ok = false;
+          break;
+        }
+        const int tk0 = original_row(d, w.g * d.G + j * kSub, sh);
+        const uint32_t bar = smem_u32(&bar_kv[s]);
+        if (elect_one()) {
+          mbar_arrive_expect_tx(bar, 2 * C::KV_BYTES);
+          for (int c = 0; c < D / 64; ++c) {
+            tma_load_4d(sK(s) + c * C::KV_ATOM, &tmK, bar, c * 64, w.kvh, tk0, w.b);
+            tma_load_4d(sV(s) + c * C::KV_ATOM, &tmV, bar, c * 64, w.kvh, tk0, w.b);
+          }
+        }
+        __syncwarp();
+      }
     }
     if (*wc.abort && lane == 0) {
-      drain_wait(smem_u32(&bar_q), 0);
-      for (int s = 0; s < ST && s < issued; ++s)
-        drain_wait(smem_u32(&bar_kv[s]), ((issued - 1 - s) / ST) & 1);
+      for (int qb = 0; qb < 2 && qb < q_issued; ++qb)
+        drain_wait(smem_u32(&bar_q[qb]), ((q_issued - 1 - qb) >> 1) & 1);
+      for (int s = 0; s < ST && s < gi; ++s) drain_wait(smem_u32(&bar_kv[s]), ((gi - 1 - s) / ST) & 1);
     }
   } else if (warp == 1) {
-    // (whole warp converged; one elected lane issues each batch)
+    // ------------------------------------------------------------ UMMA issuer
     const uint32_t idS = make_idesc_bf16(128, kSub, 0, 0);  // S = Q K^T, dP = dO V^T
     const uint32_t idQ = make_idesc_bf16(128, D, 0, 1);     // dQ += dS K (K MN-major)
-    const uint64_t dQ0 = make_sdesc_sw128(sQ, 16, 1024);               // K-major (A)
-    const uint64_t dG0 = make_sdesc_sw128(sG, 16, 1024);
+    const uint64_t dQ0 = make_sdesc_sw128(sQ(0), 16, 1024);            // K-major (A)
+    const uint64_t dG0 = make_sdesc_sw128(sG(0), 16, 1024);
     const uint64_t dKk = make_sdesc_sw128(sK(0), 16, 1024);            // K-major (B of S)
     const uint64_t dVk = make_sdesc_sw128(sV(0), 16, 1024);
     const uint64_t dKm = make_sdesc_sw128(sK(0), C::KV_ATOM, 1024);    // MN-major (B of dQ)
-    auto issue_sdp = [&](int j, int s) {
-      const uint32_t bo = (j & 1) * kSub;
+    auto issue_sdp = [&](int g, int qb) {
+      const int s = g % ST;
+      const uint32_t bo = (g & 1) * kSub;
+      const uint64_t dq = sdesc_advance(dQ0, qb * 2 * C::Q_BYTES), dgo = sdesc_advance(dG0, qb * 2 * C::Q_BYTES);
       const uint64_t dk = sdesc_advance(dKk, s * C::KV_BYTES), dv = sdesc_advance(dVk, s * C::KV_BYTES);
       if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t qo = (kk >> 2) * C::Q_ATOM + (kk & 3) * 32;
           const uint32_t ko = (kk >> 2) * C::KV_ATOM + (kk & 3) * 32;
-          umma_ss(tmem + C::TM_S + bo, sdesc_advance(dQ0, qo), sdesc_advance(dk, ko), idS, kk > 0);
+          umma_ss(tmem + C::TM_S + bo, sdesc_advance(dq, qo), sdesc_advance(dk, ko), idS, kk > 0);
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t qo = (kk >> 2) * C::Q_ATOM + (kk & 3) * 32;
           const uint32_t ko = (kk >> 2) * C::KV_ATOM + (kk & 3) * 32;
-          umma_ss(tmem + C::TM_DP + bo, sdesc_advance(dG0, qo), sdesc_advance(dv, ko), idS, kk > 0);
+          umma_ss(tmem + C::TM_DP + bo, sdesc_advance(dgo, qo), sdesc_advance(dv, ko), idS, kk > 0);
         }
-        umma_commit(smem_u32(&bar_sdp[j & 1]));
+        umma_commit(smem_u32(&bar_sdp[g & 1]));
       }
       __syncwarp();
     };
-    bool ok = warp_wait(smem_u32(&bar_q), 0, wc, 220) && warp_wait(smem_u32(&bar_kv[0]), 0, wc, 221);
-    if (ok) {
+    auto wait_inputs = [&](const DqCursor& c, int g) -> bool {
+      if (c.it == 0 && !warp_wait(smem_u32(&bar_q[c.ic.n & 1]), (c.ic.n >> 1) & 1, wc, 220)) return false;
+      if (!warp_wait(smem_u32(&bar_kv[g % ST]), (g / ST) & 1, wc, 221)) return false;
       tc_fence_after();
-      issue_sdp(0, 0);
+      return true;
+    };
+    DqCursor cur, nxt;
+    cur.first(d, ps);
+    nxt = cur;
+    nxt.next(d, ps);
+    bool ok = true;
+    if (cur.ic.valid) {
+      ok = wait_inputs(cur, 0);
+      if (ok) issue_sdp(0, cur.ic.n & 1);
     }
-    for (int j = 0; ok && j < nkv; ++j) {
-      const int s = j % ST;
-      if (j + 1 < nkv) {
-        const int s1 = (j + 1) % ST;
-        if (!warp_wait(smem_u32(&bar_kv[s1]), ((j + 1) / ST) & 1, wc, 222)) break;
-        tc_fence_after();
-        issue_sdp(j + 1, s1);
+    for (int g = 0; ok && cur.ic.valid; ++g) {
+      if (nxt.ic.valid) {
+        if (!wait_inputs(nxt, g + 1)) break;
+        issue_sdp(g + 1, nxt.ic.n & 1);
       }
-      if (!warp_wait(smem_u32(&bar_ds[j & 1]), (j >> 1) & 1, wc, 223)) break;
+      if (!warp_wait(smem_u32(&bar_ds[g & 1]), (g >> 1) & 1, wc, 223)) break;
+      if (cur.it == 0 && cur.ic.n > 0 &&
+          !warp_wait(smem_u32(&bar_acc_free), (cur.ic.n - 1) & 1, wc, 224))
+        break;
       tc_fence_after();
-      const uint32_t bo = (j & 1) * kSub;
+      const int s = g % ST;
+      const uint32_t bo = (g & 1) * kSub;
       const uint64_t dk = sdesc_advance(dKm, s * C::KV_BYTES);
+      const bool last = (cur.it == cur.iters - 1);
       if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < kSub / 16; ++kk)
           umma_ts(tmem + C::TM_DQ, tmem + C::TM_DP + bo + split_acol64(kk), sdesc_advance(dk, kk * 2048),
-                  idQ, (j > 0 || kk > 0));
+                  idQ, (cur.it > 0 || kk > 0));
         umma_commit(smem_u32(&bar_empty[s]));
+        if (last) {
+          umma_commit(smem_u32(&bar_acc_full));
+          umma_commit(smem_u32(&bar_q_empty[cur.ic.n & 1]));
+        }
       }
       __syncwarp();
+      cur = nxt;
+      nxt.next(d, ps);
     }
     if (elect_one()) {
-      umma_commit(smem_u32(&bar_done));
       umma_commit(smem_u32(&bar_drain));
       drain_wait(smem_u32(&bar_drain), 0);
     }
     __syncwarp();
   } else {
+    // ------------------------------------------------------------ dS, epilogue
     const int quarter = warp & 3;
     const int half = (warp - 2) >> 2;
     const int row = quarter * 32 + lane;  // query row inside the tile
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const float sl2 = a.scale_log2;
-    const int t = tq0 + row;
-    const size_t ridx = (static_cast<size_t>(w.b) * d.H + w.h) * d.N + t;
-    const uint64_t nl2 = f2_pack(a.nlse2[ridx], a.nlse2[ridx]);    // -lse * log2 e
-    const uint64_t nd2 = f2_pack(a.ndelta[ridx], a.ndelta[ridx]);  // -Delta
-    const uint64_t sl2x2 = f2_pack(sl2, sl2);
+    const uint64_t sl2x2 = f2_pack(a.scale_log2, a.scale_log2);
     bool ok = true;
-    for (int j = 0; j < nkv; ++j) {
-      const uint32_t bo = (j & 1) * kSub + half * 32;
-      const int koff = j * kSub - w.tile * kTile;  // kv sub-tile start minus query tile start
-      if (lane == 0) ok = mbar_wait(smem_u32(&bar_sdp[j & 1]), (j >> 1) & 1, wc, 230);
+    uint64_t nl2 = 0, nd2 = 0;
+    DqCursor cur;
+    cur.first(d, ps);
+    for (int g = 0; cur.ic.valid; ++g) {
+      const TileWork& w = cur.w;
+      const int tq0 = original_row(d, w.g * d.G + w.tile * kTile, shift_of_head(d, w.h));
+      const size_t ridx = (static_cast<size_t>(w.b) * d.H + w.h) * d.N + tq0 + row;
+      if (cur.it == 0) {
+        nl2 = f2_pack(a.nlse2[ridx], a.nlse2[ridx]);    // -lse * log2 e
+        nd2 = f2_pack(a.ndelta[ridx], a.ndelta[ridx]);  // -Delta
+      }
+      const uint32_t bo = (g & 1) * kSub + half * 32;
+      const int koff = cur.it * kSub - w.tile * kTile;  // kv sub-tile start minus query tile start
+      if (lane == 0) ok = mbar_wait(smem_u32(&bar_sdp[g & 1]), (g >> 1) & 1, wc, 230);
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       tc_fence_after();
@@ -604,23 +739,28 @@ __global__ void __launch_bounds__(320, 1)
       tmem_st16(tmem + lane_off + C::TM_DP + bo, pk);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(smem_u32(&bar_ds[j & 1]));
-    }
-    if (ok) {
-      if (lane == 0) ok = mbar_wait(smem_u32(&bar_done), 0, wc, 232);
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-    }
-    if (ok) {
-      tc_fence_after();
-      __nv_bfloat16* dqrow = static_cast<__nv_bfloat16*>(a.dq) +
-                             ((static_cast<size_t>(w.b) * d.N + t) * d.H + w.h) * D + half * (D / 2);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bar_ds[g & 1]));
+      if (cur.it == cur.iters - 1) {
+        // ---------------------------------------------------- epilogue of this item
+        if (lane == 0) ok = mbar_wait(smem_u32(&bar_acc_full), cur.ic.n & 1, wc, 232);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        tc_fence_after();
+        __nv_bfloat16* dqrow = static_cast<__nv_bfloat16*>(a.dq) +
+                               ((static_cast<size_t>(w.b) * d.N + tq0 + row) * d.H + w.h) * D + half * (D / 2);
 #pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tmem + lane_off + C::TM_DQ + half * (D / 2) + c * 32, r);
-        tmem_wait_ld();
-        store_row32(dqrow + c * 32, r, a.scale);
+        for (int c = 0; c < D / 64; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tmem + lane_off + C::TM_DQ + half * (D / 2) + c * 32, r);
+          tmem_wait_ld();
+          store_row32(dqrow + c * 32, r, a.scale);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bar_acc_free));
       }
+      cur.next(d, ps);
     }
   }
 
@@ -656,13 +796,13 @@ cudaError_t launch_bwd(const BwdMaps& m, const BwdPreArgs& pre, const BwdArgs& a
   cudaError_t e = cudaGetLastError();
   prof_after(stream);
   if (e != cudaSuccess) return e;
-  const int grid_kv = a.d.B * a.d.Hkv * a.d.n_groups * a.d.tiles;
+  const int grid_kv = a.kv_sched.pairs < num_sms ? a.kv_sched.pairs : num_sms;
   prof_before(stream, kKernelBwdDkDv);
   s2_bwd_dkdv_kernel<D><<<grid_kv, K3::THREADS, K3::SMEM_BYTES, stream>>>(m.q64, m.k128, m.v128, m.g64, a);
   e = cudaGetLastError();
   prof_after(stream);
   if (e != cudaSuccess) return e;
-  const int grid_q = a.d.B * a.d.H * a.d.n_groups * a.d.tiles;
+  const int grid_q = a.q_sched.pairs < num_sms ? a.q_sched.pairs : num_sms;
   prof_before(stream, kKernelBwdDq);
   s2_bwd_dq_kernel<D><<<grid_q, K4::THREADS, K4::SMEM_BYTES, stream>>>(m.q128, m.k64, m.v64, m.g128, a);
   e = cudaGetLastError();

@@ -72,6 +72,93 @@ __host__ __device__ __forceinline__ TileWork decode_kv_tile(const Dims& d, int x
   return w;
 }
 
+// Persistent schedule.  A "unit" is one rolled group of one (batch, head);
+// its T tiles are the work items.  Work grows (forward, dQ) or shrinks (dK/dV)
+// linearly with the tile index, so tile t is paired with tile T-1-t: every
+// pair carries the same work.  Pairs are dealt round-robin to the CTAs (one
+// per SM), consecutive pairs belong to the same unit, so the CTAs running at
+// one time share their K/V (or Q/dO) in L2.
+struct PairSched {
+  int units, T, ppu, pairs;  // ppu = pairs per unit
+};
+
+__host__ __device__ __forceinline__ PairSched make_pair_sched(int units, int T) {
+  PairSched ps;
+  ps.units = units;
+  ps.T = T;
+  ps.ppu = (T + 1) / 2;
+  ps.pairs = units * ps.ppu;
+  return ps;
+}
+
+// Item `e` (0 or 1) of pair p: its unit and tile; false if it does not exist
+// (the middle tile of an odd T has no partner).
+__host__ __device__ __forceinline__ bool pair_item(const PairSched& ps, int p, int e, int& unit,
+                                                   int& tile) {
+  if (p >= ps.pairs) return false;
+  unit = p / ps.ppu;
+  const int pj = p - unit * ps.ppu;
+  tile = (e == 0) ? pj : ps.T - 1 - pj;
+  return !(e == 1 && tile == pj);
+}
+
+// Walks the items of one CTA in order: pairs blockIdx.x, +gridDim.x, ...
+struct ItemCursor {
+  int p, e, unit, tile, n;  // n = items visited before this one
+  bool valid;
+  __device__ __forceinline__ void first(const PairSched& ps) {
+    p = blockIdx.x;
+    e = 0;
+    n = 0;
+    valid = pair_item(ps, p, e, unit, tile);
+  }
+  __device__ __forceinline__ void next(const PairSched& ps) {
+    ++n;
+    for (;;) {
+      if (e == 0) {
+        e = 1;
+      } else {
+        e = 0;
+        p += gridDim.x;
+      }
+      if (p >= ps.pairs) {
+        valid = false;
+        return;
+      }
+      if (pair_item(ps, p, e, unit, tile)) {
+        valid = true;
+        return;
+      }
+    }
+  }
+};
+
+// kv-tile work item of the dK/dV kernel from (unit, tile): unit = (b*Hkv + kvh)*ng + g.
+__host__ __device__ __forceinline__ TileWork kv_item(const Dims& d, int unit, int tile) {
+  TileWork w;
+  w.tile = tile;
+  w.g = unit % d.n_groups;
+  const int x = unit / d.n_groups;
+  w.kvh = x % d.Hkv;
+  w.b = x / d.Hkv;
+  w.h = w.kvh * d.rep;
+  return w;
+}
+
+// query-tile work item of the forward / dQ kernels: unit = ((b*Hkv + kvh)*ng + g)*rep + hr.
+__host__ __device__ __forceinline__ TileWork q_item(const Dims& d, int unit, int tile) {
+  TileWork w;
+  w.tile = tile;
+  const int hr = unit % d.rep;
+  int x = unit / d.rep;
+  w.g = x % d.n_groups;
+  x /= d.n_groups;
+  w.kvh = x % d.Hkv;
+  w.b = x / d.Hkv;
+  w.h = w.kvh * d.rep + hr;
+  return w;
+}
+
 struct FwdArgs {
   Dims d;
   float scale_log2;        // (1/sqrt(D)) * log2(e)
@@ -93,6 +180,8 @@ struct BwdPreArgs {
 
 struct BwdArgs {
   Dims d;
+  PairSched kv_sched;      // dK/dV work items (units: batch x kv-head x group)
+  PairSched q_sched;       // dQ work items (units: batch x head x group)
   float scale;             // 1/sqrt(D)
   float scale_log2;        // scale * log2(e)
   const float* ndelta;     // fp32 [B, H, N]: -Delta

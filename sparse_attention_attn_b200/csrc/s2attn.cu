@@ -320,6 +320,8 @@ int s2attn_bwd(const void* q, const void* k, const void* v, const void* o, const
   pre.status = status;
   BwdArgs a;
   a.d = d;
+  a.kv_sched = make_pair_sched(B * Hkv * d.n_groups, d.tiles);
+  a.q_sched = make_pair_sched(B * H * d.n_groups, d.tiles);
   a.scale = static_cast<float>(1.0 / __builtin_sqrt(static_cast<double>(D)));
   a.scale_log2 = static_cast<float>(1.4426950408889634 / __builtin_sqrt(static_cast<double>(D)));
   a.ndelta = ndelta;
