@@ -381,11 +381,14 @@ def main():
     ap.add_argument("--workload", default=I.LLAMA2_7B_8K.name,
                     choices=[s.name for s in I.WORKLOADS])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    ap.add_argument("--ref-step-seconds", type=float, default=5.0)
+    ap.add_argument("--ref-step-seconds", type=float, default=None,
+                    help="oracle seconds per reference step (default: ~2 minutes in total)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--dense-ratio", action="store_true", help="also time G=N on the same inputs")
     args = ap.parse_args()
     shape = {s.name: s for s in I.WORKLOADS}[args.workload]
+    if args.ref_step_seconds is None:
+        args.ref_step_seconds = min(5.0, 120.0 / max(args.steps, 1))
     world, rank, local = dist_setup()
     try:
         if args.impl == "reference":

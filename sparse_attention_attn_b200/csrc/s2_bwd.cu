@@ -125,6 +125,7 @@ __device__ __forceinline__ uint32_t split_acol64(int kk) { return kk * 8 + (kk >
 template <int D>
 struct DkvCfg {
   static constexpr int STAGES = 3;
+  // warps: 0 producer, 1 UMMA issuer A, 2..9 elementwise + epilogue, 10 UMMA issuer B
   static constexpr int KV_ATOM = kTile * 128;  // one 64-column slab of a 128-row tile
   static constexpr int Q_ATOM = kSub * 128;    // one 64-column slab of a 64-row tile
   static constexpr int KV_BYTES = kTile * D * 2;
@@ -135,7 +136,7 @@ struct DkvCfg {
   static constexpr int OFF_ROW = OFF_DO + STAGES * Q_BYTES;  // per stage: -lse2[64], -delta[64]
   static constexpr int SMEM_BYTES = OFF_ROW + STAGES * 512 + 1024;
   static constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DV = 256, TM_DK = 256 + D;
-  static constexpr int THREADS = 320;
+  static constexpr int THREADS = 352;
 };
 
 // Sub-tile cursor of the dK/dV kernel: item (kv tile) plus sub-tile index.
@@ -162,7 +163,7 @@ struct DkvCursor {
 };
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(352, 1)
     s2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmG,
                        const BwdArgs a) {
@@ -171,8 +172,10 @@ __global__ void __launch_bounds__(320, 1)
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  __shared__ __align__(8) uint64_t bar_kv[2], bar_kv_empty[2], bar_full[ST], bar_empty[ST], bar_sdp[2],
-      bar_pds[2], bar_acc_full, bar_acc_free, bar_drain;
+  // bar_s / bar_dp: S^T / dP^T of a sub-tile landed (issuers A / B);
+  // empty, kv_empty, acc_full complete once both issuers committed.
+  __shared__ __align__(8) uint64_t bar_kv[2], bar_kv_empty[2], bar_full[ST], bar_empty[ST], bar_s[2],
+      bar_dp[2], bar_pds[2], bar_acc_full, bar_acc_free, bar_drain[2];
   __shared__ uint32_t tmem_slot;
   __shared__ uint32_t abort_flag;
 
@@ -192,17 +195,18 @@ __global__ void __launch_bounds__(320, 1)
     abort_flag = 0;
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&bar_kv[i]), 1);
-      mbar_init(smem_u32(&bar_kv_empty[i]), 1);
-      mbar_init(smem_u32(&bar_sdp[i]), 1);
+      mbar_init(smem_u32(&bar_kv_empty[i]), 2);
+      mbar_init(smem_u32(&bar_s[i]), 1);
+      mbar_init(smem_u32(&bar_dp[i]), 1);
       mbar_init(smem_u32(&bar_pds[i]), 8);  // one elected arrival per elementwise warp
+      mbar_init(smem_u32(&bar_drain[i]), 1);
     }
     for (int s = 0; s < ST; ++s) {
       mbar_init(smem_u32(&bar_full[s]), 1);
-      mbar_init(smem_u32(&bar_empty[s]), 1);
+      mbar_init(smem_u32(&bar_empty[s]), 2);
     }
-    mbar_init(smem_u32(&bar_acc_full), 1);
+    mbar_init(smem_u32(&bar_acc_full), 2);
     mbar_init(smem_u32(&bar_acc_free), 8);
-    mbar_init(smem_u32(&bar_drain), 1);
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -274,37 +278,36 @@ __global__ void __launch_bounds__(320, 1)
         drain_wait(smem_u32(&bar_kv[kb]), ((kv_issued - 1 - kb) >> 1) & 1);
       for (int s = 0; s < ST && s < gi; ++s) drain_wait(smem_u32(&bar_full[s]), ((gi - 1 - s) / ST) & 1);
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ UMMA issuer
-    // (whole warp converged; one elected lane issues each batch)
-    const uint32_t idS = make_idesc_bf16(128, kSub, 0, 0);  // S^T = K Q^T, dP^T = V dO^T
-    const uint32_t idG = make_idesc_bf16(128, D, 0, 1);     // dV += P^T dO, dK += dS^T Q
-    const uint64_t dK0 = make_sdesc_sw128(sK(0), 16, 1024);         // K-major (A)
-    const uint64_t dV0 = make_sdesc_sw128(sV(0), 16, 1024);
-    const uint64_t dQk = make_sdesc_sw128(sQ(0), 16, 1024);         // K-major (B of S^T)
-    const uint64_t dGk = make_sdesc_sw128(sG(0), 16, 1024);
-    const uint64_t dQm = make_sdesc_sw128(sQ(0), C::Q_ATOM, 1024);  // MN-major (B of dK)
-    const uint64_t dGm = make_sdesc_sw128(sG(0), C::Q_ATOM, 1024);  // MN-major (B of dV)
-    // S^T and dP^T of global sub-tile g (stage g % ST, K/V buffer kb)
-    auto issue_sdp = [&](int g, int kb) {
+  } else if (warp == 1 || warp == 10) {
+    // ------------------------------------------------------------ UMMA issuers
+    // Two converged warps on different SM sub-partitions share the UMMA
+    // issue: A (warp 1) S^T = K Q^T and dV += P^T dO, B (warp 10) dP^T = V dO^T
+    // and dK += dS^T Q.  Each stream is in order on its own; they meet only at
+    // the barriers above.  (One issuing warp could not keep the tensor pipe
+    // fed while eight elementwise warps share its sub-partitions.)
+    const bool A = (warp == 1);
+    const uint32_t idS = make_idesc_bf16(128, kSub, 0, 0);  // S^T, dP^T
+    const uint32_t idG = make_idesc_bf16(128, D, 0, 1);     // dV, dK
+    // A: operand K / Q / dO, B: operand V / dO / Q
+    const uint64_t dX0 = make_sdesc_sw128(A ? sK(0) : sV(0), 16, 1024);          // K-major (A operand)
+    const uint64_t dYk = make_sdesc_sw128(A ? sQ(0) : sG(0), 16, 1024);          // K-major (B of S^T / dP^T)
+    const uint64_t dZm = make_sdesc_sw128(A ? sG(0) : sQ(0), C::Q_ATOM, 1024);   // MN-major (B of dV / dK)
+    const uint32_t tm_sp = tmem + (A ? C::TM_S : C::TM_DP);
+    const uint32_t tm_acc = tmem + (A ? C::TM_DV : C::TM_DK);
+    const uint32_t bar_ready = smem_u32(A ? &bar_s[0] : &bar_dp[0]);
+    auto issue_sp = [&](int g, int kb) {
       const int s = g % ST;
       const uint32_t bo = (g & 1) * kSub;
-      const uint64_t dk = sdesc_advance(dK0, kb * 2 * C::KV_BYTES), dv = sdesc_advance(dV0, kb * 2 * C::KV_BYTES);
-      const uint64_t dq = sdesc_advance(dQk, s * C::Q_BYTES), dg = sdesc_advance(dGk, s * C::Q_BYTES);
+      const uint64_t dx = sdesc_advance(dX0, kb * 2 * C::KV_BYTES);
+      const uint64_t dy = sdesc_advance(dYk, s * C::Q_BYTES);
       if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ko = (kk >> 2) * C::KV_ATOM + (kk & 3) * 32;
           const uint32_t qo = (kk >> 2) * C::Q_ATOM + (kk & 3) * 32;
-          umma_ss(tmem + C::TM_S + bo, sdesc_advance(dk, ko), sdesc_advance(dq, qo), idS, kk > 0);
+          umma_ss(tm_sp + bo, sdesc_advance(dx, ko), sdesc_advance(dy, qo), idS, kk > 0);
         }
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t ko = (kk >> 2) * C::KV_ATOM + (kk & 3) * 32;
-          const uint32_t qo = (kk >> 2) * C::Q_ATOM + (kk & 3) * 32;
-          umma_ss(tmem + C::TM_DP + bo, sdesc_advance(dv, ko), sdesc_advance(dg, qo), idS, kk > 0);
-        }
-        umma_commit(smem_u32(&bar_sdp[g & 1]));
+        umma_commit(bar_ready + (g & 1) * 8);
       }
       __syncwarp();
     };
@@ -322,12 +325,12 @@ __global__ void __launch_bounds__(320, 1)
     bool ok = true;
     if (cur.ic.valid) {
       ok = wait_inputs(cur, 0);
-      if (ok) issue_sdp(0, cur.ic.n & 1);
+      if (ok) issue_sp(0, cur.ic.n & 1);
     }
     for (int g = 0; ok && cur.ic.valid; ++g) {
-      if (nxt.ic.valid) {  // S^T/dP^T of the next sub-tile (possibly the next item's first)
+      if (nxt.ic.valid) {  // the next sub-tile (possibly the next item's first)
         if (!wait_inputs(nxt, g + 1)) break;
-        issue_sdp(g + 1, nxt.ic.n & 1);  // its TMEM buffer's last readers were issued before: in order
+        issue_sp(g + 1, nxt.ic.n & 1);  // its TMEM buffer's last reader was issued before: in order
       }
       if (!warp_wait(smem_u32(&bar_pds[g & 1]), (g >> 1) & 1, wc, 123)) break;
       if (cur.it == 0 && cur.ic.n > 0 &&
@@ -336,17 +339,13 @@ __global__ void __launch_bounds__(320, 1)
       tc_fence_after();
       const int s = g % ST;
       const uint32_t bo = (g & 1) * kSub;
-      const uint64_t dg = sdesc_advance(dGm, s * C::Q_BYTES), dq = sdesc_advance(dQm, s * C::Q_BYTES);
+      const uint64_t dz = sdesc_advance(dZm, s * C::Q_BYTES);
       const bool last = (cur.it == cur.iters - 1);
       if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < kSub / 16; ++kk)
-          umma_ts(tmem + C::TM_DV, tmem + C::TM_S + bo + split_acol64(kk), sdesc_advance(dg, kk * 2048),
-                  idG, (cur.it > 0 || kk > 0));
-#pragma unroll
-        for (int kk = 0; kk < kSub / 16; ++kk)
-          umma_ts(tmem + C::TM_DK, tmem + C::TM_DP + bo + split_acol64(kk), sdesc_advance(dq, kk * 2048),
-                  idG, (cur.it > 0 || kk > 0));
+          umma_ts(tm_acc, tm_sp + bo + split_acol64(kk), sdesc_advance(dz, kk * 2048), idG,
+                  (cur.it > 0 || kk > 0));
         umma_commit(smem_u32(&bar_empty[s]));
         if (last) {
           umma_commit(smem_u32(&bar_acc_full));
@@ -358,8 +357,8 @@ __global__ void __launch_bounds__(320, 1)
       nxt.next(d, ps);
     }
     if (elect_one()) {
-      umma_commit(smem_u32(&bar_drain));
-      drain_wait(smem_u32(&bar_drain), 0);
+      umma_commit(smem_u32(&bar_drain[A ? 0 : 1]));
+      drain_wait(smem_u32(&bar_drain[A ? 0 : 1]), 0);
     }
     __syncwarp();
   } else {
@@ -379,7 +378,8 @@ __global__ void __launch_bounds__(320, 1)
       const uint32_t bo = (g & 1) * kSub + half * 32;
       if (lane == 0)
         ok = mbar_wait(smem_u32(&bar_full[s]), (g / ST) & 1, wc, 130) &&
-             mbar_wait(smem_u32(&bar_sdp[g & 1]), (g >> 1) & 1, wc, 131);
+             mbar_wait(smem_u32(&bar_s[g & 1]), (g >> 1) & 1, wc, 131) &&
+             mbar_wait(smem_u32(&bar_dp[g & 1]), (g >> 1) & 1, wc, 133);
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       tc_fence_after();

@@ -1,0 +1,108 @@
+"""Host-only checks of the C ABI (no GPU needed, nothing is launched).
+
+* libs2attn.so loads and exports every function include/s2attn.h declares;
+* status codes and their names;
+* argument validation: every invalid argument returns its status code before
+  any CUDA call is made (fake, never-dereferenced pointers are passed);
+* workspace sizing.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from sparse_attention_attn_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "s2attn.h")
+
+P = 0x10000  # a 16-byte aligned fake device address (never dereferenced)
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"S2ATTN_API\s+[\w\s\*]+?\b(s2attn_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_documented_entry_points():
+    names = declared_functions()
+    for required in ("s2attn_fwd", "s2attn_bwd", "s2attn_bwd_workspace_bytes", "s2attn_device_status",
+                     "s2attn_status_string", "s2attn_bwd_noalloc"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = _lib.load()
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert name in _lib.SIGNATURES, f"binding lacks {name}"
+
+
+def test_status_strings():
+    for code, name in ((0, "S2ATTN_OK"), (1, "S2ATTN_ERR_INVALID_ARG"), (2, "S2ATTN_ERR_UNSUPPORTED"),
+                       (3, "S2ATTN_ERR_MISALIGNED"), (4, "S2ATTN_ERR_CUDA"), (5, "S2ATTN_ERR_DEVICE_TIMEOUT"),
+                       (6, "S2ATTN_ERR_WORKSPACE")):
+        assert _lib.status_string(code) == name
+    assert _lib.status_string(99) == "S2ATTN_UNKNOWN_STATUS"
+
+
+def fwd(q=P, k=P, v=P, o=P, lse=P, B=1, H=4, Hkv=4, N=1024, D=64, G=256):
+    return _lib.s2attn_fwd(q, k, v, o, lse, B, H, Hkv, N, D, G, None)
+
+
+def bwd(ptr=P, B=1, H=4, Hkv=4, N=1024, D=64, G=256, ws=P, wsb=1 << 30):
+    return _lib.s2attn_bwd(ptr, ptr, ptr, ptr, ptr, ptr, ptr, ptr, ptr, B, H, Hkv, N, D, G, ws, wsb, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), _lib.S2ATTN_ERR_INVALID_ARG),
+    (dict(lse=None), _lib.S2ATTN_ERR_INVALID_ARG),
+    (dict(B=0), _lib.S2ATTN_ERR_INVALID_ARG),          # empty batch is rejected, not a no-op
+    (dict(N=0), _lib.S2ATTN_ERR_INVALID_ARG),
+    (dict(H=-4), _lib.S2ATTN_ERR_INVALID_ARG),
+    (dict(H=4, Hkv=3), _lib.S2ATTN_ERR_INVALID_ARG),   # H % Hkv
+    (dict(N=1024, G=384), _lib.S2ATTN_ERR_INVALID_ARG),  # N % G
+    (dict(N=1024, G=2048), _lib.S2ATTN_ERR_INVALID_ARG),  # G > N
+    (dict(D=96), _lib.S2ATTN_ERR_UNSUPPORTED),
+    (dict(D=256), _lib.S2ATTN_ERR_UNSUPPORTED),
+    (dict(N=1000, G=1000), _lib.S2ATTN_ERR_UNSUPPORTED),  # ragged length (not a tile multiple)
+    (dict(N=1536, G=384), _lib.S2ATTN_ERR_UNSUPPORTED),  # shift G/2 = 192 is not a whole tile
+    (dict(H=6, Hkv=3, N=1024, G=256), _lib.S2ATTN_ERR_UNSUPPORTED),  # kv-head would mix shifts
+    (dict(q=P + 8), _lib.S2ATTN_ERR_MISALIGNED),
+    (dict(o=P + 4), _lib.S2ATTN_ERR_MISALIGNED),
+])
+def test_forward_argument_validation(kw, status):
+    assert fwd(**kw) == status
+    assert _lib.s2attn_last_launch_count() == 0
+
+
+def test_backward_argument_validation():
+    assert bwd(ptr=None) == _lib.S2ATTN_ERR_INVALID_ARG
+    assert bwd(D=80) == _lib.S2ATTN_ERR_UNSUPPORTED
+    assert bwd(ptr=P + 2) == _lib.S2ATTN_ERR_MISALIGNED
+    need = _lib.s2attn_bwd_workspace_bytes(1, 4, 4, 1024, 64, 256)
+    assert bwd(ws=None) == _lib.S2ATTN_ERR_WORKSPACE
+    assert bwd(wsb=need - 1) == _lib.S2ATTN_ERR_WORKSPACE
+    assert bwd(ws=P + 16) == _lib.S2ATTN_ERR_WORKSPACE  # workspace must be 256-byte aligned
+    assert _lib.s2attn_last_launch_count() == 0
+
+
+def test_workspace_bytes():
+    # status block + two fp32 [B, H, N] row-statistics arrays, each rounded to 256 bytes
+    assert _lib.s2attn_bwd_workspace_bytes(1, 32, 32, 8192, 128, 2048) == 256 + 2 * 32 * 8192 * 4
+    assert _lib.s2attn_bwd_workspace_bytes(1, 1, 1, 128, 64, 128) == 256 + 2 * 512
+    assert _lib.s2attn_bwd_workspace_bytes(1, 4, 3, 1024, 64, 256) == 0  # invalid shape
+
+
+def test_noalloc_rejects_oversize_before_launch():
+    # 64 heads x 131072 rows need ~64 MiB of scratch: rejected without touching the device
+    assert _lib.s2attn_bwd_noalloc(P, P, P, P, P, P, P, P, P, 1, 64, 64, 131072, 128, 131072, None) == \
+        _lib.S2ATTN_ERR_WORKSPACE
+    assert _lib.s2attn_bwd_noalloc(P, P, P, P, P, P, P, P, P, 1, 4, 3, 1024, 64, 256, None) == \
+        _lib.S2ATTN_ERR_INVALID_ARG  # invalid shape: reported by the backward's own validation
+
+
+def test_profile_api_host_side():
+    assert _lib.s2attn_profile_start(0) == _lib.S2ATTN_ERR_INVALID_ARG
+    assert _lib.s2attn_profile_stop(None, None, 0) == 0  # not started: nothing recorded
