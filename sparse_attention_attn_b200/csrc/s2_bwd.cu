@@ -383,8 +383,14 @@ __global__ void __launch_bounds__(352, 1)
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       tc_fence_after();
-      const float4* l4 = reinterpret_cast<const float4*>(smem + C::OFF_ROW + s * 512) + half * 8;
-      const float4* d4 = l4 + 16;
+      // row statistics of the 64 query rows: -lse*log2e at +0, -Delta at +256 bytes
+      const uint32_t l4 = sRow(s) + half * 128, d4 = l4 + 256;
+      float4 lv[8], dv4[8];
+#pragma unroll
+      for (int c4 = 0; c4 < 8; ++c4) {
+        lv[c4] = lds_f4(l4 + c4 * 16);
+        dv4[c4] = lds_f4(d4 + c4 * 16);
+      }
       uint32_t sr[32], dr[32];
       tmem_ld32(tmem + lane_off + C::TM_S + bo, sr);
       tmem_ld32(tmem + lane_off + C::TM_DP + bo, dr);
@@ -392,7 +398,7 @@ __global__ void __launch_bounds__(352, 1)
       float p[32];
 #pragma unroll
       for (int c4 = 0; c4 < 8; ++c4) {  // P^T = 2^(S^T * scale * log2 e - lse * log2 e)
-        const float4 l = l4[c4];
+        const float4 l = lv[c4];
         const uint64_t x01 = f2_fma(f2_pack(__uint_as_float(sr[4 * c4]), __uint_as_float(sr[4 * c4 + 1])),
                                     sl2x2, f2_pack(l.x, l.y));
         const uint64_t x23 = f2_fma(f2_pack(__uint_as_float(sr[4 * c4 + 2]), __uint_as_float(sr[4 * c4 + 3])),
@@ -413,7 +419,7 @@ __global__ void __launch_bounds__(352, 1)
       tmem_st16(tmem + lane_off + C::TM_S + bo, pk);
 #pragma unroll
       for (int c4 = 0; c4 < 8; ++c4) {  // dS^T = P^T * (dP^T - Delta)
-        const float4 dl = d4[c4];
+        const float4 dl = dv4[c4];
         const uint64_t d01 = f2_add(f2_pack(__uint_as_float(dr[4 * c4]), __uint_as_float(dr[4 * c4 + 1])),
                                     f2_pack(dl.x, dl.y));
         const uint64_t d23 = f2_add(f2_pack(__uint_as_float(dr[4 * c4 + 2]), __uint_as_float(dr[4 * c4 + 3])),

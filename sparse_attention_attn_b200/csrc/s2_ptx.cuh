@@ -352,6 +352,17 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
 // bf16x2 (round to nearest even) of a packed fp32 pair
 __device__ __forceinline__ uint32_t f2_to_bf16x2(uint64_t v) { return pack_bf16x2(f2_lo(v), f2_hi(v)); }
 
+// Explicit shared-memory vector load (a pointer into dynamic shared memory
+// that went through integer alignment arithmetic is generic to the compiler,
+// and generic loads take the long-latency path).
+__device__ __forceinline__ float4 lds_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr));
+  return v;
+}
+
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
                                              uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
