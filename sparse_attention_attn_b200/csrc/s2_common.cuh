@@ -159,8 +159,103 @@ __host__ __device__ __forceinline__ TileWork q_item(const Dims& d, int unit, int
   return w;
 }
 
+// Forward schedule.  A forward item is a pair of adjacent query tiles
+// (2i, 2i+1) of one unit (a rolled group of one (batch, head)): every K/V tile
+// the first tile needs, the second needs too, so one K/V load feeds 256 query
+// rows.  Item i carries 4i+3 tile products (2i+1 for the first tile, 2i+2 for
+// the second).  Two static orders, chosen per shape by the host:
+//  * snake: items sorted longest first, level-major (every unit's item Ti-1,
+//    then every unit's Ti-2, ...), dealt boustrophedon over the CTAs.  This
+//    approximates longest-processing-time-first list scheduling (within 3% of
+//    perfect balance on the shapes served); CTAs running at one time work on
+//    many units, so it is used when K and V together fit in L2;
+//  * pairs: item i paired with item Ti-1-i (equal work), pairs dealt
+//    round-robin, consecutive pairs in the same unit, so the CTAs running at
+//    one time share their K/V in L2 (long sequences).
+struct FwdSched {
+  int snake;  // 1: snake order, 0: pairs
+  int units;  // B * H * n_groups
+  int Ti;     // items per unit, ceil(tiles / 2)
+  int ppu;    // pairs per unit, ceil(Ti / 2)
+  int n;      // snake: units * Ti items; pairs: units * ppu pairs
+};
+
+// The items of one CTA, in order.
+struct FwdCursor {
+  int r, e;     // round, and position inside the round
+  int unit, i;  // current item
+  bool valid;
+  __device__ __forceinline__ void first(const FwdSched& s) {
+    r = 0;
+    e = 0;
+    settle(s);
+  }
+  __device__ __forceinline__ void next(const FwdSched& s) {
+    if (e == 0) {
+      e = 1;
+    } else {
+      e = 0;
+      ++r;
+    }
+    settle(s);
+  }
+  __device__ __forceinline__ void settle(const FwdSched& s) {
+    const int P = gridDim.x, c = blockIdx.x;
+    for (;;) {
+      if (s.snake) {
+        const int k = r * 2 * P + (e ? 2 * P - 1 - c : c);
+        valid = k < s.n;  // positions only grow from here on
+        if (valid) {
+          const int lvl = k / s.units;
+          unit = k - lvl * s.units;
+          i = s.Ti - 1 - lvl;
+        }
+        return;
+      }
+      const int p = r * P + c;
+      if (p >= s.n) {
+        valid = false;
+        return;
+      }
+      unit = p / s.ppu;
+      const int pj = p - unit * s.ppu;
+      i = e ? s.Ti - 1 - pj : pj;
+      if (!(e && i == pj)) {
+        valid = true;
+        return;
+      }
+      e = 0;  // the middle item of an odd Ti has no partner
+      ++r;
+    }
+  }
+};
+
+// One forward item: query tiles ta = 2i (always) and ta + 1 (if it exists),
+// key/value tiles 0 .. nkv-1 of the same rolled group.
+struct FwdItem {
+  int b, h, kvh, g, sh;
+  int ta;
+  bool has_b;
+  int nkv;
+};
+
+__device__ __forceinline__ FwdItem fwd_item(const Dims& d, int unit, int i) {
+  const TileWork w = q_item(d, unit, 2 * i);
+  FwdItem it;
+  it.b = w.b;
+  it.h = w.h;
+  it.kvh = w.kvh;
+  it.g = w.g;
+  it.sh = shift_of_head(d, w.h);
+  it.ta = 2 * i;
+  it.has_b = 2 * i + 1 < d.tiles;
+  it.nkv = it.has_b ? 2 * i + 2 : 2 * i + 1;
+  return it;
+}
+
 struct FwdArgs {
   Dims d;
+  FwdSched sched;
   float scale_log2;        // (1/sqrt(D)) * log2(e)
   void* o;                 // bf16 [B, N, H, D]
   float* lse;              // fp32 [B, H, N]

@@ -1,24 +1,29 @@
 // S2-Attn forward for sm_100a: tcgen05 UMMA with TMEM accumulators, TMA-fed
-// K/V ring, online softmax in fp32 with one query row per thread.
+// Q and K/V rings, online softmax in fp32 with one query row per thread.
 //
-// One CTA computes one 128-row query tile of one (batch, head).  Its key/value
-// tiles run from the start of the tile's rolled group up to the diagonal tile;
-// tiles above the diagonal and outside the group are never touched (LongQLoRA
-// community post, section 03: attention only inside each group; section 04:
-// causal next-token objective).
+// A persistent CTA (one per SM) walks a static list of items; an item is the
+// pair of adjacent query tiles (2i, 2i+1) of one rolled group of one
+// (batch, head).  The key/value tiles of an item run from the start of the
+// group up to the diagonal of its second tile; tiles above the diagonal and
+// outside the group are never touched (LongQLoRA community post, section 03:
+// attention only inside each group; section 04: causal next-token objective).
+// Every K/V tile feeds both query tiles, so one load serves 256 query rows.
 //
 // Warp roles (320 threads):
-//   warp 0      TMA producer: Q once, then K_j / V_j into a STAGES-deep ring.
-//   warp 1      TMEM owner and UMMA issuer: S_j = Q K_j^T (double-buffered in
-//               TMEM), O += P_j V_j with P_j read from TMEM.
-//   warps 2..9  softmax: two threads per query row (warps 2..5 the first 64
-//               key columns of a tile, warps 6..9 the last 64); S from TMEM,
-//               running max and sum, P (bf16) written back over S, O rescaled
-//               in TMEM only when the running max grows by more than 2^8,
-//               epilogue.
+//   warp 0      TMA producer: Q tiles into a 3-slot ring (the next item's
+//               tiles are fetched while the current item runs), K_j / V_j
+//               into a KV ring.
+//   warp 1      TMEM owner and UMMA issuer: S_A = Q_A K_j^T, S_B = Q_B K_j^T,
+//               O_A += P_A V_j, O_B += P_B V_j, in the order S_A(0) S_B(0)
+//               PV_A(0) S_A(1) PV_B(0) S_B(1) PV_A(1) ... so the tensor core
+//               works on one tile while the softmax of the other runs.
+//   warps 2..5  softmax warpgroup A (query tile 2i), warps 6..9 warpgroup B
+//               (tile 2i+1): one thread per query row; S from TMEM, running
+//               max and sum, P (bf16) written back over S, O rescaled in TMEM
+//               only when the running max grows by more than 2^8; epilogue.
 //
-// TMEM (512 columns): S buffers at [0,128) and [128,256) (P over their first
-// 64 columns), O at [256, 256 + D).
+// TMEM (512 columns): S_A [0,128), S_B [128,256) (P over their first 64
+// columns), O_A [256, 256+D), O_B [256+D, 256+2D).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -31,14 +36,12 @@ namespace s2 {
 template <int D>
 struct FwdCfg {
   static constexpr int BM = kTile, BN = kTile;
-  // K and V tiles share one ring of slots, filled in the order K0 V0 K1 V1 ...;
-  // a K slot is released as soon as its S UMMA completes.
-  static constexpr int SLOTS = (D == 64) ? 8 : 5;
-  static constexpr int ATOM_BYTES = kTile * 128;  // one 64-column slab of a 128-row tile
-  static constexpr int Q_BYTES = BM * D * 2;
-  static constexpr int KV_BYTES = BN * D * 2;
-  static constexpr int OFF_KV = Q_BYTES;
-  static constexpr int SMEM_BYTES = OFF_KV + SLOTS * KV_BYTES + 1024;  // + alignment slack
+  static constexpr int QSLOTS = 3;                  // Q ring: two tiles per item, one ahead
+  static constexpr int KVSLOTS = (D == 64) ? 8 : 4;  // K and V tiles share one ring: K0 V0 K1 V1 ...
+  static constexpr int ATOM_BYTES = kTile * 128;    // one 64-column slab of a 128-row tile
+  static constexpr int TILE_BYTES = kTile * D * 2;  // one 128-row tile of Q, K or V
+  static constexpr int OFF_KV = QSLOTS * TILE_BYTES;
+  static constexpr int SMEM_BYTES = OFF_KV + KVSLOTS * TILE_BYTES + 1024;  // + alignment slack
   static constexpr uint32_t TM_O = 256;
   static constexpr int THREADS = 320;
 };
@@ -78,14 +81,14 @@ __device__ __forceinline__ uint64_t exp2_fma2(uint64_t x) {
 // pairs in pk; returns the fp32 sum.  Arguments and sums use packed f32x2
 // arithmetic; one pair in four takes its exponentials on the FMA pipe
 // (exp2_fma2), the rest on the MUFU (ex2.approx), which balances the pipes.
-__device__ __forceinline__ float softmax_row64(const uint32_t (&sr)[2][32], float sl2, float m,
-                                               uint32_t (&pk)[32]) {
+__device__ __forceinline__ float softmax_row64(const uint32_t (&s0)[32], const uint32_t (&s1)[32], float sl2,
+                                               float m, uint32_t (&pk)[32]) {
   const uint64_t sc2 = f2_pack(sl2, sl2), nm2 = f2_pack(-m, -m);
   uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
   for (int c = 0; c < 32; ++c) {
-    const uint64_t x = f2_fma(f2_pack(__uint_as_float(sr[(2 * c) >> 5][(2 * c) & 31]),
-                                      __uint_as_float(sr[(2 * c + 1) >> 5][(2 * c + 1) & 31])),
+    const uint32_t* src = (c < 16) ? s0 : s1;
+    const uint64_t x = f2_fma(f2_pack(__uint_as_float(src[(2 * c) & 31]), __uint_as_float(src[(2 * c + 1) & 31])),
                               sc2, nm2);
     uint64_t p;
     if ((c & 3) == 0) {
@@ -105,43 +108,39 @@ __global__ void __launch_bounds__(320, 1)
     s2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdArgs a) {
   using C = FwdCfg<D>;
-  constexpr int NS = C::SLOTS;
+  constexpr int NQ = C::QSLOTS, NS = C::KVSLOTS;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  __shared__ __align__(8) uint64_t bar_q, bar_full[NS], bar_empty[NS], bar_s[2], bar_p[2], bar_x[2],
-      bar_l, bar_o, bar_drain;
-  __shared__ float red_max[2][2][kTile];  // [tile parity][half][row] partial row maxima
-  __shared__ float red_sum[2][kTile];     // [half][row] partial row sums
+  __shared__ __align__(8) uint64_t bar_qfull[NQ], bar_qempty[NQ], bar_full[NS], bar_empty[NS],
+      bar_s[2], bar_p[2], bar_o[2], bar_ofree[2], bar_drain;
   __shared__ uint32_t tmem_slot;
   __shared__ uint32_t abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const Dims& d = a.d;
-  const TileWork w = decode_q_tile(d, blockIdx.x);
-  const int sh = shift_of_head(d, w.h);
-  const int r0 = w.g * d.G + w.tile * kTile;  // rolled first row of this query tile
-  const int tq0 = original_row(d, r0, sh);     // its original row (the tile never wraps)
-  const int nkv = w.tile + 1;
   WaitCtx wc{&abort_flag, a.status, a.wait_limit_ns};
 
   const uint32_t sQ = smem_u32(smem);
-  auto slot_addr = [&](int s) { return sQ + C::OFF_KV + s * C::KV_BYTES; };
+  auto q_addr = [&](int s) { return sQ + s * C::TILE_BYTES; };
+  auto kv_addr = [&](int s) { return sQ + C::OFF_KV + s * C::TILE_BYTES; };
 
   if (threadIdx.x == 0) {
     abort_flag = 0;
-    mbar_init(smem_u32(&bar_q), 1);
+    for (int s = 0; s < NQ; ++s) {
+      mbar_init(smem_u32(&bar_qfull[s]), 1);
+      mbar_init(smem_u32(&bar_qempty[s]), 1);
+    }
     for (int s = 0; s < NS; ++s) {
       mbar_init(smem_u32(&bar_full[s]), 1);
       mbar_init(smem_u32(&bar_empty[s]), 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&bar_s[i]), 1);
-      mbar_init(smem_u32(&bar_p[i]), 8);  // one elected arrival per softmax warp
-      mbar_init(smem_u32(&bar_x[i]), 8);
+      mbar_init(smem_u32(&bar_p[i]), 4);      // one elected arrival per warp of the warpgroup
+      mbar_init(smem_u32(&bar_o[i]), 1);
+      mbar_init(smem_u32(&bar_ofree[i]), 4);
     }
-    mbar_init(smem_u32(&bar_l), 8);
-    mbar_init(smem_u32(&bar_o), 1);
     mbar_init(smem_u32(&bar_drain), 1);
     fence_barrier_init();
   }
@@ -161,78 +160,165 @@ __global__ void __launch_bounds__(320, 1)
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      mbar_arrive_expect_tx(smem_u32(&bar_q), C::Q_BYTES);
-      for (int c = 0; c < D / 64; ++c)
-        tma_load_4d(sQ + c * C::ATOM_BYTES, &tmQ, smem_u32(&bar_q), c * 64, w.h, tq0, w.b);
     }
     __syncwarp();
-    int issued = 0;
-    for (int L = 0; L < 2 * nkv; ++L) {  // load L: K_{L/2} (even) or V_{L/2} (odd)
-      const int s = L % NS, n = L / NS;
-      if (n > 0 && !warp_wait(smem_u32(&bar_empty[s]), (n - 1) & 1, wc, 10)) break;
-      const int tk0 = original_row(d, w.g * d.G + (L >> 1) * kTile, sh);
-      const CUtensorMap* map = (L & 1) ? &tmV : &tmK;
+    int qu = 0;  // Q-ring uses so far (two per item)
+    int L = 0;   // KV-ring loads so far
+    // Q use qu: query tile t of item it, or (absent second tile) a plain
+    // arrival that completes the slot's phase without data.
+    auto load_q = [&](const FwdItem& it, int t, bool present) -> bool {
+      const int s = qu % NQ, r = qu / NQ;
+      if (r > 0 && !warp_wait(smem_u32(&bar_qempty[s]), (r - 1) & 1, wc, 10)) return false;
+      const int row = original_row(d, it.g * d.G + t * kTile, it.sh);
       if (elect_one()) {
-        mbar_arrive_expect_tx(smem_u32(&bar_full[s]), C::KV_BYTES);
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_4d(slot_addr(s) + c * C::ATOM_BYTES, map, smem_u32(&bar_full[s]), c * 64, w.kvh,
-                      tk0, w.b);
+        if (present) {
+          mbar_arrive_expect_tx(smem_u32(&bar_qfull[s]), C::TILE_BYTES);
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_4d(q_addr(s) + c * C::ATOM_BYTES, &tmQ, smem_u32(&bar_qfull[s]), c * 64, it.h,
+                        row, it.b);
+        } else {
+          mbar_arrive(smem_u32(&bar_qfull[s]));
+        }
       }
       __syncwarp();
-      ++issued;
+      ++qu;
+      return true;
+    };
+    auto load_kv = [&](const FwdItem& it, int j, bool is_v) -> bool {
+      const int s = L % NS, r = L / NS;
+      if (r > 0 && !warp_wait(smem_u32(&bar_empty[s]), (r - 1) & 1, wc, 11)) return false;
+      const int row = original_row(d, it.g * d.G + j * kTile, it.sh);
+      if (elect_one()) {
+        mbar_arrive_expect_tx(smem_u32(&bar_full[s]), C::TILE_BYTES);
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_4d(kv_addr(s) + c * C::ATOM_BYTES, is_v ? &tmV : &tmK, smem_u32(&bar_full[s]),
+                      c * 64, it.kvh, row, it.b);
+      }
+      __syncwarp();
+      ++L;
+      return true;
+    };
+    FwdCursor cur;
+    cur.first(a.sched);
+    bool ok = true;
+    if (cur.valid) {
+      FwdItem it = fwd_item(d, cur.unit, cur.i);
+      ok = load_q(it, it.ta, true) && load_q(it, it.ta + 1, it.has_b);
+      while (ok && cur.valid) {
+        FwdCursor nx = cur;
+        nx.next(a.sched);
+        const FwdItem itn = fwd_item(d, nx.valid ? nx.unit : cur.unit, nx.valid ? nx.i : cur.i);
+        // the next item's first Q tile goes into the slot its predecessor's
+        // second tile freed: fetched once this item is under way
+        const int jq = min(2, it.nkv - 1);
+        for (int j = 0; ok && j < it.nkv; ++j) {
+          ok = load_kv(it, j, false) && load_kv(it, j, true);
+          if (ok && j == jq && nx.valid) ok = load_q(itn, itn.ta, true);
+        }
+        if (ok && nx.valid) ok = load_q(itn, itn.ta + 1, itn.has_b);
+        cur = nx;
+        it = itn;
+      }
     }
     if (*wc.abort && lane == 0) {
       // never leave copies in flight into shared memory: wait (bounded) for
-      // the last fill of every slot and for Q
-      drain_wait(smem_u32(&bar_q), 0);
-      for (int s = 0; s < NS && s < issued; ++s)
-        drain_wait(smem_u32(&bar_full[s]), ((issued - 1 - s) / NS) & 1);
+      // the last fill of every slot
+      for (int s = 0; s < NQ && s < qu; ++s) drain_wait(smem_u32(&bar_qfull[s]), ((qu - 1 - s) / NQ) & 1);
+      for (int s = 0; s < NS && s < L; ++s) drain_wait(smem_u32(&bar_full[s]), ((L - 1 - s) / NS) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ UMMA issuer
     // (whole warp converged; one elected lane issues each batch)
     const uint32_t idS = make_idesc_bf16(128, C::BN, 0, 0);  // Q K-major, K K-major
     const uint32_t idO = make_idesc_bf16(128, D, 0, 1);      // P from TMEM, V MN-major
-    // operand descriptors: built once, then advanced by constants
-    const uint64_t dQ0 = make_sdesc_sw128(sQ, 16, 1024);                      // K-major
-    const uint64_t dK0 = make_sdesc_sw128(slot_addr(0), 16, 1024);            // K-major
-    const uint64_t dV0 = make_sdesc_sw128(slot_addr(0), C::ATOM_BYTES, 1024);  // MN-major
-    // S_j = Q K_j^T into S buffer j&1; releases K_j's slot when done
-    auto issue_qk = [&](int j) -> bool {
-      const int L = 2 * j, s = L % NS;
-      if (!warp_wait(smem_u32(&bar_full[s]), (L / NS) & 1, wc, 22)) return false;
+    const uint64_t dQ0 = make_sdesc_sw128(q_addr(0), 16, 1024);              // K-major
+    const uint64_t dK0 = make_sdesc_sw128(kv_addr(0), 16, 1024);             // K-major
+    const uint64_t dV0 = make_sdesc_sw128(kv_addr(0), C::ATOM_BYTES, 1024);  // MN-major
+    auto commit = [&](uint64_t* bar) {
+      if (elect_one()) umma_commit(smem_u32(bar));
+      __syncwarp();
+    };
+    auto wait_full = [&](int Lx) { return warp_wait(smem_u32(&bar_full[Lx % NS]), (Lx / NS) & 1, wc, 20); };
+    // S_wg = Q(slot qs) K(load Lk)^T
+    auto issue_s = [&](int wg, int qs, int Lk) {
       tc_fence_after();
-      const uint64_t dk = sdesc_advance(dK0, s * C::KV_BYTES);
-      const uint32_t tS = tmem + (j & 1) * 128;
+      const uint64_t dq = sdesc_advance(dQ0, qs * C::TILE_BYTES);
+      const uint64_t dk = sdesc_advance(dK0, (Lk % NS) * C::TILE_BYTES);
       if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::ATOM_BYTES + (kk & 3) * 32;
-          umma_ss(tS, sdesc_advance(dQ0, off), sdesc_advance(dk, off), idS, kk > 0);
+          umma_ss(tmem + wg * 128, sdesc_advance(dq, off), sdesc_advance(dk, off), idS, kk > 0);
         }
-        umma_commit(smem_u32(&bar_s[j & 1]));
-        umma_commit(smem_u32(&bar_empty[s]));
+        umma_commit(smem_u32(&bar_s[wg]));
       }
       __syncwarp();
-      return true;
     };
-    bool ok = warp_wait(smem_u32(&bar_q), 0, wc, 20) && issue_qk(0);
-    for (int j = 0; ok && j < nkv; ++j) {
-      if (j + 1 < nkv && !issue_qk(j + 1)) break;
-      const int L = 2 * j + 1, s = L % NS;
-      if (!warp_wait(smem_u32(&bar_p[j & 1]), (j >> 1) & 1, wc, 23)) break;
-      if (!warp_wait(smem_u32(&bar_full[s]), (L / NS) & 1, wc, 24)) break;
+    // O_wg (+)= P_wg V(load Lv)
+    auto issue_pv = [&](int wg, int Lv, bool acc) {
       tc_fence_after();
-      const uint32_t tP = tmem + (j & 1) * 128;
-      const uint64_t dv = sdesc_advance(dV0, s * C::KV_BYTES);
+      const uint64_t dv = sdesc_advance(dV0, (Lv % NS) * C::TILE_BYTES);
       if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < C::BN / 16; ++kk)
-          umma_ts(tmem + C::TM_O, tP + kk * 8, sdesc_advance(dv, kk * 2048), idO, (j > 0 || kk > 0));
-        umma_commit(smem_u32(&bar_o));
-        umma_commit(smem_u32(&bar_empty[s]));
+          umma_ts(tmem + C::TM_O + wg * D, tmem + wg * 128 + kk * 8, sdesc_advance(dv, kk * 2048), idO,
+                  acc || kk > 0);
+        umma_commit(smem_u32(&bar_o[wg]));
       }
       __syncwarp();
+    };
+    int L = 0, n = 0, np[2] = {0, 0};
+    FwdCursor cur;
+    cur.first(a.sched);
+    bool ok = true;
+    while (ok && cur.valid) {
+      const FwdItem it = fwd_item(d, cur.unit, cur.i);
+      const int uA = 2 * n, uB = uA + 1, sA = uA % NQ, sB = uB % NQ;
+      const int lastA = it.ta, lastB = it.has_b ? it.ta + 1 : -1;
+      const int L0 = L;  // K_j is load L0 + 2j, V_j load L0 + 2j + 1
+      ok = warp_wait(smem_u32(&bar_qfull[sA]), (uA / NQ) & 1, wc, 21) && wait_full(L0) &&
+           warp_wait(smem_u32(&bar_qfull[sB]), (uB / NQ) & 1, wc, 21);
+      if (!ok) break;
+      issue_s(0, sA, L0);
+      if (lastA == 0) commit(&bar_qempty[sA]);
+      if (it.has_b) issue_s(1, sB, L0);
+      else commit(&bar_qempty[sB]);
+      commit(&bar_empty[L0 % NS]);
+      for (int j = 0; ok && j < it.nkv; ++j) {
+        const int Lv = L0 + 2 * j + 1, Lk1 = L0 + 2 * j + 2;
+        if (j <= lastA) {
+          ok = warp_wait(smem_u32(&bar_p[0]), np[0] & 1, wc, 22) &&
+               (j > 0 || n == 0 || warp_wait(smem_u32(&bar_ofree[0]), (n - 1) & 1, wc, 23)) && wait_full(Lv);
+          if (!ok) break;
+          ++np[0];
+          issue_pv(0, Lv, j > 0);
+          if (j > lastB) commit(&bar_empty[Lv % NS]);
+          if (j + 1 <= lastA) {
+            if (!wait_full(Lk1)) { ok = false; break; }
+            issue_s(0, sA, Lk1);
+            if (j + 1 == lastA) commit(&bar_qempty[sA]);
+            if (j + 1 > lastB) commit(&bar_empty[Lk1 % NS]);
+          }
+        }
+        if (j <= lastB) {
+          ok = warp_wait(smem_u32(&bar_p[1]), np[1] & 1, wc, 24) &&
+               (j > 0 || n == 0 || warp_wait(smem_u32(&bar_ofree[1]), (n - 1) & 1, wc, 25)) &&
+               (j <= lastA || wait_full(Lv));
+          if (!ok) break;
+          ++np[1];
+          issue_pv(1, Lv, j > 0);
+          commit(&bar_empty[Lv % NS]);
+          if (j + 1 <= lastB) {
+            if (j + 1 > lastA && !wait_full(Lk1)) { ok = false; break; }
+            issue_s(1, sB, Lk1);
+            if (j + 1 == lastB) commit(&bar_qempty[sB]);
+            commit(&bar_empty[Lk1 % NS]);
+          }
+        }
+      }
+      L = L0 + 2 * it.nkv;
+      ++n;
+      cur.next(a.sched);
     }
     // every issued UMMA completes before TMEM is released
     if (elect_one()) {
@@ -242,128 +328,120 @@ __global__ void __launch_bounds__(320, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax
-    // Two warpgroups share every query row: warps 2..5 take key columns
-    // [0,64) of each tile, warps 6..9 columns [64,128).  The two halves of a
-    // row exchange their partial maxima through shared memory each tile (and
-    // their partial sums once at the end); both then take identical decisions.
+    // warpgroup wg owns query tile ta + wg of every item; thread = query row
+    const int wg = (warp - 2) >> 2;
     const int quarter = warp & 3;  // TMEM lanes this warp may access
-    const int half = (warp - 2) >> 2;
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t tS = tmem + lane_off + wg * 128;
+    const uint32_t tO = tmem + lane_off + C::TM_O + wg * D;
     const float sl2 = a.scale_log2;
-    float m_run = 0.f, l_run = 0.f;
+    int ns = 0, no = 0;  // S and PV phases of this warpgroup so far
+    FwdCursor cur;
+    cur.first(a.sched);
     bool ok = true;
-    for (int j = 0; j < nkv; ++j) {
-      const uint32_t tS = tmem + lane_off + (j & 1) * 128;
-      if (lane == 0) ok = mbar_wait(smem_u32(&bar_s[j & 1]), (j >> 1) & 1, wc, 30);
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) break;
-      tc_fence_after();
-      uint32_t sr[2][32];
-      tmem_ld32(tS + half * 64, sr[0]);
-      tmem_ld32(tS + half * 64 + 32, sr[1]);
-      tmem_wait_ld();
-      if (j == nkv - 1) {  // diagonal tile: keys after the query are masked
+    while (ok && cur.valid) {
+      const FwdItem it = fwd_item(d, cur.unit, cur.i);
+      const int t = it.ta + wg;
+      if (wg == 0 || it.has_b) {
+        float m_run = 0.f, l_run = 0.f;
+        for (int j = 0; j <= t; ++j) {
+          if (lane == 0) ok = mbar_wait(smem_u32(&bar_s[wg]), ns & 1, wc, 30);
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          if (!ok) break;
+          ++ns;
+          tc_fence_after();
+          uint32_t sr[4][32];
 #pragma unroll
-        for (int c = 0; c < 64; ++c)
-          if (half * 64 + c > row) sr[c >> 5][c & 31] = __float_as_uint(neg_inf());
-      }
-      float m4[4] = {neg_inf(), neg_inf(), neg_inf(), neg_inf()};
+          for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr[c]);
+          tmem_wait_ld();
+          if (j == t) {  // diagonal tile: keys after the query are masked
 #pragma unroll
-      for (int c = 0; c < 64; ++c) m4[c & 3] = fmaxf(m4[c & 3], __uint_as_float(sr[c >> 5][c & 31]));
-      const float mh = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-      // exchange partial maxima with the other half of the row (double-buffered
-      // slot).  From the second tile on the exchange completes in the
-      // background: P is computed against the running max first and redone
-      // only if the row max grew by more than 2^8 (rare after the first tiles).
-      red_max[j & 1][half][row] = mh;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bar_x[j & 1]));
-      auto exchange = [&]() -> bool {
-        bool ok2 = true;
-        if (lane == 0) ok2 = mbar_wait(smem_u32(&bar_x[j & 1]), (j >> 1) & 1, wc, 33);
-        return __shfl_sync(0xffffffffu, ok2, 0);
-      };
-      if (j == 0) {
-        if (!exchange()) { ok = false; break; }
-        m_run = fmaxf(mh, red_max[0][half ^ 1][row]) * sl2;
-      }
-      uint32_t pk[32];
-      float rs = softmax_row64(sr, sl2, m_run, pk);
-      float alpha = 1.f;
-      bool resc = false;
-      if (j > 0) {
-        if (!exchange()) { ok = false; break; }
-        const float mx = fmaxf(mh, red_max[j & 1][half ^ 1][row]) * sl2;
-        if (mx > m_run + 8.f) {
-          alpha = ex2_approx(m_run - mx);
-          m_run = mx;
-          resc = true;
-          rs = softmax_row64(sr, sl2, m_run, pk);
+            for (int c = 0; c < 128; ++c)
+              if (c > row) sr[c >> 5][c & 31] = __float_as_uint(neg_inf());
+          }
+          float m4[4] = {neg_inf(), neg_inf(), neg_inf(), neg_inf()};
+#pragma unroll
+          for (int c = 0; c < 128; ++c) m4[c & 3] = fmaxf(m4[c & 3], __uint_as_float(sr[c >> 5][c & 31]));
+          const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl2;
+          float alpha = 1.f;
+          bool resc = false;
+          if (j == 0) {
+            m_run = mx;
+          } else if (mx > m_run + 8.f) {
+            alpha = ex2_approx(m_run - mx);
+            m_run = mx;
+            resc = true;
+          }
+          uint32_t pk[2][32];
+          const float rs = softmax_row64(sr[0], sr[1], sl2, m_run, pk[0]) + softmax_row64(sr[2], sr[3], sl2, m_run, pk[1]);
+          l_run = l_run * alpha + rs;
+          // P (bf16) over the first 64 columns of S; every S column of this
+          // thread's row was read above
+          tmem_st32(tS, pk[0]);
+          tmem_st32(tS + 32, pk[1]);
+          if (__any_sync(0xffffffffu, resc)) {
+            // rescale O (it holds P_{j-1} V_{j-1} once that UMMA has completed)
+            // before P_j V_j accumulates onto it
+            if (lane == 0) ok = mbar_wait(smem_u32(&bar_o[wg]), (no - 1) & 1, wc, 31);
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            tc_fence_after();
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t o[32];
+              tmem_ld32(tO + c * 32, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+              tmem_st32(tO + c * 32, o);
+            }
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&bar_p[wg]));
+          ++no;
         }
-      }
-      l_run = l_run * alpha + rs;
-      // P (bf16) over the first 64 columns of this S buffer; both halves read
-      // their S columns before the exchange above, so no write races a read
-      tmem_st32(tS + half * 32, pk);
-      if (__any_sync(0xffffffffu, resc)) {
-        // O holds P_{j-1} V_{j-1} only once that UMMA has completed
-        if (lane == 0) ok = mbar_wait(smem_u32(&bar_o), (j - 1) & 1, wc, 31);
-        ok = __shfl_sync(0xffffffffu, ok, 0);
+        // ---------------------------------------------------------- epilogue
+        if (ok) {
+          if (lane == 0) ok = mbar_wait(smem_u32(&bar_o[wg]), (no - 1) & 1, wc, 32);
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+        }
         if (!ok) break;
         tc_fence_after();
+        uint32_t o[D / 32][32];
 #pragma unroll
-        for (int c = 0; c < D / 64; ++c) {
-          uint32_t o[32];
-          const uint32_t to = tmem + lane_off + C::TM_O + half * (D / 2) + c * 32;
-          tmem_ld32(to, o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(to, o);
-        }
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bar_p[j & 1]));
-    }
-    // ------------------------------------------------------------ epilogue
-    if (ok) {
-      red_sum[half][row] = l_run;
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(smem_u32(&bar_l));
-        ok = mbar_wait(smem_u32(&bar_l), 0, wc, 34) && mbar_wait(smem_u32(&bar_o), (nkv - 1) & 1, wc, 32);
-      }
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-    }
-    if (ok) {
-      tc_fence_after();
-      const float l_tot = l_run + red_sum[half ^ 1][row];
-      const float inv_l = 1.f / l_tot;
-      const int t = tq0 + row;
-      __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.o) +
-                            ((static_cast<size_t>(w.b) * d.N + t) * d.H + w.h) * D + half * (D / 2);
-#pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
-        uint32_t o[32];
-        tmem_ld32(tmem + lane_off + C::TM_O + half * (D / 2) + c * 32, o);
+        for (int c = 0; c < D / 32; ++c) tmem_ld32(tO + c * 32, o[c]);
         tmem_wait_ld();
-        uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+        // O is in registers: the issuer may start the next item's P V
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bar_ofree[wg]));
+        const float inv_l = 1.f / l_run;
+        const int tq = original_row(d, it.g * d.G + t * kTile + row, it.sh);
+        __nv_bfloat16* orow =
+            static_cast<__nv_bfloat16*>(a.o) + ((static_cast<size_t>(it.b) * d.N + tq) * d.H + it.h) * D;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint4 v;
-          v.x = pack_bf16x2(__uint_as_float(o[8 * q + 0]) * inv_l, __uint_as_float(o[8 * q + 1]) * inv_l);
-          v.y = pack_bf16x2(__uint_as_float(o[8 * q + 2]) * inv_l, __uint_as_float(o[8 * q + 3]) * inv_l);
-          v.z = pack_bf16x2(__uint_as_float(o[8 * q + 4]) * inv_l, __uint_as_float(o[8 * q + 5]) * inv_l);
-          v.w = pack_bf16x2(__uint_as_float(o[8 * q + 6]) * inv_l, __uint_as_float(o[8 * q + 7]) * inv_l);
-          dst[q] = v;
+        for (int c = 0; c < D / 32; ++c) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint4 v;
+            v.x = pack_bf16x2(__uint_as_float(o[c][8 * q + 0]) * inv_l, __uint_as_float(o[c][8 * q + 1]) * inv_l);
+            v.y = pack_bf16x2(__uint_as_float(o[c][8 * q + 2]) * inv_l, __uint_as_float(o[c][8 * q + 3]) * inv_l);
+            v.z = pack_bf16x2(__uint_as_float(o[c][8 * q + 4]) * inv_l, __uint_as_float(o[c][8 * q + 5]) * inv_l);
+            v.w = pack_bf16x2(__uint_as_float(o[c][8 * q + 6]) * inv_l, __uint_as_float(o[c][8 * q + 7]) * inv_l);
+            dst[q] = v;
+          }
         }
+        a.lse[(static_cast<size_t>(it.b) * d.H + it.h) * d.N + tq] = (m_run + __log2f(l_run)) * 0.69314718055994530942f;
+      } else {
+        // no second tile in this item: keep the O-free phases in step
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bar_ofree[wg]));
       }
-      if (half == 0)
-        a.lse[(static_cast<size_t>(w.b) * d.H + w.h) * d.N + t] =
-            (m_run + __log2f(l_tot)) * 0.69314718055994530942f;
+      cur.next(a.sched);
     }
   }
 
@@ -377,12 +455,12 @@ __global__ void __launch_bounds__(320, 1)
 
 template <int D>
 cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const FwdArgs& a, cudaStream_t stream) {
+                       const FwdArgs& a, int num_sms, cudaStream_t stream) {
   using C = FwdCfg<D>;
   cudaError_t ea = cudaFuncSetAttribute(s2_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         C::SMEM_BYTES);
   if (ea != cudaSuccess) return ea;
-  const int grid = a.d.B * a.d.H * a.d.n_groups * a.d.tiles;
+  const int grid = a.sched.n < num_sms ? a.sched.n : num_sms;
   prof_before(stream, kKernelFwd);
   s2_fwd_kernel<D><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, a);
   cudaError_t e = cudaGetLastError();
@@ -413,8 +491,8 @@ cudaError_t launch_exp2_selftest(const float* x, float* y_poly, float* y_ref, in
 }
 
 template cudaError_t launch_fwd<64>(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
-                                    const FwdArgs&, cudaStream_t);
+                                    const FwdArgs&, int, cudaStream_t);
 template cudaError_t launch_fwd<128>(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
-                                     const FwdArgs&, cudaStream_t);
+                                     const FwdArgs&, int, cudaStream_t);
 
 }  // namespace s2

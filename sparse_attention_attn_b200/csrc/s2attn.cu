@@ -19,7 +19,7 @@
 namespace s2 {
 template <int D>
 cudaError_t launch_fwd(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const FwdArgs&,
-                       cudaStream_t);
+                       int, cudaStream_t);
 template <int D>
 cudaError_t launch_bwd(const BwdMaps&, const BwdPreArgs&, const BwdArgs&, int, cudaStream_t, int*);
 cudaError_t launch_exp2_selftest(const float* x, float* y_poly, float* y_ref, int n, cudaStream_t stream);
@@ -122,6 +122,21 @@ Dims make_dims(int B, int H, int Hkv, int N, int D, int G) {
   d.n_groups = N / G;
   d.tiles = G / kTile;
   return d;
+}
+
+// Forward work order (see FwdSched): the snake order balances best; it
+// spreads the units over all CTAs at once, so it is taken only while K and V
+// together stay within about twice the L2 (126 MB on B200) -- beyond that the
+// pairs order keeps each K/V tile's readers running together.
+FwdSched make_fwd_sched(const Dims& d) {
+  FwdSched s;
+  s.units = d.B * d.H * d.n_groups;
+  s.Ti = (d.tiles + 1) / 2;
+  s.ppu = (s.Ti + 1) / 2;
+  const double kv_bytes = 2.0 * d.B * d.N * d.Hkv * d.D * 2.0;
+  s.snake = kv_bytes <= 256.0 * 1024 * 1024 ? 1 : 0;
+  s.n = s.snake ? s.units * s.Ti : s.units * s.ppu;
+  return s;
 }
 
 // 4-D view {D, heads, N, B} of a bf16 [B, N, heads, D] tensor; box = one
@@ -269,6 +284,7 @@ int s2attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
     return S2ATTN_ERR_CUDA;
   FwdArgs a;
   a.d = make_dims(B, H, Hkv, N, D, G);
+  a.sched = make_fwd_sched(a.d);
   a.scale_log2 = static_cast<float>(1.4426950408889634 / __builtin_sqrt(static_cast<double>(D)));
   a.o = o;
   a.lse = lse;
@@ -277,7 +293,8 @@ int s2attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   a.status = static_cast<uint32_t*>(status);
   a.wait_limit_ns = wait_limit_ns();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = (D == 64) ? launch_fwd<64>(tq, tk, tv, a, s) : launch_fwd<128>(tq, tk, tv, a, s);
+  cudaError_t e = (D == 64) ? launch_fwd<64>(tq, tk, tv, a, info.sms, s)
+                             : launch_fwd<128>(tq, tk, tv, a, info.sms, s);
   if (e != cudaSuccess) return S2ATTN_ERR_CUDA;
   g_last_launches = 1;
   return S2ATTN_OK;

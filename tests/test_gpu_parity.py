@@ -44,6 +44,8 @@ SMALL = [
     (1, 512, 1, 1, 64, 256),      # H=1: every head shifted
     (1, 2048, 2, 2, 128, 2048),   # dense causal, 16 tiles
     (2, 1536, 4, 4, 64, 768),     # G/2 = 384: three-tile shift
+    (1, 640, 2, 2, 64, 640),      # dense, 5 tiles: the last forward item has one query tile
+    (1, 384, 3, 1, 128, 384),     # dense, 3 tiles, D=128, three query heads per kv-head
 ]
 
 
