@@ -258,6 +258,7 @@ struct FwdArgs {
   FwdSched sched;
   float scale_log2;        // (1/sqrt(D)) * log2(e)
   void* o;                 // bf16 [B, N, H, D]
+  int o_v8;                // o is 32-byte aligned: the epilogue writes whole 32-byte sectors
   float* lse;              // fp32 [B, H, N]
   uint32_t* status;        // device status words
   unsigned long long wait_limit_ns;

@@ -268,22 +268,53 @@ __global__ void __launch_bounds__(320, 1)
       __syncwarp();
     };
     int L = 0, n = 0, np[2] = {0, 0};
+    bool pre = false;  // this item's first S_A / S_B were issued at the end of the previous item
     FwdCursor cur;
     cur.first(a.sched);
     bool ok = true;
     while (ok && cur.valid) {
       const FwdItem it = fwd_item(d, cur.unit, cur.i);
+      FwdCursor nx = cur;
+      nx.next(a.sched);
+      const FwdItem itn = fwd_item(d, nx.valid ? nx.unit : cur.unit, nx.valid ? nx.i : cur.i);
       const int uA = 2 * n, uB = uA + 1, sA = uA % NQ, sB = uB % NQ;
+      const int sAn = (uA + 2) % NQ, sBn = (uB + 2) % NQ;  // the next item's Q slots
       const int lastA = it.ta, lastB = it.has_b ? it.ta + 1 : -1;
       const int L0 = L;  // K_j is load L0 + 2j, V_j load L0 + 2j + 1
-      ok = warp_wait(smem_u32(&bar_qfull[sA]), (uA / NQ) & 1, wc, 21) && wait_full(L0) &&
-           warp_wait(smem_u32(&bar_qfull[sB]), (uB / NQ) & 1, wc, 21);
-      if (!ok) break;
-      issue_s(0, sA, L0);
-      if (lastA == 0) commit(&bar_qempty[sA]);
-      if (it.has_b) issue_s(1, sB, L0);
-      else commit(&bar_qempty[sB]);
-      commit(&bar_empty[L0 % NS]);
+      const int L0n = L0 + 2 * it.nkv;
+      if (!pre) {
+        ok = warp_wait(smem_u32(&bar_qfull[sA]), (uA / NQ) & 1, wc, 21) && wait_full(L0) &&
+             warp_wait(smem_u32(&bar_qfull[sB]), (uB / NQ) & 1, wc, 21);
+        if (!ok) break;
+        issue_s(0, sA, L0);
+        if (lastA == 0) commit(&bar_qempty[sA]);
+        if (it.has_b) issue_s(1, sB, L0);
+        else commit(&bar_qempty[sB]);
+        commit(&bar_empty[L0 % NS]);
+      }
+      // The next item's first scores are computed as soon as this item's
+      // last P V of the same warpgroup has been issued (it reads P out of the
+      // S buffer before the new S overwrites it), so a warpgroup moves on to
+      // the next item without waiting for the other one to finish this item.
+      auto start_next_a = [&]() -> bool {
+        if (!nx.valid) return true;
+        if (!warp_wait(smem_u32(&bar_qfull[sAn]), ((uA + 2) / NQ) & 1, wc, 26) || !wait_full(L0n)) return false;
+        issue_s(0, sAn, L0n);
+        if (itn.ta == 0) commit(&bar_qempty[sAn]);
+        if (!itn.has_b) {
+          if (!warp_wait(smem_u32(&bar_qfull[sBn]), ((uB + 2) / NQ) & 1, wc, 26)) return false;
+          commit(&bar_qempty[sBn]);
+          commit(&bar_empty[L0n % NS]);
+        }
+        return true;
+      };
+      auto start_next_b = [&]() -> bool {
+        if (!nx.valid || !itn.has_b) return true;
+        if (!warp_wait(smem_u32(&bar_qfull[sBn]), ((uB + 2) / NQ) & 1, wc, 27)) return false;
+        issue_s(1, sBn, L0n);
+        commit(&bar_empty[L0n % NS]);
+        return true;
+      };
       for (int j = 0; ok && j < it.nkv; ++j) {
         const int Lv = L0 + 2 * j + 1, Lk1 = L0 + 2 * j + 2;
         if (j <= lastA) {
@@ -298,6 +329,8 @@ __global__ void __launch_bounds__(320, 1)
             issue_s(0, sA, Lk1);
             if (j + 1 == lastA) commit(&bar_qempty[sA]);
             if (j + 1 > lastB) commit(&bar_empty[Lk1 % NS]);
+          } else if (!(ok = start_next_a() && (lastB >= 0 || start_next_b()))) {
+            break;
           }
         }
         if (j <= lastB) {
@@ -313,12 +346,15 @@ __global__ void __launch_bounds__(320, 1)
             issue_s(1, sB, Lk1);
             if (j + 1 == lastB) commit(&bar_qempty[sB]);
             commit(&bar_empty[Lk1 % NS]);
+          } else if (!(ok = start_next_b())) {
+            break;
           }
         }
       }
-      L = L0 + 2 * it.nkv;
+      L = L0n;
       ++n;
-      cur.next(a.sched);
+      pre = nx.valid;
+      cur = nx;
     }
     // every issued UMMA completes before TMEM is released
     if (elect_one()) {
@@ -422,17 +458,30 @@ __global__ void __launch_bounds__(320, 1)
         const int tq = original_row(d, it.g * d.G + t * kTile + row, it.sh);
         __nv_bfloat16* orow =
             static_cast<__nv_bfloat16*>(a.o) + ((static_cast<size_t>(it.b) * d.N + tq) * d.H + it.h) * D;
+        if (a.o_v8) {
+          // 32-byte stores: each writes a whole sector of the row
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+          for (int c = 0; c < D / 16; ++c) {
+            uint32_t v[8];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint4 v;
-            v.x = pack_bf16x2(__uint_as_float(o[c][8 * q + 0]) * inv_l, __uint_as_float(o[c][8 * q + 1]) * inv_l);
-            v.y = pack_bf16x2(__uint_as_float(o[c][8 * q + 2]) * inv_l, __uint_as_float(o[c][8 * q + 3]) * inv_l);
-            v.z = pack_bf16x2(__uint_as_float(o[c][8 * q + 4]) * inv_l, __uint_as_float(o[c][8 * q + 5]) * inv_l);
-            v.w = pack_bf16x2(__uint_as_float(o[c][8 * q + 6]) * inv_l, __uint_as_float(o[c][8 * q + 7]) * inv_l);
-            dst[q] = v;
+            for (int q = 0; q < 8; ++q)
+              v[q] = pack_bf16x2(__uint_as_float(o[c >> 1][(c & 1) * 16 + 2 * q]) * inv_l,
+                                 __uint_as_float(o[c >> 1][(c & 1) * 16 + 2 * q + 1]) * inv_l);
+            st_global_v8(orow + c * 16, v);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              uint4 v;
+              v.x = pack_bf16x2(__uint_as_float(o[c][8 * q + 0]) * inv_l, __uint_as_float(o[c][8 * q + 1]) * inv_l);
+              v.y = pack_bf16x2(__uint_as_float(o[c][8 * q + 2]) * inv_l, __uint_as_float(o[c][8 * q + 3]) * inv_l);
+              v.z = pack_bf16x2(__uint_as_float(o[c][8 * q + 4]) * inv_l, __uint_as_float(o[c][8 * q + 5]) * inv_l);
+              v.w = pack_bf16x2(__uint_as_float(o[c][8 * q + 6]) * inv_l, __uint_as_float(o[c][8 * q + 7]) * inv_l);
+              dst[q] = v;
+            }
           }
         }
         a.lse[(static_cast<size_t>(it.b) * d.H + it.h) * d.N + tq] = (m_run + __log2f(l_run)) * 0.69314718055994530942f;

@@ -287,6 +287,7 @@ int s2attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   a.sched = make_fwd_sched(a.d);
   a.scale_log2 = static_cast<float>(1.4426950408889634 / __builtin_sqrt(static_cast<double>(D)));
   a.o = o;
+  a.o_v8 = (reinterpret_cast<uintptr_t>(o) & 31u) == 0 ? 1 : 0;
   a.lse = lse;
   void* status = nullptr;
   if (cudaGetSymbolAddress(&status, g_fwd_status) != cudaSuccess) return S2ATTN_ERR_CUDA;

@@ -162,3 +162,21 @@ def test_exp2_fma_against_cuda_exp2f():
                               torch.cuda.current_stream().cuda_stream)
     torch.cuda.synchronize()
     assert bool((yp2 >= 0).all()) and float(yp2.max()) < 1e-37
+
+
+def test_forward_output_only_16_byte_aligned():
+    """An output buffer that is 16- but not 32-byte aligned takes the 16-byte
+    store path of the epilogue; it must give the same bits as the aligned one."""
+    import sparse_attention_attn_b200 as s2
+    shape = I.Shape("align", 1, 4, 2, 128, 1024, 256)
+    q, k, v, _ = (t.to("cuda:0") for t in I.make_inputs(shape, seed_offset=3))
+    o_ref, lse_ref = s2.s2attn_forward(q, k, v, shape.G)
+    n = q.numel()
+    buf = torch.empty(n + 64, dtype=torch.bfloat16, device="cuda:0")
+    off = next(i for i in range(16) if (buf.data_ptr() + 2 * i) % 32 == 16)
+    o16 = buf[off:off + n].view_as(q)
+    assert o16.data_ptr() % 16 == 0 and o16.data_ptr() % 32 == 16
+    o_got, lse_got = s2.s2attn_forward(q, k, v, shape.G, out=o16)
+    torch.cuda.synchronize()
+    assert s2.device_status() == 0
+    assert torch.equal(o_got, o_ref) and torch.equal(lse_got, lse_ref)
