@@ -18,6 +18,7 @@ from __future__ import annotations
 
 import argparse
 import ctypes
+import hashlib
 import json
 import os
 import statistics
@@ -62,6 +63,31 @@ def load_peaks():
         with open(p) as fh:
             return json.load(fh), "measured"
     return dict(FALLBACK_PEAKS), "fallback"
+
+
+def recorded_traffic(kernel: str, workload: str, root: str = ROOT):
+    """DRAM bytes per launch of `kernel` on `workload` from the committed ncu
+    record (profiles/dram_traffic_<workload>.txt), or None when there is no
+    record or the kernel's sources changed since it was taken."""
+    path = os.path.join(root, "profiles", f"dram_traffic_{workload}.txt")
+    if not os.path.exists(path):
+        return None
+    csrc = os.path.join(root, "sparse_attention_attn_b200", "csrc")
+    with open(path) as fh:
+        for line in fh:
+            f = line.split()
+            if not f or f[0].startswith("#") or f[0] != kernel or f[1] != workload:
+                continue
+            h = hashlib.sha256()
+            for name in f[5:]:
+                src = os.path.join(csrc, name)
+                if not os.path.exists(src):
+                    return None
+                h.update(name.encode())
+                with open(src, "rb") as sf:
+                    h.update(sf.read())
+            return int(f[2]) + int(f[3]) if h.hexdigest() == f[4] else None
+    return None
 
 
 class ClockSampler:
@@ -313,7 +339,7 @@ def run_ours(args, shape, world, rank, local):
         "kernel": KERNEL_NAMES[dom_id], "bound": bound, "achieved": dom.get("achieved"),
         "peak": peaks["bf16_tflops"] if bound == "tensor" else peaks["hbm_gbs"],
         "unit": "TFLOP/s" if bound == "tensor" else "GB/s", "frac": dom.get("frac"),
-        "traffic": None, "peak_source": f"{peak_src} ({'bf16_tflops burst' if bound == 'tensor' else 'hbm_gbs'})",
+        "traffic": recorded_traffic(KERNEL_NAMES[dom_id], shape.name), "peak_source": f"{peak_src} ({'bf16_tflops burst' if bound == 'tensor' else 'hbm_gbs'})",
         "share": (sum(per_kernel[dom_id]) / sum(sum(v) for v in per_kernel.values())) if per_kernel else None,
     }
     line = {
