@@ -474,8 +474,13 @@ __global__ void __launch_bounds__(352, 1)
 // values of each item stream in 64-row sub-tiles from the group start to the
 // diagonal.  S and dP (128 x 64) are double-buffered in TMEM so the UMMAs of
 // sub-tile g+1 overlap the dS work on sub-tile g; Q/dO are double-buffered
-// across items.  TMEM: S [0,128) (two buffers), dP [128,256), dQ [256, 256+D);
-// dQ is read out by the item's epilogue before the next item overwrites it.
+// across items in shared memory and copied, one item at a time, into TMEM by
+// the dS warps, so S = Q K^T and dP = dO V^T take their A operand from TMEM
+// and read only K / V from shared memory (an SS UMMA with N = 64 would be
+// limited by shared-memory bandwidth).  TMEM: S [0,128) (two buffers),
+// dP [128,256), dQ [256, 256+D), Q [256+D, 256+3D/2), dO [256+3D/2, 256+2D)
+// (bf16 pairs); dQ is read out by the item's epilogue before the next item
+// overwrites it.
 
 template <int D>
 struct DqCfg {
@@ -489,6 +494,7 @@ struct DqCfg {
   static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
   static constexpr int SMEM_BYTES = OFF_V + STAGES * KV_BYTES + 1024;
   static constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DQ = 256;
+  static constexpr uint32_t TM_QT = 256 + D, TM_GT = 256 + D + D / 2;  // Q, dO as UMMA A operands
   static constexpr int THREADS = 320;
 };
 
@@ -523,7 +529,7 @@ __global__ void __launch_bounds__(320, 1)
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  __shared__ __align__(8) uint64_t bar_q[2], bar_q_empty[2], bar_kv[ST], bar_empty[ST], bar_sdp[2],
+  __shared__ __align__(8) uint64_t bar_q[2], bar_q_empty[2], bar_qt, bar_kv[ST], bar_empty[ST], bar_sdp[2],
       bar_ds[2], bar_acc_full, bar_acc_free, bar_drain;
   __shared__ uint32_t tmem_slot;
   __shared__ uint32_t abort_flag;
@@ -553,6 +559,7 @@ __global__ void __launch_bounds__(320, 1)
     }
     mbar_init(smem_u32(&bar_acc_full), 1);
     mbar_init(smem_u32(&bar_acc_free), 8);
+    mbar_init(smem_u32(&bar_qt), 8);  // one elected arrival per dS warp
     mbar_init(smem_u32(&bar_drain), 1);
     fence_barrier_init();
   }
@@ -618,37 +625,34 @@ __global__ void __launch_bounds__(320, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ UMMA issuer
-    const uint32_t idS = make_idesc_bf16(128, kSub, 0, 0);  // S = Q K^T, dP = dO V^T
+    const uint32_t idS = make_idesc_bf16(128, kSub, 0, 0);  // S = Q K^T, dP = dO V^T (A from TMEM)
     const uint32_t idQ = make_idesc_bf16(128, D, 0, 1);     // dQ += dS K (K MN-major)
-    const uint64_t dQ0 = make_sdesc_sw128(sQ(0), 16, 1024);            // K-major (A)
-    const uint64_t dG0 = make_sdesc_sw128(sG(0), 16, 1024);
     const uint64_t dKk = make_sdesc_sw128(sK(0), 16, 1024);            // K-major (B of S)
     const uint64_t dVk = make_sdesc_sw128(sV(0), 16, 1024);
     const uint64_t dKm = make_sdesc_sw128(sK(0), C::KV_ATOM, 1024);    // MN-major (B of dQ)
-    auto issue_sdp = [&](int g, int qb) {
+    auto issue_sdp = [&](int g) {
       const int s = g % ST;
       const uint32_t bo = (g & 1) * kSub;
-      const uint64_t dq = sdesc_advance(dQ0, qb * 2 * C::Q_BYTES), dgo = sdesc_advance(dG0, qb * 2 * C::Q_BYTES);
       const uint64_t dk = sdesc_advance(dKk, s * C::KV_BYTES), dv = sdesc_advance(dVk, s * C::KV_BYTES);
       if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t qo = (kk >> 2) * C::Q_ATOM + (kk & 3) * 32;
           const uint32_t ko = (kk >> 2) * C::KV_ATOM + (kk & 3) * 32;
-          umma_ss(tmem + C::TM_S + bo, sdesc_advance(dq, qo), sdesc_advance(dk, ko), idS, kk > 0);
+          umma_ts(tmem + C::TM_S + bo, tmem + C::TM_QT + kk * 8, sdesc_advance(dk, ko), idS, kk > 0);
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t qo = (kk >> 2) * C::Q_ATOM + (kk & 3) * 32;
           const uint32_t ko = (kk >> 2) * C::KV_ATOM + (kk & 3) * 32;
-          umma_ss(tmem + C::TM_DP + bo, sdesc_advance(dgo, qo), sdesc_advance(dv, ko), idS, kk > 0);
+          umma_ts(tmem + C::TM_DP + bo, tmem + C::TM_GT + kk * 8, sdesc_advance(dv, ko), idS, kk > 0);
         }
         umma_commit(smem_u32(&bar_sdp[g & 1]));
       }
       __syncwarp();
     };
+    // the item's Q / dO are in TMEM (copied there by the dS warps), the
+    // sub-tile's K / V in shared memory
     auto wait_inputs = [&](const DqCursor& c, int g) -> bool {
-      if (c.it == 0 && !warp_wait(smem_u32(&bar_q[c.ic.n & 1]), (c.ic.n >> 1) & 1, wc, 220)) return false;
+      if (c.it == 0 && !warp_wait(smem_u32(&bar_qt), c.ic.n & 1, wc, 220)) return false;
       if (!warp_wait(smem_u32(&bar_kv[g % ST]), (g / ST) & 1, wc, 221)) return false;
       tc_fence_after();
       return true;
@@ -660,12 +664,12 @@ __global__ void __launch_bounds__(320, 1)
     bool ok = true;
     if (cur.ic.valid) {
       ok = wait_inputs(cur, 0);
-      if (ok) issue_sdp(0, cur.ic.n & 1);
+      if (ok) issue_sdp(0);
     }
     for (int g = 0; ok && cur.ic.valid; ++g) {
       if (nxt.ic.valid) {
         if (!wait_inputs(nxt, g + 1)) break;
-        issue_sdp(g + 1, nxt.ic.n & 1);
+        issue_sdp(g + 1);
       }
       if (!warp_wait(smem_u32(&bar_ds[g & 1]), (g >> 1) & 1, wc, 223)) break;
       if (cur.it == 0 && cur.ic.n > 0 &&
@@ -705,9 +709,39 @@ __global__ void __launch_bounds__(320, 1)
     const uint64_t sl2x2 = f2_pack(a.scale_log2, a.scale_log2);
     bool ok = true;
     uint64_t nl2 = 0, nd2 = 0;
+    // Item c's Q rows (warps of half 0) or dO rows (half 1) from the swizzled
+    // shared-memory tile into TMEM as bf16 pairs: the A operand of S / dP.
+    // Called once the previous item's last S and dP have completed.
+    auto put_q = [&](const DqCursor& c) -> bool {
+      const int qb = c.ic.n & 1;
+      bool okq = true;
+      if (lane == 0) okq = mbar_wait(smem_u32(&bar_q[qb]), (c.ic.n >> 1) & 1, wc, 233);
+      if (!__shfl_sync(0xffffffffu, okq, 0)) return false;
+      const uint32_t src = (half == 0 ? sQ(qb) : sG(qb)) + row * 128;
+      const uint32_t sw = static_cast<uint32_t>(row & 7);
+#pragma unroll
+      for (int at = 0; at < D / 64; ++at) {
+        uint32_t r[32];
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          const float4 v = lds_f4(src + at * C::Q_ATOM + ((ch ^ sw) << 4));
+          r[4 * ch] = __float_as_uint(v.x);
+          r[4 * ch + 1] = __float_as_uint(v.y);
+          r[4 * ch + 2] = __float_as_uint(v.z);
+          r[4 * ch + 3] = __float_as_uint(v.w);
+        }
+        tmem_st32(tmem + lane_off + (half == 0 ? C::TM_QT : C::TM_GT) + at * 32, r);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bar_qt));
+      return true;
+    };
     DqCursor cur;
     cur.first(d, ps);
-    for (int g = 0; cur.ic.valid; ++g) {
+    if (cur.ic.valid) ok = put_q(cur);
+    for (int g = 0; ok && cur.ic.valid; ++g) {
       const TileWork& w = cur.w;
       const int tq0 = original_row(d, w.g * d.G + w.tile * kTile, shift_of_head(d, w.h));
       const size_t ridx = (static_cast<size_t>(w.b) * d.H + w.h) * d.N + tq0 + row;
@@ -721,6 +755,16 @@ __global__ void __launch_bounds__(320, 1)
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       tc_fence_after();
+      if (cur.it == cur.iters - 1) {
+        // this item's last S and dP are done with Q / dO in TMEM: bring in the
+        // next item's, so its first S / dP overlap the dS work below
+        DqCursor nq = cur;
+        nq.next(d, ps);
+        if (nq.ic.valid && !put_q(nq)) {
+          ok = false;
+          break;
+        }
+      }
       uint32_t sr[32], dr[32];
       tmem_ld32(tmem + lane_off + C::TM_S + bo, sr);
       tmem_ld32(tmem + lane_off + C::TM_DP + bo, dr);
