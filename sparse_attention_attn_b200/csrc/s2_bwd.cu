@@ -102,6 +102,18 @@ __device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const uint32_t (
 }
 
 
+// The same as two 32-byte stores (whole DRAM sectors); dst 32-byte aligned.
+__device__ __forceinline__ void store_row32_v8(__nv_bfloat16* dst, const uint32_t (&r)[32], float scale) {
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint32_t v[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      v[q] = pack_bf16x2(__uint_as_float(r[16 * h + 2 * q]) * scale, __uint_as_float(r[16 * h + 2 * q + 1]) * scale);
+    st_global_v8(dst + 16 * h, v);
+  }
+}
+
 // ------------------------------------------------------------------ dK / dV
 //
 // Persistent: one CTA per SM walks its share of 128-row kv tiles (work items,
@@ -443,18 +455,27 @@ __global__ void __launch_bounds__(352, 1)
         const size_t grow = (static_cast<size_t>(w.b) * d.N + tk0 + row) * d.Hkv + w.kvh;
         __nv_bfloat16* dvrow = static_cast<__nv_bfloat16*>(a.dv) + grow * D + half * (D / 2);
         __nv_bfloat16* dkrow = static_cast<__nv_bfloat16*>(a.dk) + grow * D + half * (D / 2);
+        uint32_t r[D / 64][32], r2[D / 64][32];
 #pragma unroll
         for (int c = 0; c < D / 64; ++c) {
-          uint32_t r[32], r2[32];
-          tmem_ld32(tmem + lane_off + C::TM_DV + half * (D / 2) + c * 32, r);
-          tmem_ld32(tmem + lane_off + C::TM_DK + half * (D / 2) + c * 32, r2);
-          tmem_wait_ld();
-          store_row32(dvrow + c * 32, r, 1.f);
-          store_row32(dkrow + c * 32, r2, a.scale);
+          tmem_ld32(tmem + lane_off + C::TM_DV + half * (D / 2) + c * 32, r[c]);
+          tmem_ld32(tmem + lane_off + C::TM_DK + half * (D / 2) + c * 32, r2[c]);
         }
+        tmem_wait_ld();
+        // dV / dK are out of TMEM: the next item's first gradient UMMAs may start
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&bar_acc_free));
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c) {
+          if (a.kv_v8) {
+            store_row32_v8(dvrow + c * 32, r[c], 1.f);
+            store_row32_v8(dkrow + c * 32, r2[c], a.scale);
+          } else {
+            store_row32(dvrow + c * 32, r[c], 1.f);
+            store_row32(dkrow + c * 32, r2[c], a.scale);
+          }
+        }
       }
       cur.next(d, ps);
     }
@@ -473,14 +494,19 @@ __global__ void __launch_bounds__(352, 1)
 // Persistent: one CTA per SM walks its share of 128-row query tiles.  Keys and
 // values of each item stream in 64-row sub-tiles from the group start to the
 // diagonal.  S and dP (128 x 64) are double-buffered in TMEM so the UMMAs of
-// sub-tile g+1 overlap the dS work on sub-tile g; Q/dO are double-buffered
-// across items in shared memory and copied, one item at a time, into TMEM by
-// the dS warps, so S = Q K^T and dP = dO V^T take their A operand from TMEM
-// and read only K / V from shared memory (an SS UMMA with N = 64 would be
-// limited by shared-memory bandwidth).  TMEM: S [0,128) (two buffers),
-// dP [128,256), dQ [256, 256+D), Q [256+D, 256+3D/2), dO [256+3D/2, 256+2D)
-// (bf16 pairs); dQ is read out by the item's epilogue before the next item
-// overwrites it.
+// sub-tile g+1 overlap the dS work on sub-tile g.  Q / dO arrive by TMA in one
+// shared-memory buffer and are copied, one item at a time, into TMEM by the dS
+// warps, so S = Q K^T and dP = dO V^T take their A operand from TMEM and read
+// only K / V from shared memory (an SS UMMA with N = 64 would be limited by
+// shared-memory bandwidth); the buffer then takes the next item's Q / dO.
+// Two UMMA issuers split the sub-tile's 20 instructions (one issuing thread
+// manages about one UMMA per 48 cycles, slower than a TS UMMA with N = 64
+// executes): warp 1 issues S, warp 10 dP and dQ += dS K, so each issuer only
+// overwrites buffers its own earlier UMMAs read.  The epilogue stages each
+// warp's 32 rows of dQ in shared memory and writes them back row-contiguous.
+// TMEM: S [0,128) (two buffers), dP [128,256), dQ [256, 256+D),
+// Q [256+D, 256+3D/2), dO [256+3D/2, 256+2D) (bf16 pairs); dQ is read out by
+// the item's epilogue before the next item overwrites it.
 
 template <int D>
 struct DqCfg {
@@ -489,13 +515,15 @@ struct DqCfg {
   static constexpr int KV_ATOM = kSub * 128;
   static constexpr int Q_BYTES = kTile * D * 2;
   static constexpr int KV_BYTES = kSub * D * 2;
-  static constexpr int OFF_Q = 0;  // [2 buffers][Q, dO]
-  static constexpr int OFF_K = 4 * Q_BYTES;
+  static constexpr int ROW_OUT = D;                 // bytes of one row's half of dQ (D/2 bf16)
+  static constexpr int OFF_Q = 0;                   // [Q, dO]
+  static constexpr int OFF_OUT = 2 * Q_BYTES;       // epilogue staging: 8 warps x 32 rows x ROW_OUT
+  static constexpr int OFF_K = OFF_OUT + 8 * 32 * ROW_OUT;
   static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
   static constexpr int SMEM_BYTES = OFF_V + STAGES * KV_BYTES + 1024;
   static constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DQ = 256;
   static constexpr uint32_t TM_QT = 256 + D, TM_GT = 256 + D + D / 2;  // Q, dO as UMMA A operands
-  static constexpr int THREADS = 320;
+  static constexpr int THREADS = 352;
 };
 
 struct DqCursor {
@@ -520,7 +548,7 @@ struct DqCursor {
 };
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(352, 1)
     s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmG,
                      const BwdArgs a) {
@@ -529,8 +557,8 @@ __global__ void __launch_bounds__(320, 1)
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  __shared__ __align__(8) uint64_t bar_q[2], bar_q_empty[2], bar_qt, bar_kv[ST], bar_empty[ST], bar_sdp[2],
-      bar_ds[2], bar_acc_full, bar_acc_free, bar_drain;
+  __shared__ __align__(8) uint64_t bar_q, bar_q_empty, bar_qt, bar_kv[ST], bar_empty[ST], bar_sdp[2], bar_ds[2],
+      bar_acc_full, bar_acc_free, bar_drain[2];
   __shared__ uint32_t tmem_slot;
   __shared__ uint32_t abort_flag;
 
@@ -540,18 +568,19 @@ __global__ void __launch_bounds__(320, 1)
   WaitCtx wc{&abort_flag, a.status, a.wait_limit_ns};
 
   const uint32_t s0 = smem_u32(smem);
-  auto sQ = [&](int qb) { return s0 + C::OFF_Q + qb * 2 * C::Q_BYTES; };
-  auto sG = [&](int qb) { return s0 + C::OFF_Q + qb * 2 * C::Q_BYTES + C::Q_BYTES; };
+  const uint32_t sQ = s0 + C::OFF_Q, sG = s0 + C::OFF_Q + C::Q_BYTES;
   auto sK = [&](int s) { return s0 + C::OFF_K + s * C::KV_BYTES; };
   auto sV = [&](int s) { return s0 + C::OFF_V + s * C::KV_BYTES; };
 
   if (threadIdx.x == 0) {
     abort_flag = 0;
+    mbar_init(smem_u32(&bar_q), 1);
+    mbar_init(smem_u32(&bar_q_empty), 8);  // the dS warps, once Q / dO are in TMEM
+    mbar_init(smem_u32(&bar_qt), 8);       // one elected arrival per dS warp
     for (int i = 0; i < 2; ++i) {
-      mbar_init(smem_u32(&bar_q[i]), 1);
-      mbar_init(smem_u32(&bar_q_empty[i]), 1);
-      mbar_init(smem_u32(&bar_sdp[i]), 1);
-      mbar_init(smem_u32(&bar_ds[i]), 8);  // one elected arrival per elementwise warp
+      mbar_init(smem_u32(&bar_sdp[i]), 2);  // S (warp 1) and dP (warp 10)
+      mbar_init(smem_u32(&bar_ds[i]), 8);   // one elected arrival per dS warp
+      mbar_init(smem_u32(&bar_drain[i]), 1);
     }
     for (int s = 0; s < ST; ++s) {
       mbar_init(smem_u32(&bar_kv[s]), 1);
@@ -559,8 +588,6 @@ __global__ void __launch_bounds__(320, 1)
     }
     mbar_init(smem_u32(&bar_acc_full), 1);
     mbar_init(smem_u32(&bar_acc_free), 8);
-    mbar_init(smem_u32(&bar_qt), 8);  // one elected arrival per dS warp
-    mbar_init(smem_u32(&bar_drain), 1);
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -587,14 +614,14 @@ __global__ void __launch_bounds__(320, 1)
     for (ic.first(ps); ok && ic.valid; ic.next(ps)) {
       const TileWork w = q_item(d, ic.unit, ic.tile);
       const int sh = shift_of_head(d, w.h);
-      const int qb = ic.n & 1;
-      if (ic.n >= 2 && !warp_wait(smem_u32(&bar_q_empty[qb]), ((ic.n >> 1) - 1) & 1, wc, 209)) break;
+      // the buffer is free once the previous item's Q / dO are in TMEM
+      if (ic.n >= 1 && !warp_wait(smem_u32(&bar_q_empty), (ic.n - 1) & 1, wc, 209)) break;
       const int tq0 = original_row(d, w.g * d.G + w.tile * kTile, sh);
       if (elect_one()) {
-        mbar_arrive_expect_tx(smem_u32(&bar_q[qb]), 2 * C::Q_BYTES);
+        mbar_arrive_expect_tx(smem_u32(&bar_q), 2 * C::Q_BYTES);
         for (int c = 0; c < D / 64; ++c) {
-          tma_load_4d(sQ(qb) + c * C::Q_ATOM, &tmQ, smem_u32(&bar_q[qb]), c * 64, w.h, tq0, w.b);
-          tma_load_4d(sG(qb) + c * C::Q_ATOM, &tmG, smem_u32(&bar_q[qb]), c * 64, w.h, tq0, w.b);
+          tma_load_4d(sQ + c * C::Q_ATOM, &tmQ, smem_u32(&bar_q), c * 64, w.h, tq0, w.b);
+          tma_load_4d(sG + c * C::Q_ATOM, &tmG, smem_u32(&bar_q), c * 64, w.h, tq0, w.b);
         }
       }
       __syncwarp();
@@ -619,85 +646,78 @@ __global__ void __launch_bounds__(320, 1)
       }
     }
     if (*wc.abort && lane == 0) {
-      for (int qb = 0; qb < 2 && qb < q_issued; ++qb)
-        drain_wait(smem_u32(&bar_q[qb]), ((q_issued - 1 - qb) >> 1) & 1);
+      if (q_issued > 0) drain_wait(smem_u32(&bar_q), (q_issued - 1) & 1);
       for (int s = 0; s < ST && s < gi; ++s) drain_wait(smem_u32(&bar_kv[s]), ((gi - 1 - s) / ST) & 1);
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ UMMA issuer
-    const uint32_t idS = make_idesc_bf16(128, kSub, 0, 0);  // S = Q K^T, dP = dO V^T (A from TMEM)
+  } else if (warp == 1 || warp == 10) {
+    // ------------------------------------------------------------ UMMA issuers
+    // warp 1: S(g) = Q K_g^T.  warp 10: dP(g) = dO V_g^T, then dQ += dS(g-1) K.
+    // Each waits for dS(g-2) before writing buffer g&1 again.
+    const bool is_s = (warp == 1);
+    const uint32_t idS = make_idesc_bf16(128, kSub, 0, 0);  // S, dP: A from TMEM, B K-major
     const uint32_t idQ = make_idesc_bf16(128, D, 0, 1);     // dQ += dS K (K MN-major)
     const uint64_t dKk = make_sdesc_sw128(sK(0), 16, 1024);            // K-major (B of S)
-    const uint64_t dVk = make_sdesc_sw128(sV(0), 16, 1024);
+    const uint64_t dVk = make_sdesc_sw128(sV(0), 16, 1024);            // K-major (B of dP)
     const uint64_t dKm = make_sdesc_sw128(sK(0), C::KV_ATOM, 1024);    // MN-major (B of dQ)
-    auto issue_sdp = [&](int g) {
-      const int s = g % ST;
+    const uint32_t tA = tmem + (is_s ? C::TM_QT : C::TM_GT);
+    const uint32_t tD = tmem + (is_s ? C::TM_S : C::TM_DP);
+    const uint64_t dB0 = is_s ? dKk : dVk;
+    // S or dP of sub-tile g (cursor c)
+    auto issue_sdp = [&](const DqCursor& c, int g) -> bool {
+      if (c.it == 0 && !warp_wait(smem_u32(&bar_qt), c.ic.n & 1, wc, 220)) return false;
+      if (!warp_wait(smem_u32(&bar_kv[g % ST]), (g / ST) & 1, wc, 221)) return false;
+      if (g >= 2 && !warp_wait(smem_u32(&bar_ds[g & 1]), ((g - 2) >> 1) & 1, wc, 222)) return false;
+      tc_fence_after();
+      const uint64_t db = sdesc_advance(dB0, (g % ST) * C::KV_BYTES);
       const uint32_t bo = (g & 1) * kSub;
-      const uint64_t dk = sdesc_advance(dKk, s * C::KV_BYTES), dv = sdesc_advance(dVk, s * C::KV_BYTES);
       if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ko = (kk >> 2) * C::KV_ATOM + (kk & 3) * 32;
-          umma_ts(tmem + C::TM_S + bo, tmem + C::TM_QT + kk * 8, sdesc_advance(dk, ko), idS, kk > 0);
-        }
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t ko = (kk >> 2) * C::KV_ATOM + (kk & 3) * 32;
-          umma_ts(tmem + C::TM_DP + bo, tmem + C::TM_GT + kk * 8, sdesc_advance(dv, ko), idS, kk > 0);
+          umma_ts(tD + bo, tA + kk * 8, sdesc_advance(db, ko), idS, kk > 0);
         }
         umma_commit(smem_u32(&bar_sdp[g & 1]));
       }
       __syncwarp();
-    };
-    // the item's Q / dO are in TMEM (copied there by the dS warps), the
-    // sub-tile's K / V in shared memory
-    auto wait_inputs = [&](const DqCursor& c, int g) -> bool {
-      if (c.it == 0 && !warp_wait(smem_u32(&bar_qt), c.ic.n & 1, wc, 220)) return false;
-      if (!warp_wait(smem_u32(&bar_kv[g % ST]), (g / ST) & 1, wc, 221)) return false;
-      tc_fence_after();
       return true;
     };
-    DqCursor cur, nxt;
-    cur.first(d, ps);
-    nxt = cur;
-    nxt.next(d, ps);
-    bool ok = true;
-    if (cur.ic.valid) {
-      ok = wait_inputs(cur, 0);
-      if (ok) issue_sdp(0);
-    }
-    for (int g = 0; ok && cur.ic.valid; ++g) {
-      if (nxt.ic.valid) {
-        if (!wait_inputs(nxt, g + 1)) break;
-        issue_sdp(g + 1);
-      }
-      if (!warp_wait(smem_u32(&bar_ds[g & 1]), (g >> 1) & 1, wc, 223)) break;
-      if (cur.it == 0 && cur.ic.n > 0 &&
-          !warp_wait(smem_u32(&bar_acc_free), (cur.ic.n - 1) & 1, wc, 224))
-        break;
+    // dQ += dS(g) K_g (warp 10)
+    auto issue_dq = [&](const DqCursor& c, int g) -> bool {
+      if (!warp_wait(smem_u32(&bar_ds[g & 1]), (g >> 1) & 1, wc, 223)) return false;
+      if (c.it == 0 && c.ic.n > 0 && !warp_wait(smem_u32(&bar_acc_free), (c.ic.n - 1) & 1, wc, 224))
+        return false;
       tc_fence_after();
       const int s = g % ST;
       const uint32_t bo = (g & 1) * kSub;
       const uint64_t dk = sdesc_advance(dKm, s * C::KV_BYTES);
-      const bool last = (cur.it == cur.iters - 1);
+      const bool last = (c.it == c.iters - 1);
       if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < kSub / 16; ++kk)
-          umma_ts(tmem + C::TM_DQ, tmem + C::TM_DP + bo + split_acol64(kk), sdesc_advance(dk, kk * 2048),
-                  idQ, (cur.it > 0 || kk > 0));
+          umma_ts(tmem + C::TM_DQ, tmem + C::TM_DP + bo + split_acol64(kk), sdesc_advance(dk, kk * 2048), idQ,
+                  (c.it > 0 || kk > 0));
+        // S(g) (warp 1) has completed: the dS warps read it before dS(g)
         umma_commit(smem_u32(&bar_empty[s]));
-        if (last) {
-          umma_commit(smem_u32(&bar_acc_full));
-          umma_commit(smem_u32(&bar_q_empty[cur.ic.n & 1]));
-        }
+        if (last) umma_commit(smem_u32(&bar_acc_full));
       }
       __syncwarp();
-      cur = nxt;
-      nxt.next(d, ps);
+      return true;
+    };
+    DqCursor cur, prev;
+    cur.first(d, ps);
+    bool ok = true;
+    int g = 0;
+    for (; ok && cur.ic.valid; ++g) {
+      ok = issue_sdp(cur, g);
+      if (ok && !is_s && g >= 1) ok = issue_dq(prev, g - 1);
+      prev = cur;
+      cur.next(d, ps);
     }
+    if (ok && !is_s && g >= 1) issue_dq(prev, g - 1);
+    // every issued UMMA completes before TMEM is released
     if (elect_one()) {
-      umma_commit(smem_u32(&bar_drain));
-      drain_wait(smem_u32(&bar_drain), 0);
+      umma_commit(smem_u32(&bar_drain[is_s ? 0 : 1]));
+      drain_wait(smem_u32(&bar_drain[is_s ? 0 : 1]), 0);
     }
     __syncwarp();
   } else {
@@ -707,17 +727,21 @@ __global__ void __launch_bounds__(320, 1)
     const int row = quarter * 32 + lane;  // query row inside the tile
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint64_t sl2x2 = f2_pack(a.scale_log2, a.scale_log2);
+    // this warp's epilogue staging: 32 rows x ROW_OUT bytes, 16-byte chunks
+    // swizzled by the row so neither the row-wise writes nor the column-wise
+    // reads conflict
+    const uint32_t stage = s0 + C::OFF_OUT + (warp - 2) * 32 * C::ROW_OUT;
+    constexpr int CH = C::ROW_OUT / 16;  // 16-byte chunks per staged row
     bool ok = true;
     uint64_t nl2 = 0, nd2 = 0;
     // Item c's Q rows (warps of half 0) or dO rows (half 1) from the swizzled
     // shared-memory tile into TMEM as bf16 pairs: the A operand of S / dP.
     // Called once the previous item's last S and dP have completed.
     auto put_q = [&](const DqCursor& c) -> bool {
-      const int qb = c.ic.n & 1;
       bool okq = true;
-      if (lane == 0) okq = mbar_wait(smem_u32(&bar_q[qb]), (c.ic.n >> 1) & 1, wc, 233);
+      if (lane == 0) okq = mbar_wait(smem_u32(&bar_q), c.ic.n & 1, wc, 233);
       if (!__shfl_sync(0xffffffffu, okq, 0)) return false;
-      const uint32_t src = (half == 0 ? sQ(qb) : sG(qb)) + row * 128;
+      const uint32_t src = (half == 0 ? sQ : sG) + row * 128;
       const uint32_t sw = static_cast<uint32_t>(row & 7);
 #pragma unroll
       for (int at = 0; at < D / 64; ++at) {
@@ -735,19 +759,33 @@ __global__ void __launch_bounds__(320, 1)
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bar_qt));
+      if (lane == 0) {
+        mbar_arrive(smem_u32(&bar_qt));
+        mbar_arrive(smem_u32(&bar_q_empty));  // the shared-memory copy may be overwritten
+      }
       return true;
+    };
+    // this thread's row statistics of item c: -lse * log2 e and -Delta
+    auto row_stats = [&](const DqCursor& c, float& l2, float& dl) {
+      const TileWork& w = c.w;
+      const int t0 = original_row(d, w.g * d.G + w.tile * kTile, shift_of_head(d, w.h));
+      const size_t ridx = (static_cast<size_t>(w.b) * d.H + w.h) * d.N + t0 + row;
+      l2 = a.nlse2[ridx];
+      dl = a.ndelta[ridx];
     };
     DqCursor cur;
     cur.first(d, ps);
-    if (cur.ic.valid) ok = put_q(cur);
+    float nl_next = 0.f, nd_next = 0.f;  // the next item's, fetched one item ahead
+    if (cur.ic.valid) {
+      ok = put_q(cur);
+      row_stats(cur, nl_next, nd_next);
+    }
     for (int g = 0; ok && cur.ic.valid; ++g) {
       const TileWork& w = cur.w;
       const int tq0 = original_row(d, w.g * d.G + w.tile * kTile, shift_of_head(d, w.h));
-      const size_t ridx = (static_cast<size_t>(w.b) * d.H + w.h) * d.N + tq0 + row;
       if (cur.it == 0) {
-        nl2 = f2_pack(a.nlse2[ridx], a.nlse2[ridx]);    // -lse * log2 e
-        nd2 = f2_pack(a.ndelta[ridx], a.ndelta[ridx]);  // -Delta
+        nl2 = f2_pack(nl_next, nl_next);
+        nd2 = f2_pack(nd_next, nd_next);
       }
       const uint32_t bo = (g & 1) * kSub + half * 32;
       const int koff = cur.it * kSub - w.tile * kTile;  // kv sub-tile start minus query tile start
@@ -760,9 +798,12 @@ __global__ void __launch_bounds__(320, 1)
         // next item's, so its first S / dP overlap the dS work below
         DqCursor nq = cur;
         nq.next(d, ps);
-        if (nq.ic.valid && !put_q(nq)) {
-          ok = false;
-          break;
+        if (nq.ic.valid) {
+          if (!put_q(nq)) {
+            ok = false;
+            break;
+          }
+          row_stats(nq, nl_next, nd_next);  // in flight during this item's last dS and epilogue
         }
       }
       uint32_t sr[32], dr[32];
@@ -797,18 +838,39 @@ __global__ void __launch_bounds__(320, 1)
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
         tc_fence_after();
-        __nv_bfloat16* dqrow = static_cast<__nv_bfloat16*>(a.dq) +
-                               ((static_cast<size_t>(w.b) * d.N + tq0 + row) * d.H + w.h) * D + half * (D / 2);
+        // this thread's row, columns [half * D/2, (half+1) * D/2), scaled,
+        // as bf16 into the staging rows
+        const uint32_t srow = stage + lane * C::ROW_OUT;
 #pragma unroll
         for (int c = 0; c < D / 64; ++c) {
           uint32_t r[32];
           tmem_ld32(tmem + lane_off + C::TM_DQ + half * (D / 2) + c * 32, r);
           tmem_wait_ld();
-          store_row32(dqrow + c * 32, r, a.scale);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int ch = c * 4 + q;
+            st_shared_v4(srow + ((ch ^ (lane % CH)) << 4),
+                         pack_bf16x2(__uint_as_float(r[8 * q]) * a.scale, __uint_as_float(r[8 * q + 1]) * a.scale),
+                         pack_bf16x2(__uint_as_float(r[8 * q + 2]) * a.scale, __uint_as_float(r[8 * q + 3]) * a.scale),
+                         pack_bf16x2(__uint_as_float(r[8 * q + 4]) * a.scale, __uint_as_float(r[8 * q + 5]) * a.scale),
+                         pack_bf16x2(__uint_as_float(r[8 * q + 6]) * a.scale, __uint_as_float(r[8 * q + 7]) * a.scale));
+          }
         }
+        // dQ is out of TMEM: the next item's first dQ UMMA may start
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&bar_acc_free));
+        // write back row-contiguous: lane l takes chunk l % CH of staged row
+        // 32/CH * i + l / CH, so each store instruction covers whole rows
+        __nv_bfloat16* dq0 = static_cast<__nv_bfloat16*>(a.dq) +
+                             ((static_cast<size_t>(w.b) * d.N + tq0 + quarter * 32) * d.H + w.h) * D + half * (D / 2);
+#pragma unroll
+        for (int i = 0; i < CH; ++i) {
+          const int rr = i * (32 / CH) + lane / CH, ch = lane % CH;
+          const float4 v = lds_f4(stage + rr * C::ROW_OUT + ((ch ^ (rr % CH)) << 4));
+          *reinterpret_cast<float4*>(dq0 + static_cast<size_t>(rr) * d.H * D + ch * 8) = v;
+        }
+        __syncwarp();
       }
       cur.next(d, ps);
     }

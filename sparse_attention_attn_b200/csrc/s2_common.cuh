@@ -285,6 +285,7 @@ struct BwdArgs {
   void* dq;                // bf16 [B, N, H, D]
   void* dk;                // bf16 [B, N, Hkv, D]
   void* dv;                // bf16 [B, N, Hkv, D]
+  int kv_v8;               // dk and dv are 32-byte aligned: whole-sector stores
   uint32_t* status;
   unsigned long long wait_limit_ns;
 };

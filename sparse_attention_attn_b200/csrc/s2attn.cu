@@ -347,6 +347,7 @@ int s2attn_bwd(const void* q, const void* k, const void* v, const void* o, const
   a.dq = dq;
   a.dk = dk;
   a.dv = dv;
+  a.kv_v8 = ((reinterpret_cast<uintptr_t>(dk) | reinterpret_cast<uintptr_t>(dv)) & 31u) == 0 ? 1 : 0;
   a.status = status;
   a.wait_limit_ns = wait_limit_ns();
   int launches = 0;

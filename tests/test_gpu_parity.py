@@ -180,3 +180,26 @@ def test_forward_output_only_16_byte_aligned():
     torch.cuda.synchronize()
     assert s2.device_status() == 0
     assert torch.equal(o_got, o_ref) and torch.equal(lse_got, lse_ref)
+
+
+def test_backward_gradients_only_16_byte_aligned():
+    """dk / dv buffers that are 16- but not 32-byte aligned take the 16-byte
+    store path of the dK/dV epilogue; the bits must match the aligned run."""
+    import sparse_attention_attn_b200 as s2
+    shape = I.Shape("align", 1, 4, 2, 128, 1024, 256)
+    q, k, v, do = (t.to("cuda:0") for t in I.make_inputs(shape, seed_offset=5))
+    o, lse = s2.s2attn_forward(q, k, v, shape.G)
+    dq_ref, dk_ref, dv_ref = s2.s2attn_backward(q, k, v, o, lse, do, shape.G)
+
+    def offset16(like):
+        n = like.numel()
+        buf = torch.empty(n + 64, dtype=like.dtype, device=like.device)
+        off = next(i for i in range(16) if (buf.data_ptr() + 2 * i) % 32 == 16)
+        return buf[off:off + n].view_as(like)
+
+    dk16, dv16 = offset16(k), offset16(v)
+    assert dk16.data_ptr() % 32 == 16 and dv16.data_ptr() % 32 == 16
+    dq, dk, dv = s2.s2attn_backward(q, k, v, o, lse, do, shape.G, dk=dk16, dv=dv16)
+    torch.cuda.synchronize()
+    assert s2.device_status() == 0
+    assert torch.equal(dq, dq_ref) and torch.equal(dk, dk_ref) and torch.equal(dv, dv_ref)
