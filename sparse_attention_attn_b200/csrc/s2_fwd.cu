@@ -111,7 +111,7 @@ __global__ void __launch_bounds__(320, 1)
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   __shared__ __align__(8) uint64_t bar_qfull[NQ], bar_qempty[NQ], bar_full[NS], bar_empty[NS],
-      bar_s[2], bar_p[2], bar_o[2], bar_ofree[2], bar_drain;
+      bar_s[2], bar_plo[2], bar_p[2], bar_o[2], bar_ofree[2], bar_drain;
   __shared__ uint32_t tmem_slot;
   __shared__ uint32_t abort_flag;
 
@@ -135,7 +135,8 @@ __global__ void __launch_bounds__(320, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&bar_s[i]), 1);
-      mbar_init(smem_u32(&bar_p[i]), 4);      // one elected arrival per warp of the warpgroup
+      mbar_init(smem_u32(&bar_plo[i]), 4);    // P keys 0..63 written: one arrival per warp of the warpgroup
+      mbar_init(smem_u32(&bar_p[i]), 4);      // P keys 64..127 written
       mbar_init(smem_u32(&bar_o[i]), 1);
       mbar_init(smem_u32(&bar_ofree[i]), 4);
     }
@@ -252,20 +253,35 @@ __global__ void __launch_bounds__(320, 1)
       }
       __syncwarp();
     };
-    // O_wg (+)= P_wg V(load Lv)
-    auto issue_pv = [&](int wg, int Lv, bool acc) {
+    int L = 0, n = 0, np[2] = {0, 0};  // ring loads and items consumed, P halves received per warpgroup
+    // O_wg (+)= P_wg V(load Lv), keys 64h .. 64h+63 (the half of P that
+    // has arrived); the second half completes the product (bar_o)
+    auto issue_pv = [&](int wg, int Lv, int h, bool acc) {
       tc_fence_after();
       const uint64_t dv = sdesc_advance(dV0, (Lv % NS) * C::TILE_BYTES);
       if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < C::BN / 16; ++kk)
+        for (int kq = 0; kq < C::BN / 32; ++kq) {
+          const int kk = h * (C::BN / 32) + kq;
           umma_ts(tmem + C::TM_O + wg * D, tmem + wg * 128 + kk * 8, sdesc_advance(dv, kk * 2048), idO,
                   acc || kk > 0);
-        umma_commit(smem_u32(&bar_o[wg]));
+        }
+        if (h == 1) umma_commit(smem_u32(&bar_o[wg]));
       }
       __syncwarp();
     };
-    int L = 0, n = 0, np[2] = {0, 0};
+    // P_wg(j) V_j: the first half as soon as P keys 0..63 are in TMEM
+    auto pv = [&](int wg, int Lv, int j, bool first_of_item) -> bool {
+      if (!warp_wait(smem_u32(&bar_plo[wg]), np[wg] & 1, wc, wg == 0 ? 22 : 24) ||
+          (first_of_item && n > 0 && !warp_wait(smem_u32(&bar_ofree[wg]), (n - 1) & 1, wc, wg == 0 ? 23 : 25)) ||
+          !wait_full(Lv))
+        return false;
+      issue_pv(wg, Lv, 0, j > 0);
+      if (!warp_wait(smem_u32(&bar_p[wg]), np[wg] & 1, wc, wg == 0 ? 28 : 29)) return false;
+      issue_pv(wg, Lv, 1, true);
+      ++np[wg];
+      return true;
+    };
     bool pre = false;  // this item's first S_A / S_B were issued at the end of the previous item
     FwdCursor cur;
     cur.first(a.sched);
@@ -316,11 +332,7 @@ __global__ void __launch_bounds__(320, 1)
       for (int j = 0; ok && j < it.nkv; ++j) {
         const int Lv = L0 + 2 * j + 1, Lk1 = L0 + 2 * j + 2;
         if (j <= lastA) {
-          ok = warp_wait(smem_u32(&bar_p[0]), np[0] & 1, wc, 22) &&
-               (j > 0 || n == 0 || warp_wait(smem_u32(&bar_ofree[0]), (n - 1) & 1, wc, 23)) && wait_full(Lv);
-          if (!ok) break;
-          ++np[0];
-          issue_pv(0, Lv, j > 0);
+          if (!(ok = pv(0, Lv, j, j == 0))) break;
           if (j > lastB) commit(&bar_empty[Lv % NS]);
           if (j + 1 <= lastA) {
             if (!wait_full(Lk1)) { ok = false; break; }
@@ -332,12 +344,7 @@ __global__ void __launch_bounds__(320, 1)
           }
         }
         if (j <= lastB) {
-          ok = warp_wait(smem_u32(&bar_p[1]), np[1] & 1, wc, 24) &&
-               (j > 0 || n == 0 || warp_wait(smem_u32(&bar_ofree[1]), (n - 1) & 1, wc, 25)) &&
-               (j <= lastA || wait_full(Lv));
-          if (!ok) break;
-          ++np[1];
-          issue_pv(1, Lv, j > 0);
+          if (!(ok = pv(1, Lv, j, j == 0))) break;
           commit(&bar_empty[Lv % NS]);
           if (j + 1 <= lastB) {
             if (j + 1 > lastA && !wait_full(Lk1)) { ok = false; break; }
@@ -407,13 +414,12 @@ __global__ void __launch_bounds__(320, 1)
             m_run = mx;
             resc = true;
           }
-          uint32_t pk[2][32];
-          const float rs = softmax_row64(sr[0], sr[1], sl2, m_run, pk[0]) + softmax_row64(sr[2], sr[3], sl2, m_run, pk[1]);
-          l_run = l_run * alpha + rs;
-          // P (bf16) over the first 64 columns of S; every S column of this
-          // thread's row was read above
-          tmem_st32(tS, pk[0]);
-          tmem_st32(tS + 32, pk[1]);
+          // P (bf16) over the first 64 columns of S, in two halves so the
+          // issuer can start P V on keys 0..63 while keys 64..127 are being
+          // computed; every S column of this thread's row was read above
+          uint32_t pk[32];
+          float rs = softmax_row64(sr[0], sr[1], sl2, m_run, pk);
+          tmem_st32(tS, pk);
           if (__any_sync(0xffffffffu, resc)) {
             // rescale O (it holds P_{j-1} V_{j-1} once that UMMA has completed)
             // before P_j V_j accumulates onto it
@@ -431,6 +437,13 @@ __global__ void __launch_bounds__(320, 1)
               tmem_st32(tO + c * 32, o);
             }
           }
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&bar_plo[wg]));
+          rs += softmax_row64(sr[2], sr[3], sl2, m_run, pk);
+          tmem_st32(tS + 32, pk);
+          l_run = l_run * alpha + rs;
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
