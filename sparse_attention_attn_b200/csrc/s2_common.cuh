@@ -257,8 +257,7 @@ struct FwdArgs {
   Dims d;
   FwdSched sched;
   float scale_log2;        // (1/sqrt(D)) * log2(e)
-  void* o;                 // bf16 [B, N, H, D]
-  int o_v8;                // o is 32-byte aligned: the epilogue writes whole 32-byte sectors
+  void* o;                 // bf16 [B, N, H, D] (written through a TMA map; kept for reference)
   float* lse;              // fp32 [B, H, N]
   uint32_t* status;        // device status words
   unsigned long long wait_limit_ns;

@@ -104,7 +104,8 @@ __device__ __forceinline__ float softmax_row64(const uint32_t (&s0)[32], const u
 template <int D>
 __global__ void __launch_bounds__(320, 1)
     s2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                  const __grid_constant__ CUtensorMap tmV, const FwdArgs a) {
+                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                  const FwdArgs a) {
   using C = FwdCfg<D>;
   constexpr int NQ = C::QSLOTS, NS = C::KVSLOTS;
   extern __shared__ unsigned char smem_raw[];
@@ -127,7 +128,7 @@ __global__ void __launch_bounds__(320, 1)
     abort_flag = 0;
     for (int s = 0; s < NQ; ++s) {
       mbar_init(smem_u32(&bar_qfull[s]), 1);
-      mbar_init(smem_u32(&bar_qempty[s]), 1);
+      mbar_init(smem_u32(&bar_qempty[s]), 4);  // the four warps whose O went out through the slot
     }
     for (int s = 0; s < NS; ++s) {
       mbar_init(smem_u32(&bar_full[s]), 1);
@@ -203,18 +204,26 @@ __global__ void __launch_bounds__(320, 1)
     if (cur.valid) {
       FwdItem it = fwd_item(d, cur.unit, cur.i);
       ok = load_q(it, it.ta, true) && load_q(it, it.ta + 1, it.has_b);
+      bool qb_pending = false;  // this item's second Q tile is still to come
       while (ok && cur.valid) {
         FwdCursor nx = cur;
         nx.next(a.sched);
         const FwdItem itn = fwd_item(d, nx.valid ? nx.unit : cur.unit, nx.valid ? nx.i : cur.i);
-        // the next item's first Q tile goes into the slot its predecessor's
-        // second tile freed: fetched once this item is under way
+        // The next item's first Q tile goes into the slot the previous item's
+        // second tile freed: fetched once this item is under way.  An item's
+        // second Q tile goes into the slot whose tile's O the epilogue stages
+        // at the end of the previous item: fetched after this item's first
+        // K/V tiles, so those never wait for that epilogue.
         const int jq = min(2, it.nkv - 1);
         for (int j = 0; ok && j < it.nkv; ++j) {
           ok = load_kv(it, j, false) && load_kv(it, j, true);
+          if (ok && j == 0 && qb_pending) {
+            ok = load_q(it, it.ta + 1, it.has_b);
+            qb_pending = false;
+          }
           if (ok && j == jq && nx.valid) ok = load_q(itn, itn.ta, true);
         }
-        if (ok && nx.valid) ok = load_q(itn, itn.ta + 1, itn.has_b);
+        qb_pending = nx.valid;
         cur = nx;
         it = itn;
       }
@@ -238,6 +247,11 @@ __global__ void __launch_bounds__(320, 1)
       __syncwarp();
     };
     auto wait_full = [&](int Lx) { return warp_wait(smem_u32(&bar_full[Lx % NS]), (Lx / NS) & 1, wc, 20); };
+    // A Q slot is normally released by the epilogue that staged its tile's O
+    // there (four warps); an item without a second tile releases that slot here.
+    auto release_q = [&](int slot) {
+      for (int i = 0; i < 4; ++i) commit(&bar_qempty[slot]);
+    };
     // S_wg = Q(slot qs) K(load Lk)^T
     auto issue_s = [&](int wg, int qs, int Lk) {
       tc_fence_after();
@@ -301,9 +315,8 @@ __global__ void __launch_bounds__(320, 1)
              warp_wait(smem_u32(&bar_qfull[sB]), (uB / NQ) & 1, wc, 21);
         if (!ok) break;
         issue_s(0, sA, L0);
-        if (lastA == 0) commit(&bar_qempty[sA]);
         if (it.has_b) issue_s(1, sB, L0);
-        else commit(&bar_qempty[sB]);
+        else release_q(sB);
         commit(&bar_empty[L0 % NS]);
       }
       // The next item's first scores are computed as soon as this item's
@@ -314,10 +327,9 @@ __global__ void __launch_bounds__(320, 1)
         if (!nx.valid) return true;
         if (!warp_wait(smem_u32(&bar_qfull[sAn]), ((uA + 2) / NQ) & 1, wc, 26) || !wait_full(L0n)) return false;
         issue_s(0, sAn, L0n);
-        if (itn.ta == 0) commit(&bar_qempty[sAn]);
         if (!itn.has_b) {
           if (!warp_wait(smem_u32(&bar_qfull[sBn]), ((uB + 2) / NQ) & 1, wc, 26)) return false;
-          commit(&bar_qempty[sBn]);
+          release_q(sBn);
           commit(&bar_empty[L0n % NS]);
         }
         return true;
@@ -337,7 +349,6 @@ __global__ void __launch_bounds__(320, 1)
           if (j + 1 <= lastA) {
             if (!wait_full(Lk1)) { ok = false; break; }
             issue_s(0, sA, Lk1);
-            if (j + 1 == lastA) commit(&bar_qempty[sA]);
             if (j + 1 > lastB) commit(&bar_empty[Lk1 % NS]);
           } else if (!(ok = start_next_a() && (lastB >= 0 || start_next_b()))) {
             break;
@@ -349,7 +360,6 @@ __global__ void __launch_bounds__(320, 1)
           if (j + 1 <= lastB) {
             if (j + 1 > lastA && !wait_full(Lk1)) { ok = false; break; }
             issue_s(1, sB, Lk1);
-            if (j + 1 == lastB) commit(&bar_qempty[sB]);
             commit(&bar_empty[Lk1 % NS]);
           } else if (!(ok = start_next_b())) {
             break;
@@ -378,6 +388,7 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t tO = tmem + lane_off + C::TM_O + wg * D;
     const float sl2 = a.scale_log2;
     int ns = 0, no = 0;  // S and PV phases of this warpgroup so far
+    int n_item = 0;      // items walked (the Q-ring use of this warpgroup's tile is 2 n_item + wg)
     FwdCursor cur;
     cur.first(a.sched);
     bool ok = true;
@@ -466,41 +477,45 @@ __global__ void __launch_bounds__(320, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&bar_ofree[wg]));
         const float inv_l = 1.f / l_run;
-        const int tq = original_row(d, it.g * d.G + t * kTile + row, it.sh);
-        __nv_bfloat16* orow =
-            static_cast<__nv_bfloat16*>(a.o) + ((static_cast<size_t>(it.b) * d.N + tq) * d.H + it.h) * D;
-        if (a.o_v8) {
-          // 32-byte stores: each writes a whole sector of the row
+        const int tq0 = original_row(d, it.g * d.G + t * kTile, it.sh);  // the tile never wraps
+        const int tq = tq0 + row;
+        // O (bf16) of this warp's 32 rows into the tile's Q slot, whose last
+        // reader (this tile's last S) has completed: 128-byte swizzled rows in
+        // the TMA layout, then one TMA store per 64-column slab; the slot goes
+        // back to the producer once the stores have read it
+        const int qs = (2 * n_item + wg) % NQ;
+        const uint32_t stage = q_addr(qs) + row * 128;
+        const uint32_t sw = static_cast<uint32_t>(row & 7);
 #pragma unroll
-          for (int c = 0; c < D / 16; ++c) {
-            uint32_t v[8];
+        for (int sl = 0; sl < D / 64; ++sl) {
 #pragma unroll
-            for (int q = 0; q < 8; ++q)
-              v[q] = pack_bf16x2(__uint_as_float(o[c >> 1][(c & 1) * 16 + 2 * q]) * inv_l,
-                                 __uint_as_float(o[c >> 1][(c & 1) * 16 + 2 * q + 1]) * inv_l);
-            st_global_v8(orow + c * 16, v);
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              uint4 v;
-              v.x = pack_bf16x2(__uint_as_float(o[c][8 * q + 0]) * inv_l, __uint_as_float(o[c][8 * q + 1]) * inv_l);
-              v.y = pack_bf16x2(__uint_as_float(o[c][8 * q + 2]) * inv_l, __uint_as_float(o[c][8 * q + 3]) * inv_l);
-              v.z = pack_bf16x2(__uint_as_float(o[c][8 * q + 4]) * inv_l, __uint_as_float(o[c][8 * q + 5]) * inv_l);
-              v.w = pack_bf16x2(__uint_as_float(o[c][8 * q + 6]) * inv_l, __uint_as_float(o[c][8 * q + 7]) * inv_l);
-              dst[q] = v;
-            }
+          for (int ch = 0; ch < 8; ++ch) {
+            const uint32_t* src = &o[2 * sl + (ch >> 2)][(ch & 3) * 8];
+            st_shared_v4(stage + sl * C::ATOM_BYTES + ((ch ^ sw) << 4),
+                         pack_bf16x2(__uint_as_float(src[0]) * inv_l, __uint_as_float(src[1]) * inv_l),
+                         pack_bf16x2(__uint_as_float(src[2]) * inv_l, __uint_as_float(src[3]) * inv_l),
+                         pack_bf16x2(__uint_as_float(src[4]) * inv_l, __uint_as_float(src[5]) * inv_l),
+                         pack_bf16x2(__uint_as_float(src[6]) * inv_l, __uint_as_float(src[7]) * inv_l));
           }
         }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          for (int sl = 0; sl < D / 64; ++sl)
+            tma_store_4d(&tmO, q_addr(qs) + sl * C::ATOM_BYTES + quarter * 32 * 128, sl * 64, it.h, tq0 + quarter * 32,
+                         it.b);
+          bulk_commit_group();
+          bulk_wait_read_all();
+          mbar_arrive(smem_u32(&bar_qempty[qs]));
+        }
+        __syncwarp();
         a.lse[(static_cast<size_t>(it.b) * d.H + it.h) * d.N + tq] = (m_run + __log2f(l_run)) * 0.69314718055994530942f;
       } else {
         // no second tile in this item: keep the O-free phases in step
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&bar_ofree[wg]));
       }
+      ++n_item;
       cur.next(a.sched);
     }
   }
@@ -515,14 +530,14 @@ __global__ void __launch_bounds__(320, 1)
 
 template <int D>
 cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const FwdArgs& a, int num_sms, cudaStream_t stream) {
+                       const CUtensorMap& to, const FwdArgs& a, int num_sms, cudaStream_t stream) {
   using C = FwdCfg<D>;
   cudaError_t ea = cudaFuncSetAttribute(s2_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         C::SMEM_BYTES);
   if (ea != cudaSuccess) return ea;
   const int grid = a.sched.n < num_sms ? a.sched.n : num_sms;
   prof_before(stream, kKernelFwd);
-  s2_fwd_kernel<D><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, a);
+  s2_fwd_kernel<D><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, to, a);
   cudaError_t e = cudaGetLastError();
   prof_after(stream);
   return e;
@@ -551,8 +566,8 @@ cudaError_t launch_exp2_selftest(const float* x, float* y_poly, float* y_ref, in
 }
 
 template cudaError_t launch_fwd<64>(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
-                                    const FwdArgs&, int, cudaStream_t);
+                                    const CUtensorMap&, const FwdArgs&, int, cudaStream_t);
 template cudaError_t launch_fwd<128>(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
-                                     const FwdArgs&, int, cudaStream_t);
+                                     const CUtensorMap&, const FwdArgs&, int, cudaStream_t);
 
 }  // namespace s2

@@ -18,8 +18,8 @@
 
 namespace s2 {
 template <int D>
-cudaError_t launch_fwd(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const FwdArgs&,
-                       int, cudaStream_t);
+cudaError_t launch_fwd(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
+                       const FwdArgs&, int, cudaStream_t);
 template <int D>
 cudaError_t launch_bwd(const BwdMaps&, const BwdPreArgs&, const BwdArgs&, int, cudaStream_t, int*);
 cudaError_t launch_exp2_selftest(const float* x, float* y_poly, float* y_ref, int n, cudaStream_t stream);
@@ -278,24 +278,23 @@ int s2attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   DeviceInfo info;
   if (!device_info(&info)) return S2ATTN_ERR_CUDA;
   if (!info.ok) return S2ATTN_ERR_UNSUPPORTED;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   if (!make_map(&tq, q, B, N, H, D) || !make_map(&tk, k, B, N, Hkv, D) ||
-      !make_map(&tv, v, B, N, Hkv, D))
+      !make_map(&tv, v, B, N, Hkv, D) || !make_map(&to, o, B, N, H, D, 32))
     return S2ATTN_ERR_CUDA;
   FwdArgs a;
   a.d = make_dims(B, H, Hkv, N, D, G);
   a.sched = make_fwd_sched(a.d);
   a.scale_log2 = static_cast<float>(1.4426950408889634 / __builtin_sqrt(static_cast<double>(D)));
   a.o = o;
-  a.o_v8 = (reinterpret_cast<uintptr_t>(o) & 31u) == 0 ? 1 : 0;
   a.lse = lse;
   void* status = nullptr;
   if (cudaGetSymbolAddress(&status, g_fwd_status) != cudaSuccess) return S2ATTN_ERR_CUDA;
   a.status = static_cast<uint32_t*>(status);
   a.wait_limit_ns = wait_limit_ns();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = (D == 64) ? launch_fwd<64>(tq, tk, tv, a, info.sms, s)
-                             : launch_fwd<128>(tq, tk, tv, a, info.sms, s);
+  cudaError_t e = (D == 64) ? launch_fwd<64>(tq, tk, tv, to, a, info.sms, s)
+                             : launch_fwd<128>(tq, tk, tv, to, a, info.sms, s);
   if (e != cudaSuccess) return S2ATTN_ERR_CUDA;
   g_last_launches = 1;
   return S2ATTN_OK;
