@@ -499,10 +499,11 @@ __global__ void __launch_bounds__(352, 1)
 // warps, so S = Q K^T and dP = dO V^T take their A operand from TMEM and read
 // only K / V from shared memory (an SS UMMA with N = 64 would be limited by
 // shared-memory bandwidth); the buffer then takes the next item's Q / dO.
-// Two UMMA issuers split the sub-tile's 20 instructions (one issuing thread
-// manages about one UMMA per 48 cycles, slower than a TS UMMA with N = 64
-// executes): warp 1 issues S, warp 10 dP and dQ += dS K, so each issuer only
-// overwrites buffers its own earlier UMMAs read.  The epilogue stages each
+// Three UMMA issuers split the sub-tile's 20 instructions (next to busy
+// elementwise warps one issuing thread spends far longer per UMMA than a TS
+// UMMA with N = 64 executes): warp 1 issues S, warp 10 dP, warp 11
+// dQ += dS K; warp 10 overwrites a dS buffer only after warp 11's dQ that
+// read it has completed (bar_dqd).  The epilogue stages each
 // warp's 32 rows of dQ in shared memory and writes them back row-contiguous.
 // TMEM: S [0,128) (two buffers), dP [128,256), dQ [256, 256+D),
 // Q [256+D, 256+3D/2), dO [256+3D/2, 256+2D) (bf16 pairs); dQ is read out by
@@ -523,7 +524,7 @@ struct DqCfg {
   static constexpr int SMEM_BYTES = OFF_V + STAGES * KV_BYTES + 1024;
   static constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DQ = 256;
   static constexpr uint32_t TM_QT = 256 + D, TM_GT = 256 + D + D / 2;  // Q, dO as UMMA A operands
-  static constexpr int THREADS = 352;
+  static constexpr int THREADS = 384;
 };
 
 struct DqCursor {
@@ -548,7 +549,7 @@ struct DqCursor {
 };
 
 template <int D>
-__global__ void __launch_bounds__(352, 1)
+__global__ void __launch_bounds__(384, 1)
     s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmG,
                      const BwdArgs a) {
@@ -558,7 +559,7 @@ __global__ void __launch_bounds__(352, 1)
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   __shared__ __align__(8) uint64_t bar_q, bar_q_empty, bar_qt, bar_kv[ST], bar_empty[ST], bar_sdp[2], bar_ds[2],
-      bar_acc_full, bar_acc_free, bar_drain[2];
+      bar_acc_full, bar_acc_free, bar_dqd[2], bar_drain[3];
   __shared__ uint32_t tmem_slot;
   __shared__ uint32_t abort_flag;
 
@@ -580,8 +581,9 @@ __global__ void __launch_bounds__(352, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&bar_sdp[i]), 2);  // S (warp 1) and dP (warp 10)
       mbar_init(smem_u32(&bar_ds[i]), 8);   // one elected arrival per dS warp
-      mbar_init(smem_u32(&bar_drain[i]), 1);
+      mbar_init(smem_u32(&bar_dqd[i]), 1);  // dQ(g) (warp 11) done with dS buffer g&1
     }
+    for (int i = 0; i < 3; ++i) mbar_init(smem_u32(&bar_drain[i]), 1);
     for (int s = 0; s < ST; ++s) {
       mbar_init(smem_u32(&bar_kv[s]), 1);
       mbar_init(smem_u32(&bar_empty[s]), 1);
@@ -649,11 +651,13 @@ __global__ void __launch_bounds__(352, 1)
       if (q_issued > 0) drain_wait(smem_u32(&bar_q), (q_issued - 1) & 1);
       for (int s = 0; s < ST && s < gi; ++s) drain_wait(smem_u32(&bar_kv[s]), ((gi - 1 - s) / ST) & 1);
     }
-  } else if (warp == 1 || warp == 10) {
+  } else if (warp == 1 || warp >= 10) {
     // ------------------------------------------------------------ UMMA issuers
-    // warp 1: S(g) = Q K_g^T.  warp 10: dP(g) = dO V_g^T, then dQ += dS(g-1) K.
-    // Each waits for dS(g-2) before writing buffer g&1 again.
+    // warp 1: S(g) = Q K_g^T.  warp 10: dP(g) = dO V_g^T.  warp 11:
+    // dQ += dS(g) K_g.  S and dP wait for dS(g-2) before writing buffer g&1
+    // again, dP also for dQ(g-2), the last reader of that dS buffer.
     const bool is_s = (warp == 1);
+    const int role = (warp == 1) ? 0 : (warp == 10 ? 1 : 2);
     const uint32_t idS = make_idesc_bf16(128, kSub, 0, 0);  // S, dP: A from TMEM, B K-major
     const uint32_t idQ = make_idesc_bf16(128, D, 0, 1);     // dQ += dS K (K MN-major)
     const uint64_t dKk = make_sdesc_sw128(sK(0), 16, 1024);            // K-major (B of S)
@@ -667,6 +671,7 @@ __global__ void __launch_bounds__(352, 1)
       if (c.it == 0 && !warp_wait(smem_u32(&bar_qt), c.ic.n & 1, wc, 220)) return false;
       if (!warp_wait(smem_u32(&bar_kv[g % ST]), (g / ST) & 1, wc, 221)) return false;
       if (g >= 2 && !warp_wait(smem_u32(&bar_ds[g & 1]), ((g - 2) >> 1) & 1, wc, 222)) return false;
+      if (role == 1 && g >= 2 && !warp_wait(smem_u32(&bar_dqd[g & 1]), ((g - 2) >> 1) & 1, wc, 225)) return false;
       tc_fence_after();
       const uint64_t db = sdesc_advance(dB0, (g % ST) * C::KV_BYTES);
       const uint32_t bo = (g & 1) * kSub;
@@ -696,28 +701,25 @@ __global__ void __launch_bounds__(352, 1)
         for (int kk = 0; kk < kSub / 16; ++kk)
           umma_ts(tmem + C::TM_DQ, tmem + C::TM_DP + bo + split_acol64(kk), sdesc_advance(dk, kk * 2048), idQ,
                   (c.it > 0 || kk > 0));
-        // S(g) (warp 1) has completed: the dS warps read it before dS(g)
+        // S(g) and dP(g) have completed: the dS warps read them before dS(g)
         umma_commit(smem_u32(&bar_empty[s]));
+        umma_commit(smem_u32(&bar_dqd[g & 1]));
         if (last) umma_commit(smem_u32(&bar_acc_full));
       }
       __syncwarp();
       return true;
     };
-    DqCursor cur, prev;
+    DqCursor cur;
     cur.first(d, ps);
     bool ok = true;
-    int g = 0;
-    for (; ok && cur.ic.valid; ++g) {
-      ok = issue_sdp(cur, g);
-      if (ok && !is_s && g >= 1) ok = issue_dq(prev, g - 1);
-      prev = cur;
+    for (int g = 0; ok && cur.ic.valid; ++g) {
+      ok = (role == 2) ? issue_dq(cur, g) : issue_sdp(cur, g);
       cur.next(d, ps);
     }
-    if (ok && !is_s && g >= 1) issue_dq(prev, g - 1);
     // every issued UMMA completes before TMEM is released
     if (elect_one()) {
-      umma_commit(smem_u32(&bar_drain[is_s ? 0 : 1]));
-      drain_wait(smem_u32(&bar_drain[is_s ? 0 : 1]), 0);
+      umma_commit(smem_u32(&bar_drain[role]));
+      drain_wait(smem_u32(&bar_drain[role]), 0);
     }
     __syncwarp();
   } else {
