@@ -21,9 +21,12 @@
 //                       sub-tiles from the group start to the diagonal: S, dP
 //                       in TMEM, dS over dP, dQ += dS K in TMEM.
 //
-// Warp roles of the two UMMA kernels (320 threads): warp 0 TMA producer,
-// warp 1 TMEM owner + UMMA issuer, warps 2..9 elementwise (thread = one TMEM
-// lane = one tile row; warps 2..5 take columns [0,64), warps 6..9 [64,128)).
+// Warp roles of the two UMMA kernels: warp 0 TMA producer, warp 1 TMEM owner
+// and UMMA issuer, warps 2..9 elementwise and epilogue (thread = one TMEM lane
+// = one tile row; warps 2..5 take the first 32 columns of each 64-column
+// sub-tile and the first D/2 output columns, warps 6..9 the rest), and more
+// UMMA issuers after them: warp 10 in dK/dV (352 threads), warps 10 and 11 in
+// dQ (384 threads).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>

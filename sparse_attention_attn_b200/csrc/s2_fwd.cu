@@ -19,11 +19,16 @@
 //               works on one tile while the softmax of the other runs.
 //   warps 2..5  softmax warpgroup A (query tile 2i), warps 6..9 warpgroup B
 //               (tile 2i+1): one thread per query row; S from TMEM, running
-//               max and sum, P (bf16) written back over S, O rescaled in TMEM
-//               only when the running max grows by more than 2^8; epilogue.
+//               max and sum, P (bf16) written back over S in two 64-key
+//               halves (P V on the first starts while the second is being
+//               computed), O rescaled in TMEM only when the running max grows
+//               by more than 2^8; epilogue: O / l staged in the tile's Q slot
+//               and written by TMA stores, lse by the threads.
 //
-// TMEM (512 columns): S_A [0,128), S_B [128,256) (P over their first 64
-// columns), O_A [256, 256+D), O_B [256+D, 256+2D).
+// The issuer starts the next item's S for a warpgroup as soon as that
+// warpgroup's last P V of the current item is issued.  TMEM (512 columns):
+// S_A [0,128), S_B [128,256) (P over their first 64 columns),
+// O_A [256, 256+D), O_B [256+D, 256+2D).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
