@@ -65,6 +65,21 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def source_digest(names, csrc: str):
+    """sha256 over the code of the named sources with comments and whitespace
+    removed, so a record stays valid across comment-only edits."""
+    import re
+    h = hashlib.sha256()
+    for name in names:
+        with open(os.path.join(csrc, name)) as fh:
+            text = fh.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        h.update(name.encode())
+        h.update(" ".join(text.split()).encode())
+    return h.hexdigest()
+
+
 def recorded_traffic(kernel: str, workload: str, root: str = ROOT):
     """DRAM bytes per launch of `kernel` on `workload` from the committed ncu
     record (profiles/dram_traffic_<workload>.txt), or None when there is no
@@ -78,15 +93,9 @@ def recorded_traffic(kernel: str, workload: str, root: str = ROOT):
             f = line.split()
             if not f or f[0].startswith("#") or f[0] != kernel or f[1] != workload:
                 continue
-            h = hashlib.sha256()
-            for name in f[5:]:
-                src = os.path.join(csrc, name)
-                if not os.path.exists(src):
-                    return None
-                h.update(name.encode())
-                with open(src, "rb") as sf:
-                    h.update(sf.read())
-            return int(f[2]) + int(f[3]) if h.hexdigest() == f[4] else None
+            if not all(os.path.exists(os.path.join(csrc, name)) for name in f[5:]):
+                return None
+            return int(f[2]) + int(f[3]) if source_digest(f[5:], csrc) == f[4] else None
     return None
 
 
