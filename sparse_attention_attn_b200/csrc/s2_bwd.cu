@@ -54,42 +54,53 @@ __device__ __forceinline__ float dot_bf16x2(uint32_t a, uint32_t b) {
 
 // ------------------------------------------------------------------ preprocess
 
+// One block per task of 128 consecutive rows t of one (batch, head): every
+// row's D values are read as 16-byte chunks by D/8 lanes (whole rows per
+// instruction), all of the task's loads are in flight at once, and the 128
+// row statistics go out as contiguous runs through shared memory.
 template <int D>
 __global__ void __launch_bounds__(256) s2_bwd_pre_kernel(const BwdPreArgs a) {
-  constexpr int LPR = D / 8;     // lanes per row: one 16-byte chunk each
-  constexpr int RPW = 32 / LPR;  // rows per warp per step
+  constexpr int LPR = D / 8;               // lanes per row: one 16-byte chunk each
+  constexpr int RPS = 256 / LPR;           // rows per step (whole block)
+  constexpr int STEPS = kTile / RPS;       // steps per 128-row task
+  __shared__ float red[kTile];
   const Dims& d = a.d;
-  const long long rows = static_cast<long long>(d.B) * d.N * d.H;
-  const int lane = threadIdx.x & 31;
-  const long long warp_id = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const long long n_warps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
-  const int sub = lane / LPR, part = lane % LPR;
+  const int tid = threadIdx.x;
+  const int part = tid % LPR, rsub = tid / LPR;
   const uint4* o = static_cast<const uint4*>(a.o);
   const uint4* g = static_cast<const uint4*>(a.dO);
-  if (blockIdx.x == 0 && threadIdx.x == 0) {
+  if (blockIdx.x == 0 && tid == 0) {
     a.status[0] = 0u;
     a.status[1] = 0u;
   }
-  for (long long base = warp_id * RPW; base < rows; base += n_warps * RPW) {
-    const long long row = base + sub;  // (b * N + t) * H + h
-    float acc = 0.f;
-    if (row < rows) {
-      const uint4 ov = ldg_stream(o + row * (D / 8) + part);
-      const uint4 gv = ldg_stream(g + row * (D / 8) + part);
-      acc = dot_bf16x2(ov.x, gv.x) + dot_bf16x2(ov.y, gv.y) + dot_bf16x2(ov.z, gv.z) +
-            dot_bf16x2(ov.w, gv.w);
+  const int tblk = d.N / kTile;
+  const long long tasks = static_cast<long long>(d.B) * d.H * tblk;
+  for (long long task = blockIdx.x; task < tasks; task += gridDim.x) {
+    const long long bh = task / tblk;  // b * H + h
+    const int t0 = static_cast<int>(task - bh * tblk) * kTile;
+    const int h = static_cast<int>(bh % d.H), b = static_cast<int>(bh / d.H);
+    uint4 ov[STEPS], gv[STEPS];
+#pragma unroll
+    for (int st = 0; st < STEPS; ++st) {
+      const long long row = (static_cast<long long>(b) * d.N + t0 + st * RPS + rsub) * d.H + h;
+      ov[st] = ldg_stream(o + row * (D / 8) + part);
+      gv[st] = ldg_stream(g + row * (D / 8) + part);
     }
 #pragma unroll
-    for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (row < rows && part == 0) {
-      const int h = static_cast<int>(row % d.H);
-      const long long bt = row / d.H;
-      const int t = static_cast<int>(bt % d.N);
-      const int b = static_cast<int>(bt / d.N);
-      const size_t idx = (static_cast<size_t>(b) * d.H + h) * d.N + t;
-      a.ndelta[idx] = -acc;
+    for (int st = 0; st < STEPS; ++st) {
+      float acc = dot_bf16x2(ov[st].x, gv[st].x) + dot_bf16x2(ov[st].y, gv[st].y) +
+                  dot_bf16x2(ov[st].z, gv[st].z) + dot_bf16x2(ov[st].w, gv[st].w);
+#pragma unroll
+      for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+      if (part == 0) red[st * RPS + rsub] = acc;
+    }
+    __syncthreads();
+    if (tid < kTile) {
+      const size_t idx = static_cast<size_t>(bh) * d.N + t0 + tid;
+      a.ndelta[idx] = -red[tid];
       a.nlse2[idx] = -a.lse[idx] * kLog2e;
     }
+    __syncthreads();
   }
 }
 
@@ -906,8 +917,8 @@ cudaError_t launch_bwd(const BwdMaps& m, const BwdPreArgs& pre, const BwdArgs& a
       !set_smem_attr(reinterpret_cast<const void*>(s2_bwd_dq_kernel<D>), K4::SMEM_BYTES))
     return cudaErrorInvalidValue;
   const long long rows = static_cast<long long>(a.d.B) * a.d.N * a.d.H;
-  const long long want = (rows * (D / 8) + 255) / 256;
-  const int pre_grid = static_cast<int>(want < 16LL * num_sms ? want : 16LL * num_sms);
+  const long long tasks = rows / kTile;  // 128-row tasks of one (batch, head)
+  const int pre_grid = static_cast<int>(tasks < 8LL * num_sms ? tasks : 8LL * num_sms);
   prof_before(stream, kKernelBwdPre);
   s2_bwd_pre_kernel<D><<<pre_grid, 256, 0, stream>>>(pre);
   cudaError_t e = cudaGetLastError();
