@@ -36,41 +36,10 @@ __host__ __device__ __forceinline__ int original_row(const Dims& d, int r, int s
   return t >= d.N ? t - d.N : t;
 }
 
-// Work item of one CTA.  Orders are unit-major so the CTAs resident at one time
-// share their K/V (or Q/dO) tiles in L2, and longest-first inside a unit.
+// A work item: one 128-row tile of one rolled group of one (batch, head).
 struct TileWork {
   int b, h, kvh, g, tile;  // tile = local tile index inside the group
 };
-
-// forward / dQ: one 128-row query tile of head h; work grows with the tile index.
-__host__ __device__ __forceinline__ TileWork decode_q_tile(const Dims& d, int x) {
-  TileWork w;
-  const int T = d.tiles;
-  w.tile = T - 1 - x % T;
-  x /= T;
-  const int hr = x % d.rep;
-  x /= d.rep;
-  w.g = x % d.n_groups;
-  x /= d.n_groups;
-  w.kvh = x % d.Hkv;
-  w.b = x / d.Hkv;
-  w.h = w.kvh * d.rep + hr;
-  return w;
-}
-
-// dK/dV: one 128-row kv tile of kv-head kvh; work shrinks with the tile index.
-__host__ __device__ __forceinline__ TileWork decode_kv_tile(const Dims& d, int x) {
-  TileWork w;
-  const int T = d.tiles;
-  w.tile = x % T;
-  x /= T;
-  w.g = x % d.n_groups;
-  x /= d.n_groups;
-  w.kvh = x % d.Hkv;
-  w.b = x / d.Hkv;
-  w.h = w.kvh * d.rep;  // first query head of the kv-head (they share one shift)
-  return w;
-}
 
 // Persistent schedule.  A "unit" is one rolled group of one (batch, head);
 // its T tiles are the work items.  Work grows (forward, dQ) or shrinks (dK/dV)
@@ -257,7 +226,6 @@ struct FwdArgs {
   Dims d;
   FwdSched sched;
   float scale_log2;        // (1/sqrt(D)) * log2(e)
-  void* o;                 // bf16 [B, N, H, D] (written through a TMA map; kept for reference)
   float* lse;              // fp32 [B, H, N]
   uint32_t* status;        // device status words
   unsigned long long wait_limit_ns;

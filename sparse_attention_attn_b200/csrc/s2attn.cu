@@ -286,8 +286,7 @@ int s2attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   a.d = make_dims(B, H, Hkv, N, D, G);
   a.sched = make_fwd_sched(a.d);
   a.scale_log2 = static_cast<float>(1.4426950408889634 / __builtin_sqrt(static_cast<double>(D)));
-  a.o = o;
-  a.lse = lse;
+  a.lse = lse;  // o is written through its TMA map
   void* status = nullptr;
   if (cudaGetSymbolAddress(&status, g_fwd_status) != cudaSuccess) return S2ATTN_ERR_CUDA;
   a.status = static_cast<uint32_t*>(status);
