@@ -123,9 +123,10 @@ S2ATTN_API const char* s2attn_status_string(int status);
 S2ATTN_API int s2attn_selftest_wait_timeout(uint32_t* status_out, uint64_t limit_ns, s2attn_stream_t stream);
 
 /*
- * Test hook for the forward kernel's FMA-pipe exponential: writes
- * y_poly[i] = the kernel's 2^x (Cody-Waite split plus a minimax cubic) and
- * y_ref[i] = CUDA's exp2f(x[i]) for n device floats.  Asynchronous on stream.
+ * Test hook for the library's FMA-pipe exponential (a Cody-Waite split plus a
+ * minimax cubic; the kernels currently compute every exponential on the MUFU,
+ * which measured faster): writes y_poly[i] = that 2^x and y_ref[i] = CUDA's
+ * exp2f(x[i]) for n device floats.  Asynchronous on stream.
  */
 S2ATTN_API int s2attn_selftest_exp2(const float* x, float* y_poly, float* y_ref, int n,
                                     s2attn_stream_t stream);
