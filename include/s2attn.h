@@ -65,8 +65,9 @@ typedef enum {
 typedef void* s2attn_stream_t;
 
 /*
- * Supported shapes (S2ATTN_ERR_UNSUPPORTED otherwise):
- *   D in {64, 128};  N % 128 == 0;  G % 128 == 0;  N % G == 0;
+ * Shapes.  G <= N, N % G == 0 and H % Hkv == 0 belong to the definition
+ * (S2ATTN_ERR_INVALID_ARG otherwise).  Supported (S2ATTN_ERR_UNSUPPORTED otherwise):
+ *   D in {64, 128};  N % 128 == 0;  G % 128 == 0;
  *   when G < N (shifted heads exist): G % 256 == 0, so the G/2 shift is a
  *   whole number of 128-row tiles, and (H/2) % (H/Hkv) == 0, so the query
  *   heads of one kv-head share one shift;  a device of compute capability 10.0.

@@ -17,15 +17,17 @@ import torch
 from . import _lib
 
 
-def _stream() -> int:
-    return torch.cuda.current_stream().cuda_stream
+def _stream(device=None) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
 
 
-def _need(name: str, t: torch.Tensor, shape, dtype=torch.bfloat16) -> None:
+def _need(name: str, t: torch.Tensor, shape, dtype=torch.bfloat16, device=None) -> None:
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device} (all operands on one device)")
     if t.dtype != dtype:
         raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
     if tuple(t.shape) != tuple(shape):
@@ -48,16 +50,18 @@ def s2attn_forward(q, k, v, group_size: int, out=None, lse=None):
     """
     B, N, H, Hkv, D = _dims(q, k)
     _need("q", q, (B, N, H, D))
-    _need("k", k, (B, N, Hkv, D))
-    _need("v", v, (B, N, Hkv, D))
+    dev = q.device
+    _need("k", k, (B, N, Hkv, D), device=dev)
+    _need("v", v, (B, N, Hkv, D), device=dev)
     if out is None:
         out = torch.empty_like(q)
     if lse is None:
-        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    _need("out", out, (B, N, H, D))
-    _need("lse", lse, (B, H, N), torch.float32)
-    st = _lib.s2attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                         B, H, Hkv, N, D, int(group_size), _stream())
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    _need("out", out, (B, N, H, D), device=dev)
+    _need("lse", lse, (B, H, N), torch.float32, device=dev)
+    with torch.cuda.device(dev):  # the C ABI launches on the current device
+        st = _lib.s2attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                             B, H, Hkv, N, D, int(group_size), _stream(dev))
     _lib._check("s2attn_fwd", st)
     return out, lse
 
@@ -73,25 +77,30 @@ def s2attn_backward(q, k, v, o, lse, do, group_size: int, dq=None, dk=None, dv=N
                     workspace=None):
     """S2-Attn backward.  Returns (dq, dk, dv); dk/dv summed over shared query heads."""
     B, N, H, Hkv, D = _dims(q, k)
-    for name, t, shp in (("q", q, (B, N, H, D)), ("k", k, (B, N, Hkv, D)), ("v", v, (B, N, Hkv, D)),
+    _need("q", q, (B, N, H, D))
+    dev = q.device
+    for name, t, shp in (("k", k, (B, N, Hkv, D)), ("v", v, (B, N, Hkv, D)),
                          ("o", o, (B, N, H, D)), ("do", do, (B, N, H, D))):
-        _need(name, t, shp)
-    _need("lse", lse, (B, H, N), torch.float32)
+        _need(name, t, shp, device=dev)
+    _need("lse", lse, (B, H, N), torch.float32, device=dev)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
-    _need("dq", dq, (B, N, H, D))
-    _need("dk", dk, (B, N, Hkv, D))
-    _need("dv", dv, (B, N, Hkv, D))
+    _need("dq", dq, (B, N, H, D), device=dev)
+    _need("dk", dk, (B, N, Hkv, D), device=dev)
+    _need("dv", dv, (B, N, Hkv, D), device=dev)
     wsb = bwd_workspace_bytes(B, H, Hkv, N, D, group_size)
     if workspace is None:
-        workspace = torch.empty(wsb, dtype=torch.uint8, device=q.device)
+        workspace = torch.empty(wsb, dtype=torch.uint8, device=dev)
+    if not isinstance(workspace, torch.Tensor) or workspace.device != dev or not workspace.is_contiguous():
+        raise ValueError(f"workspace must be a contiguous tensor on {dev}")
     if workspace.numel() * workspace.element_size() < wsb:
         raise _lib.S2AttnError("s2attn_bwd", _lib.S2ATTN_ERR_WORKSPACE)
-    st = _lib.s2attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
-                         do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
-                         B, H, Hkv, N, D, int(group_size), workspace.data_ptr(),
-                         workspace.numel() * workspace.element_size(), _stream())
+    with torch.cuda.device(dev):  # the C ABI launches on the current device
+        st = _lib.s2attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                             do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                             B, H, Hkv, N, D, int(group_size), workspace.data_ptr(),
+                             workspace.numel() * workspace.element_size(), _stream(dev))
     _lib._check("s2attn_bwd", st)
     return dq, dk, dv
 

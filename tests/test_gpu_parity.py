@@ -236,3 +236,44 @@ def test_backward_gradients_only_16_byte_aligned():
     torch.cuda.synchronize()
     assert s2.device_status() == 0
     assert torch.equal(dq, dq_ref) and torch.equal(dk, dk_ref) and torch.equal(dv, dv_ref)
+
+
+def test_binding_rejects_bad_operands():
+    """Wrong dtypes, shapes, strides, group sizes, alignment and workspaces are
+    refused before any launch, and the library stays usable afterwards."""
+    import sparse_attention_attn_b200 as s2
+    from sparse_attention_attn_b200 import _lib
+    shape = I.Shape("reject", 1, 4, 2, 64, 512, 256)
+    q, k, v, do = (t.to("cuda:0") for t in I.make_inputs(shape, seed_offset=7))
+    with pytest.raises(ValueError, match="must be torch.bfloat16"):
+        s2.s2attn_forward(q.float(), k, v, shape.G)
+    with pytest.raises(ValueError, match="has shape"):
+        s2.s2attn_forward(q, k[:, :256], v, shape.G)
+    with pytest.raises(ValueError, match="contiguous"):
+        s2.s2attn_forward(q.transpose(1, 2).contiguous().transpose(1, 2), k, v, shape.G)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        s2.s2attn_forward(q, k.cpu(), v, shape.G)
+    with pytest.raises(_lib.S2AttnError) as e:
+        s2.s2attn_forward(q, k, v, 192)  # N % G != 0
+    assert e.value.status == _lib.S2ATTN_ERR_INVALID_ARG
+    with pytest.raises(_lib.S2AttnError) as e:
+        s2.s2attn_forward(q, k, v, 128)  # shifted groups need G % 256 == 0
+    assert e.value.status == _lib.S2ATTN_ERR_UNSUPPORTED
+    n = q.numel()
+    buf = torch.empty(n + 8, dtype=torch.bfloat16, device="cuda:0")
+    off = next(i for i in range(8) if (buf.data_ptr() + 2 * i) % 16 == 8)
+    with pytest.raises(_lib.S2AttnError) as e:
+        s2.s2attn_forward(q, k, v, shape.G, out=buf[off:off + n].view_as(q))
+    assert e.value.status == _lib.S2ATTN_ERR_MISALIGNED
+    o, lse = s2.s2attn_forward(q, k, v, shape.G)
+    with pytest.raises(ValueError, match="workspace"):
+        s2.s2attn_backward(q, k, v, o, lse, do, shape.G, workspace=torch.empty(1 << 20, dtype=torch.uint8))
+    with pytest.raises(_lib.S2AttnError) as e:
+        s2.s2attn_backward(q, k, v, o, lse, do, shape.G,
+                           workspace=torch.empty(16, dtype=torch.uint8, device="cuda:0"))
+    assert e.value.status == _lib.S2ATTN_ERR_WORKSPACE
+    dq, dk, dv = s2.s2attn_backward(q, k, v, o, lse, do, shape.G)
+    torch.cuda.synchronize()
+    assert s2.device_status() == 0
+    o_ref, _ = ref.s2_attention_fwd(to64(q), to64(k), to64(v), shape.G)
+    assert rel_fro(to64(o), o_ref) <= 5e-3
