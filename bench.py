@@ -293,34 +293,75 @@ def run_ours(args, shape, world, rank, local):
         raise RuntimeError("device status reports a timeout in the timed region")
 
     # ---- end-to-end through the public API with pinned host buffers ----
+    # Every step copies its four inputs in from pinned host memory and its three
+    # gradients out to pinned host memory.  The pipelined loop is how a training
+    # input pipeline feeds the call: step i+1's inputs arrive (copy stream in) and
+    # step i-1's gradients leave (copy stream out) while step i computes, on two
+    # device sets of inputs and gradients.  The serial loop (copies and compute one
+    # after another on one stream) is reported beside it.
     hq, hk, hv, hdo = (t.pin_memory() for t in (q, k, v, do))
     hdq, hdk, hdv = (torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (dq, dk, dv))
-    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo))
-    d2h = sum(t.numel() * t.element_size() for t in (hdq, hdk, hdv))
+    host_in, host_out = (hq, hk, hv, hdo), (hdq, hdk, hdv)
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
+    dev_in = [(qd, kd, vd, dod), tuple(torch.empty_like(t) for t in (qd, kd, vd, dod))]
+    dev_out = [(dq, dk, dv), tuple(torch.empty_like(t) for t in (dq, dk, dv))]
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
 
-    def e2e_step():
-        qd.copy_(hq, non_blocking=True)
-        kd.copy_(hk, non_blocking=True)
-        vd.copy_(hv, non_blocking=True)
-        dod.copy_(hdo, non_blocking=True)
-        step()
-        hdq.copy_(dq, non_blocking=True)
-        hdk.copy_(dk, non_blocking=True)
-        hdv.copy_(dv, non_blocking=True)
+    def compute(i):
+        qi, ki, vi, doi = dev_in[i % 2]
+        dqi, dki, dvi = dev_out[i % 2]
+        s2.s2attn_forward(qi, ki, vi, shape.G, out=o, lse=lse)
+        s2.s2attn_backward(qi, ki, vi, o, lse, doi, shape.G, dq=dqi, dk=dki, dv=dvi, workspace=ws)
+
+    def e2e_serial(n):
+        for _ in range(n):
+            for d_, h_ in zip(dev_in[0], host_in):
+                d_.copy_(h_, non_blocking=True)
+            compute(0)
+            for h_, d_ in zip(host_out, dev_out[0]):
+                h_.copy_(d_, non_blocking=True)
+
+    def e2e_pipelined(n):
+        ev_in, ev_comp, ev_out = ([torch.cuda.Event() for _ in range(n)] for _ in range(3))
+        for i in range(n):
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(ev_comp[i - 2])  # the last reader of this input set
+                for d_, h_ in zip(dev_in[i % 2], host_in):
+                    d_.copy_(h_, non_blocking=True)
+                ev_in[i].record(s_in)
+            stream.wait_event(ev_in[i])
+            if i >= 2:
+                stream.wait_event(ev_out[i - 2])  # this gradient set has left the device
+            compute(i)
+            ev_comp[i].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_comp[i])
+                for h_, d_ in zip(host_out, dev_out[i % 2]):
+                    h_.copy_(d_, non_blocking=True)
+                ev_out[i].record(s_out)
+
+    def timed_e2e(loop, n, first, last):
+        loop(2)
+        torch.cuda.synchronize()
+        barrier(world)
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(first)
+        loop(n)
+        f1.record(last)
+        torch.cuda.synchronize()
+        barrier(world)
+        return max_over_ranks(f0.elapsed_time(f1) / n, world, dev)
 
     e2e_steps = max(3, min(args.steps, 20))
-    for _ in range(2):
-        e2e_step()
-    torch.cuda.synchronize()
-    barrier(world)
-    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    f0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    f1.record(stream)
-    torch.cuda.synchronize()
-    barrier(world)
-    ms_e2e = max_over_ranks(f0.elapsed_time(f1) / e2e_steps, world, dev)
+    ms_e2e_serial = timed_e2e(e2e_serial, e2e_steps, stream, stream)
+    ms_e2e = timed_e2e(e2e_pipelined, e2e_steps, s_in, s_out)
+    if s2.device_status() != 0 or s2.device_status(ws) != 0:
+        raise RuntimeError("device status reports a timeout in the end-to-end loop")
+    # every step has the same inputs: the gradients that reached the host are the device's
+    if not all(torch.equal(h_, d_.cpu()) for h_, d_ in zip(host_out, dev_out[1])):
+        raise RuntimeError("end-to-end loop: gradients on the host differ from the device's")
 
     # ---- report ----
     fwd, bwd = effective_flops(shape)
@@ -362,7 +403,10 @@ def run_ours(args, shape, world, rank, local):
                    "l2": "inputs larger than L2 (q,k,v,dO,o = %d MiB), no flush" %
                          ((4 * qd.numel() + 2 * kd.numel()) * 2 >> 20)},
         "e2e": {"value": total_flops / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e,
+                "loop": "pipelined: copies in / out on two side streams overlap the neighbouring steps' compute",
+                "serial_ms_per_step": ms_e2e_serial,
+                "serial_value": total_flops / (ms_e2e_serial * 1e-3) / 1e12},
         "gpu_launches": gpu_launches,
         "roofline": roofline,
         "kernels": kern,
