@@ -24,6 +24,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -105,14 +106,21 @@ class ClockSampler:
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, csv_dir=None):
+        """The raw samples go to `csv_dir`/clocks_rank<gpu>.csv when a directory
+        is given, else to a temporary file removed once summarised."""
         self.proc = None
         self.gpu = gpu_index
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+        self.keep = csv_dir is not None
+        if self.keep:
+            self.path = os.path.join(csv_dir, f"clocks_rank{gpu_index}.csv")
+        else:
+            fd, self.path = tempfile.mkstemp(prefix=f"s2attn_clocks{gpu_index}_", suffix=".csv")
+            os.close(fd)
 
     def start(self):
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            os.makedirs(os.path.dirname(os.path.abspath(self.path)), exist_ok=True)
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
                                           "--format=csv,noheader,nounits", "-lms", "100"],
@@ -122,6 +130,8 @@ class ClockSampler:
 
     def stop(self):
         if self.proc is None:
+            if not self.keep and os.path.exists(self.path):
+                os.remove(self.path)
             return None
         self.proc.terminate()
         try:
@@ -132,18 +142,21 @@ class ClockSampler:
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         with open(self.path) as fh:
-            for line in fh:
-                f = [x.strip() for x in line.split(",")]
-                if len(f) < 9:
-                    continue
-                try:
-                    sm.append(float(f[1]))
-                    mx = float(f[2])
-                except ValueError:
-                    continue
-                for name, val in zip(names, f[5:9]):
-                    if val.lower().startswith("active"):
-                        reasons.add(name)
+            lines = fh.readlines()
+        if not self.keep:
+            os.remove(self.path)
+        for line in lines:
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, f[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
         if not sm:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
@@ -264,7 +277,7 @@ def run_ours(args, shape, world, rank, local):
         raise RuntimeError("device status reports a timeout during warm-up")
 
     # ---- device-timed region (inputs resident in HBM) ----
-    clocks = ClockSampler(local)
+    clocks = ClockSampler(local, args.clocks_csv_dir)
     clocks.start()
     time.sleep(0.3)
     cap = 4 * args.steps + 8
@@ -463,6 +476,8 @@ def main():
     ap.add_argument("--ref-step-seconds", type=float, default=None,
                     help="oracle seconds per reference step (default: ~2 minutes in total)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--clocks-csv-dir", default=None,
+                    help="keep the raw nvidia-smi clock samples of the timed region in this directory")
     ap.add_argument("--dense-ratio", action="store_true", help="also time G=N on the same inputs")
     args = ap.parse_args()
     shape = {s.name: s for s in I.WORKLOADS}[args.workload]
