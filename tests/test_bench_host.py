@@ -1,7 +1,8 @@
 """Host logic of bench.py that needs no GPU: the roofline traffic record is
 used only while the code of the kernel sources it was measured on is
 unchanged (comment-only edits keep it); the clock sampler's summary of the
-timed region (median SM clock, throttle reasons) from nvidia-smi samples."""
+timed region (median SM clock, throttle reasons) from nvidia-smi samples; the
+reference arm's JSON line (it runs the oracle on the host, no GPU needed)."""
 import os
 
 import bench
@@ -76,3 +77,30 @@ def test_clock_sampler_without_nvidia_smi(monkeypatch):
     c.start()
     assert c.stop() is None
     assert not os.path.exists(c.path)
+
+
+def test_reference_arm_prints_the_contract_line():
+    """`bench.py --impl reference` (the fp64 oracle on the host cores) prints one
+    JSON line with the keys the benchmark contract names."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--workload", "tiny",
+                          "--steps", "2", "--warmup", "1", "--ref-step-seconds", "0.2"],
+                         capture_output=True, text=True, timeout=300, cwd=root,
+                         env={k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")})
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [l for l in out.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+                "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e", "gpu_launches"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["unit"] == "TFLOP/s" and d["value"] > 0
+    assert d["steps"] == 2 and d["warmup"] == 1 and d["higher_is_better"] is True
+    assert d["config"]["workload"] == "tiny"
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"] == {"value": d["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    assert d["gpu_launches"] == 0
