@@ -59,6 +59,8 @@ __all__ = [
     "s2_unit",
     "group_suffix_attention",
     "s2_unit_suffix",
+    "group_prefix_attention",
+    "s2_unit_prefix",
     "s2_effective_flops",
 ]
 
@@ -328,6 +330,73 @@ def s2_unit_suffix(q, k, v, do, G: int, b: int, h: int, g: int, m: int,
     dog = np.asarray(do[b, rows_all, h], dtype=np.float64)
     o, lse, dq, dk, dv, delta = group_suffix_attention(qg, kg, vg, dog, G - m, scale)
     return {"rows": rows_all[G - m:], "o": o, "lse": lse, "dq": dq, "dk_part": dk,
+            "dv_part": dv, "delta": delta, "kv_head": kh, "shift": s}
+
+
+def group_prefix_attention(qg, kg, vg, dog, m: int, scale: float, block: int = 1024):
+    """Causal attention of one group, the outputs that belong to its first rows [0, m).
+
+    Key rows j < m are read by every query row i >= j of the group, so their dk
+    and dv need the whole group: the query rows are streamed in blocks of
+    `block` rows.  Each block's softmax is taken over all the keys its rows see
+    (keys [0, i]), its O (for Delta = rowsum(dO * O)) over all of them too, and
+    only the score columns of keys [0, m) feed dk, dv.  Query rows i < m see
+    only keys [0, i], so their o, lse and dq come out of the first block whole.
+    Same definitions as group_causal_attention(_grad).  Returns
+    (o, lse, dq, dk, dv, delta) for rows [0, m).
+    """
+    n, D = qg.shape
+    dk = np.zeros((m, D))
+    dv = np.zeros((m, D))
+    o_pre = np.zeros((m, D))
+    lse_pre = np.zeros(m)
+    dq_pre = np.zeros((m, D))
+    delta_pre = np.zeros(m)
+    for i0 in range(0, n, block):
+        i1 = min(n, i0 + block)
+        s = scale * (qg[i0:i1] @ kg[:i1].T)
+        vis = np.arange(i1)[None, :] <= np.arange(i0, i1)[:, None]
+        s = np.where(vis, s, -np.inf)
+        mx = s.max(axis=1, keepdims=True)
+        e = np.exp(s - mx)
+        l = e.sum(axis=1, keepdims=True)
+        p = e / l
+        o = p @ vg[:i1]
+        dp = dog[i0:i1] @ vg[:i1].T
+        delta = np.sum(dog[i0:i1] * o, axis=1)
+        ds = p * (dp - delta[:, None])
+        kc = min(m, i1)                      # key columns of the prefix this block sees
+        dk[:kc] += scale * (ds[:, :kc].T @ qg[i0:i1])
+        dv[:kc] += p[:, :kc].T @ dog[i0:i1]
+        if i0 < m:                           # query rows of the prefix in this block
+            r1 = min(m, i1)
+            o_pre[i0:r1] = o[:r1 - i0]
+            lse_pre[i0:r1] = (mx + np.log(l))[:r1 - i0, 0]
+            dq_pre[i0:r1] = scale * (ds[:r1 - i0] @ kg[:i1])
+            delta_pre[i0:r1] = delta[:r1 - i0]
+    return o_pre, lse_pre, dq_pre, dk, dv, delta_pre
+
+
+def s2_unit_prefix(q, k, v, do, G: int, b: int, h: int, g: int, m: int,
+                   scale: float | None = None, block: int = 1024):
+    """Oracle for the first m rolled rows of unit (b, h, g), at original positions.
+
+    The counterpart of s2_unit_suffix for the start of a group: dk_part and
+    dv_part of its first m key rows (the rows every later query row of the
+    group contributes to), and o, lse, dq, delta of its first m query rows.
+    """
+    B, N, H, D = q.shape
+    Hkv = k.shape[2]
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    s = shift_of_head(h, H, N, G)
+    kh = kv_head_of(h, H, Hkv)
+    rows_all = (np.arange(g * G, (g + 1) * G) + s) % N
+    qg = np.asarray(q[b, rows_all, h], dtype=np.float64)
+    kg = np.asarray(k[b, rows_all, kh], dtype=np.float64)
+    vg = np.asarray(v[b, rows_all, kh], dtype=np.float64)
+    dog = np.asarray(do[b, rows_all, h], dtype=np.float64)
+    o, lse, dq, dk, dv, delta = group_prefix_attention(qg, kg, vg, dog, m, scale, block)
+    return {"rows": rows_all[:m], "o": o, "lse": lse, "dq": dq, "dk_part": dk,
             "dv_part": dv, "delta": delta, "kv_head": kh, "shift": s}
 
 

@@ -248,6 +248,71 @@ def test_suffix_matches_full_unit():
             np.testing.assert_allclose(suf[key], full[key][-12:], rtol=0, atol=1e-12, err_msg=key)
 
 
+@pytest.mark.parametrize("m,block", [(12, 5), (12, 64), (32, 7), (1, 3), (20, 20)])
+def test_prefix_matches_full_unit(m, block):
+    """The prefix oracle (dk/dv of a group's first key rows, which every later
+    query row reaches) equals the whole-group oracle on its rows, for query
+    blocks that do not divide the group, blocks smaller and larger than the
+    prefix, and the whole group as the prefix."""
+    B, N, G, H, Hkv, D = 1, 64, 32, 4, 2, 6
+    q, k, v, do = _qkvdo(B, N, H, Hkv, D, seed=14)
+    for h, g in ((0, 1), (3, 1), (2, 0)):
+        full = ref.s2_unit(q, k, v, do, G, b=0, h=h, g=g)
+        pre = ref.s2_unit_prefix(q, k, v, do, G, b=0, h=h, g=g, m=m, block=block)
+        np.testing.assert_array_equal(pre["rows"], full["rows"][:m])
+        for key in ("o", "lse", "dq", "dk_part", "dv_part", "delta"):
+            np.testing.assert_allclose(pre[key], full[key][:m], rtol=0, atol=1e-12, err_msg=key)
+
+
+def test_prefix_and_suffix_cover_whole_tensor_gradients():
+    """dk/dv of a kv-head assembled from prefix (first half) and suffix (second
+    half) pieces, summed over the kv-head's query heads, equal the whole-tensor
+    backward: the two sampling oracles together reach every key row."""
+    B, N, G, H, Hkv, D = 1, 48, 16, 4, 2, 5
+    q, k, v, do = _qkvdo(B, N, H, Hkv, D, seed=15)
+    _, dk, dv, _ = ref.s2_attention_bwd(q, k, v, do, G)
+    rep = H // Hkv
+    for kh in range(Hkv):
+        for g in range(N // G):
+            pk, pv = 0.0, 0.0
+            sk, sv = 0.0, 0.0
+            for h in range(kh * rep, (kh + 1) * rep):
+                pre = ref.s2_unit_prefix(q, k, v, do, G, 0, h, g, m=G // 2, block=5)
+                suf = ref.s2_unit_suffix(q, k, v, do, G, 0, h, g, m=G // 2)
+                pk, pv = pk + pre["dk_part"], pv + pre["dv_part"]
+                sk, sv = sk + suf["dk_part"], sv + suf["dv_part"]
+            np.testing.assert_allclose(pk, dk[0, pre["rows"], kh], rtol=0, atol=1e-12)
+            np.testing.assert_allclose(pv, dv[0, pre["rows"], kh], rtol=0, atol=1e-12)
+            np.testing.assert_allclose(sk, dk[0, suf["rows"], kh], rtol=0, atol=1e-12)
+            np.testing.assert_allclose(sv, dv[0, suf["rows"], kh], rtol=0, atol=1e-12)
+
+
+def test_prefix_planted_mistake_fails():
+    """Taking Delta from the prefix's key columns only (a plausible shortcut:
+    O restricted to keys [0, m)) must break the prefix pin."""
+    B, N, G, H, Hkv, D = 1, 32, 32, 2, 2, 4
+    q, k, v, do = _qkvdo(B, N, H, Hkv, D, seed=16)
+    full = ref.s2_unit(q, k, v, do, G, b=0, h=0, g=0)
+    m = 8
+    qg, kg, vg, dog = (x[0, :, 0] for x in (q, k, v, do))
+    scale = 1.0 / math.sqrt(D)
+
+    def prefix_only_delta(qg, kg, vg, dog, m, scale, block=1024):
+        n = qg.shape[0]
+        s = scale * (qg @ kg.T)
+        s = np.where(np.tril(np.ones((n, n), dtype=bool)), s, -np.inf)
+        p = np.exp(s - s.max(1, keepdims=True))
+        p /= p.sum(1, keepdims=True)
+        delta = np.sum(dog * (p[:, :m] @ vg[:m]), axis=1)
+        ds = p * (dog @ vg.T - delta[:, None])
+        return None, None, None, scale * ds[:, :m].T @ qg, p[:, :m].T @ dog, delta
+
+    good = ref.group_prefix_attention(qg, kg, vg, dog, m, scale, block=7)
+    np.testing.assert_allclose(good[3], full["dk_part"][:m], atol=1e-12, rtol=0)
+    bad = prefix_only_delta(qg, kg, vg, dog, m, scale)
+    assert np.abs(bad[3] - full["dk_part"][:m]).max() > 1e-3
+
+
 def test_rejects_mixed_shift_kv_head():
     q, k, v, _ = _qkvdo(1, 16, 4, 1, 4)
     with pytest.raises(ValueError):
