@@ -218,7 +218,21 @@ def oracle_sample(shape: I.Shape, budget_s: float, seed_offset: int = 0):
     return el, units, units * fwd_unit * 3.5, threads
 
 
+def workload_config(shape: I.Shape, world: int):
+    """The `config` object of the JSON line; both arms print the same one."""
+    q_bytes = shape.B * shape.N * shape.H * shape.D * 2
+    kv_bytes = shape.B * shape.N * shape.Hkv * shape.D * 2
+    return {"workload": shape.name, "B": shape.B, "H": shape.H, "Hkv": shape.Hkv, "D": shape.D,
+            "N": shape.N, "G": shape.G, "parallelism": f"replicas{world}" if world > 1 else "single",
+            "l2": "inputs larger than L2 (q,k,v,dO,o = %d MiB), no flush" % ((3 * q_bytes + 2 * kv_bytes) >> 20)}
+
+
 def run_reference(args, shape, world, rank):
+    """The fp64 oracle timed on the host cores.  One step is one bounded sample
+    of the workload (whole (head, group) units for about --ref-step-seconds);
+    ms_per_step is the measured wall time of such a step, and the rate is the
+    effective FLOPs the sample did divided by that time.  The time a whole
+    workload step would take at that rate is reported under its own key."""
     if rank != 0:
         return
     fwd, bwd = effective_flops(shape)
@@ -232,17 +246,18 @@ def run_reference(args, shape, world, rank):
         total_flops += fl
     tflops = total_flops / total_s / 1e12
     tokens_per_s = total_units * shape.G / total_s
-    ms_per_step = 1e3 * (fwd + bwd) / (tflops * 1e12)  # time the oracle would take for one full step
     line = {
         "impl": "reference", "metric": METRIC, "value": tflops, "unit": "TFLOP/s", "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_s / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "tokens_per_s": tokens_per_s,
-        "config": {"workload": shape.name, "B": shape.B, "H": shape.H, "Hkv": shape.Hkv, "D": shape.D,
-                   "N": shape.N, "G": shape.G},
+        "step": f"one bounded sample of the workload: whole (head, group) units of G={shape.G} rows, "
+                f"fwd+bwd, for about {args.ref_step_seconds:g} s",
+        "full_workload_step_ms_extrapolated": 1e3 * (fwd + bwd) / (tflops * 1e12),
+        "config": workload_config(shape, world),
         "cpu_baseline": {"value": tflops, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                          "sample": f"{total_units} whole (head, group) units of G={shape.G} rows, "
-                                   f"fwd+bwd, over {args.steps} steps"},
+                                   f"fwd+bwd, over {args.steps} steps ({total_s:.1f} s)"},
         "e2e": {"value": tflops, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
     }
@@ -277,11 +292,10 @@ def run_ours(args, shape, world, rank, local):
         raise RuntimeError("device status reports a timeout during warm-up")
 
     # ---- device-timed region (inputs resident in HBM) ----
+    # The headline loop runs with no per-kernel events between the launches.
     clocks = ClockSampler(local, args.clocks_csv_dir)
     clocks.start()
     time.sleep(0.3)
-    cap = 4 * args.steps + 8
-    assert _lib.s2attn_profile_start(cap) == 0
     launches[0] = 0
     barrier(world)
     torch.cuda.synchronize()
@@ -293,11 +307,18 @@ def run_ours(args, shape, world, rank, local):
     torch.cuda.synchronize()
     barrier(world)
     ms_total = e0.elapsed_time(e1)
+    gpu_launches = launches[0]
+    # Per-kernel times: a second loop of the same steps with one CUDA-event pair
+    # around each launch (on the launching stream).
+    cap = 8 * args.steps + 8
+    assert _lib.s2attn_profile_start(cap) == 0
+    for _ in range(args.steps):
+        step()
     ms_arr = (ctypes.c_float * cap)()
     id_arr = (ctypes.c_int * cap)()
     n_rec = _lib.s2attn_profile_stop(ctypes.addressof(ms_arr), ctypes.addressof(id_arr), cap)
+    torch.cuda.synchronize()
     clk = clocks.stop()
-    gpu_launches = launches[0]
     per_kernel = {}
     for i in range(max(n_rec, 0)):
         per_kernel.setdefault(id_arr[i], []).append(ms_arr[i])
@@ -411,10 +432,7 @@ def run_ours(args, shape, world, rank, local):
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "tokens_per_s": tokens,
         "frac_of_bf16_peak": tflops / (peaks["bf16_tflops"] * world),
-        "config": {"workload": shape.name, "B": shape.B, "H": shape.H, "Hkv": shape.Hkv, "D": shape.D,
-                   "N": shape.N, "G": shape.G, "parallelism": f"replicas{world}" if world > 1 else "single",
-                   "l2": "inputs larger than L2 (q,k,v,dO,o = %d MiB), no flush" %
-                         ((4 * qd.numel() + 2 * kd.numel()) * 2 >> 20)},
+        "config": workload_config(shape, world),
         "e2e": {"value": total_flops / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e,
                 "loop": "pipelined: copies in / out on two side streams overlap the neighbouring steps' compute",
@@ -425,8 +443,11 @@ def run_ours(args, shape, world, rank, local):
         "kernels": kern,
         "clocks": clk,
     }
-    if args.dense_ratio and rank == 0:
+    if not args.no_dense_ratio and rank == 0 and shape.G < shape.N:
         line["dense_comparison"] = dense_ratio(shape, dev, args)
+    if not args.no_extra_workloads and world == 1:
+        line["other_workloads"] = {s.name: other_workload(s, dev, peaks)
+                                   for s in I.WORKLOADS if s.name in args.extra_workloads.split(",")}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         el, units, fl, threads = oracle_sample(shape, args.cpu_seconds)
         line["cpu_baseline"] = {"value": fl / el / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
@@ -464,6 +485,39 @@ def dense_ratio(shape: I.Shape, dev, args):
     return {"s2_ms": t_s2, "dense_ms": t_dense, "speedup": t_dense / t_s2}
 
 
+def other_workload(shape: I.Shape, dev, peaks, steps: int = 5, warmup: int = 3):
+    """ms per fwd+bwd step and fraction of the bf16 peak on another workload
+    shape (a few steps; CUDA events on the launching stream)."""
+    import sparse_attention_attn_b200 as s2
+    q, k, v, do = (t.to(dev) for t in I.make_inputs(shape))
+    o = torch.empty_like(q)
+    lse = torch.empty((shape.B, shape.H, shape.N), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(s2.bwd_workspace_bytes(shape.B, shape.H, shape.Hkv, shape.N, shape.D, shape.G),
+                     dtype=torch.uint8, device=dev)
+
+    def step():
+        s2.s2attn_forward(q, k, v, shape.G, out=o, lse=lse)
+        s2.s2attn_backward(q, k, v, o, lse, do, shape.G, dq=dq, dk=dk, dv=dv, workspace=ws)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        step()
+    b.record()
+    torch.cuda.synchronize()
+    if s2.device_status() != 0 or s2.device_status(ws) != 0:
+        raise RuntimeError(f"device status reports a timeout on {shape.name}")
+    ms = a.elapsed_time(b) / steps
+    fwd, bwd = effective_flops(shape)
+    tflops = (fwd + bwd) / (ms * 1e-3) / 1e12
+    return {"ms_per_step": ms, "value": tflops, "unit": "TFLOP/s", "frac_of_bf16_peak": tflops / peaks["bf16_tflops"],
+            "tokens_per_s": shape.B * shape.N / (ms * 1e-3), "steps": steps, "warmup": warmup}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -478,7 +532,12 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--clocks-csv-dir", default=None,
                     help="keep the raw nvidia-smi clock samples of the timed region in this directory")
-    ap.add_argument("--dense-ratio", action="store_true", help="also time G=N on the same inputs")
+    ap.add_argument("--no-dense-ratio", action="store_true",
+                    help="skip timing G=N (dense causal) on the same inputs")
+    ap.add_argument("--no-extra-workloads", action="store_true",
+                    help="skip the few-step timing of the other workload shapes")
+    ap.add_argument("--extra-workloads", default=f"{I.QWEN3_8B_16K.name},{I.LLAMA2_70B_32K.name}",
+                    help="comma-separated workload names timed for a few steps beside the headline")
     args = ap.parse_args()
     shape = {s.name: s for s in I.WORKLOADS}[args.workload]
     if args.ref_step_seconds is None:

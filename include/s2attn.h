@@ -24,8 +24,11 @@
  *                  (scaled scores), indexed by original position.
  * All pointers are DEVICE pointers and must be 16-byte aligned.
  *
- * Ownership: the caller allocates and owns every buffer, including the
- * backward workspace.  The library never allocates or frees device memory.
+ * Ownership: the caller allocates and owns every buffer it passes, including
+ * the backward workspace; the library never allocates or frees device memory
+ * at run time.  Its own device state is fixed at module load: the forward's
+ * status block and the scratch array of s2attn_bwd_noalloc (below), both
+ * file-scope __device__ arrays held by every GPU that loads the library.
  * Calls are asynchronous on `stream` (0 = legacy default stream) and perform
  * no host synchronisation, except s2attn_device_status.
  *
@@ -116,21 +119,47 @@ S2ATTN_API int s2attn_device_status(void* workspace, s2attn_stream_t stream);
 S2ATTN_API const char* s2attn_status_string(int status);
 
 /*
+ * Backward for callers that cannot allocate device memory (no counterpart in
+ * the papers: this is a deployment variant of s2attn_bwd).  Some callers have
+ * no way to get a workspace: they run under another runtime's memory budget
+ * without an allocator handle, inside plugin hosts that forbid cudaMalloc, or
+ * must not allocate between set-up and graph capture.  This call computes
+ * exactly what s2attn_bwd computes, with the same arguments minus the
+ * workspace, and allocates nothing: its scratch (s2attn_bwd_workspace_bytes of
+ * it) is a fixed 32 MiB device array inside the library, which every GPU that
+ * loads the library holds until the process exits.  That limits it to
+ * B * H * N <= 4194272 query rows (all five workload shapes fit); larger
+ * shapes return S2ATTN_ERR_WORKSPACE without launching anything.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current) and caches it per device and context; make that
+ *     first call before any stream capture.  After the device's context is
+ *     destroyed and recreated (cudaDeviceReset), the next call looks the
+ *     address up again, so it too should come before any stream capture.
+ *   - All calls share the array and it keeps the last call's contents; each
+ *     call rewrites what it reads.  Calls that overlap on the GPU (e.g. on two
+ *     streams) race on it and must be serialised by the caller.
+ *   - A bounded-wait timeout is recorded in the array's status block, which is
+ *     not readable through s2attn_device_status; use s2attn_bwd when the
+ *     device status is needed.
+ */
+S2ATTN_API int s2attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                                  const float* lse, const void* dO, void* dq, void* dk, void* dv,
+                                  int B, int H, int Hkv, int N, int D, int G,
+                                  s2attn_stream_t stream);
+
+/* ========================================================================
+ * Test and benchmark hooks.  Not part of the operation: the test suite and
+ * the benchmark use them to exercise the bounded waits, count launches and
+ * time each kernel.  A caller of the attention needs none of them.
+ * ======================================================================== */
+
+/*
  * Self-test of the bounded wait every kernel uses: launches one block that
  * waits on an mbarrier nothing ever arrives at, with a `limit_ns` time limit,
  * and writes the resulting status code (S2ATTN_ERR_DEVICE_TIMEOUT expected)
  * to the device word *status_out.  No fault, trap or endless spin is involved.
  */
 S2ATTN_API int s2attn_selftest_wait_timeout(uint32_t* status_out, uint64_t limit_ns, s2attn_stream_t stream);
-
-/*
- * Test hook for the library's FMA-pipe exponential (a Cody-Waite split plus a
- * minimax cubic; the kernels currently compute every exponential on the MUFU,
- * which measured faster): writes y_poly[i] = that 2^x and y_ref[i] = CUDA's
- * exp2f(x[i]) for n device floats.  Asynchronous on stream.
- */
-S2ATTN_API int s2attn_selftest_exp2(const float* x, float* y_poly, float* y_ref, int n,
-                                    s2attn_stream_t stream);
 
 /* Number of kernel launches the last s2attn_fwd / s2attn_bwd call made on this host thread. */
 S2ATTN_API int s2attn_last_launch_count(void);
@@ -148,33 +177,6 @@ S2ATTN_API int s2attn_last_launch_count(void);
  */
 S2ATTN_API int s2attn_profile_start(int max_launches);
 S2ATTN_API int s2attn_profile_stop(float* ms, int* kernel_ids, int capacity);
-
-/*
- * Backward for callers that cannot allocate device memory (no counterpart in
- * the papers: this is a deployment variant of s2attn_bwd).  Some callers have
- * no way to get a workspace: they run under another runtime's memory budget
- * without an allocator handle, inside plugin hosts that forbid cudaMalloc, or
- * must not allocate between set-up and graph capture.  This call computes
- * exactly what s2attn_bwd computes, with the same arguments minus the
- * workspace, and allocates nothing: its scratch (s2attn_bwd_workspace_bytes of
- * it) is a fixed 32 MiB device array inside the library, which every GPU that
- * loads the library holds until the process exits.  That limits it to
- * B * H * N <= 4194272 query rows (all five workload shapes fit); larger
- * shapes return S2ATTN_ERR_WORKSPACE without launching anything.
- *   - The first call on a device looks up the array's device address (with
- *     that device current) and caches it; make that first call before any
- *     stream capture.
- *   - All calls share the array and it keeps the last call's contents; each
- *     call rewrites what it reads.  Calls that overlap on the GPU (e.g. on two
- *     streams) race on it and must be serialised by the caller.
- *   - A bounded-wait timeout is recorded in the array's status block, which is
- *     not readable through s2attn_device_status; use s2attn_bwd when the
- *     device status is needed.
- */
-S2ATTN_API int s2attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
-                                  const float* lse, const void* dO, void* dq, void* dk, void* dv,
-                                  int B, int H, int Hkv, int N, int D, int G,
-                                  s2attn_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -33,7 +33,6 @@ SIGNATURES = {
     "s2attn_status_string": (ctypes.c_char_p, [_i]),
     "s2attn_selftest_wait_timeout": (_i, [_vp, ctypes.c_uint64, _vp]),
     "s2attn_last_launch_count": (_i, []),
-    "s2attn_selftest_exp2": (_i, [_vp, _vp, _vp, _i, _vp]),
     "s2attn_profile_start": (_i, [_i]),
     "s2attn_profile_stop": (_i, [_vp, _vp, _i]),
     "s2attn_bwd_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
@@ -95,10 +94,6 @@ def s2attn_device_status(workspace, stream) -> int:
 
 def s2attn_selftest_wait_timeout(status_out, limit_ns, stream) -> int:
     return load().s2attn_selftest_wait_timeout(status_out, limit_ns, stream)
-
-
-def s2attn_selftest_exp2(x, y_poly, y_ref, n, stream) -> int:
-    return load().s2attn_selftest_exp2(x, y_poly, y_ref, n, stream)
 
 
 def s2attn_last_launch_count() -> int:

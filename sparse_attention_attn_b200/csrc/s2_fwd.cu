@@ -51,44 +51,9 @@ struct FwdCfg {
   static constexpr int THREADS = 320;
 };
 
-// Cubic for 2^f on [-1/2, 1/2], minimax in relative error (derived by
-// derive_exp2_poly.py in this directory; max relative error 7.5e-5 in float32).
-constexpr float kExp2C0 = 9.999280572e-01f;
-constexpr float kExp2C1 = 6.932609677e-01f;
-constexpr float kExp2C2 = 2.426111251e-01f;
-constexpr float kExp2C3 = 5.517166853e-02f;
-
-// 2^x on the FMA pipe (Cody-Waite split x = n + f, n = round(x), f in
-// [-1/2, 1/2]; 2^n added to the exponent field).  x is clamped below at -126
-// so the result stays a (tiny) non-negative float; inputs here are <= 8.
-__device__ __forceinline__ float exp2_fma(float x) {
-  x = fmaxf(x, -126.f);
-  const float t = x + 12582912.f;  // 1.5 * 2^23: round(x) lands in the low mantissa bits
-  const float f = x - (t - 12582912.f);
-  const float p = fmaf(fmaf(fmaf(kExp2C3, f, kExp2C2), f, kExp2C1), f, kExp2C0);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
-// The same on a packed pair, with f32x2 arithmetic.
-__device__ __forceinline__ uint64_t exp2_fma2(uint64_t x) {
-  const uint64_t xc = f2_pack(fmaxf(f2_lo(x), -126.f), fmaxf(f2_hi(x), -126.f));
-  const uint64_t t = f2_add(xc, f2_pack(12582912.f, 12582912.f));
-  const uint64_t f = f2_add(xc, f2_add(t, f2_pack(-12582912.f, -12582912.f)) ^ 0x8000000080000000ull);
-  uint64_t p = f2_fma(f2_pack(kExp2C3, kExp2C3), f, f2_pack(kExp2C2, kExp2C2));
-  p = f2_fma(p, f, f2_pack(kExp2C1, kExp2C1));
-  p = f2_fma(p, f, f2_pack(kExp2C0, kExp2C0));
-  const uint32_t lo = __float_as_uint(f2_lo(p)) + (static_cast<uint32_t>(t) << 23);
-  const uint32_t hi = __float_as_uint(f2_hi(p)) + (static_cast<uint32_t>(t >> 32) << 23);
-  return (static_cast<uint64_t>(hi) << 32) | lo;
-}
-
 // P for 64 scores of one query row: p = 2^(s * sl2 - m), packed to bf16
 // pairs in pk; returns the fp32 sum.  Arguments and sums use packed f32x2
-// arithmetic, the exponentials the MUFU (ex2.approx).  (Moving a share of the
-// exponentials to the FMA pipe with exp2_fma2 above measured slower in this
-// kernel -- 1/8 of the pairs: +6%, 1/4: +7% forward time at 8K tokens -- as
-// one softmax warp per SMSP is latency-bound, not MUFU-bound; exp2_fma2 is
-// kept with its self-test as a checked building block.)
+// arithmetic, the exponentials the MUFU (ex2.approx).
 __device__ __forceinline__ float softmax_row64(const uint32_t (&s0)[32], const uint32_t (&s1)[32], float sl2,
                                                float m, uint32_t (&pk)[32]) {
   const uint64_t sc2 = f2_pack(sl2, sl2), nm2 = f2_pack(-m, -m);
@@ -546,28 +511,6 @@ cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
   cudaError_t e = cudaGetLastError();
   prof_after(stream);
   return e;
-}
-
-// Test hook: the FMA-pipe exp2 next to CUDA's exp2f on the same inputs.
-// (pairs go through the packed form the softmax uses; an odd last element
-// through the scalar form)
-__global__ void s2_exp2_selftest_kernel(const float* x, float* y_poly, float* y_ref, int n) {
-  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
-  if (i + 1 < n) {
-    const uint64_t p = exp2_fma2(f2_pack(x[i], x[i + 1]));
-    y_poly[i] = f2_lo(p);
-    y_poly[i + 1] = f2_hi(p);
-    y_ref[i] = exp2f(x[i]);
-    y_ref[i + 1] = exp2f(x[i + 1]);
-  } else if (i < n) {
-    y_poly[i] = exp2_fma(x[i]);
-    y_ref[i] = exp2f(x[i]);
-  }
-}
-
-cudaError_t launch_exp2_selftest(const float* x, float* y_poly, float* y_ref, int n, cudaStream_t stream) {
-  s2_exp2_selftest_kernel<<<((n + 1) / 2 + 255) / 256, 256, 0, stream>>>(x, y_poly, y_ref, n);
-  return cudaGetLastError();
 }
 
 template cudaError_t launch_fwd<64>(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,

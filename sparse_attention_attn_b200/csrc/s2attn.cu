@@ -1,9 +1,10 @@
 // Host side of the C ABI declared in include/s2attn.h: argument validation,
 // TMA tensor-map encoding, kernel launches and status reporting.
 //
-// Nothing here allocates device memory: every buffer belongs to the caller.
-// The only library-owned device state is the forward's status block, a
-// file-scope __device__ array.
+// Nothing here allocates device memory at run time: the caller owns every
+// buffer it passes.  The library's own device state is fixed at module load:
+// the forward's status block and the scratch array of s2attn_bwd_noalloc,
+// both file-scope __device__ arrays.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -22,7 +23,6 @@ cudaError_t launch_fwd(const CUtensorMap&, const CUtensorMap&, const CUtensorMap
                        const FwdArgs&, int, cudaStream_t);
 template <int D>
 cudaError_t launch_bwd(const BwdMaps&, const BwdPreArgs&, const BwdArgs&, int, cudaStream_t, int*);
-cudaError_t launch_exp2_selftest(const float* x, float* y_poly, float* y_ref, int n, cudaStream_t stream);
 }  // namespace s2
 
 namespace {
@@ -373,16 +373,6 @@ int s2attn_device_status(void* workspace, s2attn_stream_t stream) {
   return words[0] == 0 ? S2ATTN_OK : static_cast<int>(words[0]);
 }
 
-int s2attn_selftest_exp2(const float* x, float* y_poly, float* y_ref, int n, s2attn_stream_t stream) {
-  if (!x || !y_poly || !y_ref || n <= 0) return S2ATTN_ERR_INVALID_ARG;
-  DeviceInfo info;
-  if (!device_info(&info)) return S2ATTN_ERR_CUDA;
-  if (!info.ok) return S2ATTN_ERR_UNSUPPORTED;
-  return launch_exp2_selftest(x, y_poly, y_ref, n, static_cast<cudaStream_t>(stream)) == cudaSuccess
-             ? S2ATTN_OK
-             : S2ATTN_ERR_CUDA;
-}
-
 int s2attn_selftest_wait_timeout(uint32_t* status_out, uint64_t limit_ns, s2attn_stream_t stream) {
   if (!status_out || limit_ns == 0 || limit_ns > 10000000000ull) return S2ATTN_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(status_out) & 7u) != 0) return S2ATTN_ERR_MISALIGNED;
@@ -416,18 +406,45 @@ constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB
 static __device__ __align__(256) unsigned char g_bwd_scratch[kNoAllocScratchBytes];
 
 // Device address of g_bwd_scratch on the current device.  In host code the
-// array's name is only a host-side stand-in, so the address is looked up once
-// per device, with that device current, and cached.
+// array's name is only a host-side stand-in, so the address is looked up with
+// the device current, once per device and context, and cached.  The cache is
+// keyed on the current context as well as the device index: a context torn
+// down and recreated (cudaDeviceReset) loads the module again at a new
+// address, so a changed context handle triggers a new lookup.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+
+CtxGetCurrentFn get_ctx_current() {
+  static std::once_flag once;
+  static CtxGetCurrentFn fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  return fn;
+}
+
 bool noalloc_scratch(void** out) {
   static std::mutex mu;
   static void* ptrs[64] = {};
+  static CUcontext ctxs[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  CtxGetCurrentFn ctx_current = get_ctx_current();
+  if (!ctx_current) return false;
   std::lock_guard<std::mutex> lk(mu);
-  if (ptrs[dev] == nullptr) {
+  CUcontext ctx = nullptr;
+  // the runtime makes the device's primary context current on first use;
+  // before that there is none and the lookup below creates it
+  if (ctx_current(&ctx) != CUDA_SUCCESS) return false;
+  if (ptrs[dev] == nullptr || ctx == nullptr || ctx != ctxs[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_bwd_scratch) != cudaSuccess || p == nullptr) return false;
+    if (ctx_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
     ptrs[dev] = p;
+    ctxs[dev] = ctx;
   }
   *out = ptrs[dev];
   return true;

@@ -104,3 +104,12 @@ def test_reference_arm_prints_the_contract_line():
     assert d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"] == {"value": d["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
     assert d["gpu_launches"] == 0
+    # the per-step time is the measured time of the sampled steps, which fits
+    # in the run's wall time; the extrapolated whole-workload step is separate
+    assert 0 < d["ms_per_step"] * d["steps"] < 60_000
+    assert d["full_workload_step_ms_extrapolated"] > 0
+    # both arms print the same config object for a workload
+    sys.path.insert(0, root)
+    import bench
+    from sparse_attention_attn_b200 import inputs as I
+    assert d["config"] == bench.workload_config(I.TINY, 1)

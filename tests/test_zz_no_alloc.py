@@ -11,8 +11,9 @@ import numpy as np
 import pytest
 import torch
 
+import oracle.s2_ref as ref
 from sparse_attention_attn_b200 import inputs as I
-from tests.parity_util import GRAD_REL_FRO, rel_fro, to64
+from tests.parity_util import GRAD_REL_FRO, check_grad, rel_fro, to64
 
 pytestmark = pytest.mark.gpu
 
@@ -24,6 +25,8 @@ def test_bwd_noalloc_matches_bwd_twice():
     shape = I.Shape("noalloc", 2, 8, 4, 128, 1024, 256)  # shifted heads, GQA, two batches
     q, k, v, do = (t.cuda() for t in I.make_inputs(shape, seed_offset=3))
     o, lse = s2.s2attn_forward(q, k, v, shape.G)
+    # the fp64 oracle on the same inputs, independent of either entry point
+    dq_or, dk_or, dv_or, _ = ref.s2_attention_bwd(to64(q), to64(k), to64(v), to64(do), shape.G)
     # the existing entry point, with a caller-provided workspace
     dq_ref, dk_ref, dv_ref = s2.s2attn_backward(q, k, v, o, lse, do, shape.G)
     torch.cuda.synchronize()
@@ -37,10 +40,12 @@ def test_bwd_noalloc_matches_bwd_twice():
         assert rc == 0, _lib.status_string(rc)
         assert _lib.s2attn_last_launch_count() == 3
         torch.cuda.synchronize()
-        for name, got, ref in (("dq", dq, dq_ref), ("dk", dk, dk_ref), ("dv", dv, dv_ref)):
-            g, r = to64(got), to64(ref)
+        for name, got, other, oracle_grad in (("dq", dq, dq_ref, dq_or), ("dk", dk, dk_ref, dk_or),
+                                              ("dv", dv, dv_ref, dv_or)):
+            g, r = to64(got), to64(other)
             assert np.isfinite(g).all(), (call, name)
             assert rel_fro(g, r) <= GRAD_REL_FRO, (call, name, rel_fro(g, r))
+            check_grad(name, g, oracle_grad, f" [no-alloc call {call}]")
 
 
 def test_bwd_noalloc_rejects_oversize_shape():
