@@ -1,0 +1,76 @@
+"""fp64 CPU oracle for rotary position embedding with Position Interpolation.
+
+TEST INFRASTRUCTURE ONLY: imported by the test suite, the package smoke check
+and the benchmark's CPU-baseline leg, never by the product path; it shares no
+code with the CUDA kernels.
+
+What the pages state (LongQLoRA community post):
+* §02 Introduction: LLaMA models use RoPE, rotary position encoding, so their
+  context can be extended by adjusting the rotation;
+* §03 Method, Background: Position Interpolation (from Meta) extends the
+  context length by interpolating positions, then a short fine-tune;
+* §04 Setup: Position Interpolation shrinks RoPE's rotation angles to extend
+  LLaMA2 from 4096 to 8192 tokens, before S2 attention is applied.
+
+Readings taken where the pages are silent (listed in the design notes):
+* the rotary pairs are (i, i + D/2) for i < D/2 (the "rotate half" layout);
+* the frequency of pair i is base^(-2i/D) with base 10000;
+* Position Interpolation multiplies every position by s = L_train / L_target
+  (0.5 for 4096 -> 8192), so the angle of pair i at token t is t * s * base^(-2i/D);
+* the rotation is applied to q and k at their original token positions,
+  before the shift and grouping of S2 attention, and not to v;
+* the backward of a rotation is the rotation by the opposite angle.
+
+All arithmetic is float64 numpy.  Layout: x is [B, N, heads, D].
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+from .s2_ref import s2_attention_bwd, s2_attention_fwd
+
+__all__ = ["rope_angles", "rope_rotate", "s2_rope_attention_fwd", "s2_rope_attention_bwd"]
+
+
+def rope_angles(N: int, D: int, pos_scale: float, base: float = 10000.0) -> np.ndarray:
+    """[N, D/2] rotation angles: angle[t, i] = t * pos_scale * base^(-2i/D)."""
+    i = np.arange(D // 2, dtype=np.float64)
+    freq = base ** (-2.0 * i / D)
+    t = np.arange(N, dtype=np.float64) * pos_scale
+    return t[:, None] * freq[None, :]
+
+
+def rope_rotate(x, pos_scale: float, base: float = 10000.0, inverse: bool = False) -> np.ndarray:
+    """Rotate each pair (x_i, x_{i+D/2}) of every row t by angle[t, i]
+    (by -angle[t, i] when `inverse`):
+        y_i        = x_i cos a - x_{i+D/2} sin a
+        y_{i+D/2}  = x_i sin a + x_{i+D/2} cos a
+    x is [B, N, heads, D]; returns a float64 array of the same shape."""
+    x = np.asarray(x, dtype=np.float64)
+    B, N, Hx, D = x.shape
+    a = rope_angles(N, D, pos_scale, base)
+    if inverse:
+        a = -a
+    c = np.cos(a)[None, :, None, :]
+    s = np.sin(a)[None, :, None, :]
+    x1, x2 = x[..., : D // 2], x[..., D // 2:]
+    return np.concatenate([x1 * c - x2 * s, x1 * s + x2 * c], axis=-1)
+
+
+def s2_rope_attention_fwd(q, k, v, G: int, pos_scale: float, base: float = 10000.0):
+    """S2 attention of rotated q and k: returns (o, lse, q_rot, k_rot)."""
+    qr = rope_rotate(q, pos_scale, base)
+    kr = rope_rotate(k, pos_scale, base)
+    o, lse = s2_attention_fwd(qr, kr, v, G)
+    return o, lse, qr, kr
+
+
+def s2_rope_attention_bwd(q, k, v, do, G: int, pos_scale: float, base: float = 10000.0):
+    """Gradients with respect to the unrotated q and k (and v): the S2
+    backward on the rotated inputs, then dq and dk rotated back.
+    Returns (dq, dk, dv)."""
+    qr = rope_rotate(q, pos_scale, base)
+    kr = rope_rotate(k, pos_scale, base)
+    dqr, dkr, dv, _ = s2_attention_bwd(qr, kr, v, do, G)
+    return rope_rotate(dqr, pos_scale, base, inverse=True), rope_rotate(dkr, pos_scale, base, inverse=True), dv
