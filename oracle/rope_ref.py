@@ -30,7 +30,8 @@ import numpy as np
 
 from .s2_ref import s2_attention_bwd, s2_attention_fwd
 
-__all__ = ["rope_angles", "rope_rotate", "s2_rope_attention_fwd", "s2_rope_attention_bwd"]
+__all__ = ["rope_angles", "rope_rotate", "rope_rotate_rows", "s2_rope_attention_fwd", "s2_rope_attention_bwd",
+           "s2_rope_unit"]
 
 
 def rope_angles(N: int, D: int, pos_scale: float, base: float = 10000.0) -> np.ndarray:
@@ -56,6 +57,54 @@ def rope_rotate(x, pos_scale: float, base: float = 10000.0, inverse: bool = Fals
     s = np.sin(a)[None, :, None, :]
     x1, x2 = x[..., : D // 2], x[..., D // 2:]
     return np.concatenate([x1 * c - x2 * s, x1 * s + x2 * c], axis=-1)
+
+
+def rope_rotate_rows(x, t, pos_scale: float, base: float = 10000.0, inverse: bool = False) -> np.ndarray:
+    """The same rotation for rows x [n, D] at token positions t [n] (for
+    sampling single units of long sequences)."""
+    x = np.asarray(x, dtype=np.float64)
+    D = x.shape[-1]
+    i = np.arange(D // 2, dtype=np.float64)
+    a = (np.asarray(t, dtype=np.float64) * pos_scale)[:, None] * (base ** (-2.0 * i / D))[None, :]
+    if inverse:
+        a = -a
+    c, s = np.cos(a), np.sin(a)
+    x1, x2 = x[:, : D // 2], x[:, D // 2:]
+    return np.concatenate([x1 * c - x2 * s, x1 * s + x2 * c], axis=-1)
+
+
+def s2_rope_unit(q, k, v, do, G: int, b: int, h: int, g: int, pos_scale: float, base: float = 10000.0,
+                 piece: str = "whole", m: int | None = None):
+    """One (batch b, query head h, rolled group g) unit of S2 attention on
+    rotated q and k, at original positions.  piece = "whole" (every row of the
+    group), "prefix" or "suffix" (its first / last m rows, as s2_unit_prefix /
+    s2_unit_suffix).  dq and this head's dk_part are rotated back (gradients
+    with respect to the unrotated q and k); o, lse, dv_part as in s2_ref."""
+    from .s2_ref import group_causal_attention, group_causal_attention_grad, group_prefix_attention, \
+        group_suffix_attention, kv_head_of, shift_of_head
+    B, N, H, D = q.shape
+    Hkv = k.shape[2]
+    scale = 1.0 / np.sqrt(D)
+    s = shift_of_head(h, H, N, G)
+    kh = kv_head_of(h, H, Hkv)
+    rows = (np.arange(g * G, (g + 1) * G) + s) % N
+    qg = rope_rotate_rows(q[b, rows, h], rows, pos_scale, base)
+    kg = rope_rotate_rows(k[b, rows, kh], rows, pos_scale, base)
+    vg = np.asarray(v[b, rows, kh], dtype=np.float64)
+    dog = np.asarray(do[b, rows, h], dtype=np.float64)
+    if piece == "whole":
+        og, lse, _ = group_causal_attention(qg, kg, vg, scale)
+        dq, dk, dv, _ = group_causal_attention_grad(qg, kg, vg, dog, scale)
+        r = rows
+    elif piece == "prefix":
+        og, lse, dq, dk, dv, _ = group_prefix_attention(qg, kg, vg, dog, m, scale)
+        r = rows[:m]
+    else:
+        og, lse, dq, dk, dv, _ = group_suffix_attention(qg, kg, vg, dog, G - m, scale)
+        r = rows[G - m:]
+    return {"rows": r, "o": og, "lse": lse, "kv_head": kh,
+            "dq": rope_rotate_rows(dq, r, pos_scale, base, inverse=True),
+            "dk_part": rope_rotate_rows(dk, r, pos_scale, base, inverse=True), "dv_part": dv}
 
 
 def s2_rope_attention_fwd(q, k, v, G: int, pos_scale: float, base: float = 10000.0):

@@ -135,3 +135,29 @@ def test_planted_mistakes_fail(monkeypatch):
            - np.sum(rr.s2_rope_attention_fwd(qm, k, v, 8, 0.5, 100.0)[0] * w)) / (2 * eps)
     assert abs(num - dq_good[0, 5, 1, 2]) < 1e-6
     assert abs(num - dq_bad[0, 5, 1, 2]) > 1e-4
+
+
+def test_rows_and_unit_match_whole_tensor():
+    """The row-sampling forms equal the whole-tensor oracle on their rows."""
+    import oracle.s2_ref as ref
+    B, N, G, H, Hkv, D = 1, 64, 32, 4, 2, 6
+    q, k, v, do = _rand((B, N, H, D), 20), _rand((B, N, Hkv, D), 21), _rand((B, N, Hkv, D), 22), _rand((B, N, H, D), 23)
+    rows = np.array([5, 63, 0, 17])
+    np.testing.assert_allclose(rr.rope_rotate_rows(q[0, rows, 1], rows, 0.5, 100.0),
+                               rr.rope_rotate(q, 0.5, 100.0)[0, rows, 1], rtol=0, atol=1e-13)
+    o, lse, _, _ = rr.s2_rope_attention_fwd(q, k, v, G, 0.5, 100.0)
+    dq, dk, dv = rr.s2_rope_attention_bwd(q, k, v, do, G, 0.5, 100.0)
+    for h, g in ((0, 1), (3, 1), (2, 0)):
+        kh = h // (H // Hkv)
+        parts = {}
+        for piece, m in (("whole", None), ("prefix", 12), ("suffix", 12)):
+            u = rr.s2_rope_unit(q, k, v, do, G, 0, h, g, 0.5, 100.0, piece, m)
+            np.testing.assert_allclose(u["o"], o[0, u["rows"], h], atol=1e-12, rtol=0)
+            np.testing.assert_allclose(u["lse"], lse[0, h, u["rows"]], atol=1e-12, rtol=0)
+            np.testing.assert_allclose(u["dq"], dq[0, u["rows"], h], atol=1e-12, rtol=0)
+            parts[piece] = u
+        # the kv-head's dk / dv are the sums of its query heads' parts
+        h2 = kh * (H // Hkv) + (1 - h % 2)
+        u2 = rr.s2_rope_unit(q, k, v, do, G, 0, h2, g, 0.5, 100.0)
+        np.testing.assert_allclose(parts["whole"]["dk_part"] + u2["dk_part"], dk[0, u2["rows"], kh], atol=1e-12, rtol=0)
+        np.testing.assert_allclose(parts["whole"]["dv_part"] + u2["dv_part"], dv[0, u2["rows"], kh], atol=1e-12, rtol=0)
