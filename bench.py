@@ -37,7 +37,8 @@ if ROOT not in sys.path:
 from sparse_attention_attn_b200 import inputs as I  # noqa: E402
 
 METRIC = "S2-Attn fwd+bwd TFLOP/s & tokens/s on 1 B200; % of BF16 tensor peak"
-KERNEL_NAMES = {0: "s2_fwd_kernel", 1: "s2_bwd_pre_kernel", 2: "s2_bwd_dkdv_kernel", 3: "s2_bwd_dq_kernel"}
+KERNEL_NAMES = {0: "s2_fwd_kernel", 1: "s2_bwd_pre_kernel", 2: "s2_bwd_dkdv_kernel", 3: "s2_bwd_dq_kernel",
+                4: "s2_bwd_fused_kernel", 5: "s2_bwd_dq_post_kernel", 6: "s2_rope_apply_kernel"}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -46,16 +47,20 @@ def effective_flops(s: I.Shape):
     return fwd, 2.5 * fwd
 
 
-def kernel_algorithmic(s: I.Shape):
+def kernel_algorithmic(s: I.Shape, fused: bool = False):
     """Per-launch algorithmic work of each kernel.  The UMMA kernels are
     credited the GEMMs they must issue on the causal half of every group
-    (2*B*H*N*G*D/2 FLOPs per GEMM): forward 2 (S, O), dK/dV 4 (S, dP, dV, dK),
-    dQ 3 (S, dP, dQ).  The preprocess moves bytes: O and dO read, Delta and
-    lse*log2(e) written, lse read."""
+    (2*B*H*N*G*D/2 FLOPs per GEMM): forward 2 (S, O); split backward dK/dV 4
+    (S, dP, dV, dK) and dQ 3 (S, dP, dQ); fused backward 5 (S, dP, dV, dK, dQ).
+    The preprocess moves bytes: O and dO read, Delta and lse*log2(e) written,
+    lse read, and on the fused path the fp32 dq accumulator zeroed; the dq
+    conversion reads the accumulator and writes bf16 dq."""
     gemm = 2.0 * s.B * s.H * s.N * s.G * s.D * 0.5
     rows = s.B * s.H * s.N
-    return {0: ("tensor", 2 * gemm), 2: ("tensor", 4 * gemm), 3: ("tensor", 3 * gemm),
-            1: ("hbm", 2.0 * rows * s.D * 2 + rows * 4 * 3)}
+    acc = rows * s.D * 4.0
+    return {0: ("tensor", 2 * gemm), 2: ("tensor", 4 * gemm), 3: ("tensor", 3 * gemm), 4: ("tensor", 5 * gemm),
+            1: ("hbm", 2.0 * rows * s.D * 2 + rows * 4 * 3 + (acc if fused else 0.0)),
+            5: ("hbm", acc + rows * s.D * 2.0)}
 
 
 def load_peaks():
@@ -310,7 +315,7 @@ def run_ours(args, shape, world, rank, local):
     gpu_launches = launches[0]
     # Per-kernel times: a second loop of the same steps with one CUDA-event pair
     # around each launch (on the launching stream).
-    cap = 8 * args.steps + 8
+    cap = 4 * args.steps + 8
     assert _lib.s2attn_profile_start(cap) == 0
     for _ in range(args.steps):
         step()
@@ -403,7 +408,7 @@ def run_ours(args, shape, world, rank, local):
     tflops = total_flops / (ms_step * 1e-3) / 1e12
     tokens = shape.B * shape.N * world / (ms_step * 1e-3)
     peaks, peak_src = load_peaks()
-    alg = kernel_algorithmic(shape)
+    alg = kernel_algorithmic(shape, fused=4 in per_kernel)
     kern = {}
     for kid, times in per_kernel.items():
         avg = sum(times) / len(times)
@@ -445,6 +450,8 @@ def run_ours(args, shape, world, rank, local):
     }
     if not args.no_dense_ratio and rank == 0 and shape.G < shape.N:
         line["dense_comparison"] = dense_ratio(shape, dev, args)
+    if not args.no_rope and rank == 0 and world == 1:
+        line["rope"] = rope_step(shape, dev, peaks, ms_step)
     if not args.no_extra_workloads and world == 1:
         line["other_workloads"] = {s.name: other_workload(s, dev, peaks)
                                    for s in I.WORKLOADS if s.name in args.extra_workloads.split(",")}
@@ -485,6 +492,61 @@ def dense_ratio(shape: I.Shape, dev, args):
     return {"s2_ms": t_s2, "dense_ms": t_dense, "speedup": t_dense / t_s2}
 
 
+def rope_step(shape: I.Shape, dev, peaks, ms_plain: float, steps: int = 10, warmup: int = 3):
+    """The same step with RoPE + Position Interpolation (from 4096 tokens)
+    before S2 attention: s2attn_fwd_rope (rotation passes for q and k, then the
+    forward) and s2attn_bwd_rope (back-rotation fused into the dq conversion
+    and the dK epilogue on the fused path).  Reports its time beside the plain
+    step's and the rotation pass against the HBM bandwidth (bytes: read and
+    write q and k; the table is L2-resident)."""
+    import sparse_attention_attn_b200 as s2
+    from sparse_attention_attn_b200 import _lib
+    q, k, v, do = (t.to(dev) for t in I.make_inputs(shape))
+    tab = s2.rope_table(shape.N, shape.D, min(1.0, 4096 / shape.N))
+    o = torch.empty_like(q)
+    lse = torch.empty((shape.B, shape.H, shape.N), dtype=torch.float32, device=dev)
+    qr, kr = torch.empty_like(q), torch.empty_like(k)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(s2.bwd_workspace_bytes(shape.B, shape.H, shape.Hkv, shape.N, shape.D, shape.G),
+                     dtype=torch.uint8, device=dev)
+
+    def step():
+        s2.s2attn_forward_rope(q, k, v, shape.G, tab, out=o, lse=lse, q_rot=qr, k_rot=kr)
+        s2.s2attn_backward_rope(qr, kr, v, o, lse, do, shape.G, tab, dq=dq, dk=dk, dv=dv, workspace=ws)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        step()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    cap = 8 * steps + 8
+    assert _lib.s2attn_profile_start(cap) == 0
+    for _ in range(steps):
+        step()
+    ms_arr, id_arr = (ctypes.c_float * cap)(), (ctypes.c_int * cap)()
+    n = _lib.s2attn_profile_stop(ctypes.addressof(ms_arr), ctypes.addressof(id_arr), cap)
+    if s2.device_status() != 0 or s2.device_status(ws) != 0:
+        raise RuntimeError("device status reports a timeout in the RoPE step")
+    rot = [ms_arr[i] for i in range(max(n, 0)) if id_arr[i] == 6]
+    rot_bytes = 2.0 * (q.numel() + k.numel()) * 2 / 2  # per launch on average: q (H heads) or k (Hkv heads), read + write
+    avg = sum(rot) / len(rot) if rot else None
+    fwd, bwd = effective_flops(shape)
+    out = {"ms_per_step": ms, "plain_ms_per_step": ms_plain, "overhead_ms": ms - ms_plain,
+           "value": (fwd + bwd) / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+           "pos_scale": min(1.0, 4096 / shape.N), "rope_base": 10000.0}
+    if avg:
+        out["rotation_pass"] = {"launches_per_step": len(rot) / steps, "avg_ms": avg,
+                                "achieved": rot_bytes / (avg * 1e-3) / 1e9, "unit": "GB/s",
+                                "frac": rot_bytes / (avg * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                                "bytes_per_launch": rot_bytes}
+    return out
+
+
 def other_workload(shape: I.Shape, dev, peaks, steps: int = 5, warmup: int = 3):
     """ms per fwd+bwd step and fraction of the bf16 peak on another workload
     shape (a few steps; CUDA events on the launching stream)."""
@@ -518,6 +580,76 @@ def other_workload(shape: I.Shape, dev, peaks, steps: int = 5, warmup: int = 3):
             "tokens_per_s": shape.B * shape.N / (ms * 1e-3), "steps": steps, "warmup": warmup}
 
 
+def sweep_variants(D: int):
+    """Every variant the per-shape plan can select at head dim D, as override
+    strings: forward (work order x K/V ring depth) and backward (path x stages)."""
+    slots = (2, 3, 4) if D == 128 else (4, 6, 8)
+    fwd = [f"fwd_order={o},fwd_kv={s}" for o in ("snake", "pairs") for s in slots]
+    bwd = (["bwd=fused"] if D == 128 else []) + \
+        [f"bwd=split,bwd_stages={s}" for s in ((2, 3) if D == 128 else (3, 4))]
+    return fwd, bwd
+
+
+def run_sweep(args, dev):
+    """Times each selectable variant of the forward and of the backward on
+    every workload shape (CUDA events on the launching stream, a few steps
+    after warm-up) and prints one JSON line per (workload, variant) plus the
+    plan the library selects for each shape."""
+    import sparse_attention_attn_b200 as s2
+    from sparse_attention_attn_b200 import _lib
+    torch.cuda.set_device(dev)
+    props = torch.cuda.get_device_properties(dev)
+    rows = []
+    for shape in I.WORKLOADS:
+        q, k, v, do = (t.to(dev) for t in I.make_inputs(shape))
+        o = torch.empty_like(q)
+        lse = torch.empty((shape.B, shape.H, shape.N), dtype=torch.float32, device=dev)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        steps = 10 if shape.N <= 16384 else 4
+        fwd_specs, bwd_specs = sweep_variants(shape.D)
+        _lib.s2attn_set_tile_override(None)
+        chosen = _lib.s2attn_plan(shape.B, shape.H, shape.Hkv, shape.N, shape.D, shape.G, props.multi_processor_count)
+
+        def timed(fn):
+            for _ in range(3):
+                fn()
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            for _ in range(steps):
+                fn()
+            b.record()
+            torch.cuda.synchronize()
+            return a.elapsed_time(b) / steps
+
+        for kind, specs in (("fwd", fwd_specs), ("bwd", bwd_specs)):
+            for spec in specs:
+                _lib.s2attn_set_tile_override(spec)
+                try:
+                    if kind == "fwd":
+                        ms = timed(lambda: s2.s2attn_forward(q, k, v, shape.G, out=o, lse=lse))
+                    else:
+                        s2.s2attn_forward(q, k, v, shape.G, out=o, lse=lse)
+                        ws = torch.empty(s2.bwd_workspace_bytes(shape.B, shape.H, shape.Hkv, shape.N, shape.D,
+                                                                shape.G), dtype=torch.uint8, device=dev)
+                        ms = timed(lambda: s2.s2attn_backward(q, k, v, o, lse, do, shape.G, dq=dq, dk=dk, dv=dv,
+                                                              workspace=ws))
+                        del ws
+                    if s2.device_status() != 0:
+                        raise RuntimeError(f"device status reports a timeout ({shape.name}, {spec})")
+                finally:
+                    _lib.s2attn_set_tile_override(None)
+                fwd_f, bwd_f = effective_flops(shape)
+                row = {"workload": shape.name, "kernel": kind, "variant": spec, "ms": ms,
+                       "tflops": (fwd_f if kind == "fwd" else bwd_f) / (ms * 1e-3) / 1e12, "steps": steps}
+                rows.append(row)
+                print(json.dumps(row), flush=True)
+        print(json.dumps({"workload": shape.name, "selected_plan": chosen}), flush=True)
+        del q, k, v, do, o, lse, dq, dk, dv
+        torch.cuda.empty_cache()
+    return rows
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -536,12 +668,18 @@ def main():
                     help="skip timing G=N (dense causal) on the same inputs")
     ap.add_argument("--no-extra-workloads", action="store_true",
                     help="skip the few-step timing of the other workload shapes")
+    ap.add_argument("--no-rope", action="store_true", help="skip the step with RoPE + Position Interpolation")
+    ap.add_argument("--sweep", action="store_true",
+                    help="time every selectable kernel variant on every workload shape and exit")
     ap.add_argument("--extra-workloads", default=f"{I.QWEN3_8B_16K.name},{I.LLAMA2_70B_32K.name}",
                     help="comma-separated workload names timed for a few steps beside the headline")
     args = ap.parse_args()
     shape = {s.name: s for s in I.WORKLOADS}[args.workload]
     if args.ref_step_seconds is None:
         args.ref_step_seconds = min(5.0, 120.0 / max(args.steps, 1))
+    if args.sweep:
+        run_sweep(args, torch.device("cuda", 0))
+        return
     world, rank, local = dist_setup()
     try:
         if args.impl == "reference":

@@ -88,7 +88,8 @@ S2ATTN_API int s2attn_fwd(const void* q, const void* k, const void* v, void* o, 
 /*
  * Bytes of device workspace s2attn_bwd needs: a 256-byte device status block,
  * then two fp32 [B, H, N] arrays written by the backward's first kernel:
- * -Delta (Delta_t = sum_d dO_td * O_td) and -lse_t * log2(e).
+ * -Delta (Delta_t = sum_d dO_td * O_td) and -lse_t * log2(e); at head dim 128
+ * (the fused backward) also an fp32 [B, H, N, D] accumulator for dq.
  */
 S2ATTN_API size_t s2attn_bwd_workspace_bytes(int B, int H, int Hkv, int N, int D, int G);
 
@@ -118,16 +119,74 @@ S2ATTN_API int s2attn_device_status(void* workspace, s2attn_stream_t stream);
 /* Static, human-readable name of a status code. */
 S2ATTN_API const char* s2attn_status_string(int status);
 
+/* ------------------------------------------------------------------------
+ * Rotary position embedding with Position Interpolation before S2 attention.
+ * LongQLoRA community post: LLaMA encodes positions with RoPE (section 02);
+ * Position Interpolation shrinks RoPE's rotation angles to extend the context
+ * from 4096 to 8192 tokens (section 04), and S2 attention then runs on the
+ * rotated q and k.  Pair i of a head -- elements i and i + D/2 -- at token t
+ * (original position) turns by  a(t, i) = t * pos_scale * rope_base^(-2i/D):
+ *   y_i = x_i cos a - x_{i+D/2} sin a,   y_{i+D/2} = x_i sin a + x_{i+D/2} cos a.
+ * pos_scale = L_train / L_target (0.5 for 4096 -> 8192; 1 is plain RoPE);
+ * rope_base is the frequency base (10000 for LLaMA2).  v is not rotated.
+ * ------------------------------------------------------------------------ */
+
+/* Bytes of the rotary table for N positions at head dim D (0 if unsupported). */
+S2ATTN_API size_t s2attn_rope_table_bytes(int N, int D);
+
+/*
+ * Fills `table` (device, caller-owned, s2attn_rope_table_bytes bytes, 16-byte
+ * aligned) with fp32 (cos a, sin a) pairs, [N][D/2][2].  The angles are
+ * formed and reduced in fp64 (at 100K tokens they reach ~1e5 radians).  The
+ * table depends only on (N, D, pos_scale, rope_base): build it once and reuse
+ * it across layers and steps.  D in {64, 128}, pos_scale > 0, rope_base > 1.
+ */
+S2ATTN_API int s2attn_rope_table(float* table, int N, int D, double pos_scale, double rope_base,
+                                 s2attn_stream_t stream);
+
+/*
+ * out = x rotated by the table (by the opposite angles when `inverse` != 0,
+ * which is the backward of the rotation).  x, out: bf16 [B, N, heads, D]
+ * device buffers; out == x is allowed (in place).
+ */
+S2ATTN_API int s2attn_rope_apply(const void* x, void* out, const float* table, int B, int N, int heads, int D,
+                                 int inverse, s2attn_stream_t stream);
+
+/*
+ * Forward of S2 attention on rotated inputs: q_rot = rotate(q), k_rot =
+ * rotate(k) (caller buffers shaped like q and k, kept for the backward, not
+ * aliasing q, k or each other), then o, lse = S2Attn(q_rot, k_rot, v) exactly
+ * as s2attn_fwd.  Three launches.
+ */
+S2ATTN_API int s2attn_fwd_rope(const void* q, const void* k, const void* v, void* o, float* lse, void* q_rot,
+                               void* k_rot, const float* table, int B, int H, int Hkv, int N, int D, int G,
+                               s2attn_stream_t stream);
+
+/*
+ * Backward of s2attn_fwd_rope: takes the rotated q_rot, k_rot it produced and
+ * writes the gradients with respect to the UNROTATED q and k (and v):
+ * dq = rotate^-1(dq_rot), dk = rotate^-1(dk_rot).  On the fused backward path
+ * (head dim 128) the back-rotation happens inside the dq conversion and the
+ * dK epilogue; on the split path two in-place rotation passes follow.  The
+ * workspace is that of s2attn_bwd (s2attn_bwd_workspace_bytes).
+ */
+S2ATTN_API int s2attn_bwd_rope(const void* q_rot, const void* k_rot, const void* v, const void* o,
+                               const float* lse, const void* dO, void* dq, void* dk, void* dv, const float* table,
+                               int B, int H, int Hkv, int N, int D, int G, void* workspace, size_t workspace_bytes,
+                               s2attn_stream_t stream);
+
 /*
  * Backward for callers that cannot allocate device memory (no counterpart in
  * the papers: this is a deployment variant of s2attn_bwd).  Some callers have
  * no way to get a workspace: they run under another runtime's memory budget
  * without an allocator handle, inside plugin hosts that forbid cudaMalloc, or
  * must not allocate between set-up and graph capture.  This call computes
- * exactly what s2attn_bwd computes, with the same arguments minus the
- * workspace, and allocates nothing: its scratch (s2attn_bwd_workspace_bytes of
- * it) is a fixed 32 MiB device array inside the library, which every GPU that
- * loads the library holds until the process exits.  That limits it to
+ * the same gradients as s2attn_bwd, with the same arguments minus the
+ * workspace, and allocates nothing.  It runs the split backward (preprocess,
+ * dK/dV kernel, dQ kernel), whose scratch -- status block, Delta and
+ * lse*log2(e), 256 + 2 * round_up(4 * B * H * N, 256) bytes -- is a fixed
+ * 32 MiB device array inside the library, which every GPU that loads the
+ * library holds until the process exits.  That limits it to
  * B * H * N <= 4194272 query rows (all five workload shapes fit); larger
  * shapes return S2ATTN_ERR_WORKSPACE without launching anything.
  *   - The first call on a device looks up the array's device address (with
@@ -177,6 +236,30 @@ S2ATTN_API int s2attn_last_launch_count(void);
  */
 S2ATTN_API int s2attn_profile_start(int max_launches);
 S2ATTN_API int s2attn_profile_stop(float* ms, int* kernel_ids, int capacity);
+
+/*
+ * The per-shape plan the library would use for a call with these arguments on
+ * a device with num_sms SMs (with the override below applied): out[0] forward
+ * work order (1 longest-first snake, 0 equal-work pairs), out[1] forward K/V
+ * ring depth, out[2] backward path (1 fused, 0 split), out[3] split backward
+ * pipeline stages.  Host only; returns a status code (shape validation as in
+ * s2attn_fwd).
+ */
+S2ATTN_API int s2attn_plan(int B, int H, int Hkv, int N, int D, int G, int num_sms, int* out);
+
+/*
+ * Replaces the plan override (initially the S2ATTN_TILE environment
+ * variable) that later calls in this process consult; NULL restores the
+ * environment's value.  The override forces a variant the per-shape selection
+ * would not pick, for tests and sweeps: a comma-separated list of key=value
+ * items; keys bwd=split|fused (backward path; fused exists for head dim 128),
+ * fwd_order=snake|pairs (forward work order), fwd_kv=N (forward K/V ring
+ * depth: 2-4 at head dim 128, 4/6/8 at 64), bwd_stages=N (split backward
+ * stages: 2-3 at head dim 128, 3-4 at 64); values that do not exist for a
+ * call's head dim are ignored.  s2attn_bwd_workspace_bytes answers for the
+ * path in force when it is called.  Returns S2ATTN_OK.
+ */
+S2ATTN_API int s2attn_set_tile_override(const char* spec);
 
 #ifdef __cplusplus
 }

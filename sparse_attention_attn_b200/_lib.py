@@ -35,6 +35,14 @@ SIGNATURES = {
     "s2attn_last_launch_count": (_i, []),
     "s2attn_profile_start": (_i, [_i]),
     "s2attn_profile_stop": (_i, [_vp, _vp, _i]),
+    "s2attn_set_tile_override": (_i, [ctypes.c_char_p]),
+    "s2attn_rope_table_bytes": (ctypes.c_size_t, [_i, _i]),
+    "s2attn_rope_table": (_i, [_vp, _i, _i, ctypes.c_double, ctypes.c_double, _vp]),
+    "s2attn_rope_apply": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
+    "s2attn_fwd_rope": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]),
+    "s2attn_bwd_rope": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp,
+                             ctypes.c_size_t, _vp]),
+    "s2attn_plan": (_i, [_i, _i, _i, _i, _i, _i, _i, _vp]),
     "s2attn_bwd_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
                                 _vp]),
 }
@@ -106,6 +114,41 @@ def s2attn_profile_start(max_launches) -> int:
 
 def s2attn_profile_stop(ms, kernel_ids, capacity) -> int:
     return load().s2attn_profile_stop(ms, kernel_ids, capacity)
+
+
+def s2attn_rope_table_bytes(N, D) -> int:
+    return load().s2attn_rope_table_bytes(N, D)
+
+
+def s2attn_rope_table(table, N, D, pos_scale, rope_base, stream) -> int:
+    return load().s2attn_rope_table(table, N, D, pos_scale, rope_base, stream)
+
+
+def s2attn_rope_apply(x, out, table, B, N, heads, D, inverse, stream) -> int:
+    return load().s2attn_rope_apply(x, out, table, B, N, heads, D, inverse, stream)
+
+
+def s2attn_fwd_rope(q, k, v, o, lse, q_rot, k_rot, table, B, H, Hkv, N, D, G, stream) -> int:
+    return load().s2attn_fwd_rope(q, k, v, o, lse, q_rot, k_rot, table, B, H, Hkv, N, D, G, stream)
+
+
+def s2attn_bwd_rope(q_rot, k_rot, v, o, lse, dO, dq, dk, dv, table, B, H, Hkv, N, D, G, workspace,
+                    workspace_bytes, stream) -> int:
+    return load().s2attn_bwd_rope(q_rot, k_rot, v, o, lse, dO, dq, dk, dv, table, B, H, Hkv, N, D, G, workspace,
+                                  workspace_bytes, stream)
+
+
+def s2attn_plan(B, H, Hkv, N, D, G, num_sms):
+    """The per-shape plan as a dict (host only), or raises on an invalid shape."""
+    out = (ctypes.c_int * 4)()
+    _check("s2attn_plan", load().s2attn_plan(B, H, Hkv, N, D, G, num_sms, ctypes.addressof(out)))
+    return {"fwd_order": "snake" if out[0] else "pairs", "fwd_kv_slots": out[1],
+            "bwd_path": "fused" if out[2] else "split", "bwd_stages": out[3]}
+
+
+def s2attn_set_tile_override(spec) -> int:
+    """Test / sweep hook: force a kernel variant (None restores S2ATTN_TILE)."""
+    return load().s2attn_set_tile_override(None if spec is None else spec.encode())
 
 
 def s2attn_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, B, H, Hkv, N, D, G, stream) -> int:

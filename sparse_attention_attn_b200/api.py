@@ -111,6 +111,110 @@ def device_status(workspace=None) -> int:
     return _lib.s2attn_device_status(ptr, _stream())
 
 
+def rope_table(N: int, D: int, pos_scale: float, rope_base: float = 10000.0, device=None):
+    """fp32 (cos, sin) table [N, D/2, 2] of RoPE with Position Interpolation:
+    pair i at token t turns by t * pos_scale * rope_base^(-2i/D) (LongQLoRA
+    post section 04: Position Interpolation shrinks RoPE's angles; pos_scale =
+    L_train / L_target).  Built on the GPU; reuse it across layers and steps."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    nbytes = _lib.s2attn_rope_table_bytes(N, D)
+    if nbytes == 0:
+        raise _lib.S2AttnError("s2attn_rope_table_bytes", _lib.S2ATTN_ERR_UNSUPPORTED)
+    table = torch.empty((N, D // 2, 2), dtype=torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        st = _lib.s2attn_rope_table(table.data_ptr(), N, D, float(pos_scale), float(rope_base), _stream(dev))
+    _lib._check("s2attn_rope_table", st)
+    return table
+
+
+def rope_apply(x, table, inverse: bool = False, out=None):
+    """x [B, N, heads, D] bf16 rotated by the table (the opposite way when
+    `inverse`); out may be x (in place)."""
+    B, N, Hx, D = x.shape
+    _need("x", x, (B, N, Hx, D))
+    _need("table", table, (N, D // 2, 2), torch.float32, device=x.device)
+    out = torch.empty_like(x) if out is None else out
+    _need("out", out, (B, N, Hx, D), device=x.device)
+    with torch.cuda.device(x.device):
+        st = _lib.s2attn_rope_apply(x.data_ptr(), out.data_ptr(), table.data_ptr(), B, N, Hx, D, int(inverse),
+                                    _stream(x.device))
+    _lib._check("s2attn_rope_apply", st)
+    return out
+
+
+def s2attn_forward_rope(q, k, v, group_size: int, table, out=None, lse=None, q_rot=None, k_rot=None):
+    """S2 attention on RoPE-rotated q and k.  Returns (o, lse, q_rot, k_rot);
+    q_rot and k_rot are what the backward takes."""
+    B, N, H, Hkv, D = _dims(q, k)
+    _need("q", q, (B, N, H, D))
+    dev = q.device
+    _need("k", k, (B, N, Hkv, D), device=dev)
+    _need("v", v, (B, N, Hkv, D), device=dev)
+    _need("table", table, (N, D // 2, 2), torch.float32, device=dev)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev) if lse is None else lse
+    q_rot = torch.empty_like(q) if q_rot is None else q_rot
+    k_rot = torch.empty_like(k) if k_rot is None else k_rot
+    _need("out", out, (B, N, H, D), device=dev)
+    _need("lse", lse, (B, H, N), torch.float32, device=dev)
+    _need("q_rot", q_rot, (B, N, H, D), device=dev)
+    _need("k_rot", k_rot, (B, N, Hkv, D), device=dev)
+    with torch.cuda.device(dev):
+        st = _lib.s2attn_fwd_rope(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                  q_rot.data_ptr(), k_rot.data_ptr(), table.data_ptr(), B, H, Hkv, N, D,
+                                  int(group_size), _stream(dev))
+    _lib._check("s2attn_fwd_rope", st)
+    return out, lse, q_rot, k_rot
+
+
+def s2attn_backward_rope(q_rot, k_rot, v, o, lse, do, group_size: int, table, dq=None, dk=None, dv=None,
+                         workspace=None):
+    """Backward of s2attn_forward_rope: gradients with respect to the
+    unrotated q and k, and v.  Returns (dq, dk, dv)."""
+    B, N, H, Hkv, D = _dims(q_rot, k_rot)
+    _need("q_rot", q_rot, (B, N, H, D))
+    dev = q_rot.device
+    for name, t, shp in (("k_rot", k_rot, (B, N, Hkv, D)), ("v", v, (B, N, Hkv, D)),
+                         ("o", o, (B, N, H, D)), ("do", do, (B, N, H, D))):
+        _need(name, t, shp, device=dev)
+    _need("lse", lse, (B, H, N), torch.float32, device=dev)
+    _need("table", table, (N, D // 2, 2), torch.float32, device=dev)
+    dq = torch.empty_like(q_rot) if dq is None else dq
+    dk = torch.empty_like(k_rot) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    for name, t, shp in (("dq", dq, (B, N, H, D)), ("dk", dk, (B, N, Hkv, D)), ("dv", dv, (B, N, Hkv, D))):
+        _need(name, t, shp, device=dev)
+    wsb = bwd_workspace_bytes(B, H, Hkv, N, D, group_size)
+    if workspace is None:
+        workspace = torch.empty(wsb, dtype=torch.uint8, device=dev)
+    if workspace.numel() * workspace.element_size() < wsb:
+        raise _lib.S2AttnError("s2attn_bwd_rope", _lib.S2ATTN_ERR_WORKSPACE)
+    with torch.cuda.device(dev):
+        st = _lib.s2attn_bwd_rope(q_rot.data_ptr(), k_rot.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                  do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), table.data_ptr(),
+                                  B, H, Hkv, N, D, int(group_size), workspace.data_ptr(),
+                                  workspace.numel() * workspace.element_size(), _stream(dev))
+    _lib._check("s2attn_bwd_rope", st)
+    return dq, dk, dv
+
+
+class S2RopeAttention(torch.autograd.Function):
+    """Autograd wrapper: RoPE with Position Interpolation, then S2 attention."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, group_size, table):
+        o, lse, q_rot, k_rot = s2attn_forward_rope(q, k, v, group_size, table)
+        ctx.save_for_backward(q_rot, k_rot, v, o, lse, table)
+        ctx.group_size = group_size
+        return o
+
+    @staticmethod
+    def backward(ctx, do):
+        q_rot, k_rot, v, o, lse, table = ctx.saved_tensors
+        dq, dk, dv = s2attn_backward_rope(q_rot, k_rot, v, o, lse, do.contiguous(), ctx.group_size, table)
+        return dq, dk, dv, None, None
+
+
 class S2Attention(torch.autograd.Function):
     """Autograd wrapper: the drop-in attention call of a training step."""
 

@@ -94,6 +94,12 @@ __global__ void __launch_bounds__(256) s2_bwd_pre_kernel(const BwdPreArgs a) {
       for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
       if (part == 0) red[st * RPS + rsub] = acc;
     }
+    if (a.dqacc != nullptr) {
+      // the fused backward reduces dQ partials into these 128 rows: start at zero
+      float4* z = reinterpret_cast<float4*>(a.dqacc + (static_cast<size_t>(bh) * d.N + t0) * D);
+#pragma unroll
+      for (int i = 0; i < kTile * D / 4 / 256; ++i) z[tid + i * 256] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
     __syncthreads();
     if (tid < kTile) {
       const size_t idx = static_cast<size_t>(bh) * d.N + t0 + tid;
@@ -101,30 +107,6 @@ __global__ void __launch_bounds__(256) s2_bwd_pre_kernel(const BwdPreArgs a) {
       a.nlse2[idx] = -a.lse[idx] * kLog2e;
     }
     __syncthreads();
-  }
-}
-
-// 32 fp32 values (bit patterns) times `scale` -> 32 bf16 at dst (64 bytes, 16-byte aligned).
-__device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const uint32_t (&r)[32], float scale) {
-  uint4* out = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-  for (int q = 0; q < 4; ++q)
-    out[q] = make_uint4(pack_bf16x2(__uint_as_float(r[8 * q]) * scale, __uint_as_float(r[8 * q + 1]) * scale),
-                        pack_bf16x2(__uint_as_float(r[8 * q + 2]) * scale, __uint_as_float(r[8 * q + 3]) * scale),
-                        pack_bf16x2(__uint_as_float(r[8 * q + 4]) * scale, __uint_as_float(r[8 * q + 5]) * scale),
-                        pack_bf16x2(__uint_as_float(r[8 * q + 6]) * scale, __uint_as_float(r[8 * q + 7]) * scale));
-}
-
-
-// The same as two 32-byte stores (whole DRAM sectors); dst 32-byte aligned.
-__device__ __forceinline__ void store_row32_v8(__nv_bfloat16* dst, const uint32_t (&r)[32], float scale) {
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    uint32_t v[8];
-#pragma unroll
-    for (int q = 0; q < 8; ++q)
-      v[q] = pack_bf16x2(__uint_as_float(r[16 * h + 2 * q]) * scale, __uint_as_float(r[16 * h + 2 * q + 1]) * scale);
-    st_global_v8(dst + 16 * h, v);
   }
 }
 
@@ -141,16 +123,14 @@ __device__ __forceinline__ void store_row32_v8(__nv_bfloat16* dst, const uint32_
 // dV/dK are read out by the epilogue of an item before the next item's first
 // gradient UMMA overwrites them (acc_full / acc_free handshake).
 
-constexpr int kSub = 64;  // rows of a streamed sub-tile
-
 // A-operand column of k-step kk (16 rows of K) when a 64-wide bf16 operand was
 // written by two warp halves at packed columns [0,16) and [32,48) of its
 // 64-column TMEM buffer (each half stays inside the fp32 columns it read).
 __device__ __forceinline__ uint32_t split_acol64(int kk) { return kk * 8 + (kk >= 2 ? 16 : 0); }
 
-template <int D>
+template <int D, int NST>
 struct DkvCfg {
-  static constexpr int STAGES = 3;
+  static constexpr int STAGES = NST;
   // warps: 0 producer, 1 UMMA issuer A, 2..9 elementwise + epilogue, 10 UMMA issuer B
   static constexpr int KV_ATOM = kTile * 128;  // one 64-column slab of a 128-row tile
   static constexpr int Q_ATOM = kSub * 128;    // one 64-column slab of a 64-row tile
@@ -165,35 +145,12 @@ struct DkvCfg {
   static constexpr int THREADS = 352;
 };
 
-// Sub-tile cursor of the dK/dV kernel: item (kv tile) plus sub-tile index.
-struct DkvCursor {
-  ItemCursor ic;
-  TileWork w;
-  int it, iters, nq;
-  __device__ __forceinline__ void load(const Dims& d, const PairSched& ps) {
-    if (!ic.valid) return;
-    w = kv_item(d, ic.unit, ic.tile);
-    nq = 2 * (d.tiles - w.tile);  // 64-row query sub-tiles from the diagonal to the group end
-    iters = d.rep * nq;
-    it = 0;
-  }
-  __device__ __forceinline__ void first(const Dims& d, const PairSched& ps) {
-    ic.first(ps);
-    load(d, ps);
-  }
-  __device__ __forceinline__ void next(const Dims& d, const PairSched& ps) {
-    if (++it < iters) return;
-    ic.next(ps);
-    load(d, ps);
-  }
-};
-
-template <int D>
+template <int D, int NST>
 __global__ void __launch_bounds__(352, 1)
     s2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmG,
                        const BwdArgs a) {
-  using C = DkvCfg<D>;
+  using C = DkvCfg<D, NST>;
   constexpr int ST = C::STAGES;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -523,9 +480,9 @@ __global__ void __launch_bounds__(352, 1)
 // Q [256+D, 256+3D/2), dO [256+3D/2, 256+2D) (bf16 pairs); dQ is read out by
 // the item's epilogue before the next item overwrites it.
 
-template <int D>
+template <int D, int NST>
 struct DqCfg {
-  static constexpr int STAGES = 3;
+  static constexpr int STAGES = NST;
   static constexpr int Q_ATOM = kTile * 128;
   static constexpr int KV_ATOM = kSub * 128;
   static constexpr int Q_BYTES = kTile * D * 2;
@@ -539,6 +496,7 @@ struct DqCfg {
   static constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DQ = 256;
   static constexpr uint32_t TM_QT = 256 + D, TM_GT = 256 + D + D / 2;  // Q, dO as UMMA A operands
   static constexpr int THREADS = 384;
+  static_assert(SMEM_BYTES <= 232448 - 512, "shared memory");
 };
 
 struct DqCursor {
@@ -562,12 +520,12 @@ struct DqCursor {
   }
 };
 
-template <int D>
+template <int D, int NST>
 __global__ void __launch_bounds__(384, 1)
     s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmG,
                      const BwdArgs a) {
-  using C = DqCfg<D>;
+  using C = DqCfg<D, NST>;
   constexpr int ST = C::STAGES;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -906,40 +864,69 @@ static bool set_smem_attr(const void* fn, int bytes) {
   return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
 }
 
-// Tensor maps: `*128` have 128-row boxes, `*64` 64-row boxes.  dK/dV streams
-// 64-row query sub-tiles against 128-row kv tiles; dQ the other way round.
+// The preprocess: one block per 128-row task of one (batch, head), at most
+// eight blocks per SM.
 template <int D>
-cudaError_t launch_bwd(const BwdMaps& m, const BwdPreArgs& pre, const BwdArgs& a, int num_sms,
-                       cudaStream_t stream, int* launches) {
-  using K3 = DkvCfg<D>;
-  using K4 = DqCfg<D>;
-  if (!set_smem_attr(reinterpret_cast<const void*>(s2_bwd_dkdv_kernel<D>), K3::SMEM_BYTES) ||
-      !set_smem_attr(reinterpret_cast<const void*>(s2_bwd_dq_kernel<D>), K4::SMEM_BYTES))
-    return cudaErrorInvalidValue;
-  const long long rows = static_cast<long long>(a.d.B) * a.d.N * a.d.H;
+cudaError_t launch_bwd_pre(const BwdPreArgs& pre, int num_sms, cudaStream_t stream) {
+  const long long rows = static_cast<long long>(pre.d.B) * pre.d.N * pre.d.H;
   const long long tasks = rows / kTile;  // 128-row tasks of one (batch, head)
   const int pre_grid = static_cast<int>(tasks < 8LL * num_sms ? tasks : 8LL * num_sms);
   prof_before(stream, kKernelBwdPre);
   s2_bwd_pre_kernel<D><<<pre_grid, 256, 0, stream>>>(pre);
   cudaError_t e = cudaGetLastError();
   prof_after(stream);
+  return e;
+}
+template cudaError_t launch_bwd_pre<64>(const BwdPreArgs&, int, cudaStream_t);
+template cudaError_t launch_bwd_pre<128>(const BwdPreArgs&, int, cudaStream_t);
+
+// Tensor maps: `*128` have 128-row boxes, `*64` 64-row boxes.  dK/dV streams
+// 64-row query sub-tiles against 128-row kv tiles; dQ the other way round.
+// NST: pipeline stages of both kernels' streamed operands.
+template <int D, int NST>
+cudaError_t launch_bwd_stages(const BwdMaps& m, const BwdPreArgs& pre, const BwdArgs& a, int num_sms,
+                              cudaStream_t stream, int* launches) {
+  using K3 = DkvCfg<D, NST>;
+  using K4 = DqCfg<D, NST>;
+  if (!set_smem_attr(reinterpret_cast<const void*>(s2_bwd_dkdv_kernel<D, NST>), K3::SMEM_BYTES) ||
+      !set_smem_attr(reinterpret_cast<const void*>(s2_bwd_dq_kernel<D, NST>), K4::SMEM_BYTES))
+    return cudaErrorInvalidValue;
+  cudaError_t e = launch_bwd_pre<D>(pre, num_sms, stream);
   if (e != cudaSuccess) return e;
   const int grid_kv = a.kv_sched.pairs < num_sms ? a.kv_sched.pairs : num_sms;
   prof_before(stream, kKernelBwdDkDv);
-  s2_bwd_dkdv_kernel<D><<<grid_kv, K3::THREADS, K3::SMEM_BYTES, stream>>>(m.q64, m.k128, m.v128, m.g64, a);
+  s2_bwd_dkdv_kernel<D, NST><<<grid_kv, K3::THREADS, K3::SMEM_BYTES, stream>>>(m.q64, m.k128, m.v128, m.g64, a);
   e = cudaGetLastError();
   prof_after(stream);
   if (e != cudaSuccess) return e;
   const int grid_q = a.q_sched.pairs < num_sms ? a.q_sched.pairs : num_sms;
   prof_before(stream, kKernelBwdDq);
-  s2_bwd_dq_kernel<D><<<grid_q, K4::THREADS, K4::SMEM_BYTES, stream>>>(m.q128, m.k64, m.v64, m.g128, a);
+  s2_bwd_dq_kernel<D, NST><<<grid_q, K4::THREADS, K4::SMEM_BYTES, stream>>>(m.q128, m.k64, m.v64, m.g128, a);
   e = cudaGetLastError();
   prof_after(stream);
   if (launches) *launches = 3;
   return e;
 }
 
-template cudaError_t launch_bwd<64>(const BwdMaps&, const BwdPreArgs&, const BwdArgs&, int, cudaStream_t, int*);
-template cudaError_t launch_bwd<128>(const BwdMaps&, const BwdPreArgs&, const BwdArgs&, int, cudaStream_t, int*);
+// stages: 2 or 3 at head dim 128, 3 or 4 at head dim 64 (what fits in shared
+// memory); anything else is an invalid value.
+template <int D>
+cudaError_t launch_bwd(const BwdMaps& m, const BwdPreArgs& pre, const BwdArgs& a, int num_sms,
+                       cudaStream_t stream, int* launches, int stages) {
+  if constexpr (D == 128) {
+    if (stages == 2) return launch_bwd_stages<D, 2>(m, pre, a, num_sms, stream, launches);
+    if (stages == 3) return launch_bwd_stages<D, 3>(m, pre, a, num_sms, stream, launches);
+    return cudaErrorInvalidValue;
+  } else {
+    if (stages == 3) return launch_bwd_stages<D, 3>(m, pre, a, num_sms, stream, launches);
+    if (stages == 4) return launch_bwd_stages<D, 4>(m, pre, a, num_sms, stream, launches);
+    return cudaErrorInvalidValue;
+  }
+}
+
+template cudaError_t launch_bwd<64>(const BwdMaps&, const BwdPreArgs&, const BwdArgs&, int, cudaStream_t, int*,
+                                    int);
+template cudaError_t launch_bwd<128>(const BwdMaps&, const BwdPreArgs&, const BwdArgs&, int, cudaStream_t, int*,
+                                     int);
 
 }  // namespace s2

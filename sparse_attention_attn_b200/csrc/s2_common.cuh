@@ -18,6 +18,7 @@
 namespace s2 {
 
 constexpr int kTile = 128;  // rows of every q / kv tile
+constexpr int kSub = 64;    // rows of a streamed backward sub-tile
 
 struct Dims {
   int B, H, Hkv, N, D, G;
@@ -127,6 +128,29 @@ __host__ __device__ __forceinline__ TileWork q_item(const Dims& d, int unit, int
   w.h = w.kvh * d.rep + hr;
   return w;
 }
+
+// Sub-tile cursor of the dK/dV kernel: item (kv tile) plus sub-tile index.
+struct DkvCursor {
+  ItemCursor ic;
+  TileWork w;
+  int it, iters, nq;
+  __device__ __forceinline__ void load(const Dims& d, const PairSched& ps) {
+    if (!ic.valid) return;
+    w = kv_item(d, ic.unit, ic.tile);
+    nq = 2 * (d.tiles - w.tile);  // 64-row query sub-tiles from the diagonal to the group end
+    iters = d.rep * nq;
+    it = 0;
+  }
+  __device__ __forceinline__ void first(const Dims& d, const PairSched& ps) {
+    ic.first(ps);
+    load(d, ps);
+  }
+  __device__ __forceinline__ void next(const Dims& d, const PairSched& ps) {
+    if (++it < iters) return;
+    ic.next(ps);
+    load(d, ps);
+  }
+};
 
 // Forward schedule.  A forward item is a pair of adjacent query tiles
 // (2i, 2i+1) of one unit (a rolled group of one (batch, head)): every K/V tile
@@ -238,6 +262,7 @@ struct BwdPreArgs {
   const float* lse;        // fp32 [B, H, N]
   float* ndelta;           // fp32 [B, H, N]: -Delta = -sum_d dO * O
   float* nlse2;            // fp32 [B, H, N]: -lse * log2(e)
+  float* dqacc;            // fp32 [B, H, N, D] dQ accumulator zeroed here, or null (split path)
   uint32_t* status;        // device status words, cleared here (first kernel of the call)
 };
 
@@ -250,9 +275,12 @@ struct BwdArgs {
   const float* ndelta;     // fp32 [B, H, N]: -Delta
   const float* nlse2;      // fp32 [B, H, N]: -lse * log2(e)
   void* dq;                // bf16 [B, N, H, D]
+  float* dqacc;            // fused path: fp32 [B, H, N, D] dQ accumulator (zeroed by the preprocess)
   void* dk;                // bf16 [B, N, Hkv, D]
   void* dv;                // bf16 [B, N, Hkv, D]
   int kv_v8;               // dk and dv are 32-byte aligned: whole-sector stores
+  const float* rope;       // fused path: fp32 (cos, sin) [N][D/2][2] table to rotate dq and dk back
+                           // (the inputs were rotated by it), or null
   uint32_t* status;
   unsigned long long wait_limit_ns;
 };
@@ -263,9 +291,20 @@ struct BwdMaps {
   CUtensorMap q64, k64, v64, g64;
 };
 
+template <int D>
+cudaError_t launch_bwd_pre(const BwdPreArgs& pre, int num_sms, cudaStream_t stream);
+
 // Optional per-kernel timing (s2attn_profile_start / _stop): the launchers
 // bracket every kernel with these; they do nothing unless profiling is on.
-enum KernelId : int { kKernelFwd = 0, kKernelBwdPre = 1, kKernelBwdDkDv = 2, kKernelBwdDq = 3 };
+enum KernelId : int {
+  kKernelFwd = 0,
+  kKernelBwdPre = 1,
+  kKernelBwdDkDv = 2,
+  kKernelBwdDq = 3,
+  kKernelBwdFused = 4,
+  kKernelBwdDqPost = 5,
+  kKernelRope = 6
+};
 void prof_before(cudaStream_t stream, int kernel_id);
 void prof_after(cudaStream_t stream);
 

@@ -38,17 +38,20 @@
 
 namespace s2 {
 
-template <int D>
+// KVS: slots of the K/V ring (K and V tiles share it: K0 V0 K1 V1 ...), the
+// pipeline depth the per-shape plan selects (2-4 at head dim 128, 4-8 at 64).
+template <int D, int KVS>
 struct FwdCfg {
   static constexpr int BM = kTile, BN = kTile;
   static constexpr int QSLOTS = 3;                  // Q ring: two tiles per item, one ahead
-  static constexpr int KVSLOTS = (D == 64) ? 8 : 4;  // K and V tiles share one ring: K0 V0 K1 V1 ...
+  static constexpr int KVSLOTS = KVS;
   static constexpr int ATOM_BYTES = kTile * 128;    // one 64-column slab of a 128-row tile
   static constexpr int TILE_BYTES = kTile * D * 2;  // one 128-row tile of Q, K or V
   static constexpr int OFF_KV = QSLOTS * TILE_BYTES;
   static constexpr int SMEM_BYTES = OFF_KV + KVSLOTS * TILE_BYTES + 1024;  // + alignment slack
   static constexpr uint32_t TM_O = 256;
   static constexpr int THREADS = 320;
+  static_assert(SMEM_BYTES <= 232448 - 512, "shared memory");
 };
 
 // P for 64 scores of one query row: p = 2^(s * sl2 - m), packed to bf16
@@ -71,12 +74,12 @@ __device__ __forceinline__ float softmax_row64(const uint32_t (&s0)[32], const u
   return f2_lo(s) + f2_hi(s);
 }
 
-template <int D>
+template <int D, int KVS>
 __global__ void __launch_bounds__(320, 1)
     s2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                   const FwdArgs a) {
-  using C = FwdCfg<D>;
+  using C = FwdCfg<D, KVS>;
   constexpr int NQ = C::QSLOTS, NS = C::KVSLOTS;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -498,24 +501,47 @@ __global__ void __launch_bounds__(320, 1)
   }
 }
 
-template <int D>
-cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const CUtensorMap& to, const FwdArgs& a, int num_sms, cudaStream_t stream) {
-  using C = FwdCfg<D>;
-  cudaError_t ea = cudaFuncSetAttribute(s2_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+template <int D, int KVS>
+cudaError_t launch_fwd_slots(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                             const CUtensorMap& to, const FwdArgs& a, int num_sms, cudaStream_t stream) {
+  using C = FwdCfg<D, KVS>;
+  cudaError_t ea = cudaFuncSetAttribute(s2_fwd_kernel<D, KVS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         C::SMEM_BYTES);
   if (ea != cudaSuccess) return ea;
   const int grid = a.sched.n < num_sms ? a.sched.n : num_sms;
   prof_before(stream, kKernelFwd);
-  s2_fwd_kernel<D><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, to, a);
+  s2_fwd_kernel<D, KVS><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, to, a);
   cudaError_t e = cudaGetLastError();
   prof_after(stream);
   return e;
 }
 
+// kv_slots: depth of the K/V ring, 2, 3 or 4 at head dim 128 and 4, 6 or 8
+// at head dim 64 (what fits in shared memory beside the three Q slots);
+// anything else is an invalid value.
+template <int D>
+cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const CUtensorMap& to, const FwdArgs& a, int num_sms, cudaStream_t stream, int kv_slots) {
+  if constexpr (D == 128) {
+    switch (kv_slots) {
+      case 2: return launch_fwd_slots<D, 2>(tq, tk, tv, to, a, num_sms, stream);
+      case 3: return launch_fwd_slots<D, 3>(tq, tk, tv, to, a, num_sms, stream);
+      case 4: return launch_fwd_slots<D, 4>(tq, tk, tv, to, a, num_sms, stream);
+      default: return cudaErrorInvalidValue;
+    }
+  } else {
+    switch (kv_slots) {
+      case 4: return launch_fwd_slots<D, 4>(tq, tk, tv, to, a, num_sms, stream);
+      case 6: return launch_fwd_slots<D, 6>(tq, tk, tv, to, a, num_sms, stream);
+      case 8: return launch_fwd_slots<D, 8>(tq, tk, tv, to, a, num_sms, stream);
+      default: return cudaErrorInvalidValue;
+    }
+  }
+}
+
 template cudaError_t launch_fwd<64>(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
-                                    const CUtensorMap&, const FwdArgs&, int, cudaStream_t);
+                                    const CUtensorMap&, const FwdArgs&, int, cudaStream_t, int);
 template cudaError_t launch_fwd<128>(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
-                                     const CUtensorMap&, const FwdArgs&, int, cudaStream_t);
+                                     const CUtensorMap&, const FwdArgs&, int, cudaStream_t, int);
 
 }  // namespace s2

@@ -166,6 +166,24 @@ __device__ __forceinline__ void bulk_wait_read_all() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 
+// Wait until every committed bulk operation of this thread has completed
+// (its global writes or reductions are performed).
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// Untiled bulk reduction shared -> global: dst[i] += src[i] for `bytes` / 4
+// fp32 values, performed at L2; both addresses 16-byte aligned, bytes % 16 == 0.
+// Completes through the issuing thread's bulk group.
+__device__ __forceinline__ void bulk_reduce_add_f32(void* dst, uint32_t src, uint32_t bytes) {
+  asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(
+                   reinterpret_cast<uint64_t>(dst)),
+               "r"(src), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void st_shared_f32(uint32_t addr, float v) {
+  asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+
 // Plain (untiled) bulk copy global -> shared, 16-byte aligned, size % 16 == 0.
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
                                           uint32_t bar) {
@@ -386,6 +404,31 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
                "r"(d)
                : "memory");
+}
+
+// ----------------------------------------------------------------- row stores
+
+// 32 fp32 values (bit patterns) times `scale` -> 32 bf16 at dst (64 bytes, 16-byte aligned).
+__device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const uint32_t (&r)[32], float scale) {
+  uint4* out = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    out[q] = make_uint4(pack_bf16x2(__uint_as_float(r[8 * q]) * scale, __uint_as_float(r[8 * q + 1]) * scale),
+                        pack_bf16x2(__uint_as_float(r[8 * q + 2]) * scale, __uint_as_float(r[8 * q + 3]) * scale),
+                        pack_bf16x2(__uint_as_float(r[8 * q + 4]) * scale, __uint_as_float(r[8 * q + 5]) * scale),
+                        pack_bf16x2(__uint_as_float(r[8 * q + 6]) * scale, __uint_as_float(r[8 * q + 7]) * scale));
+}
+
+// The same as two 32-byte stores (whole DRAM sectors); dst 32-byte aligned.
+__device__ __forceinline__ void store_row32_v8(__nv_bfloat16* dst, const uint32_t (&r)[32], float scale) {
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint32_t v[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      v[q] = pack_bf16x2(__uint_as_float(r[16 * h + 2 * q]) * scale, __uint_as_float(r[16 * h + 2 * q + 1]) * scale);
+    st_global_v8(dst + 16 * h, v);
+  }
 }
 
 }  // namespace s2

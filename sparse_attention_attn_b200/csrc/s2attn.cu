@@ -11,6 +11,7 @@
 #include <cstdint>
 #include <cstdlib>
 #include <mutex>
+#include <string>
 #include <vector>
 
 #include "s2_common.cuh"
@@ -20,9 +21,15 @@
 namespace s2 {
 template <int D>
 cudaError_t launch_fwd(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
-                       const FwdArgs&, int, cudaStream_t);
+                       const FwdArgs&, int, cudaStream_t, int);
 template <int D>
-cudaError_t launch_bwd(const BwdMaps&, const BwdPreArgs&, const BwdArgs&, int, cudaStream_t, int*);
+cudaError_t launch_bwd(const BwdMaps&, const BwdPreArgs&, const BwdArgs&, int, cudaStream_t, int*, int);
+template <int D>
+cudaError_t launch_bwd_fused(const BwdMaps&, const BwdPreArgs&, const BwdArgs&, int, cudaStream_t, int*);
+cudaError_t launch_rope_table(float* table, int N, int D, double pos_scale, double base, int num_sms,
+                              cudaStream_t stream);
+cudaError_t launch_rope_apply(const void* x, void* out, const float* table, int B, int N, int heads, int D,
+                              int inverse, int num_sms, cudaStream_t stream);
 }  // namespace s2
 
 namespace {
@@ -34,6 +41,12 @@ __device__ uint32_t g_fwd_status[4];  // [0] error code, [1] where
 thread_local int g_last_launches = 0;
 
 constexpr size_t kStatusBytes = 256;
+
+// Backward paths.  Split: preprocess, dK/dV kernel, dQ kernel (recomputes S
+// and dP).  Fused (head dim 128): preprocess, one kernel for dK, dV and the
+// dQ partials (reduced into an fp32 accumulator in the workspace), dq
+// conversion.
+enum BwdPath : int { kBwdSplit = 0, kBwdFused = 1 };
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -124,17 +137,90 @@ Dims make_dims(int B, int H, int Hkv, int N, int D, int G) {
   return d;
 }
 
-// Forward work order (see FwdSched): the snake order balances best; it
-// spreads the units over all CTAs at once, so it is taken only while K and V
-// together stay within about twice the L2 (126 MB on B200) -- beyond that the
-// pairs order keeps each K/V tile's readers running together.
-FwdSched make_fwd_sched(const Dims& d) {
+// ---------------------------------------------------------------- plan override
+// A plan override string ("key=value,..."), used to time or test a variant
+// that the per-shape selection would not pick.  It starts from the
+// S2ATTN_TILE environment variable and can be replaced at run time by the
+// s2attn_set_tile_override test hook.  Keys: bwd=split|fused,
+// fwd_order=snake|pairs.  Unknown keys and values are ignored.
+std::mutex g_override_mu;
+std::string g_override;
+bool g_override_init = false;
+
+std::string tile_override() {
+  std::lock_guard<std::mutex> lk(g_override_mu);
+  if (!g_override_init) {
+    const char* e = std::getenv("S2ATTN_TILE");
+    g_override = e ? e : "";
+    g_override_init = true;
+  }
+  return g_override;
+}
+
+// Value of `key` in the override string, or "" if absent.
+std::string override_value(const std::string& spec, const char* key) {
+  const std::string k = std::string(key) + "=";
+  size_t pos = 0;
+  while (pos < spec.size()) {
+    size_t end = spec.find(',', pos);
+    if (end == std::string::npos) end = spec.size();
+    const std::string item = spec.substr(pos, end - pos);
+    if (item.compare(0, k.size(), k) == 0) return item.substr(k.size());
+    pos = end + 1;
+  }
+  return "";
+}
+
+// ---------------------------------------------------------------- per-shape plan
+// The kernel variant and pipeline depths for one call, chosen from the shape
+// (D, G, N, H, Hkv, B) and the SM count; the table below follows the sweep
+// recorded under profiles/ (every variant timed on the five workload shapes).
+struct Plan {
+  int fwd_snake;     // forward work order: 1 snake (longest first), 0 equal-work pairs
+  int fwd_kv_slots;  // forward K/V ring depth: 2-4 (head dim 128), 4/6/8 (head dim 64)
+  int bwd_path;      // kBwdFused (head dim 128 only) or kBwdSplit
+  int bwd_stages;    // split backward operand stages: 2-3 (head dim 128), 3-4 (head dim 64)
+};
+
+bool valid_kv_slots(int D, int v) { return D == 128 ? (v >= 2 && v <= 4) : (v == 4 || v == 6 || v == 8); }
+bool valid_bwd_stages(int D, int v) { return D == 128 ? (v == 2 || v == 3) : (v == 3 || v == 4); }
+
+Plan select_plan(int B, int H, int Hkv, int N, int D, int G, int sms) {
+  (void)H;
+  (void)G;
+  (void)sms;
+  Plan p;
+  // The snake order balances the CTAs best but spreads the units over all of
+  // them at once, so it is taken while K and V together stay within about
+  // twice the L2 (126 MB): beyond that the pairs order keeps the readers of a
+  // K/V tile running together.
+  const double kv_bytes = 2.0 * B * N * Hkv * D * 2.0;
+  p.fwd_snake = kv_bytes <= 256.0 * 1024 * 1024 ? 1 : 0;
+  p.fwd_kv_slots = D == 128 ? 4 : 8;
+  p.bwd_path = D == 128 ? kBwdFused : kBwdSplit;
+  p.bwd_stages = 3;
+  // the override, where it names a variant that exists for this head dim
+  const std::string spec = tile_override();
+  const std::string order = override_value(spec, "fwd_order");
+  if (order == "snake") p.fwd_snake = 1;
+  if (order == "pairs") p.fwd_snake = 0;
+  const std::string kv = override_value(spec, "fwd_kv");
+  if (!kv.empty() && valid_kv_slots(D, std::atoi(kv.c_str()))) p.fwd_kv_slots = std::atoi(kv.c_str());
+  const std::string path = override_value(spec, "bwd");
+  if (path == "split") p.bwd_path = kBwdSplit;
+  if (path == "fused" && D == 128) p.bwd_path = kBwdFused;
+  const std::string st = override_value(spec, "bwd_stages");
+  if (!st.empty() && valid_bwd_stages(D, std::atoi(st.c_str()))) p.bwd_stages = std::atoi(st.c_str());
+  return p;
+}
+
+// Forward work order (see FwdSched).
+FwdSched make_fwd_sched(const Dims& d, int snake) {
   FwdSched s;
   s.units = d.B * d.H * d.n_groups;
   s.Ti = (d.tiles + 1) / 2;
   s.ppu = (s.Ti + 1) / 2;
-  const double kv_bytes = 2.0 * d.B * d.N * d.Hkv * d.D * 2.0;
-  s.snake = kv_bytes <= 256.0 * 1024 * 1024 ? 1 : 0;
+  s.snake = snake;
   s.n = s.snake ? s.units * s.Ti : s.units * s.ppu;
   return s;
 }
@@ -159,6 +245,14 @@ size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 size_t rowstat_bytes(int B, int H, int N) {
   return round_up(static_cast<size_t>(B) * H * N * sizeof(float), 256);
+}
+
+// Workspace: status block, -Delta, -lse*log2(e), and for the fused path the
+// fp32 [B, H, N, D] dQ accumulator.
+size_t workspace_bytes_for(int path, int B, int H, int N, int D) {
+  size_t n = kStatusBytes + 2 * rowstat_bytes(B, H, N);
+  if (path == kBwdFused) n += round_up(static_cast<size_t>(B) * H * N * D * sizeof(float), 256);
+  return n;
 }
 
 __global__ void s2_selftest_wait_kernel(uint32_t* status, unsigned long long limit_ns) {
@@ -264,7 +358,7 @@ int s2attn_last_launch_count(void) { return g_last_launches; }
 
 size_t s2attn_bwd_workspace_bytes(int B, int H, int Hkv, int N, int D, int G) {
   if (validate_shape(B, H, Hkv, N, D, G) != S2ATTN_OK) return 0;
-  return kStatusBytes + 2 * rowstat_bytes(B, H, N);
+  return workspace_bytes_for(select_plan(B, H, Hkv, N, D, G, 0).bwd_path, B, H, N, D);
 }
 
 int s2attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
@@ -284,7 +378,8 @@ int s2attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
     return S2ATTN_ERR_CUDA;
   FwdArgs a;
   a.d = make_dims(B, H, Hkv, N, D, G);
-  a.sched = make_fwd_sched(a.d);
+  const Plan plan = select_plan(B, H, Hkv, N, D, G, info.sms);
+  a.sched = make_fwd_sched(a.d, plan.fwd_snake);
   a.scale_log2 = static_cast<float>(1.4426950408889634 / __builtin_sqrt(static_cast<double>(D)));
   a.lse = lse;  // o is written through its TMA map
   void* status = nullptr;
@@ -292,16 +387,20 @@ int s2attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   a.status = static_cast<uint32_t*>(status);
   a.wait_limit_ns = wait_limit_ns();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = (D == 64) ? launch_fwd<64>(tq, tk, tv, to, a, info.sms, s)
-                             : launch_fwd<128>(tq, tk, tv, to, a, info.sms, s);
+  cudaError_t e = (D == 64) ? launch_fwd<64>(tq, tk, tv, to, a, info.sms, s, plan.fwd_kv_slots)
+                             : launch_fwd<128>(tq, tk, tv, to, a, info.sms, s, plan.fwd_kv_slots);
   if (e != cudaSuccess) return S2ATTN_ERR_CUDA;
   g_last_launches = 1;
   return S2ATTN_OK;
 }
 
-int s2attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
-               const void* dO, void* dq, void* dk, void* dv, int B, int H, int Hkv, int N, int D,
-               int G, void* workspace, size_t workspace_bytes, s2attn_stream_t stream) {
+}  // extern "C"
+
+namespace {
+// The backward on `path` (kBwdSplit or kBwdFused).
+int bwd_impl(int path, int stages, const void* q, const void* k, const void* v, const void* o, const float* lse,
+             const void* dO, void* dq, void* dk, void* dv, int B, int H, int Hkv, int N, int D, int G,
+             void* workspace, size_t workspace_bytes, s2attn_stream_t stream, const float* rope = nullptr) {
   g_last_launches = 0;
   if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return S2ATTN_ERR_INVALID_ARG;
   int st = validate_shape(B, H, Hkv, N, D, G);
@@ -309,7 +408,7 @@ int s2attn_bwd(const void* q, const void* k, const void* v, const void* o, const
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
       !aligned16(dO) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
     return S2ATTN_ERR_MISALIGNED;
-  const size_t need = s2attn_bwd_workspace_bytes(B, H, Hkv, N, D, G);
+  const size_t need = workspace_bytes_for(path, B, H, N, D);
   if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return S2ATTN_ERR_WORKSPACE;
   DeviceInfo info;
@@ -325,6 +424,8 @@ int s2attn_bwd(const void* q, const void* k, const void* v, const void* o, const
   uint32_t* status = reinterpret_cast<uint32_t*>(ws);
   float* ndelta = reinterpret_cast<float*>(ws + kStatusBytes);
   float* nlse2 = reinterpret_cast<float*>(ws + kStatusBytes + rowstat_bytes(B, H, N));
+  float* dqacc = path == kBwdFused ? reinterpret_cast<float*>(ws + kStatusBytes + 2 * rowstat_bytes(B, H, N))
+                                   : nullptr;
   const Dims d = make_dims(B, H, Hkv, N, D, G);
   BwdPreArgs pre;
   pre.d = d;
@@ -333,6 +434,7 @@ int s2attn_bwd(const void* q, const void* k, const void* v, const void* o, const
   pre.lse = lse;
   pre.ndelta = ndelta;
   pre.nlse2 = nlse2;
+  pre.dqacc = dqacc;
   pre.status = status;
   BwdArgs a;
   a.d = d;
@@ -343,18 +445,137 @@ int s2attn_bwd(const void* q, const void* k, const void* v, const void* o, const
   a.ndelta = ndelta;
   a.nlse2 = nlse2;
   a.dq = dq;
+  a.dqacc = dqacc;
   a.dk = dk;
   a.dv = dv;
   a.kv_v8 = ((reinterpret_cast<uintptr_t>(dk) | reinterpret_cast<uintptr_t>(dv)) & 31u) == 0 ? 1 : 0;
+  a.rope = path == kBwdFused ? rope : nullptr;
   a.status = status;
   a.wait_limit_ns = wait_limit_ns();
   int launches = 0;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = (D == 64) ? launch_bwd<64>(maps, pre, a, info.sms, s, &launches)
-                            : launch_bwd<128>(maps, pre, a, info.sms, s, &launches);
+  cudaError_t e;
+  if (path == kBwdFused)
+    e = launch_bwd_fused<128>(maps, pre, a, info.sms, s, &launches);  // the plan picks it at D == 128 only
+  else
+    e = (D == 64) ? launch_bwd<64>(maps, pre, a, info.sms, s, &launches, stages)
+                  : launch_bwd<128>(maps, pre, a, info.sms, s, &launches, stages);
+  if (e == cudaSuccess && rope != nullptr && path != kBwdFused) {
+    // the split path writes dq, dk of the rotated inputs: turn them back in place
+    e = launch_rope_apply(dq, dq, rope, B, N, H, D, 1, info.sms, s);
+    if (e == cudaSuccess) e = launch_rope_apply(dk, dk, rope, B, N, Hkv, D, 1, info.sms, s);
+    launches += 2;
+  }
   g_last_launches = launches;
   return e == cudaSuccess ? S2ATTN_OK : S2ATTN_ERR_CUDA;
 }
+
+bool rope_table_args_ok(int N, int D, double pos_scale, double base) {
+  return N > 0 && (D == 64 || D == 128) && pos_scale > 0.0 && pos_scale <= 1e6 && base > 1.0 && base < 1e30;
+}
+}  // namespace
+
+extern "C" {
+
+int s2attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+               const void* dO, void* dq, void* dk, void* dv, int B, int H, int Hkv, int N, int D,
+               int G, void* workspace, size_t workspace_bytes, s2attn_stream_t stream) {
+  const Plan plan = select_plan(B, H, Hkv, N, D, G, 0);
+  return bwd_impl(plan.bwd_path, plan.bwd_stages, q, k, v, o, lse, dO, dq, dk, dv, B, H, Hkv, N, D, G,
+                  workspace, workspace_bytes, stream);
+}
+
+size_t s2attn_rope_table_bytes(int N, int D) {
+  if (N <= 0 || (D != 64 && D != 128)) return 0;
+  return static_cast<size_t>(N) * (D / 2) * 2 * sizeof(float);
+}
+
+int s2attn_rope_table(float* table, int N, int D, double pos_scale, double rope_base, s2attn_stream_t stream) {
+  g_last_launches = 0;
+  if (!table) return S2ATTN_ERR_INVALID_ARG;
+  if (!rope_table_args_ok(N, D, pos_scale, rope_base)) return D == 64 || D == 128 ? S2ATTN_ERR_INVALID_ARG
+                                                                                 : S2ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(table)) return S2ATTN_ERR_MISALIGNED;
+  DeviceInfo info;
+  if (!device_info(&info)) return S2ATTN_ERR_CUDA;
+  if (!info.ok) return S2ATTN_ERR_UNSUPPORTED;
+  if (launch_rope_table(table, N, D, pos_scale, rope_base, info.sms, static_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
+    return S2ATTN_ERR_CUDA;
+  g_last_launches = 1;
+  return S2ATTN_OK;
+}
+
+int s2attn_rope_apply(const void* x, void* out, const float* table, int B, int N, int heads, int D, int inverse,
+                      s2attn_stream_t stream) {
+  g_last_launches = 0;
+  if (!x || !out || !table || B <= 0 || N <= 0 || heads <= 0) return S2ATTN_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return S2ATTN_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * N * heads * D >= (1LL << 40)) return S2ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(out) || !aligned16(table)) return S2ATTN_ERR_MISALIGNED;
+  DeviceInfo info;
+  if (!device_info(&info)) return S2ATTN_ERR_CUDA;
+  if (!info.ok) return S2ATTN_ERR_UNSUPPORTED;
+  if (launch_rope_apply(x, out, table, B, N, heads, D, inverse ? 1 : 0, info.sms,
+                        static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return S2ATTN_ERR_CUDA;
+  g_last_launches = 1;
+  return S2ATTN_OK;
+}
+
+int s2attn_fwd_rope(const void* q, const void* k, const void* v, void* o, float* lse, void* q_rot, void* k_rot,
+                    const float* table, int B, int H, int Hkv, int N, int D, int G, s2attn_stream_t stream) {
+  g_last_launches = 0;
+  if (!q || !k || !v || !o || !lse || !q_rot || !k_rot || !table) return S2ATTN_ERR_INVALID_ARG;
+  int st = validate_shape(B, H, Hkv, N, D, G);
+  if (st != S2ATTN_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(q_rot) || !aligned16(k_rot) || !aligned16(table))
+    return S2ATTN_ERR_MISALIGNED;
+  if (q_rot == q || k_rot == k || q_rot == k_rot) return S2ATTN_ERR_INVALID_ARG;  // the backward needs both
+  st = s2attn_rope_apply(q, q_rot, table, B, N, H, D, 0, stream);
+  if (st != S2ATTN_OK) return st;
+  st = s2attn_rope_apply(k, k_rot, table, B, N, Hkv, D, 0, stream);
+  if (st != S2ATTN_OK) return st;
+  st = s2attn_fwd(q_rot, k_rot, v, o, lse, B, H, Hkv, N, D, G, stream);
+  g_last_launches = st == S2ATTN_OK ? 3 : 0;
+  return st;
+}
+
+int s2attn_bwd_rope(const void* q_rot, const void* k_rot, const void* v, const void* o, const float* lse,
+                    const void* dO, void* dq, void* dk, void* dv, const float* table, int B, int H, int Hkv, int N,
+                    int D, int G, void* workspace, size_t workspace_bytes, s2attn_stream_t stream) {
+  g_last_launches = 0;
+  if (!table) return S2ATTN_ERR_INVALID_ARG;
+  if (!aligned16(table)) return S2ATTN_ERR_MISALIGNED;
+  const Plan plan = select_plan(B, H, Hkv, N, D, G, 0);
+  return bwd_impl(plan.bwd_path, plan.bwd_stages, q_rot, k_rot, v, o, lse, dO, dq, dk, dv, B, H, Hkv, N, D, G,
+                  workspace, workspace_bytes, stream, table);
+}
+
+int s2attn_plan(int B, int H, int Hkv, int N, int D, int G, int num_sms, int* out) {
+  if (!out) return S2ATTN_ERR_INVALID_ARG;
+  const int st = validate_shape(B, H, Hkv, N, D, G);
+  if (st != S2ATTN_OK) return st;
+  const Plan p = select_plan(B, H, Hkv, N, D, G, num_sms);
+  out[0] = p.fwd_snake;
+  out[1] = p.fwd_kv_slots;
+  out[2] = p.bwd_path;
+  out[3] = p.bwd_stages;
+  return S2ATTN_OK;
+}
+
+int s2attn_set_tile_override(const char* spec) {
+  std::lock_guard<std::mutex> lk(g_override_mu);
+  if (spec) {
+    g_override = spec;
+  } else {
+    const char* e = std::getenv("S2ATTN_TILE");
+    g_override = e ? e : "";
+  }
+  g_override_init = true;
+  return S2ATTN_OK;
+}
+
 
 int s2attn_device_status(void* workspace, s2attn_stream_t stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -457,11 +678,16 @@ extern "C" int s2attn_bwd_noalloc(const void* q, const void* k, const void* v, c
                                   int B, int H, int Hkv, int N, int D, int G,
                                   s2attn_stream_t stream) {
   g_last_launches = 0;
-  const size_t need = s2attn_bwd_workspace_bytes(B, H, Hkv, N, D, G);
+  // the split backward: its scratch (status block, Delta, lse*log2(e)) grows
+  // with B * H * N only, where the fused path would need a dQ accumulator of
+  // B * H * N * D floats
+  const bool valid = validate_shape(B, H, Hkv, N, D, G) == S2ATTN_OK;
+  const size_t need = valid ? workspace_bytes_for(kBwdSplit, B, H, N, D) : 0;
   if (need > kNoAllocScratchBytes) return S2ATTN_ERR_WORKSPACE;
   void* scratch = nullptr;
-  // need == 0 means the shape is invalid: s2attn_bwd reports which error
-  if (need != 0 && !noalloc_scratch(&scratch)) return S2ATTN_ERR_CUDA;
-  return s2attn_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, Hkv, N, D, G, scratch,
-                    kNoAllocScratchBytes, stream);
+  // an invalid shape: bwd_impl reports which error
+  if (valid && !noalloc_scratch(&scratch)) return S2ATTN_ERR_CUDA;
+  const Plan plan = select_plan(B, H, Hkv, N, D, G, 0);
+  return bwd_impl(kBwdSplit, plan.bwd_stages, q, k, v, o, lse, dO, dq, dk, dv, B, H, Hkv, N, D, G, scratch,
+                  kNoAllocScratchBytes, stream);
 }

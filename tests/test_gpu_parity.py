@@ -52,8 +52,21 @@ SMALL = [
 ]
 
 
-@pytest.mark.parametrize("B,N,H,Hkv,D,G", SMALL)
-def test_small_whole_tensor(B, N, H, Hkv, D, G):
+@pytest.fixture
+def bwd_path(request):
+    """Backward path forced through the plan override for the test's duration
+    (head dim 128 has both; head dim 64 has the split path only)."""
+    from sparse_attention_attn_b200 import _lib
+    _lib.s2attn_set_tile_override(f"bwd={request.param}")
+    yield request.param
+    _lib.s2attn_set_tile_override(None)
+
+
+SMALL_PATHS = [(*s, p) for s in SMALL for p in (("fused", "split") if s[4] == 128 else ("split",))]
+
+
+@pytest.mark.parametrize("B,N,H,Hkv,D,G,bwd_path", SMALL_PATHS, indirect=["bwd_path"])
+def test_small_whole_tensor(B, N, H, Hkv, D, G, bwd_path):
     shape = I.Shape("small", B, H, Hkv, D, N, G)
     (q, k, v, do), (o, lse, dq, dk, dv) = _run(shape, seed_offset=7)
     q64, k64, v64, do64 = (to64(t) for t in (q, k, v, do))
@@ -64,6 +77,35 @@ def test_small_whole_tensor(B, N, H, Hkv, D, G):
     check_grad("dQ", to64(dq), dq_ref)
     check_grad("dK", to64(dk), dk_ref)
     check_grad("dV", to64(dv), dv_ref)
+
+
+PLAN_VARIANTS = [
+    # every variant the per-shape plan can select, forced through the override
+    (128, "fwd_order=pairs"), (128, "fwd_kv=2"), (128, "fwd_kv=3"), (128, "bwd=split,bwd_stages=2"),
+    (64, "fwd_order=pairs"), (64, "fwd_kv=4"), (64, "fwd_kv=6"), (64, "bwd_stages=4"),
+]
+
+
+@pytest.mark.parametrize("D,spec", PLAN_VARIANTS, ids=[f"d{d}-{s}" for d, s in PLAN_VARIANTS])
+def test_plan_variants(D, spec):
+    """Each selectable kernel variant (work order, K/V ring depth, backward path
+    and stages) against the oracle on whole tensors: shifted GQA heads, two
+    batches, a group of 12 tiles (odd forward items and long pipelines)."""
+    from sparse_attention_attn_b200 import _lib
+    shape = I.Shape("plan", 2, 4, 2, D, 3072, 1536)
+    _lib.s2attn_set_tile_override(spec)
+    try:
+        (q, k, v, do), (o, lse, dq, dk, dv) = _run(shape, seed_offset=13)
+    finally:
+        _lib.s2attn_set_tile_override(None)
+    q64, k64, v64, do64 = (to64(t) for t in (q, k, v, do))
+    o_ref, lse_ref = ref.s2_attention_fwd(q64, k64, v64, shape.G)
+    dq_ref, dk_ref, dv_ref, _ = ref.s2_attention_bwd(q64, k64, v64, do64, shape.G)
+    check_o(to64(o), o_ref, f" [{spec}]")
+    assert max_abs(to64(lse), lse_ref) < 1e-3
+    check_grad("dQ", to64(dq), dq_ref, f" [{spec}]")
+    check_grad("dK", to64(dk), dk_ref, f" [{spec}]")
+    check_grad("dV", to64(dv), dv_ref, f" [{spec}]")
 
 
 @pytest.mark.parametrize("q_scale", [3.0, 0.0], ids=["large-scores", "equal-scores"])
@@ -161,6 +203,12 @@ def _check_full_size(shape: I.Shape, m: int, units=None):
 @pytest.mark.parametrize("shape", I.WORKLOADS[:4], ids=lambda s: s.name)
 def test_workload_sampled(shape):
     _check_full_size(shape, m=2048)
+
+
+@pytest.mark.parametrize("bwd_path", ["split"], indirect=True)
+def test_workload_split_backward_sampled(bwd_path):
+    """The split backward (the no-allocation entry point's path) at full size."""
+    _check_full_size(I.LLAMA2_7B_8K, m=2048)
 
 
 @pytest.mark.slow
