@@ -19,6 +19,10 @@ Readings taken where the pages are silent (listed in the design notes):
   (0.5 for 4096 -> 8192), so the angle of pair i at token t is t * s * base^(-2i/D);
 * the rotation is applied to q and k at their original token positions,
   before the shift and grouping of S2 attention, and not to v;
+* the rotated q and k are bf16 tensors, like every activation at the call
+  boundary (the forward returns them and the backward takes them), so the
+  attention sees them rounded to bf16 (round to nearest even); the gradients
+  pass through that rounding unchanged;
 * the backward of a rotation is the rotation by the opposite angle.
 
 All arithmetic is float64 numpy.  Layout: x is [B, N, heads, D].
@@ -30,8 +34,17 @@ import numpy as np
 
 from .s2_ref import s2_attention_bwd, s2_attention_fwd
 
-__all__ = ["rope_angles", "rope_rotate", "rope_rotate_rows", "s2_rope_attention_fwd", "s2_rope_attention_bwd",
-           "s2_rope_unit"]
+__all__ = ["rope_angles", "rope_rotate", "rope_rotate_rows", "round_bf16", "s2_rope_attention_fwd",
+           "s2_rope_attention_bwd", "s2_rope_unit"]
+
+
+def round_bf16(x) -> np.ndarray:
+    """Values rounded to bfloat16 (8 significant bits, round to nearest even),
+    returned as float64: first to float32 (nearest), then the low 16 bits of
+    the float32 pattern are rounded away, ties to even."""
+    u = np.ascontiguousarray(np.asarray(x, dtype=np.float64).astype(np.float32)).view(np.uint32).astype(np.uint64)
+    u = (u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000
+    return u.astype(np.uint32).view(np.float32).astype(np.float64)
 
 
 def rope_angles(N: int, D: int, pos_scale: float, base: float = 10000.0) -> np.ndarray:
@@ -74,7 +87,7 @@ def rope_rotate_rows(x, t, pos_scale: float, base: float = 10000.0, inverse: boo
 
 
 def s2_rope_unit(q, k, v, do, G: int, b: int, h: int, g: int, pos_scale: float, base: float = 10000.0,
-                 piece: str = "whole", m: int | None = None):
+                 piece: str = "whole", m: int | None = None, bf16_boundary: bool = True):
     """One (batch b, query head h, rolled group g) unit of S2 attention on
     rotated q and k, at original positions.  piece = "whole" (every row of the
     group), "prefix" or "suffix" (its first / last m rows, as s2_unit_prefix /
@@ -88,8 +101,8 @@ def s2_rope_unit(q, k, v, do, G: int, b: int, h: int, g: int, pos_scale: float, 
     s = shift_of_head(h, H, N, G)
     kh = kv_head_of(h, H, Hkv)
     rows = (np.arange(g * G, (g + 1) * G) + s) % N
-    qg = rope_rotate_rows(q[b, rows, h], rows, pos_scale, base)
-    kg = rope_rotate_rows(k[b, rows, kh], rows, pos_scale, base)
+    qg = _boundary(rope_rotate_rows(q[b, rows, h], rows, pos_scale, base), bf16_boundary)
+    kg = _boundary(rope_rotate_rows(k[b, rows, kh], rows, pos_scale, base), bf16_boundary)
     vg = np.asarray(v[b, rows, kh], dtype=np.float64)
     dog = np.asarray(do[b, rows, h], dtype=np.float64)
     if piece == "whole":
@@ -107,19 +120,26 @@ def s2_rope_unit(q, k, v, do, G: int, b: int, h: int, g: int, pos_scale: float, 
             "dk_part": rope_rotate_rows(dk, r, pos_scale, base, inverse=True), "dv_part": dv}
 
 
-def s2_rope_attention_fwd(q, k, v, G: int, pos_scale: float, base: float = 10000.0):
-    """S2 attention of rotated q and k: returns (o, lse, q_rot, k_rot)."""
+def _boundary(x, bf16: bool):
+    return round_bf16(x) if bf16 else x
+
+
+def s2_rope_attention_fwd(q, k, v, G: int, pos_scale: float, base: float = 10000.0, bf16_boundary: bool = True):
+    """S2 attention of rotated q and k: returns (o, lse, q_rot, k_rot), q_rot
+    and k_rot as the exact rotation (fp64).  With bf16_boundary the attention
+    reads them rounded to bf16 (the call boundary's dtype); without, it reads
+    the exact values (the plain composite function, for the gradient pins)."""
     qr = rope_rotate(q, pos_scale, base)
     kr = rope_rotate(k, pos_scale, base)
-    o, lse = s2_attention_fwd(qr, kr, v, G)
+    o, lse = s2_attention_fwd(_boundary(qr, bf16_boundary), _boundary(kr, bf16_boundary), v, G)
     return o, lse, qr, kr
 
 
-def s2_rope_attention_bwd(q, k, v, do, G: int, pos_scale: float, base: float = 10000.0):
+def s2_rope_attention_bwd(q, k, v, do, G: int, pos_scale: float, base: float = 10000.0, bf16_boundary: bool = True):
     """Gradients with respect to the unrotated q and k (and v): the S2
     backward on the rotated inputs, then dq and dk rotated back.
     Returns (dq, dk, dv)."""
-    qr = rope_rotate(q, pos_scale, base)
-    kr = rope_rotate(k, pos_scale, base)
+    qr = _boundary(rope_rotate(q, pos_scale, base), bf16_boundary)
+    kr = _boundary(rope_rotate(k, pos_scale, base), bf16_boundary)
     dqr, dkr, dv, _ = s2_attention_bwd(qr, kr, v, do, G)
     return rope_rotate(dqr, pos_scale, base, inverse=True), rope_rotate(dkr, pos_scale, base, inverse=True), dv

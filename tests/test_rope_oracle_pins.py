@@ -25,6 +25,17 @@ def _rand(shape, seed):
     return np.random.default_rng(seed).standard_normal(shape)
 
 
+def test_bf16_rounding_matches_torch_and_ties():
+    """round_bf16 against torch's float32 -> bfloat16 cast (a library
+    routine), and hand-picked ties: 1 + 2^-8 (halfway, even below) rounds down,
+    1 + 3*2^-8 (halfway, odd below) rounds up."""
+    import torch
+    x = np.random.default_rng(30).standard_normal(100_000).astype(np.float32) * 10.0
+    ref = torch.from_numpy(x).to(torch.bfloat16).double().numpy()
+    np.testing.assert_array_equal(rr.round_bf16(x), ref)
+    np.testing.assert_array_equal(rr.round_bf16([1 + 2**-8, 1 + 3 * 2**-8, -(1 + 2**-8)]), [1.0, 1 + 2**-6, -1.0])
+
+
 def test_golden_hand_example():
     gd = json.load(open(os.path.join(GOLDEN, "rope_pi_d4.json")))
     x = np.zeros((1, gd["t"] + 1, 1, gd["D"]))
@@ -86,11 +97,11 @@ def test_backward_finite_differences(Hkv):
     B, N, G, H, D = 1, 16, 8, 4, 4
     q, k, v = _rand((B, N, H, D), 6), _rand((B, N, Hkv, D), 7), _rand((B, N, Hkv, D), 8)
     w = _rand((B, N, H, D), 9)
-    dq, dk, dv = rr.s2_rope_attention_bwd(q, k, v, w, G, 0.5, 100.0)
+    dq, dk, dv = rr.s2_rope_attention_bwd(q, k, v, w, G, 0.5, 100.0, bf16_boundary=False)
     eps = 1e-6
 
     def loss(qq, kk, vv):
-        return float(np.sum(rr.s2_rope_attention_fwd(qq, kk, vv, G, 0.5, 100.0)[0] * w))
+        return float(np.sum(rr.s2_rope_attention_fwd(qq, kk, vv, G, 0.5, 100.0, bf16_boundary=False)[0] * w))
 
     for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
         num = np.zeros_like(x)
@@ -124,15 +135,15 @@ def test_planted_mistakes_fail(monkeypatch):
     q, k, v, w = _rand((1, 8, 2, 4), 10), _rand((1, 8, 2, 4), 11), _rand((1, 8, 2, 4), 12), _rand((1, 8, 2, 4), 13)
     good = rr.rope_rotate
     monkeypatch.setattr(rr, "rope_rotate", lambda x, s, base=10000.0, inverse=False: good(x, s, base, False))
-    dq_bad, _, _ = rr.s2_rope_attention_bwd(q, k, v, w, 8, 0.5, 100.0)
+    dq_bad, _, _ = rr.s2_rope_attention_bwd(q, k, v, w, 8, 0.5, 100.0, bf16_boundary=False)
     monkeypatch.setattr(rr, "rope_rotate", good)
-    dq_good, _, _ = rr.s2_rope_attention_bwd(q, k, v, w, 8, 0.5, 100.0)
+    dq_good, _, _ = rr.s2_rope_attention_bwd(q, k, v, w, 8, 0.5, 100.0, bf16_boundary=False)
     eps = 1e-6
     qp, qm = q.copy(), q.copy()
     qp[0, 5, 1, 2] += eps
     qm[0, 5, 1, 2] -= eps
-    num = (np.sum(rr.s2_rope_attention_fwd(qp, k, v, 8, 0.5, 100.0)[0] * w)
-           - np.sum(rr.s2_rope_attention_fwd(qm, k, v, 8, 0.5, 100.0)[0] * w)) / (2 * eps)
+    num = (np.sum(rr.s2_rope_attention_fwd(qp, k, v, 8, 0.5, 100.0, bf16_boundary=False)[0] * w)
+           - np.sum(rr.s2_rope_attention_fwd(qm, k, v, 8, 0.5, 100.0, bf16_boundary=False)[0] * w)) / (2 * eps)
     assert abs(num - dq_good[0, 5, 1, 2]) < 1e-6
     assert abs(num - dq_bad[0, 5, 1, 2]) > 1e-4
 
@@ -147,10 +158,13 @@ def test_rows_and_unit_match_whole_tensor():
                                rr.rope_rotate(q, 0.5, 100.0)[0, rows, 1], rtol=0, atol=1e-13)
     o, lse, _, _ = rr.s2_rope_attention_fwd(q, k, v, G, 0.5, 100.0)
     dq, dk, dv = rr.s2_rope_attention_bwd(q, k, v, do, G, 0.5, 100.0)
+    # the bf16 boundary is a rounding of the exact rotation, and moves o by a bf16 ulp's worth
+    o_exact, _, _, _ = rr.s2_rope_attention_fwd(q, k, v, G, 0.5, 100.0, bf16_boundary=False)
+    assert 0 < np.abs(o - o_exact).max() < 1e-2
     for h, g in ((0, 1), (3, 1), (2, 0)):
         kh = h // (H // Hkv)
         parts = {}
-        for piece, m in (("whole", None), ("prefix", 12), ("suffix", 12)):
+        for piece, m in (("whole", None), ("prefix", 12), ("suffix", 12)):  # noqa: B007
             u = rr.s2_rope_unit(q, k, v, do, G, 0, h, g, 0.5, 100.0, piece, m)
             np.testing.assert_allclose(u["o"], o[0, u["rows"], h], atol=1e-12, rtol=0)
             np.testing.assert_allclose(u["lse"], lse[0, h, u["rows"]], atol=1e-12, rtol=0)
