@@ -583,7 +583,7 @@ def other_workload(shape: I.Shape, dev, peaks, steps: int = 5, warmup: int = 3):
 def sweep_variants(D: int):
     """Every variant the per-shape plan can select at head dim D, as override
     strings: forward (work order x K/V ring depth) and backward (path x stages)."""
-    slots = (2, 3, 4) if D == 128 else (4, 6, 8)
+    slots = (4,) if D == 128 else (4, 6, 8)
     fwd = [f"fwd_order={o},fwd_kv={s}" for o in ("snake", "pairs") for s in slots]
     bwd = (["bwd=fused"] if D == 128 else []) + \
         [f"bwd=split,bwd_stages={s}" for s in ((2, 3) if D == 128 else (3, 4))]

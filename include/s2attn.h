@@ -254,7 +254,7 @@ S2ATTN_API int s2attn_plan(int B, int H, int Hkv, int N, int D, int G, int num_s
  * would not pick, for tests and sweeps: a comma-separated list of key=value
  * items; keys bwd=split|fused (backward path; fused exists for head dim 128),
  * fwd_order=snake|pairs (forward work order), fwd_kv=N (forward K/V ring
- * depth: 2-4 at head dim 128, 4/6/8 at 64), bwd_stages=N (split backward
+ * depth: 4 at head dim 128, 4/6/8 at 64), bwd_stages=N (split backward
  * stages: 2-3 at head dim 128, 3-4 at 64); values that do not exist for a
  * call's head dim are ignored.  s2attn_bwd_workspace_bytes answers for the
  * path in force when it is called.  Returns S2ATTN_OK.

@@ -39,7 +39,11 @@
 namespace s2 {
 
 // KVS: slots of the K/V ring (K and V tiles share it: K0 V0 K1 V1 ...), the
-// pipeline depth the per-shape plan selects (2-4 at head dim 128, 4-8 at 64).
+// pipeline depth the per-shape plan selects (4 at head dim 128, 4-8 at 64).
+// At least 4: the issuer starts the next item's first S (which needs the
+// next item's K_0) before it releases the current item's last V / K tiles, so
+// K_0's slot must be one released earlier -- with 4 slots it is K_ta's, the
+// last K tile both warpgroups have finished with.
 template <int D, int KVS>
 struct FwdCfg {
   static constexpr int BM = kTile, BN = kTile;
@@ -52,6 +56,7 @@ struct FwdCfg {
   static constexpr uint32_t TM_O = 256;
   static constexpr int THREADS = 320;
   static_assert(SMEM_BYTES <= 232448 - 512, "shared memory");
+  static_assert(KVSLOTS >= 4, "the next item's K_0 needs a slot released before the item ends");
 };
 
 // P for 64 scores of one query row: p = 2^(s * sl2 - m), packed to bf16
@@ -516,16 +521,14 @@ cudaError_t launch_fwd_slots(const CUtensorMap& tq, const CUtensorMap& tk, const
   return e;
 }
 
-// kv_slots: depth of the K/V ring, 2, 3 or 4 at head dim 128 and 4, 6 or 8
-// at head dim 64 (what fits in shared memory beside the three Q slots);
-// anything else is an invalid value.
+// kv_slots: depth of the K/V ring, 4 at head dim 128 and 4, 6 or 8 at head
+// dim 64 (at least 4, see FwdCfg; at most what fits in shared memory beside
+// the three Q slots); anything else is an invalid value.
 template <int D>
 cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const CUtensorMap& to, const FwdArgs& a, int num_sms, cudaStream_t stream, int kv_slots) {
   if constexpr (D == 128) {
     switch (kv_slots) {
-      case 2: return launch_fwd_slots<D, 2>(tq, tk, tv, to, a, num_sms, stream);
-      case 3: return launch_fwd_slots<D, 3>(tq, tk, tv, to, a, num_sms, stream);
       case 4: return launch_fwd_slots<D, 4>(tq, tk, tv, to, a, num_sms, stream);
       default: return cudaErrorInvalidValue;
     }

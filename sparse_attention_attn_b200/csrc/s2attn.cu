@@ -177,12 +177,12 @@ std::string override_value(const std::string& spec, const char* key) {
 // recorded under profiles/ (every variant timed on the five workload shapes).
 struct Plan {
   int fwd_snake;     // forward work order: 1 snake (longest first), 0 equal-work pairs
-  int fwd_kv_slots;  // forward K/V ring depth: 2-4 (head dim 128), 4/6/8 (head dim 64)
+  int fwd_kv_slots;  // forward K/V ring depth: 4 (head dim 128), 4/6/8 (head dim 64)
   int bwd_path;      // kBwdFused (head dim 128 only) or kBwdSplit
   int bwd_stages;    // split backward operand stages: 2-3 (head dim 128), 3-4 (head dim 64)
 };
 
-bool valid_kv_slots(int D, int v) { return D == 128 ? (v >= 2 && v <= 4) : (v == 4 || v == 6 || v == 8); }
+bool valid_kv_slots(int D, int v) { return D == 128 ? v == 4 : (v == 4 || v == 6 || v == 8); }
 bool valid_bwd_stages(int D, int v) { return D == 128 ? (v == 2 || v == 3) : (v == 3 || v == 4); }
 
 Plan select_plan(int B, int H, int Hkv, int N, int D, int G, int sms) {
@@ -197,7 +197,10 @@ Plan select_plan(int B, int H, int Hkv, int N, int D, int G, int sms) {
   const double kv_bytes = 2.0 * B * N * Hkv * D * 2.0;
   p.fwd_snake = kv_bytes <= 256.0 * 1024 * 1024 ? 1 : 0;
   p.fwd_kv_slots = D == 128 ? 4 : 8;
-  p.bwd_path = D == 128 ? kBwdFused : kBwdSplit;
+  // the split path measured faster than the fused one on every workload shape
+  // (the fused kernel is limited by its dQ reductions at L2); fused stays
+  // selectable
+  p.bwd_path = kBwdSplit;
   p.bwd_stages = 3;
   // the override, where it names a variant that exists for this head dim
   const std::string spec = tile_override();

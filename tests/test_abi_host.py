@@ -90,8 +90,8 @@ def test_backward_argument_validation():
 
 def test_workspace_bytes():
     # status block + two fp32 [B, H, N] row-statistics arrays, each rounded to 256 bytes;
-    # at head dim 128 (fused backward) also the fp32 [B, H, N, D] dq accumulator
-    assert _lib.s2attn_bwd_workspace_bytes(1, 32, 32, 8192, 128, 2048) == 256 + 2 * 32 * 8192 * 4 + 32 * 8192 * 128 * 4
+    # on the fused backward also the fp32 [B, H, N, D] dq accumulator
+    assert _lib.s2attn_bwd_workspace_bytes(1, 32, 32, 8192, 128, 2048) == 256 + 2 * 32 * 8192 * 4
     assert _lib.s2attn_bwd_workspace_bytes(1, 1, 1, 128, 64, 128) == 256 + 2 * 512
     assert _lib.s2attn_bwd_workspace_bytes(1, 4, 3, 1024, 64, 256) == 0  # invalid shape
     # the split path, forced through the override, needs no accumulator
@@ -118,16 +118,16 @@ def test_profile_api_host_side():
 
 
 def test_plan_selection_table():
-    """The per-shape plan (host logic, no GPU): head dim 128 takes the fused
-    backward, head dim 64 the split one; the forward's work order follows the
-    K/V size; depths are the selected defaults."""
+    """The per-shape plan (host logic, no GPU): the split backward (measured
+    faster), the forward's work order following the K/V size, the selected
+    depths."""
     from sparse_attention_attn_b200 import inputs as I
     expect = {
         "tiny": ("snake", 8, "split", 3),
-        "llama2-7b-n8192": ("snake", 4, "fused", 3),
-        "qwen3-8b-gqa-n16384": ("snake", 4, "fused", 3),
-        "llama2-70b-gqa-n32768": ("snake", 4, "fused", 3),
-        "llama2-7b-n102400": ("pairs", 4, "fused", 3),
+        "llama2-7b-n8192": ("snake", 4, "split", 3),
+        "qwen3-8b-gqa-n16384": ("snake", 4, "split", 3),
+        "llama2-70b-gqa-n32768": ("snake", 4, "split", 3),
+        "llama2-7b-n102400": ("pairs", 4, "split", 3),
     }
     for s in I.WORKLOADS:
         p = _lib.s2attn_plan(s.B, s.H, s.Hkv, s.N, s.D, s.G, 148)
@@ -141,8 +141,8 @@ def test_plan_override_parsing():
     that do not exist for the call's head dim."""
     try:
         _lib.s2attn_set_tile_override("fwd_order=pairs,fwd_kv=2,bwd=split,bwd_stages=2")
-        p = _lib.s2attn_plan(1, 32, 32, 8192, 128, 2048, 148)
-        assert p == {"fwd_order": "pairs", "fwd_kv_slots": 2, "bwd_path": "split", "bwd_stages": 2}
+        p = _lib.s2attn_plan(1, 32, 32, 8192, 128, 2048, 148)   # a 2-slot K/V ring does not exist
+        assert p == {"fwd_order": "pairs", "fwd_kv_slots": 4, "bwd_path": "split", "bwd_stages": 2}
         p = _lib.s2attn_plan(1, 4, 4, 1024, 64, 256, 148)   # head dim 64: kv 2 and stages 2 do not exist
         assert p == {"fwd_order": "pairs", "fwd_kv_slots": 8, "bwd_path": "split", "bwd_stages": 3}
         _lib.s2attn_set_tile_override("bwd=fused,fwd_kv=6,bwd_stages=4,junk,=,x=y")
@@ -152,4 +152,4 @@ def test_plan_override_parsing():
             {"fwd_order": "snake", "fwd_kv_slots": 4, "bwd_path": "fused", "bwd_stages": 3}
     finally:
         _lib.s2attn_set_tile_override(None)
-    assert _lib.s2attn_plan(1, 32, 32, 8192, 128, 2048, 148)["bwd_path"] == "fused"
+    assert _lib.s2attn_plan(1, 32, 32, 8192, 128, 2048, 148)["bwd_path"] == "split"

@@ -81,8 +81,8 @@ def test_small_whole_tensor(B, N, H, Hkv, D, G, bwd_path):
 
 PLAN_VARIANTS = [
     # every variant the per-shape plan can select, forced through the override
-    (128, "fwd_order=pairs"), (128, "fwd_kv=2"), (128, "fwd_kv=3"), (128, "bwd=split,bwd_stages=2"),
-    (64, "fwd_order=pairs"), (64, "fwd_kv=4"), (64, "fwd_kv=6"), (64, "bwd_stages=4"),
+    (128, "fwd_order=pairs"), (128, "bwd=split,bwd_stages=2"), (128, "bwd=split,bwd_stages=3"),
+    (128, "bwd=fused"), (64, "fwd_order=pairs"), (64, "fwd_kv=4"), (64, "fwd_kv=6"), (64, "bwd_stages=4"),
 ]
 
 
@@ -90,9 +90,11 @@ PLAN_VARIANTS = [
 def test_plan_variants(D, spec):
     """Each selectable kernel variant (work order, K/V ring depth, backward path
     and stages) against the oracle on whole tensors: shifted GQA heads, two
-    batches, a group of 12 tiles (odd forward items and long pipelines)."""
+    batches, groups of 16 tiles, more forward items (256) than a B200 has SMs
+    and two or more backward items per CTA, so every CTA crosses from one item
+    to the next (where the pipelines hand over between items)."""
     from sparse_attention_attn_b200 import _lib
-    shape = I.Shape("plan", 2, 4, 2, D, 3072, 1536)
+    shape = I.Shape("plan", 2, 4, 2, D, 8192, 2048)
     _lib.s2attn_set_tile_override(spec)
     try:
         (q, k, v, do), (o, lse, dq, dk, dv) = _run(shape, seed_offset=13)
@@ -205,9 +207,9 @@ def test_workload_sampled(shape):
     _check_full_size(shape, m=2048)
 
 
-@pytest.mark.parametrize("bwd_path", ["split"], indirect=True)
-def test_workload_split_backward_sampled(bwd_path):
-    """The split backward (the no-allocation entry point's path) at full size."""
+@pytest.mark.parametrize("bwd_path", ["fused"], indirect=True)
+def test_workload_fused_backward_sampled(bwd_path):
+    """The fused backward (selectable through the plan) at full size."""
     _check_full_size(I.LLAMA2_7B_8K, m=2048)
 
 
