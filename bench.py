@@ -398,9 +398,16 @@ def run_ours(args, shape, world, rank, local):
     ms_e2e = timed_e2e(e2e_pipelined, e2e_steps, s_in, s_out)
     if s2.device_status() != 0 or s2.device_status(ws) != 0:
         raise RuntimeError("device status reports a timeout in the end-to-end loop")
-    # every step has the same inputs: the gradients that reached the host are the device's
-    if not all(torch.equal(h_, d_.cpu()) for h_, d_ in zip(host_out, dev_out[1])):
-        raise RuntimeError("end-to-end loop: gradients on the host differ from the device's")
+    # every step has the same inputs: the gradients that reached the host are
+    # the device's -- bit for bit, except dq on the fused backward path, whose
+    # fp32 reductions at L2 arrive in no fixed order (same values up to rounding)
+    for name, h_, d_ in zip(("dq", "dk", "dv"), host_out, dev_out[1]):
+        d_ = d_.cpu()
+        if torch.equal(h_, d_):
+            continue
+        rel = float((h_.float() - d_.float()).norm() / d_.float().norm().clamp_min(1e-30))
+        if not (name == "dq" and 4 in per_kernel and rel <= 1e-3):
+            raise RuntimeError(f"end-to-end loop: {name} on the host differs from the device's (rel {rel:.2e})")
 
     # ---- report ----
     fwd, bwd = effective_flops(shape)
