@@ -175,6 +175,50 @@ S2ATTN_API int s2attn_bwd_rope(const void* q_rot, const void* k_rot, const void*
                                int B, int H, int Hkv, int N, int D, int G, void* workspace, size_t workspace_bytes,
                                s2attn_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * Chunk-wise attention over detached earlier keys (segment mode).  HGA digest
+ * (arXiv 2607.15105): segment-wise backpropagation -- only the active segment
+ * stays differentiable, older KV is detached and kept in another memory tier;
+ * SeCO / SpaCO digest (arXiv 2505.16710): each chunk of a long input builds
+ * its own graph and backpropagates locally.  The N query rows of the active
+ * chunk are the last N rows of a sequence whose keys k, v hold Nk rows
+ * (bf16 [B, Nk, Hkv, D]); with causal != 0 query row i attends keys
+ * [0, Nk - N + i] (all earlier keys and its own chunk causally), with
+ * causal == 0 every one of the Nk keys (a detached segment processed as a
+ * piece of its own).  Dense causal softmax attention, no grouping or shift,
+ * scale 1/sqrt(D); N and Nk multiples of 128; D in {64, 128}.
+ * ------------------------------------------------------------------------ */
+
+/* o bf16 [B, N, H, D], lse fp32 [B, H, N] of the segment attention. */
+S2ATTN_API int s2attn_seg_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                              int Hkv, int N, int Nk, int D, int causal, s2attn_stream_t stream);
+
+/* Workspace bytes of s2attn_seg_bwd (status block, Delta, lse*log2(e)). */
+S2ATTN_API size_t s2attn_seg_bwd_workspace_bytes(int B, int H, int Hkv, int N, int Nk, int D);
+
+/*
+ * Backward of the segment attention given the FINAL o and lse of the chunk's
+ * rows (after any lse merge of pieces): dq [B, N, H, D] through every key the
+ * rows attend; with causal != 0 also dk, dv [B, N, Hkv, D] of the chunk's own
+ * keys (the last N key rows; the earlier keys are detached and get no
+ * gradient); with causal == 0 dk and dv must be NULL (dq only).
+ * dq_accumulate != 0 adds the result to dq (summing the pieces of a query's
+ * keys).  Split kernels: preprocess, dK/dV (causal only), dQ.
+ */
+S2ATTN_API int s2attn_seg_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                              const void* dO, void* dq, void* dk, void* dv, int B, int H, int Hkv, int N, int Nk,
+                              int D, int causal, int dq_accumulate, void* workspace, size_t workspace_bytes,
+                              s2attn_stream_t stream);
+
+/*
+ * Softmax attention over two disjoint key sets from the two pieces' results:
+ * lse = log(exp(lse_a) + exp(lse_b)), o = exp(lse_a - lse) o_a + exp(lse_b - lse) o_b
+ * (o_* bf16 [B, N, H, D], lse_* fp32 [B, H, N]; a piece with lse = -inf
+ * counts for nothing).  o may be o_a and lse may be lse_a (in place).
+ */
+S2ATTN_API int s2attn_lse_merge(const void* o_a, const float* lse_a, const void* o_b, const float* lse_b, void* o,
+                                float* lse, int B, int H, int N, int D, s2attn_stream_t stream);
+
 /*
  * Backward for callers that cannot allocate device memory (no counterpart in
  * the papers: this is a deployment variant of s2attn_bwd).  Some callers have

@@ -36,6 +36,11 @@ SIGNATURES = {
     "s2attn_profile_start": (_i, [_i]),
     "s2attn_profile_stop": (_i, [_vp, _vp, _i]),
     "s2attn_set_tile_override": (_i, [ctypes.c_char_p]),
+    "s2attn_seg_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp]),
+    "s2attn_seg_bwd_workspace_bytes": (ctypes.c_size_t, [_i, _i, _i, _i, _i, _i]),
+    "s2attn_seg_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _vp,
+                            ctypes.c_size_t, _vp]),
+    "s2attn_lse_merge": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp]),
     "s2attn_rope_table_bytes": (ctypes.c_size_t, [_i, _i]),
     "s2attn_rope_table": (_i, [_vp, _i, _i, ctypes.c_double, ctypes.c_double, _vp]),
     "s2attn_rope_apply": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
@@ -114,6 +119,24 @@ def s2attn_profile_start(max_launches) -> int:
 
 def s2attn_profile_stop(ms, kernel_ids, capacity) -> int:
     return load().s2attn_profile_stop(ms, kernel_ids, capacity)
+
+
+def s2attn_seg_fwd(q, k, v, o, lse, B, H, Hkv, N, Nk, D, causal, stream) -> int:
+    return load().s2attn_seg_fwd(q, k, v, o, lse, B, H, Hkv, N, Nk, D, causal, stream)
+
+
+def s2attn_seg_bwd_workspace_bytes(B, H, Hkv, N, Nk, D) -> int:
+    return load().s2attn_seg_bwd_workspace_bytes(B, H, Hkv, N, Nk, D)
+
+
+def s2attn_seg_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, Hkv, N, Nk, D, causal, dq_accumulate, workspace,
+                   workspace_bytes, stream) -> int:
+    return load().s2attn_seg_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, Hkv, N, Nk, D, causal, dq_accumulate,
+                                 workspace, workspace_bytes, stream)
+
+
+def s2attn_lse_merge(o_a, lse_a, o_b, lse_b, o, lse, B, H, N, D, stream) -> int:
+    return load().s2attn_lse_merge(o_a, lse_a, o_b, lse_b, o, lse, B, H, N, D, stream)
 
 
 def s2attn_rope_table_bytes(N, D) -> int:

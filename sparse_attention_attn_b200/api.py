@@ -215,6 +215,110 @@ class S2RopeAttention(torch.autograd.Function):
         return dq, dk, dv, None, None
 
 
+def seg_forward(q, k, v, causal: bool = True, out=None, lse=None):
+    """Attention of a chunk's queries q [B, N, H, D] over keys k, v [B, Nk, Hkv, D]:
+    causal -- row i sees keys [0, Nk - N + i] (the earlier keys, then its own
+    chunk causally); not causal -- every key (a detached segment as a piece).
+    Returns (o, lse) of that attention."""
+    B, N, H, Hkv, D = _dims(q, k)
+    Nk = k.shape[1]
+    _need("q", q, (B, N, H, D))
+    dev = q.device
+    _need("k", k, (B, Nk, Hkv, D), device=dev)
+    _need("v", v, (B, Nk, Hkv, D), device=dev)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev) if lse is None else lse
+    _need("out", out, (B, N, H, D), device=dev)
+    _need("lse", lse, (B, H, N), torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        st = _lib.s2attn_seg_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                 B, H, Hkv, N, Nk, D, int(causal), _stream(dev))
+    _lib._check("s2attn_seg_fwd", st)
+    return out, lse
+
+
+def seg_backward(q, k, v, o, lse, do, causal: bool = True, dq=None, dk=None, dv=None, dq_accumulate=False,
+                 workspace=None):
+    """Backward of seg_forward given the chunk rows' final o and lse: dq, and
+    (causal) dk, dv of the chunk's own keys -- the last N key rows.  Not
+    causal: dq only (dk, dv returned as None).  dq_accumulate adds into dq."""
+    B, N, H, Hkv, D = _dims(q, k)
+    Nk = k.shape[1]
+    _need("q", q, (B, N, H, D))
+    dev = q.device
+    for name, t, shp in (("k", k, (B, Nk, Hkv, D)), ("v", v, (B, Nk, Hkv, D)), ("o", o, (B, N, H, D)),
+                         ("do", do, (B, N, H, D))):
+        _need(name, t, shp, device=dev)
+    _need("lse", lse, (B, H, N), torch.float32, device=dev)
+    if dq is None:
+        if dq_accumulate:
+            raise ValueError("dq_accumulate needs dq")
+        dq = torch.empty_like(q)
+    _need("dq", dq, (B, N, H, D), device=dev)
+    if causal:
+        dk = torch.empty((B, N, Hkv, D), dtype=k.dtype, device=dev) if dk is None else dk
+        dv = torch.empty((B, N, Hkv, D), dtype=v.dtype, device=dev) if dv is None else dv
+        _need("dk", dk, (B, N, Hkv, D), device=dev)
+        _need("dv", dv, (B, N, Hkv, D), device=dev)
+    else:
+        dk = dv = None
+    wsb = _lib.s2attn_seg_bwd_workspace_bytes(B, H, Hkv, N, Nk, D)
+    if wsb == 0:
+        raise _lib.S2AttnError("s2attn_seg_bwd_workspace_bytes", _lib.S2ATTN_ERR_INVALID_ARG)
+    if workspace is None:
+        workspace = torch.empty(wsb, dtype=torch.uint8, device=dev)
+    with torch.cuda.device(dev):
+        st = _lib.s2attn_seg_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                 do.data_ptr(), dq.data_ptr(), None if dk is None else dk.data_ptr(),
+                                 None if dv is None else dv.data_ptr(), B, H, Hkv, N, Nk, D, int(causal),
+                                 int(dq_accumulate), workspace.data_ptr(),
+                                 workspace.numel() * workspace.element_size(), _stream(dev))
+    _lib._check("s2attn_seg_bwd", st)
+    return dq, dk, dv
+
+
+def lse_merge(o_a, lse_a, o_b, lse_b, out=None, lse=None):
+    """Attention over the union of two disjoint key sets from the two pieces'
+    (o, lse); out / lse may be o_a / lse_a (in place)."""
+    B, N, H, D = o_a.shape
+    dev = o_a.device
+    _need("o_a", o_a, (B, N, H, D))
+    _need("o_b", o_b, (B, N, H, D), device=dev)
+    _need("lse_a", lse_a, (B, H, N), torch.float32, device=dev)
+    _need("lse_b", lse_b, (B, H, N), torch.float32, device=dev)
+    out = torch.empty_like(o_a) if out is None else out
+    lse = torch.empty_like(lse_a) if lse is None else lse
+    _need("out", out, (B, N, H, D), device=dev)
+    _need("lse", lse, (B, H, N), torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        st = _lib.s2attn_lse_merge(o_a.data_ptr(), lse_a.data_ptr(), o_b.data_ptr(), lse_b.data_ptr(),
+                                   out.data_ptr(), lse.data_ptr(), B, H, N, D, _stream(dev))
+    _lib._check("s2attn_lse_merge", st)
+    return out, lse
+
+
+class ChunkAttention(torch.autograd.Function):
+    """Chunk-wise training step: the chunk's queries attend its own keys
+    causally and the detached earlier keys fully; the two pieces are merged by
+    log-sum-exp and only q, k_act, v_act receive gradients."""
+
+    @staticmethod
+    def forward(ctx, q, k_act, v_act, k_past, v_past):
+        o_a, lse_a = seg_forward(q, k_past, v_past, causal=False)
+        o_b, lse_b = seg_forward(q, k_act, v_act, causal=True)
+        o, lse = lse_merge(o_a, lse_a, o_b, lse_b, out=o_a, lse=lse_a)
+        ctx.save_for_backward(q, k_act, v_act, k_past, v_past, o, lse)
+        return o
+
+    @staticmethod
+    def backward(ctx, do):
+        q, k_act, v_act, k_past, v_past, o, lse = ctx.saved_tensors
+        do = do.contiguous()
+        dq, _, _ = seg_backward(q, k_past, v_past, o, lse, do, causal=False)
+        dq, dk, dv = seg_backward(q, k_act, v_act, o, lse, do, causal=True, dq=dq, dq_accumulate=True)
+        return dq, dk, dv, None, None
+
+
 class S2Attention(torch.autograd.Function):
     """Autograd wrapper: the drop-in attention call of a training step."""
 

@@ -219,7 +219,9 @@ __global__ void __launch_bounds__(352, 1)
       const int sh = shift_of_head(d, w.h);
       const int kb = ic.n & 1;
       if (ic.n >= 2 && !warp_wait(smem_u32(&bar_kv_empty[kb]), ((ic.n >> 1) - 1) & 1, wc, 109)) break;
-      const int tk0 = original_row(d, w.g * d.G + w.tile * kTile, sh);
+      // the kv tiles of this kernel are the query segment's own keys, which sit
+      // at key rows qoff_t*128 onwards (0 for S2 attention)
+      const int tk0 = original_row_kv(d, d.qoff_t * kTile + w.g * d.G + w.tile * kTile, sh);
       if (elect_one()) {
         mbar_arrive_expect_tx(smem_u32(&bar_kv[kb]), 2 * C::KV_BYTES);
         for (int c = 0; c < D / 64; ++c) {
@@ -506,7 +508,9 @@ struct DqCursor {
   __device__ __forceinline__ void load(const Dims& d) {
     if (!ic.valid) return;
     w = q_item(d, ic.unit, ic.tile);
-    iters = 2 * (w.tile + 1);  // 64-row kv sub-tiles from the group start to the diagonal
+    // 64-row kv sub-tiles from the group start to the diagonal (causal), or
+    // every key (segment mode, causal = 0)
+    iters = d.causal ? 2 * (w.tile + 1 + d.qoff_t) : 2 * (d.Nk / kTile);
     it = 0;
   }
   __device__ __forceinline__ void first(const Dims& d, const PairSched& ps) {
@@ -600,14 +604,14 @@ __global__ void __launch_bounds__(384, 1)
       }
       __syncwarp();
       ++q_issued;
-      const int iters = 2 * (w.tile + 1);
+      const int iters = d.causal ? 2 * (w.tile + 1 + d.qoff_t) : 2 * (d.Nk / kTile);
       for (int j = 0; j < iters; ++j, ++gi) {
         const int s = gi % ST, f = gi / ST;
         if (f > 0 && !warp_wait(smem_u32(&bar_empty[s]), (f - 1) & 1, wc, 210)) {
           ok = false;
           break;
         }
-        const int tk0 = original_row(d, w.g * d.G + j * kSub, sh);
+        const int tk0 = original_row_kv(d, w.g * d.G + j * kSub, sh);
         const uint32_t bar = smem_u32(&bar_kv[s]);
         if (elect_one()) {
           mbar_arrive_expect_tx(bar, 2 * C::KV_BYTES);
@@ -762,7 +766,7 @@ __global__ void __launch_bounds__(384, 1)
         nd2 = f2_pack(nd_next, nd_next);
       }
       const uint32_t bo = (g & 1) * kSub + half * 32;
-      const int koff = cur.it * kSub - w.tile * kTile;  // kv sub-tile start minus query tile start
+      const int koff = cur.it * kSub - (w.tile + d.qoff_t) * kTile;  // kv sub-tile start minus query tile start
       if (lane == 0) ok = mbar_wait(smem_u32(&bar_sdp[g & 1]), (g >> 1) & 1, wc, 230);
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
@@ -791,7 +795,7 @@ __global__ void __launch_bounds__(384, 1)
         p[2 * c] = ex2_approx(f2_lo(x));
         p[2 * c + 1] = ex2_approx(f2_hi(x));
       }
-      if (koff >= 0) {  // sub-tile overlaps the diagonal: key after query is masked
+      if (d.causal && koff >= 0) {  // sub-tile overlaps the diagonal: key after query is masked
 #pragma unroll
         for (int c = 0; c < 32; ++c)
           if (koff + half * 32 + c > row) p[c] = 0.f;
@@ -841,8 +845,20 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int i = 0; i < CH; ++i) {
           const int rr = i * (32 / CH) + lane / CH, ch = lane % CH;
-          const float4 v = lds_f4(stage + rr * C::ROW_OUT + ((ch ^ (rr % CH)) << 4));
-          *reinterpret_cast<float4*>(dq0 + static_cast<size_t>(rr) * d.H * D + ch * 8) = v;
+          float4 v = lds_f4(stage + rr * C::ROW_OUT + ((ch ^ (rr % CH)) << 4));
+          float4* dst = reinterpret_cast<float4*>(dq0 + static_cast<size_t>(rr) * d.H * D + ch * 8);
+          if (a.dq_accumulate) {  // dq += this piece (8 bf16 values, summed in fp32)
+            const float4 old = *dst;
+            const uint32_t* o32 = reinterpret_cast<const uint32_t*>(&old);
+            uint32_t* n32 = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&o32[u]));
+              const float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&n32[u]));
+              n32[u] = pack_bf16x2(x.x + y.x, x.y + y.y);
+            }
+          }
+          *dst = v;
         }
         __syncwarp();
       }
@@ -893,18 +909,20 @@ cudaError_t launch_bwd_stages(const BwdMaps& m, const BwdPreArgs& pre, const Bwd
     return cudaErrorInvalidValue;
   cudaError_t e = launch_bwd_pre<D>(pre, num_sms, stream);
   if (e != cudaSuccess) return e;
-  const int grid_kv = a.kv_sched.pairs < num_sms ? a.kv_sched.pairs : num_sms;
-  prof_before(stream, kKernelBwdDkDv);
-  s2_bwd_dkdv_kernel<D, NST><<<grid_kv, K3::THREADS, K3::SMEM_BYTES, stream>>>(m.q64, m.k128, m.v128, m.g64, a);
-  e = cudaGetLastError();
-  prof_after(stream);
-  if (e != cudaSuccess) return e;
+  if (!a.no_dkdv) {
+    const int grid_kv = a.kv_sched.pairs < num_sms ? a.kv_sched.pairs : num_sms;
+    prof_before(stream, kKernelBwdDkDv);
+    s2_bwd_dkdv_kernel<D, NST><<<grid_kv, K3::THREADS, K3::SMEM_BYTES, stream>>>(m.q64, m.k128, m.v128, m.g64, a);
+    e = cudaGetLastError();
+    prof_after(stream);
+    if (e != cudaSuccess) return e;
+  }
   const int grid_q = a.q_sched.pairs < num_sms ? a.q_sched.pairs : num_sms;
   prof_before(stream, kKernelBwdDq);
   s2_bwd_dq_kernel<D, NST><<<grid_q, K4::THREADS, K4::SMEM_BYTES, stream>>>(m.q128, m.k64, m.v64, m.g128, a);
   e = cudaGetLastError();
   prof_after(stream);
-  if (launches) *launches = 3;
+  if (launches) *launches = a.no_dkdv ? 2 : 3;
   return e;
 }
 

@@ -179,7 +179,7 @@ __global__ void __launch_bounds__(384, 1)
       const int sh = shift_of_head(d, w.h);
       const int nq = 2 * (d.tiles - w.tile);
       const int iters = d.rep * nq;
-      const int tk0 = original_row(d, w.g * d.G + w.tile * kTile, sh);
+      const int tk0 = original_row_kv(d, w.g * d.G + w.tile * kTile, sh);
       // the item's first stages need only free stages, not the new K / V
       const int pre = iters < ST ? iters : ST;
       for (int it = 0; ok && it < pre; ++it) ok = load_stage(w, sh, it, nq);

@@ -25,6 +25,11 @@ struct Dims {
   int rep;        // H / Hkv, query heads per kv-head
   int n_groups;   // N / G
   int tiles;      // G / 128, tiles per group
+  // Segment mode (chunk-wise attention over detached earlier keys): the key
+  // tensors hold Nk rows and the N query rows sit at key position
+  // qoff_t * 128 onwards; causal = 1: query row i sees keys [0, qoff_t*128 + i],
+  // causal = 0: every key.  S2 attention: Nk = N, qoff_t = 0, causal = 1.
+  int Nk, qoff_t, causal;
 };
 
 __host__ __device__ __forceinline__ int shift_of_head(const Dims& d, int h) {
@@ -35,6 +40,12 @@ __host__ __device__ __forceinline__ int shift_of_head(const Dims& d, int h) {
 __host__ __device__ __forceinline__ int original_row(const Dims& d, int r, int s) {
   int t = r + s;
   return t >= d.N ? t - d.N : t;
+}
+
+// Key row of rolled key row r for a head with shift s (the key tensors hold Nk rows).
+__host__ __device__ __forceinline__ int original_row_kv(const Dims& d, int r, int s) {
+  int t = r + s;
+  return t >= d.Nk ? t - d.Nk : t;
 }
 
 // A work item: one 128-row tile of one rolled group of one (batch, head).
@@ -224,12 +235,14 @@ struct FwdCursor {
 };
 
 // One forward item: query tiles ta = 2i (always) and ta + 1 (if it exists),
-// key/value tiles 0 .. nkv-1 of the same rolled group.
+// key/value tiles 0 .. nkv-1 of the same rolled group; lastA / lastB: the
+// last key tile of tile A / B (its diagonal when causal), -1 if no tile B.
 struct FwdItem {
   int b, h, kvh, g, sh;
   int ta;
   bool has_b;
   int nkv;
+  int lastA, lastB;
 };
 
 __device__ __forceinline__ FwdItem fwd_item(const Dims& d, int unit, int i) {
@@ -242,7 +255,10 @@ __device__ __forceinline__ FwdItem fwd_item(const Dims& d, int unit, int i) {
   it.sh = shift_of_head(d, w.h);
   it.ta = 2 * i;
   it.has_b = 2 * i + 1 < d.tiles;
-  it.nkv = it.has_b ? 2 * i + 2 : 2 * i + 1;
+  const int nkt = d.Nk / kTile;
+  it.lastA = d.causal ? it.ta + d.qoff_t : nkt - 1;
+  it.lastB = it.has_b ? (d.causal ? it.ta + 1 + d.qoff_t : nkt - 1) : -1;
+  it.nkv = (it.has_b ? it.lastB : it.lastA) + 1;
   return it;
 }
 
@@ -275,6 +291,8 @@ struct BwdArgs {
   const float* ndelta;     // fp32 [B, H, N]: -Delta
   const float* nlse2;      // fp32 [B, H, N]: -lse * log2(e)
   void* dq;                // bf16 [B, N, H, D]
+  int dq_accumulate;       // split path: dq += the result instead of dq = (segment pieces)
+  int no_dkdv;             // split path: skip dK / dV (a detached key segment: dq only)
   float* dqacc;            // fused path: fp32 [B, H, N, D] dQ accumulator (zeroed by the preprocess)
   void* dk;                // bf16 [B, N, Hkv, D]
   void* dv;                // bf16 [B, N, Hkv, D]

@@ -165,7 +165,7 @@ __global__ void __launch_bounds__(320, 1)
     auto load_kv = [&](const FwdItem& it, int j, bool is_v) -> bool {
       const int s = L % NS, r = L / NS;
       if (r > 0 && !warp_wait(smem_u32(&bar_empty[s]), (r - 1) & 1, wc, 11)) return false;
-      const int row = original_row(d, it.g * d.G + j * kTile, it.sh);
+      const int row = original_row_kv(d, it.g * d.G + j * kTile, it.sh);
       if (elect_one()) {
         mbar_arrive_expect_tx(smem_u32(&bar_full[s]), C::TILE_BYTES);
         for (int c = 0; c < D / 64; ++c)
@@ -285,7 +285,7 @@ __global__ void __launch_bounds__(320, 1)
       const FwdItem itn = fwd_item(d, nx.valid ? nx.unit : cur.unit, nx.valid ? nx.i : cur.i);
       const int uA = 2 * n, uB = uA + 1, sA = uA % NQ, sB = uB % NQ;
       const int sAn = (uA + 2) % NQ, sBn = (uB + 2) % NQ;  // the next item's Q slots
-      const int lastA = it.ta, lastB = it.has_b ? it.ta + 1 : -1;
+      const int lastA = it.lastA, lastB = it.lastB;
       const int L0 = L;  // K_j is load L0 + 2j, V_j load L0 + 2j + 1
       const int L0n = L0 + 2 * it.nkv;
       if (!pre) {
@@ -373,9 +373,10 @@ __global__ void __launch_bounds__(320, 1)
     while (ok && cur.valid) {
       const FwdItem it = fwd_item(d, cur.unit, cur.i);
       const int t = it.ta + wg;
+      const int jlast = wg == 0 ? it.lastA : it.lastB;  // the diagonal key tile when causal
       if (wg == 0 || it.has_b) {
         float m_run = 0.f, l_run = 0.f;
-        for (int j = 0; j <= t; ++j) {
+        for (int j = 0; j <= jlast; ++j) {
           if (lane == 0) ok = mbar_wait(smem_u32(&bar_s[wg]), ns & 1, wc, 30);
           ok = __shfl_sync(0xffffffffu, ok, 0);
           if (!ok) break;
@@ -385,7 +386,7 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
           for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr[c]);
           tmem_wait_ld();
-          if (j == t) {  // diagonal tile: keys after the query are masked
+          if (d.causal && j == jlast) {  // diagonal tile: keys after the query are masked
 #pragma unroll
             for (int c = 0; c < 128; ++c)
               if (c > row) sr[c >> 5][c & 31] = __float_as_uint(neg_inf());

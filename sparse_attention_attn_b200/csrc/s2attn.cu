@@ -30,6 +30,8 @@ cudaError_t launch_rope_table(float* table, int N, int D, double pos_scale, doub
                               cudaStream_t stream);
 cudaError_t launch_rope_apply(const void* x, void* out, const float* table, int B, int N, int heads, int D,
                               int inverse, int num_sms, cudaStream_t stream);
+cudaError_t launch_lse_merge(const void* oa, const float* la, const void* ob, const float* lb, void* o, float* lse,
+                             int B, int H, int N, int D, int num_sms, cudaStream_t stream);
 }  // namespace s2
 
 namespace {
@@ -134,6 +136,29 @@ Dims make_dims(int B, int H, int Hkv, int N, int D, int G) {
   d.rep = H / Hkv;
   d.n_groups = N / G;
   d.tiles = G / kTile;
+  d.Nk = N;
+  d.qoff_t = 0;
+  d.causal = 1;
+  return d;
+}
+
+// Segment mode (chunk-wise attention): N query rows over Nk key rows, one
+// group, no shift; causal: query row i sees keys [0, Nk - N + i].
+int validate_segment(int B, int H, int Hkv, int N, int Nk, int D, int causal) {
+  if (B <= 0 || H <= 0 || Hkv <= 0 || N <= 0 || Nk <= 0 || D <= 0) return S2ATTN_ERR_INVALID_ARG;
+  if (H % Hkv != 0 || (causal && Nk < N)) return S2ATTN_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return S2ATTN_ERR_UNSUPPORTED;
+  if (N % kTile != 0 || Nk % kTile != 0) return S2ATTN_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * H * (N / kTile) > (1LL << 30)) return S2ATTN_ERR_UNSUPPORTED;
+  if (static_cast<long long>(Nk) * H * D >= (1LL << 40)) return S2ATTN_ERR_UNSUPPORTED;
+  return S2ATTN_OK;
+}
+
+Dims make_segment_dims(int B, int H, int Hkv, int N, int Nk, int D, int causal) {
+  Dims d = make_dims(B, H, Hkv, N, D, N);  // one group of N rows, no shift
+  d.Nk = Nk;
+  d.qoff_t = causal ? (Nk - N) / kTile : 0;
+  d.causal = causal ? 1 : 0;
   return d;
 }
 
@@ -288,6 +313,37 @@ struct ProfState {
 };
 thread_local ProfState g_prof;
 
+// The forward of a validated shape (S2 attention or a segment).
+int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, const Dims& dims,
+             s2attn_stream_t stream) {
+  const int B = dims.B, H = dims.H, Hkv = dims.Hkv, N = dims.N, D = dims.D, G = dims.G;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return S2ATTN_ERR_MISALIGNED;
+  DeviceInfo info;
+  if (!device_info(&info)) return S2ATTN_ERR_CUDA;
+  if (!info.ok) return S2ATTN_ERR_UNSUPPORTED;
+  CUtensorMap tq, tk, tv, to;
+  if (!make_map(&tq, q, B, N, H, D) || !make_map(&tk, k, B, dims.Nk, Hkv, D) ||
+      !make_map(&tv, v, B, dims.Nk, Hkv, D) || !make_map(&to, o, B, N, H, D, 32))
+    return S2ATTN_ERR_CUDA;
+  FwdArgs a;
+  a.d = dims;
+  const Plan plan = select_plan(B, H, Hkv, N, D, G, info.sms);
+  a.sched = make_fwd_sched(a.d, plan.fwd_snake);
+  a.scale_log2 = static_cast<float>(1.4426950408889634 / __builtin_sqrt(static_cast<double>(D)));
+  a.lse = lse;  // o is written through its TMA map
+  void* status = nullptr;
+  if (cudaGetSymbolAddress(&status, g_fwd_status) != cudaSuccess) return S2ATTN_ERR_CUDA;
+  a.status = static_cast<uint32_t*>(status);
+  a.wait_limit_ns = wait_limit_ns();
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = (D == 64) ? launch_fwd<64>(tq, tk, tv, to, a, info.sms, s, plan.fwd_kv_slots)
+                             : launch_fwd<128>(tq, tk, tv, to, a, info.sms, s, plan.fwd_kv_slots);
+  if (e != cudaSuccess) return S2ATTN_ERR_CUDA;
+  g_last_launches = 1;
+  return S2ATTN_OK;
+}
+
 }  // namespace
 
 namespace s2 {
@@ -370,44 +426,37 @@ int s2attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   if (!q || !k || !v || !o || !lse) return S2ATTN_ERR_INVALID_ARG;
   int st = validate_shape(B, H, Hkv, N, D, G);
   if (st != S2ATTN_OK) return st;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
-    return S2ATTN_ERR_MISALIGNED;
-  DeviceInfo info;
-  if (!device_info(&info)) return S2ATTN_ERR_CUDA;
-  if (!info.ok) return S2ATTN_ERR_UNSUPPORTED;
-  CUtensorMap tq, tk, tv, to;
-  if (!make_map(&tq, q, B, N, H, D) || !make_map(&tk, k, B, N, Hkv, D) ||
-      !make_map(&tv, v, B, N, Hkv, D) || !make_map(&to, o, B, N, H, D, 32))
-    return S2ATTN_ERR_CUDA;
-  FwdArgs a;
-  a.d = make_dims(B, H, Hkv, N, D, G);
-  const Plan plan = select_plan(B, H, Hkv, N, D, G, info.sms);
-  a.sched = make_fwd_sched(a.d, plan.fwd_snake);
-  a.scale_log2 = static_cast<float>(1.4426950408889634 / __builtin_sqrt(static_cast<double>(D)));
-  a.lse = lse;  // o is written through its TMA map
-  void* status = nullptr;
-  if (cudaGetSymbolAddress(&status, g_fwd_status) != cudaSuccess) return S2ATTN_ERR_CUDA;
-  a.status = static_cast<uint32_t*>(status);
-  a.wait_limit_ns = wait_limit_ns();
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = (D == 64) ? launch_fwd<64>(tq, tk, tv, to, a, info.sms, s, plan.fwd_kv_slots)
-                             : launch_fwd<128>(tq, tk, tv, to, a, info.sms, s, plan.fwd_kv_slots);
-  if (e != cudaSuccess) return S2ATTN_ERR_CUDA;
-  g_last_launches = 1;
-  return S2ATTN_OK;
+  return fwd_impl(q, k, v, o, lse, make_dims(B, H, Hkv, N, D, G), stream);
 }
 
+int s2attn_seg_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv,
+                   int N, int Nk, int D, int causal, s2attn_stream_t stream) {
+  g_last_launches = 0;
+  if (!q || !k || !v || !o || !lse) return S2ATTN_ERR_INVALID_ARG;
+  int st = validate_segment(B, H, Hkv, N, Nk, D, causal);
+  if (st != S2ATTN_OK) return st;
+  return fwd_impl(q, k, v, o, lse, make_segment_dims(B, H, Hkv, N, Nk, D, causal), stream);
+}
 }  // extern "C"
 
 namespace {
-// The backward on `path` (kBwdSplit or kBwdFused).
+// The backward on `path` (kBwdSplit or kBwdFused).  `seg`: segment-mode
+// dimensions (chunk-wise attention; split path only), or null for S2
+// attention of (B, H, Hkv, N, D, G).  Segment mode with causal = 0 computes dq
+// only (dk = dv = null: a detached key segment); dq_accumulate adds the
+// result to dq.
 int bwd_impl(int path, int stages, const void* q, const void* k, const void* v, const void* o, const float* lse,
              const void* dO, void* dq, void* dk, void* dv, int B, int H, int Hkv, int N, int D, int G,
-             void* workspace, size_t workspace_bytes, s2attn_stream_t stream, const float* rope = nullptr) {
+             void* workspace, size_t workspace_bytes, s2attn_stream_t stream, const float* rope = nullptr,
+             const Dims* seg = nullptr, int dq_accumulate = 0) {
   g_last_launches = 0;
-  if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return S2ATTN_ERR_INVALID_ARG;
-  int st = validate_shape(B, H, Hkv, N, D, G);
-  if (st != S2ATTN_OK) return st;
+  const bool dq_only = seg != nullptr && !seg->causal;
+  if (!q || !k || !v || !o || !lse || !dO || !dq) return S2ATTN_ERR_INVALID_ARG;
+  if (dq_only ? (dk != nullptr || dv != nullptr) : (!dk || !dv)) return S2ATTN_ERR_INVALID_ARG;
+  if (seg == nullptr) {
+    const int st = validate_shape(B, H, Hkv, N, D, G);
+    if (st != S2ATTN_OK) return st;
+  }
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
       !aligned16(dO) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
     return S2ATTN_ERR_MISALIGNED;
@@ -417,11 +466,13 @@ int bwd_impl(int path, int stages, const void* q, const void* k, const void* v, 
   DeviceInfo info;
   if (!device_info(&info)) return S2ATTN_ERR_CUDA;
   if (!info.ok) return S2ATTN_ERR_UNSUPPORTED;
+  const Dims d = seg ? *seg : make_dims(B, H, Hkv, N, D, G);
+  const int Nk = d.Nk;
   BwdMaps maps;
-  if (!make_map(&maps.q128, q, B, N, H, D) || !make_map(&maps.k128, k, B, N, Hkv, D) ||
-      !make_map(&maps.v128, v, B, N, Hkv, D) || !make_map(&maps.g128, dO, B, N, H, D) ||
-      !make_map(&maps.q64, q, B, N, H, D, 64) || !make_map(&maps.k64, k, B, N, Hkv, D, 64) ||
-      !make_map(&maps.v64, v, B, N, Hkv, D, 64) || !make_map(&maps.g64, dO, B, N, H, D, 64))
+  if (!make_map(&maps.q128, q, B, N, H, D) || !make_map(&maps.k128, k, B, Nk, Hkv, D) ||
+      !make_map(&maps.v128, v, B, Nk, Hkv, D) || !make_map(&maps.g128, dO, B, N, H, D) ||
+      !make_map(&maps.q64, q, B, N, H, D, 64) || !make_map(&maps.k64, k, B, Nk, Hkv, D, 64) ||
+      !make_map(&maps.v64, v, B, Nk, Hkv, D, 64) || !make_map(&maps.g64, dO, B, N, H, D, 64))
     return S2ATTN_ERR_CUDA;
   unsigned char* ws = static_cast<unsigned char*>(workspace);
   uint32_t* status = reinterpret_cast<uint32_t*>(ws);
@@ -429,7 +480,6 @@ int bwd_impl(int path, int stages, const void* q, const void* k, const void* v, 
   float* nlse2 = reinterpret_cast<float*>(ws + kStatusBytes + rowstat_bytes(B, H, N));
   float* dqacc = path == kBwdFused ? reinterpret_cast<float*>(ws + kStatusBytes + 2 * rowstat_bytes(B, H, N))
                                    : nullptr;
-  const Dims d = make_dims(B, H, Hkv, N, D, G);
   BwdPreArgs pre;
   pre.d = d;
   pre.o = o;
@@ -448,6 +498,8 @@ int bwd_impl(int path, int stages, const void* q, const void* k, const void* v, 
   a.ndelta = ndelta;
   a.nlse2 = nlse2;
   a.dq = dq;
+  a.dq_accumulate = dq_accumulate ? 1 : 0;
+  a.no_dkdv = dq_only ? 1 : 0;
   a.dqacc = dqacc;
   a.dk = dk;
   a.dv = dv;
@@ -553,6 +605,42 @@ int s2attn_bwd_rope(const void* q_rot, const void* k_rot, const void* v, const v
   const Plan plan = select_plan(B, H, Hkv, N, D, G, 0);
   return bwd_impl(plan.bwd_path, plan.bwd_stages, q_rot, k_rot, v, o, lse, dO, dq, dk, dv, B, H, Hkv, N, D, G,
                   workspace, workspace_bytes, stream, table);
+}
+
+size_t s2attn_seg_bwd_workspace_bytes(int B, int H, int Hkv, int N, int Nk, int D) {
+  if (validate_segment(B, H, Hkv, N, Nk, D, 0) != S2ATTN_OK) return 0;
+  return workspace_bytes_for(kBwdSplit, B, H, N, D);
+}
+
+int s2attn_seg_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                   void* dq, void* dk, void* dv, int B, int H, int Hkv, int N, int Nk, int D, int causal,
+                   int dq_accumulate, void* workspace, size_t workspace_bytes, s2attn_stream_t stream) {
+  g_last_launches = 0;
+  const int st = validate_segment(B, H, Hkv, N, Nk, D, causal);
+  if (st != S2ATTN_OK) return st;
+  const Dims d = make_segment_dims(B, H, Hkv, N, Nk, D, causal);
+  const Plan plan = select_plan(B, H, Hkv, N, D, N, 0);
+  return bwd_impl(kBwdSplit, plan.bwd_stages, q, k, v, o, lse, dO, dq, dk, dv, B, H, Hkv, N, D, N, workspace,
+                  workspace_bytes, stream, nullptr, &d, dq_accumulate);
+}
+
+int s2attn_lse_merge(const void* o_a, const float* lse_a, const void* o_b, const float* lse_b, void* o, float* lse,
+                     int B, int H, int N, int D, s2attn_stream_t stream) {
+  g_last_launches = 0;
+  if (!o_a || !lse_a || !o_b || !lse_b || !o || !lse || B <= 0 || H <= 0 || N <= 0) return S2ATTN_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return S2ATTN_ERR_UNSUPPORTED;
+  if (N % kTile != 0 || static_cast<long long>(B) * N * H * D >= (1LL << 40)) return S2ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(o_a) || !aligned16(o_b) || !aligned16(o) || !aligned16(lse_a) || !aligned16(lse_b) ||
+      !aligned16(lse))
+    return S2ATTN_ERR_MISALIGNED;
+  DeviceInfo info;
+  if (!device_info(&info)) return S2ATTN_ERR_CUDA;
+  if (!info.ok) return S2ATTN_ERR_UNSUPPORTED;
+  if (launch_lse_merge(o_a, lse_a, o_b, lse_b, o, lse, B, H, N, D, info.sms, static_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
+    return S2ATTN_ERR_CUDA;
+  g_last_launches = 1;
+  return S2ATTN_OK;
 }
 
 int s2attn_plan(int B, int H, int Hkv, int N, int D, int G, int num_sms, int* out) {
