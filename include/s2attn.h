@@ -268,6 +268,14 @@ S2ATTN_API int s2attn_selftest_wait_timeout(uint32_t* status_out, uint64_t limit
 S2ATTN_API int s2attn_last_launch_count(void);
 
 /*
+ * Diagnosis of S2ATTN_ERR_CUDA: the last CUDA runtime error code behind one
+ * on this host thread (or minus the driver's result when a TMA tensor map
+ * could not be encoded; 0 if none), and a static description of such a code.
+ */
+S2ATTN_API int s2attn_last_cuda_error(void);
+S2ATTN_API const char* s2attn_cuda_error_string(int err);
+
+/*
  * Optional per-kernel timing for benchmarks (not part of the operation).
  * s2attn_profile_start creates 2 * max_launches CUDA events (no device memory)
  * and makes the following fwd/bwd calls on this host thread record one event

@@ -33,6 +33,8 @@ SIGNATURES = {
     "s2attn_status_string": (ctypes.c_char_p, [_i]),
     "s2attn_selftest_wait_timeout": (_i, [_vp, ctypes.c_uint64, _vp]),
     "s2attn_last_launch_count": (_i, []),
+    "s2attn_last_cuda_error": (_i, []),
+    "s2attn_cuda_error_string": (ctypes.c_char_p, [_i]),
     "s2attn_profile_start": (_i, [_i]),
     "s2attn_profile_stop": (_i, [_vp, _vp, _i]),
     "s2attn_set_tile_override": (_i, [ctypes.c_char_p]),
@@ -58,7 +60,11 @@ _lib = None
 class S2AttnError(RuntimeError):
     def __init__(self, fn: str, status: int):
         self.status = status
-        super().__init__(f"{fn} failed: {status_string(status)} ({status})")
+        msg = f"{fn} failed: {status_string(status)} ({status})"
+        if status == S2ATTN_ERR_CUDA:
+            err = load().s2attn_last_cuda_error()
+            msg += f"; CUDA: {load().s2attn_cuda_error_string(err).decode()} ({err})"
+        super().__init__(msg)
 
 
 def load() -> ctypes.CDLL:

@@ -41,6 +41,9 @@ using namespace s2;
 __device__ uint32_t g_fwd_status[4];  // [0] error code, [1] where
 
 thread_local int g_last_launches = 0;
+// The last CUDA runtime error (or -(driver result) of a tensor-map encoding)
+// behind an S2ATTN_ERR_CUDA on this host thread, for diagnosis.
+thread_local int g_last_cuda_error = 0;
 
 constexpr size_t kStatusBytes = 256;
 
@@ -80,7 +83,11 @@ bool device_info(DeviceInfo* out) {
   static DeviceInfo cache[64];
   static bool known[64] = {};
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  const cudaError_t ge = cudaGetDevice(&dev);
+  if (ge != cudaSuccess || dev < 0 || dev >= 64) {
+    g_last_cuda_error = static_cast<int>(ge);
+    return false;
+  }
   std::lock_guard<std::mutex> lk(mu);
   if (!known[dev]) {
     int major = 0, minor = 0, sms = 0;
@@ -257,16 +264,21 @@ FwdSched make_fwd_sched(const Dims& d, int snake) {
 // box_rows x 64-column slab, 128-byte swizzle (the UMMA operand layout).
 bool make_map(CUtensorMap* m, const void* base, int B, int N, int heads, int D, int box_rows = kTile) {
   EncodeTiledFn enc = get_encode();
-  if (!enc) return false;
+  if (!enc) {
+    g_last_cuda_error = -1;
+    return false;
+  }
   cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(heads),
                         static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(B)};
   cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(heads) * D * 2,
                            static_cast<cuuint64_t>(N) * heads * D * 2};
   cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(box_rows), 1};
   cuuint32_t es[4] = {1, 1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) g_last_cuda_error = -static_cast<int>(r);
+  return r == CUDA_SUCCESS;
 }
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -333,13 +345,20 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, c
   a.scale_log2 = static_cast<float>(1.4426950408889634 / __builtin_sqrt(static_cast<double>(D)));
   a.lse = lse;  // o is written through its TMA map
   void* status = nullptr;
-  if (cudaGetSymbolAddress(&status, g_fwd_status) != cudaSuccess) return S2ATTN_ERR_CUDA;
+  const cudaError_t se = cudaGetSymbolAddress(&status, g_fwd_status);
+  if (se != cudaSuccess) {
+    g_last_cuda_error = static_cast<int>(se);
+    return S2ATTN_ERR_CUDA;
+  }
   a.status = static_cast<uint32_t*>(status);
   a.wait_limit_ns = wait_limit_ns();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = (D == 64) ? launch_fwd<64>(tq, tk, tv, to, a, info.sms, s, plan.fwd_kv_slots)
                              : launch_fwd<128>(tq, tk, tv, to, a, info.sms, s, plan.fwd_kv_slots);
-  if (e != cudaSuccess) return S2ATTN_ERR_CUDA;
+  if (e != cudaSuccess) {
+    g_last_cuda_error = static_cast<int>(e);
+    return S2ATTN_ERR_CUDA;
+  }
   g_last_launches = 1;
   return S2ATTN_OK;
 }
@@ -414,6 +433,13 @@ const char* s2attn_status_string(int status) {
 }
 
 int s2attn_last_launch_count(void) { return g_last_launches; }
+
+int s2attn_last_cuda_error(void) { return g_last_cuda_error; }
+
+const char* s2attn_cuda_error_string(int err) {
+  if (err < 0) return "tensor-map encoding failed (minus the driver result)";
+  return cudaGetErrorString(static_cast<cudaError_t>(err));
+}
 
 size_t s2attn_bwd_workspace_bytes(int B, int H, int Hkv, int N, int D, int G) {
   if (validate_shape(B, H, Hkv, N, D, G) != S2ATTN_OK) return 0;
@@ -522,6 +548,7 @@ int bwd_impl(int path, int stages, const void* q, const void* k, const void* v, 
     launches += 2;
   }
   g_last_launches = launches;
+  if (e != cudaSuccess) g_last_cuda_error = static_cast<int>(e);
   return e == cudaSuccess ? S2ATTN_OK : S2ATTN_ERR_CUDA;
 }
 

@@ -334,3 +334,19 @@ def test_binding_rejects_bad_operands():
     assert s2.device_status() == 0
     o_ref, _ = ref.s2_attention_fwd(to64(q), to64(k), to64(v), shape.G)
     assert rel_fro(to64(o), o_ref) <= 5e-3
+
+
+def test_autograd_wrapper_matches_direct_calls():
+    """S2Attention through torch autograd (its backward runs on autograd's
+    worker thread) gives the direct calls' results bit for bit."""
+    import sparse_attention_attn_b200 as s2
+    shape = I.Shape("autograd", 1, 4, 2, 128, 1024, 256)
+    q, k, v, do = (t.to("cuda:0") for t in I.make_inputs(shape, seed_offset=9))
+    o_ref, lse = s2.s2attn_forward(q, k, v, shape.G)
+    dq_ref, dk_ref, dv_ref = s2.s2attn_backward(q, k, v, o_ref, lse, do, shape.G)
+    qt, kt, vt = (t.clone().requires_grad_(True) for t in (q, k, v))
+    o = s2.s2_attn(qt, kt, vt, shape.G)
+    o.backward(do)
+    torch.cuda.synchronize()
+    assert torch.equal(o.detach(), o_ref)
+    assert torch.equal(qt.grad, dq_ref) and torch.equal(kt.grad, dk_ref) and torch.equal(vt.grad, dv_ref)

@@ -143,3 +143,19 @@ def test_llama2_7b_8k_sampled():
 def test_100k_sampled(s):
     shape = I.LLAMA2_7B_100K
     _check_full_size(shape, s, 1024, [(0, shape.H - 1, shape.N // shape.G - 1)])
+
+
+def test_autograd_wrapper_matches_direct_calls():
+    """S2RopeAttention through torch autograd equals the direct calls."""
+    import sparse_attention_attn_b200 as s2
+    shape = I.Shape("rope-ag", 1, 4, 2, 128, 1024, 256)
+    q, k, v, do = (t.to("cuda:0") for t in I.make_inputs(shape, seed_offset=19))
+    tab = s2.rope_table(shape.N, shape.D, 0.5)
+    o_ref, lse, qr, kr = s2.s2attn_forward_rope(q, k, v, shape.G, tab)
+    dq_ref, dk_ref, dv_ref = s2.s2attn_backward_rope(qr, kr, v, o_ref, lse, do, shape.G, tab)
+    qt, kt, vt = (t.clone().requires_grad_(True) for t in (q, k, v))
+    o = s2.S2RopeAttention.apply(qt, kt, vt, shape.G, tab)
+    o.backward(do)
+    torch.cuda.synchronize()
+    assert torch.equal(o.detach(), o_ref)
+    assert torch.equal(qt.grad, dq_ref) and torch.equal(kt.grad, dk_ref) and torch.equal(vt.grad, dv_ref)
