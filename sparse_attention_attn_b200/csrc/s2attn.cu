@@ -83,7 +83,12 @@ bool device_info(DeviceInfo* out) {
   static DeviceInfo cache[64];
   static bool known[64] = {};
   int dev = 0;
-  const cudaError_t ge = cudaGetDevice(&dev);
+  cudaError_t ge = cudaGetDevice(&dev);
+  // bind the device's primary context to this host thread: the TMA
+  // descriptors are encoded through the driver API, which needs a current
+  // context, and a thread that has made no runtime call yet (e.g. an autograd
+  // worker running a backward) may have none
+  if (ge == cudaSuccess) ge = cudaSetDevice(dev);
   if (ge != cudaSuccess || dev < 0 || dev >= 64) {
     g_last_cuda_error = static_cast<int>(ge);
     return false;
