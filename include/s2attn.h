@@ -219,6 +219,34 @@ S2ATTN_API int s2attn_seg_bwd(const void* q, const void* k, const void* v, const
 S2ATTN_API int s2attn_lse_merge(const void* o_a, const float* lse_a, const void* o_b, const float* lse_b, void* o,
                                 float* lse, int B, int H, int N, int D, s2attn_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * HGA-style block-sparse attention over gathered history (HGA digest, arXiv
+ * 2607.15105: each query block loads a bounded set of exact historical tokens;
+ * only the active segment stays differentiable).  The sequence is cut into
+ * segments of G rows (G % 256 == 0, N % G == 0; no head is shifted); a query
+ * row attends its own segment's keys causally plus the historical key tiles
+ * listed for its 256-row query block: hist is a device int32 [B, N/256, S]
+ * array of 128-row key tile indices (tile e = key rows [128 e, 128 e + 128)),
+ * shared by all heads.  A block uses its leading entries that name a tile of
+ * an EARLIER segment (0 <= e < segment start / 128); the first other entry
+ * (e.g. -1) ends its list.  Tensors, scale and lse as in s2attn_fwd.
+ * ------------------------------------------------------------------------ */
+S2ATTN_API int s2attn_hga_fwd(const void* q, const void* k, const void* v, void* o, float* lse, const int* hist,
+                              int S, int B, int H, int Hkv, int N, int D, int G, s2attn_stream_t stream);
+
+/* Workspace bytes of s2attn_hga_bwd. */
+S2ATTN_API size_t s2attn_hga_bwd_workspace_bytes(int B, int H, int Hkv, int N, int D, int G);
+
+/*
+ * Backward of s2attn_hga_fwd: dq through every key a row attends; dk, dv
+ * through the local (same-segment) attention only -- the historical keys are
+ * detached.  Split kernels (preprocess, dK/dV, dQ over the listed tiles too).
+ */
+S2ATTN_API int s2attn_hga_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                              const void* dO, void* dq, void* dk, void* dv, const int* hist, int S, int B, int H,
+                              int Hkv, int N, int D, int G, void* workspace, size_t workspace_bytes,
+                              s2attn_stream_t stream);
+
 /*
  * Backward for callers that cannot allocate device memory (no counterpart in
  * the papers: this is a deployment variant of s2attn_bwd).  Some callers have

@@ -43,6 +43,10 @@ SIGNATURES = {
     "s2attn_seg_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _vp,
                             ctypes.c_size_t, _vp]),
     "s2attn_lse_merge": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp]),
+    "s2attn_hga_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp]),
+    "s2attn_hga_bwd_workspace_bytes": (ctypes.c_size_t, [_i, _i, _i, _i, _i, _i]),
+    "s2attn_hga_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp,
+                            ctypes.c_size_t, _vp]),
     "s2attn_rope_table_bytes": (ctypes.c_size_t, [_i, _i]),
     "s2attn_rope_table": (_i, [_vp, _i, _i, ctypes.c_double, ctypes.c_double, _vp]),
     "s2attn_rope_apply": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
@@ -143,6 +147,20 @@ def s2attn_seg_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, Hkv, N, Nk, D, causal,
 
 def s2attn_lse_merge(o_a, lse_a, o_b, lse_b, o, lse, B, H, N, D, stream) -> int:
     return load().s2attn_lse_merge(o_a, lse_a, o_b, lse_b, o, lse, B, H, N, D, stream)
+
+
+def s2attn_hga_fwd(q, k, v, o, lse, hist, S, B, H, Hkv, N, D, G, stream) -> int:
+    return load().s2attn_hga_fwd(q, k, v, o, lse, hist, S, B, H, Hkv, N, D, G, stream)
+
+
+def s2attn_hga_bwd_workspace_bytes(B, H, Hkv, N, D, G) -> int:
+    return load().s2attn_hga_bwd_workspace_bytes(B, H, Hkv, N, D, G)
+
+
+def s2attn_hga_bwd(q, k, v, o, lse, dO, dq, dk, dv, hist, S, B, H, Hkv, N, D, G, workspace, workspace_bytes,
+                   stream) -> int:
+    return load().s2attn_hga_bwd(q, k, v, o, lse, dO, dq, dk, dv, hist, S, B, H, Hkv, N, D, G, workspace,
+                                 workspace_bytes, stream)
 
 
 def s2attn_rope_table_bytes(N, D) -> int:

@@ -297,6 +297,63 @@ def lse_merge(o_a, lse_a, o_b, lse_b, out=None, lse=None):
     return out, lse
 
 
+def _need_hist(hist, B, N, dev):
+    if not isinstance(hist, torch.Tensor) or hist.dtype != torch.int32 or hist.dim() != 3:
+        raise ValueError("hist must be an int32 tensor [B, N/256, S]")
+    if hist.device != dev or not hist.is_contiguous() or tuple(hist.shape[:2]) != (B, N // 256):
+        raise ValueError(f"hist must be a contiguous [B, N/256, S] tensor on {dev}")
+
+
+def hga_forward(q, k, v, group_size: int, hist, out=None, lse=None):
+    """HGA-style block-sparse attention: each row attends its own segment
+    (group_size rows, no shift) causally and the historical key tiles listed
+    for its 256-row query block in hist (int32 [B, N/256, S], tile indices of
+    earlier segments; a list ends at its first other entry, e.g. -1)."""
+    B, N, H, Hkv, D = _dims(q, k)
+    _need("q", q, (B, N, H, D))
+    dev = q.device
+    _need("k", k, (B, N, Hkv, D), device=dev)
+    _need("v", v, (B, N, Hkv, D), device=dev)
+    _need_hist(hist, B, N, dev)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev) if lse is None else lse
+    _need("out", out, (B, N, H, D), device=dev)
+    _need("lse", lse, (B, H, N), torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        st = _lib.s2attn_hga_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                 hist.data_ptr(), hist.shape[2], B, H, Hkv, N, D, int(group_size), _stream(dev))
+    _lib._check("s2attn_hga_fwd", st)
+    return out, lse
+
+
+def hga_backward(q, k, v, o, lse, do, group_size: int, hist, dq=None, dk=None, dv=None, workspace=None):
+    """Backward of hga_forward: dq through every attended key; dk, dv through
+    the local attention only (the historical keys are detached)."""
+    B, N, H, Hkv, D = _dims(q, k)
+    _need("q", q, (B, N, H, D))
+    dev = q.device
+    for name, t, shp in (("k", k, (B, N, Hkv, D)), ("v", v, (B, N, Hkv, D)), ("o", o, (B, N, H, D)),
+                         ("do", do, (B, N, H, D))):
+        _need(name, t, shp, device=dev)
+    _need("lse", lse, (B, H, N), torch.float32, device=dev)
+    _need_hist(hist, B, N, dev)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    wsb = _lib.s2attn_hga_bwd_workspace_bytes(B, H, Hkv, N, D, int(group_size))
+    if wsb == 0:
+        raise _lib.S2AttnError("s2attn_hga_bwd_workspace_bytes", _lib.S2ATTN_ERR_INVALID_ARG)
+    if workspace is None:
+        workspace = torch.empty(wsb, dtype=torch.uint8, device=dev)
+    with torch.cuda.device(dev):
+        st = _lib.s2attn_hga_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                 do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), hist.data_ptr(),
+                                 hist.shape[2], B, H, Hkv, N, D, int(group_size), workspace.data_ptr(),
+                                 workspace.numel() * workspace.element_size(), _stream(dev))
+    _lib._check("s2attn_hga_bwd", st)
+    return dq, dk, dv
+
+
 class ChunkAttention(torch.autograd.Function):
     """Chunk-wise training step: the chunk's queries attend its own keys
     causally and the detached earlier keys fully; the two pieces are merged by

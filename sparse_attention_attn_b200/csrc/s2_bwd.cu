@@ -505,22 +505,30 @@ struct DqCursor {
   ItemCursor ic;
   TileWork w;
   int it, iters;
-  __device__ __forceinline__ void load(const Dims& d) {
+  int nh;            // HGA mode: the query block's historical tiles (64-row sub-tiles j < 2 nh)
+  const int* hist;
+  __device__ __forceinline__ void load(const Dims& d, const HgaList& hl) {
     if (!ic.valid) return;
     w = q_item(d, ic.unit, ic.tile);
-    // 64-row kv sub-tiles from the group start to the diagonal (causal), or
-    // every key (segment mode, causal = 0)
-    iters = d.causal ? 2 * (w.tile + 1 + d.qoff_t) : 2 * (d.Nk / kTile);
+    nh = hga_count(d, hl, w.b, w.g, (w.g * d.G + w.tile * kTile) / kQBlock, &hist);
+    // 64-row kv sub-tiles: the listed historical tiles, then from the group
+    // start to the diagonal (causal), or every key (segment mode, causal = 0)
+    iters = d.causal ? 2 * (w.tile + 1 + d.qoff_t + nh) : 2 * (d.Nk / kTile);
     it = 0;
   }
-  __device__ __forceinline__ void first(const Dims& d, const PairSched& ps) {
+  __device__ __forceinline__ void first(const Dims& d, const PairSched& ps, const HgaList& hl) {
     ic.first(ps);
-    load(d);
+    load(d, hl);
   }
-  __device__ __forceinline__ void next(const Dims& d, const PairSched& ps) {
+  __device__ __forceinline__ void next(const Dims& d, const PairSched& ps, const HgaList& hl) {
     if (++it < iters) return;
     ic.next(ps);
-    load(d);
+    load(d, hl);
+  }
+  // key row of 64-row kv sub-tile j of this item
+  __device__ __forceinline__ int kv_row(const Dims& d, int j) const {
+    if (j < 2 * nh) return hist[j >> 1] * kTile + (j & 1) * kSub;
+    return original_row_kv(d, w.g * d.G + (j - 2 * nh) * kSub, shift_of_head(d, w.h));
   }
 };
 
@@ -588,9 +596,10 @@ __global__ void __launch_bounds__(384, 1)
     __syncwarp();
     int gi = 0, q_issued = 0;
     bool ok = true;
-    ItemCursor ic;
-    for (ic.first(ps); ok && ic.valid; ic.next(ps)) {
-      const TileWork w = q_item(d, ic.unit, ic.tile);
+    DqCursor pc;  // walks items only (it is left at 0)
+    for (pc.first(d, ps, a.hist); ok && pc.ic.valid; pc.ic.next(ps), pc.load(d, a.hist)) {
+      const ItemCursor& ic = pc.ic;
+      const TileWork w = pc.w;
       const int sh = shift_of_head(d, w.h);
       // the buffer is free once the previous item's Q / dO are in TMEM
       if (ic.n >= 1 && !warp_wait(smem_u32(&bar_q_empty), (ic.n - 1) & 1, wc, 209)) break;
@@ -604,14 +613,14 @@ __global__ void __launch_bounds__(384, 1)
       }
       __syncwarp();
       ++q_issued;
-      const int iters = d.causal ? 2 * (w.tile + 1 + d.qoff_t) : 2 * (d.Nk / kTile);
+      const int iters = pc.iters;
       for (int j = 0; j < iters; ++j, ++gi) {
         const int s = gi % ST, f = gi / ST;
         if (f > 0 && !warp_wait(smem_u32(&bar_empty[s]), (f - 1) & 1, wc, 210)) {
           ok = false;
           break;
         }
-        const int tk0 = original_row_kv(d, w.g * d.G + j * kSub, sh);
+        const int tk0 = pc.kv_row(d, j);
         const uint32_t bar = smem_u32(&bar_kv[s]);
         if (elect_one()) {
           mbar_arrive_expect_tx(bar, 2 * C::KV_BYTES);
@@ -686,11 +695,11 @@ __global__ void __launch_bounds__(384, 1)
       return true;
     };
     DqCursor cur;
-    cur.first(d, ps);
+    cur.first(d, ps, a.hist);
     bool ok = true;
     for (int g = 0; ok && cur.ic.valid; ++g) {
       ok = (role == 2) ? issue_dq(cur, g) : issue_sdp(cur, g);
-      cur.next(d, ps);
+      cur.next(d, ps, a.hist);
     }
     // every issued UMMA completes before TMEM is released
     if (elect_one()) {
@@ -752,7 +761,7 @@ __global__ void __launch_bounds__(384, 1)
       dl = a.ndelta[ridx];
     };
     DqCursor cur;
-    cur.first(d, ps);
+    cur.first(d, ps, a.hist);
     float nl_next = 0.f, nd_next = 0.f;  // the next item's, fetched one item ahead
     if (cur.ic.valid) {
       ok = put_q(cur);
@@ -766,7 +775,9 @@ __global__ void __launch_bounds__(384, 1)
         nd2 = f2_pack(nd_next, nd_next);
       }
       const uint32_t bo = (g & 1) * kSub + half * 32;
-      const int koff = cur.it * kSub - (w.tile + d.qoff_t) * kTile;  // kv sub-tile start minus query tile start
+      // kv sub-tile start minus query tile start (in the sub-tile walk: the
+      // historical tiles and the segment offset come first)
+      const int koff = cur.it * kSub - (w.tile + d.qoff_t + cur.nh) * kTile;
       if (lane == 0) ok = mbar_wait(smem_u32(&bar_sdp[g & 1]), (g >> 1) & 1, wc, 230);
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
@@ -775,7 +786,7 @@ __global__ void __launch_bounds__(384, 1)
         // this item's last S and dP are done with Q / dO in TMEM: bring in the
         // next item's, so its first S / dP overlap the dS work below
         DqCursor nq = cur;
-        nq.next(d, ps);
+        nq.next(d, ps, a.hist);
         if (nq.ic.valid) {
           if (!put_q(nq)) {
             ok = false;
@@ -862,7 +873,7 @@ __global__ void __launch_bounds__(384, 1)
         }
         __syncwarp();
       }
-      cur.next(d, ps);
+      cur.next(d, ps, a.hist);
     }
   }
 

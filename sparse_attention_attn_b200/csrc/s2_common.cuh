@@ -30,10 +30,39 @@ struct Dims {
   // qoff_t * 128 onwards; causal = 1: query row i sees keys [0, qoff_t*128 + i],
   // causal = 0: every key.  S2 attention: Nk = N, qoff_t = 0, causal = 1.
   int Nk, qoff_t, causal;
+  // HGA block-sparse mode: no head is shifted, and every 256-row query block
+  // also attends the historical 128-row key tiles listed for it (see HgaList)
+  int noshift;
 };
 
+// Historical key tiles selected per 256-row query block (HGA digest: each
+// query block loads a bounded set of exact historical tokens): int32
+// [B, N/256, S] tile indices.  A block uses its leading entries that name a
+// tile of an earlier segment (0 <= e < segment start / 128); the first entry
+// outside that range ends the list.  null: no history.
+struct HgaList {
+  const int* tiles = nullptr;
+  int S = 0;
+};
+
+constexpr int kQBlock = 256;  // query rows sharing one historical list
+
+// Number of historical tiles query block qb (in segment g) attends; *list
+// points at its entries.
+__host__ __device__ __forceinline__ int hga_count(const Dims& d, const HgaList& hl, int b, int g, int qb,
+                                                  const int** list) {
+  *list = nullptr;
+  if (hl.tiles == nullptr || hl.S <= 0) return 0;
+  const int* l = hl.tiles + (static_cast<size_t>(b) * (d.N / kQBlock) + qb) * hl.S;
+  const int lim = g * d.G / kTile;
+  int n = 0;
+  while (n < hl.S && l[n] >= 0 && l[n] < lim) ++n;
+  *list = l;
+  return n;
+}
+
 __host__ __device__ __forceinline__ int shift_of_head(const Dims& d, int h) {
-  return (d.G < d.N && h >= d.H / 2) ? d.G / 2 : 0;
+  return (d.G < d.N && h >= d.H / 2 && !d.noshift) ? d.G / 2 : 0;
 }
 
 // Original row of rolled row r for a head with shift s.
@@ -243,9 +272,11 @@ struct FwdItem {
   bool has_b;
   int nkv;
   int lastA, lastB;
+  int nh;          // historical tiles first (HGA mode): key tile j < nh is hist[j]
+  const int* hist;
 };
 
-__device__ __forceinline__ FwdItem fwd_item(const Dims& d, int unit, int i) {
+__device__ __forceinline__ FwdItem fwd_item(const Dims& d, int unit, int i, const HgaList& hl) {
   const TileWork w = q_item(d, unit, 2 * i);
   FwdItem it;
   it.b = w.b;
@@ -255,15 +286,18 @@ __device__ __forceinline__ FwdItem fwd_item(const Dims& d, int unit, int i) {
   it.sh = shift_of_head(d, w.h);
   it.ta = 2 * i;
   it.has_b = 2 * i + 1 < d.tiles;
+  it.nh = hga_count(d, hl, w.b, w.g, (w.g * d.G + it.ta * kTile) / kQBlock, &it.hist);
   const int nkt = d.Nk / kTile;
-  it.lastA = d.causal ? it.ta + d.qoff_t : nkt - 1;
-  it.lastB = it.has_b ? (d.causal ? it.ta + 1 + d.qoff_t : nkt - 1) : -1;
+  const int off = d.qoff_t + it.nh;
+  it.lastA = d.causal ? it.ta + off : nkt - 1;
+  it.lastB = it.has_b ? (d.causal ? it.ta + 1 + off : nkt - 1) : -1;
   it.nkv = (it.has_b ? it.lastB : it.lastA) + 1;
   return it;
 }
 
 struct FwdArgs {
   Dims d;
+  HgaList hist;            // HGA mode's historical tile lists (tiles = null otherwise)
   FwdSched sched;
   float scale_log2;        // (1/sqrt(D)) * log2(e)
   float* lse;              // fp32 [B, H, N]
@@ -284,6 +318,7 @@ struct BwdPreArgs {
 
 struct BwdArgs {
   Dims d;
+  HgaList hist;            // HGA mode (split path): historical tile lists for the dQ kernel
   PairSched kv_sched;      // dK/dV work items (units: batch x kv-head x group)
   PairSched q_sched;       // dQ work items (units: batch x head x group)
   float scale;             // 1/sqrt(D)

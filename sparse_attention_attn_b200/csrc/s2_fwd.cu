@@ -165,7 +165,8 @@ __global__ void __launch_bounds__(320, 1)
     auto load_kv = [&](const FwdItem& it, int j, bool is_v) -> bool {
       const int s = L % NS, r = L / NS;
       if (r > 0 && !warp_wait(smem_u32(&bar_empty[s]), (r - 1) & 1, wc, 11)) return false;
-      const int row = original_row_kv(d, it.g * d.G + j * kTile, it.sh);
+      // key tile j: a listed historical tile first (HGA mode), then the group's own
+      const int row = j < it.nh ? it.hist[j] * kTile : original_row_kv(d, it.g * d.G + (j - it.nh) * kTile, it.sh);
       if (elect_one()) {
         mbar_arrive_expect_tx(smem_u32(&bar_full[s]), C::TILE_BYTES);
         for (int c = 0; c < D / 64; ++c)
@@ -180,13 +181,13 @@ __global__ void __launch_bounds__(320, 1)
     cur.first(a.sched);
     bool ok = true;
     if (cur.valid) {
-      FwdItem it = fwd_item(d, cur.unit, cur.i);
+      FwdItem it = fwd_item(d, cur.unit, cur.i, a.hist);
       ok = load_q(it, it.ta, true) && load_q(it, it.ta + 1, it.has_b);
       bool qb_pending = false;  // this item's second Q tile is still to come
       while (ok && cur.valid) {
         FwdCursor nx = cur;
         nx.next(a.sched);
-        const FwdItem itn = fwd_item(d, nx.valid ? nx.unit : cur.unit, nx.valid ? nx.i : cur.i);
+        const FwdItem itn = fwd_item(d, nx.valid ? nx.unit : cur.unit, nx.valid ? nx.i : cur.i, a.hist);
         // The next item's first Q tile goes into the slot the previous item's
         // second tile freed: fetched once this item is under way.  An item's
         // second Q tile goes into the slot whose tile's O the epilogue stages
@@ -279,10 +280,10 @@ __global__ void __launch_bounds__(320, 1)
     cur.first(a.sched);
     bool ok = true;
     while (ok && cur.valid) {
-      const FwdItem it = fwd_item(d, cur.unit, cur.i);
+      const FwdItem it = fwd_item(d, cur.unit, cur.i, a.hist);
       FwdCursor nx = cur;
       nx.next(a.sched);
-      const FwdItem itn = fwd_item(d, nx.valid ? nx.unit : cur.unit, nx.valid ? nx.i : cur.i);
+      const FwdItem itn = fwd_item(d, nx.valid ? nx.unit : cur.unit, nx.valid ? nx.i : cur.i, a.hist);
       const int uA = 2 * n, uB = uA + 1, sA = uA % NQ, sB = uB % NQ;
       const int sAn = (uA + 2) % NQ, sBn = (uB + 2) % NQ;  // the next item's Q slots
       const int lastA = it.lastA, lastB = it.lastB;
@@ -371,7 +372,7 @@ __global__ void __launch_bounds__(320, 1)
     cur.first(a.sched);
     bool ok = true;
     while (ok && cur.valid) {
-      const FwdItem it = fwd_item(d, cur.unit, cur.i);
+      const FwdItem it = fwd_item(d, cur.unit, cur.i, a.hist);
       const int t = it.ta + wg;
       const int jlast = wg == 0 ? it.lastA : it.lastB;  // the diagonal key tile when causal
       if (wg == 0 || it.has_b) {

@@ -31,20 +31,25 @@ __global__ void __launch_bounds__(256) s2_rope_table_kernel(float2* table, int N
   }
 }
 
-// One thread per (batch, token, 8 pairs): the 8 (cos, sin) pairs of its token
-// stay in registers while it walks the heads; per head it reads 8 values of
-// each half of the row and writes the rotated 16.  `inverse` turns by -a.
-// x and out may be the same buffer.
+// One thread per (batch, token, 8 pairs, group of up to 4 heads): the 8
+// (cos, sin) pairs of its token stay in registers while it rotates its heads;
+// per head it reads 8 values of each half of the row and writes the rotated
+// 16.  `inverse` turns by -a.  x and out may be the same buffer.
 template <int D>
 __global__ void __launch_bounds__(256) s2_rope_apply_kernel(const __nv_bfloat16* x, __nv_bfloat16* out,
                                                             const float2* table, int B, int N, int heads,
                                                             int inverse) {
   constexpr int CH = D / 16;  // 8-pair chunks per head
-  const long long n = static_cast<long long>(B) * N * CH;
+  constexpr int HG = 4;       // heads per thread
+  const int ngrp = (heads + HG - 1) / HG;
+  const long long n = static_cast<long long>(B) * N * ngrp * CH;
   const float sg = inverse ? -1.f : 1.f;
   for (long long e = blockIdx.x * 256LL + threadIdx.x; e < n; e += static_cast<long long>(gridDim.x) * 256) {
-    const long long bt = e / CH;  // b * N + t
-    const int ch = static_cast<int>(e - bt * CH);
+    // consecutive threads: chunks of one head group, then the groups of a token
+    const int ch = static_cast<int>(e % CH);
+    const long long r = e / CH;
+    const int hg = static_cast<int>(r % ngrp);
+    const long long bt = r / ngrp;  // b * N + t
     const int t = static_cast<int>(bt % N);
     const float4* tp = reinterpret_cast<const float4*>(table + static_cast<size_t>(t) * (D / 2) + ch * 8);
     float c[8], s[8];
@@ -57,12 +62,21 @@ __global__ void __launch_bounds__(256) s2_rope_apply_kernel(const __nv_bfloat16*
       s[2 * j + 1] = v.w * sg;
     }
     const size_t row = static_cast<size_t>(bt) * heads * D;
-#pragma unroll 4
-    for (int h = 0; h < heads; ++h) {
-      const size_t o1 = row + static_cast<size_t>(h) * D + ch * 8, o2 = o1 + D / 2;
-      const uint4 u1 = *reinterpret_cast<const uint4*>(x + o1);
-      const uint4 u2 = *reinterpret_cast<const uint4*>(x + o2);
-      const uint32_t a1[4] = {u1.x, u1.y, u1.z, u1.w}, a2[4] = {u2.x, u2.y, u2.z, u2.w};
+    const int h0 = hg * HG, h1 = h0 + HG < heads ? h0 + HG : heads;
+    uint4 u1[HG], u2[HG];
+#pragma unroll
+    for (int k = 0; k < HG; ++k) {
+      if (h0 + k < h1) {
+        const size_t o1 = row + static_cast<size_t>(h0 + k) * D + ch * 8;
+        u1[k] = *reinterpret_cast<const uint4*>(x + o1);
+        u2[k] = *reinterpret_cast<const uint4*>(x + o1 + D / 2);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < HG; ++k) {
+      if (h0 + k >= h1) continue;
+      const size_t o1 = row + static_cast<size_t>(h0 + k) * D + ch * 8;
+      const uint32_t a1[4] = {u1[k].x, u1[k].y, u1[k].z, u1[k].w}, a2[4] = {u2[k].x, u2[k].y, u2[k].z, u2[k].w};
       uint32_t r1[4], r2[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
@@ -73,7 +87,7 @@ __global__ void __launch_bounds__(256) s2_rope_apply_kernel(const __nv_bfloat16*
         r2[j] = pack_bf16x2(fmaf(x1.x, s[k0], x2.x * c[k0]), fmaf(x1.y, s[k1], x2.y * c[k1]));
       }
       *reinterpret_cast<uint4*>(out + o1) = make_uint4(r1[0], r1[1], r1[2], r1[3]);
-      *reinterpret_cast<uint4*>(out + o2) = make_uint4(r2[0], r2[1], r2[2], r2[3]);
+      *reinterpret_cast<uint4*>(out + o1 + D / 2) = make_uint4(r2[0], r2[1], r2[2], r2[3]);
     }
   }
 }
@@ -90,7 +104,7 @@ cudaError_t launch_rope_table(float* table, int N, int D, double pos_scale, doub
 
 cudaError_t launch_rope_apply(const void* x, void* out, const float* table, int B, int N, int heads, int D,
                               int inverse, int num_sms, cudaStream_t stream) {
-  const long long n = static_cast<long long>(B) * N * (D / 16);
+  const long long n = static_cast<long long>(B) * N * ((heads + 3) / 4) * (D / 16);
   const long long blocks = (n + 255) / 256;
   const int grid = static_cast<int>(blocks < 16LL * num_sms ? blocks : 16LL * num_sms);
   const auto* xin = static_cast<const __nv_bfloat16*>(x);

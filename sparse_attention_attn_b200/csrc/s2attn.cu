@@ -151,6 +151,7 @@ Dims make_dims(int B, int H, int Hkv, int N, int D, int G) {
   d.Nk = N;
   d.qoff_t = 0;
   d.causal = 1;
+  d.noshift = 0;
   return d;
 }
 
@@ -332,7 +333,7 @@ thread_local ProfState g_prof;
 
 // The forward of a validated shape (S2 attention or a segment).
 int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, const Dims& dims,
-             s2attn_stream_t stream) {
+             s2attn_stream_t stream, HgaList hist = HgaList()) {
   const int B = dims.B, H = dims.H, Hkv = dims.Hkv, N = dims.N, D = dims.D, G = dims.G;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
     return S2ATTN_ERR_MISALIGNED;
@@ -345,6 +346,7 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, c
     return S2ATTN_ERR_CUDA;
   FwdArgs a;
   a.d = dims;
+  a.hist = hist;
   const Plan plan = select_plan(B, H, Hkv, N, D, G, info.sms);
   a.sched = make_fwd_sched(a.d, plan.fwd_snake);
   a.scale_log2 = static_cast<float>(1.4426950408889634 / __builtin_sqrt(static_cast<double>(D)));
@@ -479,7 +481,7 @@ namespace {
 int bwd_impl(int path, int stages, const void* q, const void* k, const void* v, const void* o, const float* lse,
              const void* dO, void* dq, void* dk, void* dv, int B, int H, int Hkv, int N, int D, int G,
              void* workspace, size_t workspace_bytes, s2attn_stream_t stream, const float* rope = nullptr,
-             const Dims* seg = nullptr, int dq_accumulate = 0) {
+             const Dims* seg = nullptr, int dq_accumulate = 0, HgaList hist = HgaList()) {
   g_last_launches = 0;
   const bool dq_only = seg != nullptr && !seg->causal;
   if (!q || !k || !v || !o || !lse || !dO || !dq) return S2ATTN_ERR_INVALID_ARG;
@@ -522,6 +524,7 @@ int bwd_impl(int path, int stages, const void* q, const void* k, const void* v, 
   pre.status = status;
   BwdArgs a;
   a.d = d;
+  a.hist = hist;
   a.kv_sched = make_pair_sched(B * Hkv * d.n_groups, d.tiles);
   a.q_sched = make_pair_sched(B * H * d.n_groups, d.tiles);
   a.scale = static_cast<float>(1.0 / __builtin_sqrt(static_cast<double>(D)));
@@ -673,6 +676,46 @@ int s2attn_lse_merge(const void* o_a, const float* lse_a, const void* o_b, const
     return S2ATTN_ERR_CUDA;
   g_last_launches = 1;
   return S2ATTN_OK;
+}
+
+int s2attn_hga_fwd(const void* q, const void* k, const void* v, void* o, float* lse, const int* hist, int S,
+                   int B, int H, int Hkv, int N, int D, int G, s2attn_stream_t stream) {
+  g_last_launches = 0;
+  if (!q || !k || !v || !o || !lse || (S > 0 && !hist) || S < 0 || S > 4096) return S2ATTN_ERR_INVALID_ARG;
+  int st = validate_shape(B, H, Hkv, N, D, G);
+  if (st != S2ATTN_OK) return st;
+  if (G % kQBlock != 0) return S2ATTN_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(hist) & 3u) != 0) return S2ATTN_ERR_MISALIGNED;
+  Dims d = make_dims(B, H, Hkv, N, D, G);
+  d.noshift = 1;
+  HgaList hl;
+  hl.tiles = hist;
+  hl.S = S;
+  return fwd_impl(q, k, v, o, lse, d, stream, hl);
+}
+
+int s2attn_hga_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                   void* dq, void* dk, void* dv, const int* hist, int S, int B, int H, int Hkv, int N, int D, int G,
+                   void* workspace, size_t workspace_bytes, s2attn_stream_t stream) {
+  g_last_launches = 0;
+  if ((S > 0 && !hist) || S < 0 || S > 4096) return S2ATTN_ERR_INVALID_ARG;
+  int st = validate_shape(B, H, Hkv, N, D, G);
+  if (st != S2ATTN_OK) return st;
+  if (G % kQBlock != 0) return S2ATTN_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(hist) & 3u) != 0) return S2ATTN_ERR_MISALIGNED;
+  Dims d = make_dims(B, H, Hkv, N, D, G);
+  d.noshift = 1;
+  HgaList hl;
+  hl.tiles = hist;
+  hl.S = S;
+  const Plan plan = select_plan(B, H, Hkv, N, D, G, 0);
+  return bwd_impl(kBwdSplit, plan.bwd_stages, q, k, v, o, lse, dO, dq, dk, dv, B, H, Hkv, N, D, G, workspace,
+                  workspace_bytes, stream, nullptr, &d, 0, hl);
+}
+
+size_t s2attn_hga_bwd_workspace_bytes(int B, int H, int Hkv, int N, int D, int G) {
+  if (validate_shape(B, H, Hkv, N, D, G) != S2ATTN_OK) return 0;
+  return workspace_bytes_for(kBwdSplit, B, H, N, D);
 }
 
 int s2attn_plan(int B, int H, int Hkv, int N, int D, int G, int num_sms, int* out) {
