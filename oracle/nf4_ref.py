@@ -1,0 +1,97 @@
+"""fp64 CPU oracle for 4-bit NormalFloat (NF4) weights with double
+quantization, and the QKV projection that dequantizes them.
+
+TEST INFRASTRUCTURE ONLY: imported by the test suite, the package smoke check
+and the benchmark's CPU-baseline leg, never by the product path; it shares no
+code with the CUDA kernels.
+
+What the pages state (LongQLoRA community post, section 03, QLoRA): the
+pretrained weights are quantized to 4 bits with the 4-bit NormalFloat data
+type ("theoretically optimal", better than FP4 and Int4); Double
+Quantization saves 0.37 bit per parameter on average; LongQLoRA quantizes the
+whole model this way (section 04) and the attention's q, k, v come from the
+quantized projections.
+
+Readings taken where the pages are silent (listed in the design notes):
+* NF4 levels (the QLoRA construction): 16 values, quantiles of the standard
+  normal distribution normalised to [-1, 1] with an exact zero -- 8 positive
+  levels Phi^-1(p) for p evenly spaced from 1/2 to 1 - delta (the zero is the
+  first), 7 negative ones the same way with 8 points, delta = (1/30 + 1/32)/2,
+  each side divided by Phi^-1(1 - delta);
+* first-level blocks of 64 consecutive weights of a row with an absmax scale;
+  those scales quantized to 8 bits in blocks of 256 with an fp32 second-level
+  scale: 4 + 8/64 + 32/(64*256) = 4.127 bits per weight against 4.5 with fp32
+  scales, the 0.37 bit the post states;
+* the second level is symmetric int8 absmax: scale' = round(127 scale / c) c / 127
+  with c the block's largest scale; codes are chosen against the exact
+  first-level scale (nearest level of w / absmax);
+* the projection: [q | k | v] = X W^T with W [(H + 2 Hkv) D, d_model] the
+  dequantized NF4 weight (level * scale'), X bf16 activations; q, k, v come
+  out in the (batch, sequence, heads, head_dim) layout as row blocks of W.
+
+All arithmetic float64 numpy (scipy for the normal quantiles).
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = ["NF4_DELTA", "nf4_levels", "quantize_nf4", "dequantize_nf4", "nf4_qkv_projection",
+           "bits_per_weight"]
+
+NF4_DELTA = 0.5 * (1.0 / 30.0 + 1.0 / 32.0)
+BLOCK = 64
+DQ_BLOCK = 256
+
+
+def nf4_levels() -> np.ndarray:
+    """The 16 NF4 levels, ascending (index = code)."""
+    from scipy.special import ndtri
+    top = ndtri(1.0 - NF4_DELTA)
+    pos = ndtri(np.linspace(0.5, 1.0 - NF4_DELTA, 9)) / top          # 0 and 8 positive levels
+    neg = -ndtri(np.linspace(0.5, 1.0 - NF4_DELTA, 8)[1:]) / top     # 7 negative levels
+    return np.sort(np.concatenate([neg, pos]))
+
+
+def bits_per_weight(double_quant: bool = True) -> float:
+    return 4.0 + (8.0 / BLOCK + 32.0 / (BLOCK * DQ_BLOCK) if double_quant else 32.0 / BLOCK)
+
+
+def quantize_nf4(w):
+    """w [rows, K] (K % 64 == 0, rows * K / 64 % 256 == 0) -> (codes uint8 [rows, K],
+    scale codes int8 [rows * K / 64], second-level scales float32 [rows * K / 64 / 256])."""
+    w = np.asarray(w, dtype=np.float64)
+    rows, K = w.shape
+    lv = nf4_levels()
+    blocks = w.reshape(-1, BLOCK)
+    absmax = np.abs(blocks).max(axis=1)
+    safe = np.where(absmax > 0, absmax, 1.0)
+    x = blocks / safe[:, None]
+    codes = np.abs(x[..., None] - lv[None, None, :]).argmin(axis=-1).astype(np.uint8)
+    groups = absmax.reshape(-1, DQ_BLOCK)
+    c2 = groups.max(axis=1)
+    c2s = np.where(c2 > 0, c2, 1.0)
+    sq = np.rint(groups / c2s[:, None] * 127.0).astype(np.int8)
+    return codes.reshape(rows, K), sq.reshape(-1), c2.astype(np.float32)
+
+
+def dequantize_nf4(codes, scale_codes, c2) -> np.ndarray:
+    """float64 [rows, K]: level[code] * scale_code * c2 / 127 per 64-block."""
+    codes = np.asarray(codes)
+    rows, K = codes.shape
+    lv = nf4_levels()
+    scale = (np.asarray(scale_codes, dtype=np.float64).reshape(-1, DQ_BLOCK)
+             * np.asarray(c2, dtype=np.float64)[:, None] / 127.0).reshape(-1)
+    return (lv[codes.reshape(-1, BLOCK)] * scale[:, None]).reshape(rows, K)
+
+
+def nf4_qkv_projection(x, codes, scale_codes, c2, H: int, Hkv: int, D: int):
+    """x [B, N, d_model] -> (q [B,N,H,D], k [B,N,Hkv,D], v [B,N,Hkv,D]) with
+    the dequantized weight W [(H + 2 Hkv) D, d_model]: [q | k | v] = x W^T."""
+    x = np.asarray(x, dtype=np.float64)
+    B, N, _ = x.shape
+    y = x @ dequantize_nf4(codes, scale_codes, c2).T
+    q = y[..., : H * D].reshape(B, N, H, D)
+    k = y[..., H * D:(H + Hkv) * D].reshape(B, N, Hkv, D)
+    v = y[..., (H + Hkv) * D:].reshape(B, N, Hkv, D)
+    return q, k, v

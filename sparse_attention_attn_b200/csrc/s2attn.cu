@@ -121,12 +121,12 @@ unsigned long long wait_limit_ns() {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Shape rules shared by forward and backward.  Pure host logic: no CUDA call.
-int validate_shape(int B, int H, int Hkv, int N, int D, int G) {
+int validate_shape(int B, int H, int Hkv, int N, int D, int G, bool shifted = true) {
   if (B <= 0 || H <= 0 || Hkv <= 0 || N <= 0 || D <= 0 || G <= 0) return S2ATTN_ERR_INVALID_ARG;
   if (H % Hkv != 0 || G > N || N % G != 0) return S2ATTN_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return S2ATTN_ERR_UNSUPPORTED;
   if (N % kTile != 0 || G % kTile != 0) return S2ATTN_ERR_UNSUPPORTED;
-  if (G < N) {
+  if (G < N && shifted) {  // the shifted half of the heads takes whole kv-head groups
     if (G % (2 * kTile) != 0) return S2ATTN_ERR_UNSUPPORTED;
     if ((H / 2) % (H / Hkv) != 0) return S2ATTN_ERR_UNSUPPORTED;
   }
@@ -682,7 +682,7 @@ int s2attn_hga_fwd(const void* q, const void* k, const void* v, void* o, float* 
                    int B, int H, int Hkv, int N, int D, int G, s2attn_stream_t stream) {
   g_last_launches = 0;
   if (!q || !k || !v || !o || !lse || (S > 0 && !hist) || S < 0 || S > 4096) return S2ATTN_ERR_INVALID_ARG;
-  int st = validate_shape(B, H, Hkv, N, D, G);
+  int st = validate_shape(B, H, Hkv, N, D, G, false);
   if (st != S2ATTN_OK) return st;
   if (G % kQBlock != 0) return S2ATTN_ERR_UNSUPPORTED;
   if ((reinterpret_cast<uintptr_t>(hist) & 3u) != 0) return S2ATTN_ERR_MISALIGNED;
@@ -699,7 +699,7 @@ int s2attn_hga_bwd(const void* q, const void* k, const void* v, const void* o, c
                    void* workspace, size_t workspace_bytes, s2attn_stream_t stream) {
   g_last_launches = 0;
   if ((S > 0 && !hist) || S < 0 || S > 4096) return S2ATTN_ERR_INVALID_ARG;
-  int st = validate_shape(B, H, Hkv, N, D, G);
+  int st = validate_shape(B, H, Hkv, N, D, G, false);
   if (st != S2ATTN_OK) return st;
   if (G % kQBlock != 0) return S2ATTN_ERR_UNSUPPORTED;
   if ((reinterpret_cast<uintptr_t>(hist) & 3u) != 0) return S2ATTN_ERR_MISALIGNED;
@@ -714,7 +714,7 @@ int s2attn_hga_bwd(const void* q, const void* k, const void* v, const void* o, c
 }
 
 size_t s2attn_hga_bwd_workspace_bytes(int B, int H, int Hkv, int N, int D, int G) {
-  if (validate_shape(B, H, Hkv, N, D, G) != S2ATTN_OK) return 0;
+  if (validate_shape(B, H, Hkv, N, D, G, false) != S2ATTN_OK || G % kQBlock != 0) return 0;
   return workspace_bytes_for(kBwdSplit, B, H, N, D);
 }
 
