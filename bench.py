@@ -459,6 +459,8 @@ def run_ours(args, shape, world, rank, local):
         line["dense_comparison"] = dense_ratio(shape, dev, args)
     if not args.no_rope and rank == 0 and world == 1:
         line["rope"] = rope_step(shape, dev, peaks, ms_step)
+    if not args.no_nf4 and rank == 0 and world == 1:
+        line["nf4_qkv"] = nf4_projection(dev, peaks)
     if not args.no_extra_workloads and world == 1:
         line["other_workloads"] = {s.name: other_workload(s, dev, peaks)
                                    for s in I.WORKLOADS if s.name in args.extra_workloads.split(",")}
@@ -552,6 +554,62 @@ def rope_step(shape: I.Shape, dev, peaks, ms_plain: float, steps: int = 10, warm
                                 "frac": rot_bytes / (avg * 1e-3) / 1e9 / peaks["hbm_gbs"],
                                 "bytes_per_launch": rot_bytes}
     return out
+
+
+def nf4_projection(dev, peaks, steps: int = 20, warmup: int = 3):
+    """The QKV projection that feeds the attention, from NF4 weights with
+    double quantization (LLaMA2-7B layer at 8192 tokens: x [8192, 4096],
+    W [12288, 4096]): the fused kernel (dequantization inside the tensor-core
+    GEMM) against the library's dequantization kernel followed by a cuBLAS
+    GEMM (torch.matmul) on the dequantized weight.  Inputs and outputs (x
+    64 MiB, codes 24 MiB, q/k/v 192 MiB) exceed the L2 together."""
+    import sparse_attention_attn_b200 as s2
+    c = I.NF4_LLAMA2_7B_8K
+    M, K, H, Hkv, D = c["M"], c["K"], c["H"], c["Hkv"], c["D"]
+    rows = (H + 2 * Hkv) * D
+    codes, sq, c2 = (t.to(dev) for t in I.make_nf4_weights(rows, K, seed=3))
+    x = I.randn_bf16((1, M, K), 90).to(dev)
+    q = torch.empty((1, M, H, D), dtype=torch.bfloat16, device=dev)
+    k = torch.empty((1, M, Hkv, D), dtype=torch.bfloat16, device=dev)
+    v = torch.empty_like(k)
+    w = torch.empty((rows, K), dtype=torch.bfloat16, device=dev)
+    y = torch.empty((M, rows), dtype=torch.bfloat16, device=dev)
+
+    def fused():
+        s2.nf4_qkv(x, codes, sq, c2, H, Hkv, D, q=q, k=k, v=v)
+
+    def unfused():
+        s2.nf4_dequantize(codes, sq, c2, out=w)
+        torch.matmul(x.view(M, K), w.t(), out=y)
+
+    def dequant_only():
+        s2.nf4_dequantize(codes, sq, c2, out=w)
+
+    def timed(fn):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(steps):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / steps
+
+    ms_f, ms_u, ms_d = timed(fused), timed(unfused), timed(dequant_only)
+    if s2.device_status() != 0:
+        raise RuntimeError("device status reports a timeout in the NF4 projection")
+    flops = 2.0 * M * rows * K
+    dq_bytes = rows * K / 2 + rows * K / 64 + rows * K * 2  # codes + scale codes read, bf16 W' written
+    tf = flops / (ms_f * 1e-3) / 1e12
+    return {"workload": c["name"], "M": M, "K": K, "N_out": rows, "ms": ms_f, "achieved": tf, "unit": "TFLOP/s",
+            "frac": tf / peaks["bf16_tflops"], "peak_source": "measured (bf16_tflops burst)",
+            "unfused_ms": ms_u, "unfused": "nf4 dequantization kernel + cuBLAS bf16 GEMM (torch.matmul)",
+            "speedup_vs_unfused": ms_u / ms_f,
+            "dequant_kernel": {"ms": ms_d, "achieved": dq_bytes / (ms_d * 1e-3) / 1e9, "unit": "GB/s",
+                               "frac": dq_bytes / (ms_d * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+            "steps": steps, "warmup": warmup}
 
 
 def other_workload(shape: I.Shape, dev, peaks, steps: int = 5, warmup: int = 3):
@@ -676,6 +734,7 @@ def main():
     ap.add_argument("--no-extra-workloads", action="store_true",
                     help="skip the few-step timing of the other workload shapes")
     ap.add_argument("--no-rope", action="store_true", help="skip the step with RoPE + Position Interpolation")
+    ap.add_argument("--no-nf4", action="store_true", help="skip the NF4 QKV projection timing")
     ap.add_argument("--sweep", action="store_true",
                     help="time every selectable kernel variant on every workload shape and exit")
     ap.add_argument("--extra-workloads", default=f"{I.QWEN3_8B_16K.name},{I.LLAMA2_70B_32K.name}",

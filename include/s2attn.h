@@ -247,6 +247,57 @@ S2ATTN_API int s2attn_hga_bwd(const void* q, const void* k, const void* v, const
                               int Hkv, int N, int D, int G, void* workspace, size_t workspace_bytes,
                               s2attn_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * QKV projection from 4-bit NormalFloat weights with double quantization
+ * (LongQLoRA community post, section 03 Method, QLoRA: frozen weights in 4-bit
+ * NF4, their quantization constants quantized again; section 04: the whole
+ * model is quantized so, and S2 attention takes its q, k, v from these
+ * projections).
+ *
+ * W is the [Nout, K] weight of the fused projection, Nout = (H + 2 Hkv) D:
+ * rows [0, H D) produce q, [H D, (H + Hkv) D) k, the rest v; K is the model
+ * width.  Its storage (all device memory, caller-owned, read only):
+ *   codes        uint8 [Nout, K/2]: the 4-bit code of element 2j of a row in
+ *                the low nibble of byte j, of element 2j+1 in the high nibble;
+ *   scale_codes  int8 [Nout * K/64]: the first-level scale of block (n, kb)
+ *                -- elements [64 kb, 64 kb + 64) of row n -- at n * K/64 + kb,
+ *                as a code in [-127, 127];
+ *   c2           fp32 [ceil(Nout * K/64 / 256)]: the second-level scale of
+ *                first-level blocks [256 i, 256 i + 256) at i.
+ * The dequantized weight is W'[n, k] = bf16(level[code] * s), s = code_s * c2
+ * / 127, computed in fp32 and rounded to nearest even, with level[] the 16
+ * NF4 values of s2attn_nf4_levels.
+ * ------------------------------------------------------------------------ */
+
+/* The 16 NF4 levels, ascending (level[c] for code c), as fp32 into the host
+ * array levels[16]: standard normal quantiles normalised into [-1, 1] with an
+ * exact zero (8 positive levels, 7 negative).  Host only. */
+S2ATTN_API int s2attn_nf4_levels(float* levels);
+
+/*
+ * [q | k | v] = x W'^T with the dequantization fused into the tensor-core
+ * GEMM (W' never goes to global memory).  x: bf16 [M, K] (M tokens, row
+ * major, 16-byte aligned); q: bf16 [M, H D], k and v: bf16 [M, Hkv D], row
+ * major -- i.e. [B, N, heads, D] with M = B N, the layout s2attn_fwd reads.
+ * fp32 accumulation, bf16 results rounded to nearest even.  Requires
+ * K % 64 == 0 and H D, Hkv D multiples of 128; codes, q, k, v 16-byte
+ * aligned.
+ * Returns a status code; a bounded-wait timeout inside the kernel is reported
+ * by s2attn_device_status(NULL, stream).
+ */
+S2ATTN_API int s2attn_nf4_qkv(const void* x, const void* codes, const int8_t* scale_codes, const float* c2,
+                              void* q, void* k, void* v, int M, int K, int H, int Hkv, int D,
+                              s2attn_stream_t stream);
+
+/*
+ * The dequantized weight alone: w = W' as bf16 [rows, K] (16-byte aligned),
+ * from codes [rows, K/2] (4-byte aligned), scale_codes and c2 laid out as
+ * above with `rows` in place of Nout.  K % 64 == 0.  For callers that run
+ * their own GEMM on W' (e.g. the input gradient x' = y' W').
+ */
+S2ATTN_API int s2attn_nf4_dequant(const void* codes, const int8_t* scale_codes, const float* c2, void* w,
+                                  int rows, int K, s2attn_stream_t stream);
+
 /*
  * Backward for callers that cannot allocate device memory (no counterpart in
  * the papers: this is a deployment variant of s2attn_bwd).  Some callers have
@@ -310,7 +361,8 @@ S2ATTN_API const char* s2attn_cuda_error_string(int err);
  * pair around each kernel they launch, up to max_launches launches.
  * s2attn_profile_stop turns recording off, waits for the recorded events and
  * writes per-launch durations (ms) and kernel ids (0 forward, 1 backward
- * preprocess, 2 backward dK/dV, 3 backward dQ) to caller arrays of
+ * preprocess, 2 backward dK/dV, 3 backward dQ, 4 fused backward, 5 its dq
+ * conversion, 6 RoPE rotation, 7 NF4 QKV projection, 8 NF4 dequantization) to caller arrays of
  * `capacity` entries (either may be NULL).  Returns the number of records, or
  * minus a status code.
  */
@@ -335,8 +387,9 @@ S2ATTN_API int s2attn_plan(int B, int H, int Hkv, int N, int D, int G, int num_s
  * items; keys bwd=split|fused (backward path; fused exists for head dim 128),
  * fwd_order=snake|pairs (forward work order), fwd_kv=N (forward K/V ring
  * depth: 4 at head dim 128, 4/6/8 at 64), bwd_stages=N (split backward
- * stages: 2-3 at head dim 128, 3-4 at 64); values that do not exist for a
- * call's head dim are ignored.  s2attn_bwd_workspace_bytes answers for the
+ * stages: 2-3 at head dim 128, 3-4 at 64), nf4_stages=4|6 (pipeline
+ * depth of s2attn_nf4_qkv); values that do not exist for a call's head dim
+ * are ignored.  s2attn_bwd_workspace_bytes answers for the
  * path in force when it is called.  Returns S2ATTN_OK.
  */
 S2ATTN_API int s2attn_set_tile_override(const char* spec);

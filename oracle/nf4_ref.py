@@ -36,8 +36,10 @@ from __future__ import annotations
 
 import numpy as np
 
+from oracle.rope_ref import round_bf16
+
 __all__ = ["NF4_DELTA", "nf4_levels", "quantize_nf4", "dequantize_nf4", "nf4_qkv_projection",
-           "bits_per_weight"]
+           "bits_per_weight", "round_bf16", "unpack_codes"]
 
 NF4_DELTA = 0.5 * (1.0 / 30.0 + 1.0 / 32.0)
 BLOCK = 64
@@ -85,12 +87,27 @@ def dequantize_nf4(codes, scale_codes, c2) -> np.ndarray:
     return (lv[codes.reshape(-1, BLOCK)] * scale[:, None]).reshape(rows, K)
 
 
-def nf4_qkv_projection(x, codes, scale_codes, c2, H: int, Hkv: int, D: int):
+def unpack_codes(packed) -> np.ndarray:
+    """uint8 [rows, K/2] with two codes a byte (element 2j in the low nibble)
+    -> uint8 [rows, K]."""
+    packed = np.asarray(packed, dtype=np.uint8)
+    out = np.empty((packed.shape[0], 2 * packed.shape[1]), dtype=np.uint8)
+    out[:, 0::2] = packed & 15
+    out[:, 1::2] = packed >> 4
+    return out
+
+
+def nf4_qkv_projection(x, codes, scale_codes, c2, H: int, Hkv: int, D: int, bf16_weights: bool = False):
     """x [B, N, d_model] -> (q [B,N,H,D], k [B,N,Hkv,D], v [B,N,Hkv,D]) with
-    the dequantized weight W [(H + 2 Hkv) D, d_model]: [q | k | v] = x W^T."""
+    the dequantized weight W [(H + 2 Hkv) D, d_model]: [q | k | v] = x W^T.
+    bf16_weights rounds W to bf16 first (the tensor cores' operand type, the
+    reading of the bf16 GEMM)."""
     x = np.asarray(x, dtype=np.float64)
     B, N, _ = x.shape
-    y = x @ dequantize_nf4(codes, scale_codes, c2).T
+    w = dequantize_nf4(codes, scale_codes, c2)
+    if bf16_weights:
+        w = round_bf16(w)
+    y = x @ w.T
     q = y[..., : H * D].reshape(B, N, H, D)
     k = y[..., H * D:(H + Hkv) * D].reshape(B, N, Hkv, D)
     v = y[..., (H + Hkv) * D:].reshape(B, N, Hkv, D)

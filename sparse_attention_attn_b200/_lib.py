@@ -54,6 +54,9 @@ SIGNATURES = {
     "s2attn_bwd_rope": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp,
                              ctypes.c_size_t, _vp]),
     "s2attn_plan": (_i, [_i, _i, _i, _i, _i, _i, _i, _vp]),
+    "s2attn_nf4_levels": (_i, [_vp]),
+    "s2attn_nf4_qkv": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
+    "s2attn_nf4_dequant": (_i, [_vp, _vp, _vp, _vp, _i, _i, _vp]),
     "s2attn_bwd_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
                                 _vp]),
 }
@@ -191,6 +194,21 @@ def s2attn_plan(B, H, Hkv, N, D, G, num_sms):
     _check("s2attn_plan", load().s2attn_plan(B, H, Hkv, N, D, G, num_sms, ctypes.addressof(out)))
     return {"fwd_order": "snake" if out[0] else "pairs", "fwd_kv_slots": out[1],
             "bwd_path": "fused" if out[2] else "split", "bwd_stages": out[3]}
+
+
+def s2attn_nf4_levels():
+    """The library's 16 NF4 levels (host computation) as a list of floats."""
+    out = (ctypes.c_float * 16)()
+    _check("s2attn_nf4_levels", load().s2attn_nf4_levels(ctypes.addressof(out)))
+    return list(out)
+
+
+def s2attn_nf4_qkv(x, codes, scale_codes, c2, q, k, v, M, K, H, Hkv, D, stream) -> int:
+    return load().s2attn_nf4_qkv(x, codes, scale_codes, c2, q, k, v, M, K, H, Hkv, D, stream)
+
+
+def s2attn_nf4_dequant(codes, scale_codes, c2, w, rows, K, stream) -> int:
+    return load().s2attn_nf4_dequant(codes, scale_codes, c2, w, rows, K, stream)
 
 
 def s2attn_set_tile_override(spec) -> int:

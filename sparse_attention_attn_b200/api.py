@@ -401,3 +401,60 @@ def s2_attn(q, k, v, group_size: int):
 def dense_causal_attn(q, k, v):
     """Dense causal attention through the same kernels (G = N, no shift)."""
     return S2Attention.apply(q, k, v, q.shape[1])
+
+
+# ---------------------------------------------------------------- NF4 QKV projection
+
+def _need_nf4(codes, scale_codes, c2, rows: int, K: int, dev) -> None:
+    _need("codes", codes, (rows, K // 2), torch.uint8, device=dev)
+    _need("scale_codes", scale_codes, (rows * (K // 64),), torch.int8, device=dev)
+    _need("c2", c2, ((rows * (K // 64) + 255) // 256,), torch.float32, device=dev)
+
+
+def nf4_levels():
+    """The 16 NF4 levels the kernels use (ascending; index = 4-bit code)."""
+    return _lib.s2attn_nf4_levels()
+
+
+def nf4_qkv(x, codes, scale_codes, c2, n_heads: int, n_kv_heads: int, head_dim: int, q=None, k=None, v=None):
+    """q, k, v = the QKV projection of x (bf16 [B, N, K]) through NF4 weights
+    with double quantization, dequantized inside the tensor-core GEMM.  The
+    weight is [(H + 2 Hkv) D, K]: codes uint8 [rows, K/2] (two 4-bit codes a
+    byte, the even element in the low nibble), scale_codes int8 [rows K/64],
+    c2 fp32 [ceil(rows K/64 / 256)].  Returns bf16 [B, N, H, D], [B, N, Hkv, D],
+    [B, N, Hkv, D]."""
+    if not isinstance(x, torch.Tensor) or x.dim() != 3:
+        raise ValueError("x must be a [B, N, K] tensor")
+    B, N, K = x.shape
+    H, Hkv, D = int(n_heads), int(n_kv_heads), int(head_dim)
+    dev = x.device
+    _need("x", x, (B, N, K))
+    rows = (H + 2 * Hkv) * D
+    _need_nf4(codes, scale_codes, c2, rows, K, dev)
+    q = torch.empty((B, N, H, D), dtype=torch.bfloat16, device=dev) if q is None else q
+    k = torch.empty((B, N, Hkv, D), dtype=torch.bfloat16, device=dev) if k is None else k
+    v = torch.empty((B, N, Hkv, D), dtype=torch.bfloat16, device=dev) if v is None else v
+    _need("q", q, (B, N, H, D), device=dev)
+    _need("k", k, (B, N, Hkv, D), device=dev)
+    _need("v", v, (B, N, Hkv, D), device=dev)
+    with torch.cuda.device(dev):
+        st = _lib.s2attn_nf4_qkv(x.data_ptr(), codes.data_ptr(), scale_codes.data_ptr(), c2.data_ptr(), q.data_ptr(),
+                                 k.data_ptr(), v.data_ptr(), B * N, K, H, Hkv, D, _stream(dev))
+    _lib._check("s2attn_nf4_qkv", st)
+    return q, k, v
+
+
+def nf4_dequantize(codes, scale_codes, c2, out=None):
+    """The dequantized weight W' (bf16 [rows, K]) of NF4 codes [rows, K/2]."""
+    if not isinstance(codes, torch.Tensor) or codes.dim() != 2:
+        raise ValueError("codes must be a [rows, K/2] tensor")
+    rows, K = codes.shape[0], 2 * codes.shape[1]
+    dev = codes.device
+    _need_nf4(codes, scale_codes, c2, rows, K, dev)
+    out = torch.empty((rows, K), dtype=torch.bfloat16, device=dev) if out is None else out
+    _need("out", out, (rows, K), device=dev)
+    with torch.cuda.device(dev):
+        st = _lib.s2attn_nf4_dequant(codes.data_ptr(), scale_codes.data_ptr(), c2.data_ptr(), out.data_ptr(), rows, K,
+                                     _stream(dev))
+    _lib._check("s2attn_nf4_dequant", st)
+    return out

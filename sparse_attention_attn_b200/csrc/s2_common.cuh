@@ -13,6 +13,7 @@
 
 #include <cstdint>
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 namespace s2 {
@@ -347,6 +348,29 @@ struct BwdMaps {
 template <int D>
 cudaError_t launch_bwd_pre(const BwdPreArgs& pre, int num_sms, cudaStream_t stream);
 
+// The 16 NF4 levels, ascending (index = 4-bit code), passed to the NF4 kernels.
+struct Nf4Levels {
+  float v[16];
+};
+
+// Arguments of the fused NF4 QKV projection kernel (s2_nf4.cu).
+struct Nf4Args {
+  const int8_t* sq;
+  const float* c2;
+  int width0, width1;  // features of q and of k (v has as many as k)
+  int M, K;
+  int tiles_w;  // 128-row weight tiles (Nout / 128)
+  int tiles_t;  // 256-token tiles
+  Nf4Levels lv;
+  uint32_t* status;
+  unsigned long long wait_limit_ns;
+};
+
+cudaError_t launch_nf4_qkv(const CUtensorMap& tx, const CUtensorMap& tc, const CUtensorMap* to, const Nf4Args& a,
+                           int num_sms, cudaStream_t stream, int stages);
+cudaError_t launch_nf4_dequant(const void* codes, const int8_t* sq, const float* c2, void* w, long long n_words,
+                               const Nf4Levels& lv, int num_sms, cudaStream_t stream);
+
 // Optional per-kernel timing (s2attn_profile_start / _stop): the launchers
 // bracket every kernel with these; they do nothing unless profiling is on.
 enum KernelId : int {
@@ -356,7 +380,9 @@ enum KernelId : int {
   kKernelBwdDq = 3,
   kKernelBwdFused = 4,
   kKernelBwdDqPost = 5,
-  kKernelRope = 6
+  kKernelRope = 6,
+  kKernelNf4Qkv = 7,
+  kKernelNf4Dequant = 8
 };
 void prof_before(cudaStream_t stream, int kernel_id);
 void prof_after(cudaStream_t stream);

@@ -148,6 +148,24 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+// 2-D tiled load (coordinates innermost first) completing on mbarrier `bar`.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
+      : "memory");
+}
+
+// 2-D tiled TMA store shared -> global through the issuing thread's bulk group
+// (no coordinate may be negative; rows or columns past the tensor are clipped).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int c0, int c1) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(src), "r"(c0), "r"(c1)
+               : "memory");
+}
+
 // Tiled TMA store shared -> global, completed through the issuing thread's
 // bulk group.  The innermost coordinate times the element size must be a
 // multiple of 16 bytes and no coordinate may be negative.
@@ -178,6 +196,12 @@ __device__ __forceinline__ void bulk_reduce_add_f32(void* dst, uint32_t src, uin
                    reinterpret_cast<uint64_t>(dst)),
                "r"(src), "r"(bytes)
                : "memory");
+}
+
+// One bf16 (round to nearest even) to shared memory.
+__device__ __forceinline__ void st_shared_bf16(uint32_t addr, float v) {
+  const __nv_bfloat16 b = __float2bfloat16_rn(v);
+  asm volatile("st.shared.b16 [%0], %1;" ::"r"(addr), "h"(*reinterpret_cast<const unsigned short*>(&b)) : "memory");
 }
 
 __device__ __forceinline__ void st_shared_f32(uint32_t addr, float v) {
@@ -272,6 +296,17 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
         "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
         "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+
+// 32 lanes x 16 consecutive 32-bit columns (as tmem_ld32, half as wide).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
       : "r"(taddr)
       : "memory");
 }
@@ -389,6 +424,24 @@ __device__ __forceinline__ float4 lds_f4(uint32_t addr) {
                : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
                : "r"(addr));
   return v;
+}
+
+__device__ __forceinline__ uint4 lds_u4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
+// Table lookup across the warp: every lane holds one entry, lane l the entry
+// l mod 16 (so lanes 16..31 repeat 0..15), and each lane reads the lane named
+// by bits [4:0] of `idx` (shfl.sync idx mode with clamp 31 and no segment
+// mask uses exactly those bits).  A 4-bit code in the low bits of idx selects
+// its entry whatever bit 4 holds, so callers need not mask idx.  All 32 lanes
+// must take part.
+__device__ __forceinline__ float warp_lut16(float table, uint32_t idx) {
+  float r;
+  asm volatile("shfl.sync.idx.b32 %0, %1, %2, 0x1f, 0xffffffff;" : "=f"(r) : "f"(table), "r"(idx));
+  return r;
 }
 
 // One 32-byte global store (a whole DRAM sector); the address must be 32-byte

@@ -8,6 +8,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <cmath>
 #include <cstdint>
 #include <cstdlib>
 #include <mutex>
@@ -180,7 +181,8 @@ Dims make_segment_dims(int B, int H, int Hkv, int N, int Nk, int D, int causal) 
 // that the per-shape selection would not pick.  It starts from the
 // S2ATTN_TILE environment variable and can be replaced at run time by the
 // s2attn_set_tile_override test hook.  Keys: bwd=split|fused,
-// fwd_order=snake|pairs.  Unknown keys and values are ignored.
+// fwd_order=snake|pairs, fwd_kv=N, bwd_stages=N, nf4_stages=4|6.  Unknown
+// keys and values are ignored.
 std::mutex g_override_mu;
 std::string g_override;
 bool g_override_init = false;
@@ -711,6 +713,167 @@ int s2attn_hga_bwd(const void* q, const void* k, const void* v, const void* o, c
   const Plan plan = select_plan(B, H, Hkv, N, D, G, 0);
   return bwd_impl(kBwdSplit, plan.bwd_stages, q, k, v, o, lse, dO, dq, dk, dv, B, H, Hkv, N, D, G, workspace,
                   workspace_bytes, stream, nullptr, &d, 0, hl);
+}
+
+}  // extern "C"
+
+namespace {
+// ---------------------------------------------------------------- NF4
+// Phi^-1(p), the standard normal quantile, by bisection on the normal CDF
+// written through erfc (double precision; 200 halvings of [-10, 10]).
+double normal_quantile(double p) {
+  double lo = -10.0, hi = 10.0;
+  for (int i = 0; i < 200; ++i) {
+    const double mid = 0.5 * (lo + hi);
+    if (0.5 * std::erfc(-mid / std::sqrt(2.0)) < p)
+      lo = mid;
+    else
+      hi = mid;
+  }
+  return 0.5 * (lo + hi);
+}
+
+// The 16 NF4 levels (QLoRA's 4-bit NormalFloat): standard normal quantiles
+// normalised into [-1, 1] with an exact zero.  With delta = (1/30 + 1/32) / 2
+// and top = Phi^-1(1 - delta): the zero and 8 positive levels are
+// Phi^-1(p) / top at 9 evenly spaced p from 1/2 to 1 - delta; the 7 negative
+// levels are -Phi^-1(p) / top at 8 such p, the first (the zero) dropped.
+// Ascending, so the code is the index.
+const Nf4Levels& nf4_levels() {
+  static const Nf4Levels lv = [] {
+    Nf4Levels t;
+    const double delta = 0.5 * (1.0 / 30.0 + 1.0 / 32.0);
+    const double top = normal_quantile(1.0 - delta);
+    for (int i = 1; i < 8; ++i) t.v[7 - i] = static_cast<float>(-normal_quantile(0.5 + (0.5 - delta) * i / 7.0) / top);
+    t.v[7] = 0.f;
+    for (int i = 1; i < 9; ++i) t.v[7 + i] = static_cast<float>(normal_quantile(0.5 + (0.5 - delta) * i / 8.0) / top);
+    return t;
+  }();
+  return lv;
+}
+
+// 2-D tiled view {inner, outer} of a row-major array with `row_bytes` between rows.
+bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
+                 uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) {
+    g_last_cuda_error = -1;
+    return false;
+  }
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  const CUresult r = enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) g_last_cuda_error = -static_cast<int>(r);
+  return r == CUDA_SUCCESS;
+}
+
+// Pipeline depth of the fused NF4 projection: 4 stages, or the override's
+// nf4_stages=3|4.
+int nf4_stages() {
+  const std::string v = override_value(tile_override(), "nf4_stages");
+  return v == "3" ? 3 : 4;
+}
+
+int validate_nf4(int M, int K, int H, int Hkv, int D) {
+  if (M <= 0 || K <= 0 || H <= 0 || Hkv <= 0 || D <= 0) return S2ATTN_ERR_INVALID_ARG;
+  if (K % 64 != 0) return S2ATTN_ERR_UNSUPPORTED;
+  const long long wq = static_cast<long long>(H) * D, wk = static_cast<long long>(Hkv) * D;
+  if (wq % 128 != 0 || wk % 128 != 0) return S2ATTN_ERR_UNSUPPORTED;
+  const long long nout = wq + 2 * wk;
+  if (nout >= (1LL << 24) || M >= (1 << 30) || K >= (1 << 24)) return S2ATTN_ERR_UNSUPPORTED;
+  if (nout * (K / 64) >= (1LL << 31) || static_cast<long long>(M) * K >= (1LL << 40) ||
+      static_cast<long long>(M) * nout >= (1LL << 40))
+    return S2ATTN_ERR_UNSUPPORTED;
+  return S2ATTN_OK;
+}
+}  // namespace
+
+extern "C" {
+
+int s2attn_nf4_levels(float* levels) {
+  if (!levels) return S2ATTN_ERR_INVALID_ARG;
+  for (int i = 0; i < 16; ++i) levels[i] = nf4_levels().v[i];
+  return S2ATTN_OK;
+}
+
+int s2attn_nf4_dequant(const void* codes, const int8_t* scale_codes, const float* c2, void* w, int rows, int K,
+                       s2attn_stream_t stream) {
+  g_last_launches = 0;
+  if (!codes || !scale_codes || !c2 || !w || rows <= 0 || K <= 0) return S2ATTN_ERR_INVALID_ARG;
+  if (K % 64 != 0) return S2ATTN_ERR_UNSUPPORTED;
+  const long long blocks = static_cast<long long>(rows) * (K / 64);
+  if (blocks >= (1LL << 31)) return S2ATTN_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(codes) & 3u) != 0 || (reinterpret_cast<uintptr_t>(c2) & 3u) != 0 ||
+      !aligned16(w))
+    return S2ATTN_ERR_MISALIGNED;
+  DeviceInfo info;
+  if (!device_info(&info)) return S2ATTN_ERR_CUDA;
+  if (!info.ok) return S2ATTN_ERR_UNSUPPORTED;
+  const cudaError_t e = launch_nf4_dequant(codes, scale_codes, c2, w, blocks * 8, nf4_levels(), info.sms,
+                                           static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) {
+    g_last_cuda_error = static_cast<int>(e);
+    return S2ATTN_ERR_CUDA;
+  }
+  g_last_launches = 1;
+  return S2ATTN_OK;
+}
+
+int s2attn_nf4_qkv(const void* x, const void* codes, const int8_t* scale_codes, const float* c2, void* q, void* k,
+                   void* v, int M, int K, int H, int Hkv, int D, s2attn_stream_t stream) {
+  g_last_launches = 0;
+  if (!x || !codes || !scale_codes || !c2 || !q || !k || !v) return S2ATTN_ERR_INVALID_ARG;
+  const int st = validate_nf4(M, K, H, Hkv, D);
+  if (st != S2ATTN_OK) return st;
+  if (!aligned16(x) || !aligned16(codes) || (reinterpret_cast<uintptr_t>(c2) & 3u) != 0 || !aligned16(q) ||
+      !aligned16(k) || !aligned16(v))
+    return S2ATTN_ERR_MISALIGNED;
+  DeviceInfo info;
+  if (!device_info(&info)) return S2ATTN_ERR_CUDA;
+  if (!info.ok) return S2ATTN_ERR_UNSUPPORTED;
+  const int nout = (H + 2 * Hkv) * D;
+  CUtensorMap tx, tc;
+  if (!make_map_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
+                   static_cast<uint64_t>(K) * 2, 64, 256, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&tc, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, static_cast<uint64_t>(K / 2),
+                   static_cast<uint64_t>(nout), static_cast<uint64_t>(K / 2), 32, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return S2ATTN_ERR_CUDA;
+  CUtensorMap to[3];
+  const void* outs[3] = {q, k, v};
+  const int widths[3] = {H * D, Hkv * D, Hkv * D};
+  for (int i = 0; i < 3; ++i)
+    if (!make_map_2d(&to[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, outs[i], static_cast<uint64_t>(widths[i]),
+                     static_cast<uint64_t>(M), static_cast<uint64_t>(widths[i]) * 2, 32, 256,
+                     CU_TENSOR_MAP_SWIZZLE_NONE))
+      return S2ATTN_ERR_CUDA;
+  Nf4Args a;
+  a.sq = scale_codes;
+  a.c2 = c2;
+  a.width0 = H * D;
+  a.width1 = Hkv * D;
+  a.M = M;
+  a.K = K;
+  a.tiles_w = nout / 128;
+  a.tiles_t = (M + 255) / 256;
+  a.lv = nf4_levels();
+  void* status = nullptr;
+  const cudaError_t se = cudaGetSymbolAddress(&status, g_fwd_status);
+  if (se != cudaSuccess) {
+    g_last_cuda_error = static_cast<int>(se);
+    return S2ATTN_ERR_CUDA;
+  }
+  a.status = static_cast<uint32_t*>(status);
+  a.wait_limit_ns = wait_limit_ns();
+  const cudaError_t e = launch_nf4_qkv(tx, tc, to, a, info.sms, static_cast<cudaStream_t>(stream), nf4_stages());
+  if (e != cudaSuccess) {
+    g_last_cuda_error = static_cast<int>(e);
+    return S2ATTN_ERR_CUDA;
+  }
+  g_last_launches = 1;
+  return S2ATTN_OK;
 }
 
 size_t s2attn_hga_bwd_workspace_bytes(int B, int H, int Hkv, int N, int D, int G) {

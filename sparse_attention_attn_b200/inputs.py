@@ -1,8 +1,9 @@
 """Seeded synthetic inputs shared by the CUDA path's tests, the bench and the oracle checks.
 
-This module holds no attention arithmetic: it only draws i.i.d. N(0, 1) values
-with torch's CPU generator and rounds them to bf16, the activations' dtype.
-Seeds 0, 1, 2, 3 draw q, k, v and dO respectively (an offset shifts all four).
+This module holds no attention or quantization arithmetic: it only draws
+i.i.d. N(0, 1) values with torch's CPU generator and rounds them to bf16, the
+activations' dtype, and draws uniform random NF4 weight storage.  Seeds 0, 1,
+2, 3 draw q, k, v and dO respectively (an offset shifts all four).
 """
 from __future__ import annotations
 
@@ -50,3 +51,23 @@ def make_inputs(s: Shape, seed_offset: int = 0):
     v = randn_bf16((s.B, s.N, s.Hkv, s.D), 2 + seed_offset)
     do = randn_bf16((s.B, s.N, s.H, s.D), 3 + seed_offset)
     return q, k, v, do
+
+
+# The QKV projection of the LLaMA2-7B layer at 8192 tokens: model width 4096,
+# 32 heads of 128 (q, k and v each 4096 features).
+NF4_LLAMA2_7B_8K = dict(name="llama2-7b-qkv-n8192", M=8192, K=4096, H=32, Hkv=32, D=128)
+
+
+def make_nf4_weights(rows: int, K: int, seed: int):
+    """Random NF4 weight storage for a [rows, K] weight (CPU tensors).  Codes
+    of quantized normal weights are close to uniform (the levels are normal
+    quantiles), so the codes are uniform 4-bit values: uint8 [rows, K/2], two
+    a byte; first-level scale codes int8 [rows K/64] uniform in [64, 127];
+    second-level scales fp32 [ceil(rows K/64 / 256)] uniform in [0.05, 0.08]
+    (absmax of 64 weights of a layer with std 0.02)."""
+    g = torch.Generator().manual_seed(seed)
+    codes = torch.randint(0, 256, (rows, K // 2), generator=g, dtype=torch.int32).to(torch.uint8)
+    nblk = rows * (K // 64)
+    sq = torch.randint(64, 128, (nblk,), generator=g, dtype=torch.int32).to(torch.int8)
+    c2 = 0.05 + 0.03 * torch.rand(((nblk + 255) // 256,), generator=g, dtype=torch.float32)
+    return codes, sq, c2

@@ -153,3 +153,29 @@ def test_plan_override_parsing():
     finally:
         _lib.s2attn_set_tile_override(None)
     assert _lib.s2attn_plan(1, 32, 32, 8192, 128, 2048, 148)["bwd_path"] == "split"
+
+
+def test_nf4_levels_and_argument_checks_on_the_host():
+    """The library's NF4 levels (host computation: bisection on erfc) against
+    the oracle's (scipy's inverse normal CDF), and the projection's argument
+    checks, which return before any CUDA call."""
+    import numpy as np
+    import oracle.nf4_ref as nr
+    from sparse_attention_attn_b200 import _lib
+    np.testing.assert_allclose(np.array(_lib.s2attn_nf4_levels()), nr.nf4_levels(), rtol=0, atol=6e-8)
+    lib = _lib.load()
+    p = 1 << 20  # fake, 16-byte aligned device addresses: nothing is dereferenced
+    args = dict(x=p, codes=p, sq=p, c2=p, q=p, k=p, v=p)
+
+    def call(M=16, K=256, H=2, Hkv=1, D=128, **over):
+        a = dict(args, **over)
+        return lib.s2attn_nf4_qkv(a["x"], a["codes"], a["sq"], a["c2"], a["q"], a["k"], a["v"], M, K, H, Hkv, D,
+                                  None)
+    assert call(x=None) == _lib.S2ATTN_ERR_INVALID_ARG
+    assert call(M=0) == _lib.S2ATTN_ERR_INVALID_ARG
+    assert call(K=96) == _lib.S2ATTN_ERR_UNSUPPORTED          # not a whole number of 64-element blocks
+    assert call(H=1, Hkv=1, D=64) == _lib.S2ATTN_ERR_UNSUPPORTED  # 64 features: not a whole 128-row tile
+    assert call(x=p + 8) == _lib.S2ATTN_ERR_MISALIGNED
+    assert call(q=p + 2) == _lib.S2ATTN_ERR_MISALIGNED
+    assert lib.s2attn_nf4_dequant(p, p, p, p, 4, 100, None) == _lib.S2ATTN_ERR_UNSUPPORTED
+    assert lib.s2attn_nf4_dequant(p, p, p, p + 8, 4, 128, None) == _lib.S2ATTN_ERR_MISALIGNED
