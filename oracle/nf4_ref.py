@@ -60,8 +60,9 @@ def bits_per_weight(double_quant: bool = True) -> float:
 
 
 def quantize_nf4(w):
-    """w [rows, K] (K % 64 == 0, rows * K / 64 % 256 == 0) -> (codes uint8 [rows, K],
-    scale codes int8 [rows * K / 64], second-level scales float32 [rows * K / 64 / 256])."""
+    """w [rows, K] (K % 64 == 0) -> (codes uint8 [rows, K], scale codes int8
+    [rows * K / 64], second-level scales float32 [ceil(rows * K / 64 / 256)];
+    the last second-level block may hold fewer than 256 first-level scales)."""
     w = np.asarray(w, dtype=np.float64)
     rows, K = w.shape
     lv = nf4_levels()
@@ -70,20 +71,22 @@ def quantize_nf4(w):
     safe = np.where(absmax > 0, absmax, 1.0)
     x = blocks / safe[:, None]
     codes = np.abs(x[..., None] - lv[None, None, :]).argmin(axis=-1).astype(np.uint8)
-    groups = absmax.reshape(-1, DQ_BLOCK)
-    c2 = groups.max(axis=1)
+    grp = np.arange(absmax.size) // DQ_BLOCK
+    c2 = np.zeros(grp[-1] + 1)
+    np.maximum.at(c2, grp, absmax)
     c2s = np.where(c2 > 0, c2, 1.0)
-    sq = np.rint(groups / c2s[:, None] * 127.0).astype(np.int8)
-    return codes.reshape(rows, K), sq.reshape(-1), c2.astype(np.float32)
+    sq = np.rint(absmax / c2s[grp] * 127.0).astype(np.int8)
+    return codes.reshape(rows, K), sq, c2.astype(np.float32)
 
 
 def dequantize_nf4(codes, scale_codes, c2) -> np.ndarray:
-    """float64 [rows, K]: level[code] * scale_code * c2 / 127 per 64-block."""
+    """float64 [rows, K]: level[code] * scale_code * c2 / 127 per 64-block,
+    c2 of the block's second-level block (first-level block index // 256)."""
     codes = np.asarray(codes)
     rows, K = codes.shape
     lv = nf4_levels()
-    scale = (np.asarray(scale_codes, dtype=np.float64).reshape(-1, DQ_BLOCK)
-             * np.asarray(c2, dtype=np.float64)[:, None] / 127.0).reshape(-1)
+    sq = np.asarray(scale_codes, dtype=np.float64)
+    scale = sq * np.asarray(c2, dtype=np.float64)[np.arange(sq.size) // DQ_BLOCK] / 127.0
     return (lv[codes.reshape(-1, BLOCK)] * scale[:, None]).reshape(rows, K)
 
 

@@ -75,6 +75,24 @@ def test_round_trip():
     assert np.all(np.abs(x - lv[c.reshape(-1, 64)]) <= np.abs(x[..., None] - lv).min(-1) + 1e-15)
 
 
+def test_partial_last_second_level_block():
+    """48 first-level blocks: one second-level block of 48 (ceil(48 / 256) = 1);
+    weights that are levels times a scale still come back up to the 8-bit
+    scale rounding, and the second-level scale is the largest absmax."""
+    rng = np.random.default_rng(3)
+    lv = nr.nf4_levels()
+    rows, K = 3, 1024
+    scales = rng.uniform(0.01, 0.05, size=rows * K // 64)
+    codes_in = rng.integers(0, 16, size=(rows * K // 64, 64))
+    codes_in[:, 0] = 0                                   # level -1: absmax = scale
+    w = (lv[codes_in] * scales[:, None]).reshape(rows, K)
+    codes, sq, c2 = nr.quantize_nf4(w)
+    assert c2.shape == (1,) and abs(float(c2[0]) - scales.max()) <= 2 ** -24 * scales.max()  # stored as float32
+    np.testing.assert_array_equal(codes.reshape(-1, 64), codes_in)
+    err = np.abs(nr.dequantize_nf4(codes, sq, c2) - w).max()
+    assert err <= float(c2[0]) / 127 / 2 + 1e-12
+
+
 def test_projection_row_blocks():
     rng = np.random.default_rng(2)
     B, N, dm, H, Hkv, D = 1, 8, 256, 4, 2, 32
