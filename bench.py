@@ -735,6 +735,8 @@ def main():
                     help="skip the few-step timing of the other workload shapes")
     ap.add_argument("--no-rope", action="store_true", help="skip the step with RoPE + Position Interpolation")
     ap.add_argument("--no-nf4", action="store_true", help="skip the NF4 QKV projection timing")
+    ap.add_argument("--nf4-only", action="store_true",
+                    help="time only the NF4 QKV projection (--steps / --warmup launches) and print its JSON")
     ap.add_argument("--sweep", action="store_true",
                     help="time every selectable kernel variant on every workload shape and exit")
     ap.add_argument("--extra-workloads", default=f"{I.QWEN3_8B_16K.name},{I.LLAMA2_70B_32K.name}",
@@ -745,6 +747,10 @@ def main():
         args.ref_step_seconds = min(5.0, 120.0 / max(args.steps, 1))
     if args.sweep:
         run_sweep(args, torch.device("cuda", 0))
+        return
+    if args.nf4_only:
+        print(json.dumps(nf4_projection(torch.device("cuda", 0), load_peaks()[0], steps=args.steps,
+                                        warmup=args.warmup)), flush=True)
         return
     world, rank, local = dist_setup()
     try:

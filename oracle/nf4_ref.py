@@ -25,6 +25,9 @@ Readings taken where the pages are silent (listed in the design notes):
 * the second level is symmetric int8 absmax: scale' = round(127 scale / c) c / 127
   with c the block's largest scale; codes are chosen against the exact
   first-level scale (nearest level of w / absmax);
+* the GEMM's operand: W' in bf16, formed as level * (code * c2 / 127) with
+  each operation a float32 rounding, then rounded to bf16 (a bitsandbytes-like
+  fp32 dequantization feeding a bf16 GEMM);
 * the projection: [q | k | v] = X W^T with W [(H + 2 Hkv) D, d_model] the
   dequantized NF4 weight (level * scale'), X bf16 activations; q, k, v come
   out in the (batch, sequence, heads, head_dim) layout as row blocks of W.
@@ -39,7 +42,7 @@ import numpy as np
 from oracle.rope_ref import round_bf16
 
 __all__ = ["NF4_DELTA", "nf4_levels", "quantize_nf4", "dequantize_nf4", "nf4_qkv_projection",
-           "bits_per_weight", "round_bf16", "unpack_codes"]
+           "bits_per_weight", "round_bf16", "unpack_codes", "dequantize_nf4_bf16"]
 
 NF4_DELTA = 0.5 * (1.0 / 30.0 + 1.0 / 32.0)
 BLOCK = 64
@@ -90,6 +93,23 @@ def dequantize_nf4(codes, scale_codes, c2) -> np.ndarray:
     return (lv[codes.reshape(-1, BLOCK)] * scale[:, None]).reshape(rows, K)
 
 
+def dequantize_nf4_bf16(codes, scale_codes, c2) -> np.ndarray:
+    """The dequantized weight as the GEMM's bf16 operand, in the precision the
+    design states for it (float64 result holding bf16 values): the level table
+    rounded to float32; s = float32(code) * c2 then / 127, each step a float32
+    operation rounded to nearest; level * s in float32; then rounded to the
+    nearest bf16 (ties to even).  Within one bf16 ulp of dequantize_nf4."""
+    codes = np.asarray(codes)
+    rows, K = codes.shape
+    lv32 = nf4_levels().astype(np.float32)
+    sq = np.asarray(scale_codes).astype(np.float32)
+    c2_32 = np.asarray(c2, dtype=np.float32)[np.arange(sq.size) // DQ_BLOCK]
+    s32 = (sq * c2_32) / np.float32(127.0)
+    w32 = lv32[codes.reshape(-1, BLOCK)] * s32[:, None]
+    assert w32.dtype == np.float32
+    return round_bf16(w32).reshape(rows, K)
+
+
 def unpack_codes(packed) -> np.ndarray:
     """uint8 [rows, K/2] with two codes a byte (element 2j in the low nibble)
     -> uint8 [rows, K]."""
@@ -103,13 +123,11 @@ def unpack_codes(packed) -> np.ndarray:
 def nf4_qkv_projection(x, codes, scale_codes, c2, H: int, Hkv: int, D: int, bf16_weights: bool = False):
     """x [B, N, d_model] -> (q [B,N,H,D], k [B,N,Hkv,D], v [B,N,Hkv,D]) with
     the dequantized weight W [(H + 2 Hkv) D, d_model]: [q | k | v] = x W^T.
-    bf16_weights rounds W to bf16 first (the tensor cores' operand type, the
-    reading of the bf16 GEMM)."""
+    bf16_weights takes W as the GEMM's bf16 operand (dequantize_nf4_bf16, the
+    tensor cores' operand type) instead of the exact dequantized values."""
     x = np.asarray(x, dtype=np.float64)
     B, N, _ = x.shape
-    w = dequantize_nf4(codes, scale_codes, c2)
-    if bf16_weights:
-        w = round_bf16(w)
+    w = dequantize_nf4_bf16(codes, scale_codes, c2) if bf16_weights else dequantize_nf4(codes, scale_codes, c2)
     y = x @ w.T
     q = y[..., : H * D].reshape(B, N, H, D)
     k = y[..., H * D:(H + Hkv) * D].reshape(B, N, Hkv, D)

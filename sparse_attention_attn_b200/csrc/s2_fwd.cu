@@ -392,10 +392,17 @@ __global__ void __launch_bounds__(320, 1)
             for (int c = 0; c < 128; ++c)
               if (c > row) sr[c >> 5][c & 31] = __float_as_uint(neg_inf());
           }
+          // row max with three-input max instructions (exact: the same
+          // value as pairwise maxima), four independent chains
           float m4[4] = {neg_inf(), neg_inf(), neg_inf(), neg_inf()};
 #pragma unroll
-          for (int c = 0; c < 128; ++c) m4[c & 3] = fmaxf(m4[c & 3], __uint_as_float(sr[c >> 5][c & 31]));
-          const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl2;
+          for (int c = 0; c < 128; c += 8) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              m4[u] = fmax3(m4[u], __uint_as_float(sr[c >> 5][(c & 31) + 2 * u]),
+                            __uint_as_float(sr[c >> 5][(c & 31) + 2 * u + 1]));
+          }
+          const float mx = fmax3(fmaxf(m4[0], m4[1]), m4[2], m4[3]) * sl2;
           float alpha = 1.f;
           bool resc = false;
           if (j == 0) {

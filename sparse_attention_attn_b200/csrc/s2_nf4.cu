@@ -18,7 +18,7 @@
 // s2_nf4_qkv_kernel computes [q | k | v] = x W'^T on the tensor cores with the
 // dequantization fused in: W' never exists in global memory.  The UMMA runs
 // with the weight as its A operand held in TMEM: M = 128 weight rows, N = 256
-// tokens, K = 16.  Four dequantization warps, one per TMEM lane quarter, turn
+// tokens, K = 16.  Dequantization warps, one per TMEM lane quarter, turn
 // each 64-element block of their row into 32 packed bf16 pairs and write them
 // straight into a TMEM stage with tcgen05.st, so the dequantized operand costs
 // no shared-memory traffic; x comes in by TMA (128-byte swizzle, K-major B
@@ -27,11 +27,12 @@
 // 64 elements is one first-level quantization block, so each thread forms one
 // scale per stage.
 //
-// Warp roles (320 threads, one CTA per SM, persistent over the tiles):
-//   0    producer: TMA of x [256 tokens x 64] and codes [128 rows x 32 B]
-//   1    UMMA issuer (one elected lane)
-//   2-5  dequantization into the TMEM A stages
-//   6-9  epilogue: TMEM -> bf16 staging in shared memory -> TMA store to q / k / v
+// Warp roles (448 threads, one CTA per SM, persistent over the tiles):
+//   0      producer: TMA of x [256 tokens x 64] and codes [128 rows x 32 B]
+//   1      UMMA issuer (one elected lane)
+//   2-9    dequantization into the TMEM A stages, two groups of four taking
+//          alternate stages
+//   10-13  epilogue: TMEM -> bf16 staging in shared memory -> TMA store to q / k / v
 // TMEM: accumulator columns [0, 256), A stages [256 + 32 s, 256 + 32 s + 32).
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -64,13 +65,14 @@ struct Nf4Cfg {
   static constexpr int O_WARP_BYTES = BT * 32 * 2;  // one epilogue warp's staging: 16 KB
   static constexpr int SMEM_BYTES = NS * (X_BYTES + C_BYTES) + 4 * O_WARP_BYTES + 1024;
   static constexpr int TM_A = 256;
-  static constexpr int THREADS = 320;
+  static constexpr int DQ_WARPS = 8;                // two groups of four
+  static constexpr int THREADS = 32 * (2 + DQ_WARPS + 4);
   static_assert(TM_A + 32 * NS <= 512, "A stages must fit in TMEM beside the accumulator");
   static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
 
 template <int NS>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(448, 1)
     s2_nf4_qkv_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmC,
                       const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const Nf4Args a) {
@@ -93,7 +95,7 @@ __global__ void __launch_bounds__(320, 1)
     abort_flag = 0;
     for (int s = 0; s < NS; ++s) {
       mbar_init(smem_u32(&bar_full[s]), 1);
-      mbar_init(smem_u32(&bar_afull[s]), 4);  // one arrival per dequantization warp
+      mbar_init(smem_u32(&bar_afull[s]), 4);  // one arrival per warp of the stage's dequantization group
       mbar_init(smem_u32(&bar_empty[s]), 1);
     }
     mbar_init(smem_u32(&bar_acc_full), 1);
@@ -177,30 +179,38 @@ __global__ void __launch_bounds__(320, 1)
       drain_wait(smem_u32(&bar_drain), 0);
     }
     __syncwarp();
-  } else if (warp < 6) {
+  } else if (warp < 2 + C::DQ_WARPS) {
     // ------------------------------------------------------------ dequantization
-    const int sub = warp & 3, row = 32 * sub + lane;
+    // Two groups of four warps take alternate stages (group g the stages
+    // L = g, g + 2, ...), so one group's shuffles and TMEM store overlap the
+    // other's; within a group warp w serves TMEM lanes 32 (w mod 4) + [0, 32).
+    const int sub = warp & 3, row = 32 * sub + lane, grp = (warp - 2) >> 2;
     const float table = lane_level(a.lv, lane);
     const uint32_t tA = tmem + (static_cast<uint32_t>(32 * sub) << 16) + C::TM_A;
+    auto advance = [&](int& t, int& k) {
+      if (++k == KB) {
+        k = 0;
+        t += gridDim.x;
+      }
+    };
     // scale code and second-level scale of (tile, kb) for this thread's row,
-    // fetched one stage ahead of their use
-    auto fetch = [&](int tile, int kb, int& q, float& c) {
-      const long long blk = static_cast<long long>((tile % a.tiles_w) * C::BW + row) * KB + kb;
+    // fetched one own stage ahead of their use
+    auto fetch = [&](int t, int k, int& q, float& c) {
+      const long long blk = static_cast<long long>((t % a.tiles_w) * C::BW + row) * KB + k;
       q = a.sq[blk];
       c = __ldg(a.c2 + (blk >> 8));
     };
-    int tile = blockIdx.x, kb = 0, L = 0;
+    int tile = blockIdx.x, kb = 0, L = grp;
+    if (grp == 1) advance(tile, kb);
     int qn = 0;
     float cn = 0.f;
-    if (tile < ntiles) fetch(tile, 0, qn, cn);
+    if (tile < ntiles) fetch(tile, kb, qn, cn);
     while (tile < ntiles) {
       const int q = qn;
       const float c2 = cn;
-      int ntile = tile, nkb = kb + 1;
-      if (nkb == KB) {
-        nkb = 0;
-        ntile += gridDim.x;
-      }
+      int ntile = tile, nkb = kb;
+      advance(ntile, nkb);
+      advance(ntile, nkb);
       if (ntile < ntiles) fetch(ntile, nkb, qn, cn);
       const int s = L % NS;
       if (!warp_wait(smem_u32(&bar_full[s]), (L / NS) & 1, wc, 64)) break;
@@ -224,7 +234,7 @@ __global__ void __launch_bounds__(320, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&bar_afull[s]));
-      ++L;
+      L += 2;
       tile = ntile;
       kb = nkb;
     }
@@ -257,19 +267,33 @@ __global__ void __launch_bounds__(320, 1)
       if (lane == 0) bulk_wait_read_all();
       __syncwarp();
       tc_fence_after();
+      // two halves of 128 tokens: each loaded into registers as bf16 pairs
+      // (tokens 2i, 2i + 1) and written to the staging area; the accumulator
+      // is released once the second half is in registers
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        uint32_t r[16];
-        tmem_ld16(tD + 16 * c, r);
-        tmem_wait_ld();
+      for (int h = 0; h < 2; ++h) {
+        uint32_t pk[64];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) st_shared_bf16(stage + (16 * c + j) * 64 + lane * 2, __uint_as_float(r[j]));
+        for (int c = 0; c < 8; ++c) {
+          uint32_t r[16];
+          tmem_ld16(tD + 128 * h + 16 * c, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            pk[8 * c + i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+        }
+        if (h == 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&bar_acc_empty));
+        }
+#pragma unroll
+        for (int j = 0; j < 128; ++j)
+          st_shared_u16(stage + (128 * h + j) * 64 + lane * 2, static_cast<uint16_t>(pk[j >> 1] >> (16 * (j & 1))));
       }
-      tc_fence_before();
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(smem_u32(&bar_acc_empty));
         tma_store_2d(map, stage, col, tt * C::BT);
         bulk_commit_group();
       }

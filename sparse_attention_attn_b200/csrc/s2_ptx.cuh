@@ -198,10 +198,8 @@ __device__ __forceinline__ void bulk_reduce_add_f32(void* dst, uint32_t src, uin
                : "memory");
 }
 
-// One bf16 (round to nearest even) to shared memory.
-__device__ __forceinline__ void st_shared_bf16(uint32_t addr, float v) {
-  const __nv_bfloat16 b = __float2bfloat16_rn(v);
-  asm volatile("st.shared.b16 [%0], %1;" ::"r"(addr), "h"(*reinterpret_cast<const unsigned short*>(&b)) : "memory");
+__device__ __forceinline__ void st_shared_u16(uint32_t addr, uint16_t v) {
+  asm volatile("st.shared.b16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
 }
 
 __device__ __forceinline__ void st_shared_f32(uint32_t addr, float v) {
@@ -380,6 +378,14 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// max(a, b, c) in one instruction (sm_100 three-input max; NaN inputs are
+// ignored as in fmaxf).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
 }
 
 // Two floats -> packed bf16x2 (round to nearest even); lo in the low half.

@@ -1,14 +1,14 @@
 """GPU parity of the NF4 kernels (through the C ABI) against the fp64 oracle
 in oracle/nf4_ref.py.
 
-* dequantization alone: every element of W' is within one bf16 ulp of the
-  exact level * scale, and equal to its round-to-nearest-even bf16 value for
-  all but a tiny fraction (the kernel's scale and product are fp32 roundings);
-* the fused QKV projection against the oracle's x W^T with W rounded to bf16
-  (the operand type of the GEMM): element-wise within half a bf16 ulp of the
-  result (|y| 2^-8) plus 1e-3 of the result's rms (fp32 accumulation order and the rare
-  weight that the fp32 product rounds to the neighbouring bf16), relative
-  Frobenius error within 3e-3; shapes with ragged token tails, one token, GQA
+* dequantization alone: bit-exact against the oracle's bf16 operand in the
+  stated precision (float32 steps, then bf16), within one bf16 ulp of the
+  exact level * scale everywhere and equal to its nearest bf16 for all but a
+  tiny fraction;
+* the fused QKV projection against the oracle's x W'^T with that bf16
+  operand: element-wise within half a bf16 ulp of the result (|y| 2^-8) plus
+  2e-4 of the result's rms (fp32 accumulation order), relative Frobenius error
+  within 3e-3; shapes with ragged token tails, one token, GQA
   head counts, head dim 64, and weights quantized by the oracle from normal
   draws as well as random storage;
 * the full-size projection of a LLaMA2-7B layer at 8192 tokens on sampled
@@ -36,10 +36,15 @@ def _to64(t):
 def _check_proj(name, got, ref):
     rms = float(np.sqrt(np.mean(ref ** 2)))
     err = np.abs(got - ref)
-    bound = np.abs(ref) * 2.0 ** -8 + 1e-3 * rms
+    bound = np.abs(ref) * 2.0 ** -8 + 2e-4 * rms
     worst = float(np.max(err - bound))
     frob = float(np.linalg.norm(got - ref) / np.linalg.norm(ref))
     print(f"{name}: max_abs {err.max():.3e} rms {rms:.3e} rel_frob {frob:.2e}")
+    over = np.argwhere((err - bound).reshape(-1) > 0).reshape(-1)
+    if over.size:
+        g, r = got.reshape(-1), ref.reshape(-1)
+        print(f"  {over.size} elements over the bound; first: " + ", ".join(
+            f"[{i}] ref {r[i]:.6f} got {g[i]:.6f} rn(ref) {float(nr.round_bf16(r[i])):.6f}" for i in over[:6]))
     assert worst <= 0, f"{name}: element error exceeds half an ulp + 1e-3 rms by {worst:.3e}"
     assert frob <= 3e-3, f"{name}: relative Frobenius error {frob:.2e}"
 
@@ -64,8 +69,11 @@ def test_dequant_against_oracle(rows, K):
     codes, sq, c2 = I.make_nf4_weights(rows, K, seed=rows + K)
     w = s2.nf4_dequantize(codes.to(DEV), sq.to(DEV), c2.to(DEV))
     torch.cuda.synchronize()
-    exact = nr.dequantize_nf4(nr.unpack_codes(codes.numpy()), sq.numpy(), c2.numpy())
+    c = nr.unpack_codes(codes.numpy())
+    exact = nr.dequantize_nf4(c, sq.numpy(), c2.numpy())
     got = _to64(w)
+    # the stated precision (float32 steps, then bf16): bit-exact
+    np.testing.assert_array_equal(got, nr.dequantize_nf4_bf16(c, sq.numpy(), c2.numpy()))
     rn = nr.round_bf16(exact)
     ulp = np.maximum(np.abs(rn), 1e-30) * 2.0 ** -7
     assert np.all(np.abs(got - exact) <= ulp), "an element is more than one bf16 ulp from level * scale"

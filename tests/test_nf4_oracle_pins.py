@@ -104,3 +104,32 @@ def test_projection_row_blocks():
     np.testing.assert_allclose(q[0, 3, 1], x[0, 3] @ wd[D:2 * D].T, atol=1e-12, rtol=0)
     np.testing.assert_allclose(k[0, 5, 1], x[0, 5] @ wd[(H + 1) * D:(H + 2) * D].T, atol=1e-12, rtol=0)
     np.testing.assert_allclose(v[0, 7, 0], x[0, 7] @ wd[(H + Hkv) * D:(H + Hkv + 1) * D].T, atol=1e-12, rtol=0)
+
+
+def test_bf16_operand_reading():
+    """dequantize_nf4_bf16: within one bf16 ulp of the exact dequantized value
+    everywhere, equal to its nearest bf16 almost everywhere (the float32 steps
+    decide only near-ties), and bit-exact against a hand evaluation of the
+    float32 steps for a few entries (Python floats through struct)."""
+    import struct
+
+    def f32(v):
+        return struct.unpack("f", struct.pack("f", v))[0]
+
+    rng = np.random.default_rng(9)
+    rows, K = 16, 4096
+    codes = rng.integers(0, 16, size=(rows, K)).astype(np.uint8)
+    nblk = rows * K // 64
+    sq = rng.integers(64, 128, size=nblk).astype(np.int8)
+    c2 = rng.uniform(0.05, 0.08, size=(nblk + 255) // 256).astype(np.float32)
+    exact = nr.dequantize_nf4(codes, sq, c2)
+    w = nr.dequantize_nf4_bf16(codes, sq, c2)
+    rn = nr.round_bf16(exact)
+    assert np.all(np.abs(w - exact) <= np.abs(rn) * 2.0 ** -7)
+    assert np.mean(w == rn) >= 0.999
+    lv = nr.nf4_levels()
+    for (r, k) in [(0, 0), (3, 777), (15, 4095)]:
+        blk = (r * K + k) // 64
+        s = f32(f32(float(sq[blk]) * float(c2[blk // 256])) / 127.0)
+        v = f32(f32(float(lv[codes[r, k]])) * s)
+        assert w[r, k] == float(nr.round_bf16(np.array([v]))[0])
