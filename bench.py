@@ -189,6 +189,26 @@ def max_over_ranks(x: float, world: int, device) -> float:
     return float(t.item())
 
 
+WATCHDOG_S = 120.0
+
+
+def device_sync(limit_s: float = None, poll_s: float = 0.0005):
+    """torch.cuda.synchronize() behind a host-side watchdog: an event recorded
+    on the current stream is polled (cudaEventQuery) until it completes; if
+    the device has not finished within limit_s seconds the run stops with an
+    error instead of blocking forever.  The kernels' own waits are bounded,
+    so this only catches what they cannot (a stuck copy, a driver stall)."""
+    limit_s = WATCHDOG_S if limit_s is None else limit_s
+    ev = torch.cuda.Event()
+    ev.record()
+    t0 = time.monotonic()
+    while not ev.query():
+        if time.monotonic() - t0 > limit_s:
+            raise RuntimeError(f"watchdog: the device did not finish its work within {limit_s:.0f} s")
+        time.sleep(poll_s)
+    torch.cuda.synchronize()
+
+
 def barrier(world: int):
     if world > 1:
         import torch.distributed as dist
@@ -292,7 +312,7 @@ def run_ours(args, shape, world, rank, local):
 
     for _ in range(max(args.warmup, 3)):
         step()
-    torch.cuda.synchronize()
+    device_sync()
     if s2.device_status() != 0 or s2.device_status(ws) != 0:
         raise RuntimeError("device status reports a timeout during warm-up")
 
@@ -303,13 +323,13 @@ def run_ours(args, shape, world, rank, local):
     time.sleep(0.3)
     launches[0] = 0
     barrier(world)
-    torch.cuda.synchronize()
+    device_sync()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(args.steps):
         step()
     e1.record(stream)
-    torch.cuda.synchronize()
+    device_sync()
     barrier(world)
     ms_total = e0.elapsed_time(e1)
     gpu_launches = launches[0]
@@ -322,7 +342,7 @@ def run_ours(args, shape, world, rank, local):
     ms_arr = (ctypes.c_float * cap)()
     id_arr = (ctypes.c_int * cap)()
     n_rec = _lib.s2attn_profile_stop(ctypes.addressof(ms_arr), ctypes.addressof(id_arr), cap)
-    torch.cuda.synchronize()
+    device_sync()
     clk = clocks.stop()
     per_kernel = {}
     for i in range(max(n_rec, 0)):
@@ -383,13 +403,13 @@ def run_ours(args, shape, world, rank, local):
 
     def timed_e2e(loop, n, first, last):
         loop(2)
-        torch.cuda.synchronize()
+        device_sync()
         barrier(world)
         f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         f0.record(first)
         loop(n)
         f1.record(last)
-        torch.cuda.synchronize()
+        device_sync()
         barrier(world)
         return max_over_ranks(f0.elapsed_time(f1) / n, world, dev)
 
@@ -485,14 +505,14 @@ def dense_ratio(shape: I.Shape, dev, args):
         for _ in range(3):
             o, lse = s2.s2attn_forward(q, k, v, G)
             s2.s2attn_backward(q, k, v, o, lse, do, G, workspace=ws)
-        torch.cuda.synchronize()
+        device_sync()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
         for _ in range(steps):
             o, lse = s2.s2attn_forward(q, k, v, G)
             s2.s2attn_backward(q, k, v, o, lse, do, G, workspace=ws)
         b.record()
-        torch.cuda.synchronize()
+        device_sync()
         return a.elapsed_time(b) / steps
 
     n = max(5, min(args.steps, 20))
@@ -525,13 +545,13 @@ def rope_step(shape: I.Shape, dev, peaks, ms_plain: float, steps: int = 10, warm
 
     for _ in range(warmup):
         step()
-    torch.cuda.synchronize()
+    device_sync()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record()
     for _ in range(steps):
         step()
     b.record()
-    torch.cuda.synchronize()
+    device_sync()
     ms = a.elapsed_time(b) / steps
     cap = 8 * steps + 8
     assert _lib.s2attn_profile_start(cap) == 0
@@ -588,13 +608,13 @@ def nf4_projection(dev, peaks, steps: int = 20, warmup: int = 3):
     def timed(fn):
         for _ in range(warmup):
             fn()
-        torch.cuda.synchronize()
+        device_sync()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
         for _ in range(steps):
             fn()
         b.record()
-        torch.cuda.synchronize()
+        device_sync()
         return a.elapsed_time(b) / steps
 
     ms_f, ms_u, ms_d = timed(fused), timed(unfused), timed(dequant_only)
@@ -629,13 +649,13 @@ def other_workload(shape: I.Shape, dev, peaks, steps: int = 5, warmup: int = 3):
 
     for _ in range(warmup):
         step()
-    torch.cuda.synchronize()
+    device_sync()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record()
     for _ in range(steps):
         step()
     b.record()
-    torch.cuda.synchronize()
+    device_sync()
     if s2.device_status() != 0 or s2.device_status(ws) != 0:
         raise RuntimeError(f"device status reports a timeout on {shape.name}")
     ms = a.elapsed_time(b) / steps
@@ -678,13 +698,13 @@ def run_sweep(args, dev):
         def timed(fn):
             for _ in range(3):
                 fn()
-            torch.cuda.synchronize()
+            device_sync()
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record()
             for _ in range(steps):
                 fn()
             b.record()
-            torch.cuda.synchronize()
+            device_sync()
             return a.elapsed_time(b) / steps
 
         for kind, specs in (("fwd", fwd_specs), ("bwd", bwd_specs)):

@@ -113,3 +113,40 @@ def test_reference_arm_prints_the_contract_line():
     import bench
     from sparse_attention_attn_b200 import inputs as I
     assert d["config"] == bench.workload_config(I.TINY, 1)
+
+
+def test_watchdog_sync_stops_a_stuck_device(monkeypatch):
+    """bench.device_sync polls an event and raises once the limit passes
+    (a fake event that never completes stands in for a stuck device); a
+    device that finishes returns normally."""
+    import pytest
+    import torch
+
+    import bench
+
+    class Never:
+        def record(self):
+            pass
+
+        def query(self):
+            return False
+
+    class After:
+        n = 0
+
+        def record(self):
+            pass
+
+        def query(self):
+            After.n += 1
+            return After.n > 3
+
+    synced = []
+    monkeypatch.setattr(torch.cuda, "synchronize", lambda: synced.append(1))
+    monkeypatch.setattr(torch.cuda, "Event", lambda *a, **k: Never())
+    with pytest.raises(RuntimeError, match="watchdog"):
+        bench.device_sync(limit_s=0.05)
+    assert not synced
+    monkeypatch.setattr(torch.cuda, "Event", lambda *a, **k: After())
+    bench.device_sync(limit_s=5)
+    assert synced == [1]
