@@ -61,7 +61,8 @@ typedef enum {
   S2ATTN_ERR_MISALIGNED = 3,     /* a pointer is not 16-byte aligned */
   S2ATTN_ERR_CUDA = 4,           /* a CUDA runtime/driver call or a launch failed */
   S2ATTN_ERR_DEVICE_TIMEOUT = 5, /* a kernel's bounded wait ran out (device status word) */
-  S2ATTN_ERR_WORKSPACE = 6       /* workspace missing or smaller than required */
+  S2ATTN_ERR_WORKSPACE = 6,      /* workspace missing or smaller than required */
+  S2ATTN_ERR_DEVICE_BOUNDS = 7   /* debug build only: a kernel's computed index left its tensor (device status word) */
 } s2attn_status;
 
 /* Opaque CUDA stream handle (cudaStream_t) without pulling in CUDA headers. */
@@ -343,6 +344,16 @@ S2ATTN_API int s2attn_bwd_noalloc(const void* q, const void* k, const void* v, c
  */
 S2ATTN_API int s2attn_selftest_wait_timeout(uint32_t* status_out, uint64_t limit_ns, s2attn_stream_t stream);
 
+/*
+ * 1 if this library is the debug build (libs2attn_debug.so, compiled with
+ * S2ATTN_DEBUG_CHECKS): its kernels check every computed global index
+ * against its tensor before the access, skip an access that falls outside
+ * and record S2ATTN_ERR_DEVICE_BOUNDS with the site in the device status word
+ * (read by s2attn_device_status).  0 for the default build, which has no
+ * such checks.
+ */
+S2ATTN_API int s2attn_debug_checks(void);
+
 /* Number of kernel launches the last s2attn_fwd / s2attn_bwd call made on this host thread. */
 S2ATTN_API int s2attn_last_launch_count(void);
 
@@ -387,8 +398,8 @@ S2ATTN_API int s2attn_plan(int B, int H, int Hkv, int N, int D, int G, int num_s
  * items; keys bwd=split|fused (backward path; fused exists for head dim 128),
  * fwd_order=snake|pairs (forward work order), fwd_kv=N (forward K/V ring
  * depth: 4 at head dim 128, 4/6/8 at 64), bwd_stages=N (split backward
- * stages: 2-3 at head dim 128, 3-4 at 64), nf4_stages=4|6 (pipeline
- * depth of s2attn_nf4_qkv); values that do not exist for a call's head dim
+ * stages: 2-3 at head dim 128, 3-4 at 64), nf4_stages=3|4 and nf4_dq=8|12
+ * (pipeline depth and dequantization warps of s2attn_nf4_qkv); values that do not exist for a call's head dim
  * are ignored.  s2attn_bwd_workspace_bytes answers for the
  * path in force when it is called.  Returns S2ATTN_OK.
  */

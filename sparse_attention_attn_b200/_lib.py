@@ -10,7 +10,9 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libs2attn.so")
+# S2ATTN_DEBUG=1 selects the debug build (in-kernel index checks; built by
+# `python -m sparse_attention_attn_b200.build --debug`)
+LIB_PATH = os.path.join(_HERE, "libs2attn_debug.so" if os.environ.get("S2ATTN_DEBUG") == "1" else "libs2attn.so")
 
 S2ATTN_OK = 0
 S2ATTN_ERR_INVALID_ARG = 1
@@ -19,6 +21,7 @@ S2ATTN_ERR_MISALIGNED = 3
 S2ATTN_ERR_CUDA = 4
 S2ATTN_ERR_DEVICE_TIMEOUT = 5
 S2ATTN_ERR_WORKSPACE = 6
+S2ATTN_ERR_DEVICE_BOUNDS = 7
 
 _vp = ctypes.c_void_p
 _i = ctypes.c_int
@@ -33,6 +36,7 @@ SIGNATURES = {
     "s2attn_status_string": (ctypes.c_char_p, [_i]),
     "s2attn_selftest_wait_timeout": (_i, [_vp, ctypes.c_uint64, _vp]),
     "s2attn_last_launch_count": (_i, []),
+    "s2attn_debug_checks": (_i, []),
     "s2attn_last_cuda_error": (_i, []),
     "s2attn_cuda_error_string": (ctypes.c_char_p, [_i]),
     "s2attn_profile_start": (_i, [_i]),

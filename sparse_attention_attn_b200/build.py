@@ -2,6 +2,7 @@
 
     python -m sparse_attention_attn_b200.build          # build if sources changed
     python -m sparse_attention_attn_b200.build --force  # always rebuild
+    python -m sparse_attention_attn_b200.build --debug  # libs2attn_debug.so: kernels with index checks
 
 The library is plain CUDA C++ compiled by nvcc; it links only the CUDA runtime
 (statically) and resolves cuTensorMapEncodeTiled through the runtime's driver
@@ -20,7 +21,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libs2attn.so")
-STAMP = LIB + ".srchash"
+LIB_DEBUG = os.path.join(PKG, "libs2attn_debug.so")
 
 SOURCES = ["s2attn.cu", "s2_fwd.cu", "s2_bwd.cu", "s2_bwd_fused.cu", "s2_rope.cu", "s2_segment.cu", "s2_nf4.cu"]
 HEADERS = ["s2_ptx.cuh", "s2_common.cuh"]
@@ -34,7 +35,7 @@ def nvcc_path() -> str:
     raise RuntimeError("nvcc not found: the CUDA toolkit is required to build libs2attn.so")
 
 
-def source_hash() -> str:
+def source_hash(debug: bool = False) -> str:
     h = hashlib.sha256()
     files = [os.path.join(CSRC, f) for f in SOURCES + HEADERS] + [os.path.join(INCLUDE, "s2attn.h")]
     for f in files:
@@ -43,38 +44,47 @@ def source_hash() -> str:
             h.update(fh.read())
     h.update(" ".join(ARCH).encode())
     h.update(__file__.encode())
+    h.update(b"debug" if debug else b"release")
     return h.hexdigest()
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile libs2attn.so unless an up-to-date build exists.  Returns its path."""
-    digest = source_hash()
-    if not force and os.path.exists(LIB) and os.path.exists(STAMP):
-        with open(STAMP) as fh:
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
+    """Compile libs2attn.so (or, with debug, libs2attn_debug.so: the same
+    sources with the kernels' index checks compiled in) unless an up-to-date
+    build exists.  Returns its path.  The sources compile in parallel."""
+    lib = LIB_DEBUG if debug else LIB
+    stamp = lib + ".srchash"
+    digest = source_hash(debug)
+    if not force and os.path.exists(lib) and os.path.exists(stamp):
+        with open(stamp) as fh:
             if fh.read().strip() == digest:
-                return LIB
+                return lib
     nvcc = nvcc_path()
-    objs = []
-    tmpdir = os.path.join(PKG, "_build")
+    tmpdir = os.path.join(PKG, "_build_debug" if debug else "_build")
     os.makedirs(tmpdir, exist_ok=True)
     common = ARCH + ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-fvisibility=hidden",
                      "-I" + INCLUDE, "-I" + CSRC, "--expt-relaxed-constexpr"]
+    if debug:
+        common += ["-DS2ATTN_DEBUG_CHECKS"]
     if verbose:
         common += ["-Xptxas", "-v"]
+    objs, procs = [], []
     for src in SOURCES:
         obj = os.path.join(tmpdir, src.replace(".cu", ".o"))
-        cmd = [nvcc] + common + ["-c", os.path.join(CSRC, src), "-o", obj]
-        subprocess.run(cmd, check=True)
+        procs.append((src, subprocess.Popen([nvcc] + common + ["-c", os.path.join(CSRC, src), "-o", obj])))
         objs.append(obj)
-    tmp_lib = LIB + ".tmp"
+    failed = [src for src, p in procs if p.wait() != 0]
+    if failed:
+        raise RuntimeError(f"nvcc failed on {', '.join(failed)}")
+    tmp_lib = lib + ".tmp"
     cmd = [nvcc] + ARCH + ["-shared", "-cudart", "static", "-o", tmp_lib] + objs
     subprocess.run(cmd, check=True)
-    os.replace(tmp_lib, LIB)
-    with open(STAMP, "w") as fh:
+    os.replace(tmp_lib, lib)
+    with open(stamp, "w") as fh:
         fh.write(digest)
-    return LIB
+    return lib
 
 
 if __name__ == "__main__":
-    path = build(force="--force" in sys.argv, verbose="-v" in sys.argv)
+    path = build(force="--force" in sys.argv, verbose="-v" in sys.argv, debug="--debug" in sys.argv)
     print(path)

@@ -103,8 +103,10 @@ __global__ void __launch_bounds__(256) s2_bwd_pre_kernel(const BwdPreArgs a) {
     __syncthreads();
     if (tid < kTile) {
       const size_t idx = static_cast<size_t>(bh) * d.N + t0 + tid;
-      a.ndelta[idx] = -red[tid];
-      a.nlse2[idx] = -a.lse[idx] * kLog2e;
+      if (in_bounds(a.status, static_cast<long long>(idx), static_cast<long long>(d.B) * d.H * d.N, 43)) {
+        a.ndelta[idx] = -red[tid];
+        a.nlse2[idx] = -a.lse[idx] * kLog2e;
+      }
     }
     __syncthreads();
   }
@@ -426,6 +428,8 @@ __global__ void __launch_bounds__(352, 1)
         const TileWork& w = cur.w;
         const int tk0 = original_row(d, w.g * d.G + w.tile * kTile, shift_of_head(d, w.h));
         const size_t grow = (static_cast<size_t>(w.b) * d.N + tk0 + row) * d.Hkv + w.kvh;
+        const bool grow_ok =
+            in_bounds(wc.status, static_cast<long long>(grow), static_cast<long long>(d.B) * d.N * d.Hkv, 44);
         __nv_bfloat16* dvrow = static_cast<__nv_bfloat16*>(a.dv) + grow * D + half * (D / 2);
         __nv_bfloat16* dkrow = static_cast<__nv_bfloat16*>(a.dk) + grow * D + half * (D / 2);
         uint32_t r[D / 64][32], r2[D / 64][32];
@@ -440,7 +444,7 @@ __global__ void __launch_bounds__(352, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&bar_acc_free));
 #pragma unroll
-        for (int c = 0; c < D / 64; ++c) {
+        for (int c = 0; c < D / 64 && grow_ok; ++c) {
           if (a.kv_v8) {
             store_row32_v8(dvrow + c * 32, r[c], 1.f);
             store_row32_v8(dkrow + c * 32, r2[c], a.scale);
@@ -757,8 +761,12 @@ __global__ void __launch_bounds__(384, 1)
       const TileWork& w = c.w;
       const int t0 = original_row(d, w.g * d.G + w.tile * kTile, shift_of_head(d, w.h));
       const size_t ridx = (static_cast<size_t>(w.b) * d.H + w.h) * d.N + t0 + row;
-      l2 = a.nlse2[ridx];
-      dl = a.ndelta[ridx];
+      l2 = 0.f;
+      dl = 0.f;
+      if (in_bounds(wc.status, static_cast<long long>(ridx), static_cast<long long>(d.B) * d.H * d.N, 45)) {
+        l2 = a.nlse2[ridx];
+        dl = a.ndelta[ridx];
+      }
     };
     DqCursor cur;
     cur.first(d, ps, a.hist);
@@ -857,6 +865,8 @@ __global__ void __launch_bounds__(384, 1)
         for (int i = 0; i < CH; ++i) {
           const int rr = i * (32 / CH) + lane / CH, ch = lane % CH;
           float4 v = lds_f4(stage + rr * C::ROW_OUT + ((ch ^ (rr % CH)) << 4));
+          const long long qrow = (static_cast<long long>(w.b) * d.N + tq0 + quarter * 32 + rr) * d.H + w.h;
+          if (!in_bounds(wc.status, qrow, static_cast<long long>(d.B) * d.N * d.H, 46)) continue;
           float4* dst = reinterpret_cast<float4*>(dq0 + static_cast<size_t>(rr) * d.H * D + ch * 8);
           if (a.dq_accumulate) {  // dq += this piece (8 bf16 values, summed in fp32)
             const float4 old = *dst;

@@ -348,6 +348,26 @@ struct BwdMaps {
 template <int D>
 cudaError_t launch_bwd_pre(const BwdPreArgs& pre, int num_sms, cudaStream_t stream);
 
+// Index checks of the debug build (compiled with -DS2ATTN_DEBUG_CHECKS; they
+// compile to nothing otherwise).  A computed global index outside [0, n)
+// records status code 7 (S2ATTN_ERR_DEVICE_BOUNDS in the C ABI) and the site
+// in the device status word pair -- the first failure wins -- and the caller
+// skips the access.
+constexpr uint32_t kDevBounds = 7;
+__device__ __forceinline__ bool in_bounds(uint32_t* status, long long idx, long long n, uint32_t where) {
+#ifdef S2ATTN_DEBUG_CHECKS
+  if (idx >= 0 && idx < n) return true;
+  if (status != nullptr && atomicCAS(status, 0u, kDevBounds) == 0u) status[1] = where;
+  return false;
+#else
+  (void)status;
+  (void)idx;
+  (void)n;
+  (void)where;
+  return true;
+#endif
+}
+
 // The 16 NF4 levels, ascending (index = 4-bit code), passed to the NF4 kernels.
 struct Nf4Levels {
   float v[16];
@@ -367,7 +387,7 @@ struct Nf4Args {
 };
 
 cudaError_t launch_nf4_qkv(const CUtensorMap& tx, const CUtensorMap& tc, const CUtensorMap* to, const Nf4Args& a,
-                           int num_sms, cudaStream_t stream, int stages);
+                           int num_sms, cudaStream_t stream, int stages, int dq_warps);
 cudaError_t launch_nf4_dequant(const void* codes, const int8_t* sq, const float* c2, void* w, long long n_words,
                                const Nf4Levels& lv, int num_sms, cudaStream_t stream);
 

@@ -148,6 +148,7 @@ __global__ void __launch_bounds__(320, 1)
       const int s = qu % NQ, r = qu / NQ;
       if (r > 0 && !warp_wait(smem_u32(&bar_qempty[s]), (r - 1) & 1, wc, 10)) return false;
       const int row = original_row(d, it.g * d.G + t * kTile, it.sh);
+      if (present && !in_bounds(a.status, row, d.N - kTile + 1, 41)) present = false;
       if (elect_one()) {
         if (present) {
           mbar_arrive_expect_tx(smem_u32(&bar_qfull[s]), C::TILE_BYTES);
@@ -166,7 +167,8 @@ __global__ void __launch_bounds__(320, 1)
       const int s = L % NS, r = L / NS;
       if (r > 0 && !warp_wait(smem_u32(&bar_empty[s]), (r - 1) & 1, wc, 11)) return false;
       // key tile j: a listed historical tile first (HGA mode), then the group's own
-      const int row = j < it.nh ? it.hist[j] * kTile : original_row_kv(d, it.g * d.G + (j - it.nh) * kTile, it.sh);
+      int row = j < it.nh ? it.hist[j] * kTile : original_row_kv(d, it.g * d.G + (j - it.nh) * kTile, it.sh);
+      if (!in_bounds(a.status, row, d.Nk - kTile + 1, 42)) row = 0;  // debug build: load a valid tile instead
       if (elect_one()) {
         mbar_arrive_expect_tx(smem_u32(&bar_full[s]), C::TILE_BYTES);
         for (int c = 0; c < D / 64; ++c)
@@ -496,7 +498,9 @@ __global__ void __launch_bounds__(320, 1)
           mbar_arrive(smem_u32(&bar_qempty[qs]));
         }
         __syncwarp();
-        a.lse[(static_cast<size_t>(it.b) * d.H + it.h) * d.N + tq] = (m_run + __log2f(l_run)) * 0.69314718055994530942f;
+        const long long li = (static_cast<long long>(it.b) * d.H + it.h) * d.N + tq;
+        if (in_bounds(a.status, li, static_cast<long long>(d.B) * d.H * d.N, 40))
+          a.lse[li] = (m_run + __log2f(l_run)) * 0.69314718055994530942f;
       } else {
         // no second tile in this item: keep the O-free phases in step
         __syncwarp();

@@ -57,7 +57,7 @@ __device__ __forceinline__ float lane_level(const Nf4Levels& lv, int lane) {
   return (lane & 1) ? t[1] : t[0];
 }
 
-template <int NS>
+template <int NS, int DQW>
 struct Nf4Cfg {
   static constexpr int BW = 128, BT = 256, BK = 64;
   static constexpr int X_BYTES = BT * BK * 2;  // 32 KB per stage
@@ -65,18 +65,19 @@ struct Nf4Cfg {
   static constexpr int O_WARP_BYTES = BT * 32 * 2;  // one epilogue warp's staging: 16 KB
   static constexpr int SMEM_BYTES = NS * (X_BYTES + C_BYTES) + 4 * O_WARP_BYTES + 1024;
   static constexpr int TM_A = 256;
-  static constexpr int DQ_WARPS = 8;                // two groups of four
+  static constexpr int DQ_WARPS = DQW;  // dequantization warps: groups of four
   static constexpr int THREADS = 32 * (2 + DQ_WARPS + 4);
+  static_assert(DQW % 4 == 0 && DQW >= 4, "whole groups of four dequantization warps");
   static_assert(TM_A + 32 * NS <= 512, "A stages must fit in TMEM beside the accumulator");
   static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
 
-template <int NS>
-__global__ void __launch_bounds__(448, 1)
+template <int NS, int DQW>
+__global__ void __launch_bounds__(Nf4Cfg<NS, DQW>::THREADS, 1)
     s2_nf4_qkv_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmC,
                       const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const Nf4Args a) {
-  using C = Nf4Cfg<NS>;
+  using C = Nf4Cfg<NS, DQW>;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -181,9 +182,11 @@ __global__ void __launch_bounds__(448, 1)
     __syncwarp();
   } else if (warp < 2 + C::DQ_WARPS) {
     // ------------------------------------------------------------ dequantization
-    // Two groups of four warps take alternate stages (group g the stages
-    // L = g, g + 2, ...), so one group's shuffles and TMEM store overlap the
-    // other's; within a group warp w serves TMEM lanes 32 (w mod 4) + [0, 32).
+    // DQ_GROUPS groups of four warps take the stages in turn (group g the
+    // stages L = g, g + DQ_GROUPS, ...), so one group's shuffles and TMEM
+    // store overlap the others'; within a group warp w serves TMEM lanes
+    // 32 (w mod 4) + [0, 32).
+    constexpr int NG = C::DQ_WARPS / 4;
     const int sub = warp & 3, row = 32 * sub + lane, grp = (warp - 2) >> 2;
     const float table = lane_level(a.lv, lane);
     const uint32_t tA = tmem + (static_cast<uint32_t>(32 * sub) << 16) + C::TM_A;
@@ -197,11 +200,15 @@ __global__ void __launch_bounds__(448, 1)
     // fetched one own stage ahead of their use
     auto fetch = [&](int t, int k, int& q, float& c) {
       const long long blk = static_cast<long long>((t % a.tiles_w) * C::BW + row) * KB + k;
-      q = a.sq[blk];
-      c = __ldg(a.c2 + (blk >> 8));
+      q = 0;
+      c = 0.f;
+      if (in_bounds(a.status, blk, static_cast<long long>(a.tiles_w) * C::BW * KB, 47)) {
+        q = a.sq[blk];
+        c = __ldg(a.c2 + (blk >> 8));
+      }
     };
     int tile = blockIdx.x, kb = 0, L = grp;
-    if (grp == 1) advance(tile, kb);
+    for (int i = 0; i < grp; ++i) advance(tile, kb);
     int qn = 0;
     float cn = 0.f;
     if (tile < ntiles) fetch(tile, kb, qn, cn);
@@ -209,13 +216,13 @@ __global__ void __launch_bounds__(448, 1)
       const int q = qn;
       const float c2 = cn;
       int ntile = tile, nkb = kb;
-      advance(ntile, nkb);
-      advance(ntile, nkb);
+#pragma unroll
+      for (int i = 0; i < NG; ++i) advance(ntile, nkb);
       if (ntile < ntiles) fetch(ntile, nkb, qn, cn);
-      const int s = L % NS;
-      if (!warp_wait(smem_u32(&bar_full[s]), (L / NS) & 1, wc, 64)) break;
       const float sc = static_cast<float>(q) * c2 / 127.f;
       const uint64_t sc2 = f2_pack(sc, sc);
+      const int s = L % NS;
+      if (!warp_wait(smem_u32(&bar_full[s]), (L / NS) & 1, wc, 64)) break;
       const uint32_t src = sC + s * C::C_BYTES + row * 32;
       const uint4 c0 = lds_u4(src), c1 = lds_u4(src + 16);
       const uint32_t wd[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
@@ -234,7 +241,7 @@ __global__ void __launch_bounds__(448, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&bar_afull[s]));
-      L += 2;
+      L += NG;
       tile = ntile;
       kb = nkb;
     }
@@ -339,29 +346,29 @@ __global__ void __launch_bounds__(256) s2_nf4_dequant_kernel(const uint32_t* cod
   }
 }
 
-template <int NS>
-cudaError_t launch_nf4_qkv_stages(const CUtensorMap& tx, const CUtensorMap& tc, const CUtensorMap* to,
-                                  const Nf4Args& a, int num_sms, cudaStream_t stream) {
-  using C = Nf4Cfg<NS>;
-  cudaError_t ea =
-      cudaFuncSetAttribute(s2_nf4_qkv_kernel<NS>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+template <int NS, int DQW>
+cudaError_t launch_nf4_qkv_variant(const CUtensorMap& tx, const CUtensorMap& tc, const CUtensorMap* to,
+                                   const Nf4Args& a, int num_sms, cudaStream_t stream) {
+  using C = Nf4Cfg<NS, DQW>;
+  cudaError_t ea = cudaFuncSetAttribute(s2_nf4_qkv_kernel<NS, DQW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        C::SMEM_BYTES);
   if (ea != cudaSuccess) return ea;
   const int ntiles = a.tiles_w * a.tiles_t;
   const int grid = ntiles < num_sms ? ntiles : num_sms;
   prof_before(stream, kKernelNf4Qkv);
-  s2_nf4_qkv_kernel<NS><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tx, tc, to[0], to[1], to[2], a);
+  s2_nf4_qkv_kernel<NS, DQW><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tx, tc, to[0], to[1], to[2], a);
   cudaError_t e = cudaGetLastError();
   prof_after(stream);
   return e;
 }
 
+// stages: pipeline depth 3 or 4; dq_warps: dequantization warps, 8 or 12
 cudaError_t launch_nf4_qkv(const CUtensorMap& tx, const CUtensorMap& tc, const CUtensorMap* to, const Nf4Args& a,
-                           int num_sms, cudaStream_t stream, int stages) {
-  switch (stages) {
-    case 3: return launch_nf4_qkv_stages<3>(tx, tc, to, a, num_sms, stream);
-    case 4: return launch_nf4_qkv_stages<4>(tx, tc, to, a, num_sms, stream);
-    default: return cudaErrorInvalidValue;
-  }
+                           int num_sms, cudaStream_t stream, int stages, int dq_warps) {
+  if (stages == 4 && dq_warps == 8) return launch_nf4_qkv_variant<4, 8>(tx, tc, to, a, num_sms, stream);
+  if (stages == 4 && dq_warps == 12) return launch_nf4_qkv_variant<4, 12>(tx, tc, to, a, num_sms, stream);
+  if (stages == 3 && dq_warps == 8) return launch_nf4_qkv_variant<3, 8>(tx, tc, to, a, num_sms, stream);
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_nf4_dequant(const void* codes, const int8_t* sq, const float* c2, void* w, long long n_words,

@@ -181,7 +181,7 @@ Dims make_segment_dims(int B, int H, int Hkv, int N, int Nk, int D, int causal) 
 // that the per-shape selection would not pick.  It starts from the
 // S2ATTN_TILE environment variable and can be replaced at run time by the
 // s2attn_set_tile_override test hook.  Keys: bwd=split|fused,
-// fwd_order=snake|pairs, fwd_kv=N, bwd_stages=N, nf4_stages=4|6.  Unknown
+// fwd_order=snake|pairs, fwd_kv=N, bwd_stages=N, nf4_stages=3|4, nf4_dq=8|12.  Unknown
 // keys and values are ignored.
 std::mutex g_override_mu;
 std::string g_override;
@@ -437,11 +437,20 @@ const char* s2attn_status_string(int status) {
     case S2ATTN_ERR_CUDA: return "S2ATTN_ERR_CUDA";
     case S2ATTN_ERR_DEVICE_TIMEOUT: return "S2ATTN_ERR_DEVICE_TIMEOUT";
     case S2ATTN_ERR_WORKSPACE: return "S2ATTN_ERR_WORKSPACE";
+    case S2ATTN_ERR_DEVICE_BOUNDS: return "S2ATTN_ERR_DEVICE_BOUNDS";
     default: return "S2ATTN_UNKNOWN_STATUS";
   }
 }
 
 int s2attn_last_launch_count(void) { return g_last_launches; }
+
+int s2attn_debug_checks(void) {
+#ifdef S2ATTN_DEBUG_CHECKS
+  return 1;
+#else
+  return 0;
+#endif
+}
 
 int s2attn_last_cuda_error(void) { return g_last_cuda_error; }
 
@@ -770,11 +779,15 @@ bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint6
   return r == CUDA_SUCCESS;
 }
 
-// Pipeline depth of the fused NF4 projection: 4 stages, or the override's
-// nf4_stages=3|4.
+// Variant of the fused NF4 projection: 4 stages and 8 dequantization warps,
+// or the override's nf4_stages=3|4 and nf4_dq=8|12 (12 warps with 4 stages).
 int nf4_stages() {
   const std::string v = override_value(tile_override(), "nf4_stages");
   return v == "3" ? 3 : 4;
+}
+int nf4_dq_warps() {
+  const std::string v = override_value(tile_override(), "nf4_dq");
+  return v == "12" && nf4_stages() == 4 ? 12 : 8;
 }
 
 int validate_nf4(int M, int K, int H, int Hkv, int D) {
@@ -867,7 +880,8 @@ int s2attn_nf4_qkv(const void* x, const void* codes, const int8_t* scale_codes, 
   }
   a.status = static_cast<uint32_t*>(status);
   a.wait_limit_ns = wait_limit_ns();
-  const cudaError_t e = launch_nf4_qkv(tx, tc, to, a, info.sms, static_cast<cudaStream_t>(stream), nf4_stages());
+  const cudaError_t e = launch_nf4_qkv(tx, tc, to, a, info.sms, static_cast<cudaStream_t>(stream), nf4_stages(),
+                                       nf4_dq_warps());
   if (e != cudaSuccess) {
     g_last_cuda_error = static_cast<int>(e);
     return S2ATTN_ERR_CUDA;

@@ -179,3 +179,17 @@ def test_nf4_levels_and_argument_checks_on_the_host():
     assert call(q=p + 2) == _lib.S2ATTN_ERR_MISALIGNED
     assert lib.s2attn_nf4_dequant(p, p, p, p, 4, 100, None) == _lib.S2ATTN_ERR_UNSUPPORTED
     assert lib.s2attn_nf4_dequant(p, p, p, p + 8, 4, 128, None) == _lib.S2ATTN_ERR_MISALIGNED
+
+
+def test_debug_build_exports_the_same_symbols():
+    """libs2attn_debug.so (kernels with index checks) builds and exports every
+    entry point of the header, and says it is the debug build."""
+    import ctypes
+
+    from sparse_attention_attn_b200 import build
+    path = build.build(debug=True)
+    lib = ctypes.CDLL(path)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    lib.s2attn_debug_checks.restype = ctypes.c_int
+    assert lib.s2attn_debug_checks() == 1
