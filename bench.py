@@ -481,6 +481,8 @@ def run_ours(args, shape, world, rank, local):
         line["rope"] = rope_step(shape, dev, peaks, ms_step)
     if not args.no_nf4 and rank == 0 and world == 1:
         line["nf4_qkv"] = nf4_projection(dev, peaks)
+    if not args.no_hga and rank == 0 and world == 1:
+        line["hga"] = hga_step(shape, dev, peaks)
     if not args.no_extra_workloads and world == 1:
         line["other_workloads"] = {s.name: other_workload(s, dev, peaks)
                                    for s in I.WORKLOADS if s.name in args.extra_workloads.split(",")}
@@ -574,6 +576,45 @@ def rope_step(shape: I.Shape, dev, peaks, ms_plain: float, steps: int = 10, warm
                                 "frac": rot_bytes / (avg * 1e-3) / 1e9 / peaks["hbm_gbs"],
                                 "bytes_per_launch": rot_bytes}
     return out
+
+
+def hga_step(shape: I.Shape, dev, peaks, S: int = 8, steps: int = 10, warmup: int = 3):
+    """HGA-style block-sparse attention on the workload's inputs: segments of
+    G rows attended causally (no shift) plus S listed historical 128-row tiles
+    per 256-row query block (random earlier tiles), forward + backward.
+    Effective FLOPs: the local part counts as S2's (forward 2 GEMMs, backward
+    2.5x), the historical part forward 2 GEMMs and backward 2 (dP and dQ; no
+    dK/dV for detached keys)."""
+    import sparse_attention_attn_b200 as s2
+    q, k, v, do = (t.to(dev) for t in I.make_inputs(shape))
+    hist = I.make_hga_selection(shape.B, shape.N, shape.G, S, seed=5).to(dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((shape.B, shape.H, shape.N), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+    def step():
+        s2.hga_forward(q, k, v, shape.G, hist, out=o, lse=lse)
+        s2.hga_backward(q, k, v, o, lse, do, shape.G, hist, dq=dq, dk=dk, dv=dv)
+
+    for _ in range(warmup):
+        step()
+    device_sync()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        step()
+    b.record()
+    device_sync()
+    ms = a.elapsed_time(b) / steps
+    if s2.device_status() != 0:
+        raise RuntimeError("device status reports a timeout in the HGA step")
+    n_hist = int((hist >= 0).sum().item())  # listed tiles over all blocks (each 256 rows x 128 keys)
+    fwd_local, _ = effective_flops(shape)
+    fwd_hist = 4.0 * shape.H * shape.D * n_hist * 256 * 128
+    total = 3.5 * fwd_local + 2.0 * fwd_hist
+    tf = total / (ms * 1e-3) / 1e12
+    return {"ms_per_step": ms, "value": tf, "unit": "TFLOP/s", "frac_of_bf16_peak": tf / peaks["bf16_tflops"],
+            "tiles_per_block": S, "history_tiles_listed": n_hist, "steps": steps, "warmup": warmup}
 
 
 def nf4_projection(dev, peaks, steps: int = 20, warmup: int = 3):
@@ -755,6 +796,7 @@ def main():
                     help="skip the few-step timing of the other workload shapes")
     ap.add_argument("--no-rope", action="store_true", help="skip the step with RoPE + Position Interpolation")
     ap.add_argument("--no-nf4", action="store_true", help="skip the NF4 QKV projection timing")
+    ap.add_argument("--no-hga", action="store_true", help="skip the HGA block-sparse step timing")
     ap.add_argument("--nf4-only", action="store_true",
                     help="time only the NF4 QKV projection (--steps / --warmup launches) and print its JSON")
     ap.add_argument("--sweep", action="store_true",

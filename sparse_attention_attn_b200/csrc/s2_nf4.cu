@@ -34,6 +34,8 @@
 //          alternate stages
 //   10-13  epilogue: TMEM -> bf16 staging in shared memory -> TMA store to q / k / v
 // TMEM: accumulator columns [0, 256), A stages [256 + 32 s, 256 + 32 s + 32).
+// Five stages by default: the x tiles come from L2 at about 12 TB/s over all
+// SMs, and with four the issuer measurably waited for them.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -62,7 +64,7 @@ struct Nf4Cfg {
   static constexpr int BW = 128, BT = 256, BK = 64;
   static constexpr int X_BYTES = BT * BK * 2;  // 32 KB per stage
   static constexpr int C_BYTES = BW * BK / 2;  // 4 KB per stage
-  static constexpr int O_WARP_BYTES = BT * 32 * 2;  // one epilogue warp's staging: 16 KB
+  static constexpr int O_WARP_BYTES = 128 * 32 * 2;  // one epilogue warp's staging: 8 KB (half a tile)
   static constexpr int SMEM_BYTES = NS * (X_BYTES + C_BYTES) + 4 * O_WARP_BYTES + 1024;
   static constexpr int TM_A = 256;
   static constexpr int DQ_WARPS = DQW;  // dequantization warps: groups of four
@@ -247,10 +249,12 @@ __global__ void __launch_bounds__(Nf4Cfg<NS, DQW>::THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    // Each warp owns 32 features of the tile: it moves their 256 token values
-    // from TMEM into a [256 tokens][32 features] bf16 staging area (64-byte
-    // rows), releases the accumulator, and stores the area with one TMA copy
-    // (rows past M are clipped by the copy).
+    // Each warp owns 32 features of the tile.  Per half of 128 tokens it
+    // loads their values from TMEM into registers (bf16 pairs of tokens 2i,
+    // 2i + 1), writes them to its [128 tokens][32 features] bf16 staging area
+    // (64-byte rows) and stores the area with one TMA copy (rows past M are
+    // clipped by the copy).  The accumulator is released as soon as the
+    // second half is in registers.
     const int sub = warp & 3;
     const uint32_t tD = tmem + (static_cast<uint32_t>(32 * sub) << 16);
     const uint32_t stage = sO + sub * C::O_WARP_BYTES;
@@ -270,13 +274,7 @@ __global__ void __launch_bounds__(Nf4Cfg<NS, DQW>::THREADS, 1)
         }
       }
       if (!warp_wait(smem_u32(&bar_acc_full), n & 1, wc, 65)) break;
-      // the previous tile's store has finished reading the staging area
-      if (lane == 0) bulk_wait_read_all();
-      __syncwarp();
       tc_fence_after();
-      // two halves of 128 tokens: each loaded into registers as bf16 pairs
-      // (tokens 2i, 2i + 1) and written to the staging area; the accumulator
-      // is released once the second half is in registers
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         uint32_t pk[64];
@@ -294,17 +292,21 @@ __global__ void __launch_bounds__(Nf4Cfg<NS, DQW>::THREADS, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(smem_u32(&bar_acc_empty));
         }
+        // the previous store from the staging area has finished reading it
+        if (lane == 0) bulk_wait_read_all();
+        __syncwarp();
 #pragma unroll
         for (int j = 0; j < 128; ++j)
-          st_shared_u16(stage + (128 * h + j) * 64 + lane * 2, static_cast<uint16_t>(pk[j >> 1] >> (16 * (j & 1))));
+          st_shared_u16(stage + j * 64 + lane * 2, static_cast<uint16_t>(pk[j >> 1] >> (16 * (j & 1))));
+        fence_proxy_async_smem();
+        __syncwarp();
+        const int t0 = tt * C::BT + 128 * h;
+        if (lane == 0 && t0 < a.M) {
+          tma_store_2d(map, stage, col, t0);
+          bulk_commit_group();
+        }
+        __syncwarp();
       }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        tma_store_2d(map, stage, col, tt * C::BT);
-        bulk_commit_group();
-      }
-      __syncwarp();
     }
     if (lane == 0) bulk_wait_all();
     __syncwarp();
@@ -362,12 +364,12 @@ cudaError_t launch_nf4_qkv_variant(const CUtensorMap& tx, const CUtensorMap& tc,
   return e;
 }
 
-// stages: pipeline depth 3 or 4; dq_warps: dequantization warps, 8 or 12
+// stages: pipeline depth 4 or 5; dq_warps: dequantization warps, 8 or 12
 cudaError_t launch_nf4_qkv(const CUtensorMap& tx, const CUtensorMap& tc, const CUtensorMap* to, const Nf4Args& a,
                            int num_sms, cudaStream_t stream, int stages, int dq_warps) {
+  if (stages == 5 && dq_warps == 8) return launch_nf4_qkv_variant<5, 8>(tx, tc, to, a, num_sms, stream);
+  if (stages == 5 && dq_warps == 12) return launch_nf4_qkv_variant<5, 12>(tx, tc, to, a, num_sms, stream);
   if (stages == 4 && dq_warps == 8) return launch_nf4_qkv_variant<4, 8>(tx, tc, to, a, num_sms, stream);
-  if (stages == 4 && dq_warps == 12) return launch_nf4_qkv_variant<4, 12>(tx, tc, to, a, num_sms, stream);
-  if (stages == 3 && dq_warps == 8) return launch_nf4_qkv_variant<3, 8>(tx, tc, to, a, num_sms, stream);
   return cudaErrorInvalidValue;
 }
 

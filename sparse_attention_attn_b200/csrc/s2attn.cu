@@ -181,7 +181,7 @@ Dims make_segment_dims(int B, int H, int Hkv, int N, int Nk, int D, int causal) 
 // that the per-shape selection would not pick.  It starts from the
 // S2ATTN_TILE environment variable and can be replaced at run time by the
 // s2attn_set_tile_override test hook.  Keys: bwd=split|fused,
-// fwd_order=snake|pairs, fwd_kv=N, bwd_stages=N, nf4_stages=3|4, nf4_dq=8|12.  Unknown
+// fwd_order=snake|pairs, fwd_kv=N, bwd_stages=N, nf4_stages=4|5, nf4_dq=8|12.  Unknown
 // keys and values are ignored.
 std::mutex g_override_mu;
 std::string g_override;
@@ -779,15 +779,15 @@ bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint6
   return r == CUDA_SUCCESS;
 }
 
-// Variant of the fused NF4 projection: 4 stages and 8 dequantization warps,
-// or the override's nf4_stages=3|4 and nf4_dq=8|12 (12 warps with 4 stages).
+// Variant of the fused NF4 projection: 5 stages and 8 dequantization warps,
+// or the override's nf4_stages=4|5 and nf4_dq=8|12 (12 warps with 5 stages).
 int nf4_stages() {
   const std::string v = override_value(tile_override(), "nf4_stages");
-  return v == "3" ? 3 : 4;
+  return v == "4" ? 4 : 5;
 }
 int nf4_dq_warps() {
   const std::string v = override_value(tile_override(), "nf4_dq");
-  return v == "12" && nf4_stages() == 4 ? 12 : 8;
+  return v == "12" && nf4_stages() == 5 ? 12 : 8;
 }
 
 int validate_nf4(int M, int K, int H, int Hkv, int D) {
@@ -859,7 +859,7 @@ int s2attn_nf4_qkv(const void* x, const void* codes, const int8_t* scale_codes, 
   const int widths[3] = {H * D, Hkv * D, Hkv * D};
   for (int i = 0; i < 3; ++i)
     if (!make_map_2d(&to[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, outs[i], static_cast<uint64_t>(widths[i]),
-                     static_cast<uint64_t>(M), static_cast<uint64_t>(widths[i]) * 2, 32, 256,
+                     static_cast<uint64_t>(M), static_cast<uint64_t>(widths[i]) * 2, 32, 128,
                      CU_TENSOR_MAP_SWIZZLE_NONE))
       return S2ATTN_ERR_CUDA;
   Nf4Args a;

@@ -71,3 +71,20 @@ def make_nf4_weights(rows: int, K: int, seed: int):
     sq = torch.randint(64, 128, (nblk,), generator=g, dtype=torch.int32).to(torch.int8)
     c2 = 0.05 + 0.03 * torch.rand(((nblk + 255) // 256,), generator=g, dtype=torch.float32)
     return codes, sq, c2
+
+
+def make_hga_selection(B: int, N: int, G: int, S: int, seed: int):
+    """int32 [B, N/256, S] historical tile lists for HGA-style attention:
+    for every 256-row query block, min(S, earlier tiles) distinct 128-row key
+    tiles drawn uniformly from the segments before its own (ascending), the
+    unused slots -1.  Random stand-ins for a model's chunk-summary choice."""
+    import numpy as np
+    rng = np.random.default_rng(seed)
+    sel = -np.ones((B, N // 256, S), dtype=np.int32)
+    for b in range(B):
+        for qb in range(N // 256):
+            prev = (qb * 256 // G) * G // 128
+            n = min(S, prev)
+            if n:
+                sel[b, qb, :n] = np.sort(rng.choice(prev, size=n, replace=False))
+    return torch.from_numpy(sel)
