@@ -711,8 +711,9 @@ def sweep_variants(D: int):
     strings: forward (work order x K/V ring depth) and backward (path x stages)."""
     slots = (4,) if D == 128 else (4, 6, 8)
     fwd = [f"fwd_order={o},fwd_kv={s}" for o in ("snake", "pairs") for s in slots]
-    bwd = (["bwd=fused"] if D == 128 else []) + \
-        [f"bwd=split,bwd_stages={s}" for s in ((2, 3) if D == 128 else (3, 4))]
+    stages = (2, 3) if D == 128 else (3, 4)
+    bwd = (["bwd=fused"] if D == 128 else []) + [f"bwd={p},bwd_stages={s}" for p in ("split_ds", "split")
+                                                 for s in stages]
     return fwd, bwd
 
 

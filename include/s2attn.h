@@ -384,8 +384,9 @@ S2ATTN_API int s2attn_profile_stop(float* ms, int* kernel_ids, int capacity);
  * The per-shape plan the library would use for a call with these arguments on
  * a device with num_sms SMs (with the override below applied): out[0] forward
  * work order (1 longest-first snake, 0 equal-work pairs), out[1] forward K/V
- * ring depth, out[2] backward path (1 fused, 0 split), out[3] split backward
- * pipeline stages.  Host only; returns a status code (shape validation as in
+ * ring depth, out[2] backward path (2 split-dS: dQ from the dS blocks the
+ * dK/dV kernel stores in the workspace; 0 split: dQ recomputes S and dP; 1
+ * fused), out[3] split backward pipeline stages.  Host only; returns a status code (shape validation as in
  * s2attn_fwd).
  */
 S2ATTN_API int s2attn_plan(int B, int H, int Hkv, int N, int D, int G, int num_sms, int* out);
@@ -395,7 +396,7 @@ S2ATTN_API int s2attn_plan(int B, int H, int Hkv, int N, int D, int G, int num_s
  * variable) that later calls in this process consult; NULL restores the
  * environment's value.  The override forces a variant the per-shape selection
  * would not pick, for tests and sweeps: a comma-separated list of key=value
- * items; keys bwd=split|fused (backward path; fused exists for head dim 128),
+ * items; keys bwd=split_ds|split|fused (backward path; fused exists for head dim 128),
  * fwd_order=snake|pairs (forward work order), fwd_kv=N (forward K/V ring
  * depth: 4 at head dim 128, 4/6/8 at 64), bwd_stages=N (split backward
  * stages: 2-3 at head dim 128, 3-4 at 64), nf4_stages=4|5 and nf4_dq=8|12

@@ -197,7 +197,7 @@ def s2attn_plan(B, H, Hkv, N, D, G, num_sms):
     out = (ctypes.c_int * 4)()
     _check("s2attn_plan", load().s2attn_plan(B, H, Hkv, N, D, G, num_sms, ctypes.addressof(out)))
     return {"fwd_order": "snake" if out[0] else "pairs", "fwd_kv_slots": out[1],
-            "bwd_path": "fused" if out[2] else "split", "bwd_stages": out[3]}
+            "bwd_path": {0: "split", 1: "fused", 2: "split_ds"}[out[2]], "bwd_stages": out[3]}
 
 
 def s2attn_nf4_levels():

@@ -415,6 +415,20 @@ __global__ void __launch_bounds__(352, 1)
         dk[2 * c4 + 1] = f2_to_bf16x2(f2_mul(f2_pack(p[4 * c4 + 2], p[4 * c4 + 3]), d23));
       }
       tmem_st16(tmem + lane_off + C::TM_DP + bo, dk);
+      if (a.ds != nullptr) {
+        // split-dS path: these 32 dS^T values (kv row `row`, query columns
+        // half * 32 + [0, 32) of sub-tile i64) also go to their dS block
+        const int i64 = 2 * cur.w.tile + cur.it % cur.nq;
+        const int hq = cur.w.kvh * d.rep + cur.it / cur.nq;
+        const long long blk = ds_block(d, cur.w.b, hq, cur.w.g, i64 >> 1, cur.w.tile, a.ds_tt);
+        if (in_bounds(wc.status, blk, a.ds_blocks, 48)) {
+          __nv_bfloat16* dst = a.ds + blk * (kTile * kTile) + row * kTile + (i64 & 1) * kSub + half * 32;
+          const uint32_t lo[8] = {dk[0], dk[1], dk[2], dk[3], dk[4], dk[5], dk[6], dk[7]};
+          const uint32_t hi[8] = {dk[8], dk[9], dk[10], dk[11], dk[12], dk[13], dk[14], dk[15]};
+          st_global_v8(dst, lo);
+          st_global_v8(dst + 16, hi);
+        }
+      }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -938,12 +952,13 @@ cudaError_t launch_bwd_stages(const BwdMaps& m, const BwdPreArgs& pre, const Bwd
     prof_after(stream);
     if (e != cudaSuccess) return e;
   }
+  if (launches) *launches = a.no_dkdv ? 2 : 3;
+  if (a.ds != nullptr) return launch_dq_ds<D>(m.ds, m.k128, m.dq32, a, num_sms, stream);  // dQ from the stored dS
   const int grid_q = a.q_sched.pairs < num_sms ? a.q_sched.pairs : num_sms;
   prof_before(stream, kKernelBwdDq);
   s2_bwd_dq_kernel<D, NST><<<grid_q, K4::THREADS, K4::SMEM_BYTES, stream>>>(m.q128, m.k64, m.v64, m.g128, a);
   e = cudaGetLastError();
   prof_after(stream);
-  if (launches) *launches = a.no_dkdv ? 2 : 3;
   return e;
 }
 

@@ -335,18 +335,31 @@ struct BwdArgs {
   int kv_v8;               // dk and dv are 32-byte aligned: whole-sector stores
   const float* rope;       // fused path: fp32 (cos, sin) [N][D/2][2] table to rotate dq and dk back
                            // (the inputs were rotated by it), or null
+  __nv_bfloat16* ds;       // split-dS path: the dK/dV kernel stores dS blocks here (see ds_block), or null
+  int ds_tt;               // dS blocks per (batch, head, group): T (T + 1) / 2
+  long long ds_blocks;     // dS blocks in all
   uint32_t* status;
   unsigned long long wait_limit_ns;
 };
+
+// Split-dS path: index of the 128 x 128 dS block of (query tile i, kv tile
+// j <= i) of group g of (batch b, query head h); blocks hold dS^T, kv-row-major.
+__host__ __device__ __forceinline__ long long ds_block(const Dims& d, int b, int h, int g, int i, int j, int tt) {
+  return ((static_cast<long long>(b) * d.H + h) * d.n_groups + g) * tt + i * (i + 1) / 2 + j;
+}
 
 // TMA descriptors of the backward: 128-row and 64-row boxes of each operand.
 struct BwdMaps {
   CUtensorMap q128, k128, v128, g128;
   CUtensorMap q64, k64, v64, g64;
+  CUtensorMap ds, dq32;  // split-dS path: the dS blocks (2-D, 64 x 128 boxes), dq (32-row boxes)
 };
 
 template <int D>
 cudaError_t launch_bwd_pre(const BwdPreArgs& pre, int num_sms, cudaStream_t stream);
+template <int D>
+cudaError_t launch_dq_ds(const CUtensorMap& tds, const CUtensorMap& tk, const CUtensorMap& tq32, const BwdArgs& a,
+                         int num_sms, cudaStream_t stream);
 
 // Index checks of the debug build (compiled with -DS2ATTN_DEBUG_CHECKS; they
 // compile to nothing otherwise).  A computed global index outside [0, n)
@@ -402,7 +415,8 @@ enum KernelId : int {
   kKernelBwdDqPost = 5,
   kKernelRope = 6,
   kKernelNf4Qkv = 7,
-  kKernelNf4Dequant = 8
+  kKernelNf4Dequant = 8,
+  kKernelBwdDqDs = 9
 };
 void prof_before(cudaStream_t stream, int kernel_id);
 void prof_after(cudaStream_t stream);

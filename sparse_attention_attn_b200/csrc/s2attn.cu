@@ -52,7 +52,19 @@ constexpr size_t kStatusBytes = 256;
 // and dP).  Fused (head dim 128): preprocess, one kernel for dK, dV and the
 // dQ partials (reduced into an fp32 accumulator in the workspace), dq
 // conversion.
-enum BwdPath : int { kBwdSplit = 0, kBwdFused = 1 };
+enum BwdPath : int { kBwdSplit = 0, kBwdFused = 1, kBwdSplitDs = 2 };
+
+// The split-dS path stores every dS block (32 KB per (query tile, kv tile <=
+// it) of each (batch, head, group)) in the workspace; it is planned while that
+// stays within this budget.
+constexpr double kDsBudgetBytes = 4.0 * 1024 * 1024 * 1024;
+
+// dS blocks of the split-dS path: B H (N/G) T (T+1) / 2, T = G/128.
+long long ds_blocks_for(int B, int H, int N, int G) {
+  const long long T = G / kTile;
+  return static_cast<long long>(B) * H * (N / G) * (T * (T + 1) / 2);
+}
+
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -180,7 +192,7 @@ Dims make_segment_dims(int B, int H, int Hkv, int N, int Nk, int D, int causal) 
 // A plan override string ("key=value,..."), used to time or test a variant
 // that the per-shape selection would not pick.  It starts from the
 // S2ATTN_TILE environment variable and can be replaced at run time by the
-// s2attn_set_tile_override test hook.  Keys: bwd=split|fused,
+// s2attn_set_tile_override test hook.  Keys: bwd=split_ds|split|fused,
 // fwd_order=snake|pairs, fwd_kv=N, bwd_stages=N, nf4_stages=4|5, nf4_dq=8|12.  Unknown
 // keys and values are ignored.
 std::mutex g_override_mu;
@@ -218,7 +230,7 @@ std::string override_value(const std::string& spec, const char* key) {
 struct Plan {
   int fwd_snake;     // forward work order: 1 snake (longest first), 0 equal-work pairs
   int fwd_kv_slots;  // forward K/V ring depth: 4 (head dim 128), 4/6/8 (head dim 64)
-  int bwd_path;      // kBwdFused (head dim 128 only) or kBwdSplit
+  int bwd_path;      // kBwdSplitDs, kBwdSplit, or kBwdFused (head dim 128 only)
   int bwd_stages;    // split backward operand stages: 2-3 (head dim 128), 3-4 (head dim 64)
 };
 
@@ -237,10 +249,12 @@ Plan select_plan(int B, int H, int Hkv, int N, int D, int G, int sms) {
   const double kv_bytes = 2.0 * B * N * Hkv * D * 2.0;
   p.fwd_snake = kv_bytes <= 256.0 * 1024 * 1024 ? 1 : 0;
   p.fwd_kv_slots = D == 128 ? 4 : 8;
-  // the split path measured faster than the fused one on every workload shape
-  // (the fused kernel is limited by its dQ reductions at L2); fused stays
-  // selectable
-  p.bwd_path = kBwdSplit;
+  // dQ from the dS the dK/dV kernel stores (five GEMM-units instead of
+  // seven) while the dS blocks fit the budget, else the split path that
+  // recomputes S and dP for dQ; the fused path measured slower than both and
+  // stays selectable
+  p.bwd_path = static_cast<double>(ds_blocks_for(B, H, N, G)) * kTile * kTile * 2 <= kDsBudgetBytes ? kBwdSplitDs
+                                                                                                      : kBwdSplit;
   p.bwd_stages = 3;
   // the override, where it names a variant that exists for this head dim
   const std::string spec = tile_override();
@@ -251,6 +265,7 @@ Plan select_plan(int B, int H, int Hkv, int N, int D, int G, int sms) {
   if (!kv.empty() && valid_kv_slots(D, std::atoi(kv.c_str()))) p.fwd_kv_slots = std::atoi(kv.c_str());
   const std::string path = override_value(spec, "bwd");
   if (path == "split") p.bwd_path = kBwdSplit;
+  if (path == "split_ds") p.bwd_path = kBwdSplitDs;
   if (path == "fused" && D == 128) p.bwd_path = kBwdFused;
   const std::string st = override_value(spec, "bwd_stages");
   if (!st.empty() && valid_bwd_stages(D, std::atoi(st.c_str()))) p.bwd_stages = std::atoi(st.c_str());
@@ -289,17 +304,36 @@ bool make_map(CUtensorMap* m, const void* base, int B, int N, int heads, int D, 
   return r == CUDA_SUCCESS;
 }
 
+// 2-D tiled view {inner, outer} of a row-major array with `row_bytes` between rows.
+bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
+                 uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) {
+    g_last_cuda_error = -1;
+    return false;
+  }
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  const CUresult r = enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) g_last_cuda_error = -static_cast<int>(r);
+  return r == CUDA_SUCCESS;
+}
+
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 size_t rowstat_bytes(int B, int H, int N) {
   return round_up(static_cast<size_t>(B) * H * N * sizeof(float), 256);
 }
 
-// Workspace: status block, -Delta, -lse*log2(e), and for the fused path the
-// fp32 [B, H, N, D] dQ accumulator.
-size_t workspace_bytes_for(int path, int B, int H, int N, int D) {
+// Workspace: status block, -Delta, -lse*log2(e); for the fused path the fp32
+// [B, H, N, D] dQ accumulator; for the split-dS path the dS blocks.
+size_t workspace_bytes_for(int path, int B, int H, int N, int D, int G) {
   size_t n = kStatusBytes + 2 * rowstat_bytes(B, H, N);
   if (path == kBwdFused) n += round_up(static_cast<size_t>(B) * H * N * D * sizeof(float), 256);
+  if (path == kBwdSplitDs) n += static_cast<size_t>(ds_blocks_for(B, H, N, G)) * kTile * kTile * 2;
   return n;
 }
 
@@ -461,7 +495,7 @@ const char* s2attn_cuda_error_string(int err) {
 
 size_t s2attn_bwd_workspace_bytes(int B, int H, int Hkv, int N, int D, int G) {
   if (validate_shape(B, H, Hkv, N, D, G) != S2ATTN_OK) return 0;
-  return workspace_bytes_for(select_plan(B, H, Hkv, N, D, G, 0).bwd_path, B, H, N, D);
+  return workspace_bytes_for(select_plan(B, H, Hkv, N, D, G, 0).bwd_path, B, H, N, D, G);
 }
 
 int s2attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
@@ -504,7 +538,9 @@ int bwd_impl(int path, int stages, const void* q, const void* k, const void* v, 
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
       !aligned16(dO) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
     return S2ATTN_ERR_MISALIGNED;
-  const size_t need = workspace_bytes_for(path, B, H, N, D);
+  // segment and HGA modes take the split path (the dQ kernel walks their extra keys)
+  if (seg != nullptr && path == kBwdSplitDs) path = kBwdSplit;
+  const size_t need = workspace_bytes_for(path, B, H, N, D, G);
   if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return S2ATTN_ERR_WORKSPACE;
   DeviceInfo info;
@@ -524,6 +560,15 @@ int bwd_impl(int path, int stages, const void* q, const void* k, const void* v, 
   float* nlse2 = reinterpret_cast<float*>(ws + kStatusBytes + rowstat_bytes(B, H, N));
   float* dqacc = path == kBwdFused ? reinterpret_cast<float*>(ws + kStatusBytes + 2 * rowstat_bytes(B, H, N))
                                    : nullptr;
+  __nv_bfloat16* ds = path == kBwdSplitDs
+                          ? reinterpret_cast<__nv_bfloat16*>(ws + kStatusBytes + 2 * rowstat_bytes(B, H, N))
+                          : nullptr;
+  const long long ds_blocks = path == kBwdSplitDs ? ds_blocks_for(B, H, N, G) : 0;
+  if (ds != nullptr &&
+      (!make_map_2d(&maps.ds, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ds, kTile, static_cast<uint64_t>(ds_blocks) * kTile,
+                    kTile * 2, 64, kTile, CU_TENSOR_MAP_SWIZZLE_128B) ||
+       !make_map(&maps.dq32, dq, B, N, H, D, 32)))
+    return S2ATTN_ERR_CUDA;
   BwdPreArgs pre;
   pre.d = d;
   pre.o = o;
@@ -550,6 +595,9 @@ int bwd_impl(int path, int stages, const void* q, const void* k, const void* v, 
   a.dv = dv;
   a.kv_v8 = ((reinterpret_cast<uintptr_t>(dk) | reinterpret_cast<uintptr_t>(dv)) & 31u) == 0 ? 1 : 0;
   a.rope = path == kBwdFused ? rope : nullptr;
+  a.ds = ds;
+  a.ds_tt = (G / kTile) * (G / kTile + 1) / 2;
+  a.ds_blocks = ds_blocks;
   a.status = status;
   a.wait_limit_ns = wait_limit_ns();
   int launches = 0;
@@ -655,7 +703,7 @@ int s2attn_bwd_rope(const void* q_rot, const void* k_rot, const void* v, const v
 
 size_t s2attn_seg_bwd_workspace_bytes(int B, int H, int Hkv, int N, int Nk, int D) {
   if (validate_segment(B, H, Hkv, N, Nk, D, 0) != S2ATTN_OK) return 0;
-  return workspace_bytes_for(kBwdSplit, B, H, N, D);
+  return workspace_bytes_for(kBwdSplit, B, H, N, D, N);
 }
 
 int s2attn_seg_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
@@ -759,24 +807,6 @@ const Nf4Levels& nf4_levels() {
     return t;
   }();
   return lv;
-}
-
-// 2-D tiled view {inner, outer} of a row-major array with `row_bytes` between rows.
-bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
-                 uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
-  EncodeTiledFn enc = get_encode();
-  if (!enc) {
-    g_last_cuda_error = -1;
-    return false;
-  }
-  cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {row_bytes};
-  cuuint32_t box[2] = {box_inner, box_outer};
-  cuuint32_t es[2] = {1, 1};
-  const CUresult r = enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                         sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) g_last_cuda_error = -static_cast<int>(r);
-  return r == CUDA_SUCCESS;
 }
 
 // Variant of the fused NF4 projection: 5 stages and 8 dequantization warps,
@@ -892,7 +922,7 @@ int s2attn_nf4_qkv(const void* x, const void* codes, const int8_t* scale_codes, 
 
 size_t s2attn_hga_bwd_workspace_bytes(int B, int H, int Hkv, int N, int D, int G) {
   if (validate_shape(B, H, Hkv, N, D, G, false) != S2ATTN_OK || G % kQBlock != 0) return 0;
-  return workspace_bytes_for(kBwdSplit, B, H, N, D);
+  return workspace_bytes_for(kBwdSplit, B, H, N, D, G);
 }
 
 int s2attn_plan(int B, int H, int Hkv, int N, int D, int G, int num_sms, int* out) {
@@ -1025,7 +1055,7 @@ extern "C" int s2attn_bwd_noalloc(const void* q, const void* k, const void* v, c
   // with B * H * N only, where the fused path would need a dQ accumulator of
   // B * H * N * D floats
   const bool valid = validate_shape(B, H, Hkv, N, D, G) == S2ATTN_OK;
-  const size_t need = valid ? workspace_bytes_for(kBwdSplit, B, H, N, D) : 0;
+  const size_t need = valid ? workspace_bytes_for(kBwdSplit, B, H, N, D, G) : 0;
   if (need > kNoAllocScratchBytes) return S2ATTN_ERR_WORKSPACE;
   void* scratch = nullptr;
   // an invalid shape: bwd_impl reports which error

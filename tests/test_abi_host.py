@@ -90,10 +90,15 @@ def test_backward_argument_validation():
 
 def test_workspace_bytes():
     # status block + two fp32 [B, H, N] row-statistics arrays, each rounded to 256 bytes;
-    # on the fused backward also the fp32 [B, H, N, D] dq accumulator
-    assert _lib.s2attn_bwd_workspace_bytes(1, 32, 32, 8192, 128, 2048) == 256 + 2 * 32 * 8192 * 4
-    assert _lib.s2attn_bwd_workspace_bytes(1, 1, 1, 128, 64, 128) == 256 + 2 * 512
+    # on the split-dS path (the default while its blocks fit 4 GiB) also the dS
+    # blocks: B H (N/G) T (T+1)/2 blocks of 128 x 128 bf16, T = G/128; on the
+    # fused backward the fp32 [B, H, N, D] dq accumulator instead
+    ds = 32 * 4 * (16 * 17 // 2) * 128 * 128 * 2
+    assert _lib.s2attn_bwd_workspace_bytes(1, 32, 32, 8192, 128, 2048) == 256 + 2 * 32 * 8192 * 4 + ds
+    assert _lib.s2attn_bwd_workspace_bytes(1, 1, 1, 128, 64, 128) == 256 + 2 * 512 + 128 * 128 * 2
     assert _lib.s2attn_bwd_workspace_bytes(1, 4, 3, 1024, 64, 256) == 0  # invalid shape
+    # LLaMA2-70B at 32K tokens: 17 GB of dS blocks, over the budget: the split path
+    assert _lib.s2attn_bwd_workspace_bytes(1, 64, 8, 32768, 128, 8192) == 256 + 2 * 64 * 32768 * 4
     # the split path, forced through the override, needs no accumulator
     try:
         _lib.s2attn_set_tile_override("bwd=split")
@@ -118,14 +123,14 @@ def test_profile_api_host_side():
 
 
 def test_plan_selection_table():
-    """The per-shape plan (host logic, no GPU): the split backward (measured
-    faster), the forward's work order following the K/V size, the selected
-    depths."""
+    """The per-shape plan (host logic, no GPU): the split-dS backward while its
+    dS blocks fit 4 GiB, else the split backward; the forward's work order
+    following the K/V size; the selected depths."""
     from sparse_attention_attn_b200 import inputs as I
     expect = {
-        "tiny": ("snake", 8, "split", 3),
-        "llama2-7b-n8192": ("snake", 4, "split", 3),
-        "qwen3-8b-gqa-n16384": ("snake", 4, "split", 3),
+        "tiny": ("snake", 8, "split_ds", 3),
+        "llama2-7b-n8192": ("snake", 4, "split_ds", 3),
+        "qwen3-8b-gqa-n16384": ("snake", 4, "split_ds", 3),
         "llama2-70b-gqa-n32768": ("snake", 4, "split", 3),
         "llama2-7b-n102400": ("pairs", 4, "split", 3),
     }
@@ -145,14 +150,17 @@ def test_plan_override_parsing():
         assert p == {"fwd_order": "pairs", "fwd_kv_slots": 4, "bwd_path": "split", "bwd_stages": 2}
         p = _lib.s2attn_plan(1, 4, 4, 1024, 64, 256, 148)   # head dim 64: kv 2 and stages 2 do not exist
         assert p == {"fwd_order": "pairs", "fwd_kv_slots": 8, "bwd_path": "split", "bwd_stages": 3}
-        _lib.s2attn_set_tile_override("bwd=fused,fwd_kv=6,bwd_stages=4,junk,=,x=y")
+        _lib.s2attn_set_tile_override("bwd=fused,fwd_kv=6,bwd_stages=4,junk,=,x=y")  # no fused path at D = 64
         assert _lib.s2attn_plan(1, 4, 4, 1024, 64, 256, 148) == \
-            {"fwd_order": "snake", "fwd_kv_slots": 6, "bwd_path": "split", "bwd_stages": 4}
+            {"fwd_order": "snake", "fwd_kv_slots": 6, "bwd_path": "split_ds", "bwd_stages": 4}
         assert _lib.s2attn_plan(1, 32, 32, 8192, 128, 2048, 148) == \
             {"fwd_order": "snake", "fwd_kv_slots": 4, "bwd_path": "fused", "bwd_stages": 3}
+        _lib.s2attn_set_tile_override("bwd=split_ds")  # forced even over the budget
+        assert _lib.s2attn_plan(1, 64, 8, 32768, 128, 8192, 148)["bwd_path"] == "split_ds"
     finally:
         _lib.s2attn_set_tile_override(None)
-    assert _lib.s2attn_plan(1, 32, 32, 8192, 128, 2048, 148)["bwd_path"] == "split"
+    assert _lib.s2attn_plan(1, 32, 32, 8192, 128, 2048, 148)["bwd_path"] == "split_ds"
+    assert _lib.s2attn_plan(1, 64, 8, 32768, 128, 8192, 148)["bwd_path"] == "split"
 
 
 def test_nf4_levels_and_argument_checks_on_the_host():

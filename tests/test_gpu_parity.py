@@ -62,7 +62,8 @@ def bwd_path(request):
     _lib.s2attn_set_tile_override(None)
 
 
-SMALL_PATHS = [(*s, p) for s in SMALL for p in (("fused", "split") if s[4] == 128 else ("split",))]
+SMALL_PATHS = [(*s, p) for s in SMALL
+               for p in (("split_ds", "fused", "split") if s[4] == 128 else ("split_ds", "split"))]
 
 
 @pytest.mark.parametrize("B,N,H,Hkv,D,G,bwd_path", SMALL_PATHS, indirect=["bwd_path"])
@@ -82,7 +83,8 @@ def test_small_whole_tensor(B, N, H, Hkv, D, G, bwd_path):
 PLAN_VARIANTS = [
     # every variant the per-shape plan can select, forced through the override
     (128, "fwd_order=pairs"), (128, "bwd=split,bwd_stages=2"), (128, "bwd=split,bwd_stages=3"),
-    (128, "bwd=fused"), (64, "fwd_order=pairs"), (64, "fwd_kv=4"), (64, "fwd_kv=6"), (64, "bwd_stages=4"),
+    (128, "bwd=split_ds,bwd_stages=2"), (128, "bwd=fused"), (64, "fwd_order=pairs"), (64, "fwd_kv=4"),
+    (64, "fwd_kv=6"), (64, "bwd=split,bwd_stages=4"), (64, "bwd=split_ds,bwd_stages=4"),
 ]
 
 
@@ -207,9 +209,10 @@ def test_workload_sampled(shape):
     _check_full_size(shape, m=2048)
 
 
-@pytest.mark.parametrize("bwd_path", ["fused"], indirect=True)
+@pytest.mark.parametrize("bwd_path", ["fused", "split"], indirect=True)
 def test_workload_fused_backward_sampled(bwd_path):
-    """The fused backward (selectable through the plan) at full size."""
+    """The fused and the split (S and dP recomputed for dQ) backward paths,
+    selectable through the plan, at full size."""
     _check_full_size(I.LLAMA2_7B_8K, m=2048)
 
 

@@ -83,9 +83,9 @@ def _run(shape, s, seed_offset=0):
 
 ROPE_SMALL = [
     # (B, N, H, Hkv, D, G, path)
-    (2, 512, 4, 2, 128, 256, "fused"), (2, 512, 4, 2, 128, 256, "split"),
+    (2, 512, 4, 2, 128, 256, "fused"), (2, 512, 4, 2, 128, 256, "split"), (2, 512, 4, 2, 128, 256, "split_ds"),
     (1, 2048, 2, 2, 128, 2048, "fused"), (1, 1536, 6, 2, 128, 768, "fused"),
-    (1, 1024, 4, 4, 64, 256, "split"), (1, 768, 6, 2, 64, 256, "split"),
+    (1, 1024, 4, 4, 64, 256, "split"), (1, 768, 6, 2, 64, 256, "split_ds"),
 ]
 
 
