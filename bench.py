@@ -38,7 +38,8 @@ from sparse_attention_attn_b200 import inputs as I  # noqa: E402
 
 METRIC = "S2-Attn fwd+bwd TFLOP/s & tokens/s on 1 B200; % of BF16 tensor peak"
 KERNEL_NAMES = {0: "s2_fwd_kernel", 1: "s2_bwd_pre_kernel", 2: "s2_bwd_dkdv_kernel", 3: "s2_bwd_dq_kernel",
-                4: "s2_bwd_fused_kernel", 5: "s2_bwd_dq_post_kernel", 6: "s2_rope_apply_kernel"}
+                4: "s2_bwd_fused_kernel", 5: "s2_bwd_dq_post_kernel", 6: "s2_rope_apply_kernel",
+                7: "s2_nf4_qkv_kernel", 8: "s2_nf4_dequant_kernel", 9: "s2_bwd_dq_ds_kernel"}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -54,13 +55,19 @@ def kernel_algorithmic(s: I.Shape, fused: bool = False):
     (S, dP, dV, dK) and dQ 3 (S, dP, dQ); fused backward 5 (S, dP, dV, dK, dQ).
     The preprocess moves bytes: O and dO read, Delta and lse*log2(e) written,
     lse read, and on the fused path the fp32 dq accumulator zeroed; the dq
-    conversion reads the accumulator and writes bf16 dq."""
+    conversion reads the accumulator and writes bf16 dq.  On the split-dS path
+    the dQ GEMM (one GEMM-unit, 0.04 ms of tensor work at the LLaMA2-7B shape)
+    is bound by its bytes: the dS blocks read (B H (N/G) T (T+1)/2 blocks of
+    128 x 128 bf16, T = G/128), K read once and bf16 dq written."""
     gemm = 2.0 * s.B * s.H * s.N * s.G * s.D * 0.5
     rows = s.B * s.H * s.N
     acc = rows * s.D * 4.0
+    T = s.G // 128
+    ds_bytes = s.B * s.H * (s.N // s.G) * (T * (T + 1) // 2) * 128 * 128 * 2.0
     return {0: ("tensor", 2 * gemm), 2: ("tensor", 4 * gemm), 3: ("tensor", 3 * gemm), 4: ("tensor", 5 * gemm),
             1: ("hbm", 2.0 * rows * s.D * 2 + rows * 4 * 3 + (acc if fused else 0.0)),
-            5: ("hbm", acc + rows * s.D * 2.0)}
+            5: ("hbm", acc + rows * s.D * 2.0),
+            9: ("hbm", ds_bytes + s.B * s.N * s.Hkv * s.D * 2.0 + rows * s.D * 2.0)}
 
 
 def load_peaks():
