@@ -417,12 +417,14 @@ __global__ void __launch_bounds__(352, 1)
       tmem_st16(tmem + lane_off + C::TM_DP + bo, dk);
       if (a.ds != nullptr) {
         // split-dS path: these 32 dS^T values (kv row `row`, query columns
-        // half * 32 + [0, 32) of sub-tile i64) also go to their dS block
+        // half * 32 + [0, 32) of sub-tile i64) also go to their dS block, in
+        // its 32-column slab 2 (i64 & 1) + half: the warp's 32 rows write
+        // 2 KB of consecutive bytes
         const int i64 = 2 * cur.w.tile + cur.it % cur.nq;
         const int hq = cur.w.kvh * d.rep + cur.it / cur.nq;
         const long long blk = ds_block(d, cur.w.b, hq, cur.w.g, i64 >> 1, cur.w.tile, a.ds_tt);
         if (in_bounds(wc.status, blk, a.ds_blocks, 48)) {
-          __nv_bfloat16* dst = a.ds + blk * (kTile * kTile) + row * kTile + (i64 & 1) * kSub + half * 32;
+          __nv_bfloat16* dst = a.ds + blk * (kTile * kTile) + (2 * (i64 & 1) + half) * (kTile * 32) + row * 32;
           const uint32_t lo[8] = {dk[0], dk[1], dk[2], dk[3], dk[4], dk[5], dk[6], dk[7]};
           const uint32_t hi[8] = {dk[8], dk[9], dk[10], dk[11], dk[12], dk[13], dk[14], dk[15]};
           st_global_v8(dst, lo);

@@ -3,8 +3,9 @@
 // Delta) for every (kv tile, query sub-tile) pair of a group anyway; on this
 // path its elementwise warps also store those bf16 values in the workspace, one
 // 128 x 128 block per (query tile i, kv tile j <= i) of each (batch, head,
-// group), stored kv-row-major ([kv][query], 256-byte rows).  dQ is then a
-// plain GEMM per query tile:
+// group), as four slabs of 32 query columns ([kv][32 queries], 64-byte rows,
+// so the dK/dV warps' stores are contiguous).  dQ is then a plain GEMM per
+// query tile:
 //   dQ_i = scale * sum_{j <= i} dS_ij K_j,
 // so the backward issues the five GEMM-units of work the method counts (S^T,
 // dP^T, dV, dK in the dK/dV kernel, this one) instead of recomputing S and dP.
@@ -13,8 +14,9 @@
 //
 // Persistent: one CTA per SM walks 128-row query tiles in the pair schedule
 // of the other backward kernels (tile t with tile T-1-t: equal work).  Warp 0
-// loads, per kv tile j, the dS block (two 64-column slabs, 128-byte swizzle)
-// and K_j (128 rows, D/64 slabs) into a stage; warp 1 issues the SS UMMAs
+// loads, per kv tile j, the dS block (its four slabs with the 64-byte
+// swizzle) and K_j (128 rows, D/64 slabs, 128-byte swizzle) into a stage;
+// warp 1 issues the SS UMMAs
 // (M = 128 query rows, N = D, K = 16 kv rows; A = dS block MN-major, B = K_j
 // MN-major) into one of two TMEM accumulators; warps 2-5 (one per TMEM lane
 // quarter) scale the finished dQ, stage it as bf16 with the 128-byte swizzle
@@ -32,8 +34,9 @@ namespace s2 {
 template <int D, int NST>
 struct DqDsCfg {
   static constexpr int STAGES = NST;
-  static constexpr int SLAB = kTile * 128;            // 128 rows x 64 bf16 columns
-  static constexpr int DS_BYTES = 2 * SLAB;           // one dS block (128 x 128)
+  static constexpr int SLAB = kTile * 128;            // K: 128 rows x 64 bf16 columns
+  static constexpr int DS_SLAB = kTile * 64;          // dS: 128 rows x 32 bf16 columns
+  static constexpr int DS_BYTES = 4 * DS_SLAB;        // one dS block (128 x 128)
   static constexpr int K_BYTES = (D / 64) * SLAB;     // one K tile (128 x D)
   static constexpr int STAGE_BYTES = DS_BYTES + K_BYTES;
   static constexpr int OUT_WARP = 32 * D * 2;         // one epilogue warp's 32 rows of dQ
@@ -108,12 +111,12 @@ __global__ void __launch_bounds__(192, 1)
           break;
         }
         const int tk0 = original_row_kv(d, w.g * d.G + j * kTile, sh);
-        const int srow = static_cast<int>((blk0 + j) * kTile);
+        const int srow = static_cast<int>((blk0 + j) * 4 * kTile);  // the block's first slab row
         if (elect_one()) {
           const uint32_t bar = smem_u32(&bar_full[s]);
           mbar_arrive_expect_tx(bar, C::STAGE_BYTES);
-          tma_load_2d(sS(s), &tmS, bar, 0, srow);
-          tma_load_2d(sS(s) + C::SLAB, &tmS, bar, 64, srow);
+          tma_load_2d(sS(s), &tmS, bar, 0, srow);                           // slabs 0, 1
+          tma_load_2d(sS(s) + 2 * C::DS_SLAB, &tmS, bar, 0, srow + 2 * kTile);  // slabs 2, 3
           for (int c = 0; c < D / 64; ++c) tma_load_4d(sK(s) + c * C::SLAB, &tmK, bar, c * 64, w.kvh, tk0, w.b);
         }
         __syncwarp();
@@ -125,7 +128,7 @@ __global__ void __launch_bounds__(192, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ UMMA issuer
     const uint32_t idQ = make_idesc_bf16(128, D, 1, 1);  // A = dS (query rows contiguous), B = K (MN-major)
-    const uint64_t dA0 = make_sdesc_sw128(sS(0), C::SLAB, 1024);
+    const uint64_t dA0 = make_sdesc_sw64(sS(0), C::DS_SLAB, 512);   // 32-query slabs of 64-byte rows
     const uint64_t dB0 = make_sdesc_sw128(sK(0), C::SLAB, 1024);
     int L = 0, n = 0;
     bool ok = true;
@@ -147,7 +150,7 @@ __global__ void __launch_bounds__(192, 1)
           const uint64_t db = sdesc_advance(dB0, s * C::STAGE_BYTES);
 #pragma unroll
           for (int kk = 0; kk < kTile / 16; ++kk)
-            umma_ss(tmem + ab * D, sdesc_advance(da, kk * 2048), sdesc_advance(db, kk * 2048), idQ,
+            umma_ss(tmem + ab * D, sdesc_advance(da, kk * 1024), sdesc_advance(db, kk * 2048), idQ,
                     (j > 0 || kk > 0));
           umma_commit(smem_u32(&bar_empty[s]));
           if (j == w.tile) umma_commit(smem_u32(&bar_acc_full[ab]));

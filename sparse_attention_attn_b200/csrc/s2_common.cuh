@@ -343,7 +343,8 @@ struct BwdArgs {
 };
 
 // Split-dS path: index of the 128 x 128 dS block of (query tile i, kv tile
-// j <= i) of group g of (batch b, query head h); blocks hold dS^T, kv-row-major.
+// j <= i) of group g of (batch b, query head h).  A block holds dS^T as four
+// slabs of 32 query columns, each [128 kv rows][32 queries] (64-byte rows).
 __host__ __device__ __forceinline__ long long ds_block(const Dims& d, int b, int h, int g, int i, int j, int tt) {
   return ((static_cast<long long>(b) * d.H + h) * d.n_groups + g) * tt + i * (i + 1) / 2 + j;
 }

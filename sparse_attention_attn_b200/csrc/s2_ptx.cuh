@@ -362,6 +362,18 @@ __device__ __forceinline__ uint64_t make_sdesc_sw128(uint32_t start, uint32_t lb
   return d;
 }
 
+// The same for a 64-byte-swizzled operand (layout type SWIZZLE_64B, 4): rows
+// of 64 bytes, the swizzle pattern repeating every 8 rows (512 bytes).
+__device__ __forceinline__ uint64_t make_sdesc_sw64(uint32_t start, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((start >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1u << 46;
+  d |= (uint64_t)4u << 61;
+  return d;
+}
+
 // The descriptor of the same operand `bytes` further on in shared memory.
 // The start-address field holds address >> 4 in the low 14 bits and shared
 // addresses stay below 256 KiB, so the add never carries out of the field.

@@ -565,8 +565,8 @@ int bwd_impl(int path, int stages, const void* q, const void* k, const void* v, 
                           : nullptr;
   const long long ds_blocks = path == kBwdSplitDs ? ds_blocks_for(B, H, N, G) : 0;
   if (ds != nullptr &&
-      (!make_map_2d(&maps.ds, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ds, kTile, static_cast<uint64_t>(ds_blocks) * kTile,
-                    kTile * 2, 64, kTile, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      (!make_map_2d(&maps.ds, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ds, 32, static_cast<uint64_t>(ds_blocks) * 4 * kTile,
+                    64, 32, 2 * kTile, CU_TENSOR_MAP_SWIZZLE_64B) ||
        !make_map(&maps.dq32, dq, B, N, H, D, 32)))
     return S2ATTN_ERR_CUDA;
   BwdPreArgs pre;
