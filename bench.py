@@ -713,14 +713,19 @@ def other_workload(shape: I.Shape, dev, peaks, steps: int = 5, warmup: int = 3):
             "tokens_per_s": shape.B * shape.N / (ms * 1e-3), "steps": steps, "warmup": warmup}
 
 
-def sweep_variants(D: int):
-    """Every variant the per-shape plan can select at head dim D, as override
-    strings: forward (work order x K/V ring depth) and backward (path x stages)."""
+def sweep_variants(shape: I.Shape, ds_limit_bytes: float = 8.0 * 2 ** 30):
+    """Every variant the per-shape plan can select for a workload shape, as
+    override strings: forward (work order x K/V ring depth) and backward (path
+    x stages).  The split-dS path is swept while its dS blocks stay within
+    ds_limit_bytes (so the sweep never asks for tens of GB of workspace)."""
+    D = shape.D
     slots = (4,) if D == 128 else (4, 6, 8)
     fwd = [f"fwd_order={o},fwd_kv={s}" for o in ("snake", "pairs") for s in slots]
     stages = (2, 3) if D == 128 else (3, 4)
-    bwd = (["bwd=fused"] if D == 128 else []) + [f"bwd={p},bwd_stages={s}" for p in ("split_ds", "split")
-                                                 for s in stages]
+    T = shape.G // 128
+    ds_bytes = shape.B * shape.H * (shape.N // shape.G) * (T * (T + 1) // 2) * 128 * 128 * 2
+    paths = ("split_ds", "split") if ds_bytes <= ds_limit_bytes else ("split",)
+    bwd = (["bwd=fused"] if D == 128 else []) + [f"bwd={p},bwd_stages={s}" for p in paths for s in stages]
     return fwd, bwd
 
 
@@ -740,7 +745,7 @@ def run_sweep(args, dev):
         lse = torch.empty((shape.B, shape.H, shape.N), dtype=torch.float32, device=dev)
         dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
         steps = 10 if shape.N <= 16384 else 4
-        fwd_specs, bwd_specs = sweep_variants(shape.D)
+        fwd_specs, bwd_specs = sweep_variants(shape)
         _lib.s2attn_set_tile_override(None)
         chosen = _lib.s2attn_plan(shape.B, shape.H, shape.Hkv, shape.N, shape.D, shape.G, props.multi_processor_count)
 
