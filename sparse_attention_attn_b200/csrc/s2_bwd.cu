@@ -415,11 +415,16 @@ __global__ void __launch_bounds__(352, 1)
         dk[2 * c4 + 1] = f2_to_bf16x2(f2_mul(f2_pack(p[4 * c4 + 2], p[4 * c4 + 3]), d23));
       }
       tmem_st16(tmem + lane_off + C::TM_DP + bo, dk);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bar_pds[g & 1]));
       if (a.ds != nullptr) {
         // split-dS path: these 32 dS^T values (kv row `row`, query columns
         // half * 32 + [0, 32) of sub-tile i64) also go to their dS block, in
         // its 32-column slab 2 (i64 & 1) + half: the warp's 32 rows write
-        // 2 KB of consecutive bytes
+        // 2 KB of consecutive bytes.  Issued after the arrival, so the dK
+        // UMMA never waits for them.
         const int i64 = 2 * cur.w.tile + cur.it % cur.nq;
         const int hq = cur.w.kvh * d.rep + cur.it / cur.nq;
         const long long blk = ds_block(d, cur.w.b, hq, cur.w.g, i64 >> 1, cur.w.tile, a.ds_tt);
@@ -431,10 +436,6 @@ __global__ void __launch_bounds__(352, 1)
           st_global_v8(dst + 16, hi);
         }
       }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bar_pds[g & 1]));
       if (cur.it == cur.iters - 1) {
         // ---------------------------------------------------- epilogue of this item
         if (lane == 0) ok = mbar_wait(smem_u32(&bar_acc_full), cur.ic.n & 1, wc, 132);
