@@ -507,8 +507,9 @@ def dense_ratio(shape: I.Shape, dev, args):
     import sparse_attention_attn_b200 as s2
     dense = shape.dense()
     q, k, v, do = (t.to(dev) for t in I.make_inputs(dense))
-    ws = torch.empty(s2.bwd_workspace_bytes(dense.B, dense.H, dense.Hkv, dense.N, dense.D, dense.G),
-                     dtype=torch.uint8, device=dev)
+    # one workspace for both calls: the larger of the two plans' needs
+    ws = torch.empty(max(s2.bwd_workspace_bytes(dense.B, dense.H, dense.Hkv, dense.N, dense.D, G)
+                         for G in (shape.G, dense.G)), dtype=torch.uint8, device=dev)
 
     def timed(G, steps):
         for _ in range(3):
