@@ -147,3 +147,23 @@ def test_rejections():
     codes, sq, c2 = (t.to(DEV) for t in I.make_nf4_weights(192, 128, seed=2))
     with pytest.raises(s2.S2AttnError):  # H D = 64 is not a multiple of 128
         s2.nf4_qkv(x, codes, sq, c2, 1, 1, 64)
+
+
+@pytest.mark.parametrize("spec", ["nf4_stages=4", "nf4_dq=12"])
+def test_projection_variants(spec):
+    """Each selectable variant of the NF4 kernel (pipeline depth, dequantization
+    warps) on a shape with more tiles than a B200 has SMs (every CTA crosses
+    tiles) and a ragged token tail."""
+    from sparse_attention_attn_b200 import _lib
+    B, N, K, H, Hkv, D = 1, 2600, 1024, 16, 8, 128
+    rows = (H + 2 * Hkv) * D
+    codes, sq, c2 = I.make_nf4_weights(rows, K, seed=21)
+    _lib.s2attn_set_tile_override(spec)
+    try:
+        x, q, k, v = _run_proj(B, N, K, H, Hkv, D, codes, sq, c2, seed=22)
+    finally:
+        _lib.s2attn_set_tile_override(None)
+    rq, rk, rv = nr.nf4_qkv_projection(x.float().numpy(), nr.unpack_codes(codes.numpy()), sq.numpy(), c2.numpy(),
+                                       H, Hkv, D, bf16_weights=True)
+    for name, got, ref in (("q", q, rq), ("k", k, rk), ("v", v, rv)):
+        _check_proj(f"{name} [{spec}]", _to64(got), ref)
