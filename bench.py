@@ -721,7 +721,8 @@ def sweep_variants(shape: I.Shape, ds_limit_bytes: float = 8.0 * 2 ** 30):
     ds_limit_bytes (so the sweep never asks for tens of GB of workspace)."""
     D = shape.D
     slots = (4,) if D == 128 else (4, 6, 8)
-    fwd = [f"fwd_order={o},fwd_kv={s}" for o in ("snake", "pairs") for s in slots]
+    fwd = [f"fwd_order={o},fwd_kv={s}" for o in ("snake", "pairs") for s in slots] + \
+        [f"fwd_bn=64,fwd_order={o},fwd_kv={s}" for o in ("snake", "pairs") for s in ((8,) if D == 128 else (8, 12))]
     stages = (2, 3) if D == 128 else (3, 4)
     T = shape.G // 128
     ds_bytes = shape.B * shape.H * (shape.N // shape.G) * (T * (T + 1) // 2) * 128 * 128 * 2

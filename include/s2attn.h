@@ -386,7 +386,8 @@ S2ATTN_API int s2attn_profile_stop(float* ms, int* kernel_ids, int capacity);
  * work order (1 longest-first snake, 0 equal-work pairs), out[1] forward K/V
  * ring depth, out[2] backward path (2 split-dS: dQ from the dS blocks the
  * dK/dV kernel stores in the workspace; 0 split: dQ recomputes S and dP; 1
- * fused), out[3] split backward pipeline stages.  Host only; returns a status code (shape validation as in
+ * fused), out[3] split backward pipeline stages, out[4] forward key tile (128,
+ * or 64 with double-buffered scores).  `out` holds 5 ints.  Host only; returns a status code (shape validation as in
  * s2attn_fwd).
  */
 S2ATTN_API int s2attn_plan(int B, int H, int Hkv, int N, int D, int G, int num_sms, int* out);
@@ -397,8 +398,9 @@ S2ATTN_API int s2attn_plan(int B, int H, int Hkv, int N, int D, int G, int num_s
  * environment's value.  The override forces a variant the per-shape selection
  * would not pick, for tests and sweeps: a comma-separated list of key=value
  * items; keys bwd=split_ds|split|fused (backward path; fused exists for head dim 128),
- * fwd_order=snake|pairs (forward work order), fwd_kv=N (forward K/V ring
- * depth: 4 at head dim 128, 4/6/8 at 64), bwd_stages=N (split backward
+ * fwd_order=snake|pairs (forward work order), fwd_bn=64|128 (forward key
+ * tile), fwd_kv=N (forward K/V ring depth: with 128-key tiles 4 at head dim
+ * 128, 4/6/8 at 64; with 64-key tiles 8 at head dim 128, 8/12 at 64), bwd_stages=N (split backward
  * stages: 2-3 at head dim 128, 3-4 at 64), nf4_stages=4|5 and nf4_dq=8|12
  * (pipeline depth and dequantization warps of s2attn_nf4_qkv); values that do not exist for a call's head dim
  * are ignored.  s2attn_bwd_workspace_bytes answers for the

@@ -433,6 +433,26 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
 // bf16x2 (round to nearest even) of a packed fp32 pair
 __device__ __forceinline__ uint32_t f2_to_bf16x2(uint64_t v) { return pack_bf16x2(f2_lo(v), f2_hi(v)); }
 
+// P for 64 scores of one query row: p = 2^(s * sl2 - m), packed to bf16
+// pairs in pk; returns the fp32 sum.  Arguments and sums use packed f32x2
+// arithmetic, the exponentials the MUFU (ex2.approx).
+__device__ __forceinline__ float softmax_row64(const uint32_t (&s0)[32], const uint32_t (&s1)[32], float sl2,
+                                               float m, uint32_t (&pk)[32]) {
+  const uint64_t sc2 = f2_pack(sl2, sl2), nm2 = f2_pack(-m, -m);
+  uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+  for (int c = 0; c < 32; ++c) {
+    const uint32_t* src = (c < 16) ? s0 : s1;
+    const uint64_t x = f2_fma(f2_pack(__uint_as_float(src[(2 * c) & 31]), __uint_as_float(src[(2 * c + 1) & 31])),
+                              sc2, nm2);
+    const uint64_t p = f2_pack(ex2_approx(f2_lo(x)), ex2_approx(f2_hi(x)));
+    pk[c] = f2_to_bf16x2(p);
+    acc[c & 3] = f2_add(acc[c & 3], p);
+  }
+  const uint64_t s = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
+  return f2_lo(s) + f2_hi(s);
+}
+
 // Explicit shared-memory vector load (a pointer into dynamic shared memory
 // that went through integer alignment arithmetic is generic to the compiler,
 // and generic loads take the long-latency path).

@@ -24,6 +24,9 @@ template <int D>
 cudaError_t launch_fwd(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
                        const FwdArgs&, int, cudaStream_t, int);
 template <int D>
+cudaError_t launch_fwd64(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
+                         const FwdArgs&, int, cudaStream_t, int);
+template <int D>
 cudaError_t launch_bwd(const BwdMaps&, const BwdPreArgs&, const BwdArgs&, int, cudaStream_t, int*, int);
 template <int D>
 cudaError_t launch_bwd_fused(const BwdMaps&, const BwdPreArgs&, const BwdArgs&, int, cudaStream_t, int*);
@@ -193,7 +196,7 @@ Dims make_segment_dims(int B, int H, int Hkv, int N, int Nk, int D, int causal) 
 // that the per-shape selection would not pick.  It starts from the
 // S2ATTN_TILE environment variable and can be replaced at run time by the
 // s2attn_set_tile_override test hook.  Keys: bwd=split_ds|split|fused,
-// fwd_order=snake|pairs, fwd_kv=N, bwd_stages=N, nf4_stages=4|5, nf4_dq=8|12.  Unknown
+// fwd_order=snake|pairs, fwd_bn=64|128, fwd_kv=N, bwd_stages=N, nf4_stages=4|5, nf4_dq=8|12.  Unknown
 // keys and values are ignored.
 std::mutex g_override_mu;
 std::string g_override;
@@ -229,12 +232,17 @@ std::string override_value(const std::string& spec, const char* key) {
 // recorded under profiles/ (every variant timed on the five workload shapes).
 struct Plan {
   int fwd_snake;     // forward work order: 1 snake (longest first), 0 equal-work pairs
-  int fwd_kv_slots;  // forward K/V ring depth: 4 (head dim 128), 4/6/8 (head dim 64)
+  int fwd_bn;        // forward key tile: 128 (s2_fwd.cu) or 64 with double-buffered scores (s2_fwd64.cu)
+  int fwd_kv_slots;  // forward K/V ring depth: 128-key tiles 4 (head dim 128), 4/6/8 (head dim 64);
+                     // 64-key tiles 8 (head dim 128), 8/12 (head dim 64)
   int bwd_path;      // kBwdSplitDs, kBwdSplit, or kBwdFused (head dim 128 only)
   int bwd_stages;    // split backward operand stages: 2-3 (head dim 128), 3-4 (head dim 64)
 };
 
-bool valid_kv_slots(int D, int v) { return D == 128 ? v == 4 : (v == 4 || v == 6 || v == 8); }
+bool valid_kv_slots(int D, int bn, int v) {
+  if (bn == 64) return D == 128 ? v == 8 : (v == 8 || v == 12);
+  return D == 128 ? v == 4 : (v == 4 || v == 6 || v == 8);
+}
 bool valid_bwd_stages(int D, int v) { return D == 128 ? (v == 2 || v == 3) : (v == 3 || v == 4); }
 
 Plan select_plan(int B, int H, int Hkv, int N, int D, int G, int sms) {
@@ -248,6 +256,7 @@ Plan select_plan(int B, int H, int Hkv, int N, int D, int G, int sms) {
   // K/V tile running together.
   const double kv_bytes = 2.0 * B * N * Hkv * D * 2.0;
   p.fwd_snake = kv_bytes <= 256.0 * 1024 * 1024 ? 1 : 0;
+  p.fwd_bn = 128;
   p.fwd_kv_slots = D == 128 ? 4 : 8;
   // dQ from the dS the dK/dV kernel stores (five GEMM-units instead of
   // seven) while the dS blocks fit the budget, else the split path that
@@ -261,8 +270,17 @@ Plan select_plan(int B, int H, int Hkv, int N, int D, int G, int sms) {
   const std::string order = override_value(spec, "fwd_order");
   if (order == "snake") p.fwd_snake = 1;
   if (order == "pairs") p.fwd_snake = 0;
+  const std::string bn = override_value(spec, "fwd_bn");
+  if (bn == "64" && p.fwd_bn != 64) {
+    p.fwd_bn = 64;
+    p.fwd_kv_slots = 8;
+  }
+  if (bn == "128" && p.fwd_bn != 128) {
+    p.fwd_bn = 128;
+    p.fwd_kv_slots = D == 128 ? 4 : 8;
+  }
   const std::string kv = override_value(spec, "fwd_kv");
-  if (!kv.empty() && valid_kv_slots(D, std::atoi(kv.c_str()))) p.fwd_kv_slots = std::atoi(kv.c_str());
+  if (!kv.empty() && valid_kv_slots(D, p.fwd_bn, std::atoi(kv.c_str()))) p.fwd_kv_slots = std::atoi(kv.c_str());
   const std::string path = override_value(spec, "bwd");
   if (path == "split") p.bwd_path = kBwdSplit;
   if (path == "split_ds") p.bwd_path = kBwdSplitDs;
@@ -376,14 +394,14 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, c
   DeviceInfo info;
   if (!device_info(&info)) return S2ATTN_ERR_CUDA;
   if (!info.ok) return S2ATTN_ERR_UNSUPPORTED;
+  const Plan plan = select_plan(B, H, Hkv, N, D, G, info.sms);
   CUtensorMap tq, tk, tv, to;
-  if (!make_map(&tq, q, B, N, H, D) || !make_map(&tk, k, B, dims.Nk, Hkv, D) ||
-      !make_map(&tv, v, B, dims.Nk, Hkv, D) || !make_map(&to, o, B, N, H, D, 32))
+  if (!make_map(&tq, q, B, N, H, D) || !make_map(&tk, k, B, dims.Nk, Hkv, D, plan.fwd_bn) ||
+      !make_map(&tv, v, B, dims.Nk, Hkv, D, plan.fwd_bn) || !make_map(&to, o, B, N, H, D, 32))
     return S2ATTN_ERR_CUDA;
   FwdArgs a;
   a.d = dims;
   a.hist = hist;
-  const Plan plan = select_plan(B, H, Hkv, N, D, G, info.sms);
   a.sched = make_fwd_sched(a.d, plan.fwd_snake);
   a.scale_log2 = static_cast<float>(1.4426950408889634 / __builtin_sqrt(static_cast<double>(D)));
   a.lse = lse;  // o is written through its TMA map
@@ -396,8 +414,13 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, c
   a.status = static_cast<uint32_t*>(status);
   a.wait_limit_ns = wait_limit_ns();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = (D == 64) ? launch_fwd<64>(tq, tk, tv, to, a, info.sms, s, plan.fwd_kv_slots)
-                             : launch_fwd<128>(tq, tk, tv, to, a, info.sms, s, plan.fwd_kv_slots);
+  cudaError_t e;
+  if (plan.fwd_bn == 64)
+    e = (D == 64) ? launch_fwd64<64>(tq, tk, tv, to, a, info.sms, s, plan.fwd_kv_slots)
+                  : launch_fwd64<128>(tq, tk, tv, to, a, info.sms, s, plan.fwd_kv_slots);
+  else
+    e = (D == 64) ? launch_fwd<64>(tq, tk, tv, to, a, info.sms, s, plan.fwd_kv_slots)
+                  : launch_fwd<128>(tq, tk, tv, to, a, info.sms, s, plan.fwd_kv_slots);
   if (e != cudaSuccess) {
     g_last_cuda_error = static_cast<int>(e);
     return S2ATTN_ERR_CUDA;
@@ -934,6 +957,7 @@ int s2attn_plan(int B, int H, int Hkv, int N, int D, int G, int num_sms, int* ou
   out[1] = p.fwd_kv_slots;
   out[2] = p.bwd_path;
   out[3] = p.bwd_stages;
+  out[4] = p.fwd_bn;
   return S2ATTN_OK;
 }
 

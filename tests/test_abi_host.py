@@ -137,6 +137,7 @@ def test_plan_selection_table():
     for s in I.WORKLOADS:
         p = _lib.s2attn_plan(s.B, s.H, s.Hkv, s.N, s.D, s.G, 148)
         assert (p["fwd_order"], p["fwd_kv_slots"], p["bwd_path"], p["bwd_stages"]) == expect[s.name], s.name
+        assert p["fwd_bn"] == 128
     with pytest.raises(_lib.S2AttnError):
         _lib.s2attn_plan(1, 4, 3, 1024, 64, 256, 148)
 
@@ -147,14 +148,21 @@ def test_plan_override_parsing():
     try:
         _lib.s2attn_set_tile_override("fwd_order=pairs,fwd_kv=2,bwd=split,bwd_stages=2")
         p = _lib.s2attn_plan(1, 32, 32, 8192, 128, 2048, 148)   # a 2-slot K/V ring does not exist
-        assert p == {"fwd_order": "pairs", "fwd_kv_slots": 4, "bwd_path": "split", "bwd_stages": 2}
+        assert p == {"fwd_order": "pairs", "fwd_bn": 128, "fwd_kv_slots": 4, "bwd_path": "split", "bwd_stages": 2}
         p = _lib.s2attn_plan(1, 4, 4, 1024, 64, 256, 148)   # head dim 64: kv 2 and stages 2 do not exist
-        assert p == {"fwd_order": "pairs", "fwd_kv_slots": 8, "bwd_path": "split", "bwd_stages": 3}
+        assert p == {"fwd_order": "pairs", "fwd_bn": 128, "fwd_kv_slots": 8, "bwd_path": "split", "bwd_stages": 3}
         _lib.s2attn_set_tile_override("bwd=fused,fwd_kv=6,bwd_stages=4,junk,=,x=y")  # no fused path at D = 64
         assert _lib.s2attn_plan(1, 4, 4, 1024, 64, 256, 148) == \
-            {"fwd_order": "snake", "fwd_kv_slots": 6, "bwd_path": "split_ds", "bwd_stages": 4}
+            {"fwd_order": "snake", "fwd_bn": 128, "fwd_kv_slots": 6, "bwd_path": "split_ds", "bwd_stages": 4}
         assert _lib.s2attn_plan(1, 32, 32, 8192, 128, 2048, 148) == \
-            {"fwd_order": "snake", "fwd_kv_slots": 4, "bwd_path": "fused", "bwd_stages": 3}
+            {"fwd_order": "snake", "fwd_bn": 128, "fwd_kv_slots": 4, "bwd_path": "fused", "bwd_stages": 3}
+        _lib.s2attn_set_tile_override("fwd_bn=64,fwd_kv=4")  # 4 slots do not exist for 64-key tiles
+        assert _lib.s2attn_plan(1, 32, 32, 8192, 128, 2048, 148)["fwd_bn"] == 64
+        assert _lib.s2attn_plan(1, 32, 32, 8192, 128, 2048, 148)["fwd_kv_slots"] == 8
+        assert _lib.s2attn_plan(1, 4, 4, 1024, 64, 256, 148)["fwd_kv_slots"] == 8
+        _lib.s2attn_set_tile_override("fwd_bn=64,fwd_kv=12")
+        assert _lib.s2attn_plan(1, 4, 4, 1024, 64, 256, 148)["fwd_kv_slots"] == 12
+        assert _lib.s2attn_plan(1, 32, 32, 8192, 128, 2048, 148)["fwd_kv_slots"] == 8
         _lib.s2attn_set_tile_override("bwd=split_ds")  # forced even over the budget
         assert _lib.s2attn_plan(1, 64, 8, 32768, 128, 8192, 148)["bwd_path"] == "split_ds"
     finally:

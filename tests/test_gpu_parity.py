@@ -85,6 +85,7 @@ PLAN_VARIANTS = [
     (128, "fwd_order=pairs"), (128, "bwd=split,bwd_stages=2"), (128, "bwd=split,bwd_stages=3"),
     (128, "bwd=split_ds,bwd_stages=2"), (128, "bwd=fused"), (64, "fwd_order=pairs"), (64, "fwd_kv=4"),
     (64, "fwd_kv=6"), (64, "bwd=split,bwd_stages=4"), (64, "bwd=split_ds,bwd_stages=4"),
+    (128, "fwd_bn=64"), (128, "fwd_bn=64,fwd_order=pairs"), (64, "fwd_bn=64"), (64, "fwd_bn=64,fwd_kv=12"),
 ]
 
 
