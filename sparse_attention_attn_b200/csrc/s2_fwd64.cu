@@ -57,7 +57,7 @@ __global__ void __launch_bounds__(320, 1)
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   __shared__ __align__(8) uint64_t bar_qfull[NQ], bar_qempty[NQ], bar_full[NS], bar_empty[NS], bar_s[2][2],
-      bar_p[2], bar_o[2], bar_ofree[2], bar_drain;
+      bar_p[2][2], bar_o[2], bar_ofree[2], bar_drain;
   __shared__ uint32_t tmem_slot;
   __shared__ uint32_t abort_flag;
 
@@ -85,7 +85,12 @@ __global__ void __launch_bounds__(320, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&bar_s[i][0]), 1);
       mbar_init(smem_u32(&bar_s[i][1]), 1);
-      mbar_init(smem_u32(&bar_p[i]), 4);  // P written: one arrival per warp of the warpgroup
+      // P written into buffer 0 / 1: one arrival per warp of the warpgroup.  One
+      // barrier per buffer: the softmax may run a tile ahead of the issuer (both
+      // scores of the next two tiles can be ready), so a single barrier could
+      // complete two phases before the issuer looks at the first
+      mbar_init(smem_u32(&bar_p[i][0]), 4);
+      mbar_init(smem_u32(&bar_p[i][1]), 4);
       mbar_init(smem_u32(&bar_o[i]), 1);
       mbar_init(smem_u32(&bar_ofree[i]), 4);
     }
@@ -216,11 +221,11 @@ __global__ void __launch_bounds__(320, 1)
       __syncwarp();
       return true;
     };
-    int L = 0, n = 0, np[2] = {0, 0};  // ring loads and items consumed, P tiles received per warpgroup
+    int L = 0, n = 0, np[2][2] = {{0, 0}, {0, 0}};  // ring loads, items consumed, P tiles received per buffer
     // O_wg (+)= P_wg(j) V(load Lv) once P(j) is in TMEM (and, for an item's
     // first tile, once the epilogue has read the previous item's O)
     auto pv = [&](int wg, int Lv, int j) -> bool {
-      if (!warp_wait(smem_u32(&bar_p[wg]), np[wg] & 1, wc, wg == 0 ? 22 : 24) ||
+      if (!warp_wait(smem_u32(&bar_p[wg][j & 1]), np[wg][j & 1] & 1, wc, wg == 0 ? 22 : 24) ||
           (j == 0 && n > 0 && !warp_wait(smem_u32(&bar_ofree[wg]), (n - 1) & 1, wc, wg == 0 ? 23 : 25)) ||
           !wait_full(Lv))
         return false;
@@ -234,7 +239,7 @@ __global__ void __launch_bounds__(320, 1)
         umma_commit(smem_u32(&bar_o[wg]));
       }
       __syncwarp();
-      ++np[wg];
+      ++np[wg][j & 1];
       return true;
     };
     bool pre = false;  // this item's first scores were issued during the previous item
@@ -399,7 +404,7 @@ __global__ void __launch_bounds__(320, 1)
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(smem_u32(&bar_p[wg]));
+          if (lane == 0) mbar_arrive(smem_u32(&bar_p[wg][buf]));
           ++no;
         }
         // ---------------------------------------------------------- epilogue
