@@ -385,7 +385,9 @@ __global__ void __launch_bounds__(320, 1)
           tmem_st32(tS + buf * 64, pk);
           if (__any_sync(0xffffffffu, resc)) {
             // rescale O (it holds P V up to tile j-1 once that UMMA has
-            // completed) before P(j) V(j) accumulates onto it
+            // completed) before P(j) V(j) accumulates onto it.  P V(j-2) is
+            // complete (S(j) was issued after it), so only P V(j-1) can be
+            // pending and the parity wait is unambiguous
             if (lane == 0) ok = mbar_wait(smem_u32(&bar_o[wg]), (no - 1) & 1, wc, 31);
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
@@ -408,8 +410,15 @@ __global__ void __launch_bounds__(320, 1)
           ++no;
         }
         // ---------------------------------------------------------- epilogue
+        // The last two P V may both be in flight (the softmax can be a tile
+        // ahead of the issuer): wait for them in order, or a parity wait on
+        // the last one could be answered by the phase before the other.
+        // (UMMAs complete in order, so every earlier P V is done: this tile's
+        // S was issued after P V(nt - 3).)
         if (ok) {
-          if (lane == 0) ok = mbar_wait(smem_u32(&bar_o[wg]), (no - 1) & 1, wc, 32);
+          if (lane == 0)
+            ok = mbar_wait(smem_u32(&bar_o[wg]), (no - 2) & 1, wc, 32) &&
+                 mbar_wait(smem_u32(&bar_o[wg]), (no - 1) & 1, wc, 32);
           ok = __shfl_sync(0xffffffffu, ok, 0);
         }
         if (!ok) break;
