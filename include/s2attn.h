@@ -89,8 +89,12 @@ S2ATTN_API int s2attn_fwd(const void* q, const void* k, const void* v, void* o, 
 /*
  * Bytes of device workspace s2attn_bwd needs: a 256-byte device status block,
  * then two fp32 [B, H, N] arrays written by the backward's first kernel:
- * -Delta (Delta_t = sum_d dO_td * O_td) and -lse_t * log2(e); at head dim 128
- * (the fused backward) also an fp32 [B, H, N, D] accumulator for dq.
+ * -Delta (Delta_t = sum_d dO_td * O_td) and -lse_t * log2(e); then what the
+ * planned backward path keeps (s2attn_plan out[2]): for the split-dS path the
+ * bf16 dS blocks (32 KB per 128 x 128 block, (H/Hkv) T (T+1)/2 blocks per
+ * (batch, kv head, group), T = G/128) of out[5] such units at once, at most
+ * 4 GiB unless the override asks for more; for the fused path an fp32
+ * [B, H, N, D] accumulator for dq; nothing more for the split path.
  */
 S2ATTN_API size_t s2attn_bwd_workspace_bytes(int B, int H, int Hkv, int N, int D, int G);
 
@@ -373,7 +377,8 @@ S2ATTN_API const char* s2attn_cuda_error_string(int err);
  * s2attn_profile_stop turns recording off, waits for the recorded events and
  * writes per-launch durations (ms) and kernel ids (0 forward, 1 backward
  * preprocess, 2 backward dK/dV, 3 backward dQ, 4 fused backward, 5 its dq
- * conversion, 6 RoPE rotation, 7 NF4 QKV projection, 8 NF4 dequantization) to caller arrays of
+ * conversion, 6 RoPE rotation, 7 NF4 QKV projection, 8 NF4 dequantization, 9
+ * backward dQ from the stored dS) to caller arrays of
  * `capacity` entries (either may be NULL).  Returns the number of records, or
  * minus a status code.
  */
@@ -387,8 +392,12 @@ S2ATTN_API int s2attn_profile_stop(float* ms, int* kernel_ids, int capacity);
  * ring depth, out[2] backward path (2 split-dS: dQ from the dS blocks the
  * dK/dV kernel stores in the workspace; 0 split: dQ recomputes S and dP; 1
  * fused), out[3] split backward pipeline stages, out[4] forward key tile (128,
- * or 64 with double-buffered scores).  `out` holds 5 ints.  Host only; returns a status code (shape validation as in
- * s2attn_fwd).
+ * or 64 with double-buffered scores), out[5] on the split-dS path the dK/dV
+ * units (batch x kv head x group) whose dS blocks the workspace holds at once
+ * (all of them when they fit its 4 GiB budget; fewer, and the backward runs
+ * its dK/dV work in ranges of pairs each followed by dQ for the units the
+ * range completed), else 0.  `out` holds 6 ints.  Host only; returns a status
+ * code (shape validation as in s2attn_fwd).
  */
 S2ATTN_API int s2attn_plan(int B, int H, int Hkv, int N, int D, int G, int num_sms, int* out);
 
@@ -398,6 +407,7 @@ S2ATTN_API int s2attn_plan(int B, int H, int Hkv, int N, int D, int G, int num_s
  * environment's value.  The override forces a variant the per-shape selection
  * would not pick, for tests and sweeps: a comma-separated list of key=value
  * items; keys bwd=split_ds|split|fused (backward path; fused exists for head dim 128),
+ * ds_slots=N (N >= 2: the split-dS path's workspace holds dS of N dK/dV units),
  * fwd_order=snake|pairs (forward work order), fwd_bn=64|128 (forward key
  * tile), fwd_kv=N (forward K/V ring depth: with 128-key tiles 4 at head dim
  * 128, 4/6/8 at 64; with 64-key tiles 8 at head dim 128, 8/12 at 64), bwd_stages=N (split backward

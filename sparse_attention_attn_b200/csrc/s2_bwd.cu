@@ -359,6 +359,7 @@ __global__ void __launch_bounds__(352, 1)
     bool ok = true;
     DkvCursor cur;
     cur.first(d, ps);
+    long long ds_base = 0;
     for (int g = 0; cur.ic.valid; ++g) {
       const int s = g % ST;
       const int qoff = (cur.it % cur.nq) * kSub;  // query sub-tile start minus kv tile start (rolled)
@@ -425,9 +426,12 @@ __global__ void __launch_bounds__(352, 1)
         // its 32-column slab 2 (i64 & 1) + half: the warp's 32 rows write
         // 2 KB of consecutive bytes.  Issued after the arrival, so the dK
         // UMMA never waits for them.
-        const int i64 = 2 * cur.w.tile + cur.it % cur.nq;
-        const int hq = cur.w.kvh * d.rep + cur.it / cur.nq;
-        const long long blk = ds_block(d, cur.w.b, hq, cur.w.g, i64 >> 1, cur.w.tile, a.ds_tt);
+        // the item's first block (query head kvh rep, tile 0, kv tile 0),
+        // formed once per item; then query head, query tile and kv tile as
+        // ds_block orders them
+        if (cur.it == 0) ds_base = ds_block(d, cur.w.b, cur.w.h, cur.w.g, 0, 0, a.ds_tt, a.ds_slots);
+        const int i64 = 2 * cur.w.tile + cur.it % cur.nq, i = i64 >> 1;
+        const long long blk = ds_base + static_cast<long long>(cur.it / cur.nq) * a.ds_tt + i * (i + 1) / 2 + cur.w.tile;
         if (in_bounds(wc.status, blk, a.ds_blocks, 48)) {
           __nv_bfloat16* dst = a.ds + blk * (kTile * kTile) + (2 * (i64 & 1) + half) * (kTile * 32) + row * 32;
           const uint32_t lo[8] = {dk[0], dk[1], dk[2], dk[3], dk[4], dk[5], dk[6], dk[7]};
@@ -947,8 +951,41 @@ cudaError_t launch_bwd_stages(const BwdMaps& m, const BwdPreArgs& pre, const Bwd
     return cudaErrorInvalidValue;
   cudaError_t e = launch_bwd_pre<D>(pre, num_sms, stream);
   if (e != cudaSuccess) return e;
+  if (a.ds != nullptr) {
+    // split-dS path: dK/dV over consecutive ranges of its pairs, each followed
+    // by dQ for the units the range completed (their dS blocks all stored);
+    // the workspace's slots then serve the next range's units.  One range
+    // when every unit's dS fits.
+    const int total = a.kv_sched.pairs, ppu = a.kv_sched.ppu;
+    const int chunk = ds_chunk_pairs(a.kv_sched, a.ds_slots, num_sms);
+    BwdArgs c = a;
+    int done = 0, n = 1;
+    for (int p0 = 0; p0 < total; p0 += chunk) {
+      const int p1 = p0 + chunk < total ? p0 + chunk : total;
+      c.kv_sched.p0 = p0;
+      c.kv_sched.pairs = p1;
+      prof_before(stream, kKernelBwdDkDv);
+      s2_bwd_dkdv_kernel<D, NST><<<pair_grid(c.kv_sched, num_sms), K3::THREADS, K3::SMEM_BYTES, stream>>>(
+          m.q64, m.k128, m.v128, m.g64, c);
+      e = cudaGetLastError();
+      prof_after(stream);
+      if (e != cudaSuccess) return e;
+      ++n;
+      const int upto = p1 / ppu;  // units with every pair done
+      if (upto > done) {
+        c.q_sched.p0 = done * a.d.rep * a.q_sched.ppu;
+        c.q_sched.pairs = upto * a.d.rep * a.q_sched.ppu;
+        e = launch_dq_ds<D>(m.ds, m.k128, m.dq32, c, num_sms, stream);
+        if (e != cudaSuccess) return e;
+        ++n;
+        done = upto;
+      }
+    }
+    if (launches) *launches = n;
+    return cudaSuccess;
+  }
   if (!a.no_dkdv) {
-    const int grid_kv = a.kv_sched.pairs < num_sms ? a.kv_sched.pairs : num_sms;
+    const int grid_kv = pair_grid(a.kv_sched, num_sms);
     prof_before(stream, kKernelBwdDkDv);
     s2_bwd_dkdv_kernel<D, NST><<<grid_kv, K3::THREADS, K3::SMEM_BYTES, stream>>>(m.q64, m.k128, m.v128, m.g64, a);
     e = cudaGetLastError();
@@ -956,8 +993,7 @@ cudaError_t launch_bwd_stages(const BwdMaps& m, const BwdPreArgs& pre, const Bwd
     if (e != cudaSuccess) return e;
   }
   if (launches) *launches = a.no_dkdv ? 2 : 3;
-  if (a.ds != nullptr) return launch_dq_ds<D>(m.ds, m.k128, m.dq32, a, num_sms, stream);  // dQ from the stored dS
-  const int grid_q = a.q_sched.pairs < num_sms ? a.q_sched.pairs : num_sms;
+  const int grid_q = pair_grid(a.q_sched, num_sms);
   prof_before(stream, kKernelBwdDq);
   s2_bwd_dq_kernel<D, NST><<<grid_q, K4::THREADS, K4::SMEM_BYTES, stream>>>(m.q128, m.k64, m.v64, m.g128, a);
   e = cudaGetLastError();

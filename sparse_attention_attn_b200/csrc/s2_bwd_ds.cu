@@ -103,7 +103,7 @@ __global__ void __launch_bounds__(192, 1)
     for (ic.first(ps); ok && ic.valid; ic.next(ps)) {
       const TileWork w = q_item(d, ic.unit, ic.tile);
       const int sh = shift_of_head(d, w.h);
-      const long long blk0 = ds_block(d, w.b, w.h, w.g, w.tile, 0, a.ds_tt);
+      const long long blk0 = ds_block(d, w.b, w.h, w.g, w.tile, 0, a.ds_tt, a.ds_slots);
       for (int j = 0; j <= w.tile; ++j, ++L) {
         const int s = L % ST, f = L / ST;
         if (f > 0 && !warp_wait(smem_u32(&bar_empty[s]), (f - 1) & 1, wc, 300)) {
@@ -226,7 +226,7 @@ cudaError_t launch_dq_ds_stages(const CUtensorMap& tds, const CUtensorMap& tk, c
   cudaError_t ea =
       cudaFuncSetAttribute(s2_bwd_dq_ds_kernel<D, NST>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (ea != cudaSuccess) return ea;
-  const int grid = a.q_sched.pairs < num_sms ? a.q_sched.pairs : num_sms;
+  const int grid = pair_grid(a.q_sched, num_sms);
   prof_before(stream, kKernelBwdDqDs);
   s2_bwd_dq_ds_kernel<D, NST><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tds, tk, tq32, a);
   cudaError_t e = cudaGetLastError();

@@ -576,7 +576,7 @@ cudaError_t launch_bwd_fused(const BwdMaps& m, const BwdPreArgs& pre, const BwdA
     return cudaErrorInvalidValue;
   cudaError_t e = launch_bwd_pre<D>(pre, num_sms, stream);
   if (e != cudaSuccess) return e;
-  const int grid = a.kv_sched.pairs < num_sms ? a.kv_sched.pairs : num_sms;
+  const int grid = pair_grid(a.kv_sched, num_sms);
   prof_before(stream, kKernelBwdFused);
   s2_bwd_fused_kernel<D><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(m.q64, m.k128, m.v128, m.g64, a);
   e = cudaGetLastError();

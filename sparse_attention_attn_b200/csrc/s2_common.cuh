@@ -89,8 +89,11 @@ struct TileWork {
 // pair carries the same work.  Pairs are dealt round-robin to the CTAs (one
 // per SM), consecutive pairs belong to the same unit, so the CTAs running at
 // one time share their K/V (or Q/dO) in L2.
+// A launch can take a contiguous range [p0, pairs) of the pairs (the chunks
+// of the split-dS backward); p0 = 0 and pairs = units * ppu otherwise.
 struct PairSched {
-  int units, T, ppu, pairs;  // ppu = pairs per unit
+  int units, T, ppu, pairs;  // ppu = pairs per unit; pairs = end of this launch's range
+  int p0;                    // first pair of this launch's range
 };
 
 __host__ __device__ __forceinline__ PairSched make_pair_sched(int units, int T) {
@@ -99,7 +102,14 @@ __host__ __device__ __forceinline__ PairSched make_pair_sched(int units, int T) 
   ps.T = T;
   ps.ppu = (T + 1) / 2;
   ps.pairs = units * ps.ppu;
+  ps.p0 = 0;
   return ps;
+}
+
+// CTAs of a persistent launch over the range: one per pair, at most one per SM.
+__host__ __device__ __forceinline__ int pair_grid(const PairSched& ps, int num_sms) {
+  const int n = ps.pairs - ps.p0;
+  return n < num_sms ? n : num_sms;
 }
 
 // Item `e` (0 or 1) of pair p: its unit and tile; false if it does not exist
@@ -113,12 +123,12 @@ __host__ __device__ __forceinline__ bool pair_item(const PairSched& ps, int p, i
   return !(e == 1 && tile == pj);
 }
 
-// Walks the items of one CTA in order: pairs blockIdx.x, +gridDim.x, ...
+// Walks the items of one CTA in order: pairs p0 + blockIdx.x, +gridDim.x, ...
 struct ItemCursor {
   int p, e, unit, tile, n;  // n = items visited before this one
   bool valid;
   __device__ __forceinline__ void first(const PairSched& ps) {
-    p = blockIdx.x;
+    p = ps.p0 + blockIdx.x;
     e = 0;
     n = 0;
     valid = pair_item(ps, p, e, unit, tile);
@@ -337,16 +347,35 @@ struct BwdArgs {
                            // (the inputs were rotated by it), or null
   __nv_bfloat16* ds;       // split-dS path: the dK/dV kernel stores dS blocks here (see ds_block), or null
   int ds_tt;               // dS blocks per (batch, head, group): T (T + 1) / 2
-  long long ds_blocks;     // dS blocks in all
+  int ds_slots;            // dK/dV units whose dS the workspace holds at once (unit u uses slot u mod ds_slots)
+  long long ds_blocks;     // dS blocks in all: ds_slots * rep * ds_tt
   uint32_t* status;
   unsigned long long wait_limit_ns;
 };
 
 // Split-dS path: index of the 128 x 128 dS block of (query tile i, kv tile
-// j <= i) of group g of (batch b, query head h).  A block holds dS^T as four
-// slabs of 32 query columns, each [128 kv rows][32 queries] (64-byte rows).
-__host__ __device__ __forceinline__ long long ds_block(const Dims& d, int b, int h, int g, int i, int j, int tt) {
-  return ((static_cast<long long>(b) * d.H + h) * d.n_groups + g) * tt + i * (i + 1) / 2 + j;
+// j <= i) of group g of (batch b, query head h).  The blocks of one dK/dV unit
+// u = (b Hkv + kvh) n_groups + g (its rep query heads) sit together in slot
+// u mod slots; the workspace holds `slots` units at once, and the backward
+// runs in pair ranges whose live units never share a slot.  A block holds dS^T
+// as four slabs of 32 query columns, each [128 kv rows][32 queries] (64-byte
+// rows).
+__host__ __device__ __forceinline__ long long ds_block(const Dims& d, int b, int h, int g, int i, int j, int tt,
+                                                       int slots) {
+  const int kvh = h / d.rep;
+  const int u = (b * d.Hkv + kvh) * d.n_groups + g;
+  return (static_cast<long long>(u % slots) * d.rep + (h - kvh * d.rep)) * tt + i * (i + 1) / 2 + j;
+}
+
+// Split-dS path: pairs of dK/dV work per launch when the workspace holds
+// `slots` units of dS (every unit: no chunking).  A range of c pairs starting
+// anywhere touches at most 1 + ceil((c - 1) / ppu) units, which must fit the
+// slots: c <= (slots - 1) ppu + 1.  Within that, whole rounds of `num_sms`
+// pairs, so every launch but the last keeps all CTAs busy to its end.
+__host__ __device__ __forceinline__ int ds_chunk_pairs(const PairSched& kv, int slots, int num_sms) {
+  if (slots >= kv.units) return kv.pairs;
+  const int maxc = (slots - 1) * kv.ppu + 1;
+  return maxc >= num_sms ? maxc / num_sms * num_sms : maxc;
 }
 
 // TMA descriptors of the backward: 128-row and 64-row boxes of each operand.

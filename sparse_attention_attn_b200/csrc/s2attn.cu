@@ -57,15 +57,29 @@ constexpr size_t kStatusBytes = 256;
 // conversion.
 enum BwdPath : int { kBwdSplit = 0, kBwdFused = 1, kBwdSplitDs = 2 };
 
-// The split-dS path stores every dS block (32 KB per (query tile, kv tile <=
-// it) of each (batch, head, group)) in the workspace; it is planned while that
-// stays within this budget.
+// The split-dS path stores the dS blocks (32 KB per (query tile, kv tile <=
+// it) of each (batch, head, group)) in the workspace, within this budget: all
+// of them when they fit, else those of as many dK/dV units (batch x kv head x
+// group, with its query heads) as fit, the backward then running in ranges.
 constexpr double kDsBudgetBytes = 4.0 * 1024 * 1024 * 1024;
 
-// dS blocks of the split-dS path: B H (N/G) T (T+1) / 2, T = G/128.
-long long ds_blocks_for(int B, int H, int N, int G) {
+// dS blocks of one dK/dV unit: (H/Hkv) T (T+1) / 2, T = G/128.
+long long ds_unit_blocks(int H, int Hkv, int G) {
   const long long T = G / kTile;
-  return static_cast<long long>(B) * H * (N / G) * (T * (T + 1) / 2);
+  return static_cast<long long>(H / Hkv) * (T * (T + 1) / 2);
+}
+
+// dK/dV units whose dS the workspace holds at once: every unit if they fit
+// the budget, else as many as fit if that is at least 2 (each range of the
+// backward then completes at least one unit), else 0 (no split-dS plan).
+// `want` > 0 (a plan override) asks for that many instead, from 2 up.
+int ds_slots_for(int B, int H, int Hkv, int N, int G, int want = 0) {
+  const long long units = static_cast<long long>(B) * Hkv * (N / G);
+  const double unit_bytes = static_cast<double>(ds_unit_blocks(H, Hkv, G)) * kTile * kTile * 2;
+  long long fit = static_cast<long long>(kDsBudgetBytes / unit_bytes);
+  if (want >= 2) fit = want;
+  if (fit >= units) return static_cast<int>(units);
+  return fit >= 2 ? static_cast<int>(fit) : 0;
 }
 
 
@@ -195,7 +209,7 @@ Dims make_segment_dims(int B, int H, int Hkv, int N, int Nk, int D, int causal) 
 // A plan override string ("key=value,..."), used to time or test a variant
 // that the per-shape selection would not pick.  It starts from the
 // S2ATTN_TILE environment variable and can be replaced at run time by the
-// s2attn_set_tile_override test hook.  Keys: bwd=split_ds|split|fused,
+// s2attn_set_tile_override test hook.  Keys: bwd=split_ds|split|fused, ds_slots=N,
 // fwd_order=snake|pairs, fwd_bn=64|128, fwd_kv=N, bwd_stages=N, nf4_stages=4|5, nf4_dq=8|12.  Unknown
 // keys and values are ignored.
 std::mutex g_override_mu;
@@ -237,6 +251,7 @@ struct Plan {
                      // 64-key tiles 8 (head dim 128), 8/12 (head dim 64)
   int bwd_path;      // kBwdSplitDs, kBwdSplit, or kBwdFused (head dim 128 only)
   int bwd_stages;    // split backward operand stages: 2-3 (head dim 128), 3-4 (head dim 64)
+  int ds_slots;      // split-dS path: dK/dV units whose dS the workspace holds (see ds_slots_for)
 };
 
 bool valid_kv_slots(int D, int bn, int v) {
@@ -262,8 +277,8 @@ Plan select_plan(int B, int H, int Hkv, int N, int D, int G, int sms) {
   // seven) while the dS blocks fit the budget, else the split path that
   // recomputes S and dP for dQ; the fused path measured slower than both and
   // stays selectable
-  p.bwd_path = static_cast<double>(ds_blocks_for(B, H, N, G)) * kTile * kTile * 2 <= kDsBudgetBytes ? kBwdSplitDs
-                                                                                                      : kBwdSplit;
+  p.ds_slots = ds_slots_for(B, H, Hkv, N, G);
+  p.bwd_path = p.ds_slots > 0 ? kBwdSplitDs : kBwdSplit;
   p.bwd_stages = 3;
   // the override, where it names a variant that exists for this head dim
   const std::string spec = tile_override();
@@ -283,6 +298,9 @@ Plan select_plan(int B, int H, int Hkv, int N, int D, int G, int sms) {
   if (!kv.empty() && valid_kv_slots(D, p.fwd_bn, std::atoi(kv.c_str()))) p.fwd_kv_slots = std::atoi(kv.c_str());
   const std::string path = override_value(spec, "bwd");
   if (path == "split") p.bwd_path = kBwdSplit;
+  const std::string slots = override_value(spec, "ds_slots");
+  if (!slots.empty() && std::atoi(slots.c_str()) >= 2) p.ds_slots = ds_slots_for(B, H, Hkv, N, G, std::atoi(slots.c_str()));
+  if (path == "split_ds" && p.ds_slots == 0) p.ds_slots = ds_slots_for(B, H, Hkv, N, G, 2);
   if (path == "split_ds") p.bwd_path = kBwdSplitDs;
   if (path == "fused" && D == 128) p.bwd_path = kBwdFused;
   const std::string st = override_value(spec, "bwd_stages");
@@ -347,11 +365,11 @@ size_t rowstat_bytes(int B, int H, int N) {
 }
 
 // Workspace: status block, -Delta, -lse*log2(e); for the fused path the fp32
-// [B, H, N, D] dQ accumulator; for the split-dS path the dS blocks.
-size_t workspace_bytes_for(int path, int B, int H, int N, int D, int G) {
+// [B, H, N, D] dQ accumulator; for the split-dS path `ds_blocks` dS blocks.
+size_t workspace_bytes_for(int path, int B, int H, int N, int D, long long ds_blocks = 0) {
   size_t n = kStatusBytes + 2 * rowstat_bytes(B, H, N);
   if (path == kBwdFused) n += round_up(static_cast<size_t>(B) * H * N * D * sizeof(float), 256);
-  if (path == kBwdSplitDs) n += static_cast<size_t>(ds_blocks_for(B, H, N, G)) * kTile * kTile * 2;
+  if (path == kBwdSplitDs) n += static_cast<size_t>(ds_blocks) * kTile * kTile * 2;
   return n;
 }
 
@@ -518,7 +536,8 @@ const char* s2attn_cuda_error_string(int err) {
 
 size_t s2attn_bwd_workspace_bytes(int B, int H, int Hkv, int N, int D, int G) {
   if (validate_shape(B, H, Hkv, N, D, G) != S2ATTN_OK) return 0;
-  return workspace_bytes_for(select_plan(B, H, Hkv, N, D, G, 0).bwd_path, B, H, N, D, G);
+  const Plan p = select_plan(B, H, Hkv, N, D, G, 0);
+  return workspace_bytes_for(p.bwd_path, B, H, N, D, p.ds_slots * ds_unit_blocks(H, Hkv, G));
 }
 
 int s2attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
@@ -541,12 +560,13 @@ int s2attn_seg_fwd(const void* q, const void* k, const void* v, void* o, float* 
 }  // extern "C"
 
 namespace {
-// The backward on `path` (kBwdSplit or kBwdFused).  `seg`: segment-mode
+// The backward on `path` (kBwdSplitDs, kBwdSplit or kBwdFused); ds_slots: the
+// split-dS path's dK/dV units of dS in the workspace (ds_slots_for).  `seg`: segment-mode
 // dimensions (chunk-wise attention; split path only), or null for S2
 // attention of (B, H, Hkv, N, D, G).  Segment mode with causal = 0 computes dq
 // only (dk = dv = null: a detached key segment); dq_accumulate adds the
 // result to dq.
-int bwd_impl(int path, int stages, const void* q, const void* k, const void* v, const void* o, const float* lse,
+int bwd_impl(int path, int stages, int ds_slots, const void* q, const void* k, const void* v, const void* o, const float* lse,
              const void* dO, void* dq, void* dk, void* dv, int B, int H, int Hkv, int N, int D, int G,
              void* workspace, size_t workspace_bytes, s2attn_stream_t stream, const float* rope = nullptr,
              const Dims* seg = nullptr, int dq_accumulate = 0, HgaList hist = HgaList()) {
@@ -563,7 +583,9 @@ int bwd_impl(int path, int stages, const void* q, const void* k, const void* v, 
     return S2ATTN_ERR_MISALIGNED;
   // segment and HGA modes take the split path (the dQ kernel walks their extra keys)
   if (seg != nullptr && path == kBwdSplitDs) path = kBwdSplit;
-  const size_t need = workspace_bytes_for(path, B, H, N, D, G);
+  if (path == kBwdSplitDs && ds_slots < 2 && ds_slots < B * Hkv * (N / G)) path = kBwdSplit;
+  const long long ds_blocks = path == kBwdSplitDs ? ds_slots * ds_unit_blocks(H, Hkv, G) : 0;
+  const size_t need = workspace_bytes_for(path, B, H, N, D, ds_blocks);
   if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return S2ATTN_ERR_WORKSPACE;
   DeviceInfo info;
@@ -586,7 +608,6 @@ int bwd_impl(int path, int stages, const void* q, const void* k, const void* v, 
   __nv_bfloat16* ds = path == kBwdSplitDs
                           ? reinterpret_cast<__nv_bfloat16*>(ws + kStatusBytes + 2 * rowstat_bytes(B, H, N))
                           : nullptr;
-  const long long ds_blocks = path == kBwdSplitDs ? ds_blocks_for(B, H, N, G) : 0;
   if (ds != nullptr &&
       (!make_map_2d(&maps.ds, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ds, 32, static_cast<uint64_t>(ds_blocks) * 4 * kTile,
                     64, 32, 2 * kTile, CU_TENSOR_MAP_SWIZZLE_64B) ||
@@ -620,6 +641,7 @@ int bwd_impl(int path, int stages, const void* q, const void* k, const void* v, 
   a.rope = path == kBwdFused ? rope : nullptr;
   a.ds = ds;
   a.ds_tt = (G / kTile) * (G / kTile + 1) / 2;
+  a.ds_slots = ds_slots;
   a.ds_blocks = ds_blocks;
   a.status = status;
   a.wait_limit_ns = wait_limit_ns();
@@ -653,7 +675,7 @@ int s2attn_bwd(const void* q, const void* k, const void* v, const void* o, const
                const void* dO, void* dq, void* dk, void* dv, int B, int H, int Hkv, int N, int D,
                int G, void* workspace, size_t workspace_bytes, s2attn_stream_t stream) {
   const Plan plan = select_plan(B, H, Hkv, N, D, G, 0);
-  return bwd_impl(plan.bwd_path, plan.bwd_stages, q, k, v, o, lse, dO, dq, dk, dv, B, H, Hkv, N, D, G,
+  return bwd_impl(plan.bwd_path, plan.bwd_stages, plan.ds_slots, q, k, v, o, lse, dO, dq, dk, dv, B, H, Hkv, N, D, G,
                   workspace, workspace_bytes, stream);
 }
 
@@ -720,13 +742,13 @@ int s2attn_bwd_rope(const void* q_rot, const void* k_rot, const void* v, const v
   if (!table) return S2ATTN_ERR_INVALID_ARG;
   if (!aligned16(table)) return S2ATTN_ERR_MISALIGNED;
   const Plan plan = select_plan(B, H, Hkv, N, D, G, 0);
-  return bwd_impl(plan.bwd_path, plan.bwd_stages, q_rot, k_rot, v, o, lse, dO, dq, dk, dv, B, H, Hkv, N, D, G,
+  return bwd_impl(plan.bwd_path, plan.bwd_stages, plan.ds_slots, q_rot, k_rot, v, o, lse, dO, dq, dk, dv, B, H, Hkv, N, D, G,
                   workspace, workspace_bytes, stream, table);
 }
 
 size_t s2attn_seg_bwd_workspace_bytes(int B, int H, int Hkv, int N, int Nk, int D) {
   if (validate_segment(B, H, Hkv, N, Nk, D, 0) != S2ATTN_OK) return 0;
-  return workspace_bytes_for(kBwdSplit, B, H, N, D, N);
+  return workspace_bytes_for(kBwdSplit, B, H, N, D);
 }
 
 int s2attn_seg_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
@@ -737,7 +759,7 @@ int s2attn_seg_bwd(const void* q, const void* k, const void* v, const void* o, c
   if (st != S2ATTN_OK) return st;
   const Dims d = make_segment_dims(B, H, Hkv, N, Nk, D, causal);
   const Plan plan = select_plan(B, H, Hkv, N, D, N, 0);
-  return bwd_impl(kBwdSplit, plan.bwd_stages, q, k, v, o, lse, dO, dq, dk, dv, B, H, Hkv, N, D, N, workspace,
+  return bwd_impl(kBwdSplit, plan.bwd_stages, 0, q, k, v, o, lse, dO, dq, dk, dv, B, H, Hkv, N, D, N, workspace,
                   workspace_bytes, stream, nullptr, &d, dq_accumulate);
 }
 
@@ -791,7 +813,7 @@ int s2attn_hga_bwd(const void* q, const void* k, const void* v, const void* o, c
   hl.tiles = hist;
   hl.S = S;
   const Plan plan = select_plan(B, H, Hkv, N, D, G, 0);
-  return bwd_impl(kBwdSplit, plan.bwd_stages, q, k, v, o, lse, dO, dq, dk, dv, B, H, Hkv, N, D, G, workspace,
+  return bwd_impl(kBwdSplit, plan.bwd_stages, 0, q, k, v, o, lse, dO, dq, dk, dv, B, H, Hkv, N, D, G, workspace,
                   workspace_bytes, stream, nullptr, &d, 0, hl);
 }
 
@@ -945,7 +967,7 @@ int s2attn_nf4_qkv(const void* x, const void* codes, const int8_t* scale_codes, 
 
 size_t s2attn_hga_bwd_workspace_bytes(int B, int H, int Hkv, int N, int D, int G) {
   if (validate_shape(B, H, Hkv, N, D, G, false) != S2ATTN_OK || G % kQBlock != 0) return 0;
-  return workspace_bytes_for(kBwdSplit, B, H, N, D, G);
+  return workspace_bytes_for(kBwdSplit, B, H, N, D);
 }
 
 int s2attn_plan(int B, int H, int Hkv, int N, int D, int G, int num_sms, int* out) {
@@ -958,6 +980,7 @@ int s2attn_plan(int B, int H, int Hkv, int N, int D, int G, int num_sms, int* ou
   out[2] = p.bwd_path;
   out[3] = p.bwd_stages;
   out[4] = p.fwd_bn;
+  out[5] = p.bwd_path == kBwdSplitDs ? p.ds_slots : 0;
   return S2ATTN_OK;
 }
 
@@ -1079,12 +1102,12 @@ extern "C" int s2attn_bwd_noalloc(const void* q, const void* k, const void* v, c
   // with B * H * N only, where the fused path would need a dQ accumulator of
   // B * H * N * D floats
   const bool valid = validate_shape(B, H, Hkv, N, D, G) == S2ATTN_OK;
-  const size_t need = valid ? workspace_bytes_for(kBwdSplit, B, H, N, D, G) : 0;
+  const size_t need = valid ? workspace_bytes_for(kBwdSplit, B, H, N, D) : 0;
   if (need > kNoAllocScratchBytes) return S2ATTN_ERR_WORKSPACE;
   void* scratch = nullptr;
   // an invalid shape: bwd_impl reports which error
   if (valid && !noalloc_scratch(&scratch)) return S2ATTN_ERR_CUDA;
   const Plan plan = select_plan(B, H, Hkv, N, D, G, 0);
-  return bwd_impl(kBwdSplit, plan.bwd_stages, q, k, v, o, lse, dO, dq, dk, dv, B, H, Hkv, N, D, G, scratch,
+  return bwd_impl(kBwdSplit, plan.bwd_stages, 0, q, k, v, o, lse, dO, dq, dk, dv, B, H, Hkv, N, D, G, scratch,
                   kNoAllocScratchBytes, stream);
 }

@@ -97,12 +97,21 @@ def test_workspace_bytes():
     assert _lib.s2attn_bwd_workspace_bytes(1, 32, 32, 8192, 128, 2048) == 256 + 2 * 32 * 8192 * 4 + ds
     assert _lib.s2attn_bwd_workspace_bytes(1, 1, 1, 128, 64, 128) == 256 + 2 * 512 + 128 * 128 * 2
     assert _lib.s2attn_bwd_workspace_bytes(1, 4, 3, 1024, 64, 256) == 0  # invalid shape
-    # LLaMA2-70B at 32K tokens: 17 GB of dS blocks, over the budget: the split path
-    assert _lib.s2attn_bwd_workspace_bytes(1, 64, 8, 32768, 128, 8192) == 256 + 2 * 64 * 32768 * 4
+    # LLaMA2-70B at 32K tokens: 17 GB of dS blocks in all, over the budget: the
+    # workspace holds the dS of 7 (batch, kv head, group) units of 8 query heads
+    # each (545 MB a unit), the backward running in ranges
+    unit = 8 * (64 * 65 // 2) * 128 * 128 * 2
+    assert _lib.s2attn_bwd_workspace_bytes(1, 64, 8, 32768, 128, 8192) == 256 + 2 * 64 * 32768 * 4 + 7 * unit
+    # 100K tokens, 32 heads: 6 units of 643 MB
+    unit = (200 * 201 // 2) * 128 * 128 * 2
+    assert _lib.s2attn_bwd_workspace_bytes(1, 32, 32, 102400, 128, 25600) == 256 + 2 * 32 * 102400 * 4 + 6 * unit
     # the split path, forced through the override, needs no accumulator
     try:
         _lib.s2attn_set_tile_override("bwd=split")
         assert _lib.s2attn_bwd_workspace_bytes(1, 32, 32, 8192, 128, 2048) == 256 + 2 * 32 * 8192 * 4
+        _lib.s2attn_set_tile_override("ds_slots=3")  # dS of 3 of the 128 units
+        assert _lib.s2attn_bwd_workspace_bytes(1, 32, 32, 8192, 128, 2048) == \
+            256 + 2 * 32 * 8192 * 4 + 3 * (16 * 17 // 2) * 128 * 128 * 2
         _lib.s2attn_set_tile_override("fwd_order=pairs,bwd=fused")
         assert _lib.s2attn_bwd_workspace_bytes(1, 32, 32, 8192, 128, 2048) == 256 + 2 * 32 * 8192 * 4 + 32 * 8192 * 128 * 4
     finally:
@@ -123,21 +132,26 @@ def test_profile_api_host_side():
 
 
 def test_plan_selection_table():
-    """The per-shape plan (host logic, no GPU): the split-dS backward while its
-    dS blocks fit 4 GiB, else the split backward; the forward's work order
-    following the K/V size; the selected depths."""
+    """The per-shape plan (host logic, no GPU): the split-dS backward, its
+    workspace holding every unit's dS blocks while they fit 4 GiB and as many
+    units as fit beyond that; the forward's work order following the K/V size;
+    the selected depths."""
     from sparse_attention_attn_b200 import inputs as I
     expect = {
-        "tiny": ("snake", 8, "split_ds", 3),
-        "llama2-7b-n8192": ("snake", 4, "split_ds", 3),
-        "qwen3-8b-gqa-n16384": ("snake", 4, "split_ds", 3),
-        "llama2-70b-gqa-n32768": ("snake", 4, "split", 3),
-        "llama2-7b-n102400": ("pairs", 4, "split", 3),
+        "tiny": ("snake", 8, "split_ds", 3, 16),
+        "llama2-7b-n8192": ("snake", 4, "split_ds", 3, 128),
+        "qwen3-8b-gqa-n16384": ("snake", 4, "split_ds", 3, 32),
+        "llama2-70b-gqa-n32768": ("snake", 4, "split_ds", 3, 7),
+        "llama2-7b-n102400": ("pairs", 4, "split_ds", 3, 6),
     }
     for s in I.WORKLOADS:
         p = _lib.s2attn_plan(s.B, s.H, s.Hkv, s.N, s.D, s.G, 148)
-        assert (p["fwd_order"], p["fwd_kv_slots"], p["bwd_path"], p["bwd_stages"]) == expect[s.name], s.name
+        got = (p["fwd_order"], p["fwd_kv_slots"], p["bwd_path"], p["bwd_stages"], p["ds_slots"])
+        assert got == expect[s.name], s.name
         assert p["fwd_bn"] == 128
+    # a unit whose dS alone passes half the budget leaves no room for two: the split path
+    p = _lib.s2attn_plan(1, 64, 1, 65536, 128, 65536, 148)
+    assert (p["bwd_path"], p["ds_slots"]) == ("split", 0)
     with pytest.raises(_lib.S2AttnError):
         _lib.s2attn_plan(1, 4, 3, 1024, 64, 256, 148)
 
@@ -148,14 +162,24 @@ def test_plan_override_parsing():
     try:
         _lib.s2attn_set_tile_override("fwd_order=pairs,fwd_kv=2,bwd=split,bwd_stages=2")
         p = _lib.s2attn_plan(1, 32, 32, 8192, 128, 2048, 148)   # a 2-slot K/V ring does not exist
-        assert p == {"fwd_order": "pairs", "fwd_bn": 128, "fwd_kv_slots": 4, "bwd_path": "split", "bwd_stages": 2}
+        assert p == {"fwd_order": "pairs", "fwd_bn": 128, "fwd_kv_slots": 4, "bwd_path": "split", "bwd_stages": 2,
+                     "ds_slots": 0}
         p = _lib.s2attn_plan(1, 4, 4, 1024, 64, 256, 148)   # head dim 64: kv 2 and stages 2 do not exist
-        assert p == {"fwd_order": "pairs", "fwd_bn": 128, "fwd_kv_slots": 8, "bwd_path": "split", "bwd_stages": 3}
+        assert p == {"fwd_order": "pairs", "fwd_bn": 128, "fwd_kv_slots": 8, "bwd_path": "split", "bwd_stages": 3,
+                     "ds_slots": 0}
         _lib.s2attn_set_tile_override("bwd=fused,fwd_kv=6,bwd_stages=4,junk,=,x=y")  # no fused path at D = 64
         assert _lib.s2attn_plan(1, 4, 4, 1024, 64, 256, 148) == \
-            {"fwd_order": "snake", "fwd_bn": 128, "fwd_kv_slots": 6, "bwd_path": "split_ds", "bwd_stages": 4}
+            {"fwd_order": "snake", "fwd_bn": 128, "fwd_kv_slots": 6, "bwd_path": "split_ds", "bwd_stages": 4,
+             "ds_slots": 16}
         assert _lib.s2attn_plan(1, 32, 32, 8192, 128, 2048, 148) == \
-            {"fwd_order": "snake", "fwd_bn": 128, "fwd_kv_slots": 4, "bwd_path": "fused", "bwd_stages": 3}
+            {"fwd_order": "snake", "fwd_bn": 128, "fwd_kv_slots": 4, "bwd_path": "fused", "bwd_stages": 3,
+             "ds_slots": 0}
+        _lib.s2attn_set_tile_override("ds_slots=2")
+        assert _lib.s2attn_plan(1, 32, 32, 8192, 128, 2048, 148)["ds_slots"] == 2
+        _lib.s2attn_set_tile_override("ds_slots=1000,bwd_stages=2")  # more slots than units: every unit
+        assert _lib.s2attn_plan(1, 32, 32, 8192, 128, 2048, 148)["ds_slots"] == 128
+        _lib.s2attn_set_tile_override("ds_slots=1")  # fewer than 2 slots do not exist
+        assert _lib.s2attn_plan(1, 64, 8, 32768, 128, 8192, 148)["ds_slots"] == 7
         _lib.s2attn_set_tile_override("fwd_bn=64,fwd_kv=4")  # 4 slots do not exist for 64-key tiles
         assert _lib.s2attn_plan(1, 32, 32, 8192, 128, 2048, 148)["fwd_bn"] == 64
         assert _lib.s2attn_plan(1, 32, 32, 8192, 128, 2048, 148)["fwd_kv_slots"] == 8
@@ -163,12 +187,14 @@ def test_plan_override_parsing():
         _lib.s2attn_set_tile_override("fwd_bn=64,fwd_kv=12")
         assert _lib.s2attn_plan(1, 4, 4, 1024, 64, 256, 148)["fwd_kv_slots"] == 12
         assert _lib.s2attn_plan(1, 32, 32, 8192, 128, 2048, 148)["fwd_kv_slots"] == 8
-        _lib.s2attn_set_tile_override("bwd=split_ds")  # forced even over the budget
-        assert _lib.s2attn_plan(1, 64, 8, 32768, 128, 8192, 148)["bwd_path"] == "split_ds"
+        _lib.s2attn_set_tile_override("bwd=split_ds")  # forced where not even 2 units fit: 2 slots
+        assert _lib.s2attn_plan(1, 64, 1, 65536, 128, 65536, 148)["bwd_path"] == "split_ds"
+        assert _lib.s2attn_plan(1, 64, 1, 65536, 128, 65536, 148)["ds_slots"] == 1  # one unit: all of them
+        assert _lib.s2attn_plan(2, 64, 1, 65536, 128, 65536, 148)["ds_slots"] == 2
     finally:
         _lib.s2attn_set_tile_override(None)
     assert _lib.s2attn_plan(1, 32, 32, 8192, 128, 2048, 148)["bwd_path"] == "split_ds"
-    assert _lib.s2attn_plan(1, 64, 8, 32768, 128, 8192, 148)["bwd_path"] == "split"
+    assert _lib.s2attn_plan(1, 64, 8, 32768, 128, 8192, 148)["ds_slots"] == 7
 
 
 def test_nf4_levels_and_argument_checks_on_the_host():

@@ -80,12 +80,44 @@ def test_small_whole_tensor(B, N, H, Hkv, D, G, bwd_path):
     check_grad("dV", to64(dv), dv_ref)
 
 
+# the split-dS backward with its dS workspace holding fewer (batch, kv head,
+# group) units than there are: dK/dV in ranges of pairs (ranges that end inside
+# a unit included), each followed by dQ for the units it completed, the slots
+# reused from range to range
+DS_RANGES = [
+    ((2, 512, 4, 2, 128, 256), 2),    # 2 tiles a group: one pair a unit, 8 units
+    ((1, 1024, 8, 4, 128, 512), 3),   # 4 tiles, 2 pairs a unit
+    ((2, 1536, 4, 4, 64, 768), 2),    # 6 tiles, 3 pairs a unit: ranges of 4 pairs end inside units
+    ((1, 640, 2, 2, 64, 640), 2),     # 5 tiles: the middle pair has one item
+    ((1, 768, 6, 2, 64, 256), 4),     # three query heads per kv head
+]
+
+
+@pytest.mark.parametrize("shape,slots", DS_RANGES, ids=[f"{s}-slots{n}" for s, n in DS_RANGES])
+def test_small_split_ds_ranges(shape, slots):
+    from sparse_attention_attn_b200 import _lib
+    B, N, H, Hkv, D, G = shape
+    _lib.s2attn_set_tile_override(f"bwd=split_ds,ds_slots={slots}")
+    try:
+        assert _lib.s2attn_plan(B, H, Hkv, N, D, G, 148)["ds_slots"] == slots
+        (q, k, v, do), (o, lse, dq, dk, dv) = _run(I.Shape("small", B, H, Hkv, D, N, G), seed_offset=11)
+    finally:
+        _lib.s2attn_set_tile_override(None)
+    q64, k64, v64, do64 = (to64(t) for t in (q, k, v, do))
+    dq_ref, dk_ref, dv_ref, _ = ref.s2_attention_bwd(q64, k64, v64, do64, G)
+    tag = f" [ds_slots={slots}]"
+    check_grad("dQ", to64(dq), dq_ref, tag)
+    check_grad("dK", to64(dk), dk_ref, tag)
+    check_grad("dV", to64(dv), dv_ref, tag)
+
+
 PLAN_VARIANTS = [
     # every variant the per-shape plan can select, forced through the override
     (128, "fwd_order=pairs"), (128, "bwd=split,bwd_stages=2"), (128, "bwd=split,bwd_stages=3"),
     (128, "bwd=split_ds,bwd_stages=2"), (128, "bwd=fused"), (64, "fwd_order=pairs"), (64, "fwd_kv=4"),
     (64, "fwd_kv=6"), (64, "bwd=split,bwd_stages=4"), (64, "bwd=split_ds,bwd_stages=4"),
     (128, "fwd_bn=64"), (128, "fwd_bn=64,fwd_order=pairs"), (64, "fwd_bn=64"), (64, "fwd_bn=64,fwd_kv=12"),
+    (128, "bwd=split_ds,ds_slots=2"), (128, "bwd=split_ds,ds_slots=3"), (64, "bwd=split_ds,ds_slots=2"),
 ]
 
 
@@ -242,6 +274,13 @@ def test_launch_counts():
     assert _lib.s2attn_last_launch_count() == 1
     s2.s2attn_backward(q, k, v, o, lse, do, shape.G)
     assert _lib.s2attn_last_launch_count() == 3
+    # dS of 2 of the 4 units at once: two ranges of 2 pairs, each dK/dV + dQ
+    _lib.s2attn_set_tile_override("ds_slots=2")
+    try:
+        s2.s2attn_backward(q, k, v, o, lse, do, shape.G)
+        assert _lib.s2attn_last_launch_count() == 5
+    finally:
+        _lib.s2attn_set_tile_override(None)
 
 
 def test_bounded_wait_times_out_cleanly():
