@@ -396,10 +396,14 @@ __global__ void __launch_bounds__(320, 1)
           }
           // P (bf16) over the first 64 columns of S, in two halves so the
           // issuer can start P V on keys 0..63 while keys 64..127 are being
-          // computed; every S column of this thread's row was read above
-          uint32_t pk[32];
-          float rs = softmax_row64(sr[0], sr[1], sl2, m_run, pk);
-          tmem_st32(tS, pk);
+          // computed; every S column of this thread's row was read above.
+          // Each half goes out in two 16-column pieces, which keeps the
+          // softmax within the register budget (no spills)
+          uint32_t pk[16];
+          float rs = softmax_row32(sr[0], sl2, m_run, pk);
+          tmem_st16(tS, pk);
+          rs += softmax_row32(sr[1], sl2, m_run, pk);
+          tmem_st16(tS + 16, pk);
           if (__any_sync(0xffffffffu, resc)) {
             // rescale O (it holds P_{j-1} V_{j-1} once that UMMA has completed)
             // before P_j V_j accumulates onto it
@@ -421,8 +425,10 @@ __global__ void __launch_bounds__(320, 1)
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(smem_u32(&bar_plo[wg]));
-          rs += softmax_row64(sr[2], sr[3], sl2, m_run, pk);
-          tmem_st32(tS + 32, pk);
+          rs += softmax_row32(sr[2], sl2, m_run, pk);
+          tmem_st16(tS + 32, pk);
+          rs += softmax_row32(sr[3], sl2, m_run, pk);
+          tmem_st16(tS + 48, pk);
           l_run = l_run * alpha + rs;
           tmem_wait_st();
           tc_fence_before();

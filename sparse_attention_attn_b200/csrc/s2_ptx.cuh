@@ -453,6 +453,23 @@ __device__ __forceinline__ float softmax_row64(const uint32_t (&s0)[32], const u
   return f2_lo(s) + f2_hi(s);
 }
 
+// The same for 32 keys (one 32-column TMEM load): 16 packed pairs.  The
+// forward writes P in 16-column pieces so that no more than 16 packed values
+// are live beside the 128 scores of a row.
+__device__ __forceinline__ float softmax_row32(const uint32_t (&s0)[32], float sl2, float m, uint32_t (&pk)[16]) {
+  const uint64_t sc2 = f2_pack(sl2, sl2), nm2 = f2_pack(-m, -m);
+  uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+  for (int c = 0; c < 16; ++c) {
+    const uint64_t x = f2_fma(f2_pack(__uint_as_float(s0[2 * c]), __uint_as_float(s0[2 * c + 1])), sc2, nm2);
+    const uint64_t p = f2_pack(ex2_approx(f2_lo(x)), ex2_approx(f2_hi(x)));
+    pk[c] = f2_to_bf16x2(p);
+    acc[c & 3] = f2_add(acc[c & 3], p);
+  }
+  const uint64_t s = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
+  return f2_lo(s) + f2_hi(s);
+}
+
 // Explicit shared-memory vector load (a pointer into dynamic shared memory
 // that went through integer alignment arithmetic is generic to the compiler,
 // and generic loads take the long-latency path).
