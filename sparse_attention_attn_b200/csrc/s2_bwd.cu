@@ -119,11 +119,14 @@ __global__ void __launch_bounds__(256) s2_bwd_pre_kernel(const BwdPreArgs a) {
 // S^T and dP^T (128 kv rows x 64 query columns each) are double-buffered in
 // TMEM, so the UMMAs of sub-tile g+1 run while warps 2..9 turn sub-tile g into
 // P^T and dS^T; the buffers, the Q/dO stages and their barriers run on one
-// sub-tile counter across items.  K/V tiles are double-buffered across items,
-// so the next item's K/V load overlaps the current item.  TMEM: S^T [0,128)
-// (two 64-column buffers), dP^T [128,256), dV [256, 256+D), dK [256+D, 256+2D);
-// dV/dK are read out by the epilogue of an item before the next item's first
-// gradient UMMA overwrites them (acc_full / acc_free handshake).
+// sub-tile counter across items.  One K/V buffer: it is released once the
+// item's last S^T and dP^T have completed, and the next item's K/V load runs
+// under that item's last gradient UMMAs and its epilogue (the issuers issue
+// an item's last dV/dK before they wait for the next item's K/V; measured as
+// fast as a second K/V buffer).  TMEM: S^T [0,128) (two 64-column buffers), dP^T
+// [128,256), dV [256, 256+D), dK [256+D, 256+2D); dV/dK are read out by the
+// epilogue of an item before the next item's first gradient UMMA overwrites
+// them (acc_full / acc_free handshake).
 
 // A-operand column of k-step kk (16 rows of K) when a 64-wide bf16 operand was
 // written by two warp halves at packed columns [0,16) and [32,48) of its
@@ -138,11 +141,12 @@ struct DkvCfg {
   static constexpr int Q_ATOM = kSub * 128;    // one 64-column slab of a 64-row tile
   static constexpr int KV_BYTES = kTile * D * 2;
   static constexpr int Q_BYTES = kSub * D * 2;
-  static constexpr int OFF_KV = 0;  // [2 buffers][K, V]
-  static constexpr int OFF_Q = 4 * KV_BYTES;
+  static constexpr int OFF_KV = 0;  // [K, V] of the current item
+  static constexpr int OFF_Q = 2 * KV_BYTES;
   static constexpr int OFF_DO = OFF_Q + STAGES * Q_BYTES;
   static constexpr int OFF_ROW = OFF_DO + STAGES * Q_BYTES;  // per stage: -lse2[64], -delta[64]
   static constexpr int SMEM_BYTES = OFF_ROW + STAGES * 512 + 1024;
+  static_assert(SMEM_BYTES <= 232448 - 512, "shared memory");
   static constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DV = 256, TM_DK = 256 + D;
   static constexpr int THREADS = 352;
 };
@@ -159,7 +163,7 @@ __global__ void __launch_bounds__(352, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   // bar_s / bar_dp: S^T / dP^T of a sub-tile landed (issuers A / B);
   // empty, kv_empty, acc_full complete once both issuers committed.
-  __shared__ __align__(8) uint64_t bar_kv[2], bar_kv_empty[2], bar_full[ST], bar_empty[ST], bar_s[2],
+  __shared__ __align__(8) uint64_t bar_kv, bar_kv_empty, bar_full[ST], bar_empty[ST], bar_s[2],
       bar_dp[2], bar_pds[2], bar_acc_full, bar_acc_free, bar_drain[2];
   __shared__ uint32_t tmem_slot;
   __shared__ uint32_t abort_flag;
@@ -170,17 +174,16 @@ __global__ void __launch_bounds__(352, 1)
   WaitCtx wc{&abort_flag, a.status, a.wait_limit_ns};
 
   const uint32_t s0 = smem_u32(smem);
-  auto sK = [&](int kb) { return s0 + C::OFF_KV + kb * 2 * C::KV_BYTES; };
-  auto sV = [&](int kb) { return s0 + C::OFF_KV + kb * 2 * C::KV_BYTES + C::KV_BYTES; };
+  const uint32_t sK = s0 + C::OFF_KV, sV = s0 + C::OFF_KV + C::KV_BYTES;
   auto sQ = [&](int s) { return s0 + C::OFF_Q + s * C::Q_BYTES; };
   auto sG = [&](int s) { return s0 + C::OFF_DO + s * C::Q_BYTES; };
   auto sRow = [&](int s) { return s0 + C::OFF_ROW + s * 512; };
 
   if (threadIdx.x == 0) {
     abort_flag = 0;
+    mbar_init(smem_u32(&bar_kv), 1);
+    mbar_init(smem_u32(&bar_kv_empty), 2);  // the last S^T and dP^T of an item (one commit per issuer)
     for (int i = 0; i < 2; ++i) {
-      mbar_init(smem_u32(&bar_kv[i]), 1);
-      mbar_init(smem_u32(&bar_kv_empty[i]), 2);
       mbar_init(smem_u32(&bar_s[i]), 1);
       mbar_init(smem_u32(&bar_dp[i]), 1);
       mbar_init(smem_u32(&bar_pds[i]), 8);  // one elected arrival per elementwise warp
@@ -219,16 +222,15 @@ __global__ void __launch_bounds__(352, 1)
     for (ic.first(ps); ok && ic.valid; ic.next(ps)) {
       const TileWork w = kv_item(d, ic.unit, ic.tile);
       const int sh = shift_of_head(d, w.h);
-      const int kb = ic.n & 1;
-      if (ic.n >= 2 && !warp_wait(smem_u32(&bar_kv_empty[kb]), ((ic.n >> 1) - 1) & 1, wc, 109)) break;
+      if (ic.n >= 1 && !warp_wait(smem_u32(&bar_kv_empty), (ic.n - 1) & 1, wc, 109)) break;
       // the kv tiles of this kernel are the query segment's own keys, which sit
       // at key rows qoff_t*128 onwards (0 for S2 attention)
       const int tk0 = original_row_kv(d, d.qoff_t * kTile + w.g * d.G + w.tile * kTile, sh);
       if (elect_one()) {
-        mbar_arrive_expect_tx(smem_u32(&bar_kv[kb]), 2 * C::KV_BYTES);
+        mbar_arrive_expect_tx(smem_u32(&bar_kv), 2 * C::KV_BYTES);
         for (int c = 0; c < D / 64; ++c) {
-          tma_load_4d(sK(kb) + c * C::KV_ATOM, &tmK, smem_u32(&bar_kv[kb]), c * 64, w.kvh, tk0, w.b);
-          tma_load_4d(sV(kb) + c * C::KV_ATOM, &tmV, smem_u32(&bar_kv[kb]), c * 64, w.kvh, tk0, w.b);
+          tma_load_4d(sK + c * C::KV_ATOM, &tmK, smem_u32(&bar_kv), c * 64, w.kvh, tk0, w.b);
+          tma_load_4d(sV + c * C::KV_ATOM, &tmV, smem_u32(&bar_kv), c * 64, w.kvh, tk0, w.b);
         }
       }
       __syncwarp();
@@ -260,9 +262,8 @@ __global__ void __launch_bounds__(352, 1)
     }
     if (*wc.abort && lane == 0) {
       // never leave copies in flight into shared memory: wait (bounded) for
-      // the last fill of every stage and K/V buffer
-      for (int kb = 0; kb < 2 && kb < kv_issued; ++kb)
-        drain_wait(smem_u32(&bar_kv[kb]), ((kv_issued - 1 - kb) >> 1) & 1);
+      // the last fill of every stage and of the K/V buffer
+      if (kv_issued > 0) drain_wait(smem_u32(&bar_kv), (kv_issued - 1) & 1);
       for (int s = 0; s < ST && s < gi; ++s) drain_wait(smem_u32(&bar_full[s]), ((gi - 1 - s) / ST) & 1);
     }
   } else if (warp == 1 || warp == 10) {
@@ -276,31 +277,33 @@ __global__ void __launch_bounds__(352, 1)
     const uint32_t idS = make_idesc_bf16(128, kSub, 0, 0);  // S^T, dP^T
     const uint32_t idG = make_idesc_bf16(128, D, 0, 1);     // dV, dK
     // A: operand K / Q / dO, B: operand V / dO / Q
-    const uint64_t dX0 = make_sdesc_sw128(A ? sK(0) : sV(0), 16, 1024);          // K-major (A operand)
+    const uint64_t dX0 = make_sdesc_sw128(A ? sK : sV, 16, 1024);                // K-major (A operand)
     const uint64_t dYk = make_sdesc_sw128(A ? sQ(0) : sG(0), 16, 1024);          // K-major (B of S^T / dP^T)
     const uint64_t dZm = make_sdesc_sw128(A ? sG(0) : sQ(0), C::Q_ATOM, 1024);   // MN-major (B of dV / dK)
     const uint32_t tm_sp = tmem + (A ? C::TM_S : C::TM_DP);
     const uint32_t tm_acc = tmem + (A ? C::TM_DV : C::TM_DK);
     const uint32_t bar_ready = smem_u32(A ? &bar_s[0] : &bar_dp[0]);
-    auto issue_sp = [&](int g, int kb) {
+    // S^T / dP^T of sub-tile g (cursor c); after an item's last one, the K/V
+    // buffer goes back to the producer once those UMMAs have completed
+    auto issue_sp = [&](int g, const DkvCursor& c) {
       const int s = g % ST;
       const uint32_t bo = (g & 1) * kSub;
-      const uint64_t dx = sdesc_advance(dX0, kb * 2 * C::KV_BYTES);
       const uint64_t dy = sdesc_advance(dYk, s * C::Q_BYTES);
       if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ko = (kk >> 2) * C::KV_ATOM + (kk & 3) * 32;
           const uint32_t qo = (kk >> 2) * C::Q_ATOM + (kk & 3) * 32;
-          umma_ss(tm_sp + bo, sdesc_advance(dx, ko), sdesc_advance(dy, qo), idS, kk > 0);
+          umma_ss(tm_sp + bo, sdesc_advance(dX0, ko), sdesc_advance(dy, qo), idS, kk > 0);
         }
         umma_commit(bar_ready + (g & 1) * 8);
+        if (c.it == c.iters - 1) umma_commit(smem_u32(&bar_kv_empty));
       }
       __syncwarp();
     };
     // make sub-tile g (cursor c) ready: its item's K/V and its Q/dO stage
     auto wait_inputs = [&](const DkvCursor& c, int g) -> bool {
-      if (c.it == 0 && !warp_wait(smem_u32(&bar_kv[c.ic.n & 1]), (c.ic.n >> 1) & 1, wc, 120)) return false;
+      if (c.it == 0 && !warp_wait(smem_u32(&bar_kv), c.ic.n & 1, wc, 120)) return false;
       if (!warp_wait(smem_u32(&bar_full[g % ST]), (g / ST) & 1, wc, 121)) return false;
       tc_fence_after();
       return true;
@@ -312,12 +315,17 @@ __global__ void __launch_bounds__(352, 1)
     bool ok = true;
     if (cur.ic.valid) {
       ok = wait_inputs(cur, 0);
-      if (ok) issue_sp(0, cur.ic.n & 1);
+      if (ok) issue_sp(0, cur);
     }
     for (int g = 0; ok && cur.ic.valid; ++g) {
-      if (nxt.ic.valid) {  // the next sub-tile (possibly the next item's first)
+      // the next sub-tile's S^T / dP^T (its TMEM buffer's last readers were
+      // issued before: in order), ahead of this sub-tile's gradients -- unless
+      // it opens the next item, whose K/V arrive only after this item's last
+      // S^T / dP^T: then after them, so the epilogue never waits for that load
+      const bool nxt_new = nxt.ic.valid && nxt.it == 0;
+      if (nxt.ic.valid && !nxt_new) {
         if (!wait_inputs(nxt, g + 1)) break;
-        issue_sp(g + 1, nxt.ic.n & 1);  // its TMEM buffer's last reader was issued before: in order
+        issue_sp(g + 1, nxt);
       }
       if (!warp_wait(smem_u32(&bar_pds[g & 1]), (g >> 1) & 1, wc, 123)) break;
       if (cur.it == 0 && cur.ic.n > 0 &&
@@ -334,12 +342,13 @@ __global__ void __launch_bounds__(352, 1)
           umma_ts(tm_acc, tm_sp + bo + split_acol64(kk), sdesc_advance(dz, kk * 2048), idG,
                   (cur.it > 0 || kk > 0));
         umma_commit(smem_u32(&bar_empty[s]));
-        if (last) {
-          umma_commit(smem_u32(&bar_acc_full));
-          umma_commit(smem_u32(&bar_kv_empty[cur.ic.n & 1]));
-        }
+        if (last) umma_commit(smem_u32(&bar_acc_full));
       }
       __syncwarp();
+      if (nxt_new) {
+        if (!wait_inputs(nxt, g + 1)) break;
+        issue_sp(g + 1, nxt);
+      }
       cur = nxt;
       nxt.next(d, ps);
     }
@@ -423,12 +432,14 @@ __global__ void __launch_bounds__(352, 1)
       if (a.ds != nullptr) {
         // split-dS path: these 32 dS^T values (kv row `row`, query columns
         // half * 32 + [0, 32) of sub-tile i64) also go to their dS block, in
-        // its 32-column slab 2 (i64 & 1) + half: the warp's 32 rows write
-        // 2 KB of consecutive bytes.  Issued after the arrival, so the dK
-        // UMMA never waits for them.
-        // the item's first block (query head kvh rep, tile 0, kv tile 0),
+        // its 32-column slab 2 (i64 & 1) + half, rows quarter * 32 + [0, 32):
+        // staged in this warp's 2 KB with the 64-byte swizzle the store's
+        // tensor map names (16-byte chunk c of row r at c ^ ((r >> 1) & 3),
+        // so the warp's writes are free of bank conflicts), then written by
+        // one TMA store.  After the arrival, so the dK UMMA never waits.
+        // The item's first block (query head kvh rep, tile 0, kv tile 0) is
         // formed once per item; then query head, query tile and kv tile as
-        // ds_block orders them
+        // ds_block orders them.
         if (cur.it == 0) ds_base = ds_block(d, cur.w.b, cur.w.h, cur.w.g, 0, 0, a.ds_tt, a.ds_slots);
         const int i64 = 2 * cur.w.tile + cur.it % cur.nq, i = i64 >> 1;
         const long long blk = ds_base + static_cast<long long>(cur.it / cur.nq) * a.ds_tt + i * (i + 1) / 2 + cur.w.tile;
@@ -940,14 +951,16 @@ template cudaError_t launch_bwd_pre<128>(const BwdPreArgs&, int, cudaStream_t);
 
 // Tensor maps: `*128` have 128-row boxes, `*64` 64-row boxes.  dK/dV streams
 // 64-row query sub-tiles against 128-row kv tiles; dQ the other way round.
-// NST: pipeline stages of both kernels' streamed operands.
+// NST: pipeline stages of the dK/dV kernel's streamed operands; the split
+// path's dQ kernel takes the same, at most 3 at head dim 128 (what fits).
 template <int D, int NST>
 cudaError_t launch_bwd_stages(const BwdMaps& m, const BwdPreArgs& pre, const BwdArgs& a, int num_sms,
                               cudaStream_t stream, int* launches) {
+  constexpr int QST = (D == 128 && NST > 3) ? 3 : NST;
   using K3 = DkvCfg<D, NST>;
-  using K4 = DqCfg<D, NST>;
+  using K4 = DqCfg<D, QST>;
   if (!set_smem_attr(reinterpret_cast<const void*>(s2_bwd_dkdv_kernel<D, NST>), K3::SMEM_BYTES) ||
-      !set_smem_attr(reinterpret_cast<const void*>(s2_bwd_dq_kernel<D, NST>), K4::SMEM_BYTES))
+      !set_smem_attr(reinterpret_cast<const void*>(s2_bwd_dq_kernel<D, QST>), K4::SMEM_BYTES))
     return cudaErrorInvalidValue;
   cudaError_t e = launch_bwd_pre<D>(pre, num_sms, stream);
   if (e != cudaSuccess) return e;
@@ -995,20 +1008,21 @@ cudaError_t launch_bwd_stages(const BwdMaps& m, const BwdPreArgs& pre, const Bwd
   if (launches) *launches = a.no_dkdv ? 2 : 3;
   const int grid_q = pair_grid(a.q_sched, num_sms);
   prof_before(stream, kKernelBwdDq);
-  s2_bwd_dq_kernel<D, NST><<<grid_q, K4::THREADS, K4::SMEM_BYTES, stream>>>(m.q128, m.k64, m.v64, m.g128, a);
+  s2_bwd_dq_kernel<D, QST><<<grid_q, K4::THREADS, K4::SMEM_BYTES, stream>>>(m.q128, m.k64, m.v64, m.g128, a);
   e = cudaGetLastError();
   prof_after(stream);
   return e;
 }
 
-// stages: 2 or 3 at head dim 128, 3 or 4 at head dim 64 (what fits in shared
-// memory); anything else is an invalid value.
+// stages: 2, 3 or 4 at head dim 128, 3 or 4 at head dim 64 (what fits in
+// shared memory); anything else is an invalid value.
 template <int D>
 cudaError_t launch_bwd(const BwdMaps& m, const BwdPreArgs& pre, const BwdArgs& a, int num_sms,
                        cudaStream_t stream, int* launches, int stages) {
   if constexpr (D == 128) {
     if (stages == 2) return launch_bwd_stages<D, 2>(m, pre, a, num_sms, stream, launches);
     if (stages == 3) return launch_bwd_stages<D, 3>(m, pre, a, num_sms, stream, launches);
+    if (stages == 4) return launch_bwd_stages<D, 4>(m, pre, a, num_sms, stream, launches);
     return cudaErrorInvalidValue;
   } else {
     if (stages == 3) return launch_bwd_stages<D, 3>(m, pre, a, num_sms, stream, launches);

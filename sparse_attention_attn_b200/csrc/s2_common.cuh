@@ -382,7 +382,7 @@ __host__ __device__ __forceinline__ int ds_chunk_pairs(const PairSched& kv, int 
 struct BwdMaps {
   CUtensorMap q128, k128, v128, g128;
   CUtensorMap q64, k64, v64, g64;
-  CUtensorMap ds, dq32;  // split-dS path: the dS blocks (2-D, 64 x 128 boxes), dq (32-row boxes)
+  CUtensorMap ds, dq32;  // split-dS path: the dS blocks (2-D, 32 x 256 boxes), dq (32-row boxes)
 };
 
 template <int D>

@@ -258,7 +258,7 @@ bool valid_kv_slots(int D, int bn, int v) {
   if (bn == 64) return D == 128 ? v == 8 : (v == 8 || v == 12);
   return D == 128 ? v == 4 : (v == 4 || v == 6 || v == 8);
 }
-bool valid_bwd_stages(int D, int v) { return D == 128 ? (v == 2 || v == 3) : (v == 3 || v == 4); }
+bool valid_bwd_stages(int D, int v) { return D == 128 ? (v >= 2 && v <= 4) : (v == 3 || v == 4); }
 
 Plan select_plan(int B, int H, int Hkv, int N, int D, int G, int sms) {
   (void)H;

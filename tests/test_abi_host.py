@@ -172,8 +172,11 @@ def test_plan_override_parsing():
             {"fwd_order": "snake", "fwd_bn": 128, "fwd_kv_slots": 6, "bwd_path": "split_ds", "bwd_stages": 4,
              "ds_slots": 16}
         assert _lib.s2attn_plan(1, 32, 32, 8192, 128, 2048, 148) == \
-            {"fwd_order": "snake", "fwd_bn": 128, "fwd_kv_slots": 4, "bwd_path": "fused", "bwd_stages": 3,
+            {"fwd_order": "snake", "fwd_bn": 128, "fwd_kv_slots": 4, "bwd_path": "fused", "bwd_stages": 4,
              "ds_slots": 0}
+        _lib.s2attn_set_tile_override("bwd_stages=5")  # 5 stages exist for neither head dim
+        assert _lib.s2attn_plan(1, 32, 32, 8192, 128, 2048, 148)["bwd_stages"] == 3
+        assert _lib.s2attn_plan(1, 4, 4, 1024, 64, 256, 148)["bwd_stages"] == 3
         _lib.s2attn_set_tile_override("ds_slots=2")
         assert _lib.s2attn_plan(1, 32, 32, 8192, 128, 2048, 148)["ds_slots"] == 2
         _lib.s2attn_set_tile_override("ds_slots=1000,bwd_stages=2")  # more slots than units: every unit
