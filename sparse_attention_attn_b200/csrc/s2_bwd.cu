@@ -432,14 +432,11 @@ __global__ void __launch_bounds__(352, 1)
       if (a.ds != nullptr) {
         // split-dS path: these 32 dS^T values (kv row `row`, query columns
         // half * 32 + [0, 32) of sub-tile i64) also go to their dS block, in
-        // its 32-column slab 2 (i64 & 1) + half, rows quarter * 32 + [0, 32):
-        // staged in this warp's 2 KB with the 64-byte swizzle the store's
-        // tensor map names (16-byte chunk c of row r at c ^ ((r >> 1) & 3),
-        // so the warp's writes are free of bank conflicts), then written by
-        // one TMA store.  After the arrival, so the dK UMMA never waits.
-        // The item's first block (query head kvh rep, tile 0, kv tile 0) is
-        // formed once per item; then query head, query tile and kv tile as
-        // ds_block orders them.
+        // its 32-column slab 2 (i64 & 1) + half: the warp's 32 rows write
+        // 2 KB of consecutive bytes.  Issued after the arrival, so the dK
+        // UMMA never waits for them.  The item's first block (query head
+        // kvh rep, tile 0, kv tile 0) is formed once per item; then query
+        // head, query tile and kv tile as ds_block orders them.
         if (cur.it == 0) ds_base = ds_block(d, cur.w.b, cur.w.h, cur.w.g, 0, 0, a.ds_tt, a.ds_slots);
         const int i64 = 2 * cur.w.tile + cur.it % cur.nq, i = i64 >> 1;
         const long long blk = ds_base + static_cast<long long>(cur.it / cur.nq) * a.ds_tt + i * (i + 1) / 2 + cur.w.tile;
