@@ -265,6 +265,32 @@ def test_dense_100k_sampled():
     _check_full_size(I.LLAMA2_7B_100K.dense(), m=512, units=[(0, 0, 0)])
 
 
+@pytest.mark.parametrize("shape", [I.Shape("agree", 2, 4, 2, 128, 2048, 512), I.Shape("agree64", 1, 6, 2, 64, 1536, 768),
+                                   I.LLAMA2_7B_8K], ids=lambda s: s.name)
+def test_backward_paths_agree_bitwise(shape):
+    """The split backward (dQ recomputes S, P and dS), the split-dS backward
+    (dQ from the dS the dK/dV kernel stored) and the split-dS backward in ranges
+    (two units of dS at a time) form every dS value with the same fp32 steps
+    and bf16 rounding and accumulate dQ over the kv tiles in the same order:
+    their gradients agree bit for bit."""
+    import sparse_attention_attn_b200 as s2
+    from sparse_attention_attn_b200 import _lib
+    q, k, v, do = (t.cuda() for t in I.make_inputs(shape, 5))
+    o, lse = s2.s2attn_forward(q, k, v, shape.G)
+    outs = {}
+    for spec in ("bwd=split", "bwd=split_ds", "bwd=split_ds,ds_slots=2"):
+        _lib.s2attn_set_tile_override(spec)
+        try:
+            outs[spec] = s2.s2attn_backward(q, k, v, o, lse, do, shape.G)
+            assert s2.device_status() == 0
+        finally:
+            _lib.s2attn_set_tile_override(None)
+    ref_grads = outs.pop("bwd=split")
+    for spec, grads in outs.items():
+        for name, a, b in zip(("dq", "dk", "dv"), ref_grads, grads):
+            assert torch.equal(a.view(torch.int16), b.view(torch.int16)), f"{name} differs under {spec}"
+
+
 def test_launch_counts():
     from sparse_attention_attn_b200 import _lib
     import sparse_attention_attn_b200 as s2
