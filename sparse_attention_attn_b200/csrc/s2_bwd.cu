@@ -936,7 +936,9 @@ template <int D>
 cudaError_t launch_bwd_pre(const BwdPreArgs& pre, int num_sms, cudaStream_t stream) {
   const long long rows = static_cast<long long>(pre.d.B) * pre.d.N * pre.d.H;
   const long long tasks = rows / kTile;  // 128-row tasks of one (batch, head)
-  const int pre_grid = static_cast<int>(tasks < 8LL * num_sms ? tasks : 8LL * num_sms);
+  // up to 16 blocks per SM (8 resident at a time): blocks that finish early
+  // take the remaining tasks (0.050 vs 0.054 ms at the Qwen3-8B shape with 8)
+  const int pre_grid = static_cast<int>(tasks < 16LL * num_sms ? tasks : 16LL * num_sms);
   prof_before(stream, kKernelBwdPre);
   s2_bwd_pre_kernel<D><<<pre_grid, 256, 0, stream>>>(pre);
   cudaError_t e = cudaGetLastError();
