@@ -396,8 +396,11 @@ S2ATTN_API int s2attn_profile_stop(float* ms, int* kernel_ids, int capacity);
  * units (batch x kv head x group) whose dS blocks the workspace holds at once
  * (all of them when they fit its 4 GiB budget; fewer, and the backward runs
  * its dK/dV work in ranges of pairs each followed by dQ for the units the
- * range completed), else 0.  `out` holds 6 ints.  Host only; returns a status
- * code (shape validation as in s2attn_fwd).
+ * range completed), else 0; out[6] the dK/dV kernel's query tile (64: 64-row
+ * sub-tiles; 128: 128-row tiles, whose S^T / dP^T UMMAs are twice as wide;
+ * S2 attention calls only, the chunk-wise and HGA backwards take 64).  `out`
+ * holds 7 ints.  Host only; returns a status code (shape validation as in
+ * s2attn_fwd).
  */
 S2ATTN_API int s2attn_plan(int B, int H, int Hkv, int N, int D, int G, int num_sms, int* out);
 
@@ -408,6 +411,7 @@ S2ATTN_API int s2attn_plan(int B, int H, int Hkv, int N, int D, int G, int num_s
  * would not pick, for tests and sweeps: a comma-separated list of key=value
  * items; keys bwd=split_ds|split|fused (backward path; fused exists for head dim 128),
  * ds_slots=N (N >= 2: the split-dS path's workspace holds dS of N dK/dV units),
+ * bwd_qtile=64|128 (the dK/dV kernel's query tile),
  * fwd_order=snake|pairs (forward work order), fwd_bn=64|128 (forward key
  * tile), fwd_kv=N (forward K/V ring depth: with 128-key tiles 4 at head dim
  * 128, 4/6/8 at 64; with 64-key tiles 8 at head dim 128, 8/12 at 64), bwd_stages=N (split backward

@@ -194,11 +194,11 @@ def s2attn_bwd_rope(q_rot, k_rot, v, o, lse, dO, dq, dk, dv, table, B, H, Hkv, N
 
 def s2attn_plan(B, H, Hkv, N, D, G, num_sms):
     """The per-shape plan as a dict (host only), or raises on an invalid shape."""
-    out = (ctypes.c_int * 6)()
+    out = (ctypes.c_int * 7)()
     _check("s2attn_plan", load().s2attn_plan(B, H, Hkv, N, D, G, num_sms, ctypes.addressof(out)))
     return {"fwd_order": "snake" if out[0] else "pairs", "fwd_bn": out[4], "fwd_kv_slots": out[1],
             "bwd_path": {0: "split", 1: "fused", 2: "split_ds"}[out[2]], "bwd_stages": out[3],
-            "ds_slots": out[5]}
+            "ds_slots": out[5], "bwd_qtile": out[6]}
 
 
 def s2attn_nf4_levels():

@@ -23,7 +23,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libs2attn.so")
 LIB_DEBUG = os.path.join(PKG, "libs2attn_debug.so")
 
-SOURCES = ["s2attn.cu", "s2_fwd.cu", "s2_fwd64.cu", "s2_bwd.cu", "s2_bwd_fused.cu", "s2_rope.cu", "s2_segment.cu", "s2_nf4.cu", "s2_bwd_ds.cu"]
+SOURCES = ["s2attn.cu", "s2_fwd.cu", "s2_fwd64.cu", "s2_bwd.cu", "s2_bwd_fused.cu", "s2_rope.cu", "s2_segment.cu", "s2_nf4.cu", "s2_bwd_ds.cu", "s2_bwd_kv128.cu"]
 HEADERS = ["s2_ptx.cuh", "s2_common.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

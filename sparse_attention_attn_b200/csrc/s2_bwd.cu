@@ -976,11 +976,15 @@ cudaError_t launch_bwd_stages(const BwdMaps& m, const BwdPreArgs& pre, const Bwd
       const int p1 = p0 + chunk < total ? p0 + chunk : total;
       c.kv_sched.p0 = p0;
       c.kv_sched.pairs = p1;
-      prof_before(stream, kKernelBwdDkDv);
-      s2_bwd_dkdv_kernel<D, NST><<<pair_grid(c.kv_sched, num_sms), K3::THREADS, K3::SMEM_BYTES, stream>>>(
-          m.q64, m.k128, m.v128, m.g64, c);
-      e = cudaGetLastError();
-      prof_after(stream);
+      if (a.kv_q128) {
+        e = launch_dkdv128<D>(m, c, num_sms, stream);
+      } else {
+        prof_before(stream, kKernelBwdDkDv);
+        s2_bwd_dkdv_kernel<D, NST><<<pair_grid(c.kv_sched, num_sms), K3::THREADS, K3::SMEM_BYTES, stream>>>(
+            m.q64, m.k128, m.v128, m.g64, c);
+        e = cudaGetLastError();
+        prof_after(stream);
+      }
       if (e != cudaSuccess) return e;
       ++n;
       const int upto = p1 / ppu;  // units with every pair done
@@ -996,7 +1000,10 @@ cudaError_t launch_bwd_stages(const BwdMaps& m, const BwdPreArgs& pre, const Bwd
     if (launches) *launches = n;
     return cudaSuccess;
   }
-  if (!a.no_dkdv) {
+  if (!a.no_dkdv && a.kv_q128) {
+    e = launch_dkdv128<D>(m, a, num_sms, stream);
+    if (e != cudaSuccess) return e;
+  } else if (!a.no_dkdv) {
     const int grid_kv = pair_grid(a.kv_sched, num_sms);
     prof_before(stream, kKernelBwdDkDv);
     s2_bwd_dkdv_kernel<D, NST><<<grid_kv, K3::THREADS, K3::SMEM_BYTES, stream>>>(m.q64, m.k128, m.v128, m.g64, a);

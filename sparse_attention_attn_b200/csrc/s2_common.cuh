@@ -348,6 +348,7 @@ struct BwdArgs {
   __nv_bfloat16* ds;       // split-dS path: the dK/dV kernel stores dS blocks here (see ds_block), or null
   int ds_tt;               // dS blocks per (batch, head, group): T (T + 1) / 2
   int ds_slots;            // dK/dV units whose dS the workspace holds at once (unit u uses slot u mod ds_slots)
+  int kv_q128;             // dK/dV with 128-query tiles (s2_bwd_kv128.cu) instead of 64-query sub-tiles
   long long ds_blocks;     // dS blocks in all: ds_slots * rep * ds_tt
   uint32_t* status;
   unsigned long long wait_limit_ns;
@@ -387,6 +388,9 @@ struct BwdMaps {
 
 template <int D>
 cudaError_t launch_bwd_pre(const BwdPreArgs& pre, int num_sms, cudaStream_t stream);
+// dK/dV with 128-query tiles: one launch over a.kv_sched's pair range.
+template <int D>
+cudaError_t launch_dkdv128(const BwdMaps& m, const BwdArgs& a, int num_sms, cudaStream_t stream);
 template <int D>
 cudaError_t launch_dq_ds(const CUtensorMap& tds, const CUtensorMap& tk, const CUtensorMap& tq32, const BwdArgs& a,
                          int num_sms, cudaStream_t stream);

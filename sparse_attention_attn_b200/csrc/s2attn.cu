@@ -209,7 +209,7 @@ Dims make_segment_dims(int B, int H, int Hkv, int N, int Nk, int D, int causal) 
 // A plan override string ("key=value,..."), used to time or test a variant
 // that the per-shape selection would not pick.  It starts from the
 // S2ATTN_TILE environment variable and can be replaced at run time by the
-// s2attn_set_tile_override test hook.  Keys: bwd=split_ds|split|fused, ds_slots=N,
+// s2attn_set_tile_override test hook.  Keys: bwd=split_ds|split|fused, ds_slots=N, bwd_qtile=64|128,
 // fwd_order=snake|pairs, fwd_bn=64|128, fwd_kv=N, bwd_stages=N, nf4_stages=4|5, nf4_dq=8|12.  Unknown
 // keys and values are ignored.
 std::mutex g_override_mu;
@@ -252,6 +252,7 @@ struct Plan {
   int bwd_path;      // kBwdSplitDs, kBwdSplit, or kBwdFused (head dim 128 only)
   int bwd_stages;    // split backward operand stages: 2-3 (head dim 128), 3-4 (head dim 64)
   int ds_slots;      // split-dS path: dK/dV units whose dS the workspace holds (see ds_slots_for)
+  int bwd_qtile;     // dK/dV query tile: 64 (sub-tiles, s2_bwd.cu) or 128 (s2_bwd_kv128.cu)
 };
 
 bool valid_kv_slots(int D, int bn, int v) {
@@ -280,6 +281,7 @@ Plan select_plan(int B, int H, int Hkv, int N, int D, int G, int sms) {
   p.ds_slots = ds_slots_for(B, H, Hkv, N, G);
   p.bwd_path = p.ds_slots > 0 ? kBwdSplitDs : kBwdSplit;
   p.bwd_stages = 3;
+  p.bwd_qtile = 64;
   // the override, where it names a variant that exists for this head dim
   const std::string spec = tile_override();
   const std::string order = override_value(spec, "fwd_order");
@@ -303,6 +305,9 @@ Plan select_plan(int B, int H, int Hkv, int N, int D, int G, int sms) {
   if (path == "split_ds" && p.ds_slots == 0) p.ds_slots = ds_slots_for(B, H, Hkv, N, G, 2);
   if (path == "split_ds") p.bwd_path = kBwdSplitDs;
   if (path == "fused" && D == 128) p.bwd_path = kBwdFused;
+  const std::string qt = override_value(spec, "bwd_qtile");
+  if (qt == "64") p.bwd_qtile = 64;
+  if (qt == "128") p.bwd_qtile = 128;
   const std::string st = override_value(spec, "bwd_stages");
   if (!st.empty() && valid_bwd_stages(D, std::atoi(st.c_str()))) p.bwd_stages = std::atoi(st.c_str());
   return p;
@@ -561,12 +566,13 @@ int s2attn_seg_fwd(const void* q, const void* k, const void* v, void* o, float* 
 
 namespace {
 // The backward on `path` (kBwdSplitDs, kBwdSplit or kBwdFused); ds_slots: the
-// split-dS path's dK/dV units of dS in the workspace (ds_slots_for).  `seg`: segment-mode
+// split-dS path's dK/dV units of dS in the workspace (ds_slots_for); qtile:
+// the dK/dV kernel's query tile (128 for S2 attention only; 64 otherwise).  `seg`: segment-mode
 // dimensions (chunk-wise attention; split path only), or null for S2
 // attention of (B, H, Hkv, N, D, G).  Segment mode with causal = 0 computes dq
 // only (dk = dv = null: a detached key segment); dq_accumulate adds the
 // result to dq.
-int bwd_impl(int path, int stages, int ds_slots, const void* q, const void* k, const void* v, const void* o, const float* lse,
+int bwd_impl(int path, int stages, int ds_slots, int qtile, const void* q, const void* k, const void* v, const void* o, const float* lse,
              const void* dO, void* dq, void* dk, void* dv, int B, int H, int Hkv, int N, int D, int G,
              void* workspace, size_t workspace_bytes, s2attn_stream_t stream, const float* rope = nullptr,
              const Dims* seg = nullptr, int dq_accumulate = 0, HgaList hist = HgaList()) {
@@ -642,6 +648,7 @@ int bwd_impl(int path, int stages, int ds_slots, const void* q, const void* k, c
   a.ds = ds;
   a.ds_tt = (G / kTile) * (G / kTile + 1) / 2;
   a.ds_slots = ds_slots;
+  a.kv_q128 = (qtile == 128 && seg == nullptr && hist.tiles == nullptr && path != kBwdFused) ? 1 : 0;
   a.ds_blocks = ds_blocks;
   a.status = status;
   a.wait_limit_ns = wait_limit_ns();
@@ -675,7 +682,7 @@ int s2attn_bwd(const void* q, const void* k, const void* v, const void* o, const
                const void* dO, void* dq, void* dk, void* dv, int B, int H, int Hkv, int N, int D,
                int G, void* workspace, size_t workspace_bytes, s2attn_stream_t stream) {
   const Plan plan = select_plan(B, H, Hkv, N, D, G, 0);
-  return bwd_impl(plan.bwd_path, plan.bwd_stages, plan.ds_slots, q, k, v, o, lse, dO, dq, dk, dv, B, H, Hkv, N, D, G,
+  return bwd_impl(plan.bwd_path, plan.bwd_stages, plan.ds_slots, plan.bwd_qtile, q, k, v, o, lse, dO, dq, dk, dv, B, H, Hkv, N, D, G,
                   workspace, workspace_bytes, stream);
 }
 
@@ -742,7 +749,7 @@ int s2attn_bwd_rope(const void* q_rot, const void* k_rot, const void* v, const v
   if (!table) return S2ATTN_ERR_INVALID_ARG;
   if (!aligned16(table)) return S2ATTN_ERR_MISALIGNED;
   const Plan plan = select_plan(B, H, Hkv, N, D, G, 0);
-  return bwd_impl(plan.bwd_path, plan.bwd_stages, plan.ds_slots, q_rot, k_rot, v, o, lse, dO, dq, dk, dv, B, H, Hkv, N, D, G,
+  return bwd_impl(plan.bwd_path, plan.bwd_stages, plan.ds_slots, plan.bwd_qtile, q_rot, k_rot, v, o, lse, dO, dq, dk, dv, B, H, Hkv, N, D, G,
                   workspace, workspace_bytes, stream, table);
 }
 
@@ -759,7 +766,7 @@ int s2attn_seg_bwd(const void* q, const void* k, const void* v, const void* o, c
   if (st != S2ATTN_OK) return st;
   const Dims d = make_segment_dims(B, H, Hkv, N, Nk, D, causal);
   const Plan plan = select_plan(B, H, Hkv, N, D, N, 0);
-  return bwd_impl(kBwdSplit, plan.bwd_stages, 0, q, k, v, o, lse, dO, dq, dk, dv, B, H, Hkv, N, D, N, workspace,
+  return bwd_impl(kBwdSplit, plan.bwd_stages, 0, 64, q, k, v, o, lse, dO, dq, dk, dv, B, H, Hkv, N, D, N, workspace,
                   workspace_bytes, stream, nullptr, &d, dq_accumulate);
 }
 
@@ -813,7 +820,7 @@ int s2attn_hga_bwd(const void* q, const void* k, const void* v, const void* o, c
   hl.tiles = hist;
   hl.S = S;
   const Plan plan = select_plan(B, H, Hkv, N, D, G, 0);
-  return bwd_impl(kBwdSplit, plan.bwd_stages, 0, q, k, v, o, lse, dO, dq, dk, dv, B, H, Hkv, N, D, G, workspace,
+  return bwd_impl(kBwdSplit, plan.bwd_stages, 0, 64, q, k, v, o, lse, dO, dq, dk, dv, B, H, Hkv, N, D, G, workspace,
                   workspace_bytes, stream, nullptr, &d, 0, hl);
 }
 
@@ -981,6 +988,7 @@ int s2attn_plan(int B, int H, int Hkv, int N, int D, int G, int num_sms, int* ou
   out[3] = p.bwd_stages;
   out[4] = p.fwd_bn;
   out[5] = p.bwd_path == kBwdSplitDs ? p.ds_slots : 0;
+  out[6] = p.bwd_qtile;
   return S2ATTN_OK;
 }
 
@@ -1108,6 +1116,6 @@ extern "C" int s2attn_bwd_noalloc(const void* q, const void* k, const void* v, c
   // an invalid shape: bwd_impl reports which error
   if (valid && !noalloc_scratch(&scratch)) return S2ATTN_ERR_CUDA;
   const Plan plan = select_plan(B, H, Hkv, N, D, G, 0);
-  return bwd_impl(kBwdSplit, plan.bwd_stages, 0, q, k, v, o, lse, dO, dq, dk, dv, B, H, Hkv, N, D, G, scratch,
+  return bwd_impl(kBwdSplit, plan.bwd_stages, 0, plan.bwd_qtile, q, k, v, o, lse, dO, dq, dk, dv, B, H, Hkv, N, D, G, scratch,
                   kNoAllocScratchBytes, stream);
 }

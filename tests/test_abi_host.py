@@ -163,17 +163,17 @@ def test_plan_override_parsing():
         _lib.s2attn_set_tile_override("fwd_order=pairs,fwd_kv=2,bwd=split,bwd_stages=2")
         p = _lib.s2attn_plan(1, 32, 32, 8192, 128, 2048, 148)   # a 2-slot K/V ring does not exist
         assert p == {"fwd_order": "pairs", "fwd_bn": 128, "fwd_kv_slots": 4, "bwd_path": "split", "bwd_stages": 2,
-                     "ds_slots": 0}
+                     "ds_slots": 0, "bwd_qtile": 64}
         p = _lib.s2attn_plan(1, 4, 4, 1024, 64, 256, 148)   # head dim 64: kv 2 and stages 2 do not exist
         assert p == {"fwd_order": "pairs", "fwd_bn": 128, "fwd_kv_slots": 8, "bwd_path": "split", "bwd_stages": 3,
-                     "ds_slots": 0}
+                     "ds_slots": 0, "bwd_qtile": 64}
         _lib.s2attn_set_tile_override("bwd=fused,fwd_kv=6,bwd_stages=4,junk,=,x=y")  # no fused path at D = 64
         assert _lib.s2attn_plan(1, 4, 4, 1024, 64, 256, 148) == \
             {"fwd_order": "snake", "fwd_bn": 128, "fwd_kv_slots": 6, "bwd_path": "split_ds", "bwd_stages": 4,
-             "ds_slots": 16}
+             "ds_slots": 16, "bwd_qtile": 64}
         assert _lib.s2attn_plan(1, 32, 32, 8192, 128, 2048, 148) == \
             {"fwd_order": "snake", "fwd_bn": 128, "fwd_kv_slots": 4, "bwd_path": "fused", "bwd_stages": 4,
-             "ds_slots": 0}
+             "ds_slots": 0, "bwd_qtile": 64}
         _lib.s2attn_set_tile_override("bwd_stages=5")  # 5 stages exist for neither head dim
         assert _lib.s2attn_plan(1, 32, 32, 8192, 128, 2048, 148)["bwd_stages"] == 3
         assert _lib.s2attn_plan(1, 4, 4, 1024, 64, 256, 148)["bwd_stages"] == 3

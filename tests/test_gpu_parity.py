@@ -118,6 +118,8 @@ PLAN_VARIANTS = [
     (64, "fwd_kv=6"), (64, "bwd=split,bwd_stages=4"), (64, "bwd=split_ds,bwd_stages=4"),
     (128, "fwd_bn=64"), (128, "fwd_bn=64,fwd_order=pairs"), (64, "fwd_bn=64"), (64, "fwd_bn=64,fwd_kv=12"),
     (128, "bwd=split_ds,ds_slots=2"), (128, "bwd=split_ds,ds_slots=3"), (64, "bwd=split_ds,ds_slots=2"),
+    (128, "bwd_qtile=128"), (128, "bwd_qtile=128,bwd=split"), (64, "bwd_qtile=128"),
+    (128, "bwd_qtile=128,ds_slots=3"),
 ]
 
 
@@ -270,15 +272,17 @@ def test_dense_100k_sampled():
 def test_backward_paths_agree_bitwise(shape):
     """The split backward (dQ recomputes S, P and dS), the split-dS backward
     (dQ from the dS the dK/dV kernel stored) and the split-dS backward in ranges
-    (two units of dS at a time) form every dS value with the same fp32 steps
-    and bf16 rounding and accumulate dQ over the kv tiles in the same order:
-    their gradients agree bit for bit."""
+    (two units of dS at a time), each with 64-query sub-tiles or 128-query tiles
+    in the dK/dV kernel, form every dS value with the same fp32 steps and bf16
+    rounding and accumulate dK, dV and dQ over the same 16-deep steps in the
+    same order: their gradients agree bit for bit."""
     import sparse_attention_attn_b200 as s2
     from sparse_attention_attn_b200 import _lib
     q, k, v, do = (t.cuda() for t in I.make_inputs(shape, 5))
     o, lse = s2.s2attn_forward(q, k, v, shape.G)
     outs = {}
-    for spec in ("bwd=split", "bwd=split_ds", "bwd=split_ds,ds_slots=2"):
+    for spec in ("bwd=split", "bwd=split_ds", "bwd=split_ds,ds_slots=2", "bwd=split,bwd_qtile=128",
+                 "bwd=split_ds,bwd_qtile=128", "bwd=split_ds,ds_slots=2,bwd_qtile=128"):
         _lib.s2attn_set_tile_override(spec)
         try:
             outs[spec] = s2.s2attn_backward(q, k, v, o, lse, do, shape.G)
