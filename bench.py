@@ -722,15 +722,17 @@ def other_workload(shape: I.Shape, dev, peaks, steps: int = 5, warmup: int = 3):
 def sweep_variants(shape: I.Shape):
     """Every variant the per-shape plan can select for a workload shape, as
     override strings: forward (work order x key tile x K/V ring depth) and
-    backward (path x stages).  The split-dS path keeps the plan's dS slots
-    (every unit within the 4 GiB budget, else ranges)."""
+    backward (path x stages, and the dK/dV kernel's 128-query tiles).  The
+    split-dS path keeps the plan's dS slots (every unit within the 4 GiB
+    budget, else ranges)."""
     D = shape.D
     slots = (4,) if D == 128 else (4, 6, 8)
     fwd = [f"fwd_order={o},fwd_kv={s}" for o in ("snake", "pairs") for s in slots] + \
         [f"fwd_bn=64,fwd_order={o},fwd_kv={s}" for o in ("snake", "pairs") for s in ((8,) if D == 128 else (8, 12))]
     stages = (2, 3) if D == 128 else (3, 4)
     paths = ("split_ds", "split")
-    bwd = (["bwd=fused"] if D == 128 else []) + [f"bwd={p},bwd_stages={s}" for p in paths for s in stages]
+    bwd = (["bwd=fused"] if D == 128 else []) + [f"bwd={p},bwd_stages={s}" for p in paths for s in stages] + \
+        ["bwd=split_ds,bwd_stages=3,bwd_qtile=128"]
     return fwd, bwd
 
 
