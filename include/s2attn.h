@@ -414,8 +414,9 @@ S2ATTN_API int s2attn_plan(int B, int H, int Hkv, int N, int D, int G, int num_s
  * bwd_qtile=64|128 (the dK/dV kernel's query tile),
  * fwd_order=snake|pairs (forward work order), fwd_bn=64|128 (forward key
  * tile), fwd_kv=N (forward K/V ring depth: with 128-key tiles 4 at head dim
- * 128, 4/6/8 at 64; with 64-key tiles 8 at head dim 128, 8/12 at 64), bwd_stages=N (split backward
- * stages: 2-3 at head dim 128, 3-4 at 64), nf4_stages=4|5 and nf4_dq=8|12
+ * 128, 4/6/8 at 64; with 64-key tiles 8 at head dim 128, 8/12 at 64), bwd_stages=N (dK/dV operand
+ * stages: 2-4 at head dim 128, 3-4 at 64; the split path's dQ kernel takes at
+ * most 3 at head dim 128), nf4_stages=4|5 and nf4_dq=8|12
  * (pipeline depth and dequantization warps of s2attn_nf4_qkv); values that do not exist for a call's head dim
  * are ignored.  s2attn_bwd_workspace_bytes answers for the
  * path in force when it is called.  Returns S2ATTN_OK.

@@ -931,7 +931,7 @@ static bool set_smem_attr(const void* fn, int bytes) {
 }
 
 // The preprocess: one block per 128-row task of one (batch, head), at most
-// eight blocks per SM.
+// sixteen blocks per SM.
 template <int D>
 cudaError_t launch_bwd_pre(const BwdPreArgs& pre, int num_sms, cudaStream_t stream) {
   const long long rows = static_cast<long long>(pre.d.B) * pre.d.N * pre.d.H;

@@ -250,7 +250,7 @@ struct Plan {
   int fwd_kv_slots;  // forward K/V ring depth: 128-key tiles 4 (head dim 128), 4/6/8 (head dim 64);
                      // 64-key tiles 8 (head dim 128), 8/12 (head dim 64)
   int bwd_path;      // kBwdSplitDs, kBwdSplit, or kBwdFused (head dim 128 only)
-  int bwd_stages;    // split backward operand stages: 2-3 (head dim 128), 3-4 (head dim 64)
+  int bwd_stages;    // dK/dV operand stages: 2-4 (head dim 128; the split dQ kernel at most 3), 3-4 (head dim 64)
   int ds_slots;      // split-dS path: dK/dV units whose dS the workspace holds (see ds_slots_for)
   int bwd_qtile;     // dK/dV query tile: 64 (sub-tiles, s2_bwd.cu) or 128 (s2_bwd_kv128.cu)
 };
