@@ -1,7 +1,9 @@
 """The debug build (libs2attn_debug.so: every computed global index checked
 against its tensor in the kernels) on the GPU: on valid calls no check fires
 (device status 0) and the outputs are bit-identical to the default build's,
-for the S2 forward and backward, the HGA lists and the NF4 projection.  Each
+for the S2 forward and backward (planned kernels, and the selectable 64-key
+forward, 128-query-tile dK/dV and ranged split-dS backward), the HGA lists and
+the NF4 projection.  Each
 build runs in its own process (S2ATTN_DEBUG selects the library at import)."""
 import json
 import os
@@ -29,6 +31,14 @@ dq, dk, dv = s2.s2attn_backward(q, k, v, o, lse, do, shape.G)
 torch.cuda.synchronize()
 out["s2"] = h(o, lse, dq, dk, dv)
 out["status_fwd"] = s2.device_status()
+# the selectable kernels: 64-key forward, dK/dV with 128-query tiles, split-dS in ranges
+_lib.s2attn_set_tile_override("fwd_bn=64,bwd_qtile=128,ds_slots=2")
+o3, l3 = s2.s2attn_forward(q, k, v, shape.G)
+g3 = s2.s2attn_backward(q, k, v, o3, l3, do, shape.G)
+_lib.s2attn_set_tile_override(None)
+torch.cuda.synchronize()
+out["variants"] = h(o3, l3, *g3)
+out["status_variants"] = s2.device_status()
 sel = -torch.ones((1, 4, 2), dtype=torch.int32)
 sel[0, 2, 0] = 1
 sel[0, 3, :] = torch.tensor([0, 3], dtype=torch.int32)
@@ -62,6 +72,6 @@ def test_debug_build_agrees_and_no_check_fires():
     build.build(debug=True)
     rel, dbg = _run(False), _run(True)
     assert rel["debug"] == 0 and dbg["debug"] == 1
-    assert dbg["status_fwd"] == 0 and dbg["status"] == 0, dbg
-    for key in ("s2", "hga", "nf4"):
+    assert dbg["status_fwd"] == 0 and dbg["status_variants"] == 0 and dbg["status"] == 0, dbg
+    for key in ("s2", "variants", "hga", "nf4"):
         assert dbg[key] == rel[key], f"{key}: the debug build's outputs differ from the default build's"
