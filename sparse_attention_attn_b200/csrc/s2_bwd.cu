@@ -373,11 +373,9 @@ __global__ void __launch_bounds__(352, 1)
       const int s = g % ST;
       const int qoff = (cur.it % cur.nq) * kSub;  // query sub-tile start minus kv tile start (rolled)
       const uint32_t bo = (g & 1) * kSub + half * 32;
-      if (lane == 0)
-        ok = mbar_wait(smem_u32(&bar_full[s]), (g / ST) & 1, wc, 130) &&
-             mbar_wait(smem_u32(&bar_s[g & 1]), (g >> 1) & 1, wc, 131) &&
-             mbar_wait(smem_u32(&bar_dp[g & 1]), (g >> 1) & 1, wc, 133);
-      ok = __shfl_sync(0xffffffffu, ok, 0);
+      ok = warp_wait(smem_u32(&bar_full[s]), (g / ST) & 1, wc, 130) &&
+           warp_wait(smem_u32(&bar_s[g & 1]), (g >> 1) & 1, wc, 131) &&
+           warp_wait(smem_u32(&bar_dp[g & 1]), (g >> 1) & 1, wc, 133);
       if (!ok) break;
       tc_fence_after();
       // row statistics of the 64 query rows: -lse*log2e at +0, -Delta at +256 bytes
@@ -450,8 +448,7 @@ __global__ void __launch_bounds__(352, 1)
       }
       if (cur.it == cur.iters - 1) {
         // ---------------------------------------------------- epilogue of this item
-        if (lane == 0) ok = mbar_wait(smem_u32(&bar_acc_full), cur.ic.n & 1, wc, 132);
-        ok = __shfl_sync(0xffffffffu, ok, 0);
+        ok = warp_wait(smem_u32(&bar_acc_full), cur.ic.n & 1, wc, 132);
         if (!ok) break;
         tc_fence_after();
         const TileWork& w = cur.w;
@@ -758,9 +755,7 @@ __global__ void __launch_bounds__(384, 1)
     // shared-memory tile into TMEM as bf16 pairs: the A operand of S / dP.
     // Called once the previous item's last S and dP have completed.
     auto put_q = [&](const DqCursor& c) -> bool {
-      bool okq = true;
-      if (lane == 0) okq = mbar_wait(smem_u32(&bar_q), c.ic.n & 1, wc, 233);
-      if (!__shfl_sync(0xffffffffu, okq, 0)) return false;
+      if (!warp_wait(smem_u32(&bar_q), c.ic.n & 1, wc, 233)) return false;
       const uint32_t src = (half == 0 ? sQ : sG) + row * 128;
       const uint32_t sw = static_cast<uint32_t>(row & 7);
 #pragma unroll
@@ -815,8 +810,7 @@ __global__ void __launch_bounds__(384, 1)
       // kv sub-tile start minus query tile start (in the sub-tile walk: the
       // historical tiles and the segment offset come first)
       const int koff = cur.it * kSub - (w.tile + d.qoff_t + cur.nh) * kTile;
-      if (lane == 0) ok = mbar_wait(smem_u32(&bar_sdp[g & 1]), (g >> 1) & 1, wc, 230);
-      ok = __shfl_sync(0xffffffffu, ok, 0);
+      ok = warp_wait(smem_u32(&bar_sdp[g & 1]), (g >> 1) & 1, wc, 230);
       if (!ok) break;
       tc_fence_after();
       if (cur.it == cur.iters - 1) {
@@ -860,8 +854,7 @@ __global__ void __launch_bounds__(384, 1)
       if (lane == 0) mbar_arrive(smem_u32(&bar_ds[g & 1]));
       if (cur.it == cur.iters - 1) {
         // ---------------------------------------------------- epilogue of this item
-        if (lane == 0) ok = mbar_wait(smem_u32(&bar_acc_full), cur.ic.n & 1, wc, 232);
-        ok = __shfl_sync(0xffffffffu, ok, 0);
+        ok = warp_wait(smem_u32(&bar_acc_full), cur.ic.n & 1, wc, 232);
         if (!ok) break;
         tc_fence_after();
         // this thread's row, columns [half * D/2, (half+1) * D/2), scaled,

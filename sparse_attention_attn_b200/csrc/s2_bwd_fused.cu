@@ -355,9 +355,7 @@ __global__ void __launch_bounds__(384, 1)
     // dQ^T of sub-tile gp out of TMEM into its buffer pair as fp32 [64][D]
     auto stage_dq = [&](int gp) -> bool {
       const int b = gp & 1;
-      bool okw = true;
-      if (lane == 0) okw = mbar_wait(smem_u32(&bar_mma_done[b]), (gp >> 1) & 1, wc, 353);
-      if (!__shfl_sync(0xffffffffu, okw, 0)) return false;
+      if (!warp_wait(smem_u32(&bar_mma_done[b]), (gp >> 1) & 1, wc, 353)) return false;
       tc_fence_after();
       uint32_t r[32];
       tmem_ld32(tmem + lane_off + C::TM_DQ + b * kSub + half * 32, r);
@@ -379,10 +377,8 @@ __global__ void __launch_bounds__(384, 1)
     for (; cur.ic.valid; ++g) {
       const int s = g % ST, b = g & 1;
       const int qoff = (cur.it % cur.nq) * kSub;  // query sub-tile start minus kv tile start (rolled)
-      if (lane == 0)
-        ok = mbar_wait(smem_u32(&bar_full[s]), (g / ST) & 1, wc, 350) &&
-             mbar_wait(smem_u32(&bar_s), g & 1, wc, 351) && mbar_wait(smem_u32(&bar_dp), g & 1, wc, 352);
-      ok = __shfl_sync(0xffffffffu, ok, 0);
+      ok = warp_wait(smem_u32(&bar_full[s]), (g / ST) & 1, wc, 350) &&
+           warp_wait(smem_u32(&bar_s), g & 1, wc, 351) && warp_wait(smem_u32(&bar_dp), g & 1, wc, 352);
       if (!ok) break;
       tc_fence_after();
       // row statistics of this half's 32 query rows: -lse*log2e at +0, -Delta at +256 bytes
@@ -435,8 +431,7 @@ __global__ void __launch_bounds__(384, 1)
       // the pair held the dQ partial of sub-tile g-2: wait until the bulk
       // reduction has read it
       if (g >= 2) {
-        if (lane == 0) ok = mbar_wait(smem_u32(&bar_buf_free[b]), ((g - 2) >> 1) & 1, wc, 354);
-        ok = __shfl_sync(0xffffffffu, ok, 0);
+        ok = warp_wait(smem_u32(&bar_buf_free[b]), ((g - 2) >> 1) & 1, wc, 354);
         if (!ok) break;
       }
       // P^T and dS^T rows (bf16, 128-byte swizzled): this thread's 32 query
@@ -454,8 +449,7 @@ __global__ void __launch_bounds__(384, 1)
       if (g >= 1 && !(ok = stage_dq(g - 1))) break;
       if (cur.it == cur.iters - 1) {
         // ---------------------------------------------------- dK / dV epilogue of this item
-        if (lane == 0) ok = mbar_wait(smem_u32(&bar_acc_full), cur.ic.n & 1, wc, 355);
-        ok = __shfl_sync(0xffffffffu, ok, 0);
+        ok = warp_wait(smem_u32(&bar_acc_full), cur.ic.n & 1, wc, 355);
         if (!ok) break;
         tc_fence_after();
         const TileWork& w = cur.w;

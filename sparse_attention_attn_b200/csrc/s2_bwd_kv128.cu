@@ -272,10 +272,8 @@ __global__ void __launch_bounds__(352, 1)
     for (int g = 0; cur.ic.valid; ++g) {
       const int s = g % ST;
       const bool diag = (cur.it % cur.nq) == 0;  // the query tile on the kv tile's diagonal
-      if (lane == 0)
-        ok = mbar_wait(smem_u32(&bar_full[s]), (g / ST) & 1, wc, 170) &&
-             mbar_wait(smem_u32(&bar_s), g & 1, wc, 171) && mbar_wait(smem_u32(&bar_dp), g & 1, wc, 172);
-      ok = __shfl_sync(0xffffffffu, ok, 0);
+      ok = warp_wait(smem_u32(&bar_full[s]), (g / ST) & 1, wc, 170) &&
+           warp_wait(smem_u32(&bar_s), g & 1, wc, 171) && warp_wait(smem_u32(&bar_dp), g & 1, wc, 172);
       if (!ok) break;
       tc_fence_after();
       if (a.ds != nullptr && cur.it == 0)
@@ -351,8 +349,7 @@ __global__ void __launch_bounds__(352, 1)
       }
       if (cur.it == cur.iters - 1) {
         // ---------------------------------------------------- epilogue of this item
-        if (lane == 0) ok = mbar_wait(smem_u32(&bar_acc_full), cur.ic.n & 1, wc, 173);
-        ok = __shfl_sync(0xffffffffu, ok, 0);
+        ok = warp_wait(smem_u32(&bar_acc_full), cur.ic.n & 1, wc, 173);
         if (!ok) break;
         tc_fence_after();
         const TileWork& w = cur.w;

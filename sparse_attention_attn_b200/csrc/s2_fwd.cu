@@ -360,8 +360,7 @@ __global__ void __launch_bounds__(320, 1)
       if (wg == 0 || it.has_b) {
         float m_run = 0.f, l_run = 0.f;
         for (int j = 0; j <= jlast; ++j) {
-          if (lane == 0) ok = mbar_wait(smem_u32(&bar_s[wg]), ns & 1, wc, 30);
-          ok = __shfl_sync(0xffffffffu, ok, 0);
+          ok = warp_wait(smem_u32(&bar_s[wg]), ns & 1, wc, 30);
           if (!ok) break;
           ++ns;
           tc_fence_after();
@@ -407,8 +406,7 @@ __global__ void __launch_bounds__(320, 1)
           if (__any_sync(0xffffffffu, resc)) {
             // rescale O (it holds P_{j-1} V_{j-1} once that UMMA has completed)
             // before P_j V_j accumulates onto it
-            if (lane == 0) ok = mbar_wait(smem_u32(&bar_o[wg]), (no - 1) & 1, wc, 31);
-            ok = __shfl_sync(0xffffffffu, ok, 0);
+            ok = warp_wait(smem_u32(&bar_o[wg]), (no - 1) & 1, wc, 31);
             if (!ok) break;
             tc_fence_after();
 #pragma unroll
@@ -438,8 +436,7 @@ __global__ void __launch_bounds__(320, 1)
         }
         // ---------------------------------------------------------- epilogue
         if (ok) {
-          if (lane == 0) ok = mbar_wait(smem_u32(&bar_o[wg]), (no - 1) & 1, wc, 32);
-          ok = __shfl_sync(0xffffffffu, ok, 0);
+          ok = warp_wait(smem_u32(&bar_o[wg]), (no - 1) & 1, wc, 32);
         }
         if (!ok) break;
         tc_fence_after();

@@ -345,8 +345,7 @@ __global__ void __launch_bounds__(320, 1)
         float m_run = 0.f, l_run = 0.f;
         for (int j = 0; j < nt; ++j) {
           const int buf = j & 1;
-          if (lane == 0) ok = mbar_wait(smem_u32(&bar_s[wg][buf]), nsb[buf] & 1, wc, 30);
-          ok = __shfl_sync(0xffffffffu, ok, 0);
+          ok = warp_wait(smem_u32(&bar_s[wg][buf]), nsb[buf] & 1, wc, 30);
           if (!ok) break;
           ++nsb[buf];
           tc_fence_after();
@@ -388,8 +387,7 @@ __global__ void __launch_bounds__(320, 1)
             // completed) before P(j) V(j) accumulates onto it.  P V(j-2) is
             // complete (S(j) was issued after it), so only P V(j-1) can be
             // pending and the parity wait is unambiguous
-            if (lane == 0) ok = mbar_wait(smem_u32(&bar_o[wg]), (no - 1) & 1, wc, 31);
-            ok = __shfl_sync(0xffffffffu, ok, 0);
+            ok = warp_wait(smem_u32(&bar_o[wg]), (no - 1) & 1, wc, 31);
             if (!ok) break;
             tc_fence_after();
 #pragma unroll
@@ -416,10 +414,8 @@ __global__ void __launch_bounds__(320, 1)
         // (UMMAs complete in order, so every earlier P V is done: this tile's
         // S was issued after P V(nt - 3).)
         if (ok) {
-          if (lane == 0)
-            ok = mbar_wait(smem_u32(&bar_o[wg]), (no - 2) & 1, wc, 32) &&
-                 mbar_wait(smem_u32(&bar_o[wg]), (no - 1) & 1, wc, 32);
-          ok = __shfl_sync(0xffffffffu, ok, 0);
+          ok = warp_wait(smem_u32(&bar_o[wg]), (no - 2) & 1, wc, 32) &&
+               warp_wait(smem_u32(&bar_o[wg]), (no - 1) & 1, wc, 32);
         }
         if (!ok) break;
         tc_fence_after();

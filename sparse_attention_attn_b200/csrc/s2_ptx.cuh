@@ -113,6 +113,9 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
 }
 
 // Bounded wait by a whole converged warp; every lane gets the same answer.
+// Every lane polls (one warp instruction per poll): measured faster than
+// lane 0 polling and broadcasting its answer, both for the single-thread
+// producer / issuer warps and for the compute warps.
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const WaitCtx& w,
                                           uint32_t where) {
   const bool ok = mbar_wait(bar, parity, w, where);
