@@ -246,10 +246,12 @@ __global__ void __launch_bounds__(320, 1)
       __syncwarp();
     };
     // P_wg(j) V_j: the first half as soon as P keys 0..63 are in TMEM
-    auto pv = [&](int wg, int Lv, int j, bool first_of_item) -> bool {
+    // (V_j's arrival is waited for once: by warpgroup A's P V, or by B's
+    // when A does not use tile j)
+    auto pv = [&](int wg, int Lv, int j, bool first_of_item, bool need_v) -> bool {
       if (!warp_wait(smem_u32(&bar_plo[wg]), np[wg] & 1, wc, wg == 0 ? 22 : 24) ||
           (first_of_item && n > 0 && !warp_wait(smem_u32(&bar_ofree[wg]), (n - 1) & 1, wc, wg == 0 ? 23 : 25)) ||
-          !wait_full(Lv))
+          (need_v && !wait_full(Lv)))
         return false;
       issue_pv(wg, Lv, 0, j > 0);
       if (!warp_wait(smem_u32(&bar_p[wg]), np[wg] & 1, wc, wg == 0 ? 28 : 29)) return false;
@@ -305,7 +307,7 @@ __global__ void __launch_bounds__(320, 1)
       for (int j = 0; ok && j < it.nkv; ++j) {
         const int Lv = L0 + 2 * j + 1, Lk1 = L0 + 2 * j + 2;
         if (j <= lastA) {
-          if (!(ok = pv(0, Lv, j, j == 0))) break;
+          if (!(ok = pv(0, Lv, j, j == 0, true))) break;
           if (j > lastB) commit(&bar_empty[Lv % NS]);
           if (j + 1 <= lastA) {
             if (!wait_full(Lk1)) { ok = false; break; }
@@ -316,7 +318,7 @@ __global__ void __launch_bounds__(320, 1)
           }
         }
         if (j <= lastB) {
-          if (!(ok = pv(1, Lv, j, j == 0))) break;
+          if (!(ok = pv(1, Lv, j, j == 0, j > lastA))) break;
           commit(&bar_empty[Lv % NS]);
           if (j + 1 <= lastB) {
             if (j + 1 > lastA && !wait_full(Lk1)) { ok = false; break; }
