@@ -268,6 +268,8 @@ def test_dense_100k_sampled():
 
 
 @pytest.mark.parametrize("shape", [I.Shape("agree", 2, 4, 2, 128, 2048, 512), I.Shape("agree64", 1, 6, 2, 64, 1536, 768),
+                                   I.Shape("agree-odd-tiles", 1, 2, 2, 64, 640, 640),
+                                   I.Shape("agree-odd-tiles-128", 2, 3, 1, 128, 640, 640),
                                    I.LLAMA2_7B_8K], ids=lambda s: s.name)
 def test_backward_paths_agree_bitwise(shape):
     """The split backward (dQ recomputes S, P and dS), the split-dS backward
