@@ -281,6 +281,13 @@ __global__ void __launch_bounds__(320, 1)
         if (it.has_b) issue_s(1, sB, L0);
         else release_q(sB);
         commit(&bar_empty[L0 % NS]);
+      } else if (!it.has_b) {
+        // the absent second tile's Q slot (filled without data) goes back here,
+        // once every UMMA of the previous item is issued: waiting for it any
+        // earlier could hold up that item's second-tile work, whose released
+        // K/V slots the producer needs before it reaches this slot
+        if (!(ok = warp_wait(smem_u32(&bar_qfull[sB]), (uB / NQ) & 1, wc, 26))) break;
+        release_q(sB);
       }
       // The next item's first scores are computed as soon as this item's
       // last P V of the same warpgroup has been issued (it reads P out of the
@@ -290,11 +297,7 @@ __global__ void __launch_bounds__(320, 1)
         if (!nx.valid) return true;
         if (!warp_wait(smem_u32(&bar_qfull[sAn]), ((uA + 2) / NQ) & 1, wc, 26) || !wait_full(L0n)) return false;
         issue_s(0, sAn, L0n);
-        if (!itn.has_b) {
-          if (!warp_wait(smem_u32(&bar_qfull[sBn]), ((uB + 2) / NQ) & 1, wc, 26)) return false;
-          release_q(sBn);
-          commit(&bar_empty[L0n % NS]);
-        }
+        if (!itn.has_b) commit(&bar_empty[L0n % NS]);  // its K_0 has no second reader
         return true;
       };
       auto start_next_b = [&]() -> bool {

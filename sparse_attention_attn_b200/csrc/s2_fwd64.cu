@@ -264,6 +264,12 @@ __global__ void __launch_bounds__(320, 1)
           if (ok) commit(&bar_empty[(L0 + 2 * e) % NS]);
         }
         if (!ok) break;
+      } else if (!it.has_b) {
+        // the absent second tile's Q slot goes back here, once every UMMA of
+        // the previous item is issued (any earlier could hold up that item's
+        // second-tile work, whose released K/V slots the producer needs first)
+        if (!wait_q(uB, 26)) break;
+        release_q(sB);
       }
       // the next item's first two scores of warpgroup B (after B's -- or, for
       // an item without B, A's -- last P V of this item)
@@ -288,14 +294,7 @@ __global__ void __launch_bounds__(320, 1)
             const int e = t - nA;
             if (!(ok = wait_q(uA + 2, 26) && issue_s(0, sAn, L0n + 2 * e, e))) break;
             if (!itn.has_b) commit(&bar_empty[(L0n + 2 * e) % NS]);
-            if (e == 1) {  // A's last P V of this item is issued
-              if (!itn.has_b) {
-                if (!(ok = wait_q(uB + 2, 26))) break;
-                release_q(sBn);
-              } else if (!it.has_b && !(ok = start_next_b())) {
-                break;
-              }
-            }
+            if (e == 1 && itn.has_b && !it.has_b && !(ok = start_next_b())) break;  // A's last P V is issued
           }
         }
         if (j < nB) {

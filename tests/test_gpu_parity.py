@@ -267,6 +267,33 @@ def test_dense_100k_sampled():
     _check_full_size(I.LLAMA2_7B_100K.dense(), m=512, units=[(0, 0, 0)])
 
 
+ODD_TILE_ORDERS = [(D, spec) for D in (128, 64) for spec in ("fwd_order=pairs", "fwd_order=snake",
+                                                              "fwd_bn=64,fwd_order=pairs", "fwd_bn=64,fwd_order=snake")]
+
+
+@pytest.mark.parametrize("D,spec", ODD_TILE_ORDERS, ids=[f"d{d}-{s}" for d, s in ODD_TILE_ORDERS])
+def test_forward_orders_on_odd_tile_counts(D, spec):
+    """Groups with an odd tile count end in an item without a second query
+    tile.  In the equal-work pairs order every CTA takes such an item right
+    after an item with two tiles (pair (0, last)), which once deadlocked the
+    forward's issuer (it waited to release the missing tile's Q slot while
+    that earlier item's second-tile work was still to issue).  Both orders
+    and both key tiles against the oracle, several items per CTA."""
+    import sparse_attention_attn_b200 as s2
+    from sparse_attention_attn_b200 import _lib
+    shape = I.Shape("odd", 2, 4, 2, D, 1152, 1152)  # dense, 9 tiles: items 0..4, item 4 without a second tile
+    q, k, v, do = I.make_inputs(shape, seed_offset=21)
+    _lib.s2attn_set_tile_override(spec)
+    try:
+        o, lse = s2.s2attn_forward(q.cuda(), k.cuda(), v.cuda(), shape.G)
+        assert s2.device_status() == 0, f"device status after the forward [{spec}]"
+    finally:
+        _lib.s2attn_set_tile_override(None)
+    o_ref, lse_ref = ref.s2_attention_fwd(to64(q), to64(k), to64(v), shape.G)
+    check_o(to64(o), o_ref, f" [{spec}]")
+    assert max_abs(to64(lse), lse_ref) < 1e-3
+
+
 @pytest.mark.parametrize("shape", [I.Shape("agree", 2, 4, 2, 128, 2048, 512), I.Shape("agree64", 1, 6, 2, 64, 1536, 768),
                                    I.Shape("agree-odd-tiles", 1, 2, 2, 64, 640, 640),
                                    I.Shape("agree-odd-tiles-128", 2, 3, 1, 128, 640, 640),
