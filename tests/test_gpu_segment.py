@@ -95,6 +95,35 @@ def test_two_pieces_merged(B, C, Nk, H, Hkv, D):
     check_grad("dK", to64(kt.grad), dk_ref, " [autograd]")
 
 
+@pytest.mark.parametrize("order", ["fwd_order=pairs", "fwd_order=snake"])
+def test_odd_tile_chunk_both_orders(order):
+    """A 9-tile chunk (the forward's last item has no second query tile) with
+    enough units that the pairs order hands every CTA item 0 then that item:
+    both pieces (detached keys, every key visible; own keys, causal) and the
+    merge against the one-call oracle, under both forward work orders."""
+    import sparse_attention_attn_b200 as s2
+    from sparse_attention_attn_b200 import _lib
+    B, C, Nk, H, Hkv, D = 2, 1152, 2304, 8, 2, 128
+    q, k, v, do = _inputs(B, C, Nk, H, Hkv, D, 70)
+    c0 = Nk - C
+    qd = q.cuda()
+    kp, vp = k[:, :c0].contiguous().cuda(), v[:, :c0].contiguous().cuda()
+    ka, va = k[:, c0:].contiguous().cuda(), v[:, c0:].contiguous().cuda()
+    _lib.s2attn_set_tile_override(order)
+    try:
+        o_a, lse_a = s2.seg_forward(qd, kp, vp, causal=False)
+        o_b, lse_b = s2.seg_forward(qd, ka, va, causal=True)
+        o, lse = s2.lse_merge(o_a, lse_a, o_b, lse_b)
+        torch.cuda.synchronize()
+        assert s2.device_status() == 0, f"device status [{order}]"
+    finally:
+        _lib.s2attn_set_tile_override(None)
+    q64, k64, v64 = (to64(t) for t in (q, k, v))
+    o_ref, lse_ref = cr.chunk_attention_fwd(q64, k64, v64)
+    check_o(to64(o), o_ref, f" [merged, {order}]")
+    assert max_abs(to64(lse), lse_ref) < 1e-3
+
+
 def test_merge_elementwise():
     import sparse_attention_attn_b200 as s2
     B, N, H, D = 2, 256, 4, 128
