@@ -400,6 +400,14 @@ __global__ void __launch_bounds__(320, 1)
             }
           }
           l_run = l_run * alpha + rs;
+          if (j == nt - 1) {
+            // the item's last P: P V(j-1) completes before P V(j) can be
+            // issued, so the epilogue's parity wait below finds one P V phase
+            // outstanding, never two (two would leave a parity wait on the
+            // earlier one naming a phase the barrier has already passed twice)
+            ok = warp_wait(smem_u32(&bar_o[wg]), (no - 1) & 1, wc, 33);
+            if (!ok) break;
+          }
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
@@ -407,15 +415,9 @@ __global__ void __launch_bounds__(320, 1)
           ++no;
         }
         // ---------------------------------------------------------- epilogue
-        // The last two P V may both be in flight (the softmax can be a tile
-        // ahead of the issuer): wait for them in order, or a parity wait on
-        // the last one could be answered by the phase before the other.
-        // (UMMAs complete in order, so every earlier P V is done: this tile's
-        // S was issued after P V(nt - 3).)
-        if (ok) {
-          ok = warp_wait(smem_u32(&bar_o[wg]), (no - 2) & 1, wc, 32) &&
-               warp_wait(smem_u32(&bar_o[wg]), (no - 1) & 1, wc, 32);
-        }
+        // Only the last P V can still be in flight: P V(nt - 2) was waited
+        // for before the last P went out.
+        if (ok) ok = warp_wait(smem_u32(&bar_o[wg]), (no - 1) & 1, wc, 32);
         if (!ok) break;
         tc_fence_after();
         uint32_t o[D / 32][32];

@@ -194,9 +194,10 @@ def run(items, ST, seed):
                 finished.add(c)
                 pending[c] = None
                 break
-            if op[0] == "arrive":
+            if op[0] == "arrive":  # an arrival, then any other actor may run first
                 bars[op[1]].arrive(op[2])
-                continue
+                pending[c] = None
+                break
             done = bars[op[1]].done
             if done >= op[2] + 2:
                 return [f"{c}: phase overrun on {op[1]}"]

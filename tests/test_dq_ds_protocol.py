@@ -167,9 +167,10 @@ def run(items, ST, seed):
             except StopIteration:
                 finished.add(c)
                 break
-            if op[0] == "arrive":
+            if op[0] == "arrive":  # an arrival, then any other actor may run first
                 bars[op[1]].arrive(op[2])
-                continue
+                pending[c] = None
+                break
             if op[0] == "yield":  # let the others run before this actor goes on
                 break
             if op[0] == "until":

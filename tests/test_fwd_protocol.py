@@ -2,7 +2,8 @@
 CPU: the TMA producer, the UMMA issuer, the two softmax warpgroups with their
 epilogues, the tensor pipe and the copies in flight (landing in any order), as
 programs of mbarrier waits and arrivals with the kernel's arrival counts and
-phases, interleaved at random.  It checks that
+phases, interleaved at random (after every wait and every arrival any other
+actor, the tensor pipe or a copy may go first).  It checks that
 every program finishes (no deadlock), that no wait is overrun (a barrier two
 phases ahead of the waiter, which a parity wait cannot tell apart), and that
 every UMMA reads the tile it means and nothing is overwritten while a reader
@@ -300,9 +301,10 @@ def run(items, seed):
                 finished.add(c)
                 pending[c] = None
                 break
-            if op[0] == "arrive":
+            if op[0] == "arrive":  # an arrival, then any other actor may run first
                 bars[op[1]].arrive(op[2])
-                continue
+                pending[c] = None
+                break
             done = bars[op[1]].done
             if done >= op[2] + 2:
                 return [f"{c}: phase overrun on {op[1]}"]
