@@ -224,6 +224,14 @@ __global__ void __launch_bounds__(Nf4Cfg<NS, DQW>::THREADS, 1)
       const float sc = static_cast<float>(q) * c2 / 127.f;
       const uint64_t sc2 = f2_pack(sc, sc);
       const int s = L % NS;
+      // The groups take a stage's loads in turn, so this group skips phases of
+      // bar_full[s]: before its parity wait, the stage's previous load must be
+      // known to have landed, or a barrier still a phase behind would show the
+      // parity of a completed phase and the wait would pass at once.  The
+      // UMMA of that load completing (bar_empty[s]) says so, and costs
+      // nothing in the normal order: the producer waited for it before it
+      // issued this load.
+      if (L >= NS && !warp_wait(smem_u32(&bar_empty[s]), (L / NS - 1) & 1, wc, 66)) break;
       if (!warp_wait(smem_u32(&bar_full[s]), (L / NS) & 1, wc, 64)) break;
       const uint32_t src = sC + s * C::C_BYTES + row * 32;
       const uint4 c0 = lds_u4(src), c1 = lds_u4(src + 16);

@@ -199,6 +199,8 @@ def run(items, ST, seed):
                 pending[c] = None
                 break
             done = bars[op[1]].done
+            if done < op[2]:  # the barrier is a phase behind: a parity wait would pass at once
+                return [f"{c}: parity wait ahead on {op[1]} (waits phase {op[2]}, {done} complete)"]
             if done >= op[2] + 2:
                 return [f"{c}: phase overrun on {op[1]}"]
             if done >= op[2] + 1:
