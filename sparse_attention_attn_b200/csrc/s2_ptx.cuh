@@ -96,6 +96,12 @@ static __device__ __noinline__ void record_timeout(const WaitCtx& w, uint32_t wh
 
 // Wait for phase `parity` of mbarrier `bar` to complete.  Returns false (after
 // recording the failure) if the limit runs out or another thread aborted.
+// A parity names phase k only while the barrier's open phase is k or k+1:
+// with k+2 open (k and k+1 complete) the open phase has k's parity and the
+// wait blocks; with k-1 open the open phase's parity differs from k's and the
+// wait passes at once.  Every caller keeps its barrier within that window:
+// phase k+1 needs something the waiter does after the wait, and phase k-1 is
+// complete before it (by its own earlier wait, or by a wait that implies it).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtx& w,
                                           uint32_t where) {
   if (mbar_try_wait(bar, parity)) return true;
