@@ -194,7 +194,7 @@ def cases():
     out = []
     for T in range(1, 11):
         npairs = (T + 1) // 2
-        for ST in (2, 3):
+        for ST in (2, 3, 4):  # 3 stages at head dim 128, 4 at 64
             out.append((items_for(T, range(npairs)), ST))              # a CTA's pairs of one group
             out.append((items_for(T, [0]) * 3, ST))                     # pair (0, T-1) of three groups
             out.append((items_for(T, range(npairs))[1:], ST))           # a range starting inside a pair

@@ -322,3 +322,11 @@ def test_model_finds_the_epilogue_parity_race():
     exec(src, ns)
     found = [p for items in sequences()[:12] for seed in range(8) for p in ns["run"]([dict(x) for x in items], seed)]
     assert any("phase overrun on ('o'" in p for p in found)
+
+
+def test_fwd64_protocol_twelve_slots():
+    """The 12-slot K/V ring head dim 64 can select."""
+    for items in sequences()[::3]:
+        for seed in range(4):
+            problems = run([dict(x) for x in items], seed, NS=12)
+            assert not problems, (problems, [(x["last_a"], x["last_b"], x["has_b"]) for x in items])

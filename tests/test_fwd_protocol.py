@@ -18,7 +18,7 @@ import random
 
 import pytest
 
-NS, NQ = 4, 3  # K/V ring slots (head dim 128), Q ring slots
+NQ = 3  # Q ring slots; the K/V ring has NS slots: 4 at head dim 128, 4, 6 or 8 at 64
 
 
 class Bar:
@@ -57,7 +57,7 @@ def pairs_order(T, **kw):
     return out
 
 
-def run(items, seed):
+def run(items, seed, NS=4):
     """Returns a list of problems (empty when the protocol ran clean)."""
     rnd = random.Random(seed)
     bars = {}
@@ -340,6 +340,15 @@ def test_forward_protocol_runs_clean(idx):
     for seed in range(12):
         problems = run([dict(x) for x in items], seed)
         assert not problems, (problems, [(x["last_a"], x["last_b"], x["has_b"]) for x in items])
+
+
+@pytest.mark.parametrize("NS", [6, 8])
+def test_forward_protocol_deeper_rings(NS):
+    """The K/V ring depths head dim 64 can select."""
+    for items in sequences()[::3]:
+        for seed in range(4):
+            problems = run([dict(x) for x in items], seed, NS)
+            assert not problems, (problems, NS, [(x["last_a"], x["last_b"], x["has_b"]) for x in items])
 
 
 def test_model_finds_the_fixed_deadlock():
